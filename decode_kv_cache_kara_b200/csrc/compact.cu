@@ -1,0 +1,469 @@
+// Paged compaction: Kara's compressed windows and LaCache's ladder, through one gather.
+//
+// "Kara: Efficient Reasoning LLM Serving via Sliding-Window KV Cache Compression", English
+// abstract: Kara is adapted to PagedAttention; the kept KV pairs move into fresh blocks, the
+// block table is rewritten and the old blocks are freed. "LaCache: Ladder-Shaped KV Caching
+// ...": states outside the ladder are dropped and the rest packed into a smaller cache
+// (method details), re-applied when the cache is full (iterative compaction).
+//
+// Three stream-ordered kernels per call:
+//   plan     (one CTA)   validates every due sequence, computes its page geometry and pops its
+//                        fresh blocks from the free list (sequence order, stack top first); on
+//                        any error it records the status and marks the plan invalid.
+//   gather   (wide grid) copies rows with 16-byte loads/stores: sources through the old
+//                        block table, destinations into the fresh blocks. Kara copies one KV
+//                        head's row per kept position; LaCache copies whole [Hkv, d] rows of
+//                        the ladder's kept slots (computed analytically per layer).
+//   finalize (one CTA)   rewrites the block table, pushes the old blocks, sets ctx_len and
+//                        free_top.
+// The gather reads only blocks that belong to the sequences and writes only fresh blocks, so
+// sources never alias destinations; nothing is modified unless the plan is valid.
+#include <cstdint>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace kara {
+
+namespace {
+
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanHeader = 16;   // valid, total_new, total_old, top
+constexpr int kPlanStride = 12;   // b, n, start, off, p0, n_old, n_new, base_new, base_old
+enum { P_B = 0, P_N, P_START, P_OFF, P_P0, P_NOLD, P_NNEW, P_BNEW, P_BOLD };
+
+__device__ int block_scan_add(int v, int* buf, int* total) {
+  // exclusive scan over 1024 threads (32 warps)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) buf[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = buf[lane];
+    int z = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, z, off);
+      if (lane >= off) z += y;
+    }
+    buf[lane] = z - w;        // exclusive prefix of warp totals
+    if (lane == 31) buf[32] = z;
+  }
+  __syncthreads();
+  const int res = buf[warp] + x - v;
+  *total = buf[32];
+  __syncthreads();
+  return res;
+}
+
+struct PlanParams {
+  const int32_t* block_table;
+  const int32_t* ctx_len;
+  const int32_t* free_list;
+  const int32_t* free_top;
+  const int32_t* seq_ids;
+  int32_t* plan;
+  int32_t* status;
+  int R, batch, max_blocks, num_blocks;
+  // Kara: window W and budget k. LaCache: W = 0, k = budget, min_len = sink+recent+R_max.
+  int W, k, lacache, min_len;
+};
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) {
+  __shared__ int buf[33];
+  __shared__ int err;
+  __shared__ int carry_new, carry_old;
+  int32_t* hdr = p.plan;
+  int32_t* rows = p.plan + kPlanHeader;
+  int32_t* fresh = rows + static_cast<size_t>(p.R) * kPlanStride;
+  if (threadIdx.x == 0) { err = 0; carry_new = 0; carry_old = 0; }
+  __syncthreads();
+  for (int base = 0; base < p.R; base += kPlanThreads) {
+    const int r = base + threadIdx.x;
+    int n_new = 0, n_old = 0;
+    if (r < p.R) {
+      int code = 0;
+      const int b = p.seq_ids ? p.seq_ids[r] : r;
+      if (b < 0 || b >= p.batch) code = KARA_ERR_INVALID_ARG;
+      if (!code && p.seq_ids && r > 0 && p.seq_ids[r - 1] >= b) code = KARA_ERR_INVALID_ARG;
+      const int n = code ? 0 : p.ctx_len[b];
+      int start = 0, off = 0, p0 = 0;
+      if (!code) {
+        if (p.lacache) {
+          if (n < p.min_len || n > p.max_blocks * 16) code = KARA_ERR_INVALID_ARG;
+          n_old = (n + 15) / 16;
+          n_new = (p.k + 15) / 16;
+        } else {
+          if (n < p.W || n > p.max_blocks * 16) code = KARA_ERR_INVALID_ARG;
+          start = n - p.W;
+          off = start % 16;
+          p0 = start / 16;
+          n_old = (off + p.W + 15) / 16;
+          n_new = (off + p.k + 15) / 16;
+        }
+      }
+      if (!code) {
+        for (int i = 0; i < n_old; ++i) {
+          const int blk = p.block_table[static_cast<size_t>(b) * p.max_blocks + p0 + i];
+          if (blk < 0 || blk >= p.num_blocks) { code = KARA_ERR_BAD_BLOCK; break; }
+        }
+      }
+      if (code) {
+        atomicCAS(&err, 0, code);
+        n_new = n_old = 0;
+      }
+      int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
+      row[P_B] = b;
+      row[P_N] = n;
+      row[P_START] = start;
+      row[P_OFF] = off;
+      row[P_P0] = p0;
+      row[P_NOLD] = n_old;
+      row[P_NNEW] = n_new;
+    }
+    int tot_new, tot_old;
+    const int ex_new = block_scan_add(n_new, buf, &tot_new);
+    const int ex_old = block_scan_add(n_old, buf, &tot_old);
+    if (r < p.R) {
+      int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
+      row[P_BNEW] = carry_new + ex_new;
+      row[P_BOLD] = carry_old + ex_old;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) { carry_new += tot_new; carry_old += tot_old; }
+    __syncthreads();
+  }
+  const int top = *p.free_top;
+  if (threadIdx.x == 0) {
+    int code = err;
+    if (!code && (top < 0 || top > p.num_blocks)) code = KARA_ERR_INVALID_ARG;
+    if (!code && carry_new > top) code = KARA_ERR_OUT_OF_BLOCKS;
+    // the pushes must fit: an inconsistent free list (ids still in use) is refused
+    if (!code && top - carry_new + carry_old > p.num_blocks) code = KARA_ERR_INVALID_ARG;
+    if (code) report(p.status, code);
+    hdr[0] = code ? 0 : 1;
+    hdr[1] = carry_new;
+    hdr[2] = carry_old;
+    hdr[3] = top;
+    err = code;
+  }
+  __syncthreads();
+  if (err) return;
+  for (int i = threadIdx.x; i < carry_new; i += kPlanThreads) fresh[i] = p.free_list[top - 1 - i];
+}
+
+struct FinalizeParams {
+  int32_t* block_table;
+  int32_t* ctx_len;
+  int32_t* free_list;
+  int32_t* free_top;
+  const int32_t* plan;
+  int R, max_blocks, k;   // k: kept slots (Kara) or budget (LaCache)
+};
+
+__global__ void __launch_bounds__(256) finalize_kernel(const FinalizeParams p) {
+  const int32_t* hdr = p.plan;
+  if (hdr[0] != 1) return;
+  const int32_t* rows = p.plan + kPlanHeader;
+  const int32_t* fresh = rows + static_cast<size_t>(p.R) * kPlanStride;
+  const int total_new = hdr[1], total_old = hdr[2], top = hdr[3];
+  const int push_base = top - total_new;
+  for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
+    const int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
+    const int b = row[P_B], p0 = row[P_P0], n_old = row[P_NOLD], n_new = row[P_NNEW];
+    int32_t* tab = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+    for (int i = 0; i < n_old; ++i) {
+      const int old = tab[p0 + i];
+      tab[p0 + i] = i < n_new ? fresh[row[P_BNEW] + i] : -1;
+      p.free_list[push_base + row[P_BOLD] + i] = old;
+    }
+    p.ctx_len[b] = row[P_START] + p.k;
+  }
+  if (threadIdx.x == 0) *p.free_top = push_base + total_old;
+}
+
+// ------------------------------------------------------------------------------------------
+// Kara gather: CTA = (layer, sequence, KV head, chunk of kept rows). Chunk 0 also copies the
+// prefix rows of the first window page for its head.
+// ------------------------------------------------------------------------------------------
+constexpr int kGatherThreads = 128;
+constexpr int kChunkRows = 64;
+
+struct KaraGather {
+  LayerPtrs layers;
+  const int32_t* block_table;
+  const int32_t* keep;
+  const int32_t* plan;
+  int32_t* status;
+  int R, Hkv, k, W, max_blocks;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kGatherThreads) kara_gather_kernel(const KaraGather g) {
+  const int32_t* hdr = g.plan;
+  if (hdr[0] != 1) return;
+  constexpr int kVecPerRow = D * 2 / 16;                  // 16-byte pieces per head row
+  constexpr int kRowsPerPass = kGatherThreads / kVecPerRow;
+  const int chunk = blockIdx.x;
+  const int head = blockIdx.y % g.Hkv;
+  const int r = blockIdx.y / g.Hkv;
+  const int layer = blockIdx.z;
+  const int32_t* rows = g.plan + kPlanHeader;
+  const int32_t* fresh = rows + static_cast<size_t>(g.R) * kPlanStride;
+  const int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
+  const int b = row[P_B], start = row[P_START], off = row[P_OFF], p0 = row[P_P0];
+  const int32_t* fr = fresh + row[P_BNEW];
+  const int32_t* tab = g.block_table + static_cast<size_t>(b) * g.max_blocks;
+  const int32_t* kp = g.keep + ((static_cast<size_t>(layer) * g.R + r) * g.Hkv + head) * g.k;
+  const uint4* ksrc = reinterpret_cast<const uint4*>(g.layers.k[layer]);
+  const uint4* vsrc = reinterpret_cast<const uint4*>(g.layers.v[layer]);
+  uint4* kdst = reinterpret_cast<uint4*>(g.layers.k[layer]);
+  uint4* vdst = reinterpret_cast<uint4*>(g.layers.v[layer]);
+  const int vec = threadIdx.x % kVecPerRow;
+  const int sub = threadIdx.x / kVecPerRow;
+
+  // rows handled by this CTA: prefix rows (chunk 0 only), then kept rows of the chunk
+  const int t0 = chunk * kChunkRows;
+  const int t1 = min(g.k, t0 + kChunkRows);
+  const int npre = (chunk == 0) ? off : 0;
+  const int total = npre + max(0, t1 - t0);
+  constexpr int kUnroll = 4;
+  for (int base = sub; base < total; base += kRowsPerPass * kUnroll) {
+    uint4 kv[kUnroll], vv[kUnroll];
+    size_t dsti[kUnroll];
+    bool act[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int i = base + u * kRowsPerPass;
+      act[u] = i < total;
+      if (!act[u]) continue;
+      int src_slot, dst_slot;
+      if (i < npre) {
+        src_slot = dst_slot = p0 * 16 + i;
+      } else {
+        const int t = t0 + (i - npre);
+        const int pos = kp[t];
+        if (pos < 0 || pos >= g.W) {      // keep entry outside the window: row left unwritten
+          report(g.status, KARA_ERR_INVALID_ARG);
+          act[u] = false;
+          continue;
+        }
+        src_slot = start + pos;
+        dst_slot = start + t;
+      }
+      const int sblk = tab[src_slot >> 4];
+      const int dblk = fr[(dst_slot >> 4) - p0];
+      const size_t si = ((static_cast<size_t>(sblk) * 16 + (src_slot & 15)) * g.Hkv + head) *
+                            kVecPerRow + vec;
+      dsti[u] = ((static_cast<size_t>(dblk) * 16 + (dst_slot & 15)) * g.Hkv + head) *
+                    kVecPerRow + vec;
+      kv[u] = ksrc[si];
+      vv[u] = vsrc[si];
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (!act[u]) continue;
+      kdst[dsti[u]] = kv[u];
+      vdst[dsti[u]] = vv[u];
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// LaCache gather: CTA = (layer, sequence, chunk of compacted slots); whole [Hkv, d] rows.
+// ------------------------------------------------------------------------------------------
+struct LadderGather {
+  LayerPtrs layers;
+  const int32_t* block_table;
+  const int32_t* plan;
+  int R, L, max_blocks;
+  int row_vecs;          // 16-byte pieces per slot row (Hkv * D * 2 / 16)
+  int span, overlap, rung, budget, sink, recent, r_max;
+};
+
+constexpr int kLadderSlots = 32;
+
+// Source slot of compacted slot t in `layer`, for a sequence of n slots.
+__device__ __forceinline__ int ladder_source(const LadderGather& g, int layer, int t, int n) {
+  if (t < g.sink) return t;
+  if (t >= g.budget - g.recent) return n - (g.budget - t);
+  const int stride = g.span - g.overlap;
+  const int q = g.span / stride;          // rungs one layer keeps per period
+  const int period = g.L / stride;        // rungs per period
+  const int tr = t - g.sink;
+  const int per = tr / (q * g.rung);
+  const int rem = tr % (q * g.rung);
+  const int m = rem / g.rung;             // m-th kept rung of this layer within the period
+  const int o = rem % g.rung;
+  const int a = layer / stride;
+  // kept rungs of the layer within a period: (a - u) mod period, u = 0..q-1, ascending
+  int j;
+  if (a >= q - 1) j = a - q + 1 + m;
+  else j = (m <= a) ? m : period - q + m;
+  const int region_start = n - g.recent - g.r_max;
+  return region_start + (per * period + j) * g.rung + o;
+}
+
+__global__ void __launch_bounds__(kGatherThreads) ladder_gather_kernel(const LadderGather g) {
+  const int32_t* hdr = g.plan;
+  if (hdr[0] != 1) return;
+  const int chunk = blockIdx.x;
+  const int r = blockIdx.y;
+  const int layer = blockIdx.z;
+  const int32_t* rows = g.plan + kPlanHeader;
+  const int32_t* fresh = rows + static_cast<size_t>(g.R) * kPlanStride;
+  const int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
+  const int b = row[P_B], n = row[P_N];
+  const int32_t* fr = fresh + row[P_BNEW];
+  const int32_t* tab = g.block_table + static_cast<size_t>(b) * g.max_blocks;
+  const uint4* ksrc = reinterpret_cast<const uint4*>(g.layers.k[layer]);
+  const uint4* vsrc = reinterpret_cast<const uint4*>(g.layers.v[layer]);
+  uint4* kdst = reinterpret_cast<uint4*>(g.layers.k[layer]);
+  uint4* vdst = reinterpret_cast<uint4*>(g.layers.v[layer]);
+  const int t0 = chunk * kLadderSlots;
+  const int t1 = min(g.budget, t0 + kLadderSlots);
+  const int pieces = (t1 - t0) * g.row_vecs;
+  constexpr int kUnroll = 4;
+  for (int base = threadIdx.x; base < pieces; base += kGatherThreads * kUnroll) {
+    uint4 kv[kUnroll], vv[kUnroll];
+    size_t dsti[kUnroll];
+    bool act[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int i = base + u * kGatherThreads;
+      act[u] = i < pieces;
+      if (!act[u]) continue;
+      const int t = t0 + i / g.row_vecs;
+      const int v = i % g.row_vecs;
+      const int src = ladder_source(g, layer, t, n);
+      const int sblk = tab[src >> 4];
+      const int dblk = fr[t >> 4];
+      const size_t si = (static_cast<size_t>(sblk) * 16 + (src & 15)) * g.row_vecs + v;
+      dsti[u] = (static_cast<size_t>(dblk) * 16 + (t & 15)) * g.row_vecs + v;
+      kv[u] = ksrc[si];
+      vv[u] = vsrc[si];
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (!act[u]) continue;
+      kdst[dsti[u]] = kv[u];
+      vdst[dsti[u]] = vv[u];
+    }
+  }
+}
+
+}  // namespace
+
+size_t compact_workspace_bytes(int R, int W, int k) {
+  (void)W;
+  const size_t fresh = static_cast<size_t>(R) * ((15 + k + 15) / 16);
+  return (kPlanHeader + static_cast<size_t>(R) * kPlanStride + fresh) * sizeof(int32_t);
+}
+
+size_t lacache_workspace_bytes(int R, int budget) {
+  const size_t fresh = static_cast<size_t>(R) * ((budget + 15) / 16);
+  return (kPlanHeader + static_cast<size_t>(R) * kPlanStride + fresh) * sizeof(int32_t);
+}
+
+kara_status launch_compact(const CompactLaunch& L, cudaStream_t stream) {
+  if (L.R == 0) return KARA_OK;
+  PlanParams pp;
+  pp.block_table = L.block_table;
+  pp.ctx_len = L.ctx_len;
+  pp.free_list = L.free_list;
+  pp.free_top = L.free_top;
+  pp.seq_ids = L.seq_ids;
+  pp.plan = L.plan;
+  pp.status = L.status;
+  pp.R = L.R;
+  pp.batch = L.batch;
+  pp.max_blocks = L.max_blocks;
+  pp.num_blocks = L.num_blocks;
+  pp.W = L.W;
+  pp.k = L.k;
+  pp.lacache = 0;
+  pp.min_len = 0;
+  plan_kernel<<<1, kPlanThreads, 0, stream>>>(pp);
+  KaraGather g;
+  g.layers = L.layers;
+  g.block_table = L.block_table;
+  g.keep = L.keep;
+  g.plan = L.plan;
+  g.status = L.status;
+  g.R = L.R;
+  g.Hkv = L.Hkv;
+  g.k = L.k;
+  g.W = L.W;
+  g.max_blocks = L.max_blocks;
+  dim3 grid((L.k + kChunkRows - 1) / kChunkRows, L.R * L.Hkv, L.L);
+  if (L.D == 128) kara_gather_kernel<128><<<grid, kGatherThreads, 0, stream>>>(g);
+  else kara_gather_kernel<64><<<grid, kGatherThreads, 0, stream>>>(g);
+  FinalizeParams fp;
+  fp.block_table = L.block_table;
+  fp.ctx_len = L.ctx_len;
+  fp.free_list = L.free_list;
+  fp.free_top = L.free_top;
+  fp.plan = L.plan;
+  fp.R = L.R;
+  fp.max_blocks = L.max_blocks;
+  fp.k = L.k;
+  finalize_kernel<<<1, 256, 0, stream>>>(fp);
+  return cudaGetLastError() == cudaSuccess ? KARA_OK : KARA_ERR_CUDA;
+}
+
+kara_status launch_lacache(const LacacheLaunch& L, cudaStream_t stream) {
+  if (L.R == 0) return KARA_OK;
+  const int r_max = (L.budget - L.sink - L.recent) * L.L / L.span;
+  PlanParams pp;
+  pp.block_table = L.block_table;
+  pp.ctx_len = L.ctx_len;
+  pp.free_list = L.free_list;
+  pp.free_top = L.free_top;
+  pp.seq_ids = L.seq_ids;
+  pp.plan = L.plan;
+  pp.status = L.status;
+  pp.R = L.R;
+  pp.batch = L.batch;
+  pp.max_blocks = L.max_blocks;
+  pp.num_blocks = L.num_blocks;
+  pp.W = 0;
+  pp.k = L.budget;
+  pp.lacache = 1;
+  pp.min_len = L.sink + L.recent + r_max;
+  plan_kernel<<<1, kPlanThreads, 0, stream>>>(pp);
+  LadderGather g;
+  g.layers = L.layers;
+  g.block_table = L.block_table;
+  g.plan = L.plan;
+  g.R = L.R;
+  g.L = L.L;
+  g.max_blocks = L.max_blocks;
+  g.row_vecs = L.Hkv * L.D * 2 / 16;
+  g.span = L.span;
+  g.overlap = L.overlap;
+  g.rung = L.rung;
+  g.budget = L.budget;
+  g.sink = L.sink;
+  g.recent = L.recent;
+  g.r_max = r_max;
+  dim3 grid((L.budget + kLadderSlots - 1) / kLadderSlots, L.R, L.L);
+  ladder_gather_kernel<<<grid, kGatherThreads, 0, stream>>>(g);
+  FinalizeParams fp;
+  fp.block_table = L.block_table;
+  fp.ctx_len = L.ctx_len;
+  fp.free_list = L.free_list;
+  fp.free_top = L.free_top;
+  fp.plan = L.plan;
+  fp.R = L.R;
+  fp.max_blocks = L.max_blocks;
+  fp.k = L.budget;
+  finalize_kernel<<<1, 256, 0, stream>>>(fp);
+  return cudaGetLastError() == cudaSuccess ? KARA_OK : KARA_ERR_CUDA;
+}
+
+}  // namespace kara

@@ -1,0 +1,90 @@
+// Internal launch interface between the C-ABI entry points (api.cu) and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "kara.h"
+
+namespace kara {
+
+struct ScoreLaunch {
+  const void* q_win;
+  const void* k_cache;
+  const int32_t* block_table;
+  const int32_t* ctx_len;
+  const int32_t* seq_ids;
+  float* lse;
+  float* scores;
+  int32_t* status;
+  int R, W, Hq, Hkv, D;
+  int batch, max_blocks, num_blocks;
+  float scale;
+};
+int score_lse_stride(int W);
+kara_status launch_score_kernels(const ScoreLaunch& L, cudaStream_t stream);
+
+kara_status launch_select(const float* scores, int rows, int W, int k, int32_t* sel,
+                          cudaStream_t stream);
+kara_status launch_token2chunk(const float* scores, const int32_t* sel, int rows, int W, int k,
+                               int num_anchors, int gap_limit, int widen, int32_t* keep,
+                               cudaStream_t stream);
+
+struct LayerPtrs {
+  void* k[KARA_MAX_LAYERS];
+  void* v[KARA_MAX_LAYERS];
+};
+
+struct CompactLaunch {
+  LayerPtrs layers;
+  int L;
+  int32_t* block_table;
+  int32_t* ctx_len;
+  int32_t* free_list;
+  int32_t* free_top;
+  const int32_t* seq_ids;
+  const int32_t* keep;
+  int32_t* plan;     // workspace
+  int32_t* status;
+  int R, W, k, Hkv, D;
+  int batch, max_blocks, num_blocks;
+};
+size_t compact_workspace_bytes(int R, int W, int k);
+kara_status launch_compact(const CompactLaunch& L, cudaStream_t stream);
+
+struct LacacheLaunch {
+  LayerPtrs layers;
+  int L;
+  int32_t* block_table;
+  int32_t* ctx_len;
+  int32_t* free_list;
+  int32_t* free_top;
+  const int32_t* seq_ids;
+  int32_t* plan;
+  int32_t* status;
+  int R, Hkv, D;
+  int batch, max_blocks, num_blocks;
+  int span, overlap, rung, budget, sink, recent;
+};
+size_t lacache_workspace_bytes(int R, int budget);
+kara_status launch_lacache(const LacacheLaunch& L, cudaStream_t stream);
+
+struct DecodeLaunch {
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_table;
+  const int32_t* ctx_len;
+  void* out;
+  float* partial;    // workspace
+  int32_t* status;
+  int B, Hq, Hkv, D;
+  int max_blocks, num_blocks;
+  float scale;
+};
+int decode_num_splits(int max_blocks);
+size_t decode_workspace_bytes(int B, int Hq, int D, int max_blocks);
+kara_status launch_decode(const DecodeLaunch& L, cudaStream_t stream);
+
+}  // namespace kara

@@ -1,0 +1,600 @@
+// Window scoring on tcgen05 tensor cores (sm_100a).
+//
+// Computes, per due sequence r and KV head g,
+//   score[j] = sum over the G query heads h of g and the window queries i of
+//              softmax_j(q_hi . k_j * scale),
+// bidirectional (unmasked) attention inside the compression window, column-summed
+// ("Kara: Efficient Reasoning LLM Serving via Sliding-Window KV Cache Compression", English
+// abstract: bidirectional attention scores the KV pairs of the window; gist.science explainer,
+// section 1: a token the current reasoning refers to strongly scores high).
+//
+// Two passes, both persistent and warp-specialised (warp 0: TMA producer, warp 1: UMMA
+// issuer and TMEM owner, warps 2-5: epilogue, one TMEM lane per thread):
+//   pass 1 (query-major)  S = Q K^T, 128 query rows x up to 256 keys per UMMA tile; each
+//                         epilogue thread owns one query row and keeps an online base-2
+//                         log-sum-exp; the result goes to the workspace.
+//   pass 2 (key-major)    S^T = K Q^T, 128 keys x 256 queries per tile; each epilogue thread
+//                         owns one key and sums 2^(s*scale*log2e - lse_i) over all queries.
+// Keys are read in place from the paged pool: a key tile is a run of whole 16-slot pages
+// (TMA box of one page and one KV head); slots outside [n-W, n) are masked in the epilogue.
+// Queries come from the dense window-query buffer [R, W, Hq, d]; rows past W are zero-filled
+// by TMA and carry lse = +inf, so they add nothing in pass 2.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace kara {
+
+namespace {
+
+constexpr int kThreads = 192;        // 6 warps
+constexpr int kQRows1 = 128;         // pass 1: query rows per tile (UMMA M)
+constexpr int kKRows1 = 256;         // pass 1: max keys per UMMA (N)
+constexpr int kKStages1 = 2;
+constexpr int kKRows2 = 128;         // pass 2: keys per tile (UMMA M)
+constexpr int kQRows2 = 256;         // pass 2: queries per UMMA (N)
+constexpr int kQStages2 = 2;
+constexpr int kRowBytes = 128;       // one 64-element bf16 K-chunk row (128-byte swizzle)
+constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
+
+struct ScoreArgs {
+  const int32_t* block_table;
+  const int32_t* ctx_len;
+  const int32_t* seq_ids;
+  float* lse;       // [R, Hq, Wp] base-2 log-sum-exp of scaled logits per query
+  float* scores;    // [R, Hkv, W]
+  int32_t* status;
+  int R, W, Wp, Hq, Hkv, G;
+  int batch, max_blocks, num_blocks;
+  float cs;         // scale * log2(e)
+};
+
+struct SeqInfo {
+  int b, n, start, p_first, np;  // np: pages spanned by the window
+  bool ok;
+};
+
+__device__ __forceinline__ SeqInfo seq_info(const ScoreArgs& a, int r) {
+  SeqInfo s;
+  s.b = a.seq_ids ? a.seq_ids[r] : r;
+  s.ok = s.b >= 0 && s.b < a.batch;
+  s.n = s.ok ? a.ctx_len[s.b] : 0;
+  s.ok = s.ok && s.n >= a.W && s.n <= a.max_blocks * 16;
+  s.start = s.n - a.W;
+  s.p_first = s.ok ? s.start / 16 : 0;
+  s.np = s.ok ? (s.n - 1) / 16 - s.p_first + 1 : 0;
+  return s;
+}
+
+// Block id of page p of sequence row b, with range check (an out-of-range id is reported and
+// replaced by block 0 so that the pipeline keeps its byte counts and never stalls).
+__device__ __forceinline__ int page_block(const ScoreArgs& a, int b, int p) {
+  int blk = a.block_table[static_cast<size_t>(b) * a.max_blocks + p];
+  if (blk < 0 || blk >= a.num_blocks) {
+    report(a.status, KARA_ERR_BAD_BLOCK);
+    blk = 0;
+  }
+  return blk;
+}
+
+// ----------------------------------------------------------------------------------------
+// Pass 1: per-query base-2 log-sum-exp over the window keys.
+// ----------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
+  constexpr int NCH = D / 64;
+  constexpr uint32_t kQBytes = NCH * kQRows1 * kRowBytes;
+  constexpr uint32_t kKBytes = NCH * kKRows1 * kRowBytes;
+  constexpr uint32_t kPageBytes = 16 * kRowBytes;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* q_buf = smem;                      // 2 x kQBytes
+  uint8_t* k_buf = smem + 2 * kQBytes;        // kKStages1 x kKBytes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(k_buf + kKStages1 * kKBytes);
+  uint64_t* q_full = bars;        // [2]
+  uint64_t* q_empty = bars + 2;   // [2]
+  uint64_t* k_full = bars + 4;    // [kKStages1]
+  uint64_t* k_empty = bars + 4 + kKStages1;
+  uint64_t* acc_full = bars + 4 + 2 * kKStages1;   // [2]
+  uint64_t* acc_empty = acc_full + 2;              // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const int TT = (a.W + kQRows1 - 1) / kQRows1;
+  const int num_tiles = a.R * a.Hq * TT;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+    }
+    for (int i = 0; i < kKStages1; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      int qi = 0, ki = 0;
+      uint32_t qph = 0, kph = 0;
+      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+        const int tt = t % TT;
+        const int h = (t / TT) % a.Hq;
+        const int r = t / (TT * a.Hq);
+        const SeqInfo s = seq_info(a, r);
+        if (!s.ok) continue;
+        const int g = h / a.G;
+        if (!mbar_wait(&q_empty[qi], qph ^ 1, abort_flag, a.status)) break;
+        mbar_expect_tx(&q_full[qi], kQBytes);
+        for (int c = 0; c < NCH; ++c)
+          tma_load_4d(q_buf + qi * kQBytes + c * kQRows1 * kRowBytes, &tm_q, &q_full[qi], c * 64,
+                      h, tt * kQRows1, r);
+        if (++qi == 2) { qi = 0; qph ^= 1; }
+        const int nkt = (s.np + 15) / 16;
+        bool stop = false;
+        for (int kt = 0; kt < nkt; ++kt) {
+          const int pages = min(16, s.np - kt * 16);
+          if (!mbar_wait(&k_empty[ki], kph ^ 1, abort_flag, a.status)) { stop = true; break; }
+          mbar_expect_tx(&k_full[ki], pages * NCH * kPageBytes);
+          for (int p = 0; p < pages; ++p) {
+            const int blk = page_block(a, s.b, s.p_first + kt * 16 + p);
+            for (int c = 0; c < NCH; ++c)
+              tma_load_4d(k_buf + ki * kKBytes + c * kKRows1 * kRowBytes + p * kPageBytes, &tm_k,
+                          &k_full[ki], c * 64, g, 0, blk);
+          }
+          if (++ki == kKStages1) { ki = 0; kph ^= 1; }
+        }
+        if (stop) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- UMMA issuer ----------------
+    if (lane == 0) {
+      int qi = 0, ki = 0, ab = 0;
+      uint32_t qph = 0, kph = 0, aph = 0;
+      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+        const int r = t / (TT * a.Hq);
+        const SeqInfo s = seq_info(a, r);
+        if (!s.ok) continue;
+        if (!mbar_wait(&q_full[qi], qph, abort_flag, a.status)) break;
+        const uint32_t q_addr = smem_u32(q_buf + qi * kQBytes);
+        const int nkt = (s.np + 15) / 16;
+        bool stop = false;
+        for (int kt = 0; kt < nkt; ++kt) {
+          const int pages = min(16, s.np - kt * 16);
+          if (!mbar_wait(&k_full[ki], kph, abort_flag, a.status)) { stop = true; break; }
+          if (!mbar_wait(&acc_empty[ab], aph ^ 1, abort_flag, a.status)) { stop = true; break; }
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(k_buf + ki * kKBytes);
+          const uint32_t idesc = idesc_bf16_f32(128, pages * 16);
+          const uint32_t d_tmem = tmem_base + ab * 256;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
+            const uint64_t ad = sw128_kmajor_desc(q_addr + (kk >> 2) * kQRows1 * kRowBytes + off);
+            const uint64_t bd = sw128_kmajor_desc(k_addr + (kk >> 2) * kKRows1 * kRowBytes + off);
+            umma_bf16(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&k_empty[ki]);
+          umma_commit(&acc_full[ab]);
+          if (++ki == kKStages1) { ki = 0; kph ^= 1; }
+          if (++ab == 2) { ab = 0; aph ^= 1; }
+        }
+        if (stop) break;
+        umma_commit(&q_empty[qi]);
+        if (++qi == 2) { qi = 0; qph ^= 1; }
+      }
+    }
+  } else {
+    // ---------------- epilogue: one query row per thread ----------------
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    int ab = 0;
+    uint32_t aph = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const int tt = t % TT;
+      const int h = (t / TT) % a.Hq;
+      const int r = t / (TT * a.Hq);
+      const SeqInfo s = seq_info(a, r);
+      float lse2 = INFINITY;
+      if (s.ok && !*abort_flag) {
+        float m = -INFINITY, l = 0.f;
+        const int nkt = (s.np + 15) / 16;
+        bool stop = false;
+        for (int kt = 0; kt < nkt; ++kt) {
+          const int ncols = min(16, s.np - kt * 16) * 16;
+          if (!mbar_wait(&acc_full[ab], aph, abort_flag, a.status)) { stop = true; break; }
+          tc_fence_after();
+          const int slot0 = (s.p_first + kt * 16) * 16;
+          const bool edge = (kt == 0) || (kt == nkt - 1);
+          for (int c = 0; c < ncols; c += 32) {
+            float v[32];
+            const int nvalid = min(32, ncols - c);
+            if (nvalid == 32) {
+              tmem_ld32(lane_base + ab * 256 + c, v);
+            } else {
+              float v16[16];
+              tmem_ld16(lane_base + ab * 256 + c, v16);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) { v[i] = v16[i]; v[16 + i] = -INFINITY; }
+            }
+            tmem_wait_ld();
+            if (edge) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int slot = slot0 + c + i;
+                if (slot < s.start || slot >= s.n) v[i] = -INFINITY;
+              }
+            }
+            float cmax = v[0];
+#pragma unroll
+            for (int i = 1; i < 32; ++i) cmax = fmaxf(cmax, v[i]);
+            if (cmax == -INFINITY) continue;
+            const float m_new = fmaxf(m, cmax * a.cs);
+            float sum = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sum += ex2(fmaf(v[i], a.cs, -m_new));
+            l = l * ex2(m - m_new) + sum;
+            m = m_new;
+          }
+          tc_fence_before();
+          mbar_arrive(&acc_empty[ab]);
+          if (++ab == 2) { ab = 0; aph ^= 1; }
+        }
+        if (!stop) lse2 = m + __log2f(l);
+      } else if (!s.ok && tt == 0 && h == 0 && row == 0) {
+        report(a.status, KARA_ERR_INVALID_ARG);
+      }
+      const int token = tt * kQRows1 + row;
+      float* lrow = a.lse + (static_cast<size_t>(r) * a.Hq + h) * a.Wp;
+      if (token < a.W) lrow[token] = lse2;
+      else if (token < a.Wp) lrow[token] = INFINITY;
+      if (tt == TT - 1) {
+        const int extra = TT * kQRows1 + row;
+        if (extra < a.Wp) lrow[extra] = INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------------------------------
+// Pass 2: per-key sums of the normalised probabilities.
+// ----------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
+  constexpr int NCH = D / 64;
+  constexpr uint32_t kABytes = NCH * kKRows2 * kRowBytes;
+  constexpr uint32_t kBBytes = NCH * kQRows2 * kRowBytes;
+  constexpr uint32_t kPageBytes = 16 * kRowBytes;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* a_buf = smem;                    // 2 x kABytes (key tiles)
+  uint8_t* b_buf = smem + 2 * kABytes;      // kQStages2 x kBBytes (query tiles)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(b_buf + kQStages2 * kBBytes);
+  uint64_t* a_full = bars;                  // [2]
+  uint64_t* a_empty = bars + 2;             // [2]
+  uint64_t* b_full = bars + 4;              // [kQStages2]
+  uint64_t* b_empty = bars + 4 + kQStages2;
+  uint64_t* acc_full = bars + 4 + 2 * kQStages2;   // [2]
+  uint64_t* acc_empty = acc_full + 2;              // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  // Key tiles of 8 pages; the window spans at most ceil((W+15)/16) pages.
+  const int KT = ((a.W + 15 + 15) / 16 + 7) / 8;
+  const int QT = (a.W + kQRows2 - 1) / kQRows2;
+  const int num_tiles = a.R * a.Hkv * KT;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&a_full[i], 1);
+      mbar_init(&a_empty[i], 1);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+    }
+    for (int i = 0; i < kQStages2; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      int ai = 0, bi = 0;
+      uint32_t aph = 0, bph = 0;
+      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+        const int kt = t % KT;
+        const int g = (t / KT) % a.Hkv;
+        const int r = t / (KT * a.Hkv);
+        const SeqInfo s = seq_info(a, r);
+        if (!s.ok || kt * 8 >= s.np) continue;
+        const int pages = min(8, s.np - kt * 8);
+        if (!mbar_wait(&a_empty[ai], aph ^ 1, abort_flag, a.status)) break;
+        mbar_expect_tx(&a_full[ai], pages * NCH * kPageBytes);
+        for (int p = 0; p < pages; ++p) {
+          const int blk = page_block(a, s.b, s.p_first + kt * 8 + p);
+          for (int c = 0; c < NCH; ++c)
+            tma_load_4d(a_buf + ai * kABytes + c * kKRows2 * kRowBytes + p * kPageBytes, &tm_k,
+                        &a_full[ai], c * 64, g, 0, blk);
+        }
+        if (++ai == 2) { ai = 0; aph ^= 1; }
+        bool stop = false;
+        for (int hl = 0; hl < a.G && !stop; ++hl) {
+          const int h = g * a.G + hl;
+          for (int qt = 0; qt < QT; ++qt) {
+            if (!mbar_wait(&b_empty[bi], bph ^ 1, abort_flag, a.status)) { stop = true; break; }
+            mbar_expect_tx(&b_full[bi], kBBytes);
+            for (int c = 0; c < NCH; ++c)
+              tma_load_4d(b_buf + bi * kBBytes + c * kQRows2 * kRowBytes, &tm_q, &b_full[bi],
+                          c * 64, h, qt * kQRows2, r);
+            if (++bi == kQStages2) { bi = 0; bph ^= 1; }
+          }
+        }
+        if (stop) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int ai = 0, bi = 0, ab = 0;
+      uint32_t aph = 0, bph = 0, cph = 0;
+      const uint32_t idesc = idesc_bf16_f32(128, kQRows2);
+      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+        const int kt = t % KT;
+        const int r = t / (KT * a.Hkv);
+        const SeqInfo s = seq_info(a, r);
+        if (!s.ok || kt * 8 >= s.np) continue;
+        if (!mbar_wait(&a_full[ai], aph, abort_flag, a.status)) break;
+        const uint32_t a_addr = smem_u32(a_buf + ai * kABytes);
+        bool stop = false;
+        for (int q = 0; q < a.G * QT; ++q) {
+          if (!mbar_wait(&b_full[bi], bph, abort_flag, a.status)) { stop = true; break; }
+          if (!mbar_wait(&acc_empty[ab], cph ^ 1, abort_flag, a.status)) { stop = true; break; }
+          tc_fence_after();
+          const uint32_t b_addr = smem_u32(b_buf + bi * kBBytes);
+          const uint32_t d_tmem = tmem_base + ab * 256;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            const uint64_t ad = sw128_kmajor_desc(a_addr + (kk >> 2) * kKRows2 * kRowBytes + off);
+            const uint64_t bd = sw128_kmajor_desc(b_addr + (kk >> 2) * kQRows2 * kRowBytes + off);
+            umma_bf16(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&b_empty[bi]);
+          umma_commit(&acc_full[ab]);
+          if (++bi == kQStages2) { bi = 0; bph ^= 1; }
+          if (++ab == 2) { ab = 0; cph ^= 1; }
+        }
+        if (stop) break;
+        umma_commit(&a_empty[ai]);
+        if (++ai == 2) { ai = 0; aph ^= 1; }
+      }
+    }
+  } else {
+    // ---------------- epilogue: one key per thread ----------------
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    int ab = 0;
+    uint32_t cph = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const int kt = t % KT;
+      const int g = (t / KT) % a.Hkv;
+      const int r = t / (KT * a.Hkv);
+      const SeqInfo s = seq_info(a, r);
+      float* out = a.scores + (static_cast<size_t>(r) * a.Hkv + g) * a.W;
+      if (!s.ok) {
+        const int j = kt * kKRows2 + row;
+        if (j < a.W) out[j] = 0.f;
+        continue;
+      }
+      if (kt * 8 >= s.np) continue;
+      float acc = 0.f;
+      bool stop = *abort_flag != 0;
+      for (int hl = 0; hl < a.G && !stop; ++hl) {
+        const int h = g * a.G + hl;
+        const float* lrow = a.lse + (static_cast<size_t>(r) * a.Hq + h) * a.Wp;
+        for (int qt = 0; qt < QT; ++qt) {
+          if (!mbar_wait(&acc_full[ab], cph, abort_flag, a.status)) { stop = true; break; }
+          tc_fence_after();
+          const float4* l4 = reinterpret_cast<const float4*>(lrow + qt * kQRows2);
+#pragma unroll 1
+          for (int c = 0; c < kQRows2; c += 32) {
+            float v[32];
+            tmem_ld32(lane_base + ab * 256 + c, v);
+            float lz[32];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 x = __ldg(l4 + (c >> 2) + i);
+              lz[4 * i] = x.x; lz[4 * i + 1] = x.y; lz[4 * i + 2] = x.z; lz[4 * i + 3] = x.w;
+            }
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc += ex2(fmaf(v[i], a.cs, -lz[i]));
+          }
+          tc_fence_before();
+          mbar_arrive(&acc_empty[ab]);
+          if (++ab == 2) { ab = 0; cph ^= 1; }
+        }
+      }
+      if (stop) continue;
+      const int slot = (s.p_first + kt * 8) * 16 + row;
+      const int j = slot - s.start;
+      if (row < min(8, s.np - kt * 8) * 16 && j >= 0 && j < a.W) out[j] = acc;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+template <int D>
+constexpr size_t rowstats_smem() {
+  return 1024 + 2 * (D / 64) * kQRows1 * kRowBytes + kKStages1 * (D / 64) * kKRows1 * kRowBytes +
+         256;
+}
+template <int D>
+constexpr size_t colsum_smem() {
+  return 1024 + 2 * (D / 64) * kKRows2 * kRowBytes + kQStages2 * (D / 64) * kQRows2 * kRowBytes +
+         256;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 4-D bf16 tensor map, innermost dimension first, 128-byte swizzle, box {64, 1, rows, 1}.
+bool make_map(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides[3],
+              uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t gdim[4] = {dims[0], dims[1], dims[2], dims[3]};
+  cuuint64_t gstride[3] = {strides[0], strides[1], strides[2]};
+  cuuint32_t box[4] = {64, 1, box_rows, 1};
+  cuuint32_t estride[4] = {1, 1, 1, 1};
+  CUresult res = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), gdim, gstride,
+                    box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int D>
+kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
+  const uint64_t qdims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(L.Hq),
+                             static_cast<uint64_t>(L.W), static_cast<uint64_t>(L.R)};
+  const uint64_t qstr[3] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(L.Hq) * D * 2,
+                            static_cast<uint64_t>(L.W) * L.Hq * D * 2};
+  const uint64_t kdims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(L.Hkv), 16,
+                             static_cast<uint64_t>(L.num_blocks)};
+  const uint64_t kstr[3] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(L.Hkv) * D * 2,
+                            static_cast<uint64_t>(16) * L.Hkv * D * 2};
+  CUtensorMap tq1, tq2, tk;
+  if (!make_map(&tq1, L.q_win, qdims, qstr, kQRows1) ||
+      !make_map(&tq2, L.q_win, qdims, qstr, kQRows2) || !make_map(&tk, L.k_cache, kdims, kstr, 16))
+    return KARA_ERR_CUDA;
+
+  ScoreArgs a;
+  a.block_table = L.block_table;
+  a.ctx_len = L.ctx_len;
+  a.seq_ids = L.seq_ids;
+  a.lse = L.lse;
+  a.scores = L.scores;
+  a.status = L.status;
+  a.R = L.R;
+  a.W = L.W;
+  a.Wp = score_lse_stride(L.W);
+  a.Hq = L.Hq;
+  a.Hkv = L.Hkv;
+  a.G = L.Hq / L.Hkv;
+  a.batch = L.batch;
+  a.max_blocks = L.max_blocks;
+  a.num_blocks = L.num_blocks;
+  a.cs = L.scale * 1.4426950408889634f;
+
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(score_rowstats_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(rowstats_smem<D>()));
+    cudaFuncSetAttribute(score_colsum_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(colsum_smem<D>()));
+    attr_set = true;
+  }
+  const int TT = (L.W + kQRows1 - 1) / kQRows1;
+  const int tiles1 = L.R * L.Hq * TT;
+  const int KT = ((L.W + 15 + 15) / 16 + 7) / 8;
+  const int tiles2 = L.R * L.Hkv * KT;
+  const int sms = sm_count();
+  score_rowstats_kernel<D><<<min(tiles1, sms), kThreads, rowstats_smem<D>(), stream>>>(tq1, tk, a);
+  if (cudaGetLastError() != cudaSuccess) return KARA_ERR_CUDA;
+  score_colsum_kernel<D><<<min(tiles2, sms), kThreads, colsum_smem<D>(), stream>>>(tq2, tk, a);
+  if (cudaGetLastError() != cudaSuccess) return KARA_ERR_CUDA;
+  return KARA_OK;
+}
+
+}  // namespace
+
+int score_lse_stride(int W) { return (W + 255) / 256 * 256; }
+
+kara_status launch_score_kernels(const ScoreLaunch& L, cudaStream_t stream) {
+  if (L.D == 128) return launch_score<128>(L, stream);
+  if (L.D == 64) return launch_score<64>(L, stream);
+  return KARA_ERR_UNSUPPORTED;
+}
+
+}  // namespace kara

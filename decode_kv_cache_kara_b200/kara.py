@@ -1,0 +1,332 @@
+"""Python binding of libkara (ctypes). Argument marshalling only: every step runs in the CUDA
+library declared in include/kara.h. Torch provides device memory and the current stream.
+
+The functions carry the C names:
+    kara_score, kara_select, kara_token2chunk, kara_compact, paged_decode_attn,
+    lacache_compact, kara_workspace_bytes
+There is no CPU fallback: a missing library raises ``KaraLibraryError``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+from dataclasses import dataclass
+
+import torch
+
+from . import build as _build
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_UNSUPPORTED = 2
+ERR_OUT_OF_BLOCKS = 3
+ERR_CUDA = 4
+ERR_TIMEOUT = 5
+ERR_WORKSPACE = 6
+ERR_BAD_BLOCK = 7
+
+OP_SCORE, OP_COMPACT, OP_DECODE, OP_LACACHE = 1, 2, 3, 4
+MAX_LAYERS = 128
+
+
+class KaraLibraryError(ImportError):
+    """libkara.so is missing or cannot be loaded."""
+
+
+class KaraError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_str(code)} ({code})")
+
+
+class _LayerKV(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p)]
+
+
+class _Pool(ctypes.Structure):
+    _fields_ = [("block_table", ctypes.c_void_p), ("ctx_len", ctypes.c_void_p),
+                ("free_list", ctypes.c_void_p), ("free_top", ctypes.c_void_p),
+                ("batch", ctypes.c_int32), ("max_blocks_per_seq", ctypes.c_int32),
+                ("num_blocks", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+class _LacacheParams(ctypes.Structure):
+    _fields_ = [("span", ctypes.c_int32), ("overlap", ctypes.c_int32), ("rung", ctypes.c_int32),
+                ("budget", ctypes.c_int32), ("sink", ctypes.c_int32), ("recent", ctypes.c_int32)]
+
+
+_LIB = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_F = ctypes.c_float
+_Z = ctypes.c_size_t
+
+_SIGNATURES = {
+    "kara_score": ([_P, _P, ctypes.POINTER(_Pool), _P, _I, _I, _I, _F, _P, _P, _Z, _P, _P], _I),
+    "kara_select": ([_P, _I, _I, _I, _P, _P], _I),
+    "kara_token2chunk": ([_P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
+    "kara_compact": ([ctypes.POINTER(_LayerKV), _I, ctypes.POINTER(_Pool), _P, _I, _I, _I, _P, _P,
+                      _Z, _P, _P], _I),
+    "paged_decode_attn": ([_P, _P, _P, ctypes.POINTER(_Pool), _I, _F, _P, _P, _Z, _P, _P], _I),
+    "lacache_compact": ([ctypes.POINTER(_LayerKV), _I, ctypes.POINTER(_Pool), _P, _I,
+                         ctypes.POINTER(_LacacheParams), _P, _Z, _P, _P], _I),
+    "kara_workspace_bytes": ([_I, ctypes.POINTER(_Pool), _I, _I, _I, _I], _Z),
+    "kara_status_str": ([_I], ctypes.c_char_p),
+    "kara_version": ([], ctypes.c_char_p),
+}
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib():
+    """The loaded libkara (loaded once). Raises KaraLibraryError when it is not built."""
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise KaraLibraryError(
+                f"{path} is missing: build it with `python -m decode_kv_cache_kara_b200.build`")
+        try:
+            handle = ctypes.CDLL(path)
+        except OSError as e:  # pragma: no cover - depends on the host
+            raise KaraLibraryError(f"cannot load {path}: {e}") from e
+        for name, (args, res) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = res
+        _LIB = handle
+    return _LIB
+
+
+def declared_symbols(header: str | None = None) -> list:
+    """Function names declared in include/kara.h (used by the ABI tests)."""
+    header = header or os.path.join(_build.INCLUDE, "kara.h")
+    text = open(header).read()
+    return re.findall(r"^\s*(?:kara_status|size_t|const char\*)\s+(\w+)\s*\(", text, re.M)
+
+
+def status_str(code: int) -> str:
+    return lib().kara_status_str(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise KaraError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _require(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+@dataclass
+class PagedPool:
+    """The shared block table, lengths and free list of a paged cache (device tensors)."""
+    block_table: torch.Tensor   # int32 [B, max_blocks]
+    ctx_len: torch.Tensor       # int32 [B]
+    free_list: torch.Tensor     # int32 [num_blocks]
+    free_top: torch.Tensor      # int32 [1]
+    num_blocks: int
+    num_kv_heads: int
+    head_dim: int
+    page_size: int = 16
+
+    @classmethod
+    def from_cache(cls, cache: dict) -> "PagedPool":
+        k0 = cache["k"][0]
+        return cls(cache["block_table"], cache["ctx_len"], cache["free_list"], cache["free_top"],
+                   int(k0.shape[0]), int(k0.shape[2]), int(k0.shape[3]), int(k0.shape[1]))
+
+    def c_struct(self) -> _Pool:
+        for name in ("block_table", "ctx_len", "free_list", "free_top"):
+            _require(getattr(self, name), torch.int32, name)
+        b, mb = self.block_table.shape
+        return _Pool(self.block_table.data_ptr(), self.ctx_len.data_ptr(),
+                     self.free_list.data_ptr(), self.free_top.data_ptr(), int(b), int(mb),
+                     int(self.num_blocks), int(self.page_size), int(self.num_kv_heads),
+                     int(self.head_dim))
+
+
+def new_status(device=None) -> torch.Tensor:
+    """A zeroed device status word."""
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def read_status(status: torch.Tensor) -> int:
+    """Synchronises with the status word's stream and returns its value."""
+    return int(status.item())
+
+
+def kara_workspace_bytes(op: int, pool: PagedPool | None = None, num_seqs: int = 0,
+                         window: int = 0, num_q_heads: int = 0, k_or_budget: int = 0) -> int:
+    ps = ctypes.byref(pool.c_struct()) if pool is not None else None
+    return int(lib().kara_workspace_bytes(op, ps, num_seqs, window, num_q_heads, k_or_budget))
+
+
+def _workspace(nbytes: int, device, workspace):
+    if workspace is not None:
+        return workspace
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def kara_score(q_win: torch.Tensor, k_cache: torch.Tensor, pool: PagedPool, window: int,
+               scale: float | None = None, seq_ids: torch.Tensor | None = None,
+               scores: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+               status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Window scores [R, Hkv, W] fp32 (see kara_score in include/kara.h)."""
+    _require(q_win, torch.bfloat16, "q_win")
+    _require(k_cache, torch.bfloat16, "k_cache")
+    r, w, hq, d = q_win.shape
+    if w != window:
+        raise ValueError("q_win's second dimension must equal the window")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if scores is None:
+        scores = torch.empty((r, pool.num_kv_heads, window), dtype=torch.float32,
+                             device=q_win.device)
+    _require(scores, torch.float32, "scores")
+    if seq_ids is not None:
+        _require(seq_ids, torch.int32, "seq_ids")
+    status = status if status is not None else new_status(q_win.device)
+    ps = pool.c_struct()
+    nbytes = kara_workspace_bytes(OP_SCORE, pool, r, window, hq)
+    ws = _workspace(nbytes, q_win.device, workspace)
+    _check(lib().kara_score(_ptr(q_win), _ptr(k_cache), ctypes.byref(ps), _ptr(seq_ids), r,
+                            window, hq, float(scale), _ptr(scores), _ptr(ws), ws.numel(),
+                            _ptr(status), _stream(stream)), "kara_score")
+    return scores
+
+
+def kara_select(scores: torch.Tensor, k: int, sel: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """Top-k window positions per row, ascending: [..., k] int32."""
+    _require(scores, torch.float32, "scores")
+    w = scores.shape[-1]
+    rows = scores.numel() // w if w else 0
+    if sel is None:
+        sel = torch.empty(scores.shape[:-1] + (k,), dtype=torch.int32, device=scores.device)
+    _require(sel, torch.int32, "sel")
+    _check(lib().kara_select(_ptr(scores), rows, w, k, _ptr(sel), _stream(stream)), "kara_select")
+    return sel
+
+
+def kara_token2chunk(scores: torch.Tensor, sel: torch.Tensor, num_anchors: int, gap_limit: int,
+                     widen: int, keep: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Token2Chunk expansion and trim: [..., k] int32 ascending."""
+    _require(scores, torch.float32, "scores")
+    _require(sel, torch.int32, "sel")
+    w = scores.shape[-1]
+    k = sel.shape[-1]
+    rows = scores.numel() // w if w else 0
+    if keep is None:
+        keep = torch.empty_like(sel)
+    _require(keep, torch.int32, "keep")
+    _check(lib().kara_token2chunk(_ptr(scores), _ptr(sel), rows, w, k, int(num_anchors),
+                                  int(gap_limit), int(widen), _ptr(keep), _stream(stream)),
+           "kara_token2chunk")
+    return keep
+
+
+def _layers(k_layers, v_layers):
+    if len(k_layers) != len(v_layers) or not 1 <= len(k_layers) <= MAX_LAYERS:
+        raise ValueError("k_layers and v_layers must hold 1..128 tensors each")
+    arr = (_LayerKV * len(k_layers))()
+    for i, (k, v) in enumerate(zip(k_layers, v_layers)):
+        _require(k, torch.bfloat16, f"k_layers[{i}]")
+        _require(v, torch.bfloat16, f"v_layers[{i}]")
+        arr[i].k = k.data_ptr()
+        arr[i].v = v.data_ptr()
+    return arr
+
+
+def kara_compact(k_layers, v_layers, pool: PagedPool, window: int, keep: torch.Tensor,
+                 seq_ids: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                 status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Compaction into fresh blocks (in place on the pools and the PagedPool). Returns the
+    status tensor (read it after synchronising)."""
+    _require(keep, torch.int32, "keep")
+    nl, r, hkv, k = keep.shape
+    arr = _layers(k_layers, v_layers)
+    if nl != len(arr):
+        raise ValueError("keep's first dimension must equal the number of layers")
+    if seq_ids is not None:
+        _require(seq_ids, torch.int32, "seq_ids")
+    status = status if status is not None else new_status(keep.device)
+    ps = pool.c_struct()
+    nbytes = kara_workspace_bytes(OP_COMPACT, pool, r, window, 0, k)
+    ws = _workspace(nbytes, keep.device, workspace)
+    _check(lib().kara_compact(arr, nl, ctypes.byref(ps), _ptr(seq_ids), r, window, k, _ptr(keep),
+                              _ptr(ws), ws.numel(), _ptr(status), _stream(stream)),
+           "kara_compact")
+    return status
+
+
+def paged_decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                      pool: PagedPool, scale: float | None = None, out: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """One decode step of paged GQA attention: out [B, Hq, d] bf16."""
+    _require(q, torch.bfloat16, "q")
+    _require(k_cache, torch.bfloat16, "k_cache")
+    _require(v_cache, torch.bfloat16, "v_cache")
+    b, hq, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    _require(out, torch.bfloat16, "out")
+    status = status if status is not None else new_status(q.device)
+    ps = pool.c_struct()
+    nbytes = kara_workspace_bytes(OP_DECODE, pool, 0, 0, hq, 0)
+    ws = _workspace(nbytes, q.device, workspace)
+    _check(lib().paged_decode_attn(_ptr(q), _ptr(k_cache), _ptr(v_cache), ctypes.byref(ps), hq,
+                                   float(scale), _ptr(out), _ptr(ws), ws.numel(), _ptr(status),
+                                   _stream(stream)), "paged_decode_attn")
+    return out
+
+
+def lacache_compact(k_layers, v_layers, pool: PagedPool, span: int, overlap: int, rung: int,
+                    budget: int, sink: int = 0, recent: int = 0,
+                    seq_ids: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                    status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One ladder-compaction pass (in place). Returns the status tensor."""
+    arr = _layers(k_layers, v_layers)
+    device = k_layers[0].device
+    r = int(seq_ids.numel()) if seq_ids is not None else int(pool.block_table.shape[0])
+    if seq_ids is not None:
+        _require(seq_ids, torch.int32, "seq_ids")
+    status = status if status is not None else new_status(device)
+    ps = pool.c_struct()
+    prm = _LacacheParams(span, overlap, rung, budget, sink, recent)
+    nbytes = kara_workspace_bytes(OP_LACACHE, pool, r, 0, 0, budget)
+    ws = _workspace(nbytes, device, workspace)
+    _check(lib().lacache_compact(arr, len(arr), ctypes.byref(ps), _ptr(seq_ids), r,
+                                 ctypes.byref(prm), _ptr(ws), ws.numel(), _ptr(status),
+                                 _stream(stream)), "lacache_compact")
+    return status
+
+
+def anchors_for(anchor_frac: float, k: int) -> int:
+    """ceil(anchor_frac * k) clipped to [0, k]: the num_anchors argument of Token2Chunk."""
+    n = int(math.ceil(round(anchor_frac * k, 9)))
+    return max(0, min(k, n))

@@ -1,0 +1,246 @@
+/*
+ * kara.h - C ABI of libkara, the sm_100a (B200) implementation of Kara's decode-time
+ * sliding-window KV-cache compression and of LaCache's ladder compaction over a paged
+ * (PagedAttention-style) KV cache.
+ *
+ * Sources (web pages; cited by title and section):
+ *  [KARA]  "Kara: Efficient Reasoning LLM Serving via Sliding-Window KV Cache Compression",
+ *          English abstract and "method details".
+ *  [GIST]  gist.science explainer of the same paper (German / Japanese), sections 1
+ *          (two-way attention score), 2 (Token2Chunk), 3 (periodic schedule) and results.
+ *  [LAC]   "LaCache: Ladder-Shaped KV Caching for Efficient Long-Context Modeling of Large
+ *          Language Models" (papercache.org), ladder pattern, hyper-parameters S and O,
+ *          iterative compaction.
+ *
+ * Conventions for every call:
+ *  - All tensor arguments are DEVICE pointers unless a comment says "host". The caller owns
+ *    every buffer; the library keeps no pointer after a call returns. Nothing here allocates
+ *    device memory: scratch space is passed in as `workspace` (size from
+ *    kara_workspace_bytes(), 256-byte aligned).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; 0 = legacy default stream) and
+ *    returns after enqueueing its kernels.
+ *  - The return value reports what the host can check: argument shapes, alignment (16-byte
+ *    aligned tensors), supported sizes, workspace size, and CUDA launch errors
+ *    (KARA_ERR_CUDA). On any non-OK return nothing was enqueued.
+ *  - Errors found on the device (a context shorter than the window, a block id out of range,
+ *    too few free blocks, a bounded wait that ran out) are written to `dev_status`, one int32
+ *    in device memory: the first error wins (later ones do not overwrite it) and the library
+ *    never clears it. Read it after synchronising the stream. A call that finds such an error
+ *    leaves its outputs in the state documented per call and never traps or faults.
+ *  - Layout of the paged cache (one pool per layer, all layers share one block table):
+ *      K, V:         bf16 [num_blocks, page_size, num_kv_heads, head_dim]
+ *      block_table:  int32 [batch, max_blocks_per_seq]; entry p of row b is the block that
+ *                    holds slots [16p, 16p+16) of sequence b, -1 for none
+ *      ctx_len:      int32 [batch], number of cached slots of each sequence
+ *      free_list:    int32 [num_blocks], a stack of free block ids; free_top (int32 [1])
+ *                    entries are valid, the top is free_list[free_top-1]
+ *    page_size must be 16; head_dim 64 or 128; num_q_heads a multiple of num_kv_heads with
+ *    at most 8 query heads per KV head. Query head h reads KV head h / (num_q_heads /
+ *    num_kv_heads).
+ */
+#ifndef KARA_H
+#define KARA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kara_status {
+  KARA_OK = 0,
+  KARA_ERR_INVALID_ARG = 1,   /* bad shape, size, pointer or parameter combination */
+  KARA_ERR_UNSUPPORTED = 2,   /* valid request outside what this build implements */
+  KARA_ERR_OUT_OF_BLOCKS = 3, /* free list holds fewer blocks than the compaction needs */
+  KARA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  KARA_ERR_TIMEOUT = 5,       /* a bounded on-device wait ran out (kernel returned early) */
+  KARA_ERR_WORKSPACE = 6,     /* workspace missing, too small or misaligned */
+  KARA_ERR_BAD_BLOCK = 7      /* a block-table entry out of [0, num_blocks) on the device */
+} kara_status;
+
+/* Device pointers of one layer's pools. */
+typedef struct kara_layer_kv {
+  void* k;   /* bf16 [num_blocks, page_size, num_kv_heads, head_dim] */
+  void* v;   /* bf16, same shape */
+} kara_layer_kv;
+
+/* The shared paged-cache bookkeeping (host struct holding device pointers). */
+typedef struct kara_pool {
+  int32_t* block_table;        /* device int32 [batch, max_blocks_per_seq] */
+  int32_t* ctx_len;            /* device int32 [batch] */
+  int32_t* free_list;          /* device int32 [num_blocks] */
+  int32_t* free_top;           /* device int32 [1] */
+  int32_t batch;
+  int32_t max_blocks_per_seq;
+  int32_t num_blocks;
+  int32_t page_size;           /* must be 16 */
+  int32_t num_kv_heads;
+  int32_t head_dim;            /* 64 or 128 */
+} kara_pool;
+
+/* LaCache ladder parameters ([LAC] "implementation details and key hyper-parameters"). */
+typedef struct kara_lacache_params {
+  int32_t span;     /* S: consecutive layers that keep one rung */
+  int32_t overlap;  /* O: layers shared by neighbouring rungs; stride S-O divides S and L */
+  int32_t rung;     /* slots per rung */
+  int32_t budget;   /* slots every layer keeps after compaction */
+  int32_t sink;     /* leading slots kept in every layer */
+  int32_t recent;   /* trailing slots kept in every layer */
+} kara_lacache_params;
+
+/* Operation ids for kara_workspace_bytes(). */
+typedef enum kara_op {
+  KARA_OP_SCORE = 1,
+  KARA_OP_COMPACT = 2,
+  KARA_OP_DECODE = 3,
+  KARA_OP_LACACHE = 4
+} kara_op;
+
+#define KARA_MAX_LAYERS 128
+#define KARA_MAX_WINDOW 4096
+
+/*
+ * kara_score - bidirectional attention scoring of the compression window ([KARA] abstract:
+ * "bidirectional attention to score and select informative KV pairs in the window"; [GIST]
+ * section 1: a token the current reasoning refers to strongly scores high).
+ *
+ * For due sequence r (cache row b = seq_ids ? seq_ids[r] : r, n = ctx_len[b]) the window is
+ * slots [n-window, n). For KV head g with query heads h = g*G .. g*G+G-1 (G = num_q_heads /
+ * num_kv_heads):
+ *     scores[r][g][j] = sum_h sum_i softmax_j( q_win[r][i][h] . K[slot n-window+j][g] * scale )
+ * over window queries i and keys j, unmasked (every query sees every window key).
+ *
+ *  q_win      bf16 [num_seqs, window, num_q_heads, head_dim]; q_win[r][i] is the query of
+ *             window position i (slot n-window+i), as used by the model's attention.
+ *  k_cache    this layer's K pool (layout above).
+ *  pool       host pointer; block_table and ctx_len are read, nothing is written.
+ *  seq_ids    device int32 [num_seqs] or NULL (row r is cache row r).
+ *  window     1 .. KARA_MAX_WINDOW.      scale  usually 1/sqrt(head_dim).
+ *  scores     fp32 [num_seqs, num_kv_heads, window] (written).
+ *  workspace  >= kara_workspace_bytes(KARA_OP_SCORE, ...): per-query log-sum-exp rows.
+ *  dev_status device int32: KARA_ERR_INVALID_ARG if n < window or n exceeds the table,
+ *             KARA_ERR_BAD_BLOCK for a window block id outside [0, num_blocks),
+ *             KARA_ERR_TIMEOUT if a pipeline wait ran out; the scores of such a sequence are
+ *             then zero or unspecified.
+ */
+kara_status kara_score(const void* q_win, const void* k_cache, const kara_pool* pool,
+                       const int32_t* seq_ids, int32_t num_seqs, int32_t window,
+                       int32_t num_q_heads, float scale, float* scores, void* workspace,
+                       size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * kara_select - keep the k highest-scoring window positions ([KARA] abstract: "select
+ * informative KV pairs"; [GIST] results: about 20 % kept).
+ *
+ * For each of `rows` rows of scores [rows, window]: the k positions with the largest score,
+ * ties broken towards the lower position, written ascending to sel [rows, k] (int32).
+ * -0.0 and +0.0 compare equal; NaN scores are not supported. 1 <= k <= window <=
+ * KARA_MAX_WINDOW.
+ */
+kara_status kara_select(const float* scores, int32_t rows, int32_t window, int32_t k,
+                        int32_t* sel, cudaStream_t stream);
+
+/*
+ * kara_token2chunk - expand part of the selection into flexible-length chunks and trim back
+ * to budget ([KARA] abstract: "Token2Chunk module to expand a subset of selected KV pairs into
+ * chunks"; [GIST] section 2: everything between two important points is kept as one chunk).
+ *
+ * Per row, in window positions: anchors = the num_anchors selected positions with the largest
+ * scores (ties: lower position); every position strictly between two consecutive anchors is
+ * added when there are 1..gap_limit of them; every position within `widen` of an anchor is
+ * added; the union U (which contains sel) is trimmed to the k members with the largest
+ * (priority, score, -position), priority 2 = anchor, 1 = in a run of consecutive U positions
+ * that contains an anchor, 0 = other. keep [rows, k] is written ascending.
+ *  scores fp32 [rows, window]; sel int32 [rows, k] ascending (as from kara_select).
+ *  0 <= num_anchors <= k (callers use ceil(anchor_frac * k)), gap_limit >= 0, widen >= 0.
+ */
+kara_status kara_token2chunk(const float* scores, const int32_t* sel, int32_t rows,
+                             int32_t window, int32_t k, int32_t num_anchors, int32_t gap_limit,
+                             int32_t widen, int32_t* keep, cudaStream_t stream);
+
+/*
+ * kara_compact - write the compressed windows into fresh blocks, rewrite the block table and
+ * free the old window blocks ([KARA] abstract: Kara adapted to PagedAttention).
+ *
+ * For each due sequence r (cache row b), n = ctx_len[b], start = n-window, off = start % 16,
+ * p0 = start / 16: n_new = ceil((off+k)/16) blocks are popped from the free list (sequences in
+ * order r = 0, 1, ...; each takes free_list[top-1], free_list[top-2], ... for pages p0,
+ * p0+1, ...). In every layer and KV head, slot p0*16+t receives the old slot p0*16+t for
+ * t < off, and slot start+t receives the old slot start+keep[l][r][g][t] for t < k. Then
+ * block_table[b][p0 .. p0+n_new) = fresh ids, [p0+n_new, p0+n_old) = -1 with n_old =
+ * ceil((off+window)/16), ctx_len[b] = start+k, and the n_old old window blocks are pushed on
+ * the free list (sequence order, page order). Slots of the fresh blocks past start+k are left
+ * unwritten.
+ *  layers     HOST array of num_layers (1 .. KARA_MAX_LAYERS) pool pointers.
+ *  seq_ids    device int32 [num_seqs], strictly increasing, or NULL (rows 0..num_seqs-1).
+ *  keep       int32 [num_layers, num_seqs, num_kv_heads, k], ascending window positions.
+ *  workspace  >= kara_workspace_bytes(KARA_OP_COMPACT, ...).
+ *  dev_status KARA_ERR_OUT_OF_BLOCKS / KARA_ERR_INVALID_ARG / KARA_ERR_BAD_BLOCK: then no
+ *             pool, table, length or free-list entry is modified.
+ */
+kara_status kara_compact(const kara_layer_kv* layers, int32_t num_layers, const kara_pool* pool,
+                         const int32_t* seq_ids, int32_t num_seqs, int32_t window, int32_t k,
+                         const int32_t* keep, void* workspace, size_t workspace_bytes,
+                         int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * paged_decode_attn - one decode step of grouped-query attention over the (compressed) paged
+ * cache ([KARA] abstract: the kept KV pairs serve subsequent decoding, with PagedAttention).
+ *
+ *     out[b][h] = sum_t softmax_t( q[b][h] . K[t][g(h)] * scale ) V[t][g(h)],  t < ctx_len[b]
+ *  q, out     bf16 [batch, num_q_heads, head_dim] (batch = pool->batch); an empty context
+ *             gives a zero row.
+ *  workspace  >= kara_workspace_bytes(KARA_OP_DECODE, ...): split-KV partial results.
+ *  dev_status KARA_ERR_INVALID_ARG if a context exceeds the table, KARA_ERR_BAD_BLOCK for a
+ *             block id out of range (that block is skipped).
+ */
+kara_status paged_decode_attn(const void* q, const void* k_cache, const void* v_cache,
+                              const kara_pool* pool, int32_t num_q_heads, float scale, void* out,
+                              void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                              cudaStream_t stream);
+
+/*
+ * lacache_compact - one pass of LaCache's ladder compaction ([LAC] ladder pattern and
+ * iterative compaction) through the same paged gather as kara_compact.
+ *
+ * For each due sequence (cache row b, n = ctx_len[b]) and layer l the kept slots are, in
+ * ascending order: slots [0, sink); the ladder region's kept rungs; slots [n-recent, n). The
+ * region is the R_max = (budget-sink-recent)*L/S slots before the recent tail (older slots
+ * are dropped in all layers); it is cut into rungs of `rung` slots and rung j is kept in the
+ * layers (j*(S-O) + t) mod L, t < S. Every layer keeps exactly `budget` slots; slot t of the
+ * compacted sequence holds the t-th kept slot (every KV head of the layer alike). The
+ * sequence moves to ceil(budget/16) fresh blocks (popped as in kara_compact), its ceil(n/16)
+ * old blocks are pushed afterwards, and ctx_len[b] = budget.
+ *  Requirements (host-checked): 1 <= S <= L, 0 <= O < S, (S-O) divides S and L,
+ *  budget-sink-recent > 0 and a multiple of rung*S/(S-O). Device-checked: n >= sink + recent +
+ *  R_max (a full cache), else KARA_ERR_INVALID_ARG and nothing is modified.
+ */
+kara_status lacache_compact(const kara_layer_kv* layers, int32_t num_layers,
+                            const kara_pool* pool, const int32_t* seq_ids, int32_t num_seqs,
+                            const kara_lacache_params* params, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * kara_workspace_bytes - workspace size for one call (0 if the op needs none).
+ *  KARA_OP_SCORE:   num_seqs, window, num_q_heads used.
+ *  KARA_OP_COMPACT: num_seqs, window (the budget k goes in `k_or_budget`).
+ *  KARA_OP_DECODE:  pool->batch, num_q_heads, head_dim, max_blocks_per_seq used.
+ *  KARA_OP_LACACHE: num_seqs, budget in `k_or_budget`.
+ * `pool` is a host pointer (may be NULL for SCORE).
+ */
+size_t kara_workspace_bytes(kara_op op, const kara_pool* pool, int32_t num_seqs, int32_t window,
+                            int32_t num_q_heads, int32_t k_or_budget);
+
+/* Static, human-readable name of a status code. */
+const char* kara_status_str(int32_t status);
+
+/* Library version string ("kara-b200 <major>.<minor>"). */
+const char* kara_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KARA_H */

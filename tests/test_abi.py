@@ -1,0 +1,73 @@
+"""The C-ABI library: it builds, loads without a GPU, exports every declared entry point, and
+rejects bad arguments on the host before touching the device (no compute calls here)."""
+
+import ctypes
+
+import pytest
+
+from decode_kv_cache_kara_b200 import kara as K
+
+
+def test_library_exports_every_declared_symbol(lib_path):
+    names = K.declared_symbols()
+    expected = {"kara_score", "kara_select", "kara_token2chunk", "kara_compact",
+                "paged_decode_attn", "lacache_compact", "kara_workspace_bytes",
+                "kara_status_str", "kara_version"}
+    assert expected <= set(names)
+    handle = ctypes.CDLL(lib_path)
+    for n in names:
+        assert hasattr(handle, n), n
+
+
+def test_status_strings_and_version(lib_path):
+    assert K.status_str(0) == "ok"
+    assert "free blocks" in K.status_str(K.ERR_OUT_OF_BLOCKS)
+    assert K.lib().kara_version().decode().startswith("kara-b200")
+
+
+def test_host_side_validation_returns_before_any_launch(lib_path):
+    L = K.lib()
+    null = ctypes.c_void_p(0)
+    # k > window, window too large, rows < 0
+    assert L.kara_select(null, 4, 16, 17, null, null) == K.ERR_INVALID_ARG
+    assert L.kara_select(null, 4, 5000, 8, null, null) == K.ERR_INVALID_ARG
+    assert L.kara_select(null, 0, 16, 4, null, null) == K.OK          # empty input
+    # more anchors than kept tokens
+    assert L.kara_token2chunk(null, null, 1, 16, 4, 5, 8, 1, null, null) == K.ERR_INVALID_ARG
+    # page size other than 16, head_dim other than 64/128
+    pool = K._Pool(1, 1, 1, 1, 1, 8, 64, 8, 2, 128)
+    assert L.paged_decode_attn(null, null, null, ctypes.byref(pool), 4, 1.0, null, null, 0, null,
+                               null) == K.ERR_UNSUPPORTED
+    pool = K._Pool(1, 1, 1, 1, 1, 8, 64, 16, 2, 96)
+    assert L.kara_score(null, null, ctypes.byref(pool), null, 1, 16, 4, 1.0, null, null, 0, null,
+                        null) == K.ERR_UNSUPPORTED
+    # more than 8 query heads per KV head
+    pool = K._Pool(1, 1, 1, 1, 1, 8, 64, 16, 2, 128)
+    assert L.kara_score(null, null, ctypes.byref(pool), null, 1, 16, 18, 1.0, null, null, 0, null,
+                        null) == K.ERR_UNSUPPORTED
+    # workspace missing
+    one = ctypes.c_void_p(256)
+    assert L.kara_score(one, one, ctypes.byref(pool), null, 1, 16, 4, 1.0, one, null, 0, one,
+                        null) == K.ERR_WORKSPACE
+    # LaCache: stride S-O must divide S and L
+    prm = K._LacacheParams(3, 1, 4, 64, 0, 0)
+    layers = (K._LayerKV * 8)()
+    assert L.lacache_compact(layers, 8, ctypes.byref(pool), null, 1, ctypes.byref(prm), null, 0,
+                             one, null) == K.ERR_INVALID_ARG
+
+
+def test_workspace_sizes(lib_path):
+    pool = K._Pool(1, 1, 1, 1, 32, 257, 9000, 16, 4, 128)
+    score = K.lib().kara_workspace_bytes(K.OP_SCORE, None, 32, 1000, 28, 0)
+    assert score == 32 * 28 * 1024 * 4                # rows padded to 256 queries
+    dec = K.lib().kara_workspace_bytes(K.OP_DECODE, ctypes.byref(pool), 0, 0, 28, 0)
+    assert dec == 32 * 28 * 17 * 130 * 4              # 17 splits of 16 pages, d + 2 floats
+    comp = K.lib().kara_workspace_bytes(K.OP_COMPACT, None, 32, 1024, 0, 204)
+    assert comp == (16 + 32 * 12 + 32 * 14) * 4
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(K, "_LIB", None)
+    monkeypatch.setattr(K, "library_path", lambda: str(tmp_path / "nope.so"))
+    with pytest.raises(K.KaraLibraryError):
+        K.lib()

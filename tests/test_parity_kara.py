@@ -1,0 +1,274 @@
+"""GPU parity of the Kara path (score, select, Token2Chunk, compaction) against the oracle.
+
+Scores: |gpu - oracle| <= 1e-3 |oracle| + 1e-6 (bf16 inputs, fp32 accumulation; the 1e-6 floor
+covers terms the GPU's fp32 exponential flushes below 2^-126). Selection: identical sets given
+identical scores; against oracle scores, sets equal except at near-ties (1e-3 relative).
+Token2Chunk: identical given identical inputs. Compaction: bit-exact given the same keep.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from decode_kv_cache_kara_b200 import kara as K
+from decode_kv_cache_kara_b200 import synth
+from oracle import kara as ok
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+LAYER = synth.WORKLOADS["layer"]
+SCORE_CASES = {
+    "tiny": synth.WORKLOADS["tiny"],
+    "g7_aligned": LAYER.with_(batch=3, ctx_lo=1024, ctx_hi=1024, window=256, keep=52),
+    "g7_ragged_unaligned": LAYER.with_(batch=4, ctx_lo=300, ctx_hi=700, window=200, keep=40),
+    "g7_w1024_unaligned": LAYER.with_(batch=2, ctx_lo=1030, ctx_hi=1400, window=1024, keep=204),
+    "d64_g1": synth.Workload("d64_g1", batch=2, layers=1, hq=4, hkv=4, head_dim=64, ctx_lo=140,
+                             ctx_hi=180, window=130, keep=26, heavy_frac=0.05, q_mode="neighbour",
+                             spare_blocks=8),
+    "g8_w384": synth.Workload("g8_w384", batch=2, layers=1, hq=16, hkv=2, head_dim=128,
+                              ctx_lo=384, ctx_hi=500, window=384, keep=77, heavy_frac=0.03,
+                              run_hi=16, q_mode="neighbour", spare_blocks=8),
+    "w16_ctx_eq_w": synth.Workload("w16", batch=3, layers=1, hq=2, hkv=1, head_dim=128,
+                                   ctx_lo=16, ctx_hi=16, window=16, keep=1, spare_blocks=4),
+}
+
+
+def oracle_scores(cpu, wl, seq_ids=None):
+    seq_ids = list(range(wl.batch)) if seq_ids is None else seq_ids
+    q = H.f64(cpu["q_win"][0])
+    if len(seq_ids) != wl.batch:
+        q = q[seq_ids]
+    return ok.score_batch(q, H.f64(cpu["k"][0]), H.i32(cpu["block_table"]), H.i32(cpu["ctx_len"]),
+                          seq_ids, wl.window, 1 / math.sqrt(wl.head_dim), wl.page)
+
+
+@pytest.mark.parametrize("name", list(SCORE_CASES))
+def test_score_matches_oracle(name):
+    wl = SCORE_CASES[name]
+    cpu, dev = H.make(wl, 11)
+    pool = K.PagedPool.from_cache(dev)
+    status = K.new_status()
+    scores = K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window, status=status)
+    torch.cuda.synchronize()
+    assert K.read_status(status) == 0
+    ref = oracle_scores(cpu, wl)
+    H.assert_scores_close(H.f64(scores), ref)
+    # invariant at any size: every row of scores sums to W * G
+    sums = scores.double().sum(-1).cpu().numpy()
+    assert np.allclose(sums, wl.window * wl.group, rtol=1e-4)
+
+
+def test_score_subset_of_sequences():
+    wl = SCORE_CASES["g7_ragged_unaligned"]
+    cpu, dev = H.make(wl, 5)
+    ids = [1, 3]
+    pool = K.PagedPool.from_cache(dev)
+    q = dev["q_win"][0][ids].contiguous()
+    seq = torch.tensor(ids, dtype=torch.int32, device="cuda")
+    scores = K.kara_score(q, dev["k"][0], pool, wl.window, seq_ids=seq)
+    torch.cuda.synchronize()
+    H.assert_scores_close(H.f64(scores), oracle_scores(cpu, wl, ids))
+
+
+def test_score_reports_short_context():
+    wl = SCORE_CASES["g7_aligned"]
+    cpu, dev = H.make(wl, 2)
+    dev["ctx_len"][1] = wl.window - 1
+    pool = K.PagedPool.from_cache(dev)
+    status = K.new_status()
+    scores = K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window, status=status)
+    torch.cuda.synchronize()
+    assert K.read_status(status) == K.ERR_INVALID_ARG
+    assert (scores[1] == 0).all()
+    cpu["ctx_len"][1] = wl.window - 1
+    ref = oracle_scores(cpu, wl, [0, 2])
+    H.assert_scores_close(H.f64(scores[[0, 2]]), ref)
+
+
+@pytest.mark.parametrize("name", ["tiny", "g7_ragged_unaligned", "g8_w384", "w16_ctx_eq_w"])
+def test_select_and_token2chunk(name):
+    wl = SCORE_CASES[name]
+    cpu, dev = H.make(wl, 21)
+    pool = K.PagedPool.from_cache(dev)
+    scores = K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window)
+    sel = K.kara_select(scores, wl.keep)
+    na = K.anchors_for(wl.anchor_frac, wl.keep)
+    keep = K.kara_token2chunk(scores, sel, na, wl.gap_limit, wl.widen)
+    torch.cuda.synchronize()
+    s_gpu = H.f64(scores)
+    # identical inputs -> identical outputs
+    assert np.array_equal(H.i32(sel), ok.select_batch(s_gpu, wl.keep))
+    assert np.array_equal(H.i32(keep), ok.token2chunk_batch(s_gpu, H.i32(sel), na, wl.gap_limit,
+                                                            wl.widen))
+    # against the oracle's own scores: equal up to near-ties
+    ref = oracle_scores(cpu, wl)
+    H.assert_selection_matches(H.i32(sel), ok.select_batch(ref, wl.keep), ref)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_select_ties_and_token2chunk_params(seed):
+    rng = np.random.default_rng(seed)
+    rows, w = 7, int(rng.integers(16, 2049))
+    k = int(rng.integers(1, w + 1))
+    # coarse values force many exact ties; include -0.0 and +0.0
+    s = rng.integers(0, 5, size=(rows, w)).astype(np.float32) * 0.25
+    s[0, :8] = -0.0
+    scores = torch.from_numpy(s).cuda()
+    sel = K.kara_select(scores, k)
+    na = int(rng.integers(0, k + 1))
+    gap = int(rng.integers(0, 12))
+    wid = int(rng.integers(0, 4))
+    keep = K.kara_token2chunk(scores, sel, na, gap, wid)
+    torch.cuda.synchronize()
+    assert np.array_equal(H.i32(sel), ok.select_batch(s.astype(np.float64), k))
+    assert np.array_equal(H.i32(keep), ok.token2chunk_batch(s.astype(np.float64), H.i32(sel), na,
+                                                            gap, wid))
+
+
+def test_select_max_window_and_k_equals_w():
+    rng = np.random.default_rng(3)
+    s = rng.random((3, 4096)).astype(np.float32)
+    scores = torch.from_numpy(s).cuda()
+    for k in (1, 819, 4096):
+        sel = K.kara_select(scores, k)
+        torch.cuda.synchronize()
+        assert np.array_equal(H.i32(sel), ok.select_batch(s.astype(np.float64), k))
+
+
+# ---------------------------------------------------------------- compaction
+
+def oracle_compact(cpu, wl, keep, seq_ids, layers):
+    return ok.compact([H.bits(cpu["k"][i]) for i in range(layers)],
+                      [H.bits(cpu["v"][i]) for i in range(layers)],
+                      H.i32(cpu["block_table"]), H.i32(cpu["ctx_len"]), H.i32(cpu["free_list"]),
+                      int(cpu["free_top"][0]), seq_ids, wl.window, keep, wl.page)
+
+
+def check_compaction(dev, ref, layers, seq_ids, batch):
+    st, kp, vp, bt, cl, fl, top, fresh = ref
+    assert st == ok.OK
+    assert np.array_equal(H.i32(dev["block_table"]), bt)
+    assert np.array_equal(H.i32(dev["ctx_len"]), cl)
+    assert int(dev["free_top"][0]) == top
+    assert np.array_equal(H.i32(dev["free_list"])[:top], fl[:top])
+    for layer in range(layers):
+        kg, vg = H.bits(dev["k"][layer]), H.bits(dev["v"][layer])
+        for b in range(batch):
+            n = int(cl[b])
+            assert np.array_equal(H.logical_rows(kg, bt[b], n), H.logical_rows(kp[layer], bt[b], n))
+            assert np.array_equal(H.logical_rows(vg, bt[b], n), H.logical_rows(vp[layer], bt[b], n))
+        touched = set(x for ids in fresh.values() for x in ids)
+        untouched = np.array(sorted(set(range(kg.shape[0])) - touched))
+        assert np.array_equal(kg[untouched], kp[layer][untouched])
+        assert np.array_equal(vg[untouched], vp[layer][untouched])
+
+
+@pytest.mark.parametrize("name,layers,subset", [("tiny", 1, None), ("g7_ragged_unaligned", 3, None),
+                                                ("g7_ragged_unaligned", 2, [0, 2, 3]),
+                                                ("d64_g1", 2, [1]), ("w16_ctx_eq_w", 1, None)])
+def test_compact_bit_exact(name, layers, subset):
+    wl = SCORE_CASES[name]
+    cpu, dev = H.make(wl, 31, layers=layers)
+    seq_ids = list(range(wl.batch)) if subset is None else subset
+    rng = np.random.default_rng(9)
+    keep = np.stack([synth.random_keep(rng, len(seq_ids) * wl.hkv, wl.window, wl.keep)
+                     .reshape(len(seq_ids), wl.hkv, wl.keep) for _ in range(layers)])
+    ref = oracle_compact(cpu, wl, keep, seq_ids, layers)
+    pool = K.PagedPool.from_cache(dev)
+    sid = None if subset is None else torch.tensor(subset, dtype=torch.int32, device="cuda")
+    status = K.kara_compact(dev["k"], dev["v"], pool, wl.window,
+                            torch.from_numpy(keep).cuda(), seq_ids=sid)
+    torch.cuda.synchronize()
+    assert K.read_status(status) == 0
+    check_compaction(dev, ref, layers, seq_ids, wl.batch)
+
+
+def test_compact_keep_all_window():
+    wl = SCORE_CASES["g7_ragged_unaligned"].with_(keep=200)
+    cpu, dev = H.make(wl, 8)
+    keep = np.tile(np.arange(wl.window, dtype=np.int32), (1, wl.batch, wl.hkv, 1))
+    ref = oracle_compact(cpu, wl, keep, list(range(wl.batch)), 1)
+    pool = K.PagedPool.from_cache(dev)
+    K.kara_compact(dev["k"], dev["v"], pool, wl.window, torch.from_numpy(keep).cuda())
+    torch.cuda.synchronize()
+    check_compaction(dev, ref, 1, list(range(wl.batch)), wl.batch)
+
+
+def test_compact_out_of_blocks_changes_nothing():
+    wl = SCORE_CASES["g7_ragged_unaligned"]
+    cpu, dev = H.make(wl, 4)
+    dev["free_top"][0] = 2
+    before = {k: dev[k].clone() for k in ("block_table", "ctx_len", "free_list", "free_top")}
+    kb = dev["k"][0].clone()
+    keep = np.tile(np.arange(wl.keep, dtype=np.int32), (1, wl.batch, wl.hkv, 1))
+    pool = K.PagedPool.from_cache(dev)
+    status = K.kara_compact(dev["k"], dev["v"], pool, wl.window, torch.from_numpy(keep).cuda())
+    torch.cuda.synchronize()
+    assert K.read_status(status) == K.ERR_OUT_OF_BLOCKS
+    for k, t in before.items():
+        assert torch.equal(dev[k], t)
+    assert torch.equal(dev["k"][0], kb)
+
+
+def test_compact_bad_block_id_is_reported_not_faulted():
+    wl = SCORE_CASES["g7_ragged_unaligned"]
+    cpu, dev = H.make(wl, 4)
+    n = int(cpu["ctx_len"][1])
+    dev["block_table"][1, (n - 1) // 16] = 10 ** 8
+    keep = np.tile(np.arange(wl.keep, dtype=np.int32), (1, wl.batch, wl.hkv, 1))
+    pool = K.PagedPool.from_cache(dev)
+    status = K.kara_compact(dev["k"], dev["v"], pool, wl.window, torch.from_numpy(keep).cuda())
+    scores_status = K.new_status()
+    K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window, status=scores_status)
+    torch.cuda.synchronize()
+    assert K.read_status(status) == K.ERR_BAD_BLOCK
+    assert K.read_status(scores_status) == K.ERR_BAD_BLOCK
+
+
+def test_compact_reuses_freed_blocks():
+    # A second compaction, after appending W tokens to each sequence, pops blocks the first
+    # one freed (block free and reuse).
+    wl = SCORE_CASES["g7_ragged_unaligned"].with_(spare_blocks=32)
+    cpu, dev = H.make(wl, 17)
+    rng = np.random.default_rng(2)
+    keep1 = synth.random_keep(rng, wl.batch * wl.hkv, wl.window, wl.keep).reshape(
+        1, wl.batch, wl.hkv, wl.keep)
+    ref1 = oracle_compact(cpu, wl, keep1, list(range(wl.batch)), 1)
+    pool = K.PagedPool.from_cache(dev)
+    K.kara_compact(dev["k"], dev["v"], pool, wl.window, torch.from_numpy(keep1).cuda())
+    torch.cuda.synchronize()
+    check_compaction(dev, ref1, 1, list(range(wl.batch)), wl.batch)
+    _, kp, vp, bt, cl, fl, top, fresh1 = ref1
+    old_table = H.i32(cpu["block_table"])
+    freed1 = set(old_table[old_table >= 0].tolist()) - set(bt[bt >= 0].tolist())
+    assert freed1 and freed1 <= set(fl[:top].tolist())
+    # append W slots per sequence on the host state, taking blocks from the free list top
+    # (the table gets room for the longer sequences)
+    bt = np.pad(bt, ((0, 0), (0, wl.window // 16 + 2)), constant_values=-1)
+    cl, fl = cl.copy(), fl.copy()
+    for b in range(wl.batch):
+        n = int(cl[b])
+        for p in range(n // 16 + (1 if n % 16 else 0), (n + wl.window + 15) // 16):
+            top -= 1
+            bt[b, p] = fl[top]
+        cl[b] = n + wl.window
+    cpu2 = dict(cpu)
+    cpu2["k"] = [torch.from_numpy(kp[0]).view(torch.bfloat16)]
+    cpu2["v"] = [torch.from_numpy(vp[0]).view(torch.bfloat16)]
+    cpu2["block_table"] = torch.from_numpy(bt.astype(np.int32))
+    cpu2["ctx_len"] = torch.from_numpy(cl.astype(np.int32))
+    cpu2["free_list"] = torch.from_numpy(fl.astype(np.int32))
+    cpu2["free_top"] = torch.tensor([top], dtype=torch.int32)
+    dev2 = H.to_device(cpu2)
+    keep2 = synth.random_keep(rng, wl.batch * wl.hkv, wl.window, wl.keep).reshape(
+        1, wl.batch, wl.hkv, wl.keep)
+    ref2 = oracle_compact(cpu2, wl, keep2, list(range(wl.batch)), 1)
+    pool2 = K.PagedPool.from_cache(dev2)
+    K.kara_compact(dev2["k"], dev2["v"], pool2, wl.window, torch.from_numpy(keep2).cuda())
+    torch.cuda.synchronize()
+    check_compaction(dev2, ref2, 1, list(range(wl.batch)), wl.batch)
+    used2 = set(x for ids in ref2[7].values() for x in ids) | set(bt[bt >= 0].ravel().tolist())
+    assert used2 & freed1, "the second pass should reuse blocks the first one freed"
