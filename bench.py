@@ -354,7 +354,8 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
             v["frac_of_hbm_" + src] = v["gbs"] / peaks["hbm_gbs"]
         elif v["bound"] == "tensor":
             v["frac_of_bf16_" + src] = v["useful_tflops"] / peaks["bf16_tflops"]
-    dom = max(kernels, key=lambda k: kernels[k]["ms"])
+    dom = max((k for k in kernels if kernels[k]["bound"] in ("tensor", "hbm")),
+              key=lambda k: kernels[k]["ms"])
     dk = kernels[dom]
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")

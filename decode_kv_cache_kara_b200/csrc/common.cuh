@@ -147,6 +147,14 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Ties N registers filled by tcgen05.ld to a point after tcgen05.wait::ld, so that no use of
+// them is scheduled before the wait (the asm outputs alone do not order them).
+template <int N>
+__device__ __forceinline__ void reg_fence(float* v) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
+}
+
 // 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
@@ -165,7 +173,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 }
 
 // 16 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   uint32_t r[16];
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -202,12 +210,55 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Exponentials: base-2, through the SFU.
+// Exponentials, base 2.
 // ---------------------------------------------------------------------------------------
+// Through the SFU (MUFU.EX2).
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// On the FMA pipe, so that part of the exponentials leaves the SFU: x = n + f with
+// n = round-to-nearest(x) (adding and subtracting 1.5 * 2^23 leaves n in the low mantissa
+// bits of the sum), f in [-1/2, 1/2]; 2^f by a degree-4 polynomial fitted for minimum
+// maximum relative error (csrc/gen_exp2_poly.py); 2^n by adding n to the exponent field,
+// which is (bits of the shifted sum) << 23 because the shifter's own bits vanish modulo 2^32.
+// Inputs below -125 are clamped (result ~2^-125 instead of a denormal or 0). Maximum
+// relative error over [-125, 0]: 2.7e-6.
+__device__ __forceinline__ float ex2_fma(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float n = t - 12582912.0f;
+  const float f = x - n;
+  float p = fmaf(0.009570102207362652f, f, 0.05591785907745361f);
+  p = fmaf(p, f, 0.240247443318367f);
+  p = fmaf(p, f, 0.6931217908859253f);
+  p = fmaf(p, f, 0.9999992847442627f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Packed fp32 pair arithmetic (one instruction for two lanes of work on sm_100).
+__device__ __forceinline__ uint64_t f2_bits(float2 a) { return *reinterpret_cast<uint64_t*>(&a); }
+__device__ __forceinline__ float2 bits_f2(uint64_t r) { return *reinterpret_cast<float2*>(&r); }
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return bits_f2(r);
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(r);
+}
+// Both bf16 halves of a packed word as an fp32 pair (exact).
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Named barrier among `count` threads (id 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }

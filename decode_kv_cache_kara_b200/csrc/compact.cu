@@ -74,6 +74,17 @@ struct PlanParams {
   int W, k, lacache, min_len;
 };
 
+// Row r of the plan whose [base_old, base_old + n_old) range holds flat page index i.
+__device__ __forceinline__ int plan_row_of(const int32_t* rows, int R, int i) {
+  int lo = 0, hi = R - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (rows[static_cast<size_t>(mid) * kPlanStride + P_BOLD] <= i) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) {
   __shared__ int buf[33];
   __shared__ int err;
@@ -83,6 +94,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
   int32_t* fresh = rows + static_cast<size_t>(p.R) * kPlanStride;
   if (threadIdx.x == 0) { err = 0; carry_new = 0; carry_old = 0; }
   __syncthreads();
+  // 1. geometry of every due sequence, exclusive scans of its fresh / old page counts
   for (int base = 0; base < p.R; base += kPlanThreads) {
     const int r = base + threadIdx.x;
     int n_new = 0, n_old = 0;
@@ -105,12 +117,6 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
           p0 = start / 16;
           n_old = (off + p.W + 15) / 16;
           n_new = (off + p.k + 15) / 16;
-        }
-      }
-      if (!code) {
-        for (int i = 0; i < n_old; ++i) {
-          const int blk = p.block_table[static_cast<size_t>(b) * p.max_blocks + p0 + i];
-          if (blk < 0 || blk >= p.num_blocks) { code = KARA_ERR_BAD_BLOCK; break; }
         }
       }
       if (code) {
@@ -138,6 +144,16 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
     if (threadIdx.x == 0) { carry_new += tot_new; carry_old += tot_old; }
     __syncthreads();
   }
+  // 2. every old page id of every due sequence must be a valid block (flat loop over pages)
+  const int total_old = carry_old;
+  for (int i = threadIdx.x; i < total_old; i += kPlanThreads) {
+    const int r = plan_row_of(rows, p.R, i);
+    const int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
+    const int blk = p.block_table[static_cast<size_t>(row[P_B]) * p.max_blocks + row[P_P0] +
+                                  (i - row[P_BOLD])];
+    if (blk < 0 || blk >= p.num_blocks) atomicCAS(&err, 0, KARA_ERR_BAD_BLOCK);
+  }
+  __syncthreads();
   const int top = *p.free_top;
   if (threadIdx.x == 0) {
     int code = err;
@@ -154,6 +170,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
   }
   __syncthreads();
   if (err) return;
+  // 3. pop the fresh blocks (sequence order, stack top first)
   for (int i = threadIdx.x; i < carry_new; i += kPlanThreads) fresh[i] = p.free_list[top - 1 - i];
 }
 
@@ -166,6 +183,7 @@ struct FinalizeParams {
   int R, max_blocks, k;   // k: kept slots (Kara) or budget (LaCache)
 };
 
+// One thread per old page: table entry -> fresh id or -1, old id -> free list.
 __global__ void __launch_bounds__(256) finalize_kernel(const FinalizeParams p) {
   const int32_t* hdr = p.plan;
   if (hdr[0] != 1) return;
@@ -173,18 +191,17 @@ __global__ void __launch_bounds__(256) finalize_kernel(const FinalizeParams p) {
   const int32_t* fresh = rows + static_cast<size_t>(p.R) * kPlanStride;
   const int total_new = hdr[1], total_old = hdr[2], top = hdr[3];
   const int push_base = top - total_new;
-  for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total_old; i += gridDim.x * blockDim.x) {
+    const int r = plan_row_of(rows, p.R, i);
     const int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
-    const int b = row[P_B], p0 = row[P_P0], n_old = row[P_NOLD], n_new = row[P_NNEW];
-    int32_t* tab = p.block_table + static_cast<size_t>(b) * p.max_blocks;
-    for (int i = 0; i < n_old; ++i) {
-      const int old = tab[p0 + i];
-      tab[p0 + i] = i < n_new ? fresh[row[P_BNEW] + i] : -1;
-      p.free_list[push_base + row[P_BOLD] + i] = old;
-    }
-    p.ctx_len[b] = row[P_START] + p.k;
+    const int pg = i - row[P_BOLD];
+    int32_t* entry = p.block_table + static_cast<size_t>(row[P_B]) * p.max_blocks + row[P_P0] + pg;
+    const int old = *entry;
+    *entry = pg < row[P_NNEW] ? fresh[row[P_BNEW] + pg] : -1;
+    p.free_list[push_base + i] = old;
+    if (pg == 0) p.ctx_len[row[P_B]] = row[P_START] + p.k;
   }
-  if (threadIdx.x == 0) *p.free_top = push_base + total_old;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.free_top = push_base + total_old;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -412,7 +429,7 @@ kara_status launch_compact(const CompactLaunch& L, cudaStream_t stream) {
   fp.R = L.R;
   fp.max_blocks = L.max_blocks;
   fp.k = L.k;
-  finalize_kernel<<<1, 256, 0, stream>>>(fp);
+  finalize_kernel<<<8, 256, 0, stream>>>(fp);
   return cudaGetLastError() == cudaSuccess ? KARA_OK : KARA_ERR_CUDA;
 }
 
@@ -462,7 +479,7 @@ kara_status launch_lacache(const LacacheLaunch& L, cudaStream_t stream) {
   fp.R = L.R;
   fp.max_blocks = L.max_blocks;
   fp.k = L.budget;
-  finalize_kernel<<<1, 256, 0, stream>>>(fp);
+  finalize_kernel<<<8, 256, 0, stream>>>(fp);
   return cudaGetLastError() == cudaSuccess ? KARA_OK : KARA_ERR_CUDA;
 }
 

@@ -37,13 +37,6 @@ struct DecodeArgs {
   float cs;            // scale * log2(e)
 };
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
-  f[0] = bf16lo_to_f32(u.x); f[1] = bf16hi_to_f32(u.x);
-  f[2] = bf16lo_to_f32(u.y); f[3] = bf16hi_to_f32(u.y);
-  f[4] = bf16lo_to_f32(u.z); f[5] = bf16hi_to_f32(u.z);
-  f[6] = bf16lo_to_f32(u.w); f[7] = bf16hi_to_f32(u.w);
-}
-
 template <int D, int G>
 __global__ void __launch_bounds__(kDecThreads)
 decode_split_kernel(const DecodeArgs a) {
@@ -79,13 +72,14 @@ decode_split_kernel(const DecodeArgs a) {
   }
   __syncthreads();
 
-  float m[G], l[G], acc[G][kCh];
+  float m[G], l[G];
+  float2 acc[G][kCh / 2];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     m[h] = -INFINITY;
     l[h] = 0.f;
 #pragma unroll
-    for (int c = 0; c < kCh; ++c) acc[h][c] = 0.f;
+    for (int c = 0; c < kCh / 2; ++c) acc[h][c] = make_float2(0.f, 0.f);
   }
 
   const int slot = lane >> 1, half = lane & 1;
@@ -124,29 +118,30 @@ decode_split_kernel(const DecodeArgs a) {
         for (int c = 0; c < kCh / 2; ++c) vr[s][c] = 0u;
       }
     }
-    // q . k for this lane's slot and half of d
-    float dot[G];
+    // q . k for this lane's slot and half of d, as pairs of partial sums
+    float2 dot2[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) dot[h] = 0.f;
+    for (int h = 0; h < G; ++h) dot2[h] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < kVec; ++i) {
-      float kf[8];
-      bf16x8_to_f32(kr[i], kf);
+      const float2 k01 = bf16x2_to_f2(kr[i].x), k23 = bf16x2_to_f2(kr[i].y);
+      const float2 k45 = bf16x2_to_f2(kr[i].z), k67 = bf16x2_to_f2(kr[i].w);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float4 qa = *reinterpret_cast<const float4*>(&q_s[h][2 * i][half][0]);
         const float4 qb = *reinterpret_cast<const float4*>(&q_s[h][2 * i + 1][half][0]);
-        float d0 = dot[h];
-        d0 = fmaf(kf[0], qa.x, d0); d0 = fmaf(kf[1], qa.y, d0);
-        d0 = fmaf(kf[2], qa.z, d0); d0 = fmaf(kf[3], qa.w, d0);
-        d0 = fmaf(kf[4], qb.x, d0); d0 = fmaf(kf[5], qb.y, d0);
-        d0 = fmaf(kf[6], qb.z, d0); d0 = fmaf(kf[7], qb.w, d0);
-        dot[h] = d0;
+        float2 d = dot2[h];
+        d = ffma2(k01, make_float2(qa.x, qa.y), d);
+        d = ffma2(k23, make_float2(qa.z, qa.w), d);
+        d = ffma2(k45, make_float2(qb.x, qb.y), d);
+        d = ffma2(k67, make_float2(qb.z, qb.w), d);
+        dot2[h] = d;
       }
     }
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      float d = dot[h] + __shfl_xor_sync(0xffffffffu, dot[h], 1);
+      float d = dot2[h].x + dot2[h].y;
+      d += __shfl_xor_sync(0xffffffffu, d, 1);
       if (slot >= valid) d = -INFINITY;
       float pm = d;
 #pragma unroll
@@ -160,25 +155,24 @@ decode_split_kernel(const DecodeArgs a) {
       l[h] = l[h] * corr + ps;
       m[h] = m_new;
 #pragma unroll
-      for (int c = 0; c < kCh; ++c) acc[h][c] *= corr;
+      for (int c = 0; c < kCh / 2; ++c) acc[h][c] = fmul2(acc[h][c], make_float2(corr, corr));
       if (half == 0) p_s[warp][slot][h] = pr;
     }
     __syncwarp();
     // p . v
 #pragma unroll
     for (int s = 0; s < 16; ++s) {
-      float vf[kCh];
-      if constexpr (kCh == 4) {
-        vf[0] = bf16lo_to_f32(vr[s][0]); vf[1] = bf16hi_to_f32(vr[s][0]);
-        vf[2] = bf16lo_to_f32(vr[s][1]); vf[3] = bf16hi_to_f32(vr[s][1]);
-      } else {
-        vf[0] = bf16lo_to_f32(vr[s][0]); vf[1] = bf16hi_to_f32(vr[s][0]);
-      }
+      float2 vf[kCh / 2];
+#pragma unroll
+      for (int c = 0; c < kCh / 2; ++c) vf[c] = bf16x2_to_f2(vr[s][c]);
+      const float4 p0 = *reinterpret_cast<const float4*>(&p_s[warp][s][0]);
+      const float4 p1 = *reinterpret_cast<const float4*>(&p_s[warp][s][4]);
+      const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float pr = p_s[warp][s][h];
+        const float2 pp = make_float2(pv[h], pv[h]);
 #pragma unroll
-        for (int c = 0; c < kCh; ++c) acc[h][c] = fmaf(pr, vf[c], acc[h][c]);
+        for (int c = 0; c < kCh / 2; ++c) acc[h][c] = ffma2(pp, vf[c], acc[h][c]);
       }
     }
     __syncwarp();
@@ -192,7 +186,10 @@ decode_split_kernel(const DecodeArgs a) {
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int c = 0; c < kCh; ++c) red_o[warp][h][lane * kCh + c] = acc[h][c];
+    for (int c = 0; c < kCh / 2; ++c) {
+      red_o[warp][h][lane * kCh + 2 * c] = acc[h][c].x;
+      red_o[warp][h][lane * kCh + 2 * c + 1] = acc[h][c].y;
+    }
   __syncthreads();
   for (int i = threadIdx.x; i < G * (D + 2); i += kDecThreads) {
     const int h = i / (D + 2), c = i % (D + 2);

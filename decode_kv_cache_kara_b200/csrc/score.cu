@@ -9,7 +9,8 @@
 // section 1: a token the current reasoning refers to strongly scores high).
 //
 // Two passes, both persistent and warp-specialised (warp 0: TMA producer, warp 1: UMMA
-// issuer and TMEM owner, warps 2-5: epilogue, one TMEM lane per thread):
+// issuer and TMEM owner, warps 2-9: epilogue, one TMEM lane per thread and two warps per lane
+// quadrant, each on half of the accumulator columns):
 //   pass 1 (query-major)  S = Q K^T, 128 query rows x up to 256 keys per UMMA tile; each
 //                         epilogue thread owns one query row and keeps an online base-2
 //                         log-sum-exp; the result goes to the workspace.
@@ -19,6 +20,8 @@
 // (TMA box of one page and one KV head); slots outside [n-W, n) are masked in the epilogue.
 // Queries come from the dense window-query buffer [R, W, Hq, d]; rows past W are zero-filled
 // by TMA and carry lse = +inf, so they add nothing in pass 2.
+// The epilogues are bound by exponentials: about a third of them run on the FMA pipe
+// (ex2_fma) and the rest on the SFU, so that both pipes share the load.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -32,7 +35,9 @@ namespace kara {
 
 namespace {
 
-constexpr int kThreads = 192;        // 6 warps
+constexpr int kThreads = 320;        // warp 0: TMA, warp 1: UMMA + TMEM, warps 2-9: epilogue
+constexpr int kEpiThreads = 256;
+constexpr uint32_t kEpiBarrier = 1;  // named barrier among the epilogue warps
 constexpr int kQRows1 = 128;         // pass 1: query rows per tile (UMMA M)
 constexpr int kKRows1 = 256;         // pass 1: max keys per UMMA (N)
 constexpr int kKStages1 = 2;
@@ -41,6 +46,16 @@ constexpr int kQRows2 = 256;         // pass 2: queries per UMMA (N)
 constexpr int kQStages2 = 2;
 constexpr int kRowBytes = 128;       // one 64-element bf16 K-chunk row (128-byte swizzle)
 constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
+
+// Column i of every 64-column group takes the FMA-pipe exponential when this holds (about a
+// third of the columns), the SFU one otherwise: the two pipes then finish together.
+__device__ __forceinline__ constexpr bool fma_exp_column(int i) { return i % 3 == 1; }
+
+template <int I>
+__device__ __forceinline__ float exp2_split(float x) {
+  if constexpr (fma_exp_column(I)) return ex2_fma(x);
+  else return ex2(x);
+}
 
 struct ScoreArgs {
   const int32_t* block_table;
@@ -82,6 +97,32 @@ __device__ __forceinline__ int page_block(const ScoreArgs& a, int b, int p) {
   return blk;
 }
 
+// Pass-2 work list: tiles (r, g, kt) in (r, g)-major order, ceil(np/8) key tiles per valid
+// sequence (8 pages of 16 keys each) and ceil(W/128) zero-writing tiles per invalid one. Every
+// role of a CTA walks it with its own cursor; the tile index only grows, so the cursor only
+// moves forward.
+struct TileCursor {
+  int r = 0, base = 0, per = -1;
+  SeqInfo s;
+  __device__ __forceinline__ bool seek(const ScoreArgs& a, int t, int& g, int& kt) {
+    while (true) {
+      if (r >= a.R) return false;
+      if (per < 0) {
+        s = seq_info(a, r);
+        per = s.ok ? (s.np + 7) / 8 : (a.W + kKRows2 - 1) / kKRows2;
+      }
+      if (t < base + a.Hkv * per) break;
+      base += a.Hkv * per;
+      ++r;
+      per = -1;
+    }
+    const int local = t - base;
+    g = local / per;
+    kt = local % per;
+    return true;
+  }
+};
+
 // ----------------------------------------------------------------------------------------
 // Pass 1: per-query base-2 log-sum-exp over the window keys.
 // ----------------------------------------------------------------------------------------
@@ -99,7 +140,8 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
                                              ~uintptr_t(1023));
   uint8_t* q_buf = smem;                      // 2 x kQBytes
   uint8_t* k_buf = smem + 2 * kQBytes;        // kKStages1 x kKBytes
-  uint64_t* bars = reinterpret_cast<uint64_t*>(k_buf + kKStages1 * kKBytes);
+  float2* comb = reinterpret_cast<float2*>(k_buf + kKStages1 * kKBytes);   // [128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(comb + kQRows1);
   uint64_t* q_full = bars;        // [2]
   uint64_t* q_empty = bars + 2;   // [2]
   uint64_t* k_full = bars + 4;    // [kKStages1]
@@ -119,7 +161,7 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 128);
+      mbar_init(&acc_empty[i], kEpiThreads);
     }
     for (int i = 0; i < kKStages1; ++i) {
       mbar_init(&k_full[i], 1);
@@ -197,7 +239,7 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
           const uint32_t d_tmem = tmem_base + ab * 256;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
+            const uint32_t off = (kk & 3) * 32;
             const uint64_t ad = sw128_kmajor_desc(q_addr + (kk >> 2) * kQRows1 * kRowBytes + off);
             const uint64_t bd = sw128_kmajor_desc(k_addr + (kk >> 2) * kKRows1 * kRowBytes + off);
             umma_bf16(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
@@ -213,8 +255,10 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
   } else {
-    // ---------------- epilogue: one query row per thread ----------------
+    // ------------- epilogue: one query row per TMEM lane, two warps per lane quadrant -------------
+    const int e = warp - 2;
     const int quad = warp & 3;
+    const int half = e >> 2;              // which 128 columns of each 256-column tile
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     int ab = 0;
@@ -224,63 +268,88 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int h = (t / TT) % a.Hq;
       const int r = t / (TT * a.Hq);
       const SeqInfo s = seq_info(a, r);
-      float lse2 = INFINITY;
-      if (s.ok && !*abort_flag) {
-        float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f;
+      bool stop = !s.ok;
+      if (s.ok) {
         const int nkt = (s.np + 15) / 16;
-        bool stop = false;
         for (int kt = 0; kt < nkt; ++kt) {
           const int ncols = min(16, s.np - kt * 16) * 16;
           if (!mbar_wait(&acc_full[ab], aph, abort_flag, a.status)) { stop = true; break; }
           tc_fence_after();
-          const int slot0 = (s.p_first + kt * 16) * 16;
+          const int c0 = half * 128;
+          const int nsub = max(0, min(8, (ncols - c0) / 16));
+          const int slot0 = (s.p_first + kt * 16) * 16 + c0;
           const bool edge = (kt == 0) || (kt == nkt - 1);
-          for (int c = 0; c < ncols; c += 32) {
-            float v[32];
-            const int nvalid = min(32, ncols - c);
-            if (nvalid == 32) {
-              tmem_ld32(lane_base + ab * 256 + c, v);
-            } else {
-              float v16[16];
-              tmem_ld16(lane_base + ab * 256 + c, v16);
+          for (int g0 = 0; g0 < nsub; g0 += 4) {
+            float v[64];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) { v[i] = v16[i]; v[16 + i] = -INFINITY; }
-            }
+            for (int q = 0; q < 4; ++q)
+              if (g0 + q < nsub) tmem_ld16(lane_base + ab * 256 + c0 + (g0 + q) * 16, v + 16 * q);
             tmem_wait_ld();
+            reg_fence<64>(v);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (g0 + q >= nsub) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[16 * q + i] = -INFINITY;
+              }
             if (edge) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int slot = slot0 + c + i;
+              for (int i = 0; i < 64; ++i) {
+                const int slot = slot0 + g0 * 16 + i;
                 if (slot < s.start || slot >= s.n) v[i] = -INFINITY;
               }
             }
-            float cmax = v[0];
+            float mx[8];
 #pragma unroll
-            for (int i = 1; i < 32; ++i) cmax = fmaxf(cmax, v[i]);
+            for (int j = 0; j < 8; ++j) {
+              const float a0 = fmaxf(v[8 * j], v[8 * j + 1]), a1 = fmaxf(v[8 * j + 2], v[8 * j + 3]);
+              const float a2 = fmaxf(v[8 * j + 4], v[8 * j + 5]), a3 = fmaxf(v[8 * j + 6], v[8 * j + 7]);
+              mx[j] = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+            }
+            const float cmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
             if (cmax == -INFINITY) continue;
             const float m_new = fmaxf(m, cmax * a.cs);
-            float sum = 0.f;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sum += ex2(fmaf(v[i], a.cs, -m_new));
-            l = l * ex2(m - m_new) + sum;
+            for (int i = 0; i < 64; i += 4) {
+              acc[0] += exp2_split<0>(fmaf(v[i], a.cs, -m_new));
+              acc[1] += exp2_split<1>(fmaf(v[i + 1], a.cs, -m_new));
+              acc[2] += exp2_split<2>(fmaf(v[i + 2], a.cs, -m_new));
+              acc[3] += exp2_split<3>(fmaf(v[i + 3], a.cs, -m_new));
+            }
+            l = l * ex2(m - m_new) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
             m = m_new;
           }
           tc_fence_before();
           mbar_arrive(&acc_empty[ab]);
           if (++ab == 2) { ab = 0; aph ^= 1; }
         }
-        if (!stop) lse2 = m + __log2f(l);
-      } else if (!s.ok && tt == 0 && h == 0 && row == 0) {
+      } else if (tt == 0 && h == 0 && row == 0 && half == 0) {
         report(a.status, KARA_ERR_INVALID_ARG);
       }
-      const int token = tt * kQRows1 + row;
-      float* lrow = a.lse + (static_cast<size_t>(r) * a.Hq + h) * a.Wp;
-      if (token < a.W) lrow[token] = lse2;
-      else if (token < a.Wp) lrow[token] = INFINITY;
-      if (tt == TT - 1) {
-        const int extra = TT * kQRows1 + row;
-        if (extra < a.Wp) lrow[extra] = INFINITY;
+      // merge the two column halves of the row
+      if (half == 1) comb[row] = make_float2(stop ? NAN : m, l);
+      named_barrier(kEpiBarrier, kEpiThreads);
+      if (half == 0) {
+        const float2 o = comb[row];
+        float lse2 = INFINITY;
+        if (!stop && !isnan(o.x)) {
+          const float mm = fmaxf(m, o.x);
+          const float ll = l * ex2(m - mm) + (o.x == -INFINITY ? 0.f : o.y * ex2(o.x - mm));
+          lse2 = mm + __log2f(ll);
+        }
+        const int token = tt * kQRows1 + row;
+        float* lrow = a.lse + (static_cast<size_t>(r) * a.Hq + h) * a.Wp;
+        if (token < a.W) lrow[token] = lse2;
+        else if (token < a.Wp) lrow[token] = INFINITY;
+        if (tt == TT - 1) {
+          const int extra = TT * kQRows1 + row;
+          if (extra < a.Wp) lrow[extra] = INFINITY;
+        }
       }
+      named_barrier(kEpiBarrier, kEpiThreads);
     }
   }
 
@@ -309,7 +378,9 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
                                              ~uintptr_t(1023));
   uint8_t* a_buf = smem;                    // 2 x kABytes (key tiles)
   uint8_t* b_buf = smem + 2 * kABytes;      // kQStages2 x kBBytes (query tiles)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(b_buf + kQStages2 * kBBytes);
+  float* lse_s = reinterpret_cast<float*>(b_buf + kQStages2 * kBBytes);   // [2][256]
+  float* red = lse_s + 2 * kQRows2;                                       // [128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + kKRows2);
   uint64_t* a_full = bars;                  // [2]
   uint64_t* a_empty = bars + 2;             // [2]
   uint64_t* b_full = bars + 4;              // [kQStages2]
@@ -321,17 +392,15 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   const int warp = warp_id();
   const int lane = lane_id();
-  // Key tiles of 8 pages; the window spans at most ceil((W+15)/16) pages.
-  const int KT = ((a.W + 15 + 15) / 16 + 7) / 8;
   const int QT = (a.W + kQRows2 - 1) / kQRows2;
-  const int num_tiles = a.R * a.Hkv * KT;
+  const int NQ = a.G * QT;                  // query tiles per key tile
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&a_full[i], 1);
       mbar_init(&a_empty[i], 1);
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 128);
+      mbar_init(&acc_empty[i], kEpiThreads);
     }
     for (int i = 0; i < kQStages2; ++i) {
       mbar_init(&b_full[i], 1);
@@ -355,12 +424,12 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
       tma_prefetch_desc(&tm_k);
       int ai = 0, bi = 0;
       uint32_t aph = 0, bph = 0;
-      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-        const int kt = t % KT;
-        const int g = (t / KT) % a.Hkv;
-        const int r = t / (KT * a.Hkv);
-        const SeqInfo s = seq_info(a, r);
-        if (!s.ok || kt * 8 >= s.np) continue;
+      TileCursor cur;
+      int g, kt;
+      for (int t = blockIdx.x; !*abort_flag && cur.seek(a, t, g, kt); t += gridDim.x) {
+        const SeqInfo& s = cur.s;
+        if (!s.ok) continue;
+        const int r = cur.r;
         const int pages = min(8, s.np - kt * 8);
         if (!mbar_wait(&a_empty[ai], aph ^ 1, abort_flag, a.status)) break;
         mbar_expect_tx(&a_full[ai], pages * NCH * kPageBytes);
@@ -372,16 +441,14 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         if (++ai == 2) { ai = 0; aph ^= 1; }
         bool stop = false;
-        for (int hl = 0; hl < a.G && !stop; ++hl) {
-          const int h = g * a.G + hl;
-          for (int qt = 0; qt < QT; ++qt) {
-            if (!mbar_wait(&b_empty[bi], bph ^ 1, abort_flag, a.status)) { stop = true; break; }
-            mbar_expect_tx(&b_full[bi], kBBytes);
-            for (int c = 0; c < NCH; ++c)
-              tma_load_4d(b_buf + bi * kBBytes + c * kQRows2 * kRowBytes, &tm_q, &b_full[bi],
-                          c * 64, h, qt * kQRows2, r);
-            if (++bi == kQStages2) { bi = 0; bph ^= 1; }
-          }
+        for (int q = 0; q < NQ; ++q) {
+          const int h = g * a.G + q / QT, qt = q % QT;
+          if (!mbar_wait(&b_empty[bi], bph ^ 1, abort_flag, a.status)) { stop = true; break; }
+          mbar_expect_tx(&b_full[bi], kBBytes);
+          for (int c = 0; c < NCH; ++c)
+            tma_load_4d(b_buf + bi * kBBytes + c * kQRows2 * kRowBytes, &tm_q, &b_full[bi],
+                        c * 64, h, qt * kQRows2, r);
+          if (++bi == kQStages2) { bi = 0; bph ^= 1; }
         }
         if (stop) break;
       }
@@ -391,15 +458,14 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
       int ai = 0, bi = 0, ab = 0;
       uint32_t aph = 0, bph = 0, cph = 0;
       const uint32_t idesc = idesc_bf16_f32(128, kQRows2);
-      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-        const int kt = t % KT;
-        const int r = t / (KT * a.Hkv);
-        const SeqInfo s = seq_info(a, r);
-        if (!s.ok || kt * 8 >= s.np) continue;
+      TileCursor cur;
+      int g, kt;
+      for (int t = blockIdx.x; !*abort_flag && cur.seek(a, t, g, kt); t += gridDim.x) {
+        if (!cur.s.ok) continue;
         if (!mbar_wait(&a_full[ai], aph, abort_flag, a.status)) break;
         const uint32_t a_addr = smem_u32(a_buf + ai * kABytes);
         bool stop = false;
-        for (int q = 0; q < a.G * QT; ++q) {
+        for (int q = 0; q < NQ; ++q) {
           if (!mbar_wait(&b_full[bi], bph, abort_flag, a.status)) { stop = true; break; }
           if (!mbar_wait(&acc_empty[ab], cph ^ 1, abort_flag, a.status)) { stop = true; break; }
           tc_fence_after();
@@ -423,56 +489,76 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
   } else {
-    // ---------------- epilogue: one key per thread ----------------
+    // ------------- epilogue: one key per TMEM lane, two warps per lane quadrant -------------
+    const int e = warp - 2;
+    const int etid = e * 32 + lane;       // 0..255: the query column whose lse it stages
     const int quad = warp & 3;
+    const int half = e >> 2;              // which 128 query columns of each tile
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-    int ab = 0;
+    int ab = 0, qbuf = 0;
     uint32_t cph = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      const int kt = t % KT;
-      const int g = (t / KT) % a.Hkv;
-      const int r = t / (KT * a.Hkv);
-      const SeqInfo s = seq_info(a, r);
+    bool aborted = false;
+    TileCursor cur;
+    int g, kt;
+    for (int t = blockIdx.x; cur.seek(a, t, g, kt); t += gridDim.x) {
+      const SeqInfo& s = cur.s;
+      const int r = cur.r;
       float* out = a.scores + (static_cast<size_t>(r) * a.Hkv + g) * a.W;
       if (!s.ok) {
         const int j = kt * kKRows2 + row;
-        if (j < a.W) out[j] = 0.f;
+        if (half == 0 && j < a.W) out[j] = 0.f;
         continue;
       }
-      if (kt * 8 >= s.np) continue;
-      float acc = 0.f;
-      bool stop = *abort_flag != 0;
-      for (int hl = 0; hl < a.G && !stop; ++hl) {
-        const int h = g * a.G + hl;
-        const float* lrow = a.lse + (static_cast<size_t>(r) * a.Hq + h) * a.Wp;
-        for (int qt = 0; qt < QT; ++qt) {
-          if (!mbar_wait(&acc_full[ab], cph, abort_flag, a.status)) { stop = true; break; }
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const float* lse_rows = a.lse + (static_cast<size_t>(r) * a.Hq + g * a.G) * a.Wp;
+      float lv = lse_rows[etid];
+      for (int q = 0; q < NQ; ++q) {
+        // stage this tile's 256 lse values; prefetch the next tile's into a register
+        float* ls = lse_s + qbuf * kQRows2;
+        ls[etid] = lv;
+        if (q + 1 < NQ) {
+          const int h1 = (q + 1) / QT, qt1 = (q + 1) % QT;
+          lv = lse_rows[static_cast<size_t>(h1) * a.Wp + qt1 * kQRows2 + etid];
+        }
+        named_barrier(kEpiBarrier, kEpiThreads);
+        if (!aborted && !mbar_wait(&acc_full[ab], cph, abort_flag, a.status)) aborted = true;
+        if (!aborted) {
           tc_fence_after();
-          const float4* l4 = reinterpret_cast<const float4*>(lrow + qt * kQRows2);
-#pragma unroll 1
-          for (int c = 0; c < kQRows2; c += 32) {
-            float v[32];
-            tmem_ld32(lane_base + ab * 256 + c, v);
-            float lz[32];
+          const float* lh = ls + half * 128;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 x = __ldg(l4 + (c >> 2) + i);
-              lz[4 * i] = x.x; lz[4 * i + 1] = x.y; lz[4 * i + 2] = x.z; lz[4 * i + 3] = x.w;
-            }
+          for (int g0 = 0; g0 < 8; g0 += 4) {
+            float v[64];
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+              tmem_ld16(lane_base + ab * 256 + half * 128 + (g0 + qq) * 16, v + 16 * qq);
             tmem_wait_ld();
+            reg_fence<64>(v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc += ex2(fmaf(v[i], a.cs, -lz[i]));
+            for (int i = 0; i < 64; i += 4) {
+              const float4 lz = *reinterpret_cast<const float4*>(lh + g0 * 16 + i);
+              acc[0] += exp2_split<0>(fmaf(v[i], a.cs, -lz.x));
+              acc[1] += exp2_split<1>(fmaf(v[i + 1], a.cs, -lz.y));
+              acc[2] += exp2_split<2>(fmaf(v[i + 2], a.cs, -lz.z));
+              acc[3] += exp2_split<3>(fmaf(v[i + 3], a.cs, -lz.w));
+            }
           }
           tc_fence_before();
           mbar_arrive(&acc_empty[ab]);
           if (++ab == 2) { ab = 0; cph ^= 1; }
         }
+        qbuf ^= 1;
       }
-      if (stop) continue;
-      const int slot = (s.p_first + kt * 8) * 16 + row;
-      const int j = slot - s.start;
-      if (row < min(8, s.np - kt * 8) * 16 && j >= 0 && j < a.W) out[j] = acc;
+      // merge the two query halves of each key
+      const float total = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      if (half == 1) red[row] = total;
+      named_barrier(kEpiBarrier, kEpiThreads);
+      if (half == 0 && !aborted) {
+        const int slot = (s.p_first + kt * 8) * 16 + row;
+        const int j = slot - s.start;
+        if (row < min(8, s.np - kt * 8) * 16 && j >= 0 && j < a.W) out[j] = total + red[row];
+      }
+      named_barrier(kEpiBarrier, kEpiThreads);
     }
   }
 
@@ -487,12 +573,12 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
 template <int D>
 constexpr size_t rowstats_smem() {
   return 1024 + 2 * (D / 64) * kQRows1 * kRowBytes + kKStages1 * (D / 64) * kKRows1 * kRowBytes +
-         256;
+         kQRows1 * sizeof(float2) + 256;
 }
 template <int D>
 constexpr size_t colsum_smem() {
   return 1024 + 2 * (D / 64) * kKRows2 * kRowBytes + kQStages2 * (D / 64) * kQRows2 * kRowBytes +
-         256;
+         (2 * kQRows2 + kKRows2) * sizeof(float) + 256;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -577,7 +663,7 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   }
   const int TT = (L.W + kQRows1 - 1) / kQRows1;
   const int tiles1 = L.R * L.Hq * TT;
-  const int KT = ((L.W + 15 + 15) / 16 + 7) / 8;
+  const int KT = ((L.W + 15 + 15) / 16 + 7) / 8;   // at most this many key tiles per (r, g)
   const int tiles2 = L.R * L.Hkv * KT;
   const int sms = sm_count();
   score_rowstats_kernel<D><<<min(tiles1, sms), kThreads, rowstats_smem<D>(), stream>>>(tq1, tk, a);
