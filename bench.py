@@ -43,6 +43,27 @@ WORKLOAD_DESC = ("layer: one 7B-class layer, batch 32, 28 query / 4 KV heads, he
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's batch: the layer workload's seed (1234 + config index 1), offset per
+    rank so that every rank compresses its own, independent sequences."""
+    return 1234 + 1 + 1000 * rank
+
+
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The maximum of a per-rank scalar over all ranks (the step time of the whole job)."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(tokens_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: window tokens of every rank per second of the slowest rank."""
+    return tokens_per_rank_step * world / (ms_per_step / 1e3)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -281,7 +302,7 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = WORKLOAD
-    seed = 1234 + 1 + 1000 * rank            # configs[1] seed; each rank its own batch
+    seed = rank_seed(rank)
     cache = synth.make_cache(wl, seed, dev)
     work = algorithmic_work(wl, cache)
     step = Step(cache, wl)
@@ -319,20 +340,13 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
         op_ms["paged_decode_attn"].append(e[3].elapsed_time(e[4]))
     avg = {k: sum(v) / len(v) for k, v in op_ms.items()}
 
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev, world)
     ms_step = total_ms / args.steps
     tokens_step = wl.batch * wl.window * world
-    value = tokens_step / (ms_step / 1e3)
+    value = whole_job_value(wl.batch * wl.window, world, ms_step)
 
     e2e = e2e_run(cache, wl, steps=min(args.steps, args.e2e_steps), warmup=2)
-    e2e_ms = e2e["ms_per_step"]
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e["ms_per_step"], dev, world)
     if rank != 0:
         return None
 
@@ -427,7 +441,7 @@ def reference_arm(args, rank: int) -> dict | None:
     except Exception:
         cores = os.cpu_count() or 1
     wl = WORKLOAD
-    cache_cpu = synth.make_cache(wl, 1234 + 1, "cpu")
+    cache_cpu = synth.make_cache(wl, rank_seed(0), "cpu")
     for i in range(args.warmup):
         time_cpu_oracle_sample(cache_cpu, wl, units=1, seed=i)
     total, tokens = 0.0, 0.0

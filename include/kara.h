@@ -103,8 +103,9 @@ typedef enum kara_op {
 
 /*
  * kara_score - bidirectional attention scoring of the compression window ([KARA] abstract:
- * "bidirectional attention to score and select informative KV pairs in the window"; [GIST]
- * section 1: a token the current reasoning refers to strongly scores high).
+ * the KV pairs of the window are scored with attention in both directions and the
+ * informative ones kept; [GIST] section 1: a token the current reasoning refers to strongly
+ * scores high).
  *
  * For due sequence r (cache row b = seq_ids ? seq_ids[r] : r, n = ctx_len[b]) the window is
  * slots [n-window, n). For KV head g with query heads h = g*G .. g*G+G-1 (G = num_q_heads /
@@ -131,8 +132,8 @@ kara_status kara_score(const void* q_win, const void* k_cache, const kara_pool* 
                        size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream);
 
 /*
- * kara_select - keep the k highest-scoring window positions ([KARA] abstract: "select
- * informative KV pairs"; [GIST] results: about 20 % kept).
+ * kara_select - keep the k highest-scoring window positions ([KARA] abstract: the informative
+ * KV pairs of the window are selected; [GIST] results: about 20 % kept).
  *
  * For each of `rows` rows of scores [rows, window]: the k positions with the largest score,
  * ties broken towards the lower position, written ascending to sel [rows, k] (int32).
@@ -144,8 +145,8 @@ kara_status kara_select(const float* scores, int32_t rows, int32_t window, int32
 
 /*
  * kara_token2chunk - expand part of the selection into flexible-length chunks and trim back
- * to budget ([KARA] abstract: "Token2Chunk module to expand a subset of selected KV pairs into
- * chunks"; [GIST] section 2: everything between two important points is kept as one chunk).
+ * to budget ([KARA] abstract: a Token2Chunk module grows some of the selected KV pairs into
+ * chunks; [GIST] section 2: the span between two important points is kept as one chunk).
  *
  * Per row, in window positions: anchors = the num_anchors selected positions with the largest
  * scores (ties: lower position); every position strictly between two consecutive anchors is
