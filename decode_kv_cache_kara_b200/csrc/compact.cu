@@ -19,6 +19,7 @@
 // The gather reads only blocks that belong to the sequences and writes only fresh blocks, so
 // sources never alias destinations; nothing is modified unless the plan is valid.
 #include <cstdint>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -484,3 +485,60 @@ kara_status launch_lacache(const LacacheLaunch& L, cudaStream_t stream) {
 }
 
 }  // namespace kara
+
+// ------------------------------------------------------------------------------------------
+// kara_compact_noalloc: kara_compact with its plan scratch in a fixed device array.
+//
+// For callers that cannot allocate device memory when they compress: a serving engine that
+// hands all free device memory to its KV block pool at start-up (a later cudaMalloc would
+// fail, or would have to shrink the pool), and plain C callers that hold no device
+// allocator. The caller still passes the pools, the bookkeeping and `keep`; only the plan
+// (per-sequence geometry and the popped block ids) lives here.
+// ------------------------------------------------------------------------------------------
+namespace kara {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = KARA_COMPACT_NOALLOC_SCRATCH_BYTES;
+// Every GPU that loads this library holds one copy of this array until the process exits.
+static __device__ __align__(256) int32_t g_compact_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+int32_t* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once per device
+// (in host code the array's name is only a host-side handle, not a device address).
+kara_status scratch_for_current_device(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KARA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_compact_scratch) != cudaSuccess || p == nullptr)
+      return KARA_ERR_CUDA;
+    g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_scratch_ptr[dev];
+  return KARA_OK;
+}
+
+}  // namespace
+}  // namespace kara
+
+extern "C" kara_status kara_compact_noalloc(const kara_layer_kv* layers, int32_t num_layers,
+                                            const kara_pool* pool, const int32_t* seq_ids,
+                                            int32_t num_seqs, int32_t window, int32_t k,
+                                            const int32_t* keep, int32_t* dev_status,
+                                            cudaStream_t stream) {
+  using namespace kara;
+  if (num_seqs < 0 || window < 1 || k < 1 || k > window) return KARA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return KARA_OK;
+  if (compact_workspace_bytes(num_seqs, window, k) > kNoAllocScratchBytes)
+    return KARA_ERR_WORKSPACE;   // the plan would not fit the fixed scratch array
+  int32_t* scratch = nullptr;
+  const kara_status st = scratch_for_current_device(&scratch);
+  if (st != KARA_OK) return st;
+  // The plan kernel writes every scratch entry it later reads, so nothing needs clearing.
+  return kara_compact(layers, num_layers, pool, seq_ids, num_seqs, window, k, keep, scratch,
+                      kNoAllocScratchBytes, dev_status, stream);
+}

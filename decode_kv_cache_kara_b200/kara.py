@@ -71,6 +71,8 @@ _SIGNATURES = {
     "kara_token2chunk": ([_P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "kara_compact": ([ctypes.POINTER(_LayerKV), _I, ctypes.POINTER(_Pool), _P, _I, _I, _I, _P, _P,
                       _Z, _P, _P], _I),
+    "kara_compact_noalloc": ([ctypes.POINTER(_LayerKV), _I, ctypes.POINTER(_Pool), _P, _I, _I, _I,
+                              _P, _P, _P], _I),
     "paged_decode_attn": ([_P, _P, _P, ctypes.POINTER(_Pool), _I, _F, _P, _P, _Z, _P, _P], _I),
     "lacache_compact": ([ctypes.POINTER(_LayerKV), _I, ctypes.POINTER(_Pool), _P, _I,
                          ctypes.POINTER(_LacacheParams), _P, _Z, _P, _P], _I),
@@ -278,6 +280,28 @@ def kara_compact(k_layers, v_layers, pool: PagedPool, window: int, keep: torch.T
     _check(lib().kara_compact(arr, nl, ctypes.byref(ps), _ptr(seq_ids), r, window, k, _ptr(keep),
                               _ptr(ws), ws.numel(), _ptr(status), _stream(stream)),
            "kara_compact")
+    return status
+
+
+def kara_compact_noalloc(k_layers, v_layers, pool: PagedPool, window: int, keep: torch.Tensor,
+                         seq_ids: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """kara_compact with the plan scratch in the library's fixed device array: the call
+    allocates no device memory (for callers that cannot allocate when they compress). Returns
+    the status tensor; raises KaraError(ERR_WORKSPACE) when the plan would not fit."""
+    _require(keep, torch.int32, "keep")
+    nl, r, hkv, k = keep.shape
+    arr = _layers(k_layers, v_layers)
+    if nl != len(arr):
+        raise ValueError("keep's first dimension must equal the number of layers")
+    if seq_ids is not None:
+        _require(seq_ids, torch.int32, "seq_ids")
+    if status is None:
+        raise ValueError("pass a preallocated status tensor (this call allocates nothing)")
+    ps = pool.c_struct()
+    _check(lib().kara_compact_noalloc(arr, nl, ctypes.byref(ps), _ptr(seq_ids), r, window, k,
+                                      _ptr(keep), _ptr(status), _stream(stream)),
+           "kara_compact_noalloc")
     return status
 
 

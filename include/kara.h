@@ -187,6 +187,31 @@ kara_status kara_compact(const kara_layer_kv* layers, int32_t num_layers, const 
                          int32_t* dev_status, cudaStream_t stream);
 
 /*
+ * kara_compact_noalloc - kara_compact without a workspace argument: the plan scratch lives in
+ * a fixed array of KARA_COMPACT_NOALLOC_SCRATCH_BYTES inside the library, so the call
+ * allocates no device memory. The pages print no counterpart of this call; it exists for
+ * callers that cannot allocate device memory when they compress, such as a serving engine
+ * that has given all free device memory to its KV block pool, or a C caller without a device
+ * allocator.
+ *
+ * Same arguments, semantics and device-side errors as kara_compact. Differences:
+ *  - Returns KARA_ERR_WORKSPACE, without enqueueing anything, when the plan for num_seqs
+ *    sequences and budget k would exceed the fixed array (plan size in bytes:
+ *    4 * (16 + 12 * num_seqs + num_seqs * ceil((15 + k) / 16))).
+ *  - The first call on each device looks up the array's device address (once per device,
+ *    with that device current); make that first call before any stream capture.
+ *  - Every call on a device shares the one array, which keeps the last call's contents:
+ *    calls that overlap on the GPU (other streams, or threads sharing a device without
+ *    ordering) race on it. Order them on one stream.
+ *  - Every GPU that loads the library holds the array until the process exits.
+ */
+#define KARA_COMPACT_NOALLOC_SCRATCH_BYTES (64u * 1024u)
+kara_status kara_compact_noalloc(const kara_layer_kv* layers, int32_t num_layers,
+                                 const kara_pool* pool, const int32_t* seq_ids, int32_t num_seqs,
+                                 int32_t window, int32_t k, const int32_t* keep,
+                                 int32_t* dev_status, cudaStream_t stream);
+
+/*
  * paged_decode_attn - one decode step of grouped-query attention over the (compressed) paged
  * cache ([KARA] abstract: the kept KV pairs serve subsequent decoding, with PagedAttention).
  *
