@@ -43,6 +43,25 @@ WORKLOAD_DESC = ("layer: one 7B-class layer, batch 32, 28 query / 4 KV heads, he
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def captured_traffic(op: str):
+    """DRAM bytes per launch of `op` from the committed ncu summary (profiles/traffic.txt),
+    or None when the kernel source changed since the capture (its sha256 no longer matches)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        parts = line.split()
+        if len(parts) != 4 or line.startswith("#") or parts[0] != op:
+            continue
+        src = os.path.join(ROOT, "decode_kv_cache_kara_b200", parts[1])
+        if not os.path.exists(src):
+            return None
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return int(parts[3]) if digest == parts[2] else None
+    return None
+
+
 def rank_seed(rank: int) -> int:
     """Seed of a rank's batch: the layer workload's seed (1234 + config index 1), offset per
     rank so that every rank compresses its own, independent sequences."""
@@ -371,13 +390,7 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
     dom = max((k for k in kernels if kernels[k]["bound"] in ("tensor", "hbm")),
               key=lambda k: kernels[k]["ms"])
     dk = kernels[dom]
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        try:
-            traffic = json.load(open(tpath)).get(dom)
-        except Exception:
-            traffic = None
+    traffic = captured_traffic(dom)
     if dk["bound"] == "tensor":
         roof = {"kernel": dom, "bound": "tensor", "achieved": dk["useful_tflops"],
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
