@@ -9,9 +9,13 @@
 // Grid = (split, KV head, sequence); a split covers 16 pages; each of the 4 warps walks its
 // pages with its own online softmax (base 2, scale folded into q), and the warps merge in
 // shared memory into one split partial (m, l, unnormalised o). A second kernel merges the
-// splits of each (sequence, query head). Per page a warp assigns two lanes to each of the 16
-// slots (half of d each) for q.k, then one lane per 4 channels of d for p.v; K rows are read
-// with 16-byte loads, V rows with 8-byte loads, both coalesced within a row.
+// splits of each (sequence, query head). Pages reach shared memory by TMA (one 16-row box of
+// one KV head per 64 channels, 128-byte swizzle) through a 3-stage ring per warp, so that
+// each SM keeps many pages in flight. Per page a warp assigns two lanes to each of the 16
+// slots (half of d each) for q.k, then one lane per 4 channels of d for p.v; the swizzle
+// keeps both read patterns free of bank conflicts.
+#include <cuda.h>
+
 #include <cstdint>
 
 #include "common.cuh"
@@ -37,13 +41,31 @@ struct DecodeArgs {
   float cs;            // scale * log2(e)
 };
 
+template <int D>
+__host__ __device__ constexpr int page_bytes() { return 16 * D * 2; }   // one page, one KV head
+constexpr int kStages = 3;                                  // TMA page ring depth per warp
+
 template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads)
-decode_split_kernel(const DecodeArgs a) {
-  constexpr int kHalf = D / 2;          // channels per lane in q.k
-  constexpr int kVec = kHalf / 8;       // 16-byte K loads per lane
-  constexpr int kE4 = kHalf / 4;        // float4 groups per half
-  constexpr int kCh = D / 32;           // channels per lane in p.v (4 or 2)
+constexpr size_t split_smem_bytes() {
+  // [warp][stage]{K page, V page} (1024-aligned); the warp merge reuses this space
+  return 1024 + static_cast<size_t>(kDecWarps) * kStages * 2 * page_bytes<D>() + 64 * kDecWarps;
+}
+
+// Byte offset of 16-byte granule `gi` of row `r` in a 128-byte-swizzled 16-row box.
+__device__ __forceinline__ uint32_t sw128(int r, int gi) {
+  return static_cast<uint32_t>(r * 128 + ((gi ^ (r & 7)) << 4));
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kDecThreads, 2)
+decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const DecodeArgs a) {
+  constexpr int NCH = D / 64;                 // 64-channel chunks per row
+  constexpr int kHalf = D / 2;                // channels per lane in q.k
+  constexpr int kE4 = kHalf / 4;              // float4 groups per half
+  constexpr int kCh = D / 32;                 // channels per lane in p.v (4 or 2)
+  constexpr uint32_t kPage = page_bytes<D>();
+  constexpr uint32_t kChunkBytes = 16 * 128;  // one 64-channel chunk of a page
   const int split = blockIdx.x;
   const int g = blockIdx.y;
   const int b = blockIdx.z;
@@ -59,11 +81,21 @@ decode_split_kernel(const DecodeArgs a) {
   if (p_begin >= pages) return;
   const int p_end = min(pages, p_begin + kPagesPerSplit);
 
+  extern __shared__ __align__(1024) uint8_t dsm[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* my_ring = ring + static_cast<size_t>(warp) * kStages * 2 * kPage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kDecWarps * kStages * 2 * kPage);
+  uint64_t* my_bars = bars + warp * kStages;
   __shared__ __align__(16) float q_s[G][kE4][2][4];          // pre-scaled q, half-interleaved
   __shared__ __align__(16) float p_s[kDecWarps][16][8];       // page probabilities
   __shared__ float red_m[kDecWarps][G], red_l[kDecWarps][G];
-  __shared__ __align__(16) float red_o[kDecWarps][G][D];
+  float* red_o = reinterpret_cast<float*>(ring);              // [warp][G][D], after the loop
 
+  if (lane == 0) {
+    for (int st = 0; st < kStages; ++st) mbar_init(&my_bars[st], 1);
+    fence_barrier_init();
+  }
   for (int i = threadIdx.x; i < G * D; i += kDecThreads) {
     const int h = i / D, c = i % D;
     const float qv = __bfloat162float(a.q[(static_cast<size_t>(b) * a.Hq + g * G + h) * D + c]);
@@ -71,6 +103,31 @@ decode_split_kernel(const DecodeArgs a) {
     q_s[h][e / 4][half][e % 4] = qv * a.cs;
   }
   __syncthreads();
+
+  // this warp's pages: p_begin + warp + 4k; lane k holds the block id of its k-th page
+  const int32_t* tab = a.block_table + static_cast<size_t>(b) * a.max_blocks;
+  const int my_pages = (p_end - p_begin - warp + kDecWarps - 1) / kDecWarps;
+  int my_blk = 0;
+  if (lane < my_pages) {
+    my_blk = tab[p_begin + warp + kDecWarps * lane];
+    if (my_blk < 0 || my_blk >= a.num_blocks) {
+      report(a.status, KARA_ERR_BAD_BLOCK);
+      my_blk = -1;
+    }
+  }
+  auto issue = [&](int k) {          // lane 0: page k of this warp into stage k % kStages
+    const int blk = __shfl_sync(0xffffffffu, my_blk, k);
+    if (lane == 0 && blk >= 0) {
+      uint8_t* st = my_ring + (k % kStages) * 2 * kPage;
+      uint64_t* bar = &my_bars[k % kStages];
+      mbar_expect_tx(bar, 2 * kPage);
+      for (int c = 0; c < NCH; ++c) {
+        tma_load_4d(st + c * kChunkBytes, &tm_k, bar, c * 64, g, 0, blk);
+        tma_load_4d(st + kPage + c * kChunkBytes, &tm_v, bar, c * 64, g, 0, blk);
+      }
+    }
+  };
+  for (int k = 0; k < min(kStages, my_pages); ++k) issue(k);
 
   float m[G], l[G];
   float2 acc[G][kCh / 2];
@@ -81,51 +138,33 @@ decode_split_kernel(const DecodeArgs a) {
 #pragma unroll
     for (int c = 0; c < kCh / 2; ++c) acc[h][c] = make_float2(0.f, 0.f);
   }
-
   const int slot = lane >> 1, half = lane & 1;
-  const size_t row_stride = static_cast<size_t>(a.Hkv) * D;   // elements between slots
-  const int32_t* tab = a.block_table + static_cast<size_t>(b) * a.max_blocks;
+  uint32_t phase_bits = 0;            // parity per stage
+  volatile int no_abort = 0;
 
-  for (int p = p_begin + warp; p < p_end; p += kDecWarps) {
-    const int blk = tab[p];
-    if (blk < 0 || blk >= a.num_blocks) {
-      if (lane == 0) report(a.status, KARA_ERR_BAD_BLOCK);
-      continue;
-    }
+  for (int k = 0; k < my_pages; ++k) {
+    const int p = p_begin + warp + kDecWarps * k;
+    const int blk = __shfl_sync(0xffffffffu, my_blk, k);
+    const int st = k % kStages;
+    if (blk >= 0) {                                 // a bad block id was reported; page skipped
+    const bool ok = mbar_wait(&my_bars[st], (phase_bits >> st) & 1, &no_abort, a.status);
+    phase_bits ^= 1u << st;
+    if (!ok) break;
     const int valid = min(16, n - p * 16);
-    const __nv_bfloat16* kpage = a.k + (static_cast<size_t>(blk) * 16) * row_stride + g * D;
-    const __nv_bfloat16* vpage = a.v + (static_cast<size_t>(blk) * 16) * row_stride + g * D;
-    // issue the loads of the page: K (this lane's slot, half of d) and V (all 16 slots, kCh
-    // channels of this lane)
-    uint4 kr[kVec];
-    const uint4* kp4 = reinterpret_cast<const uint4*>(kpage + slot * row_stride + half * kHalf);
-#pragma unroll
-    for (int i = 0; i < kVec; ++i) kr[i] = kp4[i];
-    uint32_t vr[16][kCh / 2];
-#pragma unroll
-    for (int s = 0; s < 16; ++s) {
-      const __nv_bfloat16* vrow = vpage + s * row_stride + lane * kCh;
-      if (s < valid) {
-        if constexpr (kCh == 4) {
-          const uint2 t = *reinterpret_cast<const uint2*>(vrow);
-          vr[s][0] = t.x;
-          vr[s][1] = t.y;
-        } else {
-          vr[s][0] = *reinterpret_cast<const uint32_t*>(vrow);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kCh / 2; ++c) vr[s][c] = 0u;
-      }
-    }
-    // q . k for this lane's slot and half of d, as pairs of partial sums
+    const uint8_t* kst = my_ring + st * 2 * kPage;
+    const uint8_t* vst = kst + kPage;
+    // q . k: this lane's slot, half of d (granules of chunk `half` for d = 128, the half of
+    // chunk 0's granules for d = 64)
     float2 dot2[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) dot2[h] = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int i = 0; i < kVec; ++i) {
-      const float2 k01 = bf16x2_to_f2(kr[i].x), k23 = bf16x2_to_f2(kr[i].y);
-      const float2 k45 = bf16x2_to_f2(kr[i].z), k67 = bf16x2_to_f2(kr[i].w);
+    for (int i = 0; i < kHalf / 8; ++i) {
+      const int chunk = NCH == 2 ? half : 0;
+      const int gi = NCH == 2 ? i : half * 4 + i;
+      const uint4 kr = *reinterpret_cast<const uint4*>(kst + chunk * kChunkBytes + sw128(slot, gi));
+      const float2 k01 = bf16x2_to_f2(kr.x), k23 = bf16x2_to_f2(kr.y);
+      const float2 k45 = bf16x2_to_f2(kr.z), k67 = bf16x2_to_f2(kr.w);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float4 qa = *reinterpret_cast<const float4*>(&q_s[h][2 * i][half][0]);
@@ -159,12 +198,19 @@ decode_split_kernel(const DecodeArgs a) {
       if (half == 0) p_s[warp][slot][h] = pr;
     }
     __syncwarp();
-    // p . v
-#pragma unroll
-    for (int s = 0; s < 16; ++s) {
+    // p . v: channels [kCh*lane, kCh*lane + kCh) of every valid slot
+    const int c0 = kCh * lane;
+    const int vchunk = c0 / 64, vgi = (c0 % 64) / 8, vsub = ((c0 % 64) % 8) * 2;
+    for (int s = 0; s < valid; ++s) {
+      const uint8_t* vrow = vst + vchunk * kChunkBytes + sw128(s, vgi) + vsub;
       float2 vf[kCh / 2];
-#pragma unroll
-      for (int c = 0; c < kCh / 2; ++c) vf[c] = bf16x2_to_f2(vr[s][c]);
+      if constexpr (kCh == 4) {
+        const uint2 t = *reinterpret_cast<const uint2*>(vrow);
+        vf[0] = bf16x2_to_f2(t.x);
+        vf[1] = bf16x2_to_f2(t.y);
+      } else {
+        vf[0] = bf16x2_to_f2(*reinterpret_cast<const uint32_t*>(vrow));
+      }
       const float4 p0 = *reinterpret_cast<const float4*>(&p_s[warp][s][0]);
       const float4 p1 = *reinterpret_cast<const float4*>(&p_s[warp][s][4]);
       const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
@@ -176,7 +222,14 @@ decode_split_kernel(const DecodeArgs a) {
       }
     }
     __syncwarp();
+    }
+    // stage st is free again: refill it with page k + kStages
+    if (k + kStages < my_pages) {
+      fence_proxy_async();
+      issue(k + kStages);
+    }
   }
+  __syncthreads();    // every warp is done with the ring: reuse it for the merge
 
   // merge the four warps of the CTA
   if (lane == 0) {
@@ -187,8 +240,8 @@ decode_split_kernel(const DecodeArgs a) {
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int c = 0; c < kCh / 2; ++c) {
-      red_o[warp][h][lane * kCh + 2 * c] = acc[h][c].x;
-      red_o[warp][h][lane * kCh + 2 * c + 1] = acc[h][c].y;
+      red_o[(warp * G + h) * D + lane * kCh + 2 * c] = acc[h][c].x;
+      red_o[(warp * G + h) * D + lane * kCh + 2 * c + 1] = acc[h][c].y;
     }
   __syncthreads();
   for (int i = threadIdx.x; i < G * (D + 2); i += kDecThreads) {
@@ -203,7 +256,7 @@ decode_split_kernel(const DecodeArgs a) {
 #pragma unroll
       for (int w = 0; w < kDecWarps; ++w) {
         const float wt = (red_m[w][h] == -INFINITY) ? 0.f : ex2(red_m[w][h] - mx);
-        val += wt * (c == 1 ? red_l[w][h] : red_o[w][h][c - 2]);
+        val += wt * (c == 1 ? red_l[w][h] : red_o[(w * G + h) * D + c - 2]);
       }
     }
     a.partial[((static_cast<size_t>(b) * a.Hq + g * G + h) * a.S + split) * (D + 2) + c] = val;
@@ -234,24 +287,33 @@ decode_combine_kernel(const DecodeArgs a, __nv_bfloat16* __restrict__ out) {
 }
 
 template <int D, int G>
-kara_status launch_dg(const DecodeArgs& a, void* out, cudaStream_t stream) {
+kara_status launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, void* out,
+                      cudaStream_t stream) {
   dim3 grid(a.S, a.Hkv, a.B);
-  decode_split_kernel<D, G><<<grid, kDecThreads, 0, stream>>>(a);
+  constexpr size_t smem = split_smem_bytes<D, G>();
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+    attr = true;
+  }
+  decode_split_kernel<D, G><<<grid, kDecThreads, smem, stream>>>(tk, tv, a);
   decode_combine_kernel<D><<<a.B * a.Hq, D, 0, stream>>>(a, static_cast<__nv_bfloat16*>(out));
   return cudaGetLastError() == cudaSuccess ? KARA_OK : KARA_ERR_CUDA;
 }
 
 template <int D>
-kara_status launch_d(const DecodeArgs& a, int G, void* out, cudaStream_t stream) {
+kara_status launch_d(const DecodeArgs& a, int G, const CUtensorMap& tk, const CUtensorMap& tv,
+                     void* out, cudaStream_t stream) {
   switch (G) {
-    case 1: return launch_dg<D, 1>(a, out, stream);
-    case 2: return launch_dg<D, 2>(a, out, stream);
-    case 3: return launch_dg<D, 3>(a, out, stream);
-    case 4: return launch_dg<D, 4>(a, out, stream);
-    case 5: return launch_dg<D, 5>(a, out, stream);
-    case 6: return launch_dg<D, 6>(a, out, stream);
-    case 7: return launch_dg<D, 7>(a, out, stream);
-    case 8: return launch_dg<D, 8>(a, out, stream);
+    case 1: return launch_dg<D, 1>(a, tk, tv, out, stream);
+    case 2: return launch_dg<D, 2>(a, tk, tv, out, stream);
+    case 3: return launch_dg<D, 3>(a, tk, tv, out, stream);
+    case 4: return launch_dg<D, 4>(a, tk, tv, out, stream);
+    case 5: return launch_dg<D, 5>(a, tk, tv, out, stream);
+    case 6: return launch_dg<D, 6>(a, tk, tv, out, stream);
+    case 7: return launch_dg<D, 7>(a, tk, tv, out, stream);
+    case 8: return launch_dg<D, 8>(a, tk, tv, out, stream);
     default: return KARA_ERR_UNSUPPORTED;
   }
 }
@@ -282,8 +344,18 @@ kara_status launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
   a.S = decode_num_splits(L.max_blocks);
   a.cs = L.scale * 1.4426950408889634f;
   const int G = L.Hq / L.Hkv;
-  if (L.D == 128) return launch_d<128>(a, G, L.out, stream);
-  if (L.D == 64) return launch_d<64>(a, G, L.out, stream);
+  // paged pools as 4-D maps {d, Hkv, 16 slots, blocks}; box = one page of one KV head, 64
+  // channels wide, 128-byte swizzle (the same map shape the scoring kernels use)
+  const uint64_t dims[4] = {static_cast<uint64_t>(L.D), static_cast<uint64_t>(L.Hkv), 16,
+                            static_cast<uint64_t>(L.num_blocks)};
+  const uint64_t strides[3] = {static_cast<uint64_t>(L.D) * 2, static_cast<uint64_t>(L.Hkv) * L.D * 2,
+                               static_cast<uint64_t>(16) * L.Hkv * L.D * 2};
+  CUtensorMap tk, tv;
+  if (!make_bf16_map_4d(&tk, L.k_cache, dims, strides, 16) ||
+      !make_bf16_map_4d(&tv, L.v_cache, dims, strides, 16))
+    return KARA_ERR_CUDA;
+  if (L.D == 128) return launch_d<128>(a, G, tk, tv, L.out, stream);
+  if (L.D == 64) return launch_d<64>(a, G, tk, tv, L.out, stream);
   return KARA_ERR_UNSUPPORTED;
 }
 

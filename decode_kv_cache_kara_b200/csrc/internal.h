@@ -3,11 +3,17 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "kara.h"
 
 namespace kara {
+
+// 4-D bf16 tensor map (innermost dimension first), 128-byte swizzle, box {64, 1, rows, 1}.
+// Defined in score.cu.
+bool make_bf16_map_4d(CUtensorMap* map, const void* base, const uint64_t dims[4],
+                      const uint64_t strides[3], uint32_t box_rows);
 
 struct ScoreLaunch {
   const void* q_win;

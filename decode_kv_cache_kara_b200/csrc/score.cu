@@ -20,8 +20,8 @@
 // (TMA box of one page and one KV head); slots outside [n-W, n) are masked in the epilogue.
 // Queries come from the dense window-query buffer [R, W, Hq, d]; rows past W are zero-filled
 // by TMA and carry lse = +inf, so they add nothing in pass 2.
-// The epilogues are bound by exponentials: about a third of them run on the FMA pipe
-// (ex2_fma) and the rest on the SFU, so that both pipes share the load.
+// The epilogues are bound by exponentials: a quarter of them run on the FMA pipe (ex2_fma)
+// and the rest on the SFU, so that both pipes share the load.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -47,9 +47,10 @@ constexpr int kQStages2 = 2;
 constexpr int kRowBytes = 128;       // one 64-element bf16 K-chunk row (128-byte swizzle)
 constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
 
-// Column i of every 64-column group takes the FMA-pipe exponential when this holds (about a
-// third of the columns), the SFU one otherwise: the two pipes then finish together.
-__device__ __forceinline__ constexpr bool fma_exp_column(int i) { return i % 3 == 1; }
+// One exponential in four goes to the FMA pipe (ex2_fma, ~10 issue slots), the other three to
+// the SFU (a quarter of the SFU rate per sub-partition): with the surrounding FFMA/FADD per
+// element this balances issue slots against SFU cycles.
+__device__ __forceinline__ constexpr bool fma_exp_column(int i) { return (i & 3) == 1; }
 
 template <int I>
 __device__ __forceinline__ float exp2_split(float x) {
@@ -180,41 +181,82 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (whole warp: lanes fetch page ids, lane 0 issues) --------
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
-      int qi = 0, ki = 0;
-      uint32_t qph = 0, kph = 0;
-      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-        const int tt = t % TT;
-        const int h = (t / TT) % a.Hq;
-        const int r = t / (TT * a.Hq);
-        const SeqInfo s = seq_info(a, r);
-        if (!s.ok) continue;
+    }
+    int qi = 0, ki = 0;
+    uint32_t qph = 0, kph = 0;
+    // the window's page ids, pages lane, lane+32, lane+64 (a window spans at most 257 pages
+    // for W <= 4096; larger spans are fetched per key tile below)
+    auto load_tile = [&](int t, SeqInfo& s, int (&ids)[3]) {
+      s = seq_info(a, t / (TT * a.Hq));
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        const int p = lane + 32 * j;
+        ids[j] = (s.ok && p < s.np) ? page_block(a, s.b, s.p_first + p) : 0;
+      }
+    };
+    SeqInfo s_cur, s_nxt;
+    int ids_cur[3] = {0, 0, 0}, ids_nxt[3] = {0, 0, 0};
+    if (static_cast<int>(blockIdx.x) < num_tiles) load_tile(blockIdx.x, s_cur, ids_cur);
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      if (t + static_cast<int>(gridDim.x) < num_tiles) load_tile(t + gridDim.x, s_nxt, ids_nxt);
+      const int tt = t % TT;
+      const int h = (t / TT) % a.Hq;
+      const int r = t / (TT * a.Hq);
+      const SeqInfo s = s_cur;
+      bool stop = __shfl_sync(0xffffffffu, *abort_flag != 0 ? 1 : 0, 0) != 0;   // warp-uniform
+      if (s.ok && !stop) {
         const int g = h / a.G;
-        if (!mbar_wait(&q_empty[qi], qph ^ 1, abort_flag, a.status)) break;
-        mbar_expect_tx(&q_full[qi], kQBytes);
-        for (int c = 0; c < NCH; ++c)
-          tma_load_4d(q_buf + qi * kQBytes + c * kQRows1 * kRowBytes, &tm_q, &q_full[qi], c * 64,
-                      h, tt * kQRows1, r);
+        int ok = 1;
+        if (lane == 0) {
+          ok = mbar_wait(&q_empty[qi], qph ^ 1, abort_flag, a.status) ? 1 : 0;
+          if (ok) {
+            mbar_expect_tx(&q_full[qi], kQBytes);
+            for (int c = 0; c < NCH; ++c)
+              tma_load_4d(q_buf + qi * kQBytes + c * kQRows1 * kRowBytes, &tm_q, &q_full[qi],
+                          c * 64, h, tt * kQRows1, r);
+          }
+        }
+        stop = __shfl_sync(0xffffffffu, ok, 0) == 0;
         if (++qi == 2) { qi = 0; qph ^= 1; }
         const int nkt = (s.np + 15) / 16;
-        bool stop = false;
-        for (int kt = 0; kt < nkt; ++kt) {
+        for (int kt = 0; kt < nkt && !stop; ++kt) {
           const int pages = min(16, s.np - kt * 16);
-          if (!mbar_wait(&k_empty[ki], kph ^ 1, abort_flag, a.status)) { stop = true; break; }
-          mbar_expect_tx(&k_full[ki], pages * NCH * kPageBytes);
-          for (int p = 0; p < pages; ++p) {
-            const int blk = page_block(a, s.b, s.p_first + kt * 16 + p);
-            for (int c = 0; c < NCH; ++c)
-              tma_load_4d(k_buf + ki * kKBytes + c * kKRows1 * kRowBytes + p * kPageBytes, &tm_k,
-                          &k_full[ki], c * 64, g, 0, blk);
+          // page ids of this key tile (from the prefetched window list when it holds them)
+          int my_blk = 0;
+          {
+            const int p = kt * 16 + (lane & 15);
+            const int src = p & 31, j = p >> 5;
+            const int v0 = __shfl_sync(0xffffffffu, ids_cur[0], src);
+            const int v1 = __shfl_sync(0xffffffffu, ids_cur[1], src);
+            const int v2 = __shfl_sync(0xffffffffu, ids_cur[2], src);
+            my_blk = j == 0 ? v0 : (j == 1 ? v1 : v2);
+            if (p >= 96 && (lane & 15) < pages) my_blk = page_block(a, s.b, s.p_first + p);
+          }
+          if (lane == 0) {
+            ok = mbar_wait(&k_empty[ki], kph ^ 1, abort_flag, a.status) ? 1 : 0;
+            if (ok) mbar_expect_tx(&k_full[ki], pages * NCH * kPageBytes);
+          }
+          stop = __shfl_sync(0xffffffffu, ok, 0) == 0;
+          if (stop) break;
+          for (int pg = 0; pg < pages; ++pg) {
+            const int blk = __shfl_sync(0xffffffffu, my_blk, pg);
+            if (lane == 0) {
+              for (int c = 0; c < NCH; ++c)
+                tma_load_4d(k_buf + ki * kKBytes + c * kKRows1 * kRowBytes + pg * kPageBytes,
+                            &tm_k, &k_full[ki], c * 64, g, 0, blk);
+            }
           }
           if (++ki == kKStages1) { ki = 0; kph ^= 1; }
         }
-        if (stop) break;
       }
+      s_cur = s_nxt;
+#pragma unroll
+      for (int j = 0; j < 3; ++j) ids_cur[j] = ids_nxt[j];
+      if (stop) break;
     }
   } else if (warp == 1) {
     // ---------------- UMMA issuer ----------------
@@ -263,11 +305,15 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     int ab = 0;
     uint32_t aph = 0;
+    SeqInfo s_nxt;
+    if (static_cast<int>(blockIdx.x) < num_tiles) s_nxt = seq_info(a, blockIdx.x / (TT * a.Hq));
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       const int tt = t % TT;
       const int h = (t / TT) % a.Hq;
       const int r = t / (TT * a.Hq);
-      const SeqInfo s = seq_info(a, r);
+      const SeqInfo s = s_nxt;
+      if (t + static_cast<int>(gridDim.x) < num_tiles)
+        s_nxt = seq_info(a, (t + gridDim.x) / (TT * a.Hq));
       float m = -INFINITY, l = 0.f;
       bool stop = !s.ok;
       if (s.ok) {
@@ -277,50 +323,60 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (!mbar_wait(&acc_full[ab], aph, abort_flag, a.status)) { stop = true; break; }
           tc_fence_after();
           const int c0 = half * 128;
-          const int nsub = max(0, min(8, (ncols - c0) / 16));
+          const int cnt = max(0, min(128, ncols - c0));     // a multiple of 16
+          const int nch = (cnt + 31) / 32;
           const int slot0 = (s.p_first + kt * 16) * 16 + c0;
           const bool edge = (kt == 0) || (kt == nkt - 1);
-          for (int g0 = 0; g0 < nsub; g0 += 4) {
-            float v[64];
+          const uint32_t col0 = lane_base + ab * 256 + c0;
+          // one 32-column chunk: masked max, rescale, exponentials (a quarter on the FMA pipe)
+          auto process = [&](float (&v)[32], int j) {
+            if (cnt - 32 * j == 16) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (g0 + q < nsub) tmem_ld16(lane_base + ab * 256 + c0 + (g0 + q) * 16, v + 16 * q);
-            tmem_wait_ld();
-            reg_fence<64>(v);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (g0 + q >= nsub) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) v[16 * q + i] = -INFINITY;
-              }
+              for (int i = 16; i < 32; ++i) v[i] = -INFINITY;
+            }
             if (edge) {
 #pragma unroll
-              for (int i = 0; i < 64; ++i) {
-                const int slot = slot0 + g0 * 16 + i;
+              for (int i = 0; i < 32; ++i) {
+                const int slot = slot0 + 32 * j + i;
                 if (slot < s.start || slot >= s.n) v[i] = -INFINITY;
               }
             }
-            float mx[8];
+            float mx[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float a0 = fmaxf(v[8 * j], v[8 * j + 1]), a1 = fmaxf(v[8 * j + 2], v[8 * j + 3]);
-              const float a2 = fmaxf(v[8 * j + 4], v[8 * j + 5]), a3 = fmaxf(v[8 * j + 6], v[8 * j + 7]);
-              mx[j] = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+            for (int q = 0; q < 4; ++q) {
+              const float a0 = fmaxf(v[8 * q], v[8 * q + 1]), a1 = fmaxf(v[8 * q + 2], v[8 * q + 3]);
+              const float a2 = fmaxf(v[8 * q + 4], v[8 * q + 5]), a3 = fmaxf(v[8 * q + 6], v[8 * q + 7]);
+              mx[q] = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
             }
-            const float cmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            if (cmax == -INFINITY) continue;
+            const float cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            if (cmax == -INFINITY) return;
             const float m_new = fmaxf(m, cmax * a.cs);
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 64; i += 4) {
-              acc[0] += exp2_split<0>(fmaf(v[i], a.cs, -m_new));
-              acc[1] += exp2_split<1>(fmaf(v[i + 1], a.cs, -m_new));
-              acc[2] += exp2_split<2>(fmaf(v[i + 2], a.cs, -m_new));
-              acc[3] += exp2_split<3>(fmaf(v[i + 3], a.cs, -m_new));
+            for (int i = 0; i < 32; ++i) {
+              const float x = fmaf(v[i], a.cs, -m_new);
+              acc[i & 3] += fma_exp_column(i) ? ex2_fma(x) : ex2(x);
             }
             l = l * ex2(m - m_new) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
             m = m_new;
+          };
+          auto issue = [&](float (&v)[32], int j) {
+            tmem_ld16(col0 + 32 * j, v);
+            if (cnt - 32 * j > 16) tmem_ld16(col0 + 32 * j + 16, v + 16);
+          };
+          float va[32], vb[32];
+          if (nch > 0) issue(va, 0);
+          for (int j = 0; j < nch; j += 2) {
+            tmem_wait_ld();
+            reg_fence<32>(va);
+            if (j + 1 < nch) issue(vb, j + 1);
+            process(va, j);
+            if (j + 1 < nch) {
+              tmem_wait_ld();
+              reg_fence<32>(vb);
+              if (j + 2 < nch) issue(va, j + 2);
+              process(vb, j + 1);
+            }
           }
           tc_fence_before();
           mbar_arrive(&acc_empty[ab]);
@@ -419,28 +475,39 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
+    // whole warp: lanes fetch the tile's page ids in parallel, lane 0 issues the copies
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
-      int ai = 0, bi = 0;
-      uint32_t aph = 0, bph = 0;
-      TileCursor cur;
-      int g, kt;
-      for (int t = blockIdx.x; !*abort_flag && cur.seek(a, t, g, kt); t += gridDim.x) {
-        const SeqInfo& s = cur.s;
-        if (!s.ok) continue;
-        const int r = cur.r;
-        const int pages = min(8, s.np - kt * 8);
-        if (!mbar_wait(&a_empty[ai], aph ^ 1, abort_flag, a.status)) break;
-        mbar_expect_tx(&a_full[ai], pages * NCH * kPageBytes);
-        for (int p = 0; p < pages; ++p) {
-          const int blk = page_block(a, s.b, s.p_first + kt * 8 + p);
+    }
+    int ai = 0, bi = 0;
+    uint32_t aph = 0, bph = 0;
+    TileCursor cur;
+    int g, kt;
+    for (int t = blockIdx.x; cur.seek(a, t, g, kt); t += gridDim.x) {
+      if (__shfl_sync(0xffffffffu, *abort_flag != 0 ? 1 : 0, 0)) break;
+      const SeqInfo& s = cur.s;
+      if (!s.ok) continue;
+      const int r = cur.r;
+      const int pages = min(8, s.np - kt * 8);
+      const int my_blk = lane < pages ? page_block(a, s.b, s.p_first + kt * 8 + lane) : 0;
+      int ok = 1;
+      if (lane == 0) {
+        ok = mbar_wait(&a_empty[ai], aph ^ 1, abort_flag, a.status) ? 1 : 0;
+        if (ok) mbar_expect_tx(&a_full[ai], pages * NCH * kPageBytes);
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      for (int p = 0; p < pages; ++p) {
+        const int blk = __shfl_sync(0xffffffffu, my_blk, p);
+        if (lane == 0) {
           for (int c = 0; c < NCH; ++c)
             tma_load_4d(a_buf + ai * kABytes + c * kKRows2 * kRowBytes + p * kPageBytes, &tm_k,
                         &a_full[ai], c * 64, g, 0, blk);
         }
-        if (++ai == 2) { ai = 0; aph ^= 1; }
-        bool stop = false;
+      }
+      if (++ai == 2) { ai = 0; aph ^= 1; }
+      bool stop = false;
+      if (lane == 0) {
         for (int q = 0; q < NQ; ++q) {
           const int h = g * a.G + q / QT, qt = q % QT;
           if (!mbar_wait(&b_empty[bi], bph ^ 1, abort_flag, a.status)) { stop = true; break; }
@@ -450,8 +517,11 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
                         c * 64, h, qt * kQRows2, r);
           if (++bi == kQStages2) { bi = 0; bph ^= 1; }
         }
-        if (stop) break;
       }
+      // lanes other than 0 track the stage index too (they only read it on the next tile)
+      bi = __shfl_sync(0xffffffffu, bi, 0);
+      bph = __shfl_sync(0xffffffffu, bph, 0);
+      if (__shfl_sync(0xffffffffu, stop ? 1 : 0, 0)) break;
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -526,22 +596,35 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!aborted) {
           tc_fence_after();
           const float* lh = ls + half * 128;
+          const uint32_t col0 = lane_base + ab * 256 + half * 128;
+          auto issue = [&](float (&v)[32], int j) {
+            tmem_ld16(col0 + 32 * j, v);
+            tmem_ld16(col0 + 32 * j + 16, v + 16);
+          };
+          auto process = [&](const float (&v)[32], int j) {
 #pragma unroll
-          for (int g0 = 0; g0 < 8; g0 += 4) {
-            float v[64];
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq)
-              tmem_ld16(lane_base + ab * 256 + half * 128 + (g0 + qq) * 16, v + 16 * qq);
-            tmem_wait_ld();
-            reg_fence<64>(v);
-#pragma unroll
-            for (int i = 0; i < 64; i += 4) {
-              const float4 lz = *reinterpret_cast<const float4*>(lh + g0 * 16 + i);
-              acc[0] += exp2_split<0>(fmaf(v[i], a.cs, -lz.x));
-              acc[1] += exp2_split<1>(fmaf(v[i + 1], a.cs, -lz.y));
-              acc[2] += exp2_split<2>(fmaf(v[i + 2], a.cs, -lz.z));
-              acc[3] += exp2_split<3>(fmaf(v[i + 3], a.cs, -lz.w));
+            for (int i = 0; i < 32; i += 4) {
+              const float4 lz = *reinterpret_cast<const float4*>(lh + 32 * j + i);
+              const float x0 = fmaf(v[i], a.cs, -lz.x), x1 = fmaf(v[i + 1], a.cs, -lz.y);
+              const float x2 = fmaf(v[i + 2], a.cs, -lz.z), x3 = fmaf(v[i + 3], a.cs, -lz.w);
+              acc[0] += fma_exp_column(i) ? ex2_fma(x0) : ex2(x0);
+              acc[1] += fma_exp_column(i + 1) ? ex2_fma(x1) : ex2(x1);
+              acc[2] += fma_exp_column(i + 2) ? ex2_fma(x2) : ex2(x2);
+              acc[3] += fma_exp_column(i + 3) ? ex2_fma(x3) : ex2(x3);
             }
+          };
+          float va[32], vb[32];
+          issue(va, 0);
+#pragma unroll
+          for (int j = 0; j < 4; j += 2) {
+            tmem_wait_ld();
+            reg_fence<32>(va);
+            issue(vb, j + 1);
+            process(va, j);
+            tmem_wait_ld();
+            reg_fence<32>(vb);
+            if (j + 2 < 4) issue(va, j + 2);
+            process(vb, j + 1);
           }
           tc_fence_before();
           mbar_arrive(&acc_empty[ab]);
@@ -674,6 +757,11 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
 }
 
 }  // namespace
+
+bool make_bf16_map_4d(CUtensorMap* map, const void* base, const uint64_t dims[4],
+                      const uint64_t strides[3], uint32_t box_rows) {
+  return make_map(map, base, dims, strides, box_rows);
+}
 
 int score_lse_stride(int W) { return (W + 255) / 256 * 256; }
 
