@@ -1,12 +1,34 @@
 // C-ABI entry points of libkara: host-side argument checks, workspace carving, launches.
 // Semantics of every call are documented in include/kara.h.
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 
 #include "internal.h"
 #include "kara.h"
 
 using namespace kara;
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+}  // namespace
+
+namespace kara {
+
+void set_last_error(const char* where, const char* what) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, what);
+}
+
+kara_status check_launch(const char* where) {
+  const cudaError_t err = cudaGetLastError();
+  if (err == cudaSuccess) return KARA_OK;
+  set_last_error(where, cudaGetErrorString(err));
+  return KARA_ERR_CUDA;
+}
+
+}  // namespace kara
 
 namespace {
 
@@ -62,6 +84,8 @@ const char* kara_status_str(int32_t status) {
 }
 
 const char* kara_version(void) { return "kara-b200 0.1"; }
+
+const char* kara_last_error(void) { return g_last_error; }
 
 size_t kara_workspace_bytes(kara_op op, const kara_pool* pool, int32_t num_seqs, int32_t window,
                             int32_t num_q_heads, int32_t k_or_budget) {

@@ -251,6 +251,33 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
   return bits_f2(r);
 }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(r);
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(r);
+}
+
+// ex2_fma on a pair, with packed fp32 arithmetic (same method and error as ex2_fma).
+__device__ __forceinline__ float2 ex2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 shifter = make_float2(12582912.0f, 12582912.0f);
+  const float2 t = fadd2(x, shifter);
+  const float2 f = fsub2(x, fsub2(t, shifter));
+  float2 p = ffma2(make_float2(0.009570102207362652f, 0.009570102207362652f), f,
+                   make_float2(0.05591785907745361f, 0.05591785907745361f));
+  p = ffma2(p, f, make_float2(0.240247443318367f, 0.240247443318367f));
+  p = ffma2(p, f, make_float2(0.6931217908859253f, 0.6931217908859253f));
+  p = ffma2(p, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // Both bf16 halves of a packed word as an fp32 pair (exact).
 __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
   return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));

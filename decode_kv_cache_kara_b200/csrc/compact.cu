@@ -431,7 +431,7 @@ kara_status launch_compact(const CompactLaunch& L, cudaStream_t stream) {
   fp.max_blocks = L.max_blocks;
   fp.k = L.k;
   finalize_kernel<<<8, 256, 0, stream>>>(fp);
-  return cudaGetLastError() == cudaSuccess ? KARA_OK : KARA_ERR_CUDA;
+  return check_launch(__func__);
 }
 
 kara_status launch_lacache(const LacacheLaunch& L, cudaStream_t stream) {
@@ -481,7 +481,7 @@ kara_status launch_lacache(const LacacheLaunch& L, cudaStream_t stream) {
   fp.max_blocks = L.max_blocks;
   fp.k = L.budget;
   finalize_kernel<<<8, 256, 0, stream>>>(fp);
-  return cudaGetLastError() == cudaSuccess ? KARA_OK : KARA_ERR_CUDA;
+  return check_launch(__func__);
 }
 
 }  // namespace kara

@@ -299,7 +299,7 @@ kara_status launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensor
   }
   decode_split_kernel<D, G><<<grid, kDecThreads, smem, stream>>>(tk, tv, a);
   decode_combine_kernel<D><<<a.B * a.Hq, D, 0, stream>>>(a, static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError() == cudaSuccess ? KARA_OK : KARA_ERR_CUDA;
+  return check_launch(__func__);
 }
 
 template <int D>

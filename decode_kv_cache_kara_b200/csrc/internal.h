@@ -15,6 +15,11 @@ namespace kara {
 bool make_bf16_map_4d(CUtensorMap* map, const void* base, const uint64_t dims[4],
                       const uint64_t strides[3], uint32_t box_rows);
 
+// Records the pending CUDA error (if any) under `where` for kara_last_error() and returns
+// KARA_OK or KARA_ERR_CUDA. Defined in api.cu.
+kara_status check_launch(const char* where);
+void set_last_error(const char* where, const char* what);
+
 struct ScoreLaunch {
   const void* q_win;
   const void* k_cache;

@@ -9,8 +9,8 @@
 // section 1: a token the current reasoning refers to strongly scores high).
 //
 // Two passes, both persistent and warp-specialised (warp 0: TMA producer, warp 1: UMMA
-// issuer and TMEM owner, warps 2-9: epilogue, one TMEM lane per thread and two warps per lane
-// quadrant, each on half of the accumulator columns):
+// issuer and TMEM owner, the other warps: epilogue, one TMEM lane per thread, kParts warps per
+// lane quadrant, each on 256/kParts of the accumulator columns):
 //   pass 1 (query-major)  S = Q K^T, 128 query rows x up to 256 keys per UMMA tile; each
 //                         epilogue thread owns one query row and keeps an online base-2
 //                         log-sum-exp; the result goes to the workspace.
@@ -20,8 +20,9 @@
 // (TMA box of one page and one KV head); slots outside [n-W, n) are masked in the epilogue.
 // Queries come from the dense window-query buffer [R, W, Hq, d]; rows past W are zero-filled
 // by TMA and carry lse = +inf, so they add nothing in pass 2.
-// The epilogues are bound by exponentials: a quarter of them run on the FMA pipe (ex2_fma)
-// and the rest on the SFU, so that both pipes share the load.
+// The epilogues are bound by exponentials: a quarter of them run on the FMA pipe (ex2_fma2)
+// and the rest on the SFU, so that both pipes share the load; the arithmetic around them
+// uses packed fp32 pairs.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -35,8 +36,14 @@ namespace kara {
 
 namespace {
 
-constexpr int kThreads = 320;        // warp 0: TMA, warp 1: UMMA + TMEM, warps 2-9: epilogue
-constexpr int kEpiThreads = 256;
+#ifndef KARA_SCORE_EPI_WARPS
+#define KARA_SCORE_EPI_WARPS 8
+#endif
+constexpr int kEpiWarps = KARA_SCORE_EPI_WARPS;  // a multiple of 4: warps per TMEM lane quadrant
+constexpr int kParts = kEpiWarps / 4;            // column parts of each 256-column accumulator
+constexpr int kThreads = 64 + 32 * kEpiWarps;    // warp 0: TMA, warp 1: UMMA + TMEM, rest: epilogue
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kPartCols = 256 / kParts;          // accumulator columns per epilogue warp and tile
 constexpr uint32_t kEpiBarrier = 1;  // named barrier among the epilogue warps
 constexpr int kQRows1 = 128;         // pass 1: query rows per tile (UMMA M)
 constexpr int kKRows1 = 256;         // pass 1: max keys per UMMA (N)
@@ -47,15 +54,13 @@ constexpr int kQStages2 = 2;
 constexpr int kRowBytes = 128;       // one 64-element bf16 K-chunk row (128-byte swizzle)
 constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
 
-// One exponential in four goes to the FMA pipe (ex2_fma, ~10 issue slots), the other three to
-// the SFU (a quarter of the SFU rate per sub-partition): with the surrounding FFMA/FADD per
-// element this balances issue slots against SFU cycles.
-__device__ __forceinline__ constexpr bool fma_exp_column(int i) { return (i & 3) == 1; }
-
-template <int I>
-__device__ __forceinline__ float exp2_split(float x) {
-  if constexpr (fma_exp_column(I)) return ex2_fma(x);
-  else return ex2(x);
+// Exponentials of 8 consecutive columns as 4 pairs: three pairs on the SFU, one pair on the
+// FMA pipe (ex2_fma2). With the packed FFMA/FADD around them this balances issue slots
+// against SFU cycles (the SFU delivers a quarter of a warp instruction per cycle per
+// sub-partition).
+__device__ __forceinline__ float2 exp2_pair(float2 x, int pair_in_group) {
+  if (pair_in_group == 3) return ex2_fma2(x);
+  return make_float2(ex2(x.x), ex2(x.y));
 }
 
 struct ScoreArgs {
@@ -141,8 +146,8 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
                                              ~uintptr_t(1023));
   uint8_t* q_buf = smem;                      // 2 x kQBytes
   uint8_t* k_buf = smem + 2 * kQBytes;        // kKStages1 x kKBytes
-  float2* comb = reinterpret_cast<float2*>(k_buf + kKStages1 * kKBytes);   // [128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(comb + kQRows1);
+  float2* comb = reinterpret_cast<float2*>(k_buf + kKStages1 * kKBytes);   // [kParts-1][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(comb + 3 * kQRows1);
   uint64_t* q_full = bars;        // [2]
   uint64_t* q_empty = bars + 2;   // [2]
   uint64_t* k_full = bars + 4;    // [kKStages1]
@@ -297,12 +302,13 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
   } else {
-    // ------------- epilogue: one query row per TMEM lane, two warps per lane quadrant -------------
+    // ---------- epilogue: one query row per TMEM lane, four warps per lane quadrant ----------
     const int e = warp - 2;
     const int quad = warp & 3;
-    const int half = e >> 2;              // which 128 columns of each 256-column tile
+    const int part = e >> 2;              // which 64 columns of each 256-column tile
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    const float2 cs2 = make_float2(a.cs, a.cs);
     int ab = 0;
     uint32_t aph = 0;
     SeqInfo s_nxt;
@@ -322,13 +328,13 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int ncols = min(16, s.np - kt * 16) * 16;
           if (!mbar_wait(&acc_full[ab], aph, abort_flag, a.status)) { stop = true; break; }
           tc_fence_after();
-          const int c0 = half * 128;
-          const int cnt = max(0, min(128, ncols - c0));     // a multiple of 16
-          const int nch = (cnt + 31) / 32;
+          const int c0 = part * kPartCols;
+          const int cnt = max(0, min(kPartCols, ncols - c0));     // a multiple of 16
           const int slot0 = (s.p_first + kt * 16) * 16 + c0;
           const bool edge = (kt == 0) || (kt == nkt - 1);
           const uint32_t col0 = lane_base + ab * 256 + c0;
-          // one 32-column chunk: masked max, rescale, exponentials (a quarter on the FMA pipe)
+          const int nch = (cnt + 31) / 32;
+          // one 32-column chunk: masked max, rescale, exponentials
           auto process = [&](float (&v)[32], int j) {
             if (cnt - 32 * j == 16) {
 #pragma unroll
@@ -351,13 +357,17 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
             const float cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             if (cmax == -INFINITY) return;
             const float m_new = fmaxf(m, cmax * a.cs);
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            const float2 nm2 = make_float2(-m_new, -m_new);
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float x = fmaf(v[i], a.cs, -m_new);
-              acc[i & 3] += fma_exp_column(i) ? ex2_fma(x) : ex2(x);
+            for (int i = 0; i < 32; i += 4) {
+              const float2 x0 = ffma2(make_float2(v[i], v[i + 1]), cs2, nm2);
+              const float2 x1 = ffma2(make_float2(v[i + 2], v[i + 3]), cs2, nm2);
+              acc0 = fadd2(acc0, exp2_pair(x0, (i >> 1) & 3));
+              acc1 = fadd2(acc1, exp2_pair(x1, ((i >> 1) + 1) & 3));
             }
-            l = l * ex2(m - m_new) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+            const float2 acc = fadd2(acc0, acc1);
+            l = l * ex2(m - m_new) + (acc.x + acc.y);
             m = m_new;
           };
           auto issue = [&](float (&v)[32], int j) {
@@ -370,30 +380,50 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
             tmem_wait_ld();
             reg_fence<32>(va);
             if (j + 1 < nch) issue(vb, j + 1);
+            if (j + 1 >= nch) {            // all of this part's columns are in registers
+              tc_fence_before();
+              mbar_arrive(&acc_empty[ab]);
+            }
             process(va, j);
             if (j + 1 < nch) {
               tmem_wait_ld();
               reg_fence<32>(vb);
               if (j + 2 < nch) issue(va, j + 2);
+              else {
+                tc_fence_before();
+                mbar_arrive(&acc_empty[ab]);
+              }
               process(vb, j + 1);
             }
           }
-          tc_fence_before();
-          mbar_arrive(&acc_empty[ab]);
+          if (nch == 0) {
+            tc_fence_before();
+            mbar_arrive(&acc_empty[ab]);
+          }
           if (++ab == 2) { ab = 0; aph ^= 1; }
         }
-      } else if (tt == 0 && h == 0 && row == 0 && half == 0) {
+      } else if (tt == 0 && h == 0 && row == 0 && part == 0) {
         report(a.status, KARA_ERR_INVALID_ARG);
       }
-      // merge the two column halves of the row
-      if (half == 1) comb[row] = make_float2(stop ? NAN : m, l);
+      // merge the four column parts of the row
+      if (part > 0) comb[(part - 1) * kQRows1 + row] = make_float2(stop ? NAN : m, l);
       named_barrier(kEpiBarrier, kEpiThreads);
-      if (half == 0) {
-        const float2 o = comb[row];
+      if (part == 0) {
         float lse2 = INFINITY;
-        if (!stop && !isnan(o.x)) {
-          const float mm = fmaxf(m, o.x);
-          const float ll = l * ex2(m - mm) + (o.x == -INFINITY ? 0.f : o.y * ex2(o.x - mm));
+        float mm = m;
+        bool bad = stop;
+        float2 o[kParts - 1];
+#pragma unroll
+        for (int q = 0; q < kParts - 1; ++q) {
+          o[q] = comb[q * kQRows1 + row];
+          bad = bad || isnan(o[q].x);
+          mm = fmaxf(mm, o[q].x);
+        }
+        if (!bad) {
+          float ll = l * ex2(m - mm);
+#pragma unroll
+          for (int q = 0; q < kParts - 1; ++q)
+            if (o[q].x != -INFINITY) ll += o[q].y * ex2(o[q].x - mm);
           lse2 = mm + __log2f(ll);
         }
         const int token = tt * kQRows1 + row;
@@ -435,8 +465,8 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint8_t* a_buf = smem;                    // 2 x kABytes (key tiles)
   uint8_t* b_buf = smem + 2 * kABytes;      // kQStages2 x kBBytes (query tiles)
   float* lse_s = reinterpret_cast<float*>(b_buf + kQStages2 * kBBytes);   // [2][256]
-  float* red = lse_s + 2 * kQRows2;                                       // [128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + kKRows2);
+  float* red = lse_s + 2 * kQRows2;                                       // [3][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 3 * kKRows2);
   uint64_t* a_full = bars;                  // [2]
   uint64_t* a_empty = bars + 2;             // [2]
   uint64_t* b_full = bars + 4;              // [kQStages2]
@@ -559,13 +589,14 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
   } else {
-    // ------------- epilogue: one key per TMEM lane, two warps per lane quadrant -------------
+    // ------------- epilogue: one key per TMEM lane, four warps per lane quadrant -------------
     const int e = warp - 2;
-    const int etid = e * 32 + lane;       // 0..255: the query column whose lse it stages
+    const int etid = e * 32 + lane;       // 0..511; the first 256 stage the tile's lse values
     const int quad = warp & 3;
-    const int half = e >> 2;              // which 128 query columns of each tile
+    const int part = e >> 2;              // which 64 query columns of each tile
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    const float2 cs2 = make_float2(a.cs, a.cs);
     int ab = 0, qbuf = 0;
     uint32_t cph = 0;
     bool aborted = false;
@@ -577,17 +608,17 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
       float* out = a.scores + (static_cast<size_t>(r) * a.Hkv + g) * a.W;
       if (!s.ok) {
         const int j = kt * kKRows2 + row;
-        if (half == 0 && j < a.W) out[j] = 0.f;
+        if (part == 0 && j < a.W) out[j] = 0.f;
         continue;
       }
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
       const float* lse_rows = a.lse + (static_cast<size_t>(r) * a.Hq + g * a.G) * a.Wp;
-      float lv = lse_rows[etid];
+      float lv = etid < kQRows2 ? lse_rows[etid] : 0.f;
       for (int q = 0; q < NQ; ++q) {
-        // stage this tile's 256 lse values; prefetch the next tile's into a register
+        // stage this tile's 256 lse values (negated); prefetch the next tile's
         float* ls = lse_s + qbuf * kQRows2;
-        ls[etid] = lv;
-        if (q + 1 < NQ) {
+        if (etid < kQRows2) ls[etid] = -lv;
+        if (q + 1 < NQ && etid < kQRows2) {
           const int h1 = (q + 1) / QT, qt1 = (q + 1) % QT;
           lv = lse_rows[static_cast<size_t>(h1) * a.Wp + qt1 * kQRows2 + etid];
         }
@@ -595,8 +626,9 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!aborted && !mbar_wait(&acc_full[ab], cph, abort_flag, a.status)) aborted = true;
         if (!aborted) {
           tc_fence_after();
-          const float* lh = ls + half * 128;
-          const uint32_t col0 = lane_base + ab * 256 + half * 128;
+          const uint32_t col0 = lane_base + ab * 256 + part * kPartCols;
+          const float* lh = ls + part * kPartCols;
+          constexpr int nch = kPartCols / 32;
           auto issue = [&](float (&v)[32], int j) {
             tmem_ld16(col0 + 32 * j, v);
             tmem_ld16(col0 + 32 * j + 16, v + 16);
@@ -604,42 +636,52 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
           auto process = [&](const float (&v)[32], int j) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
-              const float4 lz = *reinterpret_cast<const float4*>(lh + 32 * j + i);
-              const float x0 = fmaf(v[i], a.cs, -lz.x), x1 = fmaf(v[i + 1], a.cs, -lz.y);
-              const float x2 = fmaf(v[i + 2], a.cs, -lz.z), x3 = fmaf(v[i + 3], a.cs, -lz.w);
-              acc[0] += fma_exp_column(i) ? ex2_fma(x0) : ex2(x0);
-              acc[1] += fma_exp_column(i + 1) ? ex2_fma(x1) : ex2(x1);
-              acc[2] += fma_exp_column(i + 2) ? ex2_fma(x2) : ex2(x2);
-              acc[3] += fma_exp_column(i + 3) ? ex2_fma(x3) : ex2(x3);
+              const float4 nl = *reinterpret_cast<const float4*>(lh + 32 * j + i);
+              const float2 x0 = ffma2(make_float2(v[i], v[i + 1]), cs2, make_float2(nl.x, nl.y));
+              const float2 x1 = ffma2(make_float2(v[i + 2], v[i + 3]), cs2, make_float2(nl.z, nl.w));
+              acc0 = fadd2(acc0, exp2_pair(x0, (i >> 1) & 3));
+              acc1 = fadd2(acc1, exp2_pair(x1, ((i >> 1) + 1) & 3));
             }
           };
           float va[32], vb[32];
           issue(va, 0);
 #pragma unroll
-          for (int j = 0; j < 4; j += 2) {
+          for (int j = 0; j < nch; j += 2) {
             tmem_wait_ld();
             reg_fence<32>(va);
-            issue(vb, j + 1);
+            if (j + 1 < nch) issue(vb, j + 1);
+            else {
+              tc_fence_before();
+              mbar_arrive(&acc_empty[ab]);
+            }
             process(va, j);
-            tmem_wait_ld();
-            reg_fence<32>(vb);
-            if (j + 2 < 4) issue(va, j + 2);
-            process(vb, j + 1);
+            if (j + 1 < nch) {
+              tmem_wait_ld();
+              reg_fence<32>(vb);
+              if (j + 2 < nch) issue(va, j + 2);
+              else {
+                tc_fence_before();
+                mbar_arrive(&acc_empty[ab]);
+              }
+              process(vb, j + 1);
+            }
           }
-          tc_fence_before();
-          mbar_arrive(&acc_empty[ab]);
           if (++ab == 2) { ab = 0; cph ^= 1; }
         }
         qbuf ^= 1;
       }
-      // merge the two query halves of each key
-      const float total = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-      if (half == 1) red[row] = total;
+      // merge the query parts of each key
+      const float2 acc = fadd2(acc0, acc1);
+      const float total = acc.x + acc.y;
+      if (part > 0) red[(part - 1) * kKRows2 + row] = total;
       named_barrier(kEpiBarrier, kEpiThreads);
-      if (half == 0 && !aborted) {
+      if (part == 0 && !aborted) {
         const int slot = (s.p_first + kt * 8) * 16 + row;
         const int j = slot - s.start;
-        if (row < min(8, s.np - kt * 8) * 16 && j >= 0 && j < a.W) out[j] = total + red[row];
+        float sum = total;
+#pragma unroll
+        for (int q = 0; q < kParts - 1; ++q) sum += red[q * kKRows2 + row];
+        if (row < min(8, s.np - kt * 8) * 16 && j >= 0 && j < a.W) out[j] = sum;
       }
       named_barrier(kEpiBarrier, kEpiThreads);
     }
@@ -656,12 +698,26 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
 template <int D>
 constexpr size_t rowstats_smem() {
   return 1024 + 2 * (D / 64) * kQRows1 * kRowBytes + kKStages1 * (D / 64) * kKRows1 * kRowBytes +
-         kQRows1 * sizeof(float2) + 256;
+         3 * kQRows1 * sizeof(float2) + 256;
 }
 template <int D>
 constexpr size_t colsum_smem() {
   return 1024 + 2 * (D / 64) * kKRows2 * kRowBytes + kQStages2 * (D / 64) * kQRows2 * kRowBytes +
-         (2 * kQRows2 + kKRows2) * sizeof(float) + 256;
+         (2 * kQRows2 + 3 * kKRows2) * sizeof(float) + 256;
+}
+
+// Appends the kernel's resource attributes to the last-error text (after a refused launch).
+void describe_kernel(const char* name, const void* fn, int threads, size_t dyn_smem) {
+  cudaFuncAttributes at;
+  char buf[400];
+  if (cudaFuncGetAttributes(&at, fn) == cudaSuccess) {
+    std::snprintf(buf, sizeof(buf),
+                  "launch refused: %d threads, %zu B dynamic smem; kernel uses %d regs, max %d "
+                  "threads/block, %zu B static smem, max dynamic smem %d B",
+                  threads, dyn_smem, at.numRegs, at.maxThreadsPerBlock, at.sharedSizeBytes,
+                  at.maxDynamicSharedSizeBytes);
+    set_last_error(name, buf);
+  }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -715,8 +771,10 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
                             static_cast<uint64_t>(16) * L.Hkv * D * 2};
   CUtensorMap tq1, tq2, tk;
   if (!make_map(&tq1, L.q_win, qdims, qstr, kQRows1) ||
-      !make_map(&tq2, L.q_win, qdims, qstr, kQRows2) || !make_map(&tk, L.k_cache, kdims, kstr, 16))
+      !make_map(&tq2, L.q_win, qdims, qstr, kQRows2) || !make_map(&tk, L.k_cache, kdims, kstr, 16)) {
+    set_last_error("kara_score", "cuTensorMapEncodeTiled failed");
     return KARA_ERR_CUDA;
+  }
 
   ScoreArgs a;
   a.block_table = L.block_table;
@@ -750,9 +808,17 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   const int tiles2 = L.R * L.Hkv * KT;
   const int sms = sm_count();
   score_rowstats_kernel<D><<<min(tiles1, sms), kThreads, rowstats_smem<D>(), stream>>>(tq1, tk, a);
-  if (cudaGetLastError() != cudaSuccess) return KARA_ERR_CUDA;
+  if (check_launch("score_rowstats_kernel") != KARA_OK) {
+    describe_kernel("score_rowstats_kernel", reinterpret_cast<const void*>(score_rowstats_kernel<D>),
+                    kThreads, rowstats_smem<D>());
+    return KARA_ERR_CUDA;
+  }
   score_colsum_kernel<D><<<min(tiles2, sms), kThreads, colsum_smem<D>(), stream>>>(tq2, tk, a);
-  if (cudaGetLastError() != cudaSuccess) return KARA_ERR_CUDA;
+  if (check_launch("score_colsum_kernel") != KARA_OK) {
+    describe_kernel("score_colsum_kernel", reinterpret_cast<const void*>(score_colsum_kernel<D>),
+                    kThreads, colsum_smem<D>());
+    return KARA_ERR_CUDA;
+  }
   return KARA_OK;
 }
 

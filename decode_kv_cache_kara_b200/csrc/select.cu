@@ -272,7 +272,7 @@ kara_status launch_select(const float* scores, int rows, int W, int k, int32_t* 
                           cudaStream_t stream) {
   if (rows == 0) return KARA_OK;
   select_kernel<<<rows, kSelThreads, select_smem(W), stream>>>(scores, W, k, sel);
-  return cudaGetLastError() == cudaSuccess ? KARA_OK : KARA_ERR_CUDA;
+  return check_launch(__func__);
 }
 
 kara_status launch_token2chunk(const float* scores, const int32_t* sel, int rows, int W, int k,
@@ -281,7 +281,7 @@ kara_status launch_token2chunk(const float* scores, const int32_t* sel, int rows
   if (rows == 0) return KARA_OK;
   token2chunk_kernel<<<rows, kSelThreads, t2c_smem(W), stream>>>(scores, sel, W, k, num_anchors,
                                                                  gap_limit, widen, keep);
-  return cudaGetLastError() == cudaSuccess ? KARA_OK : KARA_ERR_CUDA;
+  return check_launch(__func__);
 }
 
 }  // namespace kara

@@ -39,7 +39,10 @@ class KaraLibraryError(ImportError):
 class KaraError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {status_str(code)} ({code})")
+        detail = ""
+        if code == ERR_CUDA:
+            detail = " [" + lib().kara_last_error().decode() + "]"
+        super().__init__(f"{where}: {status_str(code)} ({code}){detail}")
 
 
 class _LayerKV(ctypes.Structure):
@@ -79,6 +82,7 @@ _SIGNATURES = {
     "kara_workspace_bytes": ([_I, ctypes.POINTER(_Pool), _I, _I, _I, _I], _Z),
     "kara_status_str": ([_I], ctypes.c_char_p),
     "kara_version": ([], ctypes.c_char_p),
+    "kara_last_error": ([], ctypes.c_char_p),
 }
 
 

@@ -262,6 +262,11 @@ size_t kara_workspace_bytes(kara_op op, const kara_pool* pool, int32_t num_seqs,
 /* Static, human-readable name of a status code. */
 const char* kara_status_str(int32_t status);
 
+/* Text of the CUDA error behind the calling thread's last KARA_ERR_CUDA return (with the
+ * name of the step that failed), or "" if there was none. Valid until the thread's next
+ * call into the library. */
+const char* kara_last_error(void);
+
 /* Library version string ("kara-b200 <major>.<minor>"). */
 const char* kara_version(void);
 
