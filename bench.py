@@ -175,7 +175,7 @@ class Step:
                  K.kara_workspace_bytes(K.OP_DECODE, self.pool, 0, 0, hq, 0))
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
         self.na = K.anchors_for(wl.anchor_frac, wl.keep)
-        self.launches_per_step = 2 + 1 + 1 + 3 + 2
+        self.launches_per_step = 3 + 1 + 1 + 3 + 2
 
     def restore(self):
         for k, t in self.saved.items():

@@ -92,8 +92,7 @@ size_t kara_workspace_bytes(kara_op op, const kara_pool* pool, int32_t num_seqs,
   switch (op) {
     case KARA_OP_SCORE:
       if (num_seqs <= 0 || window <= 0 || num_q_heads <= 0) return 0;
-      return static_cast<size_t>(num_seqs) * num_q_heads * score_lse_stride(window) *
-             sizeof(float);
+      return score_workspace_bytes(num_seqs, window, num_q_heads);
     case KARA_OP_COMPACT:
       if (num_seqs <= 0 || k_or_budget <= 0) return 0;
       return compact_workspace_bytes(num_seqs, window, k_or_budget);

@@ -34,6 +34,8 @@ struct ScoreLaunch {
   float scale;
 };
 int score_lse_stride(int W);
+int score_chunks(int W);
+size_t score_workspace_bytes(int R, int W, int Hq);
 kara_status launch_score_kernels(const ScoreLaunch& L, cudaStream_t stream);
 
 kara_status launch_select(const float* scores, int rows, int W, int k, int32_t* sel,

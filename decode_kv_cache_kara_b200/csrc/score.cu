@@ -26,6 +26,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 
@@ -39,6 +40,10 @@ namespace {
 #ifndef KARA_SCORE_EPI_WARPS
 #define KARA_SCORE_EPI_WARPS 8
 #endif
+// 1: packed fp32x2 arithmetic in the epilogues; 0: scalar
+#ifndef KARA_SCORE_PACKED
+#define KARA_SCORE_PACKED 1
+#endif
 constexpr int kEpiWarps = KARA_SCORE_EPI_WARPS;  // a multiple of 4: warps per TMEM lane quadrant
 constexpr int kParts = kEpiWarps / 4;            // column parts of each 256-column accumulator
 constexpr int kThreads = 64 + 32 * kEpiWarps;    // warp 0: TMA, warp 1: UMMA + TMEM, rest: epilogue
@@ -47,7 +52,7 @@ constexpr int kPartCols = 256 / kParts;          // accumulator columns per epil
 constexpr uint32_t kEpiBarrier = 1;  // named barrier among the epilogue warps
 constexpr int kQRows1 = 128;         // pass 1: query rows per tile (UMMA M)
 constexpr int kKRows1 = 256;         // pass 1: max keys per UMMA (N)
-constexpr int kKStages1 = 2;
+constexpr int kQStages1 = 2;
 constexpr int kKRows2 = 128;         // pass 2: keys per tile (UMMA M)
 constexpr int kQRows2 = 256;         // pass 2: queries per UMMA (N)
 constexpr int kQStages2 = 2;
@@ -67,7 +72,10 @@ struct ScoreArgs {
   const int32_t* block_table;
   const int32_t* ctx_len;
   const int32_t* seq_ids;
-  float* lse;       // [R, Hq, Wp] base-2 log-sum-exp of scaled logits per query
+  float* lse;         // [R, Hq, CM, Wp] base-2 log-sum-exp of scaled logits per query and
+                      // key chunk (16 pages), from pass 1
+  float* lse_merged;  // [R, Hq, Wp] the chunks merged (+inf past the window)
+  int CM;             // key chunks per window, at most
   float* scores;    // [R, Hkv, W]
   int32_t* status;
   int R, W, Wp, Hq, Hkv, G;
@@ -129,8 +137,39 @@ struct TileCursor {
   }
 };
 
+// Pass-1 work list: tiles (r, g, c, hl) = key chunk c (16 pages of KV head g) against the
+// window queries of query head g*G + hl, for valid sequences only, (r, g, c)-major so that
+// neighbouring tiles share the key chunk in L2.
+struct RowTileCursor {
+  int r = 0, base = 0, per = -1, nc = 0;
+  SeqInfo s;
+  __device__ __forceinline__ bool seek(const ScoreArgs& a, int t, int& g, int& c, int& hl) {
+    while (true) {
+      if (r >= a.R) return false;
+      if (per < 0) {
+        s = seq_info(a, r);
+        nc = s.ok ? (s.np + 15) / 16 : 0;
+        per = a.Hkv * nc * a.G;
+      }
+      if (t < base + per) break;
+      base += per;
+      ++r;
+      per = -1;
+    }
+    int local = t - base;
+    hl = local % a.G;
+    local /= a.G;
+    c = local % nc;
+    g = local / nc;
+    return true;
+  }
+};
+
 // ----------------------------------------------------------------------------------------
-// Pass 1: per-query base-2 log-sum-exp over the window keys.
+// Pass 1: per-query base-2 log-sum-exp over each 16-page key chunk of the window.
+// The chunk (up to 256 keys) stays in shared memory while 128-query tiles of one query head
+// stream through it: S = Q K^T (UMMA M = 128 queries, N = the chunk's keys). The partial
+// results of the chunks are merged when pass 2 stages them.
 // ----------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -144,34 +183,33 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* q_buf = smem;                      // 2 x kQBytes
-  uint8_t* k_buf = smem + 2 * kQBytes;        // kKStages1 x kKBytes
-  float2* comb = reinterpret_cast<float2*>(k_buf + kKStages1 * kKBytes);   // [kParts-1][128]
+  uint8_t* k_buf = smem;                      // 2 x kKBytes (key chunks)
+  uint8_t* q_buf = smem + 2 * kKBytes;        // kQStages1 x kQBytes (query tiles)
+  float2* comb = reinterpret_cast<float2*>(q_buf + kQStages1 * kQBytes);   // [kParts-1][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(comb + 3 * kQRows1);
-  uint64_t* q_full = bars;        // [2]
-  uint64_t* q_empty = bars + 2;   // [2]
-  uint64_t* k_full = bars + 4;    // [kKStages1]
-  uint64_t* k_empty = bars + 4 + kKStages1;
-  uint64_t* acc_full = bars + 4 + 2 * kKStages1;   // [2]
+  uint64_t* k_full = bars;                    // [2]
+  uint64_t* k_empty = bars + 2;               // [2]
+  uint64_t* q_full = bars + 4;                // [kQStages1]
+  uint64_t* q_empty = bars + 4 + kQStages1;
+  uint64_t* acc_full = bars + 4 + 2 * kQStages1;   // [2]
   uint64_t* acc_empty = acc_full + 2;              // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int TT = (a.W + kQRows1 - 1) / kQRows1;
-  const int num_tiles = a.R * a.Hq * TT;
+  const int TT = (a.W + kQRows1 - 1) / kQRows1;   // query tiles per head
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], kEpiThreads);
     }
-    for (int i = 0; i < kKStages1; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
+    for (int i = 0; i < kQStages1; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -186,103 +224,71 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- TMA producer (whole warp: lanes fetch page ids, lane 0 issues) --------
+    // ---- TMA producer (whole warp: lanes fetch page ids, lane 0 issues the copies) ----
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
     }
-    int qi = 0, ki = 0;
-    uint32_t qph = 0, kph = 0;
-    // the window's page ids, pages lane, lane+32, lane+64 (a window spans at most 257 pages
-    // for W <= 4096; larger spans are fetched per key tile below)
-    auto load_tile = [&](int t, SeqInfo& s, int (&ids)[3]) {
-      s = seq_info(a, t / (TT * a.Hq));
-#pragma unroll
-      for (int j = 0; j < 3; ++j) {
-        const int p = lane + 32 * j;
-        ids[j] = (s.ok && p < s.np) ? page_block(a, s.b, s.p_first + p) : 0;
+    int ki = 0, qi = 0;
+    uint32_t kph = 0, qph = 0;
+    RowTileCursor cur;
+    int g, c, hl;
+    for (int t = blockIdx.x; cur.seek(a, t, g, c, hl); t += gridDim.x) {
+      if (__shfl_sync(0xffffffffu, *abort_flag != 0 ? 1 : 0, 0)) break;
+      const SeqInfo& s = cur.s;
+      const int r = cur.r;
+      const int h = g * a.G + hl;
+      const int pages = min(16, s.np - c * 16);
+      const int my_blk = lane < pages ? page_block(a, s.b, s.p_first + c * 16 + lane) : 0;
+      int ok = 1;
+      if (lane == 0) {
+        ok = mbar_wait(&k_empty[ki], kph ^ 1, abort_flag, a.status) ? 1 : 0;
+        if (ok) mbar_expect_tx(&k_full[ki], pages * NCH * kPageBytes);
       }
-    };
-    SeqInfo s_cur, s_nxt;
-    int ids_cur[3] = {0, 0, 0}, ids_nxt[3] = {0, 0, 0};
-    if (static_cast<int>(blockIdx.x) < num_tiles) load_tile(blockIdx.x, s_cur, ids_cur);
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      if (t + static_cast<int>(gridDim.x) < num_tiles) load_tile(t + gridDim.x, s_nxt, ids_nxt);
-      const int tt = t % TT;
-      const int h = (t / TT) % a.Hq;
-      const int r = t / (TT * a.Hq);
-      const SeqInfo s = s_cur;
-      bool stop = __shfl_sync(0xffffffffu, *abort_flag != 0 ? 1 : 0, 0) != 0;   // warp-uniform
-      if (s.ok && !stop) {
-        const int g = h / a.G;
-        int ok = 1;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      for (int p = 0; p < pages; ++p) {
+        const int blk = __shfl_sync(0xffffffffu, my_blk, p);
         if (lane == 0) {
-          ok = mbar_wait(&q_empty[qi], qph ^ 1, abort_flag, a.status) ? 1 : 0;
-          if (ok) {
-            mbar_expect_tx(&q_full[qi], kQBytes);
-            for (int c = 0; c < NCH; ++c)
-              tma_load_4d(q_buf + qi * kQBytes + c * kQRows1 * kRowBytes, &tm_q, &q_full[qi],
-                          c * 64, h, tt * kQRows1, r);
-          }
-        }
-        stop = __shfl_sync(0xffffffffu, ok, 0) == 0;
-        if (++qi == 2) { qi = 0; qph ^= 1; }
-        const int nkt = (s.np + 15) / 16;
-        for (int kt = 0; kt < nkt && !stop; ++kt) {
-          const int pages = min(16, s.np - kt * 16);
-          // page ids of this key tile (from the prefetched window list when it holds them)
-          int my_blk = 0;
-          {
-            const int p = kt * 16 + (lane & 15);
-            const int src = p & 31, j = p >> 5;
-            const int v0 = __shfl_sync(0xffffffffu, ids_cur[0], src);
-            const int v1 = __shfl_sync(0xffffffffu, ids_cur[1], src);
-            const int v2 = __shfl_sync(0xffffffffu, ids_cur[2], src);
-            my_blk = j == 0 ? v0 : (j == 1 ? v1 : v2);
-            if (p >= 96 && (lane & 15) < pages) my_blk = page_block(a, s.b, s.p_first + p);
-          }
-          if (lane == 0) {
-            ok = mbar_wait(&k_empty[ki], kph ^ 1, abort_flag, a.status) ? 1 : 0;
-            if (ok) mbar_expect_tx(&k_full[ki], pages * NCH * kPageBytes);
-          }
-          stop = __shfl_sync(0xffffffffu, ok, 0) == 0;
-          if (stop) break;
-          for (int pg = 0; pg < pages; ++pg) {
-            const int blk = __shfl_sync(0xffffffffu, my_blk, pg);
-            if (lane == 0) {
-              for (int c = 0; c < NCH; ++c)
-                tma_load_4d(k_buf + ki * kKBytes + c * kKRows1 * kRowBytes + pg * kPageBytes,
-                            &tm_k, &k_full[ki], c * 64, g, 0, blk);
-            }
-          }
-          if (++ki == kKStages1) { ki = 0; kph ^= 1; }
+          for (int ch = 0; ch < NCH; ++ch)
+            tma_load_4d(k_buf + ki * kKBytes + ch * kKRows1 * kRowBytes + p * kPageBytes, &tm_k,
+                        &k_full[ki], ch * 64, g, 0, blk);
         }
       }
-      s_cur = s_nxt;
-#pragma unroll
-      for (int j = 0; j < 3; ++j) ids_cur[j] = ids_nxt[j];
-      if (stop) break;
+      if (++ki == 2) { ki = 0; kph ^= 1; }
+      bool stop = false;
+      if (lane == 0) {
+        for (int qt = 0; qt < TT; ++qt) {
+          if (!mbar_wait(&q_empty[qi], qph ^ 1, abort_flag, a.status)) { stop = true; break; }
+          mbar_expect_tx(&q_full[qi], kQBytes);
+          for (int ch = 0; ch < NCH; ++ch)
+            tma_load_4d(q_buf + qi * kQBytes + ch * kQRows1 * kRowBytes, &tm_q, &q_full[qi],
+                        ch * 64, h, qt * kQRows1, r);
+          if (++qi == kQStages1) { qi = 0; qph ^= 1; }
+        }
+      }
+      qi = __shfl_sync(0xffffffffu, qi, 0);
+      qph = __shfl_sync(0xffffffffu, qph, 0);
+      if (__shfl_sync(0xffffffffu, stop ? 1 : 0, 0)) break;
     }
   } else if (warp == 1) {
     // ---------------- UMMA issuer ----------------
     if (lane == 0) {
-      int qi = 0, ki = 0, ab = 0;
-      uint32_t qph = 0, kph = 0, aph = 0;
-      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-        const int r = t / (TT * a.Hq);
-        const SeqInfo s = seq_info(a, r);
-        if (!s.ok) continue;
-        if (!mbar_wait(&q_full[qi], qph, abort_flag, a.status)) break;
-        const uint32_t q_addr = smem_u32(q_buf + qi * kQBytes);
-        const int nkt = (s.np + 15) / 16;
+      int ki = 0, qi = 0, ab = 0;
+      uint32_t kph = 0, qph = 0, aph = 0;
+      RowTileCursor cur;
+      int g, c, hl;
+      for (int t = blockIdx.x; !*abort_flag && cur.seek(a, t, g, c, hl); t += gridDim.x) {
+        const SeqInfo& s = cur.s;
+        const int pages = min(16, s.np - c * 16);
+        if (!mbar_wait(&k_full[ki], kph, abort_flag, a.status)) break;
+        const uint32_t k_addr = smem_u32(k_buf + ki * kKBytes);
+        const uint32_t idesc = idesc_bf16_f32(128, pages * 16);
         bool stop = false;
-        for (int kt = 0; kt < nkt; ++kt) {
-          const int pages = min(16, s.np - kt * 16);
-          if (!mbar_wait(&k_full[ki], kph, abort_flag, a.status)) { stop = true; break; }
+        for (int qt = 0; qt < TT; ++qt) {
+          if (!mbar_wait(&q_full[qi], qph, abort_flag, a.status)) { stop = true; break; }
           if (!mbar_wait(&acc_empty[ab], aph ^ 1, abort_flag, a.status)) { stop = true; break; }
           tc_fence_after();
-          const uint32_t k_addr = smem_u32(k_buf + ki * kKBytes);
-          const uint32_t idesc = idesc_bf16_f32(128, pages * 16);
+          const uint32_t q_addr = smem_u32(q_buf + qi * kQBytes);
           const uint32_t d_tmem = tmem_base + ab * 256;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -291,49 +297,47 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
             const uint64_t bd = sw128_kmajor_desc(k_addr + (kk >> 2) * kKRows1 * kRowBytes + off);
             umma_bf16(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
           }
-          umma_commit(&k_empty[ki]);
+          umma_commit(&q_empty[qi]);
           umma_commit(&acc_full[ab]);
-          if (++ki == kKStages1) { ki = 0; kph ^= 1; }
+          if (++qi == kQStages1) { qi = 0; qph ^= 1; }
           if (++ab == 2) { ab = 0; aph ^= 1; }
         }
         if (stop) break;
-        umma_commit(&q_empty[qi]);
-        if (++qi == 2) { qi = 0; qph ^= 1; }
+        umma_commit(&k_empty[ki]);
+        if (++ki == 2) { ki = 0; kph ^= 1; }
       }
     }
   } else {
-    // ---------- epilogue: one query row per TMEM lane, four warps per lane quadrant ----------
+    // ------- epilogue: one query row per TMEM lane, kParts warps per lane quadrant -------
     const int e = warp - 2;
     const int quad = warp & 3;
-    const int part = e >> 2;              // which 64 columns of each 256-column tile
+    const int part = e >> 2;              // which kPartCols columns of each tile
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     const float2 cs2 = make_float2(a.cs, a.cs);
     int ab = 0;
     uint32_t aph = 0;
-    SeqInfo s_nxt;
-    if (static_cast<int>(blockIdx.x) < num_tiles) s_nxt = seq_info(a, blockIdx.x / (TT * a.Hq));
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      const int tt = t % TT;
-      const int h = (t / TT) % a.Hq;
-      const int r = t / (TT * a.Hq);
-      const SeqInfo s = s_nxt;
-      if (t + static_cast<int>(gridDim.x) < num_tiles)
-        s_nxt = seq_info(a, (t + gridDim.x) / (TT * a.Hq));
-      float m = -INFINITY, l = 0.f;
-      bool stop = !s.ok;
-      if (s.ok) {
-        const int nkt = (s.np + 15) / 16;
-        for (int kt = 0; kt < nkt; ++kt) {
-          const int ncols = min(16, s.np - kt * 16) * 16;
-          if (!mbar_wait(&acc_full[ab], aph, abort_flag, a.status)) { stop = true; break; }
+    bool aborted = false;
+    RowTileCursor cur;
+    int g, c, hl;
+    for (int t = blockIdx.x; cur.seek(a, t, g, c, hl); t += gridDim.x) {
+      const SeqInfo& s = cur.s;
+      const int r = cur.r;
+      const int h = g * a.G + hl;
+      const int nc = cur.nc;
+      const int ncols = min(16, s.np - c * 16) * 16;
+      const int c0 = part * kPartCols;
+      const int cnt = max(0, min(kPartCols, ncols - c0));     // a multiple of 16
+      const int nch = (cnt + 31) / 32;
+      const int slot0 = (s.p_first + c * 16) * 16 + c0;
+      const bool edge = (c == 0) || (c == nc - 1);
+      float* lrow = a.lse + ((static_cast<size_t>(r) * a.Hq + h) * a.CM + c) * a.Wp;
+      for (int qt = 0; qt < TT; ++qt) {
+        float m = -INFINITY, l = 0.f;
+        if (!aborted && !mbar_wait(&acc_full[ab], aph, abort_flag, a.status)) aborted = true;
+        if (!aborted) {
           tc_fence_after();
-          const int c0 = part * kPartCols;
-          const int cnt = max(0, min(kPartCols, ncols - c0));     // a multiple of 16
-          const int slot0 = (s.p_first + kt * 16) * 16 + c0;
-          const bool edge = (kt == 0) || (kt == nkt - 1);
           const uint32_t col0 = lane_base + ab * 256 + c0;
-          const int nch = (cnt + 31) / 32;
           // one 32-column chunk: masked max, rescale, exponentials
           auto process = [&](float (&v)[32], int j) {
             if (cnt - 32 * j == 16) {
@@ -357,6 +361,7 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
             const float cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             if (cmax == -INFINITY) return;
             const float m_new = fmaxf(m, cmax * a.cs);
+#if KARA_SCORE_PACKED
             const float2 nm2 = make_float2(-m_new, -m_new);
             float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -368,6 +373,15 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             const float2 acc = fadd2(acc0, acc1);
             l = l * ex2(m - m_new) + (acc.x + acc.y);
+#else
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float x = fmaf(v[i], a.cs, -m_new);
+              acc[i & 3] += ((i & 7) == 7) ? ex2_fma(x) : ex2(x);
+            }
+            l = l * ex2(m - m_new) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+#endif
             m = m_new;
           };
           auto issue = [&](float (&v)[32], int j) {
@@ -402,40 +416,26 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
           if (++ab == 2) { ab = 0; aph ^= 1; }
         }
-      } else if (tt == 0 && h == 0 && row == 0 && part == 0) {
-        report(a.status, KARA_ERR_INVALID_ARG);
-      }
-      // merge the four column parts of the row
-      if (part > 0) comb[(part - 1) * kQRows1 + row] = make_float2(stop ? NAN : m, l);
-      named_barrier(kEpiBarrier, kEpiThreads);
-      if (part == 0) {
-        float lse2 = INFINITY;
-        float mm = m;
-        bool bad = stop;
-        float2 o[kParts - 1];
+        // merge the column parts of the row; part 0 writes the chunk's partial lse
+        if (part > 0) comb[(part - 1) * kQRows1 + row] = make_float2(m, l);
+        named_barrier(kEpiBarrier, kEpiThreads);
+        if (part == 0) {
+          float mm = m;
+          float2 o[kParts - 1];
 #pragma unroll
-        for (int q = 0; q < kParts - 1; ++q) {
-          o[q] = comb[q * kQRows1 + row];
-          bad = bad || isnan(o[q].x);
-          mm = fmaxf(mm, o[q].x);
-        }
-        if (!bad) {
-          float ll = l * ex2(m - mm);
+          for (int q = 0; q < kParts - 1; ++q) {
+            o[q] = comb[q * kQRows1 + row];
+            mm = fmaxf(mm, o[q].x);
+          }
+          float ll = (m == -INFINITY) ? 0.f : l * ex2(m - mm);
 #pragma unroll
           for (int q = 0; q < kParts - 1; ++q)
             if (o[q].x != -INFINITY) ll += o[q].y * ex2(o[q].x - mm);
-          lse2 = mm + __log2f(ll);
+          const int token = qt * kQRows1 + row;
+          if (token < a.Wp) lrow[token] = (aborted || ll == 0.f) ? -INFINITY : mm + __log2f(ll);
         }
-        const int token = tt * kQRows1 + row;
-        float* lrow = a.lse + (static_cast<size_t>(r) * a.Hq + h) * a.Wp;
-        if (token < a.W) lrow[token] = lse2;
-        else if (token < a.Wp) lrow[token] = INFINITY;
-        if (tt == TT - 1) {
-          const int extra = TT * kQRows1 + row;
-          if (extra < a.Wp) lrow[extra] = INFINITY;
-        }
+        named_barrier(kEpiBarrier, kEpiThreads);
       }
-      named_barrier(kEpiBarrier, kEpiThreads);
     }
   }
 
@@ -444,6 +444,33 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------------------------------
+// Merge of the per-chunk partial log-sum-exps: lse = log2(sum_c 2^lse_c), one thread per query.
+// ----------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) score_lse_merge_kernel(const ScoreArgs a) {
+  const size_t total = static_cast<size_t>(a.R) * a.Hq * a.Wp;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int token = static_cast<int>(i % a.Wp);
+    const size_t rh = i / a.Wp;
+    const int r = static_cast<int>(rh / a.Hq);
+    float out = INFINITY;
+    if (token < a.W) {
+      const SeqInfo s = seq_info(a, r);
+      if (s.ok) {
+        const int nc = (s.np + 15) / 16;
+        const float* p = a.lse + rh * a.CM * a.Wp + token;
+        float mx = -INFINITY;
+        for (int c = 0; c < nc; ++c) mx = fmaxf(mx, p[static_cast<size_t>(c) * a.Wp]);
+        float sum = 0.f;
+        for (int c = 0; c < nc; ++c) sum += ex2(p[static_cast<size_t>(c) * a.Wp] - mx);
+        out = mx + __log2f(sum);
+      }
+    }
+    a.lse_merged[i] = out;
   }
 }
 
@@ -609,18 +636,21 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (!s.ok) {
         const int j = kt * kKRows2 + row;
         if (part == 0 && j < a.W) out[j] = 0.f;
+        if (kt == 0 && g == 0 && etid == 0) report(a.status, KARA_ERR_INVALID_ARG);
         continue;
       }
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-      const float* lse_rows = a.lse + (static_cast<size_t>(r) * a.Hq + g * a.G) * a.Wp;
+      // merged lse of the tile's 256 queries, staged negated; the next tile's is prefetched
+      const float* lse_rows = a.lse_merged + (static_cast<size_t>(r) * a.Hq + g * a.G) * a.Wp;
       float lv = etid < kQRows2 ? lse_rows[etid] : 0.f;
       for (int q = 0; q < NQ; ++q) {
-        // stage this tile's 256 lse values (negated); prefetch the next tile's
         float* ls = lse_s + qbuf * kQRows2;
-        if (etid < kQRows2) ls[etid] = -lv;
-        if (q + 1 < NQ && etid < kQRows2) {
-          const int h1 = (q + 1) / QT, qt1 = (q + 1) % QT;
-          lv = lse_rows[static_cast<size_t>(h1) * a.Wp + qt1 * kQRows2 + etid];
+        if (etid < kQRows2) {
+          ls[etid] = -lv;
+          if (q + 1 < NQ) {
+            const int h1 = (q + 1) / QT, qt1 = (q + 1) % QT;
+            lv = lse_rows[static_cast<size_t>(h1) * a.Wp + qt1 * kQRows2 + etid];
+          }
         }
         named_barrier(kEpiBarrier, kEpiThreads);
         if (!aborted && !mbar_wait(&acc_full[ab], cph, abort_flag, a.status)) aborted = true;
@@ -634,6 +664,7 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
             tmem_ld16(col0 + 32 * j + 16, v + 16);
           };
           auto process = [&](const float (&v)[32], int j) {
+#if KARA_SCORE_PACKED
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
               const float4 nl = *reinterpret_cast<const float4*>(lh + 32 * j + i);
@@ -642,6 +673,18 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
               acc0 = fadd2(acc0, exp2_pair(x0, (i >> 1) & 3));
               acc1 = fadd2(acc1, exp2_pair(x1, ((i >> 1) + 1) & 3));
             }
+#else
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 nl = *reinterpret_cast<const float4*>(lh + 32 * j + i);
+              const float x0 = fmaf(v[i], a.cs, nl.x), x1 = fmaf(v[i + 1], a.cs, nl.y);
+              const float x2 = fmaf(v[i + 2], a.cs, nl.z), x3 = fmaf(v[i + 3], a.cs, nl.w);
+              acc0.x += ex2(x0);
+              acc0.y += ex2(x1);
+              acc1.x += ex2(x2);
+              acc1.y += ((i & 4) != 0) ? ex2_fma(x3) : ex2(x3);
+            }
+#endif
           };
           float va[32], vb[32];
           issue(va, 0);
@@ -697,7 +740,7 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 template <int D>
 constexpr size_t rowstats_smem() {
-  return 1024 + 2 * (D / 64) * kQRows1 * kRowBytes + kKStages1 * (D / 64) * kKRows1 * kRowBytes +
+  return 1024 + 2 * (D / 64) * kKRows1 * kRowBytes + kQStages1 * (D / 64) * kQRows1 * kRowBytes +
          3 * kQRows1 * sizeof(float2) + 256;
 }
 template <int D>
@@ -781,11 +824,13 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   a.ctx_len = L.ctx_len;
   a.seq_ids = L.seq_ids;
   a.lse = L.lse;
+  a.lse_merged = L.lse + static_cast<size_t>(L.R) * L.Hq * score_chunks(L.W) * score_lse_stride(L.W);
   a.scores = L.scores;
   a.status = L.status;
   a.R = L.R;
   a.W = L.W;
   a.Wp = score_lse_stride(L.W);
+  a.CM = score_chunks(L.W);
   a.Hq = L.Hq;
   a.Hkv = L.Hkv;
   a.G = L.Hq / L.Hkv;
@@ -802,8 +847,7 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
                          static_cast<int>(colsum_smem<D>()));
     attr_set = true;
   }
-  const int TT = (L.W + kQRows1 - 1) / kQRows1;
-  const int tiles1 = L.R * L.Hq * TT;
+  const int tiles1 = L.R * L.Hkv * score_chunks(L.W) * (L.Hq / L.Hkv);   // upper bound
   const int KT = ((L.W + 15 + 15) / 16 + 7) / 8;   // at most this many key tiles per (r, g)
   const int tiles2 = L.R * L.Hkv * KT;
   const int sms = sm_count();
@@ -812,6 +856,12 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
     describe_kernel("score_rowstats_kernel", reinterpret_cast<const void*>(score_rowstats_kernel<D>),
                     kThreads, rowstats_smem<D>());
     return KARA_ERR_CUDA;
+  }
+  {
+    const size_t n = static_cast<size_t>(L.R) * L.Hq * score_lse_stride(L.W);
+    const int blocks = static_cast<int>(std::min<size_t>((n + 255) / 256, static_cast<size_t>(sms) * 8));
+    score_lse_merge_kernel<<<blocks, 256, 0, stream>>>(a);
+    if (check_launch("score_lse_merge_kernel") != KARA_OK) return KARA_ERR_CUDA;
   }
   score_colsum_kernel<D><<<min(tiles2, sms), kThreads, colsum_smem<D>(), stream>>>(tq2, tk, a);
   if (check_launch("score_colsum_kernel") != KARA_OK) {
@@ -830,6 +880,13 @@ bool make_bf16_map_4d(CUtensorMap* map, const void* base, const uint64_t dims[4]
 }
 
 int score_lse_stride(int W) { return (W + 255) / 256 * 256; }
+
+// 16-page key chunks a window of W slots can span (its pages: at most ceil((W + 15) / 16)).
+int score_chunks(int W) { return ((W + 15 + 15) / 16 + 15) / 16; }
+
+size_t score_workspace_bytes(int R, int W, int Hq) {
+  return static_cast<size_t>(R) * Hq * (score_chunks(W) + 1) * score_lse_stride(W) * sizeof(float);
+}
 
 kara_status launch_score_kernels(const ScoreLaunch& L, cudaStream_t stream) {
   if (L.D == 128) return launch_score<128>(L, stream);

@@ -59,7 +59,8 @@ def test_host_side_validation_returns_before_any_launch(lib_path):
 def test_workspace_sizes(lib_path):
     pool = K._Pool(1, 1, 1, 1, 32, 257, 9000, 16, 4, 128)
     score = K.lib().kara_workspace_bytes(K.OP_SCORE, None, 32, 1000, 28, 0)
-    assert score == 32 * 28 * 1024 * 4                # rows padded to 256 queries
+    assert score == 32 * 28 * 5 * 1024 * 4            # 4 key chunks + merged, rows padded to 256
+    assert K.lib().kara_workspace_bytes(K.OP_SCORE, None, 1, 1024, 1, 0) == 6 * 1024 * 4
     dec = K.lib().kara_workspace_bytes(K.OP_DECODE, ctypes.byref(pool), 0, 0, 28, 0)
     assert dec == 32 * 28 * 17 * 130 * 4              # 17 splits of 16 pages, d + 2 floats
     comp = K.lib().kara_workspace_bytes(K.OP_COMPACT, None, 32, 1024, 0, 204)
