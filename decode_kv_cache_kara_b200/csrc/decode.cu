@@ -6,14 +6,18 @@
 // adapted to PagedAttention).
 //
 // HBM-bound: every K and V row of a KV head is loaded once for all G query heads of its group.
-// Grid = (split, KV head, sequence); a split covers 16 pages; each of the 4 warps walks its
-// pages with its own online softmax (base 2, scale folded into q), and the warps merge in
-// shared memory into one split partial (m, l, unnormalised o). A second kernel merges the
-// splits of each (sequence, query head). Pages reach shared memory by TMA (one 16-row box of
-// one KV head per 64 channels, 128-byte swizzle) through a 3-stage ring per warp, so that
-// each SM keeps many pages in flight. Per page a warp assigns two lanes to each of the 16
-// slots (half of d each) for q.k, then one lane per 4 channels of d for p.v; the swizzle
-// keeps both read patterns free of bank conflicts.
+// Persistent kernel (CTAs of 4 warps, as many per SM as registers and shared memory allow);
+// every warp is an independent stream over work units (sequence, KV head, 8-page split) and
+// leaves one partial (m, l, unnormalised o) per unit and query head; a second kernel merges the
+// partials of each (sequence, query head). Pages reach shared memory by TMA (one 16-row box of
+// one KV head per 64 channels, 128-byte swizzle) through a per-warp ring of single pages that
+// carries a unit's K pages, then its V pages, and keeps streaming across unit boundaries.
+//
+// The per-page products run on warp-level mma.sync (m16n8k16, bf16 in, fp32 accumulate) with
+// the group's query heads as the 8-wide N side: with G = 7 heads a page costs 1792 FMAs per 256
+// bytes of K and V, close to the point where CUDA-core issue rather than HBM binds, so the
+// tensor cores here cut the instruction stream (about 40 per page instead of about 1400) rather
+// than add arithmetic throughput.
 #include <cuda.h>
 
 #include <cstdint>
@@ -27,7 +31,7 @@ namespace {
 
 constexpr int kDecThreads = 128;
 constexpr int kDecWarps = 4;
-constexpr int kPagesPerSplit = 16;
+constexpr int kUnitPages = 8;      // pages per work unit (one partial per unit)
 
 struct DecodeArgs {
   const __nv_bfloat16* q;
@@ -43,12 +47,13 @@ struct DecodeArgs {
 
 template <int D>
 __host__ __device__ constexpr int page_bytes() { return 16 * D * 2; }   // one page, one KV head
-constexpr int kStages = 3;                                  // TMA page ring depth per warp
+constexpr int kStages = 4;          // TMA ring depth per warp, in single pages (K or V)
+constexpr int kDecMinBlocks = 3;    // resident CTAs per SM the register budget is sized for
 
 template <int D, int G>
-constexpr size_t split_smem_bytes() {
-  // [warp][stage]{K page, V page} (1024-aligned); the warp merge reuses this space
-  return 1024 + static_cast<size_t>(kDecWarps) * kStages * 2 * page_bytes<D>() + 64 * kDecWarps;
+constexpr size_t stream_smem_bytes() {
+  // [warp][stage] one page (1024-aligned) + the warps' ring barriers
+  return 1024 + static_cast<size_t>(kDecWarps) * kStages * page_bytes<D>() + 8 * kStages * kDecWarps;
 }
 
 // Byte offset of 16-byte granule `gi` of row `r` in a 128-byte-swizzled 16-row box.
@@ -56,210 +61,331 @@ __device__ __forceinline__ uint32_t sw128(int r, int gi) {
   return static_cast<uint32_t>(r * 128 + ((gi ^ (r & 7)) << 4));
 }
 
+// Work units (b, g, split), (b, g)-major: split s covers pages [8s, 8s+8) of sequence b.
+struct Unit {
+  int b, g, split, n, p0, np;   // np: pages of the unit
+  bool ok;
+};
+
+struct UnitCursor {
+  int b = 0, base = 0, per = -1, n = 0, npages = 0;
+  __device__ __forceinline__ Unit seek(const DecodeArgs& a, int u) {
+    Unit x;
+    x.ok = false;
+    while (true) {
+      if (b >= a.B) return x;
+      if (per < 0) {
+        n = a.ctx_len[b];
+        if (n > a.max_blocks * 16) {
+          report(a.status, KARA_ERR_INVALID_ARG);
+          n = a.max_blocks * 16;
+        }
+        if (n < 0) n = 0;
+        npages = (n + 15) / 16;
+        per = a.Hkv * ((npages + kUnitPages - 1) / kUnitPages);
+      }
+      if (u < base + per) break;
+      base += per;
+      ++b;
+      per = -1;
+    }
+    const int ns = per / a.Hkv;
+    const int local = u - base;
+    x.b = b;
+    x.g = local / ns;
+    x.split = local % ns;
+    x.n = n;
+    x.p0 = x.split * kUnitPages;
+    x.np = min(kUnitPages, npages - x.p0);
+    x.ok = true;
+    return x;
+  }
+};
+
+// ldmatrix / movmatrix / mma.sync helpers (m16n8k16, bf16 inputs, fp32 accumulators).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Persistent, one independent stream per warp: the warp walks units u = warp_id, +num_warps,
+// ...; its TMA ring (kStages single pages) streams, per unit, the unit's K pages and then its
+// V pages, and keeps streaming across unit boundaries (the next unit's block ids and queries
+// are fetched ahead). Every unit leaves one partial (m, l, o) per query head for the combine
+// kernel.
+//
+// The G <= 8 query heads of the group are the N = 8 side of warp-level m16n8k16 products, so
+// no fragment row is padding: per K page, S^T (16 slots x 8 heads) = K (16 x d) Q^T over d/16
+// steps, with K fragments read from the swizzled page by ldmatrix and Q^T held in registers
+// for the whole unit. The unit's scores stay in registers (4 per thread per page); one max per
+// head over the unit fixes the exponent base, so the accumulators are never rescaled. P^T goes
+// to bf16 and, transposed in registers by movmatrix, becomes the B operand of O^T (d x 8) +=
+// V^T (d x 16) P^T (16 x 8), with V^T fragments read by ldmatrix.trans.
 template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads, 2)
-decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                    const DecodeArgs a) {
+__global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
+decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
+  static_assert(G <= 8, "at most 8 query heads per KV head");
   constexpr int NCH = D / 64;                 // 64-channel chunks per row
-  constexpr int kHalf = D / 2;                // channels per lane in q.k
-  constexpr int kE4 = kHalf / 4;              // float4 groups per half
-  constexpr int kCh = D / 32;                 // channels per lane in p.v (4 or 2)
+  constexpr int KS = D / 16;                  // k-steps of S^T, m-tiles of O^T
   constexpr uint32_t kPage = page_bytes<D>();
   constexpr uint32_t kChunkBytes = 16 * 128;  // one 64-channel chunk of a page
-  const int split = blockIdx.x;
-  const int g = blockIdx.y;
-  const int b = blockIdx.z;
   const int warp = warp_id(), lane = lane_id();
-
-  int n = a.ctx_len[b];
-  if (n > a.max_blocks * 16) {
-    if (threadIdx.x == 0 && split == 0 && g == 0) report(a.status, KARA_ERR_INVALID_ARG);
-    n = a.max_blocks * 16;
-  }
-  const int pages = (n + 15) / 16;
-  const int p_begin = split * kPagesPerSplit;
-  if (p_begin >= pages) return;
-  const int p_end = min(pages, p_begin + kPagesPerSplit);
+  const int grp = lane >> 2, tig = lane & 3;  // fragment row / column pair
+  const int mtx = lane >> 3, mrow = lane & 7; // ldmatrix: lane feeds row mrow of matrix mtx
 
   extern __shared__ __align__(1024) uint8_t dsm[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* my_ring = ring + static_cast<size_t>(warp) * kStages * 2 * kPage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kDecWarps * kStages * 2 * kPage);
-  uint64_t* my_bars = bars + warp * kStages;
-  __shared__ __align__(16) float q_s[G][kE4][2][4];          // pre-scaled q, half-interleaved
-  __shared__ __align__(16) float p_s[kDecWarps][16][8];       // page probabilities
-  __shared__ float red_m[kDecWarps][G], red_l[kDecWarps][G];
-  float* red_o = reinterpret_cast<float*>(ring);              // [warp][G][D], after the loop
+  uint8_t* my_ring = ring + static_cast<size_t>(warp) * kStages * kPage;
+  uint64_t* my_bars = reinterpret_cast<uint64_t*>(ring + kDecWarps * kStages * kPage) +
+                      warp * kStages;
+  const uint32_t ring_u32 = smem_u32(my_ring);
 
   if (lane == 0) {
     for (int st = 0; st < kStages; ++st) mbar_init(&my_bars[st], 1);
     fence_barrier_init();
   }
-  for (int i = threadIdx.x; i < G * D; i += kDecThreads) {
-    const int h = i / D, c = i % D;
-    const float qv = __bfloat162float(a.q[(static_cast<size_t>(b) * a.Hq + g * G + h) * D + c]);
-    const int half = c / kHalf, e = c % kHalf;
-    q_s[h][e / 4][half][e % 4] = qv * a.cs;
-  }
   __syncthreads();
 
-  // this warp's pages: p_begin + warp + 4k; lane k holds the block id of its k-th page
-  const int32_t* tab = a.block_table + static_cast<size_t>(b) * a.max_blocks;
-  const int my_pages = (p_end - p_begin - warp + kDecWarps - 1) / kDecWarps;
-  int my_blk = 0;
-  if (lane < my_pages) {
-    my_blk = tab[p_begin + warp + kDecWarps * lane];
-    if (my_blk < 0 || my_blk >= a.num_blocks) {
+  const int num_warps = gridDim.x * kDecWarps;
+  UnitCursor cursor;
+  int u = blockIdx.x * kDecWarps + warp;
+  Unit cu = cursor.seek(a, u);
+  if (!cu.ok) return;
+  Unit nu = cursor.seek(a, u + num_warps);
+
+  auto load_ids = [&](const Unit& x) -> int {
+    if (!x.ok || lane >= x.np) return -1;
+    int blk = a.block_table[static_cast<size_t>(x.b) * a.max_blocks + x.p0 + lane];
+    if (blk < 0 || blk >= a.num_blocks) {
       report(a.status, KARA_ERR_BAD_BLOCK);
-      my_blk = -1;
+      blk = -1;
     }
-  }
-  auto issue = [&](int k) {          // lane 0: page k of this warp into stage k % kStages
-    const int blk = __shfl_sync(0xffffffffu, my_blk, k);
-    if (lane == 0 && blk >= 0) {
-      uint8_t* st = my_ring + (k % kStages) * 2 * kPage;
-      uint64_t* bar = &my_bars[k % kStages];
-      mbar_expect_tx(bar, 2 * kPage);
-      for (int c = 0; c < NCH; ++c) {
-        tma_load_4d(st + c * kChunkBytes, &tm_k, bar, c * 64, g, 0, blk);
-        tma_load_4d(st + kPage + c * kChunkBytes, &tm_v, bar, c * 64, g, 0, blk);
-      }
+    return blk;
+  };
+  // B fragments of Q^T (column grp = query head g*G + grp when grp < G, else 0): for k-step
+  // ks, qb[ks][0] = channels ks*16 + 2*tig + {0,1}, qb[ks][1] = channels ks*16 + 8 + 2*tig + {0,1}
+  auto load_q = [&](const Unit& x, uint32_t (&qb)[KS][2]) {
+    const bool row_ok = x.ok && grp < G;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+        a.q + (static_cast<size_t>(x.b) * a.Hq + x.g * G + (row_ok ? grp : 0)) * D);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      qb[ks][0] = row_ok ? qrow[ks * 8 + tig] : 0u;
+      qb[ks][1] = row_ok ? qrow[ks * 8 + 4 + tig] : 0u;
     }
   };
-  for (int k = 0; k < min(kStages, my_pages); ++k) issue(k);
 
-  float m[G], l[G];
-  float2 acc[G][kCh / 2];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
-#pragma unroll
-    for (int c = 0; c < kCh / 2; ++c) acc[h][c] = make_float2(0.f, 0.f);
-  }
-  const int slot = lane >> 1, half = lane & 1;
-  uint32_t phase_bits = 0;            // parity per stage
+  int ids_cu = load_ids(cu), ids_nu = load_ids(nu);
+  uint32_t qb[KS][2], qn[KS][2];
+  load_q(cu, qb);
+  load_q(nu, qn);
+
+  // Stream entries: unit x contributes 2*x.np entries, K pages then V pages.
+  int ustart = 0;          // stream index of cu's first entry
+  int issued = 0, done = 0;
+  uint32_t phase = 0;      // parity bit per stage
+  uint32_t pending = 0;    // stages with a load issued and not yet consumed
   volatile int no_abort = 0;
+  auto top_up = [&]() {
+    const int avail = ustart + 2 * cu.np + (nu.ok ? 2 * nu.np : 0);
+    while (issued < done + kStages && issued < avail) {
+      const int e = issued - ustart;
+      const bool in_cu = e < 2 * cu.np;
+      const int e2 = in_cu ? e : e - 2 * cu.np;
+      const int npx = in_cu ? cu.np : nu.np;
+      const bool is_v = e2 >= npx;
+      const int j = is_v ? e2 - npx : e2;
+      const int bc = __shfl_sync(0xffffffffu, ids_cu, j & 31);
+      const int bn = __shfl_sync(0xffffffffu, ids_nu, j & 31);
+      const int blk = in_cu ? bc : bn;
+      const int g = in_cu ? cu.g : nu.g;
+      const int st = issued % kStages;
+      if (blk >= 0) pending |= 1u << st;
+      if (lane == 0 && blk >= 0) {
+        uint8_t* dst = my_ring + st * kPage;
+        mbar_expect_tx(&my_bars[st], kPage);
+        const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
+        for (int c = 0; c < NCH; ++c) tma_load_4d(dst + c * kChunkBytes, tm, &my_bars[st], c * 64, g, 0, blk);
+      }
+      ++issued;
+    }
+  };
+  // Consumes stream entry t: returns the stage's shared address, or 0 when the page was
+  // skipped (bad block, reported) or the wait gave up (sets aborted).
+  bool aborted = false;
+  auto acquire = [&](int t, int blk) -> uint32_t {
+    top_up();
+    done = t + 1;
+    if (blk < 0) return 0u;
+    const int st = t % kStages;
+    if (!mbar_wait(&my_bars[st], (phase >> st) & 1, &no_abort, a.status)) {
+      aborted = true;
+      return 0u;
+    }
+    phase ^= 1u << st;
+    pending &= ~(1u << st);
+    return ring_u32 + st * kPage;
+  };
 
-  for (int k = 0; k < my_pages; ++k) {
-    const int p = p_begin + warp + kDecWarps * k;
-    const int blk = __shfl_sync(0xffffffffu, my_blk, k);
-    const int st = k % kStages;
-    if (blk >= 0) {                                 // a bad block id was reported; page skipped
-    const bool ok = mbar_wait(&my_bars[st], (phase_bits >> st) & 1, &no_abort, a.status);
-    phase_bits ^= 1u << st;
-    if (!ok) break;
-    const int valid = min(16, n - p * 16);
-    const uint8_t* kst = my_ring + st * 2 * kPage;
-    const uint8_t* vst = kst + kPage;
-    // q . k: this lane's slot, half of d (granules of chunk `half` for d = 128, the half of
-    // chunk 0's granules for d = 64)
-    float2 dot2[G];
+  while (cu.ok) {
+    // ---- K pages: S^T for every page of the unit ----
+    float sc[kUnitPages][4];
 #pragma unroll
-    for (int h = 0; h < G; ++h) dot2[h] = make_float2(0.f, 0.f);
+    for (int j = 0; j < kUnitPages; ++j) {
+      sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = -INFINITY;
+      if (j < cu.np && !aborted) {
+        const int blk = __shfl_sync(0xffffffffu, ids_cu, j);
+        const uint32_t kst = acquire(ustart + j, blk);
+        if (kst != 0u) {
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < kHalf / 8; ++i) {
-      const int chunk = NCH == 2 ? half : 0;
-      const int gi = NCH == 2 ? i : half * 4 + i;
-      const uint4 kr = *reinterpret_cast<const uint4*>(kst + chunk * kChunkBytes + sw128(slot, gi));
-      const float2 k01 = bf16x2_to_f2(kr.x), k23 = bf16x2_to_f2(kr.y);
-      const float2 k45 = bf16x2_to_f2(kr.z), k67 = bf16x2_to_f2(kr.w);
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float4 qa = *reinterpret_cast<const float4*>(&q_s[h][2 * i][half][0]);
-        const float4 qb = *reinterpret_cast<const float4*>(&q_s[h][2 * i + 1][half][0]);
-        float2 d = dot2[h];
-        d = ffma2(k01, make_float2(qa.x, qa.y), d);
-        d = ffma2(k23, make_float2(qa.z, qa.w), d);
-        d = ffma2(k45, make_float2(qb.x, qb.y), d);
-        d = ffma2(k67, make_float2(qb.z, qb.w), d);
-        dot2[h] = d;
+          for (int ks = 0; ks < KS; ++ks) {
+            // matrices: (slots 0-7, d lo), (slots 8-15, d lo), (slots 0-7, d hi), (slots 8-15, d hi)
+            const int slot = (mtx & 1) * 8 + mrow;
+            const int d0 = ks * 16 + (mtx >> 1) * 8;
+            uint32_t ka[4];
+            ldsm_x4(kst + (d0 >> 6) * kChunkBytes + sw128(slot, (d0 & 63) >> 3), ka);
+            mma_16816(acc, ka, qb[ks][0], qb[ks][1]);
+          }
+          // acc: (slot grp, heads 2tig, 2tig+1), (slot grp+8, heads 2tig, 2tig+1)
+          const int valid = min(16, cu.n - (cu.p0 + j) * 16);
+          const bool lo_ok = grp < valid, hi_ok = grp + 8 < valid;
+          sc[j][0] = lo_ok ? acc[0] * a.cs : -INFINITY;
+          sc[j][1] = lo_ok ? acc[1] * a.cs : -INFINITY;
+          sc[j][2] = hi_ok ? acc[2] * a.cs : -INFINITY;
+          sc[j][3] = hi_ok ? acc[3] * a.cs : -INFINITY;
+        }
+        __syncwarp();
       }
     }
+    if (aborted) break;
+    // ---- one exponent base per head over the unit (heads 2tig and 2tig+1) ----
+    float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float d = dot2[h].x + dot2[h].y;
-      d += __shfl_xor_sync(0xffffffffu, d, 1);
-      if (slot >= valid) d = -INFINITY;
-      float pm = d;
-#pragma unroll
-      for (int off = 2; off < 32; off <<= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, off));
-      const float m_new = fmaxf(m[h], pm);
-      const float corr = ex2(m[h] - m_new);
-      const float pr = ex2(d - m_new);
-      float ps = pr;
-#pragma unroll
-      for (int off = 2; off < 32; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-      l[h] = l[h] * corr + ps;
-      m[h] = m_new;
-#pragma unroll
-      for (int c = 0; c < kCh / 2; ++c) acc[h][c] = fmul2(acc[h][c], make_float2(corr, corr));
-      if (half == 0) p_s[warp][slot][h] = pr;
+    for (int j = 0; j < kUnitPages; ++j) {
+      m0 = fmaxf(m0, fmaxf(sc[j][0], sc[j][2]));
+      m1 = fmaxf(m1, fmaxf(sc[j][1], sc[j][3]));
     }
-    __syncwarp();
-    // p . v: channels [kCh*lane, kCh*lane + kCh) of every valid slot
-    const int c0 = kCh * lane;
-    const int vchunk = c0 / 64, vgi = (c0 % 64) / 8, vsub = ((c0 % 64) % 8) * 2;
-    for (int s = 0; s < valid; ++s) {
-      const uint8_t* vrow = vst + vchunk * kChunkBytes + sw128(s, vgi) + vsub;
-      float2 vf[kCh / 2];
-      if constexpr (kCh == 4) {
-        const uint2 t = *reinterpret_cast<const uint2*>(vrow);
-        vf[0] = bf16x2_to_f2(t.x);
-        vf[1] = bf16x2_to_f2(t.y);
-      } else {
-        vf[0] = bf16x2_to_f2(*reinterpret_cast<const uint32_t*>(vrow));
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, off));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, off));
+    }
+    const float b0 = m0 == -INFINITY ? 0.f : m0;   // a head with no valid slot: all P = 0
+    const float b1 = m1 == -INFINITY ? 0.f : m1;
+    float l0 = 0.f, l1 = 0.f;
+    uint32_t pb[kUnitPages][2];   // P^T B fragments per page: slots 2tig.. and 8+2tig.., head grp
+#pragma unroll
+    for (int j = 0; j < kUnitPages; ++j) {
+      const float p0 = ex2(sc[j][0] - b0), p1 = ex2(sc[j][1] - b1);
+      const float p2 = ex2(sc[j][2] - b0), p3 = ex2(sc[j][3] - b1);
+      l0 += p0 + p2;
+      l1 += p1 + p3;
+      pb[j][0] = movmatrix_trans(pack_bf16(p0, p1));
+      pb[j][1] = movmatrix_trans(pack_bf16(p2, p3));
+    }
+    // ---- V pages: O^T += V^T P^T ----
+    float o[KS][4];
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kUnitPages; ++j) {
+      if (j < cu.np && !aborted) {
+        const int blk = __shfl_sync(0xffffffffu, ids_cu, j);
+        const uint32_t vst = acquire(ustart + cu.np + j, blk);
+        if (vst != 0u) {
+          const int valid = min(16, cu.n - (cu.p0 + j) * 16);
+          // slots past the context may hold any bits (even NaN); P is 0 there, V is zeroed
+          const int s_lo = 2 * tig, s_hi = 8 + 2 * tig;
+          const uint32_t mlo = (s_lo < valid ? 0xffffu : 0u) | (s_lo + 1 < valid ? 0xffff0000u : 0u);
+          const uint32_t mhi = (s_hi < valid ? 0xffffu : 0u) | (s_hi + 1 < valid ? 0xffff0000u : 0u);
+          const bool partial_page = valid < 16;
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            // matrices: (slots 0-7, ch lo), (slots 0-7, ch hi), (slots 8-15, ch lo), (slots 8-15, ch hi)
+            const int slot = (mtx >> 1) * 8 + mrow;
+            const int c0 = mt * 16 + (mtx & 1) * 8;
+            uint32_t va[4];
+            ldsm_x4_trans(vst + (c0 >> 6) * kChunkBytes + sw128(slot, (c0 & 63) >> 3), va);
+            if (partial_page) {
+              va[0] &= mlo;
+              va[1] &= mlo;
+              va[2] &= mhi;
+              va[3] &= mhi;
+            }
+            mma_16816(o[mt], va, pb[j][0], pb[j][1]);
+          }
+        }
+        __syncwarp();
       }
-      const float4 p0 = *reinterpret_cast<const float4*>(&p_s[warp][s][0]);
-      const float4 p1 = *reinterpret_cast<const float4*>(&p_s[warp][s][4]);
-      const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    }
+    if (aborted) break;
+    // ---- the unit's partial: heads 2tig, 2tig+1 own o[mt][0/2] and o[mt][1/3] ----
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float2 pp = make_float2(pv[h], pv[h]);
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
 #pragma unroll
-        for (int c = 0; c < kCh / 2; ++c) acc[h][c] = ffma2(pp, vf[c], acc[h][c]);
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * tig + e;
+      if (h < G) {
+        float* dst = a.partial +
+                     ((static_cast<size_t>(cu.b) * a.Hq + cu.g * G + h) * a.S + cu.split) * (D + 2);
+        if (grp == 0) {
+          dst[0] = e == 0 ? m0 : m1;
+          dst[1] = e == 0 ? l0 : l1;
+        }
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          dst[2 + mt * 16 + grp] = o[mt][e];
+          dst[2 + mt * 16 + 8 + grp] = o[mt][2 + e];
+        }
       }
     }
-    __syncwarp();
+    // advance: the next unit becomes current, fetch the one after it
+    ustart += 2 * cu.np;
+    cu = nu;
+    ids_cu = ids_nu;
+    if (!cu.ok) break;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      qb[ks][0] = qn[ks][0];
+      qb[ks][1] = qn[ks][1];
     }
-    // stage st is free again: refill it with page k + kStages
-    if (k + kStages < my_pages) {
-      fence_proxy_async();
-      issue(k + kStages);
-    }
+    u += num_warps;
+    nu = cursor.seek(a, u + num_warps);
+    ids_nu = load_ids(nu);
+    load_q(nu, qn);
   }
-  __syncthreads();    // every warp is done with the ring: reuse it for the merge
-
-  // merge the four warps of the CTA
-  if (lane == 0) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) { red_m[warp][h] = m[h]; red_l[warp][h] = l[h]; }
-  }
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int c = 0; c < kCh / 2; ++c) {
-      red_o[(warp * G + h) * D + lane * kCh + 2 * c] = acc[h][c].x;
-      red_o[(warp * G + h) * D + lane * kCh + 2 * c + 1] = acc[h][c].y;
-    }
-  __syncthreads();
-  for (int i = threadIdx.x; i < G * (D + 2); i += kDecThreads) {
-    const int h = i / (D + 2), c = i % (D + 2);
-    float mx = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) mx = fmaxf(mx, red_m[w][h]);
-    float val = 0.f;
-    if (c == 0) {
-      val = mx;
-    } else {
-#pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) {
-        const float wt = (red_m[w][h] == -INFINITY) ? 0.f : ex2(red_m[w][h] - mx);
-        val += wt * (c == 1 ? red_l[w][h] : red_o[(w * G + h) * D + c - 2]);
-      }
-    }
-    a.partial[((static_cast<size_t>(b) * a.Hq + g * G + h) * a.S + split) * (D + 2) + c] = val;
+  if (aborted) {
+    // a wait gave up (reported): let this warp's loads still in flight land before exiting
+    volatile int give_up = 0;
+    for (int st = 0; st < kStages; ++st)
+      if ((pending >> st) & 1u) mbar_wait(&my_bars[st], (phase >> st) & 1, &give_up, a.status);
   }
 }
 
@@ -270,7 +396,7 @@ decode_combine_kernel(const DecodeArgs a, __nv_bfloat16* __restrict__ out) {
   const int b = bh / a.Hq;
   int n = a.ctx_len[b];
   n = min(n, a.max_blocks * 16);
-  const int splits = (((n + 15) / 16) + kPagesPerSplit - 1) / kPagesPerSplit;
+  const int splits = (((n + 15) / 16) + kUnitPages - 1) / kUnitPages;
   const float* part = a.partial + static_cast<size_t>(bh) * a.S * (D + 2);
   float mx = -INFINITY;
   for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part[s * (D + 2)]);
@@ -289,15 +415,19 @@ decode_combine_kernel(const DecodeArgs a, __nv_bfloat16* __restrict__ out) {
 template <int D, int G>
 kara_status launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, void* out,
                       cudaStream_t stream) {
-  dim3 grid(a.S, a.Hkv, a.B);
-  constexpr size_t smem = split_smem_bytes<D, G>();
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  constexpr size_t smem = stream_smem_bytes<D, G>();
+  static int per_sm = 0;   // resident CTAs per SM, queried once
+  if (per_sm == 0) {
+    cudaFuncSetAttribute(decode_stream_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
-    attr = true;
+    int n = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_stream_kernel<D, G>, kDecThreads, smem);
+    per_sm = n > 0 ? n : 1;
   }
-  decode_split_kernel<D, G><<<grid, kDecThreads, smem, stream>>>(tk, tv, a);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  decode_stream_kernel<D, G><<<per_sm * sms, kDecThreads, smem, stream>>>(tk, tv, a);
   decode_combine_kernel<D><<<a.B * a.Hq, D, 0, stream>>>(a, static_cast<__nv_bfloat16*>(out));
   return check_launch(__func__);
 }
@@ -320,7 +450,7 @@ kara_status launch_d(const DecodeArgs& a, int G, const CUtensorMap& tk, const CU
 
 }  // namespace
 
-int decode_num_splits(int max_blocks) { return (max_blocks + kPagesPerSplit - 1) / kPagesPerSplit; }
+int decode_num_splits(int max_blocks) { return (max_blocks + kUnitPages - 1) / kUnitPages; }
 
 size_t decode_workspace_bytes(int B, int Hq, int D, int max_blocks) {
   return static_cast<size_t>(B) * Hq * decode_num_splits(max_blocks) * (D + 2) * sizeof(float);

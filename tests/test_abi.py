@@ -62,7 +62,7 @@ def test_workspace_sizes(lib_path):
     assert score == 32 * 28 * 5 * 1024 * 4            # 4 key chunks + merged, rows padded to 256
     assert K.lib().kara_workspace_bytes(K.OP_SCORE, None, 1, 1024, 1, 0) == 6 * 1024 * 4
     dec = K.lib().kara_workspace_bytes(K.OP_DECODE, ctypes.byref(pool), 0, 0, 28, 0)
-    assert dec == 32 * 28 * 17 * 130 * 4              # 17 splits of 16 pages, d + 2 floats
+    assert dec == 32 * 28 * 33 * 130 * 4              # 33 units of 8 pages, d + 2 floats
     comp = K.lib().kara_workspace_bytes(K.OP_COMPACT, None, 32, 1024, 0, 204)
     assert comp == (16 + 32 * 12 + 32 * 14) * 4
 
