@@ -21,6 +21,7 @@
 #include <cuda.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -39,7 +40,8 @@ struct DecodeArgs {
   const __nv_bfloat16* v;
   const int32_t* block_table;
   const int32_t* ctx_len;
-  float* partial;      // [B, Hq, S, D + 2]: m, l, o[D]
+  float* part_o;       // [B, Hq, S, D]: unnormalised o per split (16-byte aligned rows)
+  float2* part_ml;     // [B, Hq, S]: (m, l) per split
   int32_t* status;
   int B, Hq, Hkv, max_blocks, num_blocks, S;
   float cs;            // scale * log2(e)
@@ -61,7 +63,9 @@ __device__ __forceinline__ uint32_t sw128(int r, int gi) {
   return static_cast<uint32_t>(r * 128 + ((gi ^ (r & 7)) << 4));
 }
 
-// Work units (b, g, split), (b, g)-major: split s covers pages [8s, 8s+8) of sequence b.
+// Work units (b, split, g), g fastest: split s covers pages [8s, 8s+8) of sequence b. Warps
+// with consecutive unit ids (the warps of one CTA) read the KV heads of the same blocks at about
+// the same time, so each block's DRAM rows are fetched together.
 struct Unit {
   int b, g, split, n, p0, np;   // np: pages of the unit
   bool ok;
@@ -89,11 +93,10 @@ struct UnitCursor {
       ++b;
       per = -1;
     }
-    const int ns = per / a.Hkv;
     const int local = u - base;
     x.b = b;
-    x.g = local / ns;
-    x.split = local % ns;
+    x.g = local % a.Hkv;
+    x.split = local / a.Hkv;
     x.n = n;
     x.p0 = x.split * kUnitPages;
     x.np = min(kUnitPages, npages - x.p0);
@@ -168,6 +171,8 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
     fence_barrier_init();
   }
   __syncthreads();
+  // the combine kernel may be scheduled now; it waits for this grid's results itself
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int num_warps = gridDim.x * kDecWarps;
   UnitCursor cursor;
@@ -218,9 +223,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
       const int npx = in_cu ? cu.np : nu.np;
       const bool is_v = e2 >= npx;
       const int j = is_v ? e2 - npx : e2;
-      const int bc = __shfl_sync(0xffffffffu, ids_cu, j & 31);
-      const int bn = __shfl_sync(0xffffffffu, ids_nu, j & 31);
-      const int blk = in_cu ? bc : bn;
+      const int blk = __shfl_sync(0xffffffffu, in_cu ? ids_cu : ids_nu, j & 31);
       const int g = in_cu ? cu.g : nu.g;
       const int st = issued % kStages;
       if (blk >= 0) pending |= 1u << st;
@@ -260,7 +263,8 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
         const int blk = __shfl_sync(0xffffffffu, ids_cu, j);
         const uint32_t kst = acquire(ustart + j, blk);
         if (kst != 0u) {
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          // two independent accumulator chains (even / odd k-steps), added at the end
+          float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
           for (int ks = 0; ks < KS; ++ks) {
             // matrices: (slots 0-7, d lo), (slots 8-15, d lo), (slots 0-7, d hi), (slots 8-15, d hi)
@@ -268,15 +272,17 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
             const int d0 = ks * 16 + (mtx >> 1) * 8;
             uint32_t ka[4];
             ldsm_x4(kst + (d0 >> 6) * kChunkBytes + sw128(slot, (d0 & 63) >> 3), ka);
-            mma_16816(acc, ka, qb[ks][0], qb[ks][1]);
+            mma_16816(acc[ks & 1], ka, qb[ks][0], qb[ks][1]);
           }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[0][e] += acc[1][e];
           // acc: (slot grp, heads 2tig, 2tig+1), (slot grp+8, heads 2tig, 2tig+1)
           const int valid = min(16, cu.n - (cu.p0 + j) * 16);
           const bool lo_ok = grp < valid, hi_ok = grp + 8 < valid;
-          sc[j][0] = lo_ok ? acc[0] * a.cs : -INFINITY;
-          sc[j][1] = lo_ok ? acc[1] * a.cs : -INFINITY;
-          sc[j][2] = hi_ok ? acc[2] * a.cs : -INFINITY;
-          sc[j][3] = hi_ok ? acc[3] * a.cs : -INFINITY;
+          sc[j][0] = lo_ok ? acc[0][0] * a.cs : -INFINITY;
+          sc[j][1] = lo_ok ? acc[0][1] * a.cs : -INFINITY;
+          sc[j][2] = hi_ok ? acc[0][2] * a.cs : -INFINITY;
+          sc[j][3] = hi_ok ? acc[0][3] * a.cs : -INFINITY;
         }
         __syncwarp();
       }
@@ -353,16 +359,13 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
     for (int e = 0; e < 2; ++e) {
       const int h = 2 * tig + e;
       if (h < G) {
-        float* dst = a.partial +
-                     ((static_cast<size_t>(cu.b) * a.Hq + cu.g * G + h) * a.S + cu.split) * (D + 2);
-        if (grp == 0) {
-          dst[0] = e == 0 ? m0 : m1;
-          dst[1] = e == 0 ? l0 : l1;
-        }
+        const size_t row = (static_cast<size_t>(cu.b) * a.Hq + cu.g * G + h) * a.S + cu.split;
+        float* dst = a.part_o + row * D;
+        if (grp == 0) a.part_ml[row] = make_float2(e == 0 ? m0 : m1, e == 0 ? l0 : l1);
 #pragma unroll
         for (int mt = 0; mt < KS; ++mt) {
-          dst[2 + mt * 16 + grp] = o[mt][e];
-          dst[2 + mt * 16 + 8 + grp] = o[mt][2 + e];
+          dst[mt * 16 + grp] = o[mt][e];
+          dst[mt * 16 + 8 + grp] = o[mt][2 + e];
         }
       }
     }
@@ -389,27 +392,81 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
 }
 
+// Merge of the split partials of each (sequence, query head): one CTA of kCombWarps warps per
+// pair; warp w takes the splits w, w + kCombWarps, ..., lane l owns D/32 consecutive channels,
+// and every lane keeps kCombBatch independent loads in flight before it accumulates them. The
+// warps' sums meet in shared memory. Launched as a programmatic dependent of the stream kernel:
+// its CTAs may start early and wait for the stream kernel's results.
+constexpr int kCombWarps = 4;
+constexpr int kCombBatch = 8;
+
 template <int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(32 * kCombWarps)
 decode_combine_kernel(const DecodeArgs a, __nv_bfloat16* __restrict__ out) {
+  constexpr int V = D / 32;   // channels per lane
+  using VecT = typename std::conditional<V == 4, float4, float2>::type;
+  __shared__ float red_o[kCombWarps][D];
+  __shared__ float red_l[kCombWarps];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x;
+  const int warp = warp_id(), lane = lane_id();
   const int b = bh / a.Hq;
   int n = a.ctx_len[b];
-  n = min(n, a.max_blocks * 16);
+  n = max(0, min(n, a.max_blocks * 16));
   const int splits = (((n + 15) / 16) + kUnitPages - 1) / kUnitPages;
-  const float* part = a.partial + static_cast<size_t>(bh) * a.S * (D + 2);
+  const float2* ml = a.part_ml + static_cast<size_t>(bh) * a.S;
+  const float* po = a.part_o + static_cast<size_t>(bh) * a.S * D + lane * V;
   float mx = -INFINITY;
-  for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part[s * (D + 2)]);
-  float lsum = 0.f, o = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float ms = part[s * (D + 2)];
-    if (ms == -INFINITY) continue;
-    const float w = ex2(ms - mx);
-    lsum += w * part[s * (D + 2) + 1];
-    o += w * part[s * (D + 2) + 2 + threadIdx.x];
+  for (int s0 = lane; s0 < splits; s0 += 32) mx = fmaxf(mx, ml[s0].x);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  float acc[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) acc[v] = 0.f;
+  float lsum = 0.f;
+  for (int s0 = warp; s0 < splits; s0 += kCombWarps * kCombBatch) {
+    VecT x[kCombBatch];
+    float2 mlv[kCombBatch];
+#pragma unroll
+    for (int i = 0; i < kCombBatch; ++i) {
+      const int sp = s0 + i * kCombWarps;
+      if (sp < splits) {
+        x[i] = *reinterpret_cast<const VecT*>(po + static_cast<size_t>(sp) * D);
+        mlv[i] = ml[sp];
+      } else {
+        mlv[i] = make_float2(-INFINITY, 0.f);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kCombBatch; ++i) {
+      if (mlv[i].x == -INFINITY) continue;
+      const float w = ex2(mlv[i].x - mx);
+      lsum += w * mlv[i].y;
+      const float* xv = reinterpret_cast<const float*>(&x[i]);
+#pragma unroll
+      for (int v = 0; v < V; ++v) acc[v] += w * xv[v];
+    }
   }
-  const float res = lsum > 0.f ? o / lsum : 0.f;
-  out[static_cast<size_t>(bh) * D + threadIdx.x] = __float2bfloat16_rn(res);
+#pragma unroll
+  for (int v = 0; v < V; ++v) red_o[warp][lane * V + v] = acc[v];
+  if (lane == 0) red_l[warp] = lsum;
+  __syncthreads();
+  if (warp == 0) {
+    float l = 0.f, r[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) r[v] = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombWarps; ++w) {
+      l += red_l[w];
+#pragma unroll
+      for (int v = 0; v < V; ++v) r[v] += red_o[w][lane * V + v];
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    __nv_bfloat16* dst = out + static_cast<size_t>(bh) * D + lane * V;
+#pragma unroll
+    for (int v = 0; v < V; v += 2)
+      *reinterpret_cast<__nv_bfloat162*>(dst + v) = __floats2bfloat162_rn(r[v] * inv, r[v + 1] * inv);
+  }
 }
 
 template <int D, int G>
@@ -428,7 +485,16 @@ kara_status launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensor
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   decode_stream_kernel<D, G><<<per_sm * sms, kDecThreads, smem, stream>>>(tk, tv, a);
-  decode_combine_kernel<D><<<a.B * a.Hq, D, 0, stream>>>(a, static_cast<__nv_bfloat16*>(out));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.B * a.Hq);
+  cfg.blockDim = dim3(32 * kCombWarps);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, a, static_cast<__nv_bfloat16*>(out));
   return check_launch(__func__);
 }
 
@@ -464,14 +530,16 @@ kara_status launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
   a.v = static_cast<const __nv_bfloat16*>(L.v_cache);
   a.block_table = L.block_table;
   a.ctx_len = L.ctx_len;
-  a.partial = L.partial;
+  // workspace: o rows [B, Hq, S, D] first, then (m, l) pairs [B, Hq, S]
+  a.S = decode_num_splits(L.max_blocks);
+  a.part_o = L.partial;
+  a.part_ml = reinterpret_cast<float2*>(L.partial + static_cast<size_t>(L.B) * L.Hq * a.S * L.D);
   a.status = L.status;
   a.B = L.B;
   a.Hq = L.Hq;
   a.Hkv = L.Hkv;
   a.max_blocks = L.max_blocks;
   a.num_blocks = L.num_blocks;
-  a.S = decode_num_splits(L.max_blocks);
   a.cs = L.scale * 1.4426950408889634f;
   const int G = L.Hq / L.Hkv;
   // paged pools as 4-D maps {d, Hkv, 16 slots, blocks}; box = one page of one KV head, 64
