@@ -30,6 +30,8 @@
 #include <cmath>
 #include <cstdio>
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -738,6 +740,472 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
 }
 
+// ----------------------------------------------------------------------------------------
+// Fused scoring: one exponential per score, on a cluster of CL = W / 128 CTAs.
+//
+// Work items are (r, g, hl): query head g*G + hl of a valid sequence r against the window
+// keys of KV head g; all CTAs of a cluster take the same items, CTA `rank` owns the 128 window
+// keys [start + 128 rank, start + 128 rank + 128). Per 128-query tile each CTA
+//   1. computes S = Q K^T over its keys (UMMA M = 128 queries, N = 144 key rows: the 9 pages
+//      that cover its 128 keys at any slot offset; only the owned columns are read);
+//   2. in the epilogue (8 warps: a TMEM lane quadrant and 64 owned keys each) takes the row
+//      max m_p over its 64 keys, P' = 2^(s*c - m_p + 15) and the row sum l_p, and stores P' as
+//      fp16 in shared memory, MN-major (rows along K) for the next product;
+//   3. combines the two parts of each row and sends (m, l) of its 128 keys to every CTA of the
+//      cluster (st.async into their shared memory, counted on their mbarrier);
+//   4. once all CL partials of a row are in: M = max m, L = sum l 2^(m - M), and the row
+//      weight of part p is w = 2^(m_p - M + 15) / L (so that P' w = 2^15 softmax); w goes to
+//      fp16 as three B columns (w1 + w2 + 2^-24 w3, exact to about 2^-36);
+//   5. D (128 keys x 16) += P'^T W: the column sums of the tile's softmax rows on the tensor
+//      cores (UMMA M = 128 keys, K = 128 queries, N = 16), accumulated over the item's tiles.
+// Step 4 of a tile runs in the epilogue after steps 1-3 of the next tile, so the exchange
+// latency hides behind a tile of work; P', the weights and the exchange slots are multi-
+// buffered for that. After the item's last tile, D (times 2^-15) gives the head's per-key
+// scores; a second kernel sums the G heads.
+// ----------------------------------------------------------------------------------------
+constexpr int kFEpiWarps = 16;                    // two teams of 8, tiles alternate between them
+constexpr int kFParts = 2;                        // per team: 2 warps per TMEM lane quadrant
+constexpr int kFPartKeys = 128 / kFParts;         // 64 keys per warp
+constexpr int kFThreads = 96 + 32 * kFEpiWarps;   // TMA, S issuer, column-sum issuer, epilogue
+constexpr int kFEpiThreads = 32 * kFEpiWarps;
+constexpr int kFKeys = 128;            // window keys owned per CTA
+constexpr int kFKRows = 144;           // key rows loaded per CTA (9 pages)
+constexpr int kFQRows = 128;           // queries per tile
+constexpr int kFMaxCluster = 8;
+constexpr int kFXStages = 4;           // exchange slots (a peer sends tile T only after every
+                                       // CTA has read its partials of tile T - 4)
+constexpr uint32_t kFEpiBarrier = 1;
+constexpr uint32_t kFSCols = 256;      // TMEM column stride of the two S buffers
+constexpr uint32_t kFDCol = 160;       // TMEM columns of the two D buffers: 160, 176
+
+// Work items (r, g) over valid sequences: KV head g of sequence r with all G of its query
+// heads (G * W / 128 query tiles).
+struct ItemCursor {
+  int r = 0, base = 0, per = -1;
+  SeqInfo s;
+  __device__ __forceinline__ bool seek(const ScoreArgs& a, int t, int& g) {
+    while (true) {
+      if (r >= a.R) return false;
+      if (per < 0) {
+        s = seq_info(a, r);
+        per = s.ok ? a.Hkv : 0;
+      }
+      if (t < base + per) break;
+      base += per;
+      ++r;
+      per = -1;
+    }
+    g = t - base;
+    return true;
+  }
+};
+
+template <int D>
+struct FusedSmem {
+  static constexpr int NCH = D / 64;
+  static constexpr uint32_t kKChunk = kFKRows * kRowBytes;     // one 64-channel chunk of K
+  static constexpr uint32_t kKBytes = NCH * kKChunk;
+  static constexpr uint32_t kQChunk = kFQRows * kRowBytes;
+  static constexpr uint32_t kQBytes = NCH * kQChunk;
+  static constexpr uint32_t kPAtom = 64 * kFQRows * 2;         // 64 keys x 128 queries, fp16
+  static constexpr uint32_t kPBytes = 2 * kPAtom;
+  static constexpr uint32_t kWBytes = 2 * 16 * kRowBytes;      // [k chunk][16 n rows][128 B]
+  static constexpr uint32_t kXBytes = kFXStages * kFMaxCluster * kFQRows * 8;
+  static constexpr uint32_t k_off = 0;
+  static constexpr uint32_t q_off = k_off + kKBytes;
+  static constexpr uint32_t p_off = q_off + 2 * kQBytes;
+  static constexpr uint32_t w_off = p_off + 2 * kPBytes;
+  static constexpr uint32_t x_off = w_off + 2 * kWBytes;
+  static constexpr uint32_t comb_off = x_off + kXBytes;         // [team][128] float2
+  static constexpr uint32_t bar_off = comb_off + 2 * kFQRows * 8;
+  static constexpr uint32_t kBars = 2 + 2 * 9 + kFXStages;
+  static constexpr uint32_t end = bar_off + kBars * 8 + 16;
+  static constexpr size_t bytes = 1024 + end;
+};
+
+// Byte offset of (n, k) in a K-major 128-byte-swizzled 16-row B operand [k chunk][n][128 B].
+__device__ __forceinline__ uint32_t w_offset(int n, int k) {
+  return static_cast<uint32_t>((k >> 6) * 2048 + n * 128 + ((((k & 63) >> 3) ^ (n & 7)) << 4) +
+                               (k & 7) * 2);
+}
+
+template <int D, int CL>
+__global__ void __launch_bounds__(kFThreads, 1)
+score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
+  using L = FusedSmem<D>;
+  constexpr int NCH = L::NCH;
+  constexpr uint32_t kPageBytes = 16 * kRowBytes;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* k_buf = smem + L::k_off;
+  uint8_t* q_buf = smem + L::q_off;
+  uint8_t* p_buf = smem + L::p_off;
+  uint8_t* w_buf = smem + L::w_off;
+  float2* x_buf = reinterpret_cast<float2*>(smem + L::x_off);     // [stage][src rank][row]
+  float2* comb = reinterpret_cast<float2*>(smem + L::comb_off);   // [team][row]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bar_off);
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = bars + 1;
+  uint64_t* q_full = bars + 2;     // [2]
+  uint64_t* q_empty = bars + 4;
+  uint64_t* s_full = bars + 6;
+  uint64_t* s_empty = bars + 8;
+  uint64_t* p_full = bars + 10;
+  uint64_t* w_full = bars + 12;
+  uint64_t* p_empty = bars + 14;
+  uint64_t* d_full = bars + 16;
+  uint64_t* d_empty = bars + 18;
+  uint64_t* x_full = bars + 20;    // [kFXStages]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const uint32_t rank = cluster_ctarank();
+  const int cid = static_cast<int>(cluster_id_x());
+  const int ncl = static_cast<int>(cluster_count_x());
+
+  if (threadIdx.x == 0) {
+    mbar_init(k_full, 1);
+    mbar_init(k_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], kFEpiThreads / 2);     // one team per tile
+      mbar_init(&p_full[i], kFEpiThreads / 2);
+      mbar_init(&w_full[i], kFEpiThreads / 2);
+      mbar_init(&p_empty[i], 1);
+      mbar_init(&d_full[i], 1);
+      mbar_init(&d_empty[i], kFEpiThreads / 2);
+    }
+    for (int i = 0; i < kFXStages; ++i) mbar_init(&x_full[i], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp >= 3) {
+    // the weight operands' unused rows (n = 3 * parts .. 15) stay zero
+    constexpr int kZ = 16 - 3 * kFParts;
+    static_assert(kZ * 8 * 2 * 2 <= kFEpiThreads * 8, "zero fill");
+    const int t = threadIdx.x - 96;
+    for (int i = t; i < 2 * 2 * kZ * 8; i += kFEpiThreads) {
+      const int buf = i / (16 * kZ), rem = i % (16 * kZ), kc = rem / (8 * kZ);
+      const int n = 3 * kFParts + (rem % (8 * kZ)) / 8, c = rem % 8;
+      *reinterpret_cast<uint4*>(w_buf + buf * L::kWBytes + kc * 2048 + n * 128 + c * 16) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  cluster_sync_all();     // every CTA's barriers exist before any peer signals them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // rows of invalid sequences: zero scores, reported (this cluster's share of them)
+    for (int r = cid * CL + static_cast<int>(rank); r < a.R; r += ncl * CL) {
+      if (seq_info(a, r).ok) continue;
+      for (int i = lane; i < a.Hkv * a.W; i += 32) a.scores[static_cast<size_t>(r) * a.Hkv * a.W + i] = 0.f;
+      if (lane == 0) report(a.status, KARA_ERR_INVALID_ARG);
+    }
+    // ---- TMA producer: the item's key pages, then its query tiles; the next item's page
+    // ids are fetched while this item's tiles stream ----
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+    }
+    const int TPI = a.G * CL;
+    ItemCursor cur;
+    int g = 0, T = 0;
+    bool have = cur.seek(a, cid, g);
+    auto page_ids = [&](const SeqInfo& s, int& npg) {
+      const int key0 = s.start + static_cast<int>(rank) * kFKeys;
+      npg = (key0 % 16) != 0 ? 9 : 8;
+      return lane < npg ? page_block(a, s.b, key0 / 16 + lane) : 0;
+    };
+    int npg = 0;
+    int my_blk = have ? page_ids(cur.s, npg) : 0;
+    for (int I = 0; have; ++I) {
+      if (__shfl_sync(0xffffffffu, *abort_flag != 0 ? 1 : 0, 0)) break;
+      const int r = cur.r, gi = g;
+      int ok = 1;
+      if (lane == 0) {
+        ok = mbar_wait(k_empty, (I & 1) ^ 1, abort_flag, a.status) ? 1 : 0;
+        if (ok) mbar_expect_tx(k_full, npg * NCH * kPageBytes);
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      for (int p = 0; p < npg; ++p) {
+        const int blk = __shfl_sync(0xffffffffu, my_blk, p);
+        if (lane == 0)
+          for (int ch = 0; ch < NCH; ++ch)
+            tma_load_4d(k_buf + ch * L::kKChunk + p * kPageBytes, &tm_k, k_full, ch * 64, gi, 0, blk);
+      }
+      // the next item's page ids (their loads overlap this item's query tiles)
+      have = cur.seek(a, cid + (I + 1) * ncl, g);
+      if (have) my_blk = page_ids(cur.s, npg);
+      bool stop = false;
+      if (lane == 0) {
+        for (int tq = 0; tq < TPI; ++tq, ++T) {
+          const int st = T & 1;
+          const int h = gi * a.G + tq / CL, qt = tq % CL;
+          if (!mbar_wait(&q_empty[st], ((T >> 1) & 1) ^ 1, abort_flag, a.status)) { stop = true; break; }
+          mbar_expect_tx(&q_full[st], L::kQBytes);
+          for (int ch = 0; ch < NCH; ++ch)
+            tma_load_4d(q_buf + st * L::kQBytes + ch * L::kQChunk, &tm_q, &q_full[st], ch * 64, h,
+                        qt * kFQRows, r);
+        }
+      }
+      T = __shfl_sync(0xffffffffu, T, 0);
+      if (__shfl_sync(0xffffffffu, stop ? 1 : 0, 0)) break;
+    }
+  } else if (warp == 1) {
+    // ---- UMMA issuer for S: runs ahead of the epilogue by one tile ----
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, kFKRows);
+      const int TPI = a.G * CL;
+      ItemCursor cur;
+      int g, T = 0, I = 0;
+      bool ok = true;
+      for (int it = cid; ok && !*abort_flag && cur.seek(a, it, g); it += ncl, ++I) {
+        if (!mbar_wait(k_full, I & 1, abort_flag, a.status)) break;
+        const uint32_t k_addr = smem_u32(k_buf);
+        for (int tq = 0; tq < TPI; ++tq, ++T) {
+          const int st = T & 1;
+          const uint32_t ph = (T >> 1) & 1;
+          if (!mbar_wait(&q_full[st], ph, abort_flag, a.status) ||
+              !mbar_wait(&s_empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t q_addr = smem_u32(q_buf + st * L::kQBytes);
+          const uint32_t d_tmem = tmem_base + st * kFSCols;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            const uint64_t ad = sw128_kmajor_desc(q_addr + (kk >> 2) * L::kQChunk + off);
+            const uint64_t bd = sw128_kmajor_desc(k_addr + (kk >> 2) * L::kKChunk + off);
+            umma_bf16(d_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&q_empty[st]);
+          umma_commit(&s_full[st]);
+          if (tq == TPI - 1) umma_commit(k_empty);
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ---- UMMA issuer for the column sums: D += P'^T W, tile by tile ----
+    if (lane == 0) {
+      const uint32_t idesc_c = idesc_f16_f32(128, 16, true);
+      const int TPI = a.G * CL;
+      ItemCursor cur;
+      int g, Tc = 0, Ic = 0;
+      for (int it = cid; !*abort_flag && cur.seek(a, it, g); it += ncl, ++Ic) {
+        bool ok = true;
+        for (int qt = 0; qt < TPI; ++qt, ++Tc) {
+          const int st = Tc & 1;
+          const uint32_t ph = (Tc >> 1) & 1;
+          if (!mbar_wait(&p_full[st], ph, abort_flag, a.status) ||
+              !mbar_wait(&w_full[st], ph, abort_flag, a.status) ||
+              (qt == 0 &&
+               !mbar_wait(&d_empty[Ic & 1], ((Ic >> 1) & 1) ^ 1, abort_flag, a.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t p_addr = smem_u32(p_buf + st * L::kPBytes);
+          const uint32_t w_addr = smem_u32(w_buf + st * L::kWBytes);
+          const uint32_t d_tmem = tmem_base + kFDCol + (Ic & 1) * 16;
+#pragma unroll
+          for (int ks = 0; ks < kFQRows / 16; ++ks) {
+            const uint64_t ad = sw128_mnmajor_desc(p_addr + ks * 2048, L::kPAtom, 1024);
+            const uint64_t bd = sw128_kmajor_desc(w_addr + (ks >> 2) * 2048 + (ks & 3) * 32);
+            umma_bf16(d_tmem, ad, bd, idesc_c, (ks > 0 || qt > 0) ? 1u : 0u);
+          }
+          umma_commit(&p_empty[st]);
+          if (qt == TPI - 1) umma_commit(&d_full[Ic & 1]);
+        }
+        if (!ok) break;
+      }
+    }
+  } else {
+    // ---- epilogue: two teams of 8 warps take alternate tiles (team = tile parity), so that
+    // one team's exponentials overlap the other's exchange and weights. In a team, warp
+    // (quad, part) owns TMEM lane quadrant `quad` and keys [64 part, 64 part + 64). ----
+    const int e = warp - 3;
+    const int team = e >> 3;
+    const int quad = warp & 3;
+    const int part = (e & 7) >> 2;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    const float2 cs2 = make_float2(a.cs, a.cs);
+    const uint32_t x_full_u32 = smem_u32(x_full);
+    const uint32_t x_buf_u32 = smem_u32(x_buf);
+    // warp-uniform bounded waits (a wait that gives up marks the whole warp aborted)
+    bool aborted = false;
+    auto wait_cta = [&](uint64_t* bar, uint32_t parity) {
+      const bool ok = aborted ? false : mbar_wait(bar, parity, abort_flag, a.status);
+      aborted = __any_sync(0xffffffffu, !ok) != 0;
+    };
+    auto wait_cluster = [&](uint64_t* bar, uint32_t parity) {
+      const bool ok = aborted ? false : mbar_wait_cluster(bar, parity, abort_flag, a.status);
+      aborted = __any_sync(0xffffffffu, !ok) != 0;
+    };
+    const int TPI = a.G * CL;
+    ItemCursor cur;
+    int g = 0, item_seen = -1;
+    for (int T = team;; T += 2) {
+      const int I = T / TPI;
+      if (I != item_seen) {
+        if (!cur.seek(a, cid + I * ncl, g)) break;
+        item_seen = I;
+      }
+      const int st = T & 1;     // = team: S, P and weight buffers
+      const uint32_t ph = (T >> 1) & 1;
+      const uint32_t scol = lane_base + st * kFSCols +
+                            ((cur.s.start + static_cast<int>(rank) * kFKeys) % 16) + part * kFPartKeys;
+      // (1) row max over this warp's 64 keys (first pass over TMEM)
+      wait_cta(&s_full[st], ph);
+      float mx = 0.f, l = 0.f;
+      if (!aborted) {
+        tc_fence_after();
+        float v[32];
+        float mm = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          tmem_ld16(scol + 32 * h, v);
+          tmem_ld16(scol + 32 * h + 16, v + 16);
+          tmem_wait_ld();
+          reg_fence<32>(v);
+          float mq[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float a0 = fmaxf(v[8 * q], v[8 * q + 1]), a1 = fmaxf(v[8 * q + 2], v[8 * q + 3]);
+            const float a2 = fmaxf(v[8 * q + 4], v[8 * q + 5]), a3 = fmaxf(v[8 * q + 6], v[8 * q + 7]);
+            mq[q] = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+          }
+          mm = fmaxf(mm, fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])));
+        }
+        mx = mm * a.cs;
+        wait_cta(&p_empty[st], ph ^ 1);
+      }
+      // (2) P' = 2^(s c - m + 15) as fp16 in shared memory (second pass), and the row sum
+      if (!aborted) {
+        const float2 nb2 = make_float2(15.f - mx, 15.f - mx);
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        uint8_t* prow = p_buf + st * L::kPBytes + part * L::kPAtom + (row >> 3) * 1024 +
+                        (row & 7) * 128;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float v[32];
+          tmem_ld16(scol + 32 * h, v);
+          tmem_ld16(scol + 32 * h + 16, v + 16);
+          tmem_wait_ld();
+          reg_fence<32>(v);
+          if (h == 1) {
+            tc_fence_before();
+            mbar_arrive(&s_empty[st]);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 8; i += 4) {
+              const int j = 8 * c + i;
+              const float2 x0 = ffma2(make_float2(v[j], v[j + 1]), cs2, nb2);
+              const float2 x1 = ffma2(make_float2(v[j + 2], v[j + 3]), cs2, nb2);
+              const float2 e0 = exp2_pair(x0, (j >> 1) & 3);
+              const float2 e1 = exp2_pair(x1, ((j >> 1) + 1) & 3);
+              acc0 = fadd2(acc0, e0);
+              acc1 = fadd2(acc1, e1);
+              pk[i / 2] = pack_f16x2(e0.x, e0.y);
+              pk[i / 2 + 1] = pack_f16x2(e1.x, e1.y);
+            }
+            const int cc = 4 * h + c;
+            *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+        l = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+        fence_proxy_async();
+        mbar_arrive(&p_full[st]);
+      }
+      // (3) the CTA's (m, l) of each row to every CTA of the cluster
+      const int xs = T % kFXStages;
+      if ((e & 7) == 0 && lane == 0) mbar_expect_tx(&x_full[xs], CL * kFQRows * 8);
+      if (part == 1) comb[team * kFQRows + row] = make_float2(mx, l);
+      named_barrier(kFEpiBarrier + team * 4 + quad, 64);   // the two warps sharing these rows
+      if (part == 0 && !aborted) {
+        const float2 o = comb[team * kFQRows + row];
+        const float M = fmaxf(mx, o.x);
+        const float Lc = l * ex2(mx - M) + o.y * ex2(o.x - M);
+        const uint32_t slot = x_buf_u32 + ((xs * kFMaxCluster + rank) * kFQRows + row) * 8;
+        const uint32_t xb = x_full_u32 + xs * 8;
+#pragma unroll
+        for (int c = 0; c < CL; ++c) st_async_f2(map_to_rank(slot, c), M, Lc, map_to_rank(xb, c));
+      }
+      // (4) once every CTA's partials are in: this part's weights w = 2^(m_p - M + 15) / L as
+      // three fp16 columns of the B operand
+      wait_cluster(&x_full[xs], (T / kFXStages) & 1);
+      if (!aborted) {
+        const float2* xr = x_buf + xs * kFMaxCluster * kFQRows + row;
+        float2 xv[CL];
+#pragma unroll
+        for (int c = 0; c < CL; ++c) xv[c] = xr[c * kFQRows];
+        float M = xv[0].x;
+#pragma unroll
+        for (int c = 1; c < CL; ++c) M = fmaxf(M, xv[c].x);
+        // (FMA-pipe exponentials: the SFU is busy with the other team's tile)
+        float Lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < CL; ++c) Lsum += xv[c].y * ex2_fma(xv[c].x - M);
+        const float w = ex2_fma(mx - M + 15.f) / Lsum;
+        const __half w1 = __float2half_rn(w);
+        const float r1 = w - __half2float(w1);
+        const __half w2 = __float2half_rn(r1);
+        const float r2 = r1 - __half2float(w2);
+        const __half w3 = __float2half_rn(r2 * 16777216.f);
+        uint8_t* wb = w_buf + st * L::kWBytes;
+        *reinterpret_cast<__half*>(wb + w_offset(3 * part, row)) = w1;
+        *reinterpret_cast<__half*>(wb + w_offset(3 * part + 1, row)) = w2;
+        *reinterpret_cast<__half*>(wb + w_offset(3 * part + 2, row)) = w3;
+        fence_proxy_async();
+        mbar_arrive(&w_full[st]);
+      }
+      // (5) the item's last tile: the per-key sums over all G heads, read by this team
+      if (T % TPI == TPI - 1) {
+        wait_cta(&d_full[I & 1], (I >> 1) & 1);
+        if (!aborted) {
+          tc_fence_after();
+          if (part == 0) {
+            // lane quadrant `quad` holds keys [32 quad, 32 quad + 32): part quad / 2's columns
+            float d[4];
+            tmem_ld4(lane_base + kFDCol + (I & 1) * 16 + 3 * (quad >> 1), d);
+            tmem_wait_ld();
+            reg_fence<4>(d);
+            const float val = (d[0] + d[1] + d[2] * (1.f / 16777216.f)) * (1.f / 32768.f);
+            a.scores[(static_cast<size_t>(cur.r) * a.Hkv + g) * a.W + rank * kFKeys + row] = val;
+          }
+          tc_fence_before();
+          mbar_arrive(&d_empty[I & 1]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+  cluster_sync_all();     // no CTA leaves while a peer may still write into its shared memory
+}
+
 template <int D>
 constexpr size_t rowstats_smem() {
   return 1024 + 2 * (D / 64) * kKRows1 * kRowBytes + kQStages1 * (D / 64) * kQRows1 * kRowBytes +
@@ -838,6 +1306,49 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   a.max_blocks = L.max_blocks;
   a.num_blocks = L.num_blocks;
   a.cs = L.scale * 1.4426950408889634f;
+
+
+  // Windows of 128, 256, 512 or 1024 keys: the fused single-exponential kernel on clusters of
+  // W / 128 CTAs.
+  if (L.W == 128 || L.W == 256 || L.W == 512 || L.W == 1024) {
+    const int CL = L.W / kFKeys;
+    auto kern = CL == 1 ? score_fused_kernel<D, 1>
+              : CL == 2 ? score_fused_kernel<D, 2>
+              : CL == 4 ? score_fused_kernel<D, 4> : score_fused_kernel<D, 8>;
+    constexpr size_t smem = FusedSmem<D>::bytes;
+    static int max_clusters[kFMaxCluster + 1] = {0};   // per cluster size, queried once
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kFThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (max_clusters[CL] == 0) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
+      cfg.gridDim = dim3(CL * (sm_count() / CL));
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+        check_launch("score_fused_kernel occupancy");
+        return KARA_ERR_CUDA;
+      }
+      max_clusters[CL] = n;
+    }
+    const int items = L.R * L.Hkv;    // upper bound (valid sequences only are walked)
+    const int ncl = std::max(1, std::min(max_clusters[CL], items));
+    cfg.gridDim = dim3(ncl * CL);
+    cudaLaunchKernelEx(&cfg, kern, tq1, tk, a);
+    if (check_launch("score_fused_kernel") != KARA_OK) {
+      describe_kernel("score_fused_kernel", reinterpret_cast<const void*>(kern), kFThreads, smem);
+      return KARA_ERR_CUDA;
+    }
+    return KARA_OK;
+  }
 
   static bool attr_set = false;
   if (!attr_set) {
