@@ -816,8 +816,8 @@ struct FusedSmem {
   static constexpr uint32_t p_off = q_off + 2 * kQBytes;
   static constexpr uint32_t w_off = p_off + 2 * kPBytes;
   static constexpr uint32_t x_off = w_off + 2 * kWBytes;
-  static constexpr uint32_t comb_off = x_off + kXBytes;         // [team][128] float2
-  static constexpr uint32_t bar_off = comb_off + 2 * kFQRows * 8;
+  static constexpr uint32_t comb_off = x_off + kXBytes;         // [team][part][128] float2
+  static constexpr uint32_t bar_off = comb_off + 2 * 2 * kFQRows * 8;
   static constexpr uint32_t kBars = 2 + 2 * 9 + kFXStages;
   static constexpr uint32_t end = bar_off + kBars * 8 + 16;
   static constexpr size_t bytes = 1024 + end;
@@ -845,7 +845,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint8_t* p_buf = smem + L::p_off;
   uint8_t* w_buf = smem + L::w_off;
   float2* x_buf = reinterpret_cast<float2*>(smem + L::x_off);     // [stage][src rank][row]
-  float2* comb = reinterpret_cast<float2*>(smem + L::comb_off);   // [team][row]
+  float2* comb = reinterpret_cast<float2*>(smem + L::comb_off);   // [team][part][row]: (m, l)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bar_off);
   uint64_t* k_full = bars;
   uint64_t* k_empty = bars + 1;
@@ -877,7 +877,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], kFEpiThreads / 2);     // one team per tile
       mbar_init(&p_full[i], kFEpiThreads / 2);
-      mbar_init(&w_full[i], kFEpiThreads / 2);
+      mbar_init(&w_full[i], kFEpiThreads / 4);      // the team's part-1 threads
       mbar_init(&p_empty[i], 1);
       mbar_init(&d_full[i], 1);
       mbar_init(&d_empty[i], kFEpiThreads / 2);
@@ -1057,13 +1057,10 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     };
     const int TPI = a.G * CL;
     ItemCursor cur;
-    int g = 0, item_seen = -1;
-    for (int T = team;; T += 2) {
-      const int I = T / TPI;
-      if (I != item_seen) {
-        if (!cur.seek(a, cid + I * ncl, g)) break;
-        item_seen = I;
-      }
+    int g = 0, I = 0, tq = team;          // item index and tile within the item (no divisions:
+    while (tq >= TPI) { tq -= TPI; ++I; }  // they would queue behind the exponentials)
+    bool have = cur.seek(a, cid + I * ncl, g);
+    for (int T = team; have; T += 2) {
       const int st = T & 1;     // = team: S, P and weight buffers
       const uint32_t ph = (T >> 1) & 1;
       const uint32_t scol = lane_base + st * kFSCols +
@@ -1081,14 +1078,13 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
           tmem_ld16(scol + 32 * h + 16, v + 16);
           tmem_wait_ld();
           reg_fence<32>(v);
-          float mq[4];
+          float mq[11];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float a0 = fmaxf(v[8 * q], v[8 * q + 1]), a1 = fmaxf(v[8 * q + 2], v[8 * q + 3]);
-            const float a2 = fmaxf(v[8 * q + 4], v[8 * q + 5]), a3 = fmaxf(v[8 * q + 6], v[8 * q + 7]);
-            mq[q] = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
-          }
-          mm = fmaxf(mm, fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])));
+          for (int q = 0; q < 10; ++q) mq[q] = fmax3(v[3 * q], v[3 * q + 1], v[3 * q + 2]);
+          mq[10] = fmaxf(v[30], v[31]);
+          const float m0 = fmax3(mq[0], mq[1], mq[2]), m1 = fmax3(mq[3], mq[4], mq[5]);
+          const float m2 = fmax3(mq[6], mq[7], mq[8]), m3 = fmax3(mq[9], mq[10], mm);
+          mm = fmaxf(fmax3(m0, m1, m2), m3);
         }
         mx = mm * a.cs;
         wait_cta(&p_empty[st], ph ^ 1);
@@ -1118,8 +1114,8 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
               const int j = 8 * c + i;
               const float2 x0 = ffma2(make_float2(v[j], v[j + 1]), cs2, nb2);
               const float2 x1 = ffma2(make_float2(v[j + 2], v[j + 3]), cs2, nb2);
-              const float2 e0 = exp2_pair(x0, (j >> 1) & 3);
-              const float2 e1 = exp2_pair(x1, ((j >> 1) + 1) & 3);
+              const float2 e0 = make_float2(ex2(x0.x), ex2(x0.y));
+              const float2 e1 = make_float2(ex2(x1.x), ex2(x1.y));
               acc0 = fadd2(acc0, e0);
               acc1 = fadd2(acc1, e1);
               pk[i / 2] = pack_f16x2(e0.x, e0.y);
@@ -1137,10 +1133,11 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       // (3) the CTA's (m, l) of each row to every CTA of the cluster
       const int xs = T % kFXStages;
       if ((e & 7) == 0 && lane == 0) mbar_expect_tx(&x_full[xs], CL * kFQRows * 8);
-      if (part == 1) comb[team * kFQRows + row] = make_float2(mx, l);
+      float2* cb = comb + team * 2 * kFQRows;
+      cb[part * kFQRows + row] = make_float2(mx, l);
       named_barrier(kFEpiBarrier + team * 4 + quad, 64);   // the two warps sharing these rows
       if (part == 0 && !aborted) {
-        const float2 o = comb[team * kFQRows + row];
+        const float2 o = cb[kFQRows + row];
         const float M = fmaxf(mx, o.x);
         const float Lc = l * ex2(mx - M) + o.y * ex2(o.x - M);
         const uint32_t slot = x_buf_u32 + ((xs * kFMaxCluster + rank) * kFQRows + row) * 8;
@@ -1148,10 +1145,11 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int c = 0; c < CL; ++c) st_async_f2(map_to_rank(slot, c), M, Lc, map_to_rank(xb, c));
       }
-      // (4) once every CTA's partials are in: this part's weights w = 2^(m_p - M + 15) / L as
-      // three fp16 columns of the B operand
-      wait_cluster(&x_full[xs], (T / kFXStages) & 1);
-      if (!aborted) {
+      // (4) meanwhile, once every CTA's partials are in, the row's thread of part 1 writes the
+      // weights of both parts, w_p = 2^(m_p - M + 15) / L, as three fp16 columns each of the B
+      // operand (FMA-pipe exponentials: the SFU is busy with the other team's tile)
+      if (part == 1) wait_cluster(&x_full[xs], (T / kFXStages) & 1);
+      if (part == 1 && !aborted) {
         const float2* xr = x_buf + xs * kFMaxCluster * kFQRows + row;
         float2 xv[CL];
 #pragma unroll
@@ -1159,25 +1157,29 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
         float M = xv[0].x;
 #pragma unroll
         for (int c = 1; c < CL; ++c) M = fmaxf(M, xv[c].x);
-        // (FMA-pipe exponentials: the SFU is busy with the other team's tile)
         float Lsum = 0.f;
 #pragma unroll
-        for (int c = 0; c < CL; ++c) Lsum += xv[c].y * ex2_fma(xv[c].x - M);
-        const float w = ex2_fma(mx - M + 15.f) / Lsum;
-        const __half w1 = __float2half_rn(w);
-        const float r1 = w - __half2float(w1);
-        const __half w2 = __float2half_rn(r1);
-        const float r2 = r1 - __half2float(w2);
-        const __half w3 = __float2half_rn(r2 * 16777216.f);
+        for (int c = 0; c < CL; ++c) Lsum += xv[c].y * ex2(xv[c].x - M);
+        const float inv = 1.f / Lsum;
+        const float m_part0 = cb[row].x;
         uint8_t* wb = w_buf + st * L::kWBytes;
-        *reinterpret_cast<__half*>(wb + w_offset(3 * part, row)) = w1;
-        *reinterpret_cast<__half*>(wb + w_offset(3 * part + 1, row)) = w2;
-        *reinterpret_cast<__half*>(wb + w_offset(3 * part + 2, row)) = w3;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const float w = ex2((q == 0 ? m_part0 : mx) - M + 15.f) * inv;
+          const __half w1 = __float2half_rn(w);
+          const float r1 = w - __half2float(w1);
+          const __half w2 = __float2half_rn(r1);
+          const float r2 = r1 - __half2float(w2);
+          const __half w3 = __float2half_rn(r2 * 16777216.f);
+          *reinterpret_cast<__half*>(wb + w_offset(3 * q, row)) = w1;
+          *reinterpret_cast<__half*>(wb + w_offset(3 * q + 1, row)) = w2;
+          *reinterpret_cast<__half*>(wb + w_offset(3 * q + 2, row)) = w3;
+        }
         fence_proxy_async();
         mbar_arrive(&w_full[st]);
       }
       // (5) the item's last tile: the per-key sums over all G heads, read by this team
-      if (T % TPI == TPI - 1) {
+      if (tq == TPI - 1) {
         wait_cta(&d_full[I & 1], (I >> 1) & 1);
         if (!aborted) {
           tc_fence_after();
@@ -1193,6 +1195,13 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
           tc_fence_before();
           mbar_arrive(&d_empty[I & 1]);
         }
+      }
+      tq += 2;
+      if (tq >= TPI) {
+        tq -= TPI;
+        ++I;
+        if (tq >= TPI) { tq -= TPI; ++I; }   // TPI = 1
+        have = cur.seek(a, cid + I * ncl, g);
       }
     }
   }
