@@ -173,7 +173,8 @@ kara_status kara_compact(const kara_layer_kv* layers, int32_t num_layers, const 
   kara_status st = check_pool(pool);
   if (st != KARA_OK) return st;
   if (pool->free_list == nullptr || pool->free_top == nullptr) return KARA_ERR_INVALID_ARG;
-  if (num_seqs < 0 || window < 1 || k < 1 || k > window) return KARA_ERR_INVALID_ARG;
+  if (num_seqs < 0 || window < 1 || window > KARA_MAX_WINDOW || k < 1 || k > window)
+    return KARA_ERR_INVALID_ARG;
   if (num_seqs == 0) return KARA_OK;
   if (keep == nullptr || dev_status == nullptr) return KARA_ERR_INVALID_ARG;
   CompactLaunch L;

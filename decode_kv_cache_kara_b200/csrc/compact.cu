@@ -6,16 +6,20 @@
 // ...": states outside the ladder are dropped and the rest packed into a smaller cache
 // (method details), re-applied when the cache is full (iterative compaction).
 //
-// Three stream-ordered kernels per call:
+// Two stream-ordered kernels per call:
 //   plan     (one CTA)   validates every due sequence, computes its page geometry and pops its
 //                        fresh blocks from the free list (sequence order, stack top first); on
 //                        any error it records the status and marks the plan invalid.
-//   gather   (wide grid) copies rows with 16-byte loads/stores: sources through the old
-//                        block table, destinations into the fresh blocks. Kara copies one KV
-//                        head's row per kept position; LaCache copies whole [Hkv, d] rows of
-//                        the ladder's kept slots (computed analytically per layer).
-//   finalize (one CTA)   rewrites the block table, pushes the old blocks, sets ctx_len and
-//                        free_top.
+//   gather   (wide grid, launched as a programmatic dependent of the plan) copies rows with
+//                        16-byte loads/stores, all of a thread's rows in flight at once:
+//                        sources through the old block table, destinations into the fresh
+//                        blocks. Kara copies one KV head's row per kept position; LaCache copies
+//                        whole [Hkv, d] rows of the ladder's kept slots (computed analytically
+//                        per layer). Per sequence, the CTA that finishes last (a counter in
+//                        the sequence's plan row, zeroed by the plan) rewrites the sequence's
+//                        block table entries, pushes its old blocks and sets its ctx_len;
+//                        every CTA that reads that sequence's old table entries is done by
+//                        then. The plan sets free_top (nothing later in the call reads it).
 // The gather reads only blocks that belong to the sequences and writes only fresh blocks, so
 // sources never alias destinations; nothing is modified unless the plan is valid.
 #include <cstdint>
@@ -30,8 +34,8 @@ namespace {
 
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanHeader = 16;   // valid, total_new, total_old, top
-constexpr int kPlanStride = 12;   // b, n, start, off, p0, n_old, n_new, base_new, base_old
-enum { P_B = 0, P_N, P_START, P_OFF, P_P0, P_NOLD, P_NNEW, P_BNEW, P_BOLD };
+constexpr int kPlanStride = 12;   // b, n, start, off, p0, n_old, n_new, base_new, base_old, done
+enum { P_B = 0, P_N, P_START, P_OFF, P_P0, P_NOLD, P_NNEW, P_BNEW, P_BOLD, P_DONE };
 
 __device__ int block_scan_add(int v, int* buf, int* total) {
   // exclusive scan over 1024 threads (32 warps)
@@ -66,7 +70,7 @@ struct PlanParams {
   const int32_t* block_table;
   const int32_t* ctx_len;
   const int32_t* free_list;
-  const int32_t* free_top;
+  int32_t* free_top;
   const int32_t* seq_ids;
   int32_t* plan;
   int32_t* status;
@@ -75,17 +79,6 @@ struct PlanParams {
   int W, k, lacache, min_len;
 };
 
-// Row r of the plan whose [base_old, base_old + n_old) range holds flat page index i.
-__device__ __forceinline__ int plan_row_of(const int32_t* rows, int R, int i) {
-  int lo = 0, hi = R - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (rows[static_cast<size_t>(mid) * kPlanStride + P_BOLD] <= i) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
-}
-
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) {
   __shared__ int buf[33];
   __shared__ int err;
@@ -93,8 +86,16 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
   int32_t* hdr = p.plan;
   int32_t* rows = p.plan + kPlanHeader;
   int32_t* fresh = rows + static_cast<size_t>(p.R) * kPlanStride;
-  if (threadIdx.x == 0) { err = 0; carry_new = 0; carry_old = 0; }
+  __shared__ int s_top;
+  if (threadIdx.x == 0) {
+    err = 0;
+    carry_new = 0;
+    carry_old = 0;
+    s_top = *p.free_top;     // read once, early: thread 0 also writes the new top below
+  }
   __syncthreads();
+  // the gather may be scheduled now; it waits for this grid's results itself
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // 1. geometry of every due sequence, exclusive scans of its fresh / old page counts
   for (int base = 0; base < p.R; base += kPlanThreads) {
     const int r = base + threadIdx.x;
@@ -132,6 +133,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
       row[P_P0] = p0;
       row[P_NOLD] = n_old;
       row[P_NNEW] = n_new;
+      row[P_DONE] = 0;     // gather CTAs of this sequence done
     }
     int tot_new, tot_old;
     const int ex_new = block_scan_add(n_new, buf, &tot_new);
@@ -145,18 +147,27 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
     if (threadIdx.x == 0) { carry_new += tot_new; carry_old += tot_old; }
     __syncthreads();
   }
-  // 2. every old page id of every due sequence must be a valid block (flat loop over pages)
-  const int total_old = carry_old;
-  for (int i = threadIdx.x; i < total_old; i += kPlanThreads) {
-    const int r = plan_row_of(rows, p.R, i);
-    const int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
-    const int blk = p.block_table[static_cast<size_t>(row[P_B]) * p.max_blocks + row[P_P0] +
-                                  (i - row[P_BOLD])];
-    if (blk < 0 || blk >= p.num_blocks) atomicCAS(&err, 0, KARA_ERR_BAD_BLOCK);
+  // 2. every old page id of every due sequence must be a valid block (a warp per sequence);
+  // the fresh blocks are popped at the same time (sequence order, stack top first; they are
+  // used only if the plan turns out valid)
+  {
+    const int top = s_top;
+    if (top >= 0 && top <= p.num_blocks && carry_new <= top)
+      for (int i = threadIdx.x; i < carry_new; i += kPlanThreads) fresh[i] = p.free_list[top - 1 - i];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int r = warp; r < p.R; r += kPlanThreads / 32) {
+      const int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
+      const int n_old = row[P_NOLD];
+      const int32_t* tab = p.block_table + static_cast<size_t>(row[P_B]) * p.max_blocks + row[P_P0];
+      for (int pg = lane; pg < n_old; pg += 32) {
+        const int blk = tab[pg];
+        if (blk < 0 || blk >= p.num_blocks) atomicCAS(&err, 0, KARA_ERR_BAD_BLOCK);
+      }
+    }
   }
   __syncthreads();
-  const int top = *p.free_top;
   if (threadIdx.x == 0) {
+    const int top = s_top;
     int code = err;
     if (!code && (top < 0 || top > p.num_blocks)) code = KARA_ERR_INVALID_ARG;
     if (!code && carry_new > top) code = KARA_ERR_OUT_OF_BLOCKS;
@@ -167,42 +178,47 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
     hdr[1] = carry_new;
     hdr[2] = carry_old;
     hdr[3] = top;
+    // pops [top - new, top), pushes [top - new, top - new + old): the final top
+    if (!code) *p.free_top = top - carry_new + carry_old;
     err = code;
   }
-  __syncthreads();
-  if (err) return;
-  // 3. pop the fresh blocks (sequence order, stack top first)
-  for (int i = threadIdx.x; i < carry_new; i += kPlanThreads) fresh[i] = p.free_list[top - 1 - i];
 }
 
 struct FinalizeParams {
   int32_t* block_table;
   int32_t* ctx_len;
   int32_t* free_list;
-  int32_t* free_top;
-  const int32_t* plan;
+  int32_t* plan;
   int R, max_blocks, k;   // k: kept slots (Kara) or budget (LaCache)
 };
 
-// One thread per old page: table entry -> fresh id or -1, old id -> free list.
-__global__ void __launch_bounds__(256) finalize_kernel(const FinalizeParams p) {
-  const int32_t* hdr = p.plan;
-  if (hdr[0] != 1) return;
-  const int32_t* rows = p.plan + kPlanHeader;
-  const int32_t* fresh = rows + static_cast<size_t>(p.R) * kPlanStride;
-  const int total_new = hdr[1], total_old = hdr[2], top = hdr[3];
-  const int push_base = top - total_new;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total_old; i += gridDim.x * blockDim.x) {
-    const int r = plan_row_of(rows, p.R, i);
-    const int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
-    const int pg = i - row[P_BOLD];
-    int32_t* entry = p.block_table + static_cast<size_t>(row[P_B]) * p.max_blocks + row[P_P0] + pg;
-    const int old = *entry;
-    *entry = pg < row[P_NNEW] ? fresh[row[P_BNEW] + pg] : -1;
-    p.free_list[push_base + i] = old;
-    if (pg == 0) p.ctx_len[row[P_B]] = row[P_START] + p.k;
+// Called by every thread of each gather CTA when its copies are done; `per_seq` CTAs work on
+// sequence row r. The last of them rewrites the sequence's table entries of its old pages
+// (fresh id or -1), pushes the old ids onto the free list and sets the sequence's ctx_len.
+// `s_old` / `s_fresh`: the sequence's old and fresh ids staged in shared memory (or null).
+__device__ void finalize_if_last(const FinalizeParams& p, int r, int per_seq,
+                                 const int* s_old = nullptr, const int* s_fresh = nullptr) {
+  __shared__ int s_last;
+  int32_t* row = p.plan + kPlanHeader + static_cast<size_t>(r) * kPlanStride;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(&row[P_DONE], 1) == per_seq - 1;
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) *p.free_top = push_base + total_old;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int32_t* hdr = p.plan;
+  const int32_t* fresh = p.plan + kPlanHeader + static_cast<size_t>(p.R) * kPlanStride;
+  const int push_base = hdr[3] - hdr[1];
+  const int n_old = row[P_NOLD], n_new = row[P_NNEW], bnew = row[P_BNEW], bold = row[P_BOLD];
+  int32_t* tab = p.block_table + static_cast<size_t>(row[P_B]) * p.max_blocks + row[P_P0];
+  for (int pg = threadIdx.x; pg < n_old; pg += blockDim.x) {
+    const int old = s_old ? s_old[pg] : tab[pg];
+    tab[pg] = pg < n_new ? (s_fresh ? s_fresh[pg] : fresh[bnew + pg]) : -1;
+    p.free_list[push_base + bold + pg] = old;
+  }
+  if (threadIdx.x == 0 && n_old > 0) p.ctx_len[row[P_B]] = row[P_START] + p.k;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -219,10 +235,18 @@ struct KaraGather {
   const int32_t* plan;
   int32_t* status;
   int R, Hkv, k, W, max_blocks;
+  FinalizeParams fin;
 };
+
+// Pages a window can span (KARA_MAX_WINDOW slots at any slot offset), plus one.
+constexpr int kMaxWindowPages = (KARA_MAX_WINDOW + 15 + 15) / 16 + 1;
 
 template <int D>
 __global__ void __launch_bounds__(kGatherThreads) kara_gather_kernel(const KaraGather g) {
+  __shared__ int s_old[kMaxWindowPages];     // old block ids of the window's pages
+  __shared__ int s_fresh[kMaxWindowPages];   // the sequence's fresh block ids
+  __shared__ int s_keep[kChunkRows];         // this chunk's kept positions
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int32_t* hdr = g.plan;
   if (hdr[0] != 1) return;
   constexpr int kVecPerRow = D * 2 / 16;                  // 16-byte pieces per head row
@@ -235,9 +259,17 @@ __global__ void __launch_bounds__(kGatherThreads) kara_gather_kernel(const KaraG
   const int32_t* fresh = rows + static_cast<size_t>(g.R) * kPlanStride;
   const int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
   const int b = row[P_B], start = row[P_START], off = row[P_OFF], p0 = row[P_P0];
+  const int n_old = row[P_NOLD], n_new = row[P_NNEW];
+  const int t0 = chunk * kChunkRows;
+  const int t1 = min(g.k, t0 + kChunkRows);
+  // one round trip for every index this CTA needs
+  const int32_t* tab = g.block_table + static_cast<size_t>(b) * g.max_blocks + p0;
   const int32_t* fr = fresh + row[P_BNEW];
-  const int32_t* tab = g.block_table + static_cast<size_t>(b) * g.max_blocks;
   const int32_t* kp = g.keep + ((static_cast<size_t>(layer) * g.R + r) * g.Hkv + head) * g.k;
+  for (int i = threadIdx.x; i < n_old; i += kGatherThreads) s_old[i] = tab[i];
+  for (int i = threadIdx.x; i < n_new; i += kGatherThreads) s_fresh[i] = fr[i];
+  for (int i = threadIdx.x; i < t1 - t0; i += kGatherThreads) s_keep[i] = kp[t0 + i];
+  __syncthreads();
   const uint4* ksrc = reinterpret_cast<const uint4*>(g.layers.k[layer]);
   const uint4* vsrc = reinterpret_cast<const uint4*>(g.layers.v[layer]);
   uint4* kdst = reinterpret_cast<uint4*>(g.layers.k[layer]);
@@ -246,11 +278,9 @@ __global__ void __launch_bounds__(kGatherThreads) kara_gather_kernel(const KaraG
   const int sub = threadIdx.x / kVecPerRow;
 
   // rows handled by this CTA: prefix rows (chunk 0 only), then kept rows of the chunk
-  const int t0 = chunk * kChunkRows;
-  const int t1 = min(g.k, t0 + kChunkRows);
   const int npre = (chunk == 0) ? off : 0;
   const int total = npre + max(0, t1 - t0);
-  constexpr int kUnroll = 4;
+  constexpr int kUnroll = 8;
   for (int base = sub; base < total; base += kRowsPerPass * kUnroll) {
     uint4 kv[kUnroll], vv[kUnroll];
     size_t dsti[kUnroll];
@@ -265,7 +295,7 @@ __global__ void __launch_bounds__(kGatherThreads) kara_gather_kernel(const KaraG
         src_slot = dst_slot = p0 * 16 + i;
       } else {
         const int t = t0 + (i - npre);
-        const int pos = kp[t];
+        const int pos = s_keep[i - npre];
         if (pos < 0 || pos >= g.W) {      // keep entry outside the window: row left unwritten
           report(g.status, KARA_ERR_INVALID_ARG);
           act[u] = false;
@@ -274,8 +304,8 @@ __global__ void __launch_bounds__(kGatherThreads) kara_gather_kernel(const KaraG
         src_slot = start + pos;
         dst_slot = start + t;
       }
-      const int sblk = tab[src_slot >> 4];
-      const int dblk = fr[(dst_slot >> 4) - p0];
+      const int sblk = s_old[(src_slot >> 4) - p0];
+      const int dblk = s_fresh[(dst_slot >> 4) - p0];
       const size_t si = ((static_cast<size_t>(sblk) * 16 + (src_slot & 15)) * g.Hkv + head) *
                             kVecPerRow + vec;
       dsti[u] = ((static_cast<size_t>(dblk) * 16 + (dst_slot & 15)) * g.Hkv + head) *
@@ -290,6 +320,7 @@ __global__ void __launch_bounds__(kGatherThreads) kara_gather_kernel(const KaraG
       vdst[dsti[u]] = vv[u];
     }
   }
+  finalize_if_last(g.fin, r, gridDim.x * g.Hkv * gridDim.z, s_old, s_fresh);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -302,6 +333,7 @@ struct LadderGather {
   int R, L, max_blocks;
   int row_vecs;          // 16-byte pieces per slot row (Hkv * D * 2 / 16)
   int span, overlap, rung, budget, sink, recent, r_max;
+  FinalizeParams fin;
 };
 
 constexpr int kLadderSlots = 32;
@@ -328,6 +360,7 @@ __device__ __forceinline__ int ladder_source(const LadderGather& g, int layer, i
 }
 
 __global__ void __launch_bounds__(kGatherThreads) ladder_gather_kernel(const LadderGather g) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int32_t* hdr = g.plan;
   if (hdr[0] != 1) return;
   const int chunk = blockIdx.x;
@@ -373,6 +406,23 @@ __global__ void __launch_bounds__(kGatherThreads) ladder_gather_kernel(const Lad
       vdst[dsti[u]] = vv[u];
     }
   }
+  finalize_if_last(g.fin, r, gridDim.x * gridDim.z);
+}
+
+// Launches `kernel` on `grid` x kGatherThreads as a programmatic dependent of the previous
+// kernel in the stream (the plan).
+template <typename Arg>
+void launch_dependent(void (*kernel)(Arg), dim3 grid, const Arg& arg, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kGatherThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, arg);
 }
 
 }  // namespace
@@ -418,19 +468,16 @@ kara_status launch_compact(const CompactLaunch& L, cudaStream_t stream) {
   g.k = L.k;
   g.W = L.W;
   g.max_blocks = L.max_blocks;
+  g.fin.block_table = L.block_table;
+  g.fin.ctx_len = L.ctx_len;
+  g.fin.free_list = L.free_list;
+  g.fin.plan = L.plan;
+  g.fin.R = L.R;
+  g.fin.max_blocks = L.max_blocks;
+  g.fin.k = L.k;
   dim3 grid((L.k + kChunkRows - 1) / kChunkRows, L.R * L.Hkv, L.L);
-  if (L.D == 128) kara_gather_kernel<128><<<grid, kGatherThreads, 0, stream>>>(g);
-  else kara_gather_kernel<64><<<grid, kGatherThreads, 0, stream>>>(g);
-  FinalizeParams fp;
-  fp.block_table = L.block_table;
-  fp.ctx_len = L.ctx_len;
-  fp.free_list = L.free_list;
-  fp.free_top = L.free_top;
-  fp.plan = L.plan;
-  fp.R = L.R;
-  fp.max_blocks = L.max_blocks;
-  fp.k = L.k;
-  finalize_kernel<<<8, 256, 0, stream>>>(fp);
+  if (L.D == 128) launch_dependent(kara_gather_kernel<128>, grid, g, stream);
+  else launch_dependent(kara_gather_kernel<64>, grid, g, stream);
   return check_launch(__func__);
 }
 
@@ -469,18 +516,15 @@ kara_status launch_lacache(const LacacheLaunch& L, cudaStream_t stream) {
   g.sink = L.sink;
   g.recent = L.recent;
   g.r_max = r_max;
+  g.fin.block_table = L.block_table;
+  g.fin.ctx_len = L.ctx_len;
+  g.fin.free_list = L.free_list;
+  g.fin.plan = L.plan;
+  g.fin.R = L.R;
+  g.fin.max_blocks = L.max_blocks;
+  g.fin.k = L.budget;
   dim3 grid((L.budget + kLadderSlots - 1) / kLadderSlots, L.R, L.L);
-  ladder_gather_kernel<<<grid, kGatherThreads, 0, stream>>>(g);
-  FinalizeParams fp;
-  fp.block_table = L.block_table;
-  fp.ctx_len = L.ctx_len;
-  fp.free_list = L.free_list;
-  fp.free_top = L.free_top;
-  fp.plan = L.plan;
-  fp.R = L.R;
-  fp.max_blocks = L.max_blocks;
-  fp.k = L.budget;
-  finalize_kernel<<<8, 256, 0, stream>>>(fp);
+  launch_dependent(ladder_gather_kernel, grid, g, stream);
   return check_launch(__func__);
 }
 
