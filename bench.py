@@ -319,6 +319,54 @@ def e2e_run(cache: dict, wl: synth.Workload, steps: int, warmup: int) -> dict:
     return {"ms_per_step": ms, "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes}
 
 
+def lacache_run(dev, batch: int, reps: int = 5, warmup: int = 3) -> dict:
+    """One LaCache ladder-compaction pass (all 32 layers, 64K -> 8192 slots per layer) on the
+    LaCache workload, timed with CUDA events; the block table, lengths and free list are
+    restored between passes (the pass only writes fresh blocks), so every pass sees the same
+    full cache."""
+    from decode_kv_cache_kara_b200 import kara as K
+    wl = synth.WORKLOADS["lacache"].with_(batch=batch)
+    ex = wl.extra
+    cache = synth.make_cache(wl, 1234 + 4, dev, with_queries=False)
+    pool = K.PagedPool.from_cache(cache)
+    saved = {k: cache[k].clone() for k in ("block_table", "ctx_len", "free_list", "free_top")}
+    ws = torch.empty(K.kara_workspace_bytes(K.OP_LACACHE, pool, wl.batch, 0, 0, ex["budget"]),
+                     dtype=torch.uint8, device=dev)
+    status = K.new_status(dev)
+
+    def one():
+        K.lacache_compact(cache["k"], cache["v"], pool, ex["span"], ex["overlap"], ex["rung"],
+                          ex["budget"], ex["sink"], ex["recent"], workspace=ws, status=status)
+
+    def restore():
+        for k, t in saved.items():
+            cache[k].copy_(t)
+
+    for _ in range(warmup):
+        one()
+        restore()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        one()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+        restore()
+    torch.cuda.synchronize()
+    st = K.read_status(status)
+    ms = sum(times) / len(times)
+    # every layer keeps `budget` slots: K and V rows of [Hkv, d] read once and written once
+    nbytes = 2 * 2 * wl.batch * wl.layers * ex["budget"] * wl.hkv * wl.head_dim * 2
+    del cache, saved, ws
+    torch.cuda.empty_cache()
+    return {"ms": ms, "bound": "hbm", "gbs": nbytes / ms / 1e6, "bytes": nbytes, "status": st,
+            "workload": f"lacache: batch {wl.batch}, 32 layers, 8 KV heads, d=128, 64K-token "
+                        f"caches, S=8, O=4, rung 64, budget 8192 per layer; one pass (all layers)"}
+
+
 def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
     import torch.distributed as dist
     from decode_kv_cache_kara_b200 import kara as K
@@ -417,6 +465,11 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
                 "unit": "GB/s", "frac": dk["gbs"] / peaks["hbm_gbs"], "traffic": traffic,
                 "peak_source": f"{src} HBM copy (MEASURED_PEAKS.json hbm_gbs)"}
 
+    if world == 1 and not args.no_lacache:
+        lac = lacache_run(dev, args.lacache_batch)
+        lac["frac_of_hbm_" + src] = lac["gbs"] / peaks["hbm_gbs"]
+        kernels["lacache_compact"] = lac
+
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(seed)
@@ -503,6 +556,9 @@ def main():
     ap.add_argument("--impl", choices=["kara", "reference"], default="kara")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-lacache", action="store_true",
+                    help="skip the LaCache ladder-compaction measurement (1 GPU only)")
+    ap.add_argument("--lacache-batch", type=int, default=8)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
