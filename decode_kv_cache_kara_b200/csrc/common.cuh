@@ -64,19 +64,23 @@ constexpr long long kWaitBudgetCycles = 4000000000LL;
 // Waits for the phase of `bar` with the given parity. Returns false (after reporting
 // KARA_ERR_TIMEOUT and raising *abort) when the budget runs out or another role already
 // aborted. `abort` lives in shared memory and is polled so every role unwinds together.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int32_t* status) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              int32_t* status, long long budget_cycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) {
+    if (clock64() - t0 > budget_cycles) {
       *abort = 1;
       report(status, KARA_ERR_TIMEOUT);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          int32_t* status) {
+  return mbar_wait_for(bar, parity, abort, status, kWaitBudgetCycles);
 }
 
 __device__ __forceinline__ void fence_barrier_init() {

@@ -83,6 +83,7 @@ _SIGNATURES = {
     "kara_status_str": ([_I], ctypes.c_char_p),
     "kara_version": ([], ctypes.c_char_p),
     "kara_last_error": ([], ctypes.c_char_p),
+    "kara_wait_probe": ([_I, _P, _P], _I),
 }
 
 
@@ -351,6 +352,15 @@ def lacache_compact(k_layers, v_layers, pool: PagedPool, span: int, overlap: int
     _check(lib().lacache_compact(arr, len(arr), ctypes.byref(ps), _ptr(seq_ids), r,
                                  ctypes.byref(prm), _ptr(ws), ws.numel(), _ptr(status),
                                  _stream(stream)), "lacache_compact")
+    return status
+
+
+def kara_wait_probe(wait_ms: int, status: torch.Tensor | None = None, device="cuda",
+                    stream=None) -> torch.Tensor:
+    """Runs the bounded-wait probe (a wait that times out after about `wait_ms`). Returns the
+    status tensor, which holds KARA_ERR_TIMEOUT once the stream completes."""
+    status = status if status is not None else new_status(torch.device(device))
+    _check(lib().kara_wait_probe(int(wait_ms), _ptr(status), _stream(stream)), "kara_wait_probe")
     return status
 
 

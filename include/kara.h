@@ -271,6 +271,19 @@ const char* kara_last_error(void);
 /* Library version string ("kara-b200 <major>.<minor>"). */
 const char* kara_version(void);
 
+/*
+ * kara_wait_probe - exercises the bounded-wait failure path on the device. The pages have no
+ * counterpart of it: it exists so that failure detection can be tested without a GPU fault.
+ *  One CTA; thread 0 of warp 0 waits on an mbarrier that nothing arrives on, with a budget of
+ *  about `wait_ms` milliseconds of SM clock, then reports KARA_ERR_TIMEOUT to dev_status and
+ *  raises the CTA's abort flag; thread 0 of warp 1 waits on a second such barrier with the
+ *  library's default budget (about 2 s) and must unwind through that flag. The kernel then
+ *  returns, and the context stays usable.
+ *  wait_ms     1 .. 2000 (host-checked, else KARA_ERR_INVALID_ARG).
+ *  dev_status  device int32, written on the device (first error wins).
+ */
+kara_status kara_wait_probe(int32_t wait_ms, int32_t* dev_status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

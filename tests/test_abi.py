@@ -54,6 +54,13 @@ def test_host_side_validation_returns_before_any_launch(lib_path):
     layers = (K._LayerKV * 8)()
     assert L.lacache_compact(layers, 8, ctypes.byref(pool), null, 1, ctypes.byref(prm), null, 0,
                              one, null) == K.ERR_INVALID_ARG
+    # the wait probe: budget outside 1..2000 ms, or no status buffer
+    assert L.kara_wait_probe(0, one, null) == K.ERR_INVALID_ARG
+    assert L.kara_wait_probe(2001, one, null) == K.ERR_INVALID_ARG
+    assert L.kara_wait_probe(100, null, null) == K.ERR_INVALID_ARG
+    # compaction window above KARA_MAX_WINDOW
+    assert L.kara_compact(layers, 1, ctypes.byref(pool), null, 1, 5000, 8, one, one, 1 << 20, one,
+                          null) == K.ERR_INVALID_ARG
 
 
 def test_workspace_sizes(lib_path):
