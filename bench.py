@@ -160,10 +160,20 @@ class Step:
         self.K = K
         self.wl = wl
         self.c = cache
-        self.pool = K.PagedPool.from_cache(cache)
         dev = cache["k"][0].device
-        self.saved = {k: cache[k].clone() for k in ("block_table", "ctx_len", "free_list",
-                                                     "free_top")}
+        # the pool bookkeeping as views into one int32 buffer, so that the per-step restore
+        # is a single copy
+        names = ("block_table", "ctx_len", "free_list", "free_top")
+        sizes = [cache[n].numel() for n in names]
+        self.book = torch.empty(sum(sizes), dtype=torch.int32, device=dev)
+        off = 0
+        for n, sz in zip(names, sizes):
+            view = self.book[off:off + sz].view(cache[n].shape)
+            view.copy_(cache[n])
+            cache[n] = view
+            off += sz
+        self.saved_book = self.book.clone()
+        self.pool = K.PagedPool.from_cache(cache)
         self.status = K.new_status(dev)
         r, hq = wl.batch, wl.hq
         self.scores = torch.empty((r, wl.hkv, wl.window), dtype=torch.float32, device=dev)
@@ -182,8 +192,7 @@ class Step:
         self.score_fused = fused
 
     def restore(self):
-        for k, t in self.saved.items():
-            self.c[k].copy_(t, non_blocking=True)
+        self.book.copy_(self.saved_book, non_blocking=True)
 
     def run(self, events=None, restore=True):
         K, wl, c = self.K, self.wl, self.c
