@@ -322,6 +322,14 @@ __device__ __forceinline__ void st_async_f2(uint32_t remote, float x, float y, u
       "f"(x), "f"(y), "r"(remote_bar)
       : "memory");
 }
+// Stores one float into another CTA's shared memory and counts its 4 bytes on that CTA's
+// mbarrier (both addresses from map_to_rank).
+__device__ __forceinline__ void st_async_f1(uint32_t remote, float x, uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote),
+      "r"(__float_as_uint(x)), "r"(remote_bar)
+      : "memory");
+}
 // mbarrier wait with cluster-scope acquire (data written by other CTAs of the cluster).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
