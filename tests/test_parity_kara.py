@@ -33,6 +33,11 @@ SCORE_CASES = {
                               run_hi=16, q_mode="neighbour", spare_blocks=8),
     "w16_ctx_eq_w": synth.Workload("w16", batch=3, layers=1, hq=2, hkv=1, head_dim=128,
                                    ctx_lo=16, ctx_hi=16, window=16, keep=1, spare_blocks=4),
+    # windows of 128 * c keys take the fused cluster kernel (c CTAs per cluster)
+    "g7_w512_ragged": LAYER.with_(batch=4, ctx_lo=520, ctx_hi=900, window=512, keep=102),
+    "d64_g4_w256": synth.Workload("d64_g4_w256", batch=3, layers=1, hq=8, hkv=2, head_dim=64,
+                                  ctx_lo=260, ctx_hi=400, window=256, keep=51, heavy_frac=0.05,
+                                  q_mode="neighbour", spare_blocks=8),
 }
 
 
@@ -61,10 +66,12 @@ def test_score_matches_oracle(name):
     assert np.allclose(sums, wl.window * wl.group, rtol=1e-4)
 
 
-def test_score_subset_of_sequences():
-    wl = SCORE_CASES["g7_ragged_unaligned"]
+@pytest.mark.parametrize("name", ["g7_ragged_unaligned", "g7_w512_ragged"])
+def test_score_subset_of_sequences(name):
+    wl = SCORE_CASES[name]
     cpu, dev = H.make(wl, 5)
     ids = [1, 3]
+    assert wl.batch > max(ids)
     pool = K.PagedPool.from_cache(dev)
     q = dev["q_win"][0][ids].contiguous()
     seq = torch.tensor(ids, dtype=torch.int32, device="cuda")
