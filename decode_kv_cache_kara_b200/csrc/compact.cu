@@ -80,6 +80,7 @@ struct PlanParams {
 };
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
   __shared__ int buf[33];
   __shared__ int err;
   __shared__ int carry_new, carry_old;
@@ -456,7 +457,7 @@ kara_status launch_compact(const CompactLaunch& L, cudaStream_t stream) {
   pp.k = L.k;
   pp.lacache = 0;
   pp.min_len = 0;
-  plan_kernel<<<1, kPlanThreads, 0, stream>>>(pp);
+  launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), 0, stream, pp);
   KaraGather g;
   g.layers = L.layers;
   g.block_table = L.block_table;
@@ -500,7 +501,7 @@ kara_status launch_lacache(const LacacheLaunch& L, cudaStream_t stream) {
   pp.k = L.budget;
   pp.lacache = 1;
   pp.min_len = L.sink + L.recent + r_max;
-  plan_kernel<<<1, kPlanThreads, 0, stream>>>(pp);
+  launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), 0, stream, pp);
   LadderGather g;
   g.layers = L.layers;
   g.block_table = L.block_table;

@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
   static_assert(G <= 8, "at most 8 query heads per KV head");
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
   constexpr int NCH = D / 64;                 // 64-channel chunks per row
   constexpr int KS = D / 16;                  // k-steps of S^T, m-tiles of O^T
   constexpr uint32_t kPage = page_bytes<D>();
@@ -484,7 +485,8 @@ kara_status launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensor
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  decode_stream_kernel<D, G><<<per_sm * sms, kDecThreads, smem, stream>>>(tk, tv, a);
+  launch_pdl(decode_stream_kernel<D, G>, dim3(per_sm * sms), dim3(kDecThreads), smem, stream, tk,
+             tv, a);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.B * a.Hq);
   cfg.blockDim = dim3(32 * kCombWarps);

@@ -10,6 +10,26 @@
 
 namespace kara {
 
+// Launches `kernel` as a programmatic dependent of the previous kernel in `stream`: it may
+// start while that kernel finishes, and it must execute griddepcontrol.wait (which returns once
+// the previous kernel has completed and its memory is visible) before it touches memory.
+// Every library kernel launched this way does so at entry, so stream order holds as usual.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // 4-D bf16 tensor map (innermost dimension first), 128-byte swizzle, box {64, 1, rows, 1}.
 // Defined in score.cu.
 bool make_bf16_map_4d(CUtensorMap* map, const void* base, const uint64_t dims[4],

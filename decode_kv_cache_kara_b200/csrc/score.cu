@@ -177,6 +177,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
   constexpr int NCH = D / 64;
   constexpr uint32_t kQBytes = NCH * kQRows1 * kRowBytes;
   constexpr uint32_t kKBytes = NCH * kKRows1 * kRowBytes;
@@ -453,6 +454,7 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
 // Merge of the per-chunk partial log-sum-exps: lse = log2(sum_c 2^lse_c), one thread per query.
 // ----------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) score_lse_merge_kernel(const ScoreArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
   const size_t total = static_cast<size_t>(a.R) * a.Hq * a.Wp;
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
@@ -483,6 +485,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
   constexpr int NCH = D / 64;
   constexpr uint32_t kABytes = NCH * kKRows2 * kRowBytes;
   constexpr uint32_t kBBytes = NCH * kQRows2 * kRowBytes;
@@ -833,6 +836,7 @@ template <int D, int CL>
 __global__ void __launch_bounds__(kFThreads, 1)
 score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
   using L = FusedSmem<D>;
   constexpr int NCH = L::NCH;
   constexpr uint32_t kPageBytes = 16 * kRowBytes;
@@ -1330,19 +1334,24 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
     cfg.blockDim = dim3(kFThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // kernel waits at entry
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (max_clusters[CL] == 0) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
       cfg.gridDim = dim3(CL * (sm_count() / CL));
+      cfg.numAttrs = 1;                    // the query sees the cluster shape only
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+      const cudaError_t qe = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+      cfg.numAttrs = 2;
+      if (qe != cudaSuccess || n <= 0) {
         check_launch("score_fused_kernel occupancy");
         return KARA_ERR_CUDA;
       }
@@ -1371,7 +1380,8 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   const int KT = ((L.W + 15 + 15) / 16 + 7) / 8;   // at most this many key tiles per (r, g)
   const int tiles2 = L.R * L.Hkv * KT;
   const int sms = sm_count();
-  score_rowstats_kernel<D><<<min(tiles1, sms), kThreads, rowstats_smem<D>(), stream>>>(tq1, tk, a);
+  launch_pdl(score_rowstats_kernel<D>, dim3(min(tiles1, sms)), dim3(kThreads), rowstats_smem<D>(),
+             stream, tq1, tk, a);
   if (check_launch("score_rowstats_kernel") != KARA_OK) {
     describe_kernel("score_rowstats_kernel", reinterpret_cast<const void*>(score_rowstats_kernel<D>),
                     kThreads, rowstats_smem<D>());
@@ -1380,10 +1390,11 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   {
     const size_t n = static_cast<size_t>(L.R) * L.Hq * score_lse_stride(L.W);
     const int blocks = static_cast<int>(std::min<size_t>((n + 255) / 256, static_cast<size_t>(sms) * 8));
-    score_lse_merge_kernel<<<blocks, 256, 0, stream>>>(a);
+    launch_pdl(score_lse_merge_kernel, dim3(blocks), dim3(256), 0, stream, a);
     if (check_launch("score_lse_merge_kernel") != KARA_OK) return KARA_ERR_CUDA;
   }
-  score_colsum_kernel<D><<<min(tiles2, sms), kThreads, colsum_smem<D>(), stream>>>(tq2, tk, a);
+  launch_pdl(score_colsum_kernel<D>, dim3(min(tiles2, sms)), dim3(kThreads), colsum_smem<D>(),
+             stream, tq2, tk, a);
   if (check_launch("score_colsum_kernel") != KARA_OK) {
     describe_kernel("score_colsum_kernel", reinterpret_cast<const void*>(score_colsum_kernel<D>),
                     kThreads, colsum_smem<D>());

@@ -130,6 +130,7 @@ __device__ void block_compact_write(const uint8_t* flag, int W, int E, int32_t* 
 
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(const float* __restrict__ scores, int W, int k, int32_t* __restrict__ sel) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
   extern __shared__ __align__(16) uint8_t smem[];
   SelectSmem* ss = reinterpret_cast<SelectSmem*>(smem);
   uint32_t* key = reinterpret_cast<uint32_t*>(smem + sizeof(SelectSmem));
@@ -151,6 +152,7 @@ select_kernel(const float* __restrict__ scores, int W, int k, int32_t* __restric
 __global__ void __launch_bounds__(kSelThreads)
 token2chunk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ sel, int W,
                    int k, int num_anchors, int gap_limit, int widen, int32_t* __restrict__ keep) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
   extern __shared__ __align__(16) uint8_t smem[];
   SelectSmem* ss = reinterpret_cast<SelectSmem*>(smem);
   uint32_t* key = reinterpret_cast<uint32_t*>(smem + sizeof(SelectSmem));
@@ -271,7 +273,8 @@ size_t t2c_smem(int W) { return sizeof(SelectSmem) + static_cast<size_t>(W) * 14
 kara_status launch_select(const float* scores, int rows, int W, int k, int32_t* sel,
                           cudaStream_t stream) {
   if (rows == 0) return KARA_OK;
-  select_kernel<<<rows, kSelThreads, select_smem(W), stream>>>(scores, W, k, sel);
+  launch_pdl(select_kernel, dim3(rows), dim3(kSelThreads), select_smem(W), stream, scores, W, k,
+             sel);
   return check_launch(__func__);
 }
 
@@ -279,8 +282,8 @@ kara_status launch_token2chunk(const float* scores, const int32_t* sel, int rows
                                int num_anchors, int gap_limit, int widen, int32_t* keep,
                                cudaStream_t stream) {
   if (rows == 0) return KARA_OK;
-  token2chunk_kernel<<<rows, kSelThreads, t2c_smem(W), stream>>>(scores, sel, W, k, num_anchors,
-                                                                 gap_limit, widen, keep);
+  launch_pdl(token2chunk_kernel, dim3(rows), dim3(kSelThreads), t2c_smem(W), stream, scores, sel,
+             W, k, num_anchors, gap_limit, widen, keep);
   return check_launch(__func__);
 }
 
