@@ -769,7 +769,9 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
 constexpr int kFEpiWarps = 16;                    // two teams of 8, tiles alternate between them
 constexpr int kFParts = 2;                        // per team: 2 warps per TMEM lane quadrant
 constexpr int kFPartKeys = 128 / kFParts;         // 64 keys per warp
-constexpr int kFThreads = 96 + 32 * kFEpiWarps;   // TMA, S issuer, column-sum issuer, epilogue
+// warps 0-3: TMA producer, S issuer, column-sum issuer, and a spare, so that each of the four
+// SM sub-partitions holds one such warp beside its four epilogue warps
+constexpr int kFThreads = 128 + 32 * kFEpiWarps;
 constexpr int kFEpiThreads = 32 * kFEpiWarps;
 constexpr int kFKeys = 128;            // window keys owned per CTA
 constexpr int kFKRows = 144;           // key rows loaded per CTA (9 pages)
@@ -890,11 +892,11 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp >= 3) {
+  if (warp >= 4) {
     // the weight operands' unused rows (n = 3 * parts .. 15) stay zero
     constexpr int kZ = 16 - 3 * kFParts;
     static_assert(kZ * 8 * 2 * 2 <= kFEpiThreads * 8, "zero fill");
-    const int t = threadIdx.x - 96;
+    const int t = threadIdx.x - 128;
     for (int i = t; i < 2 * 2 * kZ * 8; i += kFEpiThreads) {
       const int buf = i / (16 * kZ), rem = i % (16 * kZ), kc = rem / (8 * kZ);
       const int n = 3 * kFParts + (rem % (8 * kZ)) / 8, c = rem % 8;
@@ -1036,11 +1038,11 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!ok) break;
       }
     }
-  } else {
+  } else if (warp >= 4) {
     // ---- epilogue: two teams of 8 warps take alternate tiles (team = tile parity), so that
     // one team's exponentials overlap the other's exchange and weights. In a team, warp
     // (quad, part) owns TMEM lane quadrant `quad` and keys [64 part, 64 part + 64). ----
-    const int e = warp - 3;
+    const int e = warp - 4;
     const int team = e >> 3;
     const int quad = warp & 3;
     const int part = (e & 7) >> 2;
