@@ -160,23 +160,6 @@ __device__ __forceinline__ void reg_fence(float* v) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 // 16 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   uint32_t r[16];
@@ -251,11 +234,6 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
   return bits_f2(r);
 }
-__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
-  return bits_f2(r);
-}
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
@@ -281,11 +259,6 @@ __device__ __forceinline__ float2 ex2_fma2(float2 x) {
   p = ffma2(p, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
   return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
-// Both bf16 halves of a packed word as an fp32 pair (exact).
-__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
-  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
 // ---------------------------------------------------------------------------------------
@@ -320,14 +293,6 @@ __device__ __forceinline__ void st_async_f2(uint32_t remote, float x, float y, u
       "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
           remote),
       "f"(x), "f"(y), "r"(remote_bar)
-      : "memory");
-}
-// Stores one float into another CTA's shared memory and counts its 4 bytes on that CTA's
-// mbarrier (both addresses from map_to_rank).
-__device__ __forceinline__ void st_async_f1(uint32_t remote, float x, uint32_t remote_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote),
-      "r"(__float_as_uint(x)), "r"(remote_bar)
       : "memory");
 }
 // mbarrier wait with cluster-scope acquire (data written by other CTAs of the cluster).

@@ -39,14 +39,7 @@ namespace kara {
 
 namespace {
 
-#ifndef KARA_SCORE_EPI_WARPS
-#define KARA_SCORE_EPI_WARPS 8
-#endif
-// 1: packed fp32x2 arithmetic in the epilogues; 0: scalar
-#ifndef KARA_SCORE_PACKED
-#define KARA_SCORE_PACKED 1
-#endif
-constexpr int kEpiWarps = KARA_SCORE_EPI_WARPS;  // a multiple of 4: warps per TMEM lane quadrant
+constexpr int kEpiWarps = 8;                     // a multiple of 4: warps per TMEM lane quadrant
 constexpr int kParts = kEpiWarps / 4;            // column parts of each 256-column accumulator
 constexpr int kThreads = 64 + 32 * kEpiWarps;    // warp 0: TMA, warp 1: UMMA + TMEM, rest: epilogue
 constexpr int kEpiThreads = 32 * kEpiWarps;
@@ -364,7 +357,6 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
             const float cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             if (cmax == -INFINITY) return;
             const float m_new = fmaxf(m, cmax * a.cs);
-#if KARA_SCORE_PACKED
             const float2 nm2 = make_float2(-m_new, -m_new);
             float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -376,15 +368,6 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             const float2 acc = fadd2(acc0, acc1);
             l = l * ex2(m - m_new) + (acc.x + acc.y);
-#else
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float x = fmaf(v[i], a.cs, -m_new);
-              acc[i & 3] += ((i & 7) == 7) ? ex2_fma(x) : ex2(x);
-            }
-            l = l * ex2(m - m_new) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
-#endif
             m = m_new;
           };
           auto issue = [&](float (&v)[32], int j) {
@@ -669,7 +652,6 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
             tmem_ld16(col0 + 32 * j + 16, v + 16);
           };
           auto process = [&](const float (&v)[32], int j) {
-#if KARA_SCORE_PACKED
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
               const float4 nl = *reinterpret_cast<const float4*>(lh + 32 * j + i);
@@ -678,18 +660,6 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
               acc0 = fadd2(acc0, exp2_pair(x0, (i >> 1) & 3));
               acc1 = fadd2(acc1, exp2_pair(x1, ((i >> 1) + 1) & 3));
             }
-#else
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const float4 nl = *reinterpret_cast<const float4*>(lh + 32 * j + i);
-              const float x0 = fmaf(v[i], a.cs, nl.x), x1 = fmaf(v[i + 1], a.cs, nl.y);
-              const float x2 = fmaf(v[i + 2], a.cs, nl.z), x3 = fmaf(v[i + 3], a.cs, nl.w);
-              acc0.x += ex2(x0);
-              acc0.y += ex2(x1);
-              acc1.x += ex2(x2);
-              acc1.y += ((i & 4) != 0) ? ex2_fma(x3) : ex2(x3);
-            }
-#endif
           };
           float va[32], vb[32];
           issue(va, 0);
