@@ -206,6 +206,11 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // On the FMA pipe, so that part of the exponentials leaves the SFU: x = n + f with
 // n = round-to-nearest(x) (adding and subtracting 1.5 * 2^23 leaves n in the low mantissa
@@ -293,6 +298,12 @@ __device__ __forceinline__ void st_async_f2(uint32_t remote, float x, float y, u
       "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
           remote),
       "f"(x), "f"(y), "r"(remote_bar)
+      : "memory");
+}
+__device__ __forceinline__ void st_async_f32(uint32_t remote, float x, uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote),
+      "r"(__float_as_uint(x)), "r"(remote_bar)
       : "memory");
 }
 // mbarrier wait with cluster-scope acquire (data written by other CTAs of the cluster).

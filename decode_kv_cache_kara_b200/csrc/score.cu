@@ -716,25 +716,29 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
 // ----------------------------------------------------------------------------------------
 // Fused scoring: one exponential per score, on a cluster of CL = W / 128 CTAs.
 //
-// Work items are (r, g, hl): query head g*G + hl of a valid sequence r against the window
-// keys of KV head g; all CTAs of a cluster take the same items, CTA `rank` owns the 128 window
-// keys [start + 128 rank, start + 128 rank + 128). Per 128-query tile each CTA
+// Work items are (r, g): the G query heads of KV head g of a valid sequence r against the
+// window keys of that KV head (G * W / 128 query tiles); all CTAs of a cluster take the same
+// items, CTA `rank` owns the 128 window keys [start + 128 rank, start + 128 rank + 128). Per
+// 128-query tile each CTA
 //   1. computes S = Q K^T over its keys (UMMA M = 128 queries, N = 144 key rows: the 9 pages
 //      that cover its 128 keys at any slot offset; only the owned columns are read);
 //   2. in the epilogue (8 warps: a TMEM lane quadrant and 64 owned keys each) takes the row
 //      max m_p over its 64 keys, P' = 2^(s*c - m_p + 15) and the row sum l_p, and stores P' as
 //      fp16 in shared memory, MN-major (rows along K) for the next product;
-//   3. combines the two parts of each row and sends (m, l) of its 128 keys to every CTA of the
-//      cluster (st.async into their shared memory, counted on their mbarrier);
-//   4. once all CL partials of a row are in: M = max m, L = sum l 2^(m - M), and the row
+//   3. combines the two parts of each row and sends the partial log-sum-exp of its 128 keys,
+//      lse = m + log2(l), to every CTA of the cluster (st.async into their shared memory,
+//      counted on their mbarrier);
+//   4. once all CL partials of a row are in: M = max lse, L = sum 2^(lse - M), and the row
 //      weight of part p is w = 2^(m_p - M + 15) / L (so that P' w = 2^15 softmax); w goes to
 //      fp16 as three B columns (w1 + w2 + 2^-24 w3, exact to about 2^-36);
 //   5. D (128 keys x 16) += P'^T W: the column sums of the tile's softmax rows on the tensor
 //      cores (UMMA M = 128 keys, K = 128 queries, N = 16), accumulated over the item's tiles.
-// Step 4 of a tile runs in the epilogue after steps 1-3 of the next tile, so the exchange
-// latency hides behind a tile of work; P', the weights and the exchange slots are multi-
-// buffered for that. After the item's last tile, D (times 2^-15) gives the head's per-key
-// scores; a second kernel sums the G heads.
+// Two teams of epilogue warps take alternate tiles, so one team's exponentials overlap the
+// other's exchange and weights. P' and the weights have three buffers, taken round-robin by
+// tile: a team's next tile writes the buffer of the other team's previous tile, so the wait
+// for a buffer (exchange, weights and column-sum product of its last tile) gets one more tile
+// of slack than with a buffer per team. After the item's last tile, D (times 2^-15) holds the
+// per-key scores summed over the item's G heads.
 // ----------------------------------------------------------------------------------------
 constexpr int kFEpiWarps = 16;                    // two teams of 8, tiles alternate between them
 constexpr int kFParts = 2;                        // per team: 2 warps per TMEM lane quadrant
@@ -747,8 +751,11 @@ constexpr int kFKeys = 128;            // window keys owned per CTA
 constexpr int kFKRows = 144;           // key rows loaded per CTA (9 pages)
 constexpr int kFQRows = 128;           // queries per tile
 constexpr int kFMaxCluster = 8;
-constexpr int kFXStages = 4;           // exchange slots (a peer sends tile T only after every
-                                       // CTA has read its partials of tile T - 4)
+constexpr int kFPBufs = 3;             // P' and weight buffers, tile T in buffer T mod 3
+constexpr int kFQSlots = 3;            // query ring slots of one 64-channel chunk each
+constexpr int kFXStages = 5;           // exchange slots: a peer sends tile T + 5 only after this
+                                       // CTA's exponentials of tile T + 2, which its team starts
+                                       // after reading the partials of tile T
 constexpr uint32_t kFEpiBarrier = 1;
 constexpr uint32_t kFSCols = 256;      // TMEM column stride of the two S buffers
 constexpr uint32_t kFDCol = 160;       // TMEM columns of the two D buffers: 160, 176
@@ -781,21 +788,21 @@ struct FusedSmem {
   static constexpr uint32_t kKChunk = kFKRows * kRowBytes;     // one 64-channel chunk of K
   static constexpr uint32_t kKBytes = NCH * kKChunk;
   static constexpr uint32_t kQChunk = kFQRows * kRowBytes;
-  static constexpr uint32_t kQBytes = NCH * kQChunk;
   static constexpr uint32_t kPAtom = 64 * kFQRows * 2;         // 64 keys x 128 queries, fp16
   static constexpr uint32_t kPBytes = 2 * kPAtom;
   static constexpr uint32_t kWBytes = 2 * 16 * kRowBytes;      // [k chunk][16 n rows][128 B]
-  static constexpr uint32_t kXBytes = kFXStages * kFMaxCluster * kFQRows * 8;
+  static constexpr uint32_t kXBytes = kFXStages * kFMaxCluster * kFQRows * 4;
   static constexpr uint32_t k_off = 0;
-  static constexpr uint32_t q_off = k_off + kKBytes;
-  static constexpr uint32_t p_off = q_off + 2 * kQBytes;
-  static constexpr uint32_t w_off = p_off + 2 * kPBytes;
-  static constexpr uint32_t x_off = w_off + 2 * kWBytes;
-  static constexpr uint32_t comb_off = x_off + kXBytes;         // [team][part][128] float2
-  static constexpr uint32_t bar_off = comb_off + 2 * 2 * kFQRows * 8;
-  static constexpr uint32_t kBars = 2 + 2 * 9 + kFXStages;
+  static constexpr uint32_t q_off = k_off + kKBytes;            // [slot] one chunk each
+  static constexpr uint32_t p_off = q_off + kFQSlots * kQChunk;
+  static constexpr uint32_t w_off = p_off + kFPBufs * kPBytes;
+  static constexpr uint32_t x_off = w_off + kFPBufs * kWBytes;
+  static constexpr uint32_t comb_off = x_off + kXBytes;  // [team][tile parity][part][128] float2
+  static constexpr uint32_t bar_off = comb_off + 2 * 2 * 2 * kFQRows * 8;
+  static constexpr uint32_t kBars = 2 + 2 * kFQSlots + 2 * 2 + 3 * kFPBufs + 2 * 2 + kFXStages;
   static constexpr uint32_t end = bar_off + kBars * 8 + 16;
   static constexpr size_t bytes = 1024 + end;
+  static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 // Byte offset of (n, k) in a K-major 128-byte-swizzled 16-row B operand [k chunk][n][128 B].
@@ -820,21 +827,21 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint8_t* q_buf = smem + L::q_off;
   uint8_t* p_buf = smem + L::p_off;
   uint8_t* w_buf = smem + L::w_off;
-  float2* x_buf = reinterpret_cast<float2*>(smem + L::x_off);     // [stage][src rank][row]
-  float2* comb = reinterpret_cast<float2*>(smem + L::comb_off);   // [team][part][row]: (m, l)
+  float* x_buf = reinterpret_cast<float*>(smem + L::x_off);       // [stage][src rank][row]: lse
+  float2* comb = reinterpret_cast<float2*>(smem + L::comb_off);   // [team][par][part][row]: (m, l)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bar_off);
   uint64_t* k_full = bars;
   uint64_t* k_empty = bars + 1;
-  uint64_t* q_full = bars + 2;     // [2]
-  uint64_t* q_empty = bars + 4;
-  uint64_t* s_full = bars + 6;
-  uint64_t* s_empty = bars + 8;
-  uint64_t* p_full = bars + 10;
-  uint64_t* w_full = bars + 12;
-  uint64_t* p_empty = bars + 14;
-  uint64_t* d_full = bars + 16;
-  uint64_t* d_empty = bars + 18;
-  uint64_t* x_full = bars + 20;    // [kFXStages]
+  uint64_t* q_full = bars + 2;                     // [kFQSlots]
+  uint64_t* q_empty = q_full + kFQSlots;
+  uint64_t* s_full = q_empty + kFQSlots;           // [2]
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* p_full = s_empty + 2;                  // [kFPBufs]
+  uint64_t* w_full = p_full + kFPBufs;
+  uint64_t* p_empty = w_full + kFPBufs;
+  uint64_t* d_full = p_empty + kFPBufs;            // [2]
+  uint64_t* d_empty = d_full + 2;
+  uint64_t* x_full = d_empty + 2;                  // [kFXStages]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -847,14 +854,18 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (threadIdx.x == 0) {
     mbar_init(k_full, 1);
     mbar_init(k_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kFQSlots; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], kFEpiThreads / 2);     // one team per tile
-      mbar_init(&p_full[i], kFEpiThreads / 2);
+    }
+    for (int i = 0; i < kFPBufs; ++i) {
+      mbar_init(&p_full[i], kFEpiThreads / 2);      // one team per tile
       mbar_init(&w_full[i], kFEpiThreads / 4);      // the team's part-1 threads
       mbar_init(&p_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], kFEpiThreads / 2);
       mbar_init(&d_full[i], 1);
       mbar_init(&d_empty[i], kFEpiThreads / 2);
     }
@@ -865,9 +876,8 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (warp >= 4) {
     // the weight operands' unused rows (n = 3 * parts .. 15) stay zero
     constexpr int kZ = 16 - 3 * kFParts;
-    static_assert(kZ * 8 * 2 * 2 <= kFEpiThreads * 8, "zero fill");
     const int t = threadIdx.x - 128;
-    for (int i = t; i < 2 * 2 * kZ * 8; i += kFEpiThreads) {
+    for (int i = t; i < kFPBufs * 2 * kZ * 8; i += kFEpiThreads) {
       const int buf = i / (16 * kZ), rem = i % (16 * kZ), kc = rem / (8 * kZ);
       const int n = 3 * kFParts + (rem % (8 * kZ)) / 8, c = rem % 8;
       *reinterpret_cast<uint4*>(w_buf + buf * L::kWBytes + kc * 2048 + n * 128 + c * 16) =
@@ -899,7 +909,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     const int TPI = a.G * CL;
     ItemCursor cur;
-    int g = 0, T = 0;
+    int g = 0, C = 0;   // query chunks issued
     bool have = cur.seek(a, cid, g);
     auto page_ids = [&](const SeqInfo& s, int& npg) {
       const int key0 = s.start + static_cast<int>(rank) * kFKeys;
@@ -928,17 +938,22 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (have) my_blk = page_ids(cur.s, npg);
       bool stop = false;
       if (lane == 0) {
-        for (int tq = 0; tq < TPI; ++tq, ++T) {
-          const int st = T & 1;
+        for (int tq = 0; tq < TPI && !stop; ++tq) {
           const int h = gi * a.G + tq / CL, qt = tq % CL;
-          if (!mbar_wait(&q_empty[st], ((T >> 1) & 1) ^ 1, abort_flag, a.status)) { stop = true; break; }
-          mbar_expect_tx(&q_full[st], L::kQBytes);
-          for (int ch = 0; ch < NCH; ++ch)
-            tma_load_4d(q_buf + st * L::kQBytes + ch * L::kQChunk, &tm_q, &q_full[st], ch * 64, h,
+          for (int ch = 0; ch < NCH; ++ch) {   // chunk C of the ring: slot C mod 3
+            const int slot = C % kFQSlots;
+            if (!mbar_wait(&q_empty[slot], ((C / kFQSlots) & 1) ^ 1, abort_flag, a.status)) {
+              stop = true;
+              break;
+            }
+            mbar_expect_tx(&q_full[slot], L::kQChunk);
+            tma_load_4d(q_buf + slot * L::kQChunk, &tm_q, &q_full[slot], ch * 64, h,
                         qt * kFQRows, r);
+            ++C;
+          }
         }
       }
-      T = __shfl_sync(0xffffffffu, T, 0);
+      C = __shfl_sync(0xffffffffu, C, 0);
       if (__shfl_sync(0xffffffffu, stop ? 1 : 0, 0)) break;
     }
   } else if (warp == 1) {
@@ -947,27 +962,30 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t idesc_s = idesc_bf16_f32(128, kFKRows);
       const int TPI = a.G * CL;
       ItemCursor cur;
-      int g, T = 0, I = 0;
+      int g, T = 0, I = 0, C = 0;   // tiles, items, query chunks
       bool ok = true;
       for (int it = cid; ok && !*abort_flag && cur.seek(a, it, g); it += ncl, ++I) {
         if (!mbar_wait(k_full, I & 1, abort_flag, a.status)) break;
         const uint32_t k_addr = smem_u32(k_buf);
-        for (int tq = 0; tq < TPI; ++tq, ++T) {
+        for (int tq = 0; tq < TPI && ok; ++tq, ++T) {
           const int st = T & 1;
           const uint32_t ph = (T >> 1) & 1;
-          if (!mbar_wait(&q_full[st], ph, abort_flag, a.status) ||
-              !mbar_wait(&s_empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t q_addr = smem_u32(q_buf + st * L::kQBytes);
+          if (!mbar_wait(&s_empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
           const uint32_t d_tmem = tmem_base + st * kFSCols;
+          for (int ch = 0; ch < NCH; ++ch, ++C) {
+            const int slot = C % kFQSlots;
+            if (!mbar_wait(&q_full[slot], (C / kFQSlots) & 1, abort_flag, a.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t q_addr = smem_u32(q_buf + slot * L::kQChunk);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk & 3) * 32;
-            const uint64_t ad = sw128_kmajor_desc(q_addr + (kk >> 2) * L::kQChunk + off);
-            const uint64_t bd = sw128_kmajor_desc(k_addr + (kk >> 2) * L::kKChunk + off);
-            umma_bf16(d_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sw128_kmajor_desc(q_addr + kk * 32);
+              const uint64_t bd = sw128_kmajor_desc(k_addr + ch * L::kKChunk + kk * 32);
+              umma_bf16(d_tmem, ad, bd, idesc_s, (ch > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&q_empty[slot]);
           }
-          umma_commit(&q_empty[st]);
+          if (!ok) break;
           umma_commit(&s_full[st]);
           if (tq == TPI - 1) umma_commit(k_empty);
         }
@@ -983,8 +1001,8 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (int it = cid; !*abort_flag && cur.seek(a, it, g); it += ncl, ++Ic) {
         bool ok = true;
         for (int qt = 0; qt < TPI; ++qt, ++Tc) {
-          const int st = Tc & 1;
-          const uint32_t ph = (Tc >> 1) & 1;
+          const int st = Tc % kFPBufs;
+          const uint32_t ph = (Tc / kFPBufs) & 1;
           if (!mbar_wait(&p_full[st], ph, abort_flag, a.status) ||
               !mbar_wait(&w_full[st], ph, abort_flag, a.status) ||
               (qt == 0 &&
@@ -1036,9 +1054,12 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     int g = 0, I = 0, tq = team;          // item index and tile within the item (no divisions:
     while (tq >= TPI) { tq -= TPI; ++I; }  // they would queue behind the exponentials)
     bool have = cur.seek(a, cid + I * ncl, g);
+    // running T mod 3 / T div 3 (P' and weight buffers) and T mod 5 / T div 5 (exchange slots)
+    int pb = team, pq = 0, xs = team, xq = 0;
     for (int T = team; have; T += 2) {
-      const int st = T & 1;     // = team: S, P and weight buffers
+      const int st = T & 1;     // = team: S buffer
       const uint32_t ph = (T >> 1) & 1;
+      const uint32_t pph = pq & 1;
       const uint32_t scol = lane_base + st * kFSCols +
                             ((cur.s.start + static_cast<int>(rank) * kFKeys) % 16) + part * kFPartKeys;
       // (1) row max over this warp's 64 keys (first pass over TMEM)
@@ -1063,13 +1084,13 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
           mm = fmaxf(fmax3(m0, m1, m2), m3);
         }
         mx = mm * a.cs;
-        wait_cta(&p_empty[st], ph ^ 1);
+        wait_cta(&p_empty[pb], pph ^ 1);
       }
       // (2) P' = 2^(s c - m + 15) as fp16 in shared memory (second pass), and the row sum
       if (!aborted) {
         const float2 nb2 = make_float2(15.f - mx, 15.f - mx);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-        uint8_t* prow = p_buf + st * L::kPBytes + part * L::kPAtom + (row >> 3) * 1024 +
+        uint8_t* prow = p_buf + pb * L::kPBytes + part * L::kPAtom + (row >> 3) * 1024 +
                         (row & 7) * 128;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -1104,41 +1125,42 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         l = (acc0.x + acc0.y) + (acc1.x + acc1.y);
         fence_proxy_async();
-        mbar_arrive(&p_full[st]);
+        mbar_arrive(&p_full[pb]);
       }
-      // (3) the CTA's (m, l) of each row to every CTA of the cluster
-      const int xs = T % kFXStages;
-      if ((e & 7) == 0 && lane == 0) mbar_expect_tx(&x_full[xs], CL * kFQRows * 8);
-      float2* cb = comb + team * 2 * kFQRows;
+      // (3) the CTA's partial log-sum-exp of each row to every CTA of the cluster
+      if ((e & 7) == 0 && lane == 0) mbar_expect_tx(&x_full[xs], CL * kFQRows * 4);
+      // two halves by the team's tile parity: part 0 rewrites a half only after the named
+      // barrier of the team's next tile, which part 1 reaches after reading it for this one
+      float2* cb = comb + (team * 2 + static_cast<int>(ph)) * 2 * kFQRows;
       cb[part * kFQRows + row] = make_float2(mx, l);
       named_barrier(kFEpiBarrier + team * 4 + quad, 64);   // the two warps sharing these rows
       if (part == 0 && !aborted) {
         const float2 o = cb[kFQRows + row];
         const float M = fmaxf(mx, o.x);
-        const float Lc = l * ex2(mx - M) + o.y * ex2(o.x - M);
-        const uint32_t slot = x_buf_u32 + ((xs * kFMaxCluster + rank) * kFQRows + row) * 8;
+        const float lse = M + lg2(l * ex2(mx - M) + o.y * ex2(o.x - M));
+        const uint32_t slot = x_buf_u32 + ((xs * kFMaxCluster + rank) * kFQRows + row) * 4;
         const uint32_t xb = x_full_u32 + xs * 8;
 #pragma unroll
-        for (int c = 0; c < CL; ++c) st_async_f2(map_to_rank(slot, c), M, Lc, map_to_rank(xb, c));
+        for (int c = 0; c < CL; ++c) st_async_f32(map_to_rank(slot, c), lse, map_to_rank(xb, c));
       }
       // (4) meanwhile, once every CTA's partials are in, the row's thread of part 1 writes the
       // weights of both parts, w_p = 2^(m_p - M + 15) / L, as three fp16 columns each of the B
-      // operand (FMA-pipe exponentials: the SFU is busy with the other team's tile)
-      if (part == 1) wait_cluster(&x_full[xs], (T / kFXStages) & 1);
+      // operand
+      if (part == 1) wait_cluster(&x_full[xs], xq & 1);
       if (part == 1 && !aborted) {
-        const float2* xr = x_buf + xs * kFMaxCluster * kFQRows + row;
-        float2 xv[CL];
+        const float* xr = x_buf + xs * kFMaxCluster * kFQRows + row;
+        float xv[CL];
 #pragma unroll
         for (int c = 0; c < CL; ++c) xv[c] = xr[c * kFQRows];
-        float M = xv[0].x;
+        float M = xv[0];
 #pragma unroll
-        for (int c = 1; c < CL; ++c) M = fmaxf(M, xv[c].x);
+        for (int c = 1; c < CL; ++c) M = fmaxf(M, xv[c]);
         float Lsum = 0.f;
 #pragma unroll
-        for (int c = 0; c < CL; ++c) Lsum += xv[c].y * ex2(xv[c].x - M);
+        for (int c = 0; c < CL; ++c) Lsum += ex2(xv[c] - M);
         const float inv = 1.f / Lsum;
         const float m_part0 = cb[row].x;
-        uint8_t* wb = w_buf + st * L::kWBytes;
+        uint8_t* wb = w_buf + pb * L::kWBytes;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const float w = ex2((q == 0 ? m_part0 : mx) - M + 15.f) * inv;
@@ -1152,7 +1174,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
           *reinterpret_cast<__half*>(wb + w_offset(3 * q + 2, row)) = w3;
         }
         fence_proxy_async();
-        mbar_arrive(&w_full[st]);
+        mbar_arrive(&w_full[pb]);
       }
       // (5) the item's last tile: the per-key sums over all G heads, read by this team
       if (tq == TPI - 1) {
@@ -1172,6 +1194,10 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
           mbar_arrive(&d_empty[I & 1]);
         }
       }
+      pb += 2;
+      if (pb >= kFPBufs) { pb -= kFPBufs; ++pq; }
+      xs += 2;
+      if (xs >= kFXStages) { xs -= kFXStages; ++xq; }
       tq += 2;
       if (tq >= TPI) {
         tq -= TPI;
