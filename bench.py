@@ -185,11 +185,10 @@ class Step:
                  K.kara_workspace_bytes(K.OP_DECODE, self.pool, 0, 0, hq, 0))
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
         self.na = K.anchors_for(wl.anchor_frac, wl.keep)
-        # scoring: the fused cluster kernel for windows of 128/256/512/1024 keys, else two
-        # passes and a merge; select; Token2Chunk; compaction plan + gather; decode + combine
-        fused = wl.window in (128, 256, 512, 1024)
-        self.launches_per_step = (1 if fused else 3) + 1 + 1 + 2 + 2
-        self.score_fused = fused
+        # scoring: the fused cluster kernel for windows of 128/256/512/1024 keys (plus the
+        # split-item sum when a cluster range ends inside an item), else two passes and a
+        # merge; select; Token2Chunk; compaction plan + gather; decode + combine
+        self.score_fused = wl.window in (128, 256, 512, 1024)
 
     def restore(self):
         self.book.copy_(self.saved_book, non_blocking=True)
@@ -399,10 +398,12 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    launches0 = K.kara_launch_count()
     t0.record()
     for i in range(args.steps):
         step.run(ev[i])
     t1.record()
+    launches = K.kara_launch_count() - launches0
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -498,7 +499,7 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
         "e2e": {"value": tokens_step / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                 "d2h_bytes_per_step": e2e["d2h_bytes_per_step"], "ms_per_step": e2e_ms},
-        "gpu_launches": step.launches_per_step * args.steps,
+        "gpu_launches": launches,
         "clocks": clocks,
     }
     return line

@@ -1,5 +1,6 @@
 // C-ABI entry points of libkara: host-side argument checks, workspace carving, launches.
 // Semantics of every call are documented in include/kara.h.
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -12,6 +13,7 @@ using namespace kara;
 namespace {
 
 thread_local char g_last_error[512] = "";
+std::atomic<uint64_t> g_launches{0};
 
 }  // namespace
 
@@ -19,6 +21,10 @@ namespace kara {
 
 void set_last_error(const char* where, const char* what) {
   std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, what);
+}
+
+void count_launch(cudaError_t err) {
+  if (err == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
 }
 
 kara_status check_launch(const char* where) {
@@ -86,6 +92,8 @@ const char* kara_status_str(int32_t status) {
 const char* kara_version(void) { return "kara-b200 0.1"; }
 
 const char* kara_last_error(void) { return g_last_error; }
+
+uint64_t kara_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 size_t kara_workspace_bytes(kara_op op, const kara_pool* pool, int32_t num_seqs, int32_t window,
                             int32_t num_q_heads, int32_t k_or_budget) {

@@ -423,7 +423,7 @@ void launch_dependent(void (*kernel)(Arg), dim3 grid, const Arg& arg, cudaStream
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, kernel, arg);
+  count_launch(cudaLaunchKernelEx(&cfg, kernel, arg));
 }
 
 }  // namespace

@@ -496,7 +496,8 @@ kara_status launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensor
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, a, static_cast<__nv_bfloat16*>(out));
+  count_launch(cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, a,
+                                  static_cast<__nv_bfloat16*>(out)));
   return check_launch(__func__);
 }
 

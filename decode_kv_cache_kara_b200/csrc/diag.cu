@@ -42,5 +42,7 @@ extern "C" kara_status kara_wait_probe(int32_t wait_ms, int32_t* dev_status, cud
     return check_launch("kara_wait_probe");
   const long long budget = static_cast<long long>(wait_ms) * khz;   // cycles at the rated clock
   wait_probe_kernel<<<1, 64, 0, stream>>>(dev_status, budget);
-  return check_launch("kara_wait_probe");
+  const kara_status st = check_launch("kara_wait_probe");
+  if (st == KARA_OK) count_launch(cudaSuccess);
+  return st;
 }

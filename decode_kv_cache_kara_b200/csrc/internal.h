@@ -10,6 +10,9 @@
 
 namespace kara {
 
+// Counts a kernel launch call that returned cudaSuccess (kara_launch_count). Defined in api.cu.
+void count_launch(cudaError_t err);
+
 // Launches `kernel` as a programmatic dependent of the previous kernel in `stream`: it may
 // start while that kernel finishes, and it must execute griddepcontrol.wait (which returns once
 // the previous kernel has completed and its memory is visible) before it touches memory.
@@ -27,7 +30,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, args...);
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, args...);
+  count_launch(err);
+  return err;
 }
 
 // 4-D bf16 tensor map (innermost dimension first), 128-byte swizzle, box {64, 1, rows, 1}.

@@ -72,6 +72,8 @@ struct ScoreArgs {
   float* lse_merged;  // [R, Hq, Wp] the chunks merged (+inf past the window)
   int CM;             // key chunks per window, at most
   float* scores;    // [R, Hkv, W]
+  float* part;      // fused kernel, split items: [split - 1][head part, tail part][W] key sums
+  int streamk;      // fused kernel: cluster ranges split items (else they hold whole items)
   int32_t* status;
   int R, W, Wp, Hq, Hkv, G;
   int batch, max_blocks, num_blocks;
@@ -760,25 +762,44 @@ constexpr uint32_t kFEpiBarrier = 1;
 constexpr uint32_t kFSCols = 256;      // TMEM column stride of the two S buffers
 constexpr uint32_t kFDCol = 160;       // TMEM columns of the two D buffers: 160, 176
 
-// Work items (r, g) over valid sequences: KV head g of sequence r with all G of its query
-// heads (G * W / 128 query tiles).
-struct ItemCursor {
-  int r = 0, base = 0, per = -1;
+// Work items (r, g): KV head g of sequence r with all G of its query heads, TPI = G * W / 128
+// query tiles (tile tq: head g * G + tq / CL, queries 128 (tq % CL) ..). Cluster c of ncl takes
+// a contiguous range of the sequence of (item, tile) pairs, items in order:
+//  - streamk: tiles [c N / ncl, (c + 1) N / ncl) of N = R * Hkv * TPI, so every cluster has the
+//    same share within a tile. A boundary inside an item splits it into a head part (ending
+//    cluster c - 1's range) and a tail part (starting cluster c's); each writes its key sums
+//    to its slot of split c and a second kernel adds the two. Ranges are at least TPI tiles
+//    long, so an item holds at most one boundary;
+//  - otherwise: whole items [c I / ncl, (c + 1) I / ncl) of I = R * Hkv.
+// A segment is the range's part of one item, tiles [q0, q1); items of invalid sequences are
+// skipped.
+struct SegCursor {
+  long long t = 0, t1 = 0;
+  int r = 0, g = 0, q0 = 0, q1 = 0;
   SeqInfo s;
-  __device__ __forceinline__ bool seek(const ScoreArgs& a, int t, int& g) {
-    while (true) {
-      if (r >= a.R) return false;
-      if (per < 0) {
-        s = seq_info(a, r);
-        per = s.ok ? a.Hkv : 0;
-      }
-      if (t < base + per) break;
-      base += per;
-      ++r;
-      per = -1;
+  __device__ __forceinline__ void init(const ScoreArgs& a, int c, int ncl, int TPI) {
+    const long long items = static_cast<long long>(a.R) * a.Hkv;
+    if (a.streamk) {
+      const long long n = items * TPI;
+      t = c * n / ncl;
+      t1 = (c + 1) * n / ncl;
+    } else {
+      t = c * items / ncl * TPI;
+      t1 = (c + 1) * items / ncl * TPI;
     }
-    g = t - base;
-    return true;
+  }
+  __device__ __forceinline__ bool next(const ScoreArgs& a, int TPI) {
+    while (t < t1) {
+      const long long item = t / TPI;
+      q0 = static_cast<int>(t - item * TPI);
+      q1 = t1 - t < TPI - q0 ? q0 + static_cast<int>(t1 - t) : TPI;
+      t += q1 - q0;
+      r = static_cast<int>(item / a.Hkv);
+      g = static_cast<int>(item - static_cast<long long>(r) * a.Hkv);
+      s = seq_info(a, r);
+      if (s.ok) return true;
+    }
+    return false;
   }
 };
 
@@ -908,9 +929,10 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       tma_prefetch_desc(&tm_k);
     }
     const int TPI = a.G * CL;
-    ItemCursor cur;
-    int g = 0, C = 0;   // query chunks issued
-    bool have = cur.seek(a, cid, g);
+    SegCursor cur;
+    cur.init(a, cid, ncl, TPI);
+    int C = 0;   // query chunks issued
+    bool have = cur.next(a, TPI);
     auto page_ids = [&](const SeqInfo& s, int& npg) {
       const int key0 = s.start + static_cast<int>(rank) * kFKeys;
       npg = (key0 % 16) != 0 ? 9 : 8;
@@ -920,7 +942,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     int my_blk = have ? page_ids(cur.s, npg) : 0;
     for (int I = 0; have; ++I) {
       if (__shfl_sync(0xffffffffu, *abort_flag != 0 ? 1 : 0, 0)) break;
-      const int r = cur.r, gi = g;
+      const int r = cur.r, gi = cur.g, q0 = cur.q0, q1 = cur.q1;
       int ok = 1;
       if (lane == 0) {
         ok = mbar_wait(k_empty, (I & 1) ^ 1, abort_flag, a.status) ? 1 : 0;
@@ -933,12 +955,12 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int ch = 0; ch < NCH; ++ch)
             tma_load_4d(k_buf + ch * L::kKChunk + p * kPageBytes, &tm_k, k_full, ch * 64, gi, 0, blk);
       }
-      // the next item's page ids (their loads overlap this item's query tiles)
-      have = cur.seek(a, cid + (I + 1) * ncl, g);
+      // the next segment's page ids (their loads overlap this segment's query tiles)
+      have = cur.next(a, TPI);
       if (have) my_blk = page_ids(cur.s, npg);
       bool stop = false;
       if (lane == 0) {
-        for (int tq = 0; tq < TPI && !stop; ++tq) {
+        for (int tq = q0; tq < q1 && !stop; ++tq) {
           const int h = gi * a.G + tq / CL, qt = tq % CL;
           for (int ch = 0; ch < NCH; ++ch) {   // chunk C of the ring: slot C mod 3
             const int slot = C % kFQSlots;
@@ -961,13 +983,14 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, kFKRows);
       const int TPI = a.G * CL;
-      ItemCursor cur;
-      int g, T = 0, I = 0, C = 0;   // tiles, items, query chunks
+      SegCursor cur;
+      cur.init(a, cid, ncl, TPI);
+      int T = 0, I = 0, C = 0;   // tiles, segments, query chunks
       bool ok = true;
-      for (int it = cid; ok && !*abort_flag && cur.seek(a, it, g); it += ncl, ++I) {
+      for (; ok && !*abort_flag && cur.next(a, TPI); ++I) {
         if (!mbar_wait(k_full, I & 1, abort_flag, a.status)) break;
         const uint32_t k_addr = smem_u32(k_buf);
-        for (int tq = 0; tq < TPI && ok; ++tq, ++T) {
+        for (int tq = cur.q0; tq < cur.q1 && ok; ++tq, ++T) {
           const int st = T & 1;
           const uint32_t ph = (T >> 1) & 1;
           if (!mbar_wait(&s_empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
@@ -987,7 +1010,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
           if (!ok) break;
           umma_commit(&s_full[st]);
-          if (tq == TPI - 1) umma_commit(k_empty);
+          if (tq == cur.q1 - 1) umma_commit(k_empty);
         }
       }
     }
@@ -996,16 +1019,17 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (lane == 0) {
       const uint32_t idesc_c = idesc_f16_f32(128, 16, true);
       const int TPI = a.G * CL;
-      ItemCursor cur;
-      int g, Tc = 0, Ic = 0;
-      for (int it = cid; !*abort_flag && cur.seek(a, it, g); it += ncl, ++Ic) {
+      SegCursor cur;
+      cur.init(a, cid, ncl, TPI);
+      int Tc = 0, Ic = 0;
+      for (; !*abort_flag && cur.next(a, TPI); ++Ic) {
         bool ok = true;
-        for (int qt = 0; qt < TPI; ++qt, ++Tc) {
+        for (int qt = cur.q0; qt < cur.q1; ++qt, ++Tc) {
           const int st = Tc % kFPBufs;
           const uint32_t ph = (Tc / kFPBufs) & 1;
           if (!mbar_wait(&p_full[st], ph, abort_flag, a.status) ||
               !mbar_wait(&w_full[st], ph, abort_flag, a.status) ||
-              (qt == 0 &&
+              (qt == cur.q0 &&
                !mbar_wait(&d_empty[Ic & 1], ((Ic >> 1) & 1) ^ 1, abort_flag, a.status))) {
             ok = false;
             break;
@@ -1018,10 +1042,10 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int ks = 0; ks < kFQRows / 16; ++ks) {
             const uint64_t ad = sw128_mnmajor_desc(p_addr + ks * 2048, L::kPAtom, 1024);
             const uint64_t bd = sw128_kmajor_desc(w_addr + (ks >> 2) * 2048 + (ks & 3) * 32);
-            umma_bf16(d_tmem, ad, bd, idesc_c, (ks > 0 || qt > 0) ? 1u : 0u);
+            umma_bf16(d_tmem, ad, bd, idesc_c, (ks > 0 || qt > cur.q0) ? 1u : 0u);
           }
           umma_commit(&p_empty[st]);
-          if (qt == TPI - 1) umma_commit(&d_full[Ic & 1]);
+          if (qt == cur.q1 - 1) umma_commit(&d_full[Ic & 1]);
         }
         if (!ok) break;
       }
@@ -1050,10 +1074,15 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       aborted = __any_sync(0xffffffffu, !ok) != 0;
     };
     const int TPI = a.G * CL;
-    ItemCursor cur;
-    int g = 0, I = 0, tq = team;          // item index and tile within the item (no divisions:
-    while (tq >= TPI) { tq -= TPI; ++I; }  // they would queue behind the exponentials)
-    bool have = cur.seek(a, cid + I * ncl, g);
+    SegCursor cur;
+    cur.init(a, cid, ncl, TPI);
+    int I = 0, tp = team;                 // segment index and tile within the segment (no
+    bool have = cur.next(a, TPI);         // divisions per tile: they would queue behind the
+    while (have && tp >= cur.q1 - cur.q0) {   // exponentials)
+      tp -= cur.q1 - cur.q0;
+      ++I;
+      have = cur.next(a, TPI);
+    }
     // running T mod 3 / T div 3 (P' and weight buffers) and T mod 5 / T div 5 (exchange slots)
     int pb = team, pq = 0, xs = team, xq = 0;
     for (int T = team; have; T += 2) {
@@ -1176,8 +1205,8 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
         fence_proxy_async();
         mbar_arrive(&w_full[pb]);
       }
-      // (5) the item's last tile: the per-key sums over all G heads, read by this team
-      if (tq == TPI - 1) {
+      // (5) the segment's last tile: the per-key sums over its heads, read by this team
+      if (tp == cur.q1 - cur.q0 - 1) {
         wait_cta(&d_full[I & 1], (I >> 1) & 1);
         if (!aborted) {
           tc_fence_after();
@@ -1188,7 +1217,16 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
             tmem_wait_ld();
             reg_fence<4>(d);
             const float val = (d[0] + d[1] + d[2] * (1.f / 16777216.f)) * (1.f / 32768.f);
-            a.scores[(static_cast<size_t>(cur.r) * a.Hkv + g) * a.W + rank * kFKeys + row] = val;
+            float* dst;
+            if (cur.q0 == 0 && cur.q1 == TPI) {
+              dst = a.scores + (static_cast<size_t>(cur.r) * a.Hkv + cur.g) * a.W;
+            } else {   // the head part ends this cluster's range (split cid + 1), the tail
+                       // part starts it (split cid)
+              const int side = cur.q0 == 0 ? 0 : 1;
+              const int split = side == 0 ? cid + 1 : cid;
+              dst = a.part + (static_cast<size_t>(split - 1) * 2 + side) * a.W;
+            }
+            dst[rank * kFKeys + row] = val;
           }
           tc_fence_before();
           mbar_arrive(&d_empty[I & 1]);
@@ -1198,12 +1236,11 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (pb >= kFPBufs) { pb -= kFPBufs; ++pq; }
       xs += 2;
       if (xs >= kFXStages) { xs -= kFXStages; ++xq; }
-      tq += 2;
-      if (tq >= TPI) {
-        tq -= TPI;
+      tp += 2;
+      while (have && tp >= cur.q1 - cur.q0) {
+        tp -= cur.q1 - cur.q0;
         ++I;
-        if (tq >= TPI) { tq -= TPI; ++I; }   // TPI = 1
-        have = cur.seek(a, cid + I * ncl, g);
+        have = cur.next(a, TPI);
       }
     }
   }
@@ -1215,6 +1252,26 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     tmem_dealloc(tmem_base, kTmemCols);
   }
   cluster_sync_all();     // no CTA leaves while a peer may still write into its shared memory
+}
+
+// Items split between two clusters of the fused kernel: scores = head part + tail part (in
+// that order, so the result does not depend on which part finished first). One CTA per
+// range boundary k = 1 .. ncl - 1; boundaries on an item boundary have nothing to add.
+__global__ void __launch_bounds__(256)
+score_split_sum_kernel(const ScoreArgs a, int ncl, int TPI) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // the fused kernel's writes are visible
+  const int k = blockIdx.x + 1;
+  const long long n = static_cast<long long>(a.R) * a.Hkv * TPI;
+  const long long t = k * n / ncl;
+  const long long item = t / TPI;
+  if (t == item * TPI) return;
+  const int r = static_cast<int>(item / a.Hkv);
+  const int g = static_cast<int>(item - static_cast<long long>(r) * a.Hkv);
+  if (!seq_info(a, r).ok) return;
+  const float* head = a.part + static_cast<size_t>(k - 1) * 2 * a.W;
+  const float* tail = head + a.W;
+  float* dst = a.scores + (static_cast<size_t>(r) * a.Hkv + g) * a.W;
+  for (int j = threadIdx.x; j < a.W; j += blockDim.x) dst[j] = head[j] + tail[j];
 }
 
 template <int D>
@@ -1355,13 +1412,29 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
       }
       max_clusters[CL] = n;
     }
-    const int items = L.R * L.Hkv;    // upper bound (valid sequences only are walked)
-    const int ncl = std::max(1, std::min(max_clusters[CL], items));
+    const long long items = static_cast<long long>(L.R) * L.Hkv;
+    const int ncl = static_cast<int>(std::max<long long>(1, std::min<long long>(max_clusters[CL], items)));
+    // Tile-granular ranges whenever the split slots fit in the workspace (they do whenever
+    // ncl <= items, which the grid guarantees; checked all the same). The ranges are then at
+    // least TPI tiles long, as the kernel assumes.
+    const int TPI = a.G * CL;
+    const long long ntiles = items * TPI;
+    const size_t part_bytes = static_cast<size_t>(ncl - 1) * 2 * L.W * sizeof(float);
+    a.part = L.lse;
+    a.streamk = ncl > 1 && ntiles / ncl >= TPI &&
+                part_bytes <= score_workspace_bytes(L.R, L.W, L.Hq);
+    bool any_split = false;
+    for (int k = 1; a.streamk && k < ncl && !any_split; ++k)
+      any_split = (k * ntiles / ncl) % TPI != 0;
     cfg.gridDim = dim3(ncl * CL);
-    cudaLaunchKernelEx(&cfg, kern, tq1, tk, a);
+    count_launch(cudaLaunchKernelEx(&cfg, kern, tq1, tk, a));
     if (check_launch("score_fused_kernel") != KARA_OK) {
       describe_kernel("score_fused_kernel", reinterpret_cast<const void*>(kern), kFThreads, smem);
       return KARA_ERR_CUDA;
+    }
+    if (any_split) {
+      launch_pdl(score_split_sum_kernel, dim3(ncl - 1), dim3(256), 0, stream, a, ncl, TPI);
+      if (check_launch("score_split_sum_kernel") != KARA_OK) return KARA_ERR_CUDA;
     }
     return KARA_OK;
   }

@@ -83,6 +83,7 @@ _SIGNATURES = {
     "kara_status_str": ([_I], ctypes.c_char_p),
     "kara_version": ([], ctypes.c_char_p),
     "kara_last_error": ([], ctypes.c_char_p),
+    "kara_launch_count": ([], ctypes.c_uint64),
     "kara_wait_probe": ([_I, _P, _P], _I),
 }
 
@@ -115,7 +116,13 @@ def declared_symbols(header: str | None = None) -> list:
     """Function names declared in include/kara.h (used by the ABI tests)."""
     header = header or os.path.join(_build.INCLUDE, "kara.h")
     text = open(header).read()
-    return re.findall(r"^\s*(?:kara_status|size_t|const char\*)\s+(\w+)\s*\(", text, re.M)
+    return re.findall(r"^\s*(?:kara_status|size_t|uint64_t|const char\*)\s+(\w+)\s*\(", text,
+                      re.M)
+
+
+def kara_launch_count() -> int:
+    """Kernel launches the library has issued in this process (difference two readings)."""
+    return int(lib().kara_launch_count())
 
 
 def status_str(code: int) -> str:

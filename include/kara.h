@@ -268,6 +268,11 @@ const char* kara_status_str(int32_t status);
  * call into the library. */
 const char* kara_last_error(void);
 
+/* Number of kernel launches the library has issued in this process (launch calls that
+ * returned cudaSuccess, all threads and devices), so that a caller can count the kernels a
+ * sequence of calls runs: take the difference of two readings. */
+uint64_t kara_launch_count(void);
+
 /* Library version string ("kara-b200 <major>.<minor>"). */
 const char* kara_version(void);
 

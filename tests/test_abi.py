@@ -12,7 +12,7 @@ def test_library_exports_every_declared_symbol(lib_path):
     names = K.declared_symbols()
     expected = {"kara_score", "kara_select", "kara_token2chunk", "kara_compact",
                 "paged_decode_attn", "lacache_compact", "kara_workspace_bytes",
-                "kara_status_str", "kara_version"}
+                "kara_status_str", "kara_version", "kara_launch_count"}
     assert expected <= set(names)
     handle = ctypes.CDLL(lib_path)
     for n in names:
@@ -27,6 +27,7 @@ def test_status_strings_and_version(lib_path):
 
 def test_host_side_validation_returns_before_any_launch(lib_path):
     L = K.lib()
+    launches = K.kara_launch_count()
     null = ctypes.c_void_p(0)
     # k > window, window too large, rows < 0
     assert L.kara_select(null, 4, 16, 17, null, null) == K.ERR_INVALID_ARG
@@ -61,6 +62,8 @@ def test_host_side_validation_returns_before_any_launch(lib_path):
     # compaction window above KARA_MAX_WINDOW
     assert L.kara_compact(layers, 1, ctypes.byref(pool), null, 1, 5000, 8, one, one, 1 << 20, one,
                           null) == K.ERR_INVALID_ARG
+    # none of these reached a kernel launch
+    assert K.kara_launch_count() == launches
 
 
 def test_workspace_sizes(lib_path):

@@ -38,6 +38,14 @@ SCORE_CASES = {
     "d64_g4_w256": synth.Workload("d64_g4_w256", batch=3, layers=1, hq=8, hkv=2, head_dim=64,
                                   ctx_lo=260, ctx_hi=400, window=256, keep=51, heavy_frac=0.05,
                                   q_mode="neighbour", spare_blocks=8),
+    # more (sequence, KV head) items than resident clusters: cluster ranges end inside items,
+    # whose two parts are summed by the split kernel
+    "w128_split_items": synth.Workload("w128_split", batch=40, layers=1, hq=8, hkv=4,
+                                       head_dim=128, ctx_lo=130, ctx_hi=300, window=128, keep=26,
+                                       heavy_frac=0.05, q_mode="neighbour", spare_blocks=8),
+    "w256_split_items": synth.Workload("w256_split", batch=24, layers=1, hq=8, hkv=4,
+                                       head_dim=128, ctx_lo=260, ctx_hi=420, window=256, keep=51,
+                                       heavy_frac=0.05, spare_blocks=8),
 }
 
 
@@ -93,6 +101,37 @@ def test_score_reports_short_context():
     cpu["ctx_len"][1] = wl.window - 1
     ref = oracle_scores(cpu, wl, [0, 2])
     H.assert_scores_close(H.f64(scores[[0, 2]]), ref)
+
+
+def test_score_split_items_skip_short_contexts():
+    """Every third sequence too short for the window: its items drop out of the cluster ranges
+    (and of the split sums), its rows are zero and reported; the rest match the oracle."""
+    wl = SCORE_CASES["w128_split_items"]
+    cpu, dev = H.make(wl, 4)
+    bad = list(range(1, wl.batch, 3))
+    good = [r for r in range(wl.batch) if r not in bad]
+    dev["ctx_len"][bad] = wl.window - 1
+    pool = K.PagedPool.from_cache(dev)
+    status = K.new_status()
+    scores = K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window, status=status)
+    torch.cuda.synchronize()
+    assert K.read_status(status) == K.ERR_INVALID_ARG
+    assert (scores[bad] == 0).all()
+    cpu["ctx_len"][bad] = wl.window - 1
+    H.assert_scores_close(H.f64(scores[good]), oracle_scores(cpu, wl, good))
+
+
+@pytest.mark.parametrize("name,launches", [("g7_w1024_unaligned", 1), ("w128_split_items", 2)])
+def test_score_launch_count(name, launches):
+    """The fused kernel alone when every cluster range holds whole items; with the split sum
+    when more items than resident clusters make ranges end inside items."""
+    wl = SCORE_CASES[name]
+    cpu, dev = H.make(wl, 1)
+    pool = K.PagedPool.from_cache(dev)
+    c0 = K.kara_launch_count()
+    K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window)
+    torch.cuda.synchronize()
+    assert K.kara_launch_count() - c0 == launches
 
 
 @pytest.mark.parametrize("name", ["tiny", "g7_ragged_unaligned", "g8_w384", "w16_ctx_eq_w"])
