@@ -115,14 +115,15 @@ def fresh_blocks_needed(wl: Workload) -> int:
 
 @torch.no_grad()
 def make_cache(wl: Workload, seed: int, device="cpu", layers: int | None = None,
-               with_queries: bool = True, dtype=torch.bfloat16) -> dict:
+               with_queries: bool = True, dtype=torch.bfloat16, extra_pages: int = 0) -> dict:
     """Build one seeded paged cache for a workload.
 
     Returns a dict with ``k``/``v`` (lists, one [num_blocks, page, Hkv, d] tensor per layer),
     ``block_table`` [B, max_blocks] int32 (-1 = no block), ``ctx_len`` [B] int32,
     ``free_list`` [num_blocks] int32, ``free_top`` [1] int32, and when ``with_queries`` the
     window queries ``q_win`` (list per layer of [B, W, Hq, d]) and decode queries ``q_dec``
-    [B, Hq, d]. Layers default to ``wl.layers``.
+    [B, Hq, d]. Layers default to ``wl.layers``. ``extra_pages`` adds that many table
+    columns per sequence and as many spare blocks per sequence, room for a decode loop.
     """
     device = torch.device(device)
     nlayers = wl.layers if layers is None else layers
@@ -135,8 +136,8 @@ def make_cache(wl: Workload, seed: int, device="cpu", layers: int | None = None,
     else:
         ctx = rng.integers(wl.ctx_lo, wl.ctx_hi + 1, size=wl.batch)
     pages = [math.ceil(int(n) / wl.page) for n in ctx]
-    max_blocks = max(pages) + 1
-    num_blocks = sum(pages) + fresh_blocks_needed(wl) + wl.spare_blocks
+    max_blocks = max(pages) + 1 + extra_pages
+    num_blocks = sum(pages) + fresh_blocks_needed(wl) + wl.spare_blocks + wl.batch * extra_pages
     perm = rng.permutation(num_blocks).astype(np.int64)
 
     table = np.full((wl.batch, max_blocks), -1, dtype=np.int32)
@@ -182,6 +183,26 @@ def make_cache(wl: Workload, seed: int, device="cpu", layers: int | None = None,
     if with_queries:
         out["q_dec"] = torch.randn((wl.batch, wl.hq, wl.head_dim), generator=gen, device=device,
                                    dtype=torch.float32).to(dtype)
+    return out
+
+
+@torch.no_grad()
+def decode_step_inputs(wl: Workload, seed: int, step: int, layers: int | None = None,
+                       dtype=torch.bfloat16) -> list:
+    """Seeded inputs of decode step ``step`` (CPU tensors), one dict per layer: the new
+    token's ``k`` and ``v`` [B, Hkv, d] ~ N(0, 1) and its query ``q`` [B, Hq, d], each query
+    head the new key of its KV head plus N(0, 0.5^2) noise (so the window queries resemble
+    the window keys, as in the window-query recipe)."""
+    nlayers = wl.layers if layers is None else layers
+    gen = torch.Generator()
+    gen.manual_seed(seed * 1_000_003 + step)
+    out = []
+    for _ in range(nlayers):
+        k = torch.randn((wl.batch, wl.hkv, wl.head_dim), generator=gen)
+        v = torch.randn((wl.batch, wl.hkv, wl.head_dim), generator=gen)
+        noise = torch.randn((wl.batch, wl.hq, wl.head_dim), generator=gen)
+        q = k.repeat_interleave(wl.group, dim=1) + 0.5 * noise
+        out.append({"q": q.to(dtype), "k": k.to(dtype), "v": v.to(dtype)})
     return out
 
 

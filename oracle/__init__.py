@@ -19,8 +19,10 @@ Modules:
 * ``kara``    - window scoring, top-k selection, Token2Chunk, paged compaction.
 * ``decode``  - paged GQA decode attention over the (compressed) cache.
 * ``lacache`` - the ladder keep map and ladder compaction.
+* ``decode_loop`` - the decode loop around them: block allocation for new slots, the fused
+  append + attention step, the tail-W trigger checked periodically, the window-query ring.
 
 Parity status of every function is stated in its module header.
 """
 
-from . import kara, decode, lacache  # noqa: F401
+from . import kara, decode, lacache, decode_loop  # noqa: F401
