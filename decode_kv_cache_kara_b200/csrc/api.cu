@@ -71,6 +71,84 @@ kara_status fill_layers(const kara_layer_kv* layers, int32_t num_layers, LayerPt
   return KARA_OK;
 }
 
+
+kara_status score_impl(const void* q_win, int ring, const void* k_cache, const kara_pool* pool,
+                       const int32_t* seq_ids, int32_t num_seqs, int32_t window,
+                       int32_t num_q_heads, float scale, float* scores, void* workspace,
+                       size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
+  kara_status st = check_pool(pool);
+  if (st != KARA_OK) return st;
+  if ((st = check_heads(pool, num_q_heads)) != KARA_OK) return st;
+  if (num_seqs < 0 || window < 1 || window > KARA_MAX_WINDOW) return KARA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return KARA_OK;
+  if (q_win == nullptr || k_cache == nullptr || scores == nullptr || dev_status == nullptr)
+    return KARA_ERR_INVALID_ARG;
+  if (!aligned16(q_win) || !aligned16(k_cache) || !aligned16(scores)) return KARA_ERR_INVALID_ARG;
+  const size_t need = kara_workspace_bytes(KARA_OP_SCORE, pool, num_seqs, window, num_q_heads, 0);
+  if (workspace == nullptr || workspace_bytes < need || !aligned256(workspace))
+    return KARA_ERR_WORKSPACE;
+  ScoreLaunch L;
+  L.q_win = q_win;
+  L.k_cache = k_cache;
+  L.block_table = pool->block_table;
+  L.ctx_len = pool->ctx_len;
+  L.seq_ids = seq_ids;
+  L.lse = static_cast<float*>(workspace);
+  L.scores = scores;
+  L.status = dev_status;
+  L.R = num_seqs;
+  L.W = window;
+  L.Hq = num_q_heads;
+  L.Hkv = pool->num_kv_heads;
+  L.D = pool->head_dim;
+  L.batch = pool->batch;
+  L.max_blocks = pool->max_blocks_per_seq;
+  L.num_blocks = pool->num_blocks;
+  L.scale = scale;
+  L.ring = ring;
+  return launch_score_kernels(L, stream);
+}
+
+
+kara_status decode_impl(const void* q, const void* k_new, const void* v_new, const void* k_cache,
+                        const void* v_cache, const kara_pool* pool, int32_t num_q_heads,
+                        float scale, void* q_ring, int32_t window, void* out, void* workspace,
+                        size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
+  kara_status st = check_pool(pool);
+  if (st != KARA_OK) return st;
+  if ((st = check_heads(pool, num_q_heads)) != KARA_OK) return st;
+  if (pool->batch == 0) return KARA_OK;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || out == nullptr ||
+      dev_status == nullptr)
+    return KARA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return KARA_ERR_INVALID_ARG;
+  const size_t need = kara_workspace_bytes(KARA_OP_DECODE, pool, 0, 0, num_q_heads, 0);
+  if (workspace == nullptr || workspace_bytes < need || !aligned256(workspace))
+    return KARA_ERR_WORKSPACE;
+  DecodeLaunch L;
+  L.q = q;
+  L.k_cache = k_cache;
+  L.v_cache = v_cache;
+  L.block_table = pool->block_table;
+  L.ctx_len = pool->ctx_len;
+  L.out = out;
+  L.partial = static_cast<float*>(workspace);
+  L.status = dev_status;
+  L.B = pool->batch;
+  L.Hq = num_q_heads;
+  L.Hkv = pool->num_kv_heads;
+  L.D = pool->head_dim;
+  L.max_blocks = pool->max_blocks_per_seq;
+  L.num_blocks = pool->num_blocks;
+  L.scale = scale;
+  L.k_new = k_new;
+  L.v_new = v_new;
+  L.q_ring = q_ring;
+  L.ring_w = window;
+  return launch_decode(L, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -116,40 +194,21 @@ size_t kara_workspace_bytes(kara_op op, const kara_pool* pool, int32_t num_seqs,
   }
 }
 
+
 kara_status kara_score(const void* q_win, const void* k_cache, const kara_pool* pool,
                        const int32_t* seq_ids, int32_t num_seqs, int32_t window,
                        int32_t num_q_heads, float scale, float* scores, void* workspace,
                        size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
-  kara_status st = check_pool(pool);
-  if (st != KARA_OK) return st;
-  if ((st = check_heads(pool, num_q_heads)) != KARA_OK) return st;
-  if (num_seqs < 0 || window < 1 || window > KARA_MAX_WINDOW) return KARA_ERR_INVALID_ARG;
-  if (num_seqs == 0) return KARA_OK;
-  if (q_win == nullptr || k_cache == nullptr || scores == nullptr || dev_status == nullptr)
-    return KARA_ERR_INVALID_ARG;
-  if (!aligned16(q_win) || !aligned16(k_cache) || !aligned16(scores)) return KARA_ERR_INVALID_ARG;
-  const size_t need = kara_workspace_bytes(KARA_OP_SCORE, pool, num_seqs, window, num_q_heads, 0);
-  if (workspace == nullptr || workspace_bytes < need || !aligned256(workspace))
-    return KARA_ERR_WORKSPACE;
-  ScoreLaunch L;
-  L.q_win = q_win;
-  L.k_cache = k_cache;
-  L.block_table = pool->block_table;
-  L.ctx_len = pool->ctx_len;
-  L.seq_ids = seq_ids;
-  L.lse = static_cast<float*>(workspace);
-  L.scores = scores;
-  L.status = dev_status;
-  L.R = num_seqs;
-  L.W = window;
-  L.Hq = num_q_heads;
-  L.Hkv = pool->num_kv_heads;
-  L.D = pool->head_dim;
-  L.batch = pool->batch;
-  L.max_blocks = pool->max_blocks_per_seq;
-  L.num_blocks = pool->num_blocks;
-  L.scale = scale;
-  return launch_score_kernels(L, stream);
+  return score_impl(q_win, 0, k_cache, pool, seq_ids, num_seqs, window, num_q_heads, scale,
+                    scores, workspace, workspace_bytes, dev_status, stream);
+}
+
+kara_status kara_score_ring(const void* q_ring, const void* k_cache, const kara_pool* pool,
+                            const int32_t* seq_ids, int32_t num_seqs, int32_t window,
+                            int32_t num_q_heads, float scale, float* scores, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
+  return score_impl(q_ring, 1, k_cache, pool, seq_ids, num_seqs, window, num_q_heads, scale,
+                    scores, workspace, workspace_bytes, dev_status, stream);
 }
 
 kara_status kara_select(const float* scores, int32_t rows, int32_t window, int32_t k,
@@ -210,39 +269,53 @@ kara_status kara_compact(const kara_layer_kv* layers, int32_t num_layers, const 
   return launch_compact(L, stream);
 }
 
+
 kara_status paged_decode_attn(const void* q, const void* k_cache, const void* v_cache,
                               const kara_pool* pool, int32_t num_q_heads, float scale, void* out,
                               void* workspace, size_t workspace_bytes, int32_t* dev_status,
                               cudaStream_t stream) {
+  return decode_impl(q, nullptr, nullptr, k_cache, v_cache, pool, num_q_heads, scale, nullptr, 0,
+                     out, workspace, workspace_bytes, dev_status, stream);
+}
+
+kara_status kara_decode_append(const void* q, const void* k_new, const void* v_new,
+                               void* k_cache, void* v_cache, const kara_pool* pool,
+                               int32_t num_q_heads, float scale, void* q_ring, int32_t window,
+                               void* out, void* workspace, size_t workspace_bytes,
+                               int32_t* dev_status, cudaStream_t stream) {
+  if (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new))
+    return KARA_ERR_INVALID_ARG;
+  if (q_ring != nullptr && (window < 1 || window > KARA_MAX_WINDOW || !aligned16(q_ring)))
+    return KARA_ERR_INVALID_ARG;
+  return decode_impl(q, k_new, v_new, k_cache, v_cache, pool, num_q_heads, scale, q_ring,
+                     window, out, workspace, workspace_bytes, dev_status, stream);
+}
+
+kara_status kara_step_begin(const kara_pool* pool, int32_t* dev_status, cudaStream_t stream) {
   kara_status st = check_pool(pool);
   if (st != KARA_OK) return st;
-  if ((st = check_heads(pool, num_q_heads)) != KARA_OK) return st;
+  if (pool->free_list == nullptr || pool->free_top == nullptr || dev_status == nullptr)
+    return KARA_ERR_INVALID_ARG;
   if (pool->batch == 0) return KARA_OK;
-  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || out == nullptr ||
-      dev_status == nullptr)
+  return launch_step_begin(pool, dev_status, stream);
+}
+
+kara_status kara_step_end(const kara_pool* pool, int32_t* tail, int32_t window, int32_t check,
+                          int32_t* due, int32_t* due_count, cudaStream_t stream) {
+  kara_status st = check_pool(pool);
+  if (st != KARA_OK) return st;
+  if (check != 0 && (tail == nullptr || due == nullptr || due_count == nullptr || window < 1))
     return KARA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-    return KARA_ERR_INVALID_ARG;
-  const size_t need = kara_workspace_bytes(KARA_OP_DECODE, pool, 0, 0, num_q_heads, 0);
-  if (workspace == nullptr || workspace_bytes < need || !aligned256(workspace))
-    return KARA_ERR_WORKSPACE;
-  DecodeLaunch L;
-  L.q = q;
-  L.k_cache = k_cache;
-  L.v_cache = v_cache;
-  L.block_table = pool->block_table;
-  L.ctx_len = pool->ctx_len;
-  L.out = out;
-  L.partial = static_cast<float*>(workspace);
-  L.status = dev_status;
-  L.B = pool->batch;
-  L.Hq = num_q_heads;
-  L.Hkv = pool->num_kv_heads;
-  L.D = pool->head_dim;
-  L.max_blocks = pool->max_blocks_per_seq;
-  L.num_blocks = pool->num_blocks;
-  L.scale = scale;
-  return launch_decode(L, stream);
+  if (pool->batch == 0) return KARA_OK;
+  return launch_step_end(pool, tail, window, check != 0 ? 1 : 0, due, due_count, stream);
+}
+
+kara_status kara_reset_tails(int32_t* tail, const int32_t* seq_ids, int32_t num_seqs,
+                             int32_t batch, cudaStream_t stream) {
+  if (num_seqs < 0 || batch < 0) return KARA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return KARA_OK;
+  if (tail == nullptr || seq_ids == nullptr) return KARA_ERR_INVALID_ARG;
+  return launch_reset_tails(tail, seq_ids, num_seqs, batch, stream);
 }
 
 kara_status lacache_compact(const kara_layer_kv* layers, int32_t num_layers,

@@ -19,6 +19,36 @@ __device__ __forceinline__ void report(int32_t* status, int32_t code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
+// Exclusive prefix sum of one int per thread over a block of 1024 threads (32 warps); *total
+// gets the block's sum. buf: 33 ints of shared memory. Every thread of the block must call it.
+__device__ __forceinline__ int block_scan_add(int v, int* buf, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) buf[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = buf[lane];
+    int z = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, z, off);
+      if (lane >= off) z += y;
+    }
+    buf[lane] = z - w;        // exclusive prefix of warp totals
+    if (lane == 31) buf[32] = z;
+  }
+  __syncthreads();
+  const int res = buf[warp] + x - v;
+  *total = buf[32];
+  __syncthreads();
+  return res;
+}
+
 // ---------------------------------------------------------------------------------------
 // bf16 <-> fp32 (bit-level; bf16 -> fp32 is exact)
 // ---------------------------------------------------------------------------------------

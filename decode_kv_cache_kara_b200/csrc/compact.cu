@@ -37,34 +37,6 @@ constexpr int kPlanHeader = 16;   // valid, total_new, total_old, top
 constexpr int kPlanStride = 12;   // b, n, start, off, p0, n_old, n_new, base_new, base_old, done
 enum { P_B = 0, P_N, P_START, P_OFF, P_P0, P_NOLD, P_NNEW, P_BNEW, P_BOLD, P_DONE };
 
-__device__ int block_scan_add(int v, int* buf, int* total) {
-  // exclusive scan over 1024 threads (32 warps)
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, off);
-    if (lane >= off) x += y;
-  }
-  if (lane == 31) buf[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int w = buf[lane];
-    int z = w;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, z, off);
-      if (lane >= off) z += y;
-    }
-    buf[lane] = z - w;        // exclusive prefix of warp totals
-    if (lane == 31) buf[32] = z;
-  }
-  __syncthreads();
-  const int res = buf[warp] + x - v;
-  *total = buf[32];
-  __syncthreads();
-  return res;
-}
 
 struct PlanParams {
   const int32_t* block_table;

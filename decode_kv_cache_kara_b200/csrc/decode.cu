@@ -45,6 +45,14 @@ struct DecodeArgs {
   int32_t* status;
   int B, Hq, Hkv, max_blocks, num_blocks, S;
   float cs;            // scale * log2(e)
+  // fused decode step (append): the new token of every sequence at slot n = ctx_len
+  int append;
+  const __nv_bfloat16* k_new;   // [B, Hkv, D]
+  const __nv_bfloat16* v_new;
+  __nv_bfloat16* k_dst;         // the caches the new token is written to (= k, v)
+  __nv_bfloat16* v_dst;
+  __nv_bfloat16* q_ring;        // [B, 2W, Hq, D] or null
+  int ring_w;                   // W
 };
 
 template <int D>
@@ -398,6 +406,12 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
 // and every lane keeps kCombBatch independent loads in flight before it accumulates them. The
 // warps' sums meet in shared memory. Launched as a programmatic dependent of the stream kernel:
 // its CTAs may start early and wait for the stream kernel's results.
+//
+// Fused decode step (a.append): the new token at slot n = ctx_len is one more term of the
+// softmax, taken from the inputs (s = q . k_new * scale, value v_new); the CTA of the group's
+// first query head writes k_new / v_new to slot n of the cache (its block was taken by
+// kara_step_begin), and every CTA writes its query to rows n mod W and n mod W + W of the
+// window-query ring. The stream kernel, which reads slots [0, n) only, has finished by then.
 constexpr int kCombWarps = 4;
 constexpr int kCombBatch = 8;
 
@@ -421,6 +435,21 @@ decode_combine_kernel(const DecodeArgs a, __nv_bfloat16* __restrict__ out) {
   for (int s0 = lane; s0 < splits; s0 += 32) mx = fmaxf(mx, ml[s0].x);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  // the new token's logit (base 2), in every warp; it joins the exponent base
+  const int h = bh - b * a.Hq;
+  const int g = h / (a.Hq / a.Hkv);
+  float s_new = -INFINITY;
+  if (a.append) {
+    const __nv_bfloat16* qr = a.q + static_cast<size_t>(bh) * D + lane * V;
+    const __nv_bfloat16* kr = a.k_new + (static_cast<size_t>(b) * a.Hkv + g) * D + lane * V;
+    float dot = 0.f;
+#pragma unroll
+    for (int v = 0; v < V; ++v) dot = fmaf(__bfloat162float(qr[v]), __bfloat162float(kr[v]), dot);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    s_new = dot * a.cs;
+    mx = fmaxf(mx, s_new);
+  }
   float acc[V];
 #pragma unroll
   for (int v = 0; v < V; ++v) acc[v] = 0.f;
@@ -462,11 +491,50 @@ decode_combine_kernel(const DecodeArgs a, __nv_bfloat16* __restrict__ out) {
 #pragma unroll
       for (int v = 0; v < V; ++v) r[v] += red_o[w][lane * V + v];
     }
+    if (a.append) {
+      const float w = ex2(s_new - mx);
+      const __nv_bfloat16* vr = a.v_new + (static_cast<size_t>(b) * a.Hkv + g) * D + lane * V;
+      l += w;
+#pragma unroll
+      for (int v = 0; v < V; ++v) r[v] = fmaf(w, __bfloat162float(vr[v]), r[v]);
+    }
     const float inv = l > 0.f ? 1.f / l : 0.f;
     __nv_bfloat16* dst = out + static_cast<size_t>(bh) * D + lane * V;
 #pragma unroll
     for (int v = 0; v < V; v += 2)
       *reinterpret_cast<__nv_bfloat162*>(dst + v) = __floats2bfloat162_rn(r[v] * inv, r[v + 1] * inv);
+  } else if (warp == 1 && a.append) {
+    // the new token into the cache (one CTA per KV head) and its query into the ring
+    const int n_raw = a.ctx_len[b];
+    if (n_raw < 0 || n_raw >= a.max_blocks * 16) {
+      if (lane == 0) report(a.status, KARA_ERR_INVALID_ARG);
+    } else {
+      if (h % (a.Hq / a.Hkv) == 0) {
+        const int blk = a.block_table[static_cast<size_t>(b) * a.max_blocks + n_raw / 16];
+        if (blk < 0 || blk >= a.num_blocks) {
+          if (lane == 0) report(a.status, KARA_ERR_BAD_BLOCK);
+        } else {
+          const size_t row = ((static_cast<size_t>(blk) * 16 + n_raw % 16) * a.Hkv + g) * D + lane * V;
+          const size_t src = (static_cast<size_t>(b) * a.Hkv + g) * D + lane * V;
+#pragma unroll
+          for (int v = 0; v < V; ++v) {
+            a.k_dst[row + v] = a.k_new[src + v];
+            a.v_dst[row + v] = a.v_new[src + v];
+          }
+        }
+      }
+      if (a.q_ring != nullptr) {
+        const int p = n_raw % a.ring_w;
+        const __nv_bfloat16* qr = a.q + static_cast<size_t>(bh) * D + lane * V;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          __nv_bfloat16* dq = a.q_ring +
+              ((static_cast<size_t>(b) * 2 * a.ring_w + p + e * a.ring_w) * a.Hq + h) * D + lane * V;
+#pragma unroll
+          for (int v = 0; v < V; ++v) dq[v] = qr[v];
+        }
+      }
+    }
   }
 }
 
@@ -544,6 +612,13 @@ kara_status launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
   a.max_blocks = L.max_blocks;
   a.num_blocks = L.num_blocks;
   a.cs = L.scale * 1.4426950408889634f;
+  a.append = L.k_new != nullptr ? 1 : 0;
+  a.k_new = static_cast<const __nv_bfloat16*>(L.k_new);
+  a.v_new = static_cast<const __nv_bfloat16*>(L.v_new);
+  a.k_dst = static_cast<__nv_bfloat16*>(const_cast<void*>(L.k_cache));
+  a.v_dst = static_cast<__nv_bfloat16*>(const_cast<void*>(L.v_cache));
+  a.q_ring = static_cast<__nv_bfloat16*>(L.q_ring);
+  a.ring_w = L.ring_w;
   const int G = L.Hq / L.Hkv;
   // paged pools as 4-D maps {d, Hkv, 16 slots, blocks}; box = one page of one KV head, 64
   // channels wide, 128-byte swizzle (the same map shape the scoring kernels use)

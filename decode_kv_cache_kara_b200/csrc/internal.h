@@ -57,6 +57,7 @@ struct ScoreLaunch {
   int R, W, Hq, Hkv, D;
   int batch, max_blocks, num_blocks;
   float scale;
+  int ring = 0;   // q_win is the window-query ring [batch, 2W, Hq, d]
 };
 int score_lse_stride(int W);
 int score_chunks(int W);
@@ -120,9 +121,19 @@ struct DecodeLaunch {
   int B, Hq, Hkv, D;
   int max_blocks, num_blocks;
   float scale;
+  // fused decode step: the new token (null for plain decode) and the window-query ring
+  const void* k_new = nullptr;
+  const void* v_new = nullptr;
+  void* q_ring = nullptr;
+  int ring_w = 0;
 };
 int decode_num_splits(int max_blocks);
 size_t decode_workspace_bytes(int B, int Hq, int D, int max_blocks);
 kara_status launch_decode(const DecodeLaunch& L, cudaStream_t stream);
+kara_status launch_step_begin(const kara_pool* pool, int32_t* dev_status, cudaStream_t stream);
+kara_status launch_step_end(const kara_pool* pool, int32_t* tail, int32_t window, int32_t check,
+                            int32_t* due, int32_t* due_count, cudaStream_t stream);
+kara_status launch_reset_tails(int32_t* tail, const int32_t* seq_ids, int32_t num_seqs,
+                               int32_t batch, cudaStream_t stream);
 
 }  // namespace kara

@@ -74,6 +74,7 @@ struct ScoreArgs {
   float* scores;    // [R, Hkv, W]
   float* part;      // fused kernel, split items: [split - 1][head part, tail part][W] key sums
   int streamk;      // fused kernel: cluster ranges split items (else they hold whole items)
+  int ring;         // queries from the window-query ring [batch, 2W, Hq, d] (else q_win)
   int32_t* status;
   int R, W, Wp, Hq, Hkv, G;
   int batch, max_blocks, num_blocks;
@@ -95,6 +96,17 @@ __device__ __forceinline__ SeqInfo seq_info(const ScoreArgs& a, int r) {
   s.p_first = s.ok ? s.start / 16 : 0;
   s.np = s.ok ? (s.n - 1) / 16 - s.p_first + 1 : 0;
   return s;
+}
+
+// Row and batch coordinates of the query tile that starts at window position row0: in the
+// dense q_win [R, W, Hq, d] (due sequence r), or in the window-query ring [batch, 2W, Hq, d]
+// (cache row b; window position 0 is ring row (n - W) mod W, and the W rows from there are
+// contiguous because every query is stored at rows s mod W and s mod W + W).
+__device__ __forceinline__ int q_tile_row(const ScoreArgs& a, const SeqInfo& s, int row0) {
+  return a.ring ? s.start % a.W + row0 : row0;
+}
+__device__ __forceinline__ int q_tile_batch(const ScoreArgs& a, const SeqInfo& s, int r) {
+  return a.ring ? s.b : r;
 }
 
 // Block id of page p of sequence row b, with range check (an out-of-range id is reported and
@@ -260,7 +272,7 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
           mbar_expect_tx(&q_full[qi], kQBytes);
           for (int ch = 0; ch < NCH; ++ch)
             tma_load_4d(q_buf + qi * kQBytes + ch * kQRows1 * kRowBytes, &tm_q, &q_full[qi],
-                        ch * 64, h, qt * kQRows1, r);
+                        ch * 64, h, q_tile_row(a, s, qt * kQRows1), q_tile_batch(a, s, r));
           if (++qi == kQStages1) { qi = 0; qph ^= 1; }
         }
       }
@@ -561,7 +573,7 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
           mbar_expect_tx(&b_full[bi], kBBytes);
           for (int c = 0; c < NCH; ++c)
             tma_load_4d(b_buf + bi * kBBytes + c * kQRows2 * kRowBytes, &tm_q, &b_full[bi],
-                        c * 64, h, qt * kQRows2, r);
+                        c * 64, h, q_tile_row(a, s, qt * kQRows2), q_tile_batch(a, s, r));
           if (++bi == kQStages2) { bi = 0; bph ^= 1; }
         }
       }
@@ -943,6 +955,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int I = 0; have; ++I) {
       if (__shfl_sync(0xffffffffu, *abort_flag != 0 ? 1 : 0, 0)) break;
       const int r = cur.r, gi = cur.g, q0 = cur.q0, q1 = cur.q1;
+      const SeqInfo si = cur.s;
       int ok = 1;
       if (lane == 0) {
         ok = mbar_wait(k_empty, (I & 1) ^ 1, abort_flag, a.status) ? 1 : 0;
@@ -970,7 +983,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             mbar_expect_tx(&q_full[slot], L::kQChunk);
             tma_load_4d(q_buf + slot * L::kQChunk, &tm_q, &q_full[slot], ch * 64, h,
-                        qt * kFQRows, r);
+                        q_tile_row(a, si, qt * kFQRows), q_tile_batch(a, si, r));
             ++C;
           }
         }
@@ -1340,10 +1353,12 @@ int sm_count() {
 
 template <int D>
 kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
-  const uint64_t qdims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(L.Hq),
-                             static_cast<uint64_t>(L.W), static_cast<uint64_t>(L.R)};
+  // queries: q_win [R, W, Hq, d], or the window-query ring [batch, 2W, Hq, d]
+  const uint64_t qrows = static_cast<uint64_t>(L.ring ? 2 * L.W : L.W);
+  const uint64_t qdims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(L.Hq), qrows,
+                             static_cast<uint64_t>(L.ring ? L.batch : L.R)};
   const uint64_t qstr[3] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(L.Hq) * D * 2,
-                            static_cast<uint64_t>(L.W) * L.Hq * D * 2};
+                            qrows * L.Hq * D * 2};
   const uint64_t kdims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(L.Hkv), 16,
                              static_cast<uint64_t>(L.num_blocks)};
   const uint64_t kstr[3] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(L.Hkv) * D * 2,
@@ -1374,6 +1389,9 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   a.max_blocks = L.max_blocks;
   a.num_blocks = L.num_blocks;
   a.cs = L.scale * 1.4426950408889634f;
+  a.ring = L.ring;
+  a.part = nullptr;
+  a.streamk = 0;
 
 
   // Windows of 128, 256, 512 or 1024 keys: the fused single-exponential kernel on clusters of

@@ -85,6 +85,13 @@ _SIGNATURES = {
     "kara_last_error": ([], ctypes.c_char_p),
     "kara_launch_count": ([], ctypes.c_uint64),
     "kara_wait_probe": ([_I, _P, _P], _I),
+    "kara_score_ring": ([_P, _P, ctypes.POINTER(_Pool), _P, _I, _I, _I, _F, _P, _P, _Z, _P, _P],
+                        _I),
+    "kara_decode_append": ([_P, _P, _P, _P, _P, ctypes.POINTER(_Pool), _I, _F, _P, _I, _P, _P, _Z,
+                            _P, _P], _I),
+    "kara_step_begin": ([ctypes.POINTER(_Pool), _P, _P], _I),
+    "kara_step_end": ([ctypes.POINTER(_Pool), _P, _I, _I, _P, _P, _P], _I),
+    "kara_reset_tails": ([_P, _P, _I, _I, _P], _I),
 }
 
 
@@ -339,6 +346,89 @@ def paged_decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Ten
                                    float(scale), _ptr(out), _ptr(ws), ws.numel(), _ptr(status),
                                    _stream(stream)), "paged_decode_attn")
     return out
+
+
+def kara_score_ring(q_ring: torch.Tensor, k_cache: torch.Tensor, pool: PagedPool, window: int,
+                    seq_ids: torch.Tensor, num_seqs: int, scale: float | None = None,
+                    scores: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                    status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Window scores [num_seqs, Hkv, W] fp32 with the queries read from the window-query ring
+    q_ring [B, 2W, Hq, d] (see kara_score_ring in include/kara.h)."""
+    _require(q_ring, torch.bfloat16, "q_ring")
+    _require(k_cache, torch.bfloat16, "k_cache")
+    _require(seq_ids, torch.int32, "seq_ids")
+    b, rows, hq, d = q_ring.shape
+    if rows != 2 * window:
+        raise ValueError("q_ring's second dimension must be 2 * window")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if scores is None:
+        scores = torch.empty((num_seqs, pool.num_kv_heads, window), dtype=torch.float32,
+                             device=q_ring.device)
+    _require(scores, torch.float32, "scores")
+    status = status if status is not None else new_status(q_ring.device)
+    ps = pool.c_struct()
+    ws = _workspace(kara_workspace_bytes(OP_SCORE, pool, num_seqs, window, hq), q_ring.device,
+                    workspace)
+    _check(lib().kara_score_ring(_ptr(q_ring), _ptr(k_cache), ctypes.byref(ps), _ptr(seq_ids),
+                                 num_seqs, window, hq, float(scale), _ptr(scores), _ptr(ws),
+                                 ws.numel(), _ptr(status), _stream(stream)), "kara_score_ring")
+    return scores
+
+
+def kara_decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                       k_cache: torch.Tensor, v_cache: torch.Tensor, pool: PagedPool,
+                       q_ring: torch.Tensor | None = None, window: int = 0,
+                       scale: float | None = None, out: torch.Tensor | None = None,
+                       workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """One layer of a decode step, fused: attention of the new token (slot ctx_len) over the
+    cache and itself, its K/V written to the cache and its query to the ring. out [B, Hq, d]."""
+    for t, name in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"),
+                    (v_cache, "v_cache")):
+        _require(t, torch.bfloat16, name)
+    if q_ring is not None:
+        _require(q_ring, torch.bfloat16, "q_ring")
+    b, hq, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    _require(out, torch.bfloat16, "out")
+    status = status if status is not None else new_status(q.device)
+    ps = pool.c_struct()
+    ws = _workspace(kara_workspace_bytes(OP_DECODE, pool, 0, 0, hq, 0), q.device, workspace)
+    _check(lib().kara_decode_append(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                    _ptr(v_cache), ctypes.byref(ps), hq, float(scale),
+                                    _ptr(q_ring), int(window), _ptr(out), _ptr(ws), ws.numel(),
+                                    _ptr(status), _stream(stream)), "kara_decode_append")
+    return out
+
+
+def kara_step_begin(pool: PagedPool, status: torch.Tensor, stream=None) -> None:
+    """Blocks for the slots a decode step appends (see include/kara.h)."""
+    ps = pool.c_struct()
+    _check(lib().kara_step_begin(ctypes.byref(ps), _ptr(status), _stream(stream)),
+           "kara_step_begin")
+
+
+def kara_step_end(pool: PagedPool, tail: torch.Tensor | None = None, window: int = 0,
+                  check: bool = False, due: torch.Tensor | None = None,
+                  due_count: torch.Tensor | None = None, stream=None) -> None:
+    """ctx_len + 1 and tail + 1; on a check step the due sequences and their count."""
+    if tail is not None:
+        _require(tail, torch.int32, "tail")
+    ps = pool.c_struct()
+    _check(lib().kara_step_end(ctypes.byref(ps), _ptr(tail), int(window), 1 if check else 0,
+                               _ptr(due), _ptr(due_count), _stream(stream)), "kara_step_end")
+
+
+def kara_reset_tails(tail: torch.Tensor, seq_ids: torch.Tensor, num_seqs: int,
+                     stream=None) -> None:
+    _require(tail, torch.int32, "tail")
+    _require(seq_ids, torch.int32, "seq_ids")
+    _check(lib().kara_reset_tails(_ptr(tail), _ptr(seq_ids), int(num_seqs), int(tail.numel()),
+                                  _stream(stream)), "kara_reset_tails")
 
 
 def lacache_compact(k_layers, v_layers, pool: PagedPool, span: int, overlap: int, rung: int,

@@ -229,6 +229,83 @@ kara_status paged_decode_attn(const void* q, const void* k_cache, const void* v_
                               cudaStream_t stream);
 
 /*
+ * The decode loop around the compression calls ([KARA] abstract: compression happens during
+ * decoding, on the recently generated context, instead of on a fill threshold; [GIST]
+ * section 3 "Der 'Periodische' Zeitplan (KvLLM)": on a fixed schedule, every 100 steps, the
+ * oldest part of the current reasoning of some selected requests is cleaned up). One decode
+ * step, for a batch of `pool->batch` sequences:
+ *
+ *   kara_step_begin                        blocks for the slots the step appends
+ *   for every layer: kara_decode_append    attention of the new token, which joins the cache
+ *   kara_step_end                          ctx_len + 1; on a check step, the due sequences
+ *
+ * and on a check step with due sequences: kara_score_ring (per layer), kara_select,
+ * kara_token2chunk, kara_compact (all layers), kara_reset_tails. State beyond the pool:
+ * tail (device int32 [batch], the tokens appended since the sequence's last compression,
+ * zero at the start) and, per layer, a window-query ring q_ring (bf16 [batch, 2W, Hq, d]):
+ * the query of the token at slot s is kept at rows s mod W and s mod W + W, so the queries
+ * of the window [n-W, n) are the W contiguous rows from (n-W) mod W. A due sequence (tail >= W
+ * at a check step) is compressed over its last W slots; tail then returns to 0.
+ */
+
+/*
+ * kara_step_begin - before the layers of a decode step: every sequence whose next slot
+ * n = ctx_len[b] starts a page (n % 16 == 0) takes the block of page n/16 from the top of
+ * the free list (stack[top-1] first, sequences in ascending order), written into its table.
+ * Device-checked, all or nothing: n < 0 or n >= 16 * max_blocks_per_seq gives
+ * KARA_ERR_INVALID_ARG, fewer free blocks than sequences that need one gives
+ * KARA_ERR_OUT_OF_BLOCKS; then nothing changes. Needs pool->free_list and free_top.
+ */
+kara_status kara_step_begin(const kara_pool* pool, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * kara_decode_append - one layer of a decode step, fused: the attention of the new token and
+ * its entry into the cache and the window-query ring.
+ *
+ *     out[b][h] = sum_{t <= n} softmax_t( q[b][h] . K[t][g(h)] * scale ) V[t][g(h)]
+ * with n = ctx_len[b] (not changed here) and slot n = the new token: K[n] = k_new[b],
+ * V[n] = v_new[b]. Slot n is written into k_cache / v_cache (its block taken by
+ * kara_step_begin), and q[b] into rows n mod window and n mod window + window of q_ring.
+ *  q, out        bf16 [batch, num_q_heads, head_dim]; k_new, v_new bf16 [batch, Hkv, head_dim].
+ *  q_ring        bf16 [batch, 2*window, num_q_heads, head_dim] or NULL (no ring).
+ *  workspace     >= kara_workspace_bytes(KARA_OP_DECODE, ...).
+ *  dev_status    as paged_decode_attn; KARA_ERR_INVALID_ARG if slot n is past the table,
+ *                KARA_ERR_BAD_BLOCK if its block id is out of range (the write is skipped).
+ */
+kara_status kara_decode_append(const void* q, const void* k_new, const void* v_new,
+                               void* k_cache, void* v_cache, const kara_pool* pool,
+                               int32_t num_q_heads, float scale, void* q_ring, int32_t window,
+                               void* out, void* workspace, size_t workspace_bytes,
+                               int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * kara_step_end - after the layers of a decode step: ctx_len[b] += 1 and tail[b] += 1 for
+ * every sequence (tail may be NULL when check == 0). On a check step (check != 0): the
+ * sequences with tail[b] >= window, ascending, go to due (device int32 [batch]) and their
+ * number to due_count (device int32 [1]); the caller reads the count to size the compression.
+ */
+kara_status kara_step_end(const kara_pool* pool, int32_t* tail, int32_t window, int32_t check,
+                          int32_t* due, int32_t* due_count, cudaStream_t stream);
+
+/*
+ * kara_score_ring - kara_score with the window queries read from the window-query ring:
+ * window position i of due sequence r (cache row b = seq_ids ? seq_ids[r] : r, n = ctx_len[b])
+ * is q_ring[b][(n - window) mod window + i]. q_ring bf16 [batch, 2*window, num_q_heads,
+ * head_dim]; every other argument, the output and the errors as kara_score.
+ */
+kara_status kara_score_ring(const void* q_ring, const void* k_cache, const kara_pool* pool,
+                            const int32_t* seq_ids, int32_t num_seqs, int32_t window,
+                            int32_t num_q_heads, float scale, float* scores, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * kara_reset_tails - tail[seq_ids[i]] = 0 for i < num_seqs (after their compression); ids
+ * outside [0, batch) are skipped.
+ */
+kara_status kara_reset_tails(int32_t* tail, const int32_t* seq_ids, int32_t num_seqs,
+                             int32_t batch, cudaStream_t stream);
+
+/*
  * lacache_compact - one pass of LaCache's ladder compaction ([LAC] ladder pattern and
  * iterative compaction) through the same paged gather as kara_compact.
  *

@@ -62,6 +62,17 @@ def test_host_side_validation_returns_before_any_launch(lib_path):
     # compaction window above KARA_MAX_WINDOW
     assert L.kara_compact(layers, 1, ctypes.byref(pool), null, 1, 5000, 8, one, one, 1 << 20, one,
                           null) == K.ERR_INVALID_ARG
+    # decode loop: a check step needs the tail and due buffers; the fused step needs the new
+    # token; a ring needs a window in range; negative counts
+    assert L.kara_step_end(ctypes.byref(pool), null, 16, 1, one, one, null) == K.ERR_INVALID_ARG
+    assert L.kara_decode_append(one, null, one, one, one, ctypes.byref(pool), 4, 1.0, null, 0, one,
+                                one, 1 << 20, one, null) == K.ERR_INVALID_ARG
+    assert L.kara_decode_append(one, one, one, one, one, ctypes.byref(pool), 4, 1.0, one, 0, one,
+                                one, 1 << 20, one, null) == K.ERR_INVALID_ARG
+    assert L.kara_reset_tails(one, one, -1, 4, null) == K.ERR_INVALID_ARG
+    assert L.kara_reset_tails(one, one, 0, 4, null) == K.OK             # nothing to reset
+    assert L.kara_score_ring(one, one, ctypes.byref(pool), null, 1, 5000, 4, 1.0, one, one,
+                             1 << 20, one, null) == K.ERR_INVALID_ARG
     # none of these reached a kernel launch
     assert K.kara_launch_count() == launches
 
