@@ -375,6 +375,92 @@ def lacache_run(dev, batch: int, reps: int = 5, warmup: int = 3) -> dict:
                         f"caches, S=8, O=4, rung 64, budget 8192 per layer; one pass (all layers)"}
 
 
+def decode_loop_run(dev, steps: int = 300, period: int = 100, warm: int = 20) -> dict:
+    """The decode loop on the layer workload's shapes (batch 32, 28 query / 4 KV heads, d=128,
+    4096-token contexts, W=1024, keep 204, one layer): every step kara_step_begin,
+    kara_decode_append and kara_step_end; every `period` steps the due sequences (tail >= W)
+    are compressed (kara_score_ring, kara_select, kara_token2chunk, kara_compact,
+    kara_reset_tails). Tails start spread over [0, W) and the query ring holds seeded queries,
+    as in the middle of a generation. Timed with CUDA events per step; a check step includes
+    the host read of the due count that sizes its compression."""
+    from decode_kv_cache_kara_b200 import kara as K
+    wl = WORKLOAD
+    W, B = wl.window, wl.batch
+    cache = synth.make_cache(wl, 1234 + 5, dev, with_queries=False,
+                             extra_pages=(steps + warm) // wl.page + 2)
+    pool = K.PagedPool.from_cache(cache)
+    k0, v0 = cache["k"][0], cache["v"][0]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + 6)
+    ring = torch.randn((B, 2 * W, wl.hq, wl.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+    tail = torch.randint(0, W, (B,), generator=gen, device=dev, dtype=torch.int32)
+    inputs = [[torch.randn(shape, generator=gen, device=dev).to(torch.bfloat16)
+               for shape in ((B, wl.hq, wl.head_dim), (B, wl.hkv, wl.head_dim),
+                             (B, wl.hkv, wl.head_dim))] for _ in range(16)]
+    out = torch.empty((B, wl.hq, wl.head_dim), dtype=torch.bfloat16, device=dev)
+    ws_dec = torch.empty(K.kara_workspace_bytes(K.OP_DECODE, pool, 0, 0, wl.hq, 0),
+                         dtype=torch.uint8, device=dev)
+    ws_sc = torch.empty(K.kara_workspace_bytes(K.OP_SCORE, pool, B, W, wl.hq), dtype=torch.uint8,
+                        device=dev)
+    ws_cp = torch.empty(K.kara_workspace_bytes(K.OP_COMPACT, pool, B, W, 0, wl.keep),
+                        dtype=torch.uint8, device=dev)
+    scores = torch.empty((B, wl.hkv, W), dtype=torch.float32, device=dev)
+    sel = torch.empty((B, wl.hkv, wl.keep), dtype=torch.int32, device=dev)
+    keep = torch.empty((1, B, wl.hkv, wl.keep), dtype=torch.int32, device=dev)
+    due = torch.zeros(B, dtype=torch.int32, device=dev)
+    due_count = torch.zeros(1, dtype=torch.int32, device=dev)
+    status = K.new_status(dev)
+    na = K.anchors_for(wl.anchor_frac, wl.keep)
+
+    def step(t, check):
+        q, kn, vn = inputs[t % len(inputs)]
+        K.kara_step_begin(pool, status)
+        K.kara_decode_append(q, kn, vn, k0, v0, pool, ring, W, out=out, workspace=ws_dec,
+                             status=status)
+        K.kara_step_end(pool, tail, W, check, due, due_count)
+        if not check:
+            return 0
+        cnt = int(due_count.item())
+        if cnt:
+            seq = due[:cnt]
+            K.kara_score_ring(ring, k0, pool, W, seq, cnt, scores=scores[:cnt], workspace=ws_sc,
+                              status=status)
+            K.kara_select(scores[:cnt], wl.keep, sel=sel[:cnt])
+            K.kara_token2chunk(scores[:cnt], sel[:cnt], na, wl.gap_limit, wl.widen,
+                               keep=keep[0, :cnt])
+            K.kara_compact([k0], [v0], pool, W, keep[:, :cnt], seq_ids=seq, workspace=ws_cp,
+                           status=status)
+            K.kara_reset_tails(tail, seq, cnt)
+        return cnt
+
+    for t in range(warm):
+        step(t, False)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    dues, checks = [], []
+    for t in range(steps):
+        check = (t + 1) % period == 0
+        ev[t][0].record()
+        n = step(warm + t, check)
+        ev[t][1].record()
+        if check:
+            dues.append(n)
+            checks.append(t)
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    plain = sorted(m for t, m in enumerate(ms) if t not in checks)
+    st = K.read_status(status)
+    total = sum(ms)
+    return {"steps": steps, "period": period, "ms_per_step": total / steps,
+            "decode_step_ms": plain[len(plain) // 2],
+            "check_step_ms": [ms[t] for t in checks], "due_per_check": dues,
+            "tokens_per_s": B * steps / (total / 1e3), "status": st,
+            "workload": f"decode loop: batch {B}, 28 query / 4 KV heads, d=128, 4096-token "
+                        f"contexts, W={W}, keep {wl.keep}, one layer, check every {period} "
+                        f"steps, tails spread over [0, W)"}
+
+
 def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
     import torch.distributed as dist
     from decode_kv_cache_kara_b200 import kara as K
@@ -479,6 +565,8 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
         lac = lacache_run(dev, args.lacache_batch)
         lac["frac_of_hbm_" + src] = lac["gbs"] / peaks["hbm_gbs"]
         kernels["lacache_compact"] = lac
+    if world == 1 and not args.no_loop:
+        kernels["decode_loop"] = decode_loop_run(dev)
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -569,6 +657,8 @@ def main():
     ap.add_argument("--no-lacache", action="store_true",
                     help="skip the LaCache ladder-compaction measurement (1 GPU only)")
     ap.add_argument("--lacache-batch", type=int, default=8)
+    ap.add_argument("--no-loop", action="store_true",
+                    help="skip the decode-loop measurement (kernels.decode_loop)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
