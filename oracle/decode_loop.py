@@ -26,6 +26,11 @@ Readings taken where the pages are silent (each one is used identically by the C
   calls take, and its tail returns to 0 after the compression. With a check every step the
   window is exactly the uncompressed tail; with a longer period up to period - 1 older
   uncompressed tokens stay where they are.
+* LaCache in the same loop ("LaCache: Ladder-Shaped KV Caching ...", iterative compaction:
+  the ladder is applied again whenever the cache fills up; experimental setup: a fixed
+  budget per layer): at a check step a sequence is also due when its length reaches the
+  capacity sink + recent + R_max, the length at which one ladder pass keeps exactly the
+  budget in every layer; the pass then runs over its whole cache (lacache.lacache_compact).
 * The window queries come from a per-sequence ring of 2W rows per layer: the query of the
   token at slot s is stored at rows s mod W and s mod W + W, so the queries of slots
   [n-W, n) are rows (n-W) mod W .. (n-W) mod W + W - 1, contiguous.
@@ -90,11 +95,15 @@ def decode_append(q: np.ndarray, k_new: np.ndarray, v_new: np.ndarray, k_pool: n
     return out, kp, vp, ring
 
 
-def step_end(ctx_len: np.ndarray, tail: np.ndarray, window: int, check: bool):
-    """ctx_len + 1, tail + 1, and on a check step the due sequences (ascending): tail >= W."""
+def step_end(ctx_len: np.ndarray, tail: np.ndarray | None, window: int, check: bool,
+             capacity: int = 0):
+    """ctx_len + 1, tail + 1, and on a check step the due sequences (ascending): tail >= W
+    (when W > 0, Kara) or ctx_len >= capacity (when capacity > 0, LaCache)."""
     cl = ctx_len + 1
-    tl = tail + 1
-    due = [b for b in range(len(cl)) if check and int(tl[b]) >= window]
+    tl = None if tail is None else tail + 1
+    due = [b for b in range(len(cl))
+           if check and ((window > 0 and tl is not None and int(tl[b]) >= window)
+                         or (capacity > 0 and int(cl[b]) >= capacity))]
     return cl, tl, due
 
 

@@ -11,6 +11,7 @@ import pytest
 from decode_kv_cache_kara_b200 import synth
 from oracle import decode_loop as dl
 from oracle import kara as ok
+from oracle import lacache as ol
 
 LOOP = synth.Workload("loop", batch=3, layers=2, hq=4, hkv=2, head_dim=16, ctx_lo=20, ctx_hi=37,
                       window=16, keep=5, heavy_frac=0.0, spare_blocks=4)
@@ -148,3 +149,82 @@ def test_trigger_and_ring_rows():
         ring[0, s % W, 0, 0] = ring[0, s % W + W, 0, 0] = s
     win = dl.window_queries(ring, np.array([13]), [0], W)
     assert list(win[0, :, 0, 0]) == [9, 10, 11, 12]
+
+
+def test_trigger_capacity():
+    cl, tl, due = dl.step_end(np.array([38, 39, 40]), None, 0, check=True, capacity=40)
+    assert tl is None and list(cl) == [39, 40, 41] and due == [1, 2]
+    _, _, due = dl.step_end(np.array([38, 39, 40]), None, 0, check=False, capacity=40)
+    assert due == []
+
+
+LAC_LOOP = synth.Workload("lacloop", batch=3, layers=4, hq=4, hkv=2, head_dim=16, ctx_lo=20,
+                          ctx_hi=35, window=0, keep=0, spare_blocks=4)
+LAC = dict(span=2, overlap=1, rung=4, budget=24, sink=4, recent=4)
+
+
+def test_lacache_loop_matches_dense_model():
+    """LaCache inside the decode loop: at check steps every sequence that reached the capacity
+    is laddered over its whole cache. The dense model keeps, per layer, the slots that
+    ladder_keep_slots names, by list surgery."""
+    wl, seed, steps, period = LAC_LOOP, 4, 60, 4
+    assert ol.check_params(wl.layers, LAC["span"], LAC["overlap"], LAC["rung"], LAC["budget"],
+                           LAC["sink"], LAC["recent"])
+    cap = LAC["sink"] + LAC["recent"] + ol.region_capacity(wl.layers, LAC["span"], LAC["budget"],
+                                                          LAC["sink"], LAC["recent"])
+    cache = synth.make_cache(wl, seed, "cpu", with_queries=False, extra_pages=6)
+    page, L, G = wl.page, wl.layers, wl.group
+    scale = 1 / math.sqrt(wl.head_dim)
+    kp = [np32(t) for t in cache["k"]]
+    vp = [np32(t) for t in cache["v"]]
+    bt = cache["block_table"].numpy().astype(np.int64)
+    cl = cache["ctx_len"].numpy().astype(np.int64)
+    fl = cache["free_list"].numpy().astype(np.int64)
+    top = int(cache["free_top"][0])
+    dk = [[[kp[l][bt[b, s // page], s % page] for s in range(cl[b])] for b in range(wl.batch)]
+          for l in range(L)]
+    dv = [[[vp[l][bt[b, s // page], s % page] for s in range(cl[b])] for b in range(wl.batch)]
+          for l in range(L)]
+    passes = 0
+    for t in range(steps):
+        st, bt, top = dl.step_begin(bt, cl, fl, top, page)
+        assert st == dl.OK
+        for l in range(L):
+            inp = synth.decode_step_inputs(wl, seed, t, layers=L)[l]
+            q, kn, vn = np32(inp["q"]), np32(inp["k"]), np32(inp["v"])
+            out, kp[l], vp[l], _ = dl.decode_append(q, kn, vn, kp[l], vp[l], bt, cl, scale,
+                                                    page, None, 1)
+            for b in range(wl.batch):
+                dk[l][b].append(kn[b])
+                dv[l][b].append(vn[b])
+                for h in range(wl.hq):
+                    rows_k = [r[h // G] for r in dk[l][b]]
+                    rows_v = [r[h // G] for r in dv[l][b]]
+                    assert np.allclose(out[b, h], dense_attention(q[b, h], rows_k, rows_v, scale),
+                                       rtol=1e-12, atol=1e-12)
+        cl, _, due = dl.step_end(cl, None, 0, (t + 1) % period == 0, capacity=cap)
+        assert all(int(cl[b]) >= cap for b in due)
+        if due:
+            st, kp, vp, bt, cl2, fl, top = ol.lacache_compact(
+                kp, vp, bt, cl, fl, top, due, LAC["span"], LAC["overlap"], LAC["rung"],
+                LAC["budget"], LAC["sink"], LAC["recent"], page)
+            assert st == ol.OK
+            for b in due:
+                n = int(cl[b])
+                for l in range(L):
+                    slots = ol.ladder_keep_slots(n, L, LAC["span"], LAC["overlap"], LAC["rung"],
+                                                 LAC["budget"], LAC["sink"], LAC["recent"])[l]
+                    dk[l][b] = [dk[l][b][int(x)] for x in slots]
+                    dv[l][b] = [dv[l][b][int(x)] for x in slots]
+                assert int(cl2[b]) == LAC["budget"]
+            cl = cl2
+            passes += len(due)
+        for l in range(L):
+            for b in range(wl.batch):
+                assert len(dk[l][b]) == cl[b]
+                for s in range(int(cl[b])):
+                    assert np.array_equal(kp[l][bt[b, s // page], s % page], dk[l][b][s])
+                    assert np.array_equal(vp[l][bt[b, s // page], s % page], dv[l][b][s])
+        used = [int(x) for x in bt[bt >= 0].ravel()]
+        assert sorted(used + [int(x) for x in fl[:top]]) == list(range(cache["num_blocks"]))
+    assert passes >= 2 * wl.batch       # every sequence laddered at least twice
