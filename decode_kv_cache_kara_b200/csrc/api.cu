@@ -300,14 +300,17 @@ kara_status kara_step_begin(const kara_pool* pool, int32_t* dev_status, cudaStre
   return launch_step_begin(pool, dev_status, stream);
 }
 
-kara_status kara_step_end(const kara_pool* pool, int32_t* tail, int32_t window, int32_t check,
-                          int32_t* due, int32_t* due_count, cudaStream_t stream) {
+kara_status kara_step_end(const kara_pool* pool, int32_t* tail, int32_t window,
+                          int32_t capacity, int32_t check, int32_t* due, int32_t* due_count,
+                          cudaStream_t stream) {
   kara_status st = check_pool(pool);
   if (st != KARA_OK) return st;
-  if (check != 0 && (tail == nullptr || due == nullptr || due_count == nullptr || window < 1))
+  if (window < 0 || capacity < 0 || (window > 0 && tail == nullptr)) return KARA_ERR_INVALID_ARG;
+  if (check != 0 && (due == nullptr || due_count == nullptr || (window == 0 && capacity == 0)))
     return KARA_ERR_INVALID_ARG;
   if (pool->batch == 0) return KARA_OK;
-  return launch_step_end(pool, tail, window, check != 0 ? 1 : 0, due, due_count, stream);
+  return launch_step_end(pool, tail, window, capacity, check != 0 ? 1 : 0, due, due_count,
+                         stream);
 }
 
 kara_status kara_reset_tails(int32_t* tail, const int32_t* seq_ids, int32_t num_seqs,

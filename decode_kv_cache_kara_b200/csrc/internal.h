@@ -131,8 +131,9 @@ int decode_num_splits(int max_blocks);
 size_t decode_workspace_bytes(int B, int Hq, int D, int max_blocks);
 kara_status launch_decode(const DecodeLaunch& L, cudaStream_t stream);
 kara_status launch_step_begin(const kara_pool* pool, int32_t* dev_status, cudaStream_t stream);
-kara_status launch_step_end(const kara_pool* pool, int32_t* tail, int32_t window, int32_t check,
-                            int32_t* due, int32_t* due_count, cudaStream_t stream);
+kara_status launch_step_end(const kara_pool* pool, int32_t* tail, int32_t window,
+                            int32_t capacity, int32_t check, int32_t* due, int32_t* due_count,
+                            cudaStream_t stream);
 kara_status launch_reset_tails(int32_t* tail, const int32_t* seq_ids, int32_t num_seqs,
                                int32_t batch, cudaStream_t stream);
 

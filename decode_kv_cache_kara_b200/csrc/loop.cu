@@ -8,6 +8,9 @@
 // of the current reasoning of some selected requests is cleaned up. Here a sequence is due at
 // a check step when the tokens appended since its last compression (its tail) reach the
 // window W; its window is then its last W slots, the window of kara_score / kara_compact.
+// LaCache in the same loop ("LaCache: Ladder-Shaped KV Caching ...", iterative compaction with
+// a fixed budget per layer): a sequence is due when its length reaches the capacity
+// sink + recent + R_max, at which one ladder pass keeps exactly the budget in every layer.
 //
 // One CTA of 1024 threads per call: the counts are one int per sequence, and allocation in
 // ascending sequence order is a block-wide prefix sum.
@@ -31,7 +34,7 @@ struct LoopArgs {
   int32_t* due;         // check steps: ascending due sequences
   int32_t* due_count;
   int32_t* status;
-  int B, max_blocks, num_blocks, window, check;
+  int B, max_blocks, num_blocks, window, capacity, check;
 };
 
 // Sequences whose next slot n = ctx_len starts a page take the block for page n / 16, in
@@ -78,7 +81,7 @@ __global__ void __launch_bounds__(kLoopThreads) step_begin_kernel(const LoopArgs
 }
 
 // ctx_len += 1 and tail += 1 for every sequence; on a check step the sequences with
-// tail >= W, ascending, and their count.
+// tail >= W (W > 0) or ctx_len >= capacity (capacity > 0), ascending, and their count.
 __global__ void __launch_bounds__(kLoopThreads) step_end_kernel(const LoopArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ int buf[33];
@@ -87,12 +90,14 @@ __global__ void __launch_bounds__(kLoopThreads) step_end_kernel(const LoopArgs a
     const int b = base + static_cast<int>(threadIdx.x);
     int is_due = 0;
     if (b < a.B) {
-      a.ctx_len[b] += 1;
+      const int n = a.ctx_len[b] + 1;
+      a.ctx_len[b] = n;
       if (a.tail != nullptr) {
         const int t = a.tail[b] + 1;
         a.tail[b] = t;
-        is_due = a.check && t >= a.window ? 1 : 0;
+        is_due = a.check && a.window > 0 && t >= a.window ? 1 : 0;
       }
+      if (a.check && a.capacity > 0 && n >= a.capacity) is_due = 1;
     }
     if (a.check) {
       int chunk;
@@ -128,8 +133,9 @@ kara_status launch_step_begin(const kara_pool* pool, int32_t* dev_status, cudaSt
   return check_launch("kara_step_begin");
 }
 
-kara_status launch_step_end(const kara_pool* pool, int32_t* tail, int32_t window, int32_t check,
-                            int32_t* due, int32_t* due_count, cudaStream_t stream) {
+kara_status launch_step_end(const kara_pool* pool, int32_t* tail, int32_t window,
+                            int32_t capacity, int32_t check, int32_t* due, int32_t* due_count,
+                            cudaStream_t stream) {
   LoopArgs a = {};
   a.ctx_len = pool->ctx_len;
   a.tail = tail;
@@ -137,6 +143,7 @@ kara_status launch_step_end(const kara_pool* pool, int32_t* tail, int32_t window
   a.due_count = due_count;
   a.B = pool->batch;
   a.window = window;
+  a.capacity = capacity;
   a.check = check;
   launch_pdl(step_end_kernel, dim3(1), dim3(kLoopThreads), 0, stream, a);
   return check_launch("kara_step_end");

@@ -90,7 +90,7 @@ _SIGNATURES = {
     "kara_decode_append": ([_P, _P, _P, _P, _P, ctypes.POINTER(_Pool), _I, _F, _P, _I, _P, _P, _Z,
                             _P, _P], _I),
     "kara_step_begin": ([ctypes.POINTER(_Pool), _P, _P], _I),
-    "kara_step_end": ([ctypes.POINTER(_Pool), _P, _I, _I, _P, _P, _P], _I),
+    "kara_step_end": ([ctypes.POINTER(_Pool), _P, _I, _I, _I, _P, _P, _P], _I),
     "kara_reset_tails": ([_P, _P, _I, _I, _P], _I),
 }
 
@@ -414,13 +414,16 @@ def kara_step_begin(pool: PagedPool, status: torch.Tensor, stream=None) -> None:
 
 def kara_step_end(pool: PagedPool, tail: torch.Tensor | None = None, window: int = 0,
                   check: bool = False, due: torch.Tensor | None = None,
-                  due_count: torch.Tensor | None = None, stream=None) -> None:
-    """ctx_len + 1 and tail + 1; on a check step the due sequences and their count."""
+                  due_count: torch.Tensor | None = None, capacity: int = 0,
+                  stream=None) -> None:
+    """ctx_len + 1 and tail + 1; on a check step the due sequences (tail >= window, or
+    ctx_len >= capacity) and their count."""
     if tail is not None:
         _require(tail, torch.int32, "tail")
     ps = pool.c_struct()
-    _check(lib().kara_step_end(ctypes.byref(ps), _ptr(tail), int(window), 1 if check else 0,
-                               _ptr(due), _ptr(due_count), _stream(stream)), "kara_step_end")
+    _check(lib().kara_step_end(ctypes.byref(ps), _ptr(tail), int(window), int(capacity),
+                               1 if check else 0, _ptr(due), _ptr(due_count), _stream(stream)),
+           "kara_step_end")
 
 
 def kara_reset_tails(tail: torch.Tensor, seq_ids: torch.Tensor, num_seqs: int,

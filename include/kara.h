@@ -279,13 +279,18 @@ kara_status kara_decode_append(const void* q, const void* k_new, const void* v_n
                                int32_t* dev_status, cudaStream_t stream);
 
 /*
- * kara_step_end - after the layers of a decode step: ctx_len[b] += 1 and tail[b] += 1 for
- * every sequence (tail may be NULL when check == 0). On a check step (check != 0): the
- * sequences with tail[b] >= window, ascending, go to due (device int32 [batch]) and their
- * number to due_count (device int32 [1]); the caller reads the count to size the compression.
+ * kara_step_end - after the layers of a decode step: ctx_len[b] += 1, and tail[b] += 1 when
+ * tail is not NULL. On a check step (check != 0) a sequence is due when tail[b] >= window
+ * (window > 0: Kara's tail-W trigger; tail required) or when ctx_len[b] >= capacity
+ * (capacity > 0: LaCache's full cache, capacity = sink + recent + R_max of the ladder, after
+ * which lacache_compact keeps `budget` slots per layer; [LAC] iterative compaction). The due
+ * sequences, ascending, go to due (device int32 [batch]) and their number to due_count
+ * (device int32 [1]); the caller reads the count to size the compression. window = 0 and
+ * capacity = 0 on a check step is KARA_ERR_INVALID_ARG.
  */
-kara_status kara_step_end(const kara_pool* pool, int32_t* tail, int32_t window, int32_t check,
-                          int32_t* due, int32_t* due_count, cudaStream_t stream);
+kara_status kara_step_end(const kara_pool* pool, int32_t* tail, int32_t window,
+                          int32_t capacity, int32_t check, int32_t* due, int32_t* due_count,
+                          cudaStream_t stream);
 
 /*
  * kara_score_ring - kara_score with the window queries read from the window-query ring:

@@ -64,7 +64,8 @@ def test_host_side_validation_returns_before_any_launch(lib_path):
                           null) == K.ERR_INVALID_ARG
     # decode loop: a check step needs the tail and due buffers; the fused step needs the new
     # token; a ring needs a window in range; negative counts
-    assert L.kara_step_end(ctypes.byref(pool), null, 16, 1, one, one, null) == K.ERR_INVALID_ARG
+    assert L.kara_step_end(ctypes.byref(pool), null, 16, 0, 1, one, one, null) == K.ERR_INVALID_ARG
+    assert L.kara_step_end(ctypes.byref(pool), null, 0, 0, 1, one, one, null) == K.ERR_INVALID_ARG
     assert L.kara_decode_append(one, null, one, one, one, ctypes.byref(pool), 4, 1.0, null, 0, one,
                                 one, 1 << 20, one, null) == K.ERR_INVALID_ARG
     assert L.kara_decode_append(one, one, one, one, one, ctypes.byref(pool), 4, 1.0, one, 0, one,

@@ -161,3 +161,71 @@ def test_step_begin_out_of_blocks_changes_nothing():
     assert K.read_status(status) == K.ERR_OUT_OF_BLOCKS
     assert np.array_equal(H.i32(dev["block_table"]), before)
     assert int(dev["free_top"][0]) == 2
+
+
+def test_lacache_loop_matches_oracle():
+    """LaCache inside the decode loop: at check steps the sequences whose length reached the
+    capacity sink + recent + R_max are laddered over their whole cache (lacache_compact), then
+    decoding goes on; every sequence is laddered at least twice. Outputs, due lists and the
+    whole cache state in lockstep with the oracle."""
+    from oracle import lacache as ol
+    wl = synth.Workload("lacloop", batch=3, layers=4, hq=4, hkv=2, head_dim=64, ctx_lo=20,
+                        ctx_hi=35, window=0, keep=0, spare_blocks=4)
+    lac = dict(span=2, overlap=1, rung=4, budget=24, sink=4, recent=4)
+    seed, steps, period, page, L = 4, 60, 4, wl.page, wl.layers
+    cap = lac["sink"] + lac["recent"] + ol.region_capacity(L, lac["span"], lac["budget"],
+                                                          lac["sink"], lac["recent"])
+    scale = 1 / math.sqrt(wl.head_dim)
+    cpu = synth.make_cache(wl, seed, "cpu", with_queries=False, extra_pages=6)
+    dev = H.to_device(cpu)
+    pool = K.PagedPool.from_cache(dev)
+    status = K.new_status()
+    due = torch.zeros(wl.batch, dtype=torch.int32, device="cuda")
+    due_count = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kp = [f32(t) for t in cpu["k"]]
+    vp = [f32(t) for t in cpu["v"]]
+    bt, cl = H.i32(cpu["block_table"]), H.i32(cpu["ctx_len"])
+    fl, top = H.i32(cpu["free_list"]), int(cpu["free_top"][0])
+    passes = 0
+    for t in range(steps):
+        K.kara_step_begin(pool, status)
+        st, bt, top = dl.step_begin(bt, cl, fl, top, page)
+        assert st == dl.OK
+        inputs = synth.decode_step_inputs(wl, seed, t)
+        for layer in range(L):
+            q, kn, vn = (inputs[layer][x].cuda() for x in ("q", "k", "v"))
+            out = K.kara_decode_append(q, kn, vn, dev["k"][layer], dev["v"][layer], pool,
+                                       status=status)
+            ref, kp[layer], vp[layer], _ = dl.decode_append(f32(q), f32(kn), f32(vn), kp[layer],
+                                                            vp[layer], bt, cl, scale, page, None, 1)
+            assert np.allclose(H.f64(out), ref, atol=2e-2, rtol=1e-2), (t, layer)
+        check = (t + 1) % period == 0
+        K.kara_step_end(pool, None, 0, check, due, due_count, capacity=cap)
+        cl, _, odue = dl.step_end(cl, None, 0, check, capacity=cap)
+        if not check:
+            continue
+        torch.cuda.synchronize()
+        cnt = int(due_count[0])
+        assert list(H.i32(due)[:cnt]) == odue
+        if cnt == 0:
+            continue
+        K.lacache_compact(dev["k"], dev["v"], pool, lac["span"], lac["overlap"], lac["rung"],
+                          lac["budget"], lac["sink"], lac["recent"], seq_ids=due[:cnt],
+                          status=status)
+        torch.cuda.synchronize()
+        assert K.read_status(status) == 0
+        st, kp, vp, bt, cl, fl, top = ol.lacache_compact(
+            kp, vp, bt, cl, fl, top, odue, lac["span"], lac["overlap"], lac["rung"],
+            lac["budget"], lac["sink"], lac["recent"], page)
+        assert st == ol.OK
+        assert np.array_equal(H.i32(dev["block_table"]), bt)
+        assert np.array_equal(H.i32(dev["ctx_len"]), cl)
+        assert int(dev["free_top"][0]) == top
+        assert np.array_equal(H.i32(dev["free_list"])[:top], fl[:top])
+        for layer in range(L):
+            assert rows_equal(f32(dev["k"][layer]), kp[layer], bt, cl, page)
+            assert rows_equal(f32(dev["v"][layer]), vp[layer], bt, cl, page)
+        passes += cnt
+    torch.cuda.synchronize()
+    assert K.read_status(status) == 0
+    assert passes >= 2 * wl.batch
