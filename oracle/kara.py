@@ -28,11 +28,17 @@ Readings taken where the pages are silent (each one is used identically by the C
 * Compaction = deterministic allocation of fresh blocks from a LIFO free list, copy of the
   first window page's prefix rows and of the kept rows, block-table rewrite, free of the old
   window blocks; see ``compact``.
+* Variants the pages leave open (``window_scores_agg``, ``shared_keep``): the mean (the sum
+  over its G * W pairs) and the max (the largest probability any query gives the key) in
+  place of the sum, and one selection per layer shared by its KV heads (selection and
+  Token2Chunk on the head-summed scores).
 
 Parity pins (tests/test_oracle_kara.py): closed forms for two keys, a dominant key (catches a
 transposed sum), equal keys, GQA group mapping, scale, the W*G total, brute force by pairwise
 dominance for selection and trim, hand-worked golden cases, invariants of Token2Chunk and of
-compaction (conservation, untouched blocks). No function here is unpinned.
+compaction (conservation, untouched blocks); for the variants, a brute-force max with its
+bounds, closed forms, the mean against the sum, and the shared selection against the selection
+of the head sum. No function here is unpinned.
 """
 
 from __future__ import annotations
@@ -91,6 +97,40 @@ def window_scores(q_win: np.ndarray, k_win: np.ndarray, scale: float) -> np.ndar
     for h in range(hq):
         out[h // group] += p[h].sum(axis=0)
     return out
+
+
+def window_scores_agg(q_win: np.ndarray, k_win: np.ndarray, scale: float,
+                      agg: str) -> np.ndarray:
+    """Aggregation variants of the window scores, [Hkv, W] (the pages name no aggregation;
+    sum is the main reading, these are the variants it leaves open):
+    "sum"  - window_scores;
+    "mean" - the sum divided by the G * W (query head, window query) pairs it runs over;
+    "max"  - the largest softmax probability any window query of any query head of the group
+             gives the key."""
+    if agg == "sum":
+        return window_scores(q_win, k_win, scale)
+    hq = q_win.shape[1]
+    hkv = k_win.shape[1]
+    group = hq // hkv
+    if agg == "mean":
+        return window_scores(q_win, k_win, scale) / (group * q_win.shape[0])
+    if agg == "max":
+        p = window_probs(q_win, k_win, scale)
+        out = np.zeros((hkv, q_win.shape[0]))
+        for h in range(hq):
+            out[h // group] = np.maximum(out[h // group], p[h].max(axis=0))
+        return out
+    raise ValueError(agg)
+
+
+def shared_keep(scores: np.ndarray, k: int, num_anchors: int, gap_limit: int,
+                widen: int) -> np.ndarray:
+    """A selection shared by the KV heads of a layer (a variant the pages leave open): the
+    per-head scores [Hkv, W] are summed over the heads, selection and Token2Chunk run once on
+    the sum, and every head keeps the same positions. Returns keep [Hkv, k]."""
+    total = scores.sum(axis=0)
+    keep = token2chunk(total, select_topk(total, k), num_anchors, gap_limit, widen)
+    return np.repeat(keep[None, :], scores.shape[0], axis=0)
 
 
 def score_batch(q_win: np.ndarray, k_pool: np.ndarray, block_table: np.ndarray,

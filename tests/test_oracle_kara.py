@@ -374,3 +374,60 @@ def test_compact_out_of_blocks_changes_nothing():
     st, kp, vp, bt, cl, fl, top, _ = ok.compact(ks, vs, table, ctx, free, 0, [0], 12, keep, page)
     assert st == ok.ERR_OUT_OF_BLOCKS
     assert (bt == table).all() and (cl == ctx).all() and top == 0
+
+
+# ---- aggregation variants and the shared selection (variants the pages leave open) ----
+
+def _rand_window(seed, w=9, hq=4, hkv=2, d=8):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((w, hq, d)), rng.standard_normal((w, hkv, d))
+
+
+def test_mean_is_the_sum_over_its_pairs():
+    q, k = _rand_window(1)
+    s = ok.window_scores(q, k, 0.5)
+    m = ok.window_scores_agg(q, k, 0.5, "mean")
+    assert np.allclose(m * (2 * 9), s, rtol=1e-13)
+    assert np.allclose(m.sum(axis=1), 1.0, rtol=1e-12)     # the mean of softmax rows sums to 1
+
+
+def test_max_brute_force_and_bounds():
+    q, k = _rand_window(2, w=6, hq=4, hkv=2, d=5)
+    mx = ok.window_scores_agg(q, k, 0.7, "max")
+    for g in range(2):
+        for j in range(6):
+            best = 0.0
+            for h in (2 * g, 2 * g + 1):
+                for i in range(6):
+                    logits = [float(q[i, h] @ k[jj, g]) * 0.7 for jj in range(6)]
+                    top = max(logits)
+                    den = sum(math.exp(x - top) for x in logits)
+                    best = max(best, math.exp(logits[j] - top) / den)
+            assert abs(mx[g, j] - best) < 1e-13
+    s = ok.window_scores(q, k, 0.7)
+    assert np.all(mx <= s + 1e-15) and np.all(mx >= s / (2 * 6) - 1e-15)
+
+
+def test_max_closed_forms():
+    # equal keys: every probability is 1/W
+    q = np.random.default_rng(3).standard_normal((5, 2, 4))
+    k = np.ones((5, 1, 4))
+    assert np.allclose(ok.window_scores_agg(q, k, 1.0, "max"), 1 / 5)
+    # two keys, one query, one head: max = the logistic probabilities themselves
+    q = np.array([[[1.0, 0.0]], [[0.0, 0.0]]])
+    k = np.array([[[2.0, 0.0]], [[0.0, 0.0]]])
+    p0 = 1 / (1 + math.exp(-2.0))
+    mx = ok.window_scores_agg(q, k, 1.0, "max")
+    assert np.allclose(mx[0], [p0, 0.5])      # query 1 has equal logits: 0.5 for both keys
+
+
+def test_shared_keep_is_the_selection_of_the_head_sum():
+    rng = np.random.default_rng(4)
+    sc = rng.random((3, 40))
+    keep = ok.shared_keep(sc, 8, 4, 8, 1)
+    total = sc.sum(axis=0)
+    ref = ok.token2chunk(total, ok.select_topk(total, 8), 4, 8, 1)
+    assert keep.shape == (3, 8) and all(np.array_equal(row, ref) for row in keep)
+    one = sc[:1]                               # one KV head: the per-head selection itself
+    assert np.array_equal(ok.shared_keep(one, 8, 4, 8, 1)[0],
+                          ok.token2chunk(one[0], ok.select_topk(one[0], 8), 4, 8, 1))
