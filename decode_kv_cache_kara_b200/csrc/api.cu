@@ -74,8 +74,11 @@ kara_status fill_layers(const kara_layer_kv* layers, int32_t num_layers, LayerPt
 
 kara_status score_impl(const void* q_win, int ring, const void* k_cache, const kara_pool* pool,
                        const int32_t* seq_ids, int32_t num_seqs, int32_t window,
-                       int32_t num_q_heads, float scale, float* scores, void* workspace,
-                       size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
+                       int32_t num_q_heads, float scale, int32_t agg, float* scores,
+                       void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                       cudaStream_t stream) {
+  if (agg != KARA_AGG_SUM && agg != KARA_AGG_MEAN && agg != KARA_AGG_MAX)
+    return KARA_ERR_INVALID_ARG;
   kara_status st = check_pool(pool);
   if (st != KARA_OK) return st;
   if ((st = check_heads(pool, num_q_heads)) != KARA_OK) return st;
@@ -106,6 +109,7 @@ kara_status score_impl(const void* q_win, int ring, const void* k_cache, const k
   L.num_blocks = pool->num_blocks;
   L.scale = scale;
   L.ring = ring;
+  L.agg = agg;
   return launch_score_kernels(L, stream);
 }
 
@@ -200,7 +204,34 @@ kara_status kara_score(const void* q_win, const void* k_cache, const kara_pool* 
                        int32_t num_q_heads, float scale, float* scores, void* workspace,
                        size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
   return score_impl(q_win, 0, k_cache, pool, seq_ids, num_seqs, window, num_q_heads, scale,
-                    scores, workspace, workspace_bytes, dev_status, stream);
+                    KARA_AGG_SUM, scores, workspace, workspace_bytes, dev_status, stream);
+}
+
+kara_status kara_score_ex(const void* q, int32_t q_is_ring, const void* k_cache,
+                          const kara_pool* pool, const int32_t* seq_ids, int32_t num_seqs,
+                          int32_t window, int32_t num_q_heads, float scale, int32_t agg,
+                          float* scores, void* workspace, size_t workspace_bytes,
+                          int32_t* dev_status, cudaStream_t stream) {
+  return score_impl(q, q_is_ring != 0 ? 1 : 0, k_cache, pool, seq_ids, num_seqs, window,
+                    num_q_heads, scale, agg, scores, workspace, workspace_bytes, dev_status,
+                    stream);
+}
+
+kara_status kara_sum_heads(const float* scores, int32_t rows, int32_t num_kv_heads,
+                           int32_t window, float* out, cudaStream_t stream) {
+  if (rows < 0 || num_kv_heads < 1 || window < 1 || window > KARA_MAX_WINDOW)
+    return KARA_ERR_INVALID_ARG;
+  if (rows == 0) return KARA_OK;
+  if (scores == nullptr || out == nullptr) return KARA_ERR_INVALID_ARG;
+  return launch_sum_heads(scores, rows, num_kv_heads, window, out, stream);
+}
+
+kara_status kara_expand_keep(const int32_t* keep_shared, int32_t rows, int32_t num_kv_heads,
+                             int32_t k, int32_t* keep, cudaStream_t stream) {
+  if (rows < 0 || num_kv_heads < 1 || k < 1) return KARA_ERR_INVALID_ARG;
+  if (rows == 0) return KARA_OK;
+  if (keep_shared == nullptr || keep == nullptr) return KARA_ERR_INVALID_ARG;
+  return launch_expand_keep(keep_shared, rows, num_kv_heads, k, keep, stream);
 }
 
 kara_status kara_score_ring(const void* q_ring, const void* k_cache, const kara_pool* pool,
@@ -208,7 +239,7 @@ kara_status kara_score_ring(const void* q_ring, const void* k_cache, const kara_
                             int32_t num_q_heads, float scale, float* scores, void* workspace,
                             size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
   return score_impl(q_ring, 1, k_cache, pool, seq_ids, num_seqs, window, num_q_heads, scale,
-                    scores, workspace, workspace_bytes, dev_status, stream);
+                    KARA_AGG_SUM, scores, workspace, workspace_bytes, dev_status, stream);
 }
 
 kara_status kara_select(const float* scores, int32_t rows, int32_t window, int32_t k,

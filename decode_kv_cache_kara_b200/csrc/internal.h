@@ -58,6 +58,7 @@ struct ScoreLaunch {
   int batch, max_blocks, num_blocks;
   float scale;
   int ring = 0;   // q_win is the window-query ring [batch, 2W, Hq, d]
+  int agg = 0;    // KARA_AGG_SUM / MEAN / MAX
 };
 int score_lse_stride(int W);
 int score_chunks(int W);
@@ -66,6 +67,10 @@ kara_status launch_score_kernels(const ScoreLaunch& L, cudaStream_t stream);
 
 kara_status launch_select(const float* scores, int rows, int W, int k, int32_t* sel,
                           cudaStream_t stream);
+kara_status launch_sum_heads(const float* scores, int rows, int hkv, int W, float* out,
+                             cudaStream_t stream);
+kara_status launch_expand_keep(const int32_t* keep_shared, int rows, int hkv, int k,
+                               int32_t* keep, cudaStream_t stream);
 kara_status launch_token2chunk(const float* scores, const int32_t* sel, int rows, int W, int k,
                                int num_anchors, int gap_limit, int widen, int32_t* keep,
                                cudaStream_t stream);

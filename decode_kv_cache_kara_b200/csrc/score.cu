@@ -75,6 +75,7 @@ struct ScoreArgs {
   float* part;      // fused kernel, split items: [split - 1][head part, tail part][W] key sums
   int streamk;      // fused kernel: cluster ranges split items (else they hold whole items)
   int ring;         // queries from the window-query ring [batch, 2W, Hq, d] (else q_win)
+  float out_scale;  // 1, or 1 / (G W) for the mean aggregation
   int32_t* status;
   int R, W, Wp, Hq, Hkv, G;
   int batch, max_blocks, num_blocks;
@@ -478,7 +479,9 @@ __global__ void __launch_bounds__(256) score_lse_merge_kernel(const ScoreArgs a)
 // ----------------------------------------------------------------------------------------
 // Pass 2: per-key sums of the normalised probabilities.
 // ----------------------------------------------------------------------------------------
-template <int D>
+// kMax: the largest probability of each key over the group's queries in place of the sum:
+// max_i 2^(s c - lse_i) = 2^(max_i (s c - lse_i)), one exponential per key.
+template <int D, bool kMax>
 __global__ void __launch_bounds__(kThreads, 1)
 score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
@@ -641,7 +644,8 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (kt == 0 && g == 0 && etid == 0) report(a.status, KARA_ERR_INVALID_ARG);
         continue;
       }
-      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+      const float init = kMax ? -INFINITY : 0.f;
+      float2 acc0 = make_float2(init, init), acc1 = make_float2(init, init);
       // merged lse of the tile's 256 queries, staged negated; the next tile's is prefetched
       const float* lse_rows = a.lse_merged + (static_cast<size_t>(r) * a.Hq + g * a.G) * a.Wp;
       float lv = etid < kQRows2 ? lse_rows[etid] : 0.f;
@@ -671,8 +675,13 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
               const float4 nl = *reinterpret_cast<const float4*>(lh + 32 * j + i);
               const float2 x0 = ffma2(make_float2(v[i], v[i + 1]), cs2, make_float2(nl.x, nl.y));
               const float2 x1 = ffma2(make_float2(v[i + 2], v[i + 3]), cs2, make_float2(nl.z, nl.w));
-              acc0 = fadd2(acc0, exp2_pair(x0, (i >> 1) & 3));
-              acc1 = fadd2(acc1, exp2_pair(x1, ((i >> 1) + 1) & 3));
+              if (kMax) {
+                acc0 = make_float2(fmaxf(acc0.x, x0.x), fmaxf(acc0.y, x0.y));
+                acc1 = make_float2(fmaxf(acc1.x, x1.x), fmaxf(acc1.y, x1.y));
+              } else {
+                acc0 = fadd2(acc0, exp2_pair(x0, (i >> 1) & 3));
+                acc1 = fadd2(acc1, exp2_pair(x1, ((i >> 1) + 1) & 3));
+              }
             }
           };
           float va[32], vb[32];
@@ -703,8 +712,8 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
         qbuf ^= 1;
       }
       // merge the query parts of each key
-      const float2 acc = fadd2(acc0, acc1);
-      const float total = acc.x + acc.y;
+      const float total = kMax ? fmaxf(fmaxf(acc0.x, acc0.y), fmaxf(acc1.x, acc1.y))
+                               : (acc0.x + acc1.x) + (acc0.y + acc1.y);
       if (part > 0) red[(part - 1) * kKRows2 + row] = total;
       named_barrier(kEpiBarrier, kEpiThreads);
       if (part == 0 && !aborted) {
@@ -712,8 +721,10 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int j = slot - s.start;
         float sum = total;
 #pragma unroll
-        for (int q = 0; q < kParts - 1; ++q) sum += red[q * kKRows2 + row];
-        if (row < min(8, s.np - kt * 8) * 16 && j >= 0 && j < a.W) out[j] = sum;
+        for (int q = 0; q < kParts - 1; ++q)
+          sum = kMax ? fmaxf(sum, red[q * kKRows2 + row]) : sum + red[q * kKRows2 + row];
+        if (row < min(8, s.np - kt * 8) * 16 && j >= 0 && j < a.W)
+          out[j] = kMax ? exp2f(sum) : sum * a.out_scale;
       }
       named_barrier(kEpiBarrier, kEpiThreads);
     }
@@ -1229,7 +1240,8 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
             tmem_ld4(lane_base + kFDCol + (I & 1) * 16 + 3 * (quad >> 1), d);
             tmem_wait_ld();
             reg_fence<4>(d);
-            const float val = (d[0] + d[1] + d[2] * (1.f / 16777216.f)) * (1.f / 32768.f);
+            const float val =
+                (d[0] + d[1] + d[2] * (1.f / 16777216.f)) * (1.f / 32768.f) * a.out_scale;
             float* dst;
             if (cur.q0 == 0 && cur.q1 == TPI) {
               dst = a.scores + (static_cast<size_t>(cur.r) * a.Hkv + cur.g) * a.W;
@@ -1392,11 +1404,13 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   a.ring = L.ring;
   a.part = nullptr;
   a.streamk = 0;
+  a.out_scale = L.agg == KARA_AGG_MEAN ? 1.f / (static_cast<float>(a.G) * L.W) : 1.f;
+  const bool agg_max = L.agg == KARA_AGG_MAX;
 
 
   // Windows of 128, 256, 512 or 1024 keys: the fused single-exponential kernel on clusters of
-  // W / 128 CTAs.
-  if (L.W == 128 || L.W == 256 || L.W == 512 || L.W == 1024) {
+  // W / 128 CTAs (sum and mean; the max aggregation takes the two-pass path).
+  if (!agg_max && (L.W == 128 || L.W == 256 || L.W == 512 || L.W == 1024)) {
     const int CL = L.W / kFKeys;
     auto kern = CL == 1 ? score_fused_kernel<D, 1>
               : CL == 2 ? score_fused_kernel<D, 2>
@@ -1461,7 +1475,9 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   if (!attr_set) {
     cudaFuncSetAttribute(score_rowstats_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(rowstats_smem<D>()));
-    cudaFuncSetAttribute(score_colsum_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(score_colsum_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(colsum_smem<D>()));
+    cudaFuncSetAttribute(score_colsum_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(colsum_smem<D>()));
     attr_set = true;
   }
@@ -1482,11 +1498,12 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
     launch_pdl(score_lse_merge_kernel, dim3(blocks), dim3(256), 0, stream, a);
     if (check_launch("score_lse_merge_kernel") != KARA_OK) return KARA_ERR_CUDA;
   }
-  launch_pdl(score_colsum_kernel<D>, dim3(min(tiles2, sms)), dim3(kThreads), colsum_smem<D>(),
-             stream, tq2, tk, a);
+  auto colsum = agg_max ? score_colsum_kernel<D, true> : score_colsum_kernel<D, false>;
+  launch_pdl(colsum, dim3(min(tiles2, sms)), dim3(kThreads), colsum_smem<D>(), stream, tq2, tk,
+             a);
   if (check_launch("score_colsum_kernel") != KARA_OK) {
-    describe_kernel("score_colsum_kernel", reinterpret_cast<const void*>(score_colsum_kernel<D>),
-                    kThreads, colsum_smem<D>());
+    describe_kernel("score_colsum_kernel", reinterpret_cast<const void*>(colsum), kThreads,
+                    colsum_smem<D>());
     return KARA_ERR_CUDA;
   }
   return KARA_OK;

@@ -287,4 +287,55 @@ kara_status launch_token2chunk(const float* scores, const int32_t* sel, int rows
   return check_launch(__func__);
 }
 
+namespace {
+
+// A selection shared by the KV heads of a layer: the head-summed scores (heads added in
+// ascending order, so the result is reproducible) ...
+__global__ void sum_heads_kernel(const float* __restrict__ scores, int rows, int hkv, int W,
+                                 float* __restrict__ out) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const size_t total = static_cast<size_t>(rows) * W;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t r = i / W, j = i - r * W;
+    const float* p = scores + r * hkv * W + j;
+    float s = 0.f;
+    for (int g = 0; g < hkv; ++g) s += p[static_cast<size_t>(g) * W];
+    out[i] = s;
+  }
+}
+
+// ... and the one keep set copied to every head.
+__global__ void expand_keep_kernel(const int32_t* __restrict__ keep_shared, int rows, int hkv,
+                                   int k, int32_t* __restrict__ keep) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const size_t total = static_cast<size_t>(rows) * hkv * k;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t t = i % k, r = i / (static_cast<size_t>(hkv) * k);
+    keep[i] = keep_shared[r * k + t];
+  }
+}
+
+int grid_for(size_t n) {
+  const size_t b = (n + 255) / 256;
+  return static_cast<int>(b < 1 ? 1 : (b > 4096 ? 4096 : b));
+}
+
+}  // namespace
+
+kara_status launch_sum_heads(const float* scores, int rows, int hkv, int W, float* out,
+                             cudaStream_t stream) {
+  launch_pdl(sum_heads_kernel, dim3(grid_for(static_cast<size_t>(rows) * W)), dim3(256), 0,
+             stream, scores, rows, hkv, W, out);
+  return check_launch("kara_sum_heads");
+}
+
+kara_status launch_expand_keep(const int32_t* keep_shared, int rows, int hkv, int k,
+                               int32_t* keep, cudaStream_t stream) {
+  launch_pdl(expand_keep_kernel, dim3(grid_for(static_cast<size_t>(rows) * hkv * k)), dim3(256),
+             0, stream, keep_shared, rows, hkv, k, keep);
+  return check_launch("kara_expand_keep");
+}
+
 }  // namespace kara

@@ -92,6 +92,10 @@ _SIGNATURES = {
     "kara_step_begin": ([ctypes.POINTER(_Pool), _P, _P], _I),
     "kara_step_end": ([ctypes.POINTER(_Pool), _P, _I, _I, _I, _P, _P, _P], _I),
     "kara_reset_tails": ([_P, _P, _I, _I, _P], _I),
+    "kara_score_ex": ([_P, _I, _P, ctypes.POINTER(_Pool), _P, _I, _I, _I, _F, _I, _P, _P, _Z, _P,
+                       _P], _I),
+    "kara_sum_heads": ([_P, _I, _I, _I, _P, _P], _I),
+    "kara_expand_keep": ([_P, _I, _I, _I, _P, _P], _I),
 }
 
 
@@ -236,6 +240,69 @@ def kara_score(q_win: torch.Tensor, k_cache: torch.Tensor, pool: PagedPool, wind
                             window, hq, float(scale), _ptr(scores), _ptr(ws), ws.numel(),
                             _ptr(status), _stream(stream)), "kara_score")
     return scores
+
+
+AGG_SUM, AGG_MEAN, AGG_MAX = 0, 1, 2
+
+
+def kara_score_ex(q: torch.Tensor, k_cache: torch.Tensor, pool: PagedPool, window: int,
+                  agg: int = AGG_SUM, ring: bool = False, seq_ids: torch.Tensor | None = None,
+                  num_seqs: int | None = None, scale: float | None = None,
+                  scores: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                  status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Window scores [R, Hkv, W] with the aggregation agg (AGG_SUM / AGG_MEAN / AGG_MAX), the
+    queries from q_win [R, W, Hq, d] or, with ring=True, from the ring [B, 2W, Hq, d]."""
+    _require(q, torch.bfloat16, "q")
+    _require(k_cache, torch.bfloat16, "k_cache")
+    rows, w2, hq, d = q.shape
+    if w2 != (2 * window if ring else window):
+        raise ValueError("q's second dimension must be the window (2 * window for a ring)")
+    if num_seqs is None:
+        num_seqs = int(seq_ids.numel()) if seq_ids is not None else rows
+    if seq_ids is not None:
+        _require(seq_ids, torch.int32, "seq_ids")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if scores is None:
+        scores = torch.empty((num_seqs, pool.num_kv_heads, window), dtype=torch.float32,
+                             device=q.device)
+    _require(scores, torch.float32, "scores")
+    status = status if status is not None else new_status(q.device)
+    ps = pool.c_struct()
+    ws = _workspace(kara_workspace_bytes(OP_SCORE, pool, num_seqs, window, hq), q.device,
+                    workspace)
+    _check(lib().kara_score_ex(_ptr(q), 1 if ring else 0, _ptr(k_cache), ctypes.byref(ps),
+                               _ptr(seq_ids), num_seqs, window, hq, float(scale), int(agg),
+                               _ptr(scores), _ptr(ws), ws.numel(), _ptr(status),
+                               _stream(stream)), "kara_score_ex")
+    return scores
+
+
+def kara_sum_heads(scores: torch.Tensor, out: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """[..., Hkv, W] scores summed over the heads: [..., W] fp32."""
+    _require(scores, torch.float32, "scores")
+    hkv, w = scores.shape[-2], scores.shape[-1]
+    rows = scores.numel() // (hkv * w) if hkv * w else 0
+    if out is None:
+        out = torch.empty(scores.shape[:-2] + (w,), dtype=torch.float32, device=scores.device)
+    _check(lib().kara_sum_heads(_ptr(scores), rows, hkv, w, _ptr(out), _stream(stream)),
+           "kara_sum_heads")
+    return out
+
+
+def kara_expand_keep(keep_shared: torch.Tensor, num_kv_heads: int,
+                     keep: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """[..., k] keep sets copied to every KV head: [..., Hkv, k] int32."""
+    _require(keep_shared, torch.int32, "keep_shared")
+    k = keep_shared.shape[-1]
+    rows = keep_shared.numel() // k if k else 0
+    if keep is None:
+        keep = torch.empty(keep_shared.shape[:-1] + (num_kv_heads, k), dtype=torch.int32,
+                           device=keep_shared.device)
+    _check(lib().kara_expand_keep(_ptr(keep_shared), rows, num_kv_heads, k, _ptr(keep),
+                                  _stream(stream)), "kara_expand_keep")
+    return keep
 
 
 def kara_select(scores: torch.Tensor, k: int, sel: torch.Tensor | None = None,

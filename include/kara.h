@@ -90,6 +90,14 @@ typedef struct kara_lacache_params {
   int32_t recent;   /* trailing slots kept in every layer */
 } kara_lacache_params;
 
+/* Aggregations of the window scores for kara_score_ex (the pages name none; the sum is the
+ * main reading, the others are the variants it leaves open). */
+typedef enum kara_agg {
+  KARA_AGG_SUM = 0,    /* sum over the G query heads and the W window queries */
+  KARA_AGG_MEAN = 1,   /* that sum divided by G * W */
+  KARA_AGG_MAX = 2     /* the largest probability any of those queries gives the key */
+} kara_agg;
+
 /* Operation ids for kara_workspace_bytes(). */
 typedef enum kara_op {
   KARA_OP_SCORE = 1,
@@ -131,6 +139,31 @@ kara_status kara_score(const void* q_win, const void* k_cache, const kara_pool* 
                        const int32_t* seq_ids, int32_t num_seqs, int32_t window,
                        int32_t num_q_heads, float scale, float* scores, void* workspace,
                        size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * kara_score_ex - kara_score (q_is_ring == 0: q is q_win [R, W, Hq, d]) or kara_score_ring
+ * (q_is_ring != 0: q is the window-query ring [batch, 2W, Hq, d]) with the aggregation `agg`
+ * (kara_agg). KARA_AGG_MAX runs the two-pass kernels for every window; sum and mean run the
+ * fused kernel for windows of 128 * c keys (c <= 8). Other arguments, output and errors as
+ * kara_score; an unknown agg is KARA_ERR_INVALID_ARG.
+ */
+kara_status kara_score_ex(const void* q, int32_t q_is_ring, const void* k_cache,
+                          const kara_pool* pool, const int32_t* seq_ids, int32_t num_seqs,
+                          int32_t window, int32_t num_q_heads, float scale, int32_t agg,
+                          float* scores, void* workspace, size_t workspace_bytes,
+                          int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * kara_sum_heads / kara_expand_keep - a selection shared by the KV heads of a layer (a
+ * variant the pages leave open): out[r][j] = sum over g of scores[r][g][j] (heads added in
+ * ascending order), fp32 [rows, window]; kara_select and kara_token2chunk then run once per
+ * row on it, and kara_expand_keep copies each row's keep [rows, k] to every head:
+ * keep[r][g][t] = keep_shared[r][t], int32 [rows, num_kv_heads, k], ready for kara_compact.
+ */
+kara_status kara_sum_heads(const float* scores, int32_t rows, int32_t num_kv_heads,
+                           int32_t window, float* out, cudaStream_t stream);
+kara_status kara_expand_keep(const int32_t* keep_shared, int32_t rows, int32_t num_kv_heads,
+                             int32_t k, int32_t* keep, cudaStream_t stream);
 
 /*
  * kara_select - keep the k highest-scoring window positions ([KARA] abstract: the informative
