@@ -375,6 +375,46 @@ def lacache_run(dev, batch: int, reps: int = 5, warmup: int = 3) -> dict:
                         f"caches, S=8, O=4, rung 64, budget 8192 per layer; one pass (all layers)"}
 
 
+def variants_run(step, reps: int = 10) -> dict:
+    """The score and selection variants on the layer workload (its window queries and cache,
+    not changed by them): kara_score_ex with the mean and with the max aggregation, and the
+    selection shared across KV heads (head sums, select, Token2Chunk, expansion to every
+    head). Average times with CUDA events over `reps` calls after one untimed call."""
+    K, wl, c = step.K, step.wl, step.c
+    tot = torch.empty((wl.batch, wl.window), dtype=torch.float32, device=step.scores.device)
+    shared = torch.empty((wl.batch, wl.keep), dtype=torch.int32, device=tot.device)
+    sel = torch.empty((wl.batch, wl.keep), dtype=torch.int32, device=tot.device)
+
+    def score(agg):
+        K.kara_score_ex(c["q_win"][0], c["k"][0], step.pool, wl.window, agg=agg,
+                        scores=step.scores, workspace=step.ws, status=step.status)
+
+    def shared_select():
+        K.kara_sum_heads(step.scores, out=tot)
+        K.kara_select(tot, wl.keep, sel=sel)
+        K.kara_token2chunk(tot, sel, step.na, wl.gap_limit, wl.widen, keep=shared)
+        K.kara_expand_keep(shared, wl.hkv, keep=step.keep[0])
+
+    out = {}
+    for name, fn in (("score_mean_ms", lambda: score(K.AGG_MEAN)),
+                     ("score_max_ms", lambda: score(K.AGG_MAX)),
+                     ("shared_select_ms", shared_select)):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = e0.elapsed_time(e1) / reps
+    out["status"] = K.read_status(step.status)
+    out["note"] = ("layer workload; max runs the two-pass kernels (a max, not a sum, per key); "
+                   "shared = head sums, one select + Token2Chunk per (sequence, layer), keep "
+                   "copied to the 4 KV heads")
+    return out
+
+
 def decode_loop_run(dev, steps: int = 300, period: int = 100, warm: int = 20) -> dict:
     """The decode loop on the layer workload's shapes (batch 32, 28 query / 4 KV heads, d=128,
     4096-token contexts, W=1024, keep 204, one layer): every step kara_step_begin,
@@ -567,6 +607,7 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
         kernels["lacache_compact"] = lac
     if world == 1 and not args.no_loop:
         kernels["decode_loop"] = decode_loop_run(dev)
+        kernels["variants"] = variants_run(step)
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
