@@ -187,7 +187,7 @@ class Step:
         self.na = K.anchors_for(wl.anchor_frac, wl.keep)
         # scoring: the fused cluster kernel for windows of 128/256/512/1024 keys (plus the
         # split-item sum when a cluster range ends inside an item), else two passes and a
-        # merge; select; Token2Chunk; compaction plan + gather; decode + combine
+        # merge; select + Token2Chunk in one kernel; compaction plan + gather; decode + combine
         self.score_fused = wl.window in (128, 256, 512, 1024)
 
     def restore(self):
@@ -200,9 +200,8 @@ class Step:
         K.kara_score(c["q_win"][0], c["k"][0], self.pool, wl.window, scores=self.scores,
                      workspace=self.ws, status=self.status)
         rec(1)
-        K.kara_select(self.scores, wl.keep, sel=self.sel)
-        K.kara_token2chunk(self.scores, self.sel, self.na, wl.gap_limit, wl.widen,
-                           keep=self.keep[0])
+        K.kara_select_chunks(self.scores, wl.keep, self.na, wl.gap_limit, wl.widen,
+                             keep=self.keep[0])
         rec(2)
         K.kara_compact(c["k"], c["v"], self.pool, wl.window, self.keep, workspace=self.ws,
                        status=self.status)
@@ -396,9 +395,15 @@ def variants_run(step, reps: int = 10) -> dict:
         K.kara_expand_keep(shared, wl.hkv, keep=step.keep[0])
 
     out = {}
+    def select_then_chunks():
+        K.kara_select(step.scores, wl.keep, sel=step.sel)
+        K.kara_token2chunk(step.scores, step.sel, step.na, wl.gap_limit, wl.widen,
+                           keep=step.keep[0])
+
     for name, fn in (("score_mean_ms", lambda: score(K.AGG_MEAN)),
                      ("score_max_ms", lambda: score(K.AGG_MAX)),
-                     ("shared_select_ms", shared_select)):
+                     ("shared_select_ms", shared_select),
+                     ("select_then_token2chunk_ms", select_then_chunks)):
         fn()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -411,7 +416,8 @@ def variants_run(step, reps: int = 10) -> dict:
     out["status"] = K.read_status(step.status)
     out["note"] = ("layer workload; max runs the two-pass kernels (a max, not a sum, per key); "
                    "shared = head sums, one select + Token2Chunk per (sequence, layer), keep "
-                   "copied to the 4 KV heads")
+                   "copied to the 4 KV heads; select_then_token2chunk = the two calls the "
+                   "step's fused kara_select_chunks replaces")
     return out
 
 

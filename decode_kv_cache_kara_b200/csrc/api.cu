@@ -264,6 +264,19 @@ kara_status kara_token2chunk(const float* scores, const int32_t* sel, int32_t ro
                             stream);
 }
 
+kara_status kara_select_chunks(const float* scores, int32_t rows, int32_t window, int32_t k,
+                               int32_t num_anchors, int32_t gap_limit, int32_t widen,
+                               int32_t* sel, int32_t* keep, cudaStream_t stream) {
+  if (rows < 0 || window < 1 || window > KARA_MAX_WINDOW || k < 1 || k > window)
+    return KARA_ERR_INVALID_ARG;
+  if (num_anchors < 0 || num_anchors > k || gap_limit < 0 || widen < 0)
+    return KARA_ERR_INVALID_ARG;
+  if (rows == 0) return KARA_OK;
+  if (scores == nullptr || keep == nullptr) return KARA_ERR_INVALID_ARG;
+  return launch_select_chunks(scores, rows, window, k, num_anchors, gap_limit, widen, sel, keep,
+                              stream);
+}
+
 kara_status kara_compact(const kara_layer_kv* layers, int32_t num_layers, const kara_pool* pool,
                          const int32_t* seq_ids, int32_t num_seqs, int32_t window, int32_t k,
                          const int32_t* keep, void* workspace, size_t workspace_bytes,

@@ -149,10 +149,13 @@ select_kernel(const float* __restrict__ scores, int W, int k, int32_t* __restric
   block_compact_write(flag, W, E, sel + static_cast<size_t>(row) * k, ss->ibuf);
 }
 
-__global__ void __launch_bounds__(kSelThreads)
-token2chunk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ sel, int W,
-                   int k, int num_anchors, int gap_limit, int widen, int32_t* __restrict__ keep) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
+// Token2Chunk of one row (block-level); the selection comes from `sel` (k positions in
+// global memory) or, when kSelIn is false, is selected here first (the fused
+// select + Token2Chunk of kara_select_chunks, which may also write the selection to sel).
+template <bool kSelIn>
+__device__ void token2chunk_row(const float* __restrict__ scores, int32_t* __restrict__ sel,
+                                int W, int k, int num_anchors, int gap_limit, int widen,
+                                int32_t* __restrict__ keep) {
   extern __shared__ __align__(16) uint8_t smem[];
   SelectSmem* ss = reinterpret_cast<SelectSmem*>(smem);
   uint32_t* key = reinterpret_cast<uint32_t*>(smem + sizeof(SelectSmem));
@@ -167,7 +170,7 @@ token2chunk_kernel(const float* __restrict__ scores, const int32_t* __restrict__
 
   const int row = blockIdx.x;
   const float* s = scores + static_cast<size_t>(row) * W;
-  const int32_t* sl = sel + static_cast<size_t>(row) * k;
+  const int32_t* sl = kSelIn ? sel + static_cast<size_t>(row) * k : nullptr;
   const int tid = threadIdx.x;
   const int E = (W + kSelThreads - 1) / kSelThreads;
   const int lo = tid * E, hi = min(W, lo + E);
@@ -177,13 +180,21 @@ token2chunk_kernel(const float* __restrict__ scores, const int32_t* __restrict__
     in_sel[j] = 0;
     anchor[j] = 0;
     flag[j] = 0;
+    if (!kSelIn) cand[j] = 1;
   }
   __syncthreads();
-  for (int i = tid; i < k; i += kSelThreads) {
-    const int p = sl[i];
-    if (p >= 0 && p < W) in_sel[p] = 1;
+  if (kSelIn) {
+    for (int i = tid; i < k; i += kSelThreads) {
+      const int p = sl[i];
+      if (p >= 0 && p < W) in_sel[p] = 1;
+    }
+    __syncthreads();
+  } else {
+    // the selection itself: the k largest scores (ties: lower position) into in_sel
+    block_select(key, cand, in_sel, W, E, k, ss);
+    if (sel != nullptr) block_compact_write(in_sel, W, E, sel + static_cast<size_t>(row) * k, ss->ibuf);
+    __syncthreads();
   }
-  __syncthreads();
 
   // a. anchors: top num_anchors of the selection
   block_select(key, in_sel, anchor, W, E, num_anchors, ss);
@@ -265,6 +276,21 @@ token2chunk_kernel(const float* __restrict__ scores, const int32_t* __restrict__
   block_compact_write(flag, W, E, keep + static_cast<size_t>(row) * k, ss->ibuf);
 }
 
+__global__ void __launch_bounds__(kSelThreads)
+token2chunk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ sel, int W,
+                   int k, int num_anchors, int gap_limit, int widen, int32_t* __restrict__ keep) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
+  token2chunk_row<true>(scores, const_cast<int32_t*>(sel), W, k, num_anchors, gap_limit, widen,
+                        keep);
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+select_chunks_kernel(const float* __restrict__ scores, int32_t* __restrict__ sel, int W, int k,
+                     int num_anchors, int gap_limit, int widen, int32_t* __restrict__ keep) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
+  token2chunk_row<false>(scores, sel, W, k, num_anchors, gap_limit, widen, keep);
+}
+
 size_t select_smem(int W) { return sizeof(SelectSmem) + static_cast<size_t>(W) * 6 + 64; }
 size_t t2c_smem(int W) { return sizeof(SelectSmem) + static_cast<size_t>(W) * 14 + 64; }
 
@@ -284,6 +310,15 @@ kara_status launch_token2chunk(const float* scores, const int32_t* sel, int rows
   if (rows == 0) return KARA_OK;
   launch_pdl(token2chunk_kernel, dim3(rows), dim3(kSelThreads), t2c_smem(W), stream, scores, sel,
              W, k, num_anchors, gap_limit, widen, keep);
+  return check_launch(__func__);
+}
+
+kara_status launch_select_chunks(const float* scores, int rows, int W, int k, int num_anchors,
+                                 int gap_limit, int widen, int32_t* sel, int32_t* keep,
+                                 cudaStream_t stream) {
+  if (rows == 0) return KARA_OK;
+  launch_pdl(select_chunks_kernel, dim3(rows), dim3(kSelThreads), t2c_smem(W), stream, scores,
+             sel, W, k, num_anchors, gap_limit, widen, keep);
   return check_launch(__func__);
 }
 

@@ -96,6 +96,7 @@ _SIGNATURES = {
                        _P], _I),
     "kara_sum_heads": ([_P, _I, _I, _I, _P, _P], _I),
     "kara_expand_keep": ([_P, _I, _I, _I, _P, _P], _I),
+    "kara_select_chunks": ([_P, _I, _I, _I, _I, _I, _I, _P, _P, _P], _I),
 }
 
 
@@ -276,6 +277,25 @@ def kara_score_ex(q: torch.Tensor, k_cache: torch.Tensor, pool: PagedPool, windo
                                _ptr(scores), _ptr(ws), ws.numel(), _ptr(status),
                                _stream(stream)), "kara_score_ex")
     return scores
+
+
+def kara_select_chunks(scores: torch.Tensor, k: int, num_anchors: int, gap_limit: int,
+                       widen: int, keep: torch.Tensor | None = None,
+                       sel: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """kara_select + kara_token2chunk in one kernel: keep [..., k] int32 (sel, if given, gets
+    the selection)."""
+    _require(scores, torch.float32, "scores")
+    w = scores.shape[-1]
+    rows = scores.numel() // w if w else 0
+    if keep is None:
+        keep = torch.empty(scores.shape[:-1] + (k,), dtype=torch.int32, device=scores.device)
+    _require(keep, torch.int32, "keep")
+    if sel is not None:
+        _require(sel, torch.int32, "sel")
+    _check(lib().kara_select_chunks(_ptr(scores), rows, w, k, num_anchors, gap_limit, widen,
+                                    _ptr(sel), _ptr(keep), _stream(stream)),
+           "kara_select_chunks")
+    return keep
 
 
 def kara_sum_heads(scores: torch.Tensor, out: torch.Tensor | None = None,

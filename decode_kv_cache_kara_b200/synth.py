@@ -64,7 +64,8 @@ class Workload:
         return replace(self, **kw)
 
 
-# The five workloads of the method's benchmark suite (see the design doc for the recipe).
+# The five workloads: tiny (the parity case), one 7B-class layer, a 28-layer step with ragged
+# contexts, an 8B-class GQA model and the LaCache workload; each line states its sizes.
 WORKLOADS = {
     # 1 sequence, 4q/2kv heads, d=64, 512-token cache, window 128, keep 32, 5 % heavy window keys
     "tiny": Workload("tiny", batch=1, layers=1, hq=4, hkv=2, head_dim=64, ctx_lo=512, ctx_hi=512,

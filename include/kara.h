@@ -196,6 +196,16 @@ kara_status kara_token2chunk(const float* scores, const int32_t* sel, int32_t ro
                              int32_t widen, int32_t* keep, cudaStream_t stream);
 
 /*
+ * kara_select_chunks - kara_select and kara_token2chunk in one kernel per row: the selection
+ * stays in shared memory and one launch replaces two. keep as kara_token2chunk of
+ * kara_select's output, bit for bit. sel may be NULL; otherwise
+ * the selection is written there too. Arguments and limits as the two calls.
+ */
+kara_status kara_select_chunks(const float* scores, int32_t rows, int32_t window, int32_t k,
+                               int32_t num_anchors, int32_t gap_limit, int32_t widen,
+                               int32_t* sel, int32_t* keep, cudaStream_t stream);
+
+/*
  * kara_compact - write the compressed windows into fresh blocks, rewrite the block table and
  * free the old window blocks ([KARA] abstract: Kara adapted to PagedAttention).
  *

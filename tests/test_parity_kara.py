@@ -318,3 +318,27 @@ def test_compact_reuses_freed_blocks():
     check_compaction(dev2, ref2, 1, list(range(wl.batch)), wl.batch)
     used2 = set(x for ids in ref2[7].values() for x in ids) | set(bt[bt >= 0].ravel().tolist())
     assert used2 & freed1, "the second pass should reuse blocks the first one freed"
+
+
+@pytest.mark.parametrize("name", ["g7_ragged_unaligned", "g8_w384", "w16_ctx_eq_w"])
+def test_select_chunks_equals_select_then_token2chunk(name):
+    """The fused select + Token2Chunk kernel gives the separate calls' keep (and selection)
+    bit for bit, and both equal the oracle's on the same scores."""
+    wl = SCORE_CASES[name]
+    cpu, dev = H.make(wl, 12)
+    pool = K.PagedPool.from_cache(dev)
+    sc = K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window)
+    na = K.anchors_for(wl.anchor_frac, wl.keep)
+    sel = K.kara_select(sc, wl.keep)
+    keep = K.kara_token2chunk(sc, sel, na, wl.gap_limit, wl.widen)
+    sel2 = torch.empty_like(sel)
+    keep2 = K.kara_select_chunks(sc, wl.keep, na, wl.gap_limit, wl.widen, sel=sel2)
+    keep3 = K.kara_select_chunks(sc, wl.keep, na, wl.gap_limit, wl.widen)
+    torch.cuda.synchronize()
+    assert torch.equal(keep, keep2) and torch.equal(sel, sel2) and torch.equal(keep, keep3)
+    s = H.f64(sc)
+    for r in range(wl.batch):
+        for g in range(wl.hkv):
+            ref = ok.token2chunk(s[r, g], ok.select_topk(s[r, g], wl.keep), na, wl.gap_limit,
+                                 wl.widen)
+            assert np.array_equal(H.i32(keep2[r, g]), ref)
