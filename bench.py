@@ -2,8 +2,8 @@
 
 One step = one pass of the whole hot path over one batch of the "layer" workload (one
 7B-class layer, batch 32, 28 query / 4 KV heads, d = 128, 4096-token paged caches, window
-1024, keep 204): kara_score -> kara_select -> kara_token2chunk -> kara_compact ->
-paged_decode_attn over the compressed cache, then the block table, lengths and free list are
+1024, keep 204): kara_score -> kara_select_chunks (select and Token2Chunk in one kernel) ->
+kara_compact -> paged_decode_attn over the compressed cache, then the block table, lengths and free list are
 restored so that every step sees the same input. Metric: compressed KV tokens per second
 (window tokens of all due sequences / step time), whole job over all ranks.
 
@@ -425,7 +425,7 @@ def decode_loop_run(dev, steps: int = 300, period: int = 100, warm: int = 20) ->
     """The decode loop on the layer workload's shapes (batch 32, 28 query / 4 KV heads, d=128,
     4096-token contexts, W=1024, keep 204, one layer): every step kara_step_begin,
     kara_decode_append and kara_step_end; every `period` steps the due sequences (tail >= W)
-    are compressed (kara_score_ring, kara_select, kara_token2chunk, kara_compact,
+    are compressed (kara_score_ring, kara_select_chunks, kara_compact,
     kara_reset_tails). Tails start spread over [0, W) and the query ring holds seeded queries,
     as in the middle of a generation. Timed with CUDA events per step; a check step includes
     the host read of the due count that sizes its compression."""
@@ -471,9 +471,8 @@ def decode_loop_run(dev, steps: int = 300, period: int = 100, warm: int = 20) ->
             seq = due[:cnt]
             K.kara_score_ring(ring, k0, pool, W, seq, cnt, scores=scores[:cnt], workspace=ws_sc,
                               status=status)
-            K.kara_select(scores[:cnt], wl.keep, sel=sel[:cnt])
-            K.kara_token2chunk(scores[:cnt], sel[:cnt], na, wl.gap_limit, wl.widen,
-                               keep=keep[0, :cnt])
+            K.kara_select_chunks(scores[:cnt], wl.keep, na, wl.gap_limit, wl.widen,
+                                 keep=keep[0, :cnt])
             K.kara_compact([k0], [v0], pool, W, keep[:, :cnt], seq_ids=seq, workspace=ws_cp,
                            status=status)
             K.kara_reset_tails(tail, seq, cnt)
