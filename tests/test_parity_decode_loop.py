@@ -229,3 +229,38 @@ def test_lacache_loop_matches_oracle():
     torch.cuda.synchronize()
     assert K.read_status(status) == 0
     assert passes >= 2 * wl.batch
+
+
+def test_decode_append_empty_context_and_no_ring():
+    """A sequence with an empty cache: its block comes from kara_step_begin, the new token is
+    the only one, so the output is its V row (bf16, exactly); no ring is passed, and a step
+    end without a check only advances the lengths."""
+    wl = synth.Workload("empty", batch=3, layers=1, hq=4, hkv=2, head_dim=128, ctx_lo=20,
+                        ctx_hi=40, window=16, keep=4)
+    cpu = synth.make_cache(wl, 13, "cpu", with_queries=False, extra_pages=2)
+    cpu["ctx_len"][1] = 0
+    cpu["block_table"][1].fill_(-1)
+    # the emptied sequence's old blocks stay out of the free list (they are simply unused)
+    dev = H.to_device(cpu)
+    pool = K.PagedPool.from_cache(dev)
+    status = K.new_status()
+    K.kara_step_begin(pool, status)
+    inp = synth.decode_step_inputs(wl, 13, 0)[0]
+    q, kn, vn = (inp[x].cuda() for x in ("q", "k", "v"))
+    out = K.kara_decode_append(q, kn, vn, dev["k"][0], dev["v"][0], pool, status=status)
+    K.kara_step_end(pool)
+    torch.cuda.synchronize()
+    assert K.read_status(status) == 0
+    assert int(dev["ctx_len"][1]) == 1 and int(dev["ctx_len"][0]) == int(cpu["ctx_len"][0]) + 1
+    g_of_h = torch.arange(wl.hq) // wl.group
+    assert torch.equal(out[1].cpu(), vn[1].cpu()[g_of_h])
+    blk = int(dev["block_table"][1, 0])
+    assert blk >= 0
+    assert torch.equal(dev["k"][0][blk, 0].cpu(), kn[1].cpu())
+    assert torch.equal(dev["v"][0][blk, 0].cpu(), vn[1].cpu())
+    # the other sequences against the oracle
+    scale = 1 / math.sqrt(wl.head_dim)
+    bt = H.i32(dev["block_table"])
+    ref, _, _, _ = dl.decode_append(f32(q), f32(kn), f32(vn), f32(cpu["k"][0]), f32(cpu["v"][0]),
+                                    bt, H.i32(cpu["ctx_len"]), scale, wl.page, None, 1)
+    assert np.allclose(H.f64(out), ref, atol=2e-2, rtol=1e-2)

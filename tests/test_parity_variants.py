@@ -124,3 +124,21 @@ def test_shared_selection_across_kv_heads():
             n = int(cl[b])
             assert np.array_equal(H.logical_rows(kg, bt[b], n), H.logical_rows(kpo[layer], bt[b], n))
             assert np.array_equal(H.logical_rows(vg, bt[b], n), H.logical_rows(vpo[layer], bt[b], n))
+
+
+def test_mean_from_the_ring_equals_mean_from_q_win_and_one_head_sums():
+    wl = CASES["w512_fused"]
+    cpu, dev = H.make(wl, 14)
+    pool = K.PagedPool.from_cache(dev)
+    W = wl.window
+    ring = torch.zeros((wl.batch, 2 * W, wl.hq, wl.head_dim), device="cuda", dtype=torch.bfloat16)
+    for b in range(wl.batch):
+        off = (int(cpu["ctx_len"][b]) - W) % W
+        ring[b, off:off + W] = dev["q_win"][0][b]
+    seq = torch.arange(wl.batch, dtype=torch.int32, device="cuda")
+    a = K.kara_score_ex(dev["q_win"][0], dev["k"][0], pool, W, agg=K.AGG_MEAN)
+    b = K.kara_score_ex(ring, dev["k"][0], pool, W, agg=K.AGG_MEAN, ring=True, seq_ids=seq)
+    one = K.kara_sum_heads(a[:, :1].contiguous())          # one KV head: the row itself
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert torch.equal(one, a[:, 0])
