@@ -201,7 +201,7 @@ class Step:
                      workspace=self.ws, status=self.status)
         rec(1)
         K.kara_select_chunks(self.scores, wl.keep, self.na, wl.gap_limit, wl.widen,
-                             keep=self.keep[0])
+                             keep=self.keep[0], sel=self.sel)
         rec(2)
         K.kara_compact(c["k"], c["v"], self.pool, wl.window, self.keep, workspace=self.ws,
                        status=self.status)
