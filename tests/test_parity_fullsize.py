@@ -1,8 +1,8 @@
 """Parity at full size, in the launch configuration bench.py times.
 
 The layer workload (batch 32, 28 q / 4 kv heads, d=128, 4096-token caches, W=1024, k=204) goes
-through the same calls as one bench step (bench.Step): kara_score -> kara_select ->
-kara_token2chunk -> kara_compact -> paged_decode_attn. Checks: sampled score rows against the
+through the same calls as one bench step (bench.Step): kara_score -> kara_select_chunks
+(selection and Token2Chunk in one kernel, both written) -> kara_compact -> paged_decode_attn. Checks: sampled score rows against the
 oracle, and the W*G row sums on every row; select and Token2Chunk exactly on sampled rows;
 compaction bit-exact on every sequence; decode on sampled (sequence, query head) pairs. The
 LaCache ladder runs at its workload's sequence length (64K tokens, 32 layers, 8 KV heads) with
