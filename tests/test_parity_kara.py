@@ -182,6 +182,16 @@ def test_select_max_window_and_k_equals_w():
         sel = K.kara_select(scores, k)
         torch.cuda.synchronize()
         assert np.array_equal(H.i32(sel), ok.select_batch(s.astype(np.float64), k))
+    # Token2Chunk at the largest window (58 KB of shared memory), separately and fused
+    sel = K.kara_select(scores, 819)
+    keep = K.kara_token2chunk(scores, sel, 410, 8, 1)
+    keep2 = K.kara_select_chunks(scores, 819, 410, 8, 1)
+    torch.cuda.synchronize()
+    assert torch.equal(keep, keep2)
+    s64 = s.astype(np.float64)
+    for r in range(3):
+        assert np.array_equal(H.i32(keep[r]), ok.token2chunk(s64[r], ok.select_topk(s64[r], 819),
+                                                            410, 8, 1))
 
 
 # ---------------------------------------------------------------- compaction
