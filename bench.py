@@ -413,6 +413,33 @@ def variants_run(step, reps: int = 10) -> dict:
         e1.record()
         torch.cuda.synchronize()
         out[name] = e0.elapsed_time(e1) / reps
+    # selection, Token2Chunk and compaction: two calls (three kernels) against kara_compress
+    # (plan + one fused kernel); the bookkeeping is restored between repetitions, untimed
+    def compact_pair():
+        K.kara_select_chunks(step.scores, wl.keep, step.na, wl.gap_limit, wl.widen,
+                             keep=step.keep[0])
+        K.kara_compact(c["k"], c["v"], step.pool, wl.window, step.keep, workspace=step.ws,
+                       status=step.status)
+
+    def compress():
+        K.kara_compress(step.scores[None], c["k"], c["v"], step.pool, wl.window, wl.keep, step.na,
+                        wl.gap_limit, wl.widen, keep=step.keep, workspace=step.ws,
+                        status=step.status)
+
+    for name, fn in (("select_chunks_then_compact_ms", compact_pair), ("compress_ms", compress)):
+        fn()
+        step.restore()
+        torch.cuda.synchronize()
+        total = 0.0
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            step.restore()
+            torch.cuda.synchronize()
+            total += e0.elapsed_time(e1)
+        out[name] = total / reps
     out["status"] = K.read_status(step.status)
     out["note"] = ("layer workload; max runs the two-pass kernels (a max, not a sum, per key); "
                    "shared = head sums, one select + Token2Chunk per (sequence, layer), keep "

@@ -313,6 +313,50 @@ kara_status kara_compact(const kara_layer_kv* layers, int32_t num_layers, const 
   return launch_compact(L, stream);
 }
 
+kara_status kara_compress(const float* scores, const kara_layer_kv* layers, int32_t num_layers,
+                          const kara_pool* pool, const int32_t* seq_ids, int32_t num_seqs,
+                          int32_t window, int32_t k, int32_t num_anchors, int32_t gap_limit,
+                          int32_t widen, int32_t* keep, void* workspace, size_t workspace_bytes,
+                          int32_t* dev_status, cudaStream_t stream) {
+  kara_status st = check_pool(pool);
+  if (st != KARA_OK) return st;
+  if (pool->free_list == nullptr || pool->free_top == nullptr) return KARA_ERR_INVALID_ARG;
+  if (num_seqs < 0 || window < 1 || window > KARA_MAX_WINDOW || k < 1 || k > window)
+    return KARA_ERR_INVALID_ARG;
+  if (num_anchors < 0 || num_anchors > k || gap_limit < 0 || widen < 0)
+    return KARA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return KARA_OK;
+  if (scores == nullptr || dev_status == nullptr) return KARA_ERR_INVALID_ARG;
+  CompactLaunch L;
+  if ((st = fill_layers(layers, num_layers, &L.layers)) != KARA_OK) return st;
+  const size_t need = kara_workspace_bytes(KARA_OP_COMPACT, pool, num_seqs, window, 0, k);
+  if (workspace == nullptr || workspace_bytes < need || !aligned256(workspace))
+    return KARA_ERR_WORKSPACE;
+  L.L = num_layers;
+  L.block_table = pool->block_table;
+  L.ctx_len = pool->ctx_len;
+  L.free_list = pool->free_list;
+  L.free_top = pool->free_top;
+  L.seq_ids = seq_ids;
+  L.keep = nullptr;
+  L.plan = static_cast<int32_t*>(workspace);
+  L.status = dev_status;
+  L.R = num_seqs;
+  L.W = window;
+  L.k = k;
+  L.Hkv = pool->num_kv_heads;
+  L.D = pool->head_dim;
+  L.batch = pool->batch;
+  L.max_blocks = pool->max_blocks_per_seq;
+  L.num_blocks = pool->num_blocks;
+  L.scores = scores;
+  L.keep_out = keep;
+  L.num_anchors = num_anchors;
+  L.gap_limit = gap_limit;
+  L.widen = widen;
+  return launch_compact(L, stream);
+}
+
 
 kara_status paged_decode_attn(const void* q, const void* k_cache, const void* v_cache,
                               const kara_pool* pool, int32_t num_q_heads, float scale, void* out,

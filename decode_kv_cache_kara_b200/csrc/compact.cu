@@ -27,6 +27,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "select_row.cuh"
 
 namespace kara {
 
@@ -297,6 +298,102 @@ __global__ void __launch_bounds__(kGatherThreads) kara_gather_kernel(const KaraG
 }
 
 // ------------------------------------------------------------------------------------------
+// Fused compression: CTA = (layer, sequence, KV head) of kSelThreads threads. The compaction
+// plan depends only on (n, W, k) of each sequence, not on which positions are kept, so it
+// runs first; each CTA then selects and expands its row in shared memory (select_row.cuh),
+// copies the head's prefix rows of the first window page and its k kept rows into the fresh
+// blocks, and the sequence's last CTA finalizes it. keep_out (optional) gets the keep sets.
+// ------------------------------------------------------------------------------------------
+struct CompressArgs {
+  KaraGather g;                  // g.keep unused
+  const float* scores;           // [L, R, Hkv, W]
+  int32_t* keep_out;             // [L, R, Hkv, k] or null
+  int num_anchors, gap_limit, widen;
+};
+
+__host__ __device__ constexpr size_t compress_keep_off(int W) {
+  return (t2c_smem(W) + 15) / 16 * 16;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) compress_kernel(const CompressArgs c) {
+  __shared__ int s_old[kMaxWindowPages];
+  __shared__ int s_fresh[kMaxWindowPages];
+  extern __shared__ __align__(16) uint8_t dsm[];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const KaraGather& g = c.g;
+  const int head = blockIdx.y % g.Hkv;
+  const int r = blockIdx.y / g.Hkv;
+  const int layer = blockIdx.z;
+  const size_t rowi = (static_cast<size_t>(layer) * g.R + r) * g.Hkv + head;
+  int32_t* s_keep = reinterpret_cast<int32_t*>(dsm + compress_keep_off(g.W));
+  // 1. selection and Token2Chunk of the row, the keep set into shared memory
+  token2chunk_row(c.scores + rowi * g.W, nullptr, nullptr, g.W, g.k, c.num_anchors,
+                  c.gap_limit, c.widen, s_keep, dsm);
+  __syncthreads();
+  if (c.keep_out != nullptr)
+    for (int i = threadIdx.x; i < g.k; i += kSelThreads) c.keep_out[rowi * g.k + i] = s_keep[i];
+  const int32_t* hdr = g.plan;
+  if (hdr[0] != 1) return;        // the plan refused (and reported): nothing moves
+  // 2. the gather of the row's prefix rows and kept rows
+  constexpr int kVecPerRow = D * 2 / 16;
+  constexpr int kRowsPerPass = kSelThreads / kVecPerRow;
+  const int32_t* rows = g.plan + kPlanHeader;
+  const int32_t* fresh = rows + static_cast<size_t>(g.R) * kPlanStride;
+  const int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
+  const int b = row[P_B], start = row[P_START], off = row[P_OFF], p0 = row[P_P0];
+  const int n_old = row[P_NOLD], n_new = row[P_NNEW];
+  const int32_t* tab = g.block_table + static_cast<size_t>(b) * g.max_blocks + p0;
+  const int32_t* fr = fresh + row[P_BNEW];
+  for (int i = threadIdx.x; i < n_old; i += kSelThreads) s_old[i] = tab[i];
+  for (int i = threadIdx.x; i < n_new; i += kSelThreads) s_fresh[i] = fr[i];
+  __syncthreads();
+  const uint4* ksrc = reinterpret_cast<const uint4*>(g.layers.k[layer]);
+  const uint4* vsrc = reinterpret_cast<const uint4*>(g.layers.v[layer]);
+  uint4* kdst = reinterpret_cast<uint4*>(g.layers.k[layer]);
+  uint4* vdst = reinterpret_cast<uint4*>(g.layers.v[layer]);
+  const int vec = threadIdx.x % kVecPerRow;
+  const int sub = threadIdx.x / kVecPerRow;
+  const int total = off + g.k;
+  constexpr int kUnroll = 8;
+  for (int base = sub; base < total; base += kRowsPerPass * kUnroll) {
+    uint4 kv[kUnroll], vv[kUnroll];
+    size_t dsti[kUnroll];
+    bool act[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int i = base + u * kRowsPerPass;
+      act[u] = i < total;
+      if (!act[u]) continue;
+      int src_slot, dst_slot;
+      if (i < off) {
+        src_slot = dst_slot = p0 * 16 + i;
+      } else {
+        src_slot = start + s_keep[i - off];
+        dst_slot = start + (i - off);
+      }
+      const int sblk = s_old[(src_slot >> 4) - p0];
+      const int dblk = s_fresh[(dst_slot >> 4) - p0];
+      const size_t si = ((static_cast<size_t>(sblk) * 16 + (src_slot & 15)) * g.Hkv + head) *
+                            kVecPerRow + vec;
+      dsti[u] = ((static_cast<size_t>(dblk) * 16 + (dst_slot & 15)) * g.Hkv + head) *
+                    kVecPerRow + vec;
+      kv[u] = ksrc[si];
+      vv[u] = vsrc[si];
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (!act[u]) continue;
+      kdst[dsti[u]] = kv[u];
+      vdst[dsti[u]] = vv[u];
+    }
+  }
+  // 3. the sequence's last CTA (of L x Hkv) rewrites its table, frees its old blocks and
+  // sets its length
+  finalize_if_last(g.fin, r, g.Hkv * gridDim.z, s_old, s_fresh);
+}
+
+// ------------------------------------------------------------------------------------------
 // LaCache gather: CTA = (layer, sequence, chunk of compacted slots); whole [Hkv, d] rows.
 // ------------------------------------------------------------------------------------------
 struct LadderGather {
@@ -448,6 +545,28 @@ kara_status launch_compact(const CompactLaunch& L, cudaStream_t stream) {
   g.fin.R = L.R;
   g.fin.max_blocks = L.max_blocks;
   g.fin.k = L.k;
+  if (L.scores != nullptr) {
+    CompressArgs c;
+    c.g = g;
+    c.scores = L.scores;
+    c.keep_out = L.keep_out;
+    c.num_anchors = L.num_anchors;
+    c.gap_limit = L.gap_limit;
+    c.widen = L.widen;
+    const size_t smem = compress_keep_off(L.W) + static_cast<size_t>(L.k) * sizeof(int32_t);
+    static bool attr = false;
+    if (!attr) {
+      const int most = static_cast<int>(compress_keep_off(KARA_MAX_WINDOW) +
+                                        KARA_MAX_WINDOW * sizeof(int32_t));
+      cudaFuncSetAttribute(compress_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      cudaFuncSetAttribute(compress_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      attr = true;
+    }
+    const dim3 grid(1, L.R * L.Hkv, L.L);
+    if (L.D == 128) launch_pdl(compress_kernel<128>, grid, dim3(kSelThreads), smem, stream, c);
+    else launch_pdl(compress_kernel<64>, grid, dim3(kSelThreads), smem, stream, c);
+    return check_launch("kara_compress");
+  }
   dim3 grid((L.k + kChunkRows - 1) / kChunkRows, L.R * L.Hkv, L.L);
   if (L.D == 128) launch_dependent(kara_gather_kernel<128>, grid, g, stream);
   else launch_dependent(kara_gather_kernel<64>, grid, g, stream);

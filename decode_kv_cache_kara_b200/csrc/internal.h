@@ -96,6 +96,11 @@ struct CompactLaunch {
   int32_t* status;
   int R, W, k, Hkv, D;
   int batch, max_blocks, num_blocks;
+  // fused compression (kara_compress): the keep sets come from these scores [L, R, Hkv, W]
+  // through selection and Token2Chunk in the gather's CTAs (keep may then be an output)
+  const float* scores = nullptr;
+  int32_t* keep_out = nullptr;
+  int num_anchors = 0, gap_limit = 0, widen = 0;
 };
 size_t compact_workspace_bytes(int R, int W, int k);
 kara_status launch_compact(const CompactLaunch& L, cudaStream_t stream);

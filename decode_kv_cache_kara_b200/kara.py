@@ -97,6 +97,8 @@ _SIGNATURES = {
     "kara_sum_heads": ([_P, _I, _I, _I, _P, _P], _I),
     "kara_expand_keep": ([_P, _I, _I, _I, _P, _P], _I),
     "kara_select_chunks": ([_P, _I, _I, _I, _I, _I, _I, _P, _P, _P], _I),
+    "kara_compress": ([_P, ctypes.POINTER(_LayerKV), _I, ctypes.POINTER(_Pool), _P, _I, _I, _I, _I,
+                       _I, _I, _P, _P, _Z, _P, _P], _I),
 }
 
 
@@ -296,6 +298,32 @@ def kara_select_chunks(scores: torch.Tensor, k: int, num_anchors: int, gap_limit
                                     _ptr(sel), _ptr(keep), _stream(stream)),
            "kara_select_chunks")
     return keep
+
+
+def kara_compress(scores: torch.Tensor, k_layers, v_layers, pool: PagedPool, window: int, k: int,
+                  num_anchors: int, gap_limit: int, widen: int,
+                  seq_ids: torch.Tensor | None = None, keep: torch.Tensor | None = None,
+                  workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """Selection, Token2Chunk and compaction of all layers from their scores
+    [L, R, Hkv, W] (in place on the pools and the PagedPool). Returns the status tensor."""
+    _require(scores, torch.float32, "scores")
+    nl, r, hkv, w = scores.shape
+    arr = _layers(k_layers, v_layers)
+    if nl != len(arr) or w != window:
+        raise ValueError("scores must be [layers, sequences, KV heads, window]")
+    if seq_ids is not None:
+        _require(seq_ids, torch.int32, "seq_ids")
+    if keep is not None:
+        _require(keep, torch.int32, "keep")
+    status = status if status is not None else new_status(scores.device)
+    ps = pool.c_struct()
+    ws = _workspace(kara_workspace_bytes(OP_COMPACT, pool, r, window, 0, k), scores.device,
+                    workspace)
+    _check(lib().kara_compress(_ptr(scores), arr, nl, ctypes.byref(ps), _ptr(seq_ids), r, window,
+                               k, num_anchors, gap_limit, widen, _ptr(keep), _ptr(ws),
+                               ws.numel(), _ptr(status), _stream(stream)), "kara_compress")
+    return status
 
 
 def kara_sum_heads(scores: torch.Tensor, out: torch.Tensor | None = None,

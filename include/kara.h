@@ -206,6 +206,23 @@ kara_status kara_select_chunks(const float* scores, int32_t rows, int32_t window
                                int32_t* sel, int32_t* keep, cudaStream_t stream);
 
 /*
+ * kara_compress - selection, Token2Chunk and compaction in two kernels (the compaction plan,
+ * which depends only on the windows' geometry, then one kernel per (layer, due sequence, KV
+ * head) that selects and expands the row in shared memory and gathers it into the fresh
+ * blocks; the last CTA of each sequence finalizes it). The result equals kara_select_chunks
+ * on each layer's scores followed by kara_compact, bit for bit.
+ *  scores   fp32 [num_layers, num_seqs, Hkv, window] (kara_score's output per layer).
+ *  keep     int32 [num_layers, num_seqs, Hkv, k] or NULL: the keep sets, written when given.
+ *  Other arguments, the workspace (KARA_OP_COMPACT), the device errors and their
+ *  all-or-nothing rule as kara_compact; selection arguments and limits as kara_select_chunks.
+ */
+kara_status kara_compress(const float* scores, const kara_layer_kv* layers, int32_t num_layers,
+                          const kara_pool* pool, const int32_t* seq_ids, int32_t num_seqs,
+                          int32_t window, int32_t k, int32_t num_anchors, int32_t gap_limit,
+                          int32_t widen, int32_t* keep, void* workspace, size_t workspace_bytes,
+                          int32_t* dev_status, cudaStream_t stream);
+
+/*
  * kara_compact - write the compressed windows into fresh blocks, rewrite the block table and
  * free the old window blocks ([KARA] abstract: Kara adapted to PagedAttention).
  *

@@ -352,3 +352,65 @@ def test_select_chunks_equals_select_then_token2chunk(name):
             ref = ok.token2chunk(s[r, g], ok.select_topk(s[r, g], wl.keep), na, wl.gap_limit,
                                  wl.widen)
             assert np.array_equal(H.i32(keep2[r, g]), ref)
+
+
+@pytest.mark.parametrize("name,layers,subset", [("g7_ragged_unaligned", 2, False),
+                                                ("g7_w512_ragged", 1, True),
+                                                ("d64_g4_w256", 3, False)])
+def test_compress_equals_select_chunks_then_compact(name, layers, subset):
+    """kara_compress (plan, then selection + Token2Chunk + gather in one kernel per row) leaves
+    the same cache, table, lengths, free list and keep sets as kara_select_chunks on every
+    layer followed by kara_compact, bit for bit; both against the oracle."""
+    wl = SCORE_CASES[name].with_(layers=layers)
+    cpu, dev_a = H.make(wl, 15)
+    dev_b = H.to_device(cpu)
+    ids = [1, 3] if subset else list(range(wl.batch))
+    assert wl.batch > max(ids)
+    seq = torch.tensor(ids, dtype=torch.int32, device="cuda")
+    na = K.anchors_for(wl.anchor_frac, wl.keep)
+    pool_a, pool_b = K.PagedPool.from_cache(dev_a), K.PagedPool.from_cache(dev_b)
+    scores = torch.stack([K.kara_score(dev_a["q_win"][l][ids].contiguous(), dev_a["k"][l], pool_a,
+                                       wl.window, seq_ids=seq) for l in range(layers)])
+    keep_a = torch.empty((layers, len(ids), wl.hkv, wl.keep), dtype=torch.int32, device="cuda")
+    for l in range(layers):
+        K.kara_select_chunks(scores[l], wl.keep, na, wl.gap_limit, wl.widen, keep=keep_a[l])
+    st_a = K.kara_compact(dev_a["k"], dev_a["v"], pool_a, wl.window, keep_a, seq_ids=seq)
+    keep_b = torch.empty_like(keep_a)
+    st_b = K.kara_compress(scores, dev_b["k"], dev_b["v"], pool_b, wl.window, wl.keep, na,
+                           wl.gap_limit, wl.widen, seq_ids=seq, keep=keep_b)
+    torch.cuda.synchronize()
+    assert K.read_status(st_a) == 0 and K.read_status(st_b) == 0
+    assert torch.equal(keep_a, keep_b)
+    for key in ("block_table", "ctx_len", "free_top"):
+        assert torch.equal(dev_a[key], dev_b[key])
+    top = int(dev_a["free_top"][0])
+    assert torch.equal(dev_a["free_list"][:top], dev_b["free_list"][:top])
+    bt, cl = H.i32(dev_a["block_table"]), H.i32(dev_a["ctx_len"])
+    for l in range(layers):
+        ka, kb = H.bits(dev_a["k"][l]), H.bits(dev_b["k"][l])
+        va, vb = H.bits(dev_a["v"][l]), H.bits(dev_b["v"][l])
+        for b in range(wl.batch):
+            n = int(cl[b])
+            assert np.array_equal(H.logical_rows(ka, bt[b], n), H.logical_rows(kb, bt[b], n))
+            assert np.array_equal(H.logical_rows(va, bt[b], n), H.logical_rows(vb, bt[b], n))
+    # and the oracle's compaction with those keep sets
+    check_compaction(dev_b, oracle_compact(cpu, wl, H.i32(keep_b), ids, layers), layers, ids,
+                     wl.batch)
+
+
+def test_compress_out_of_blocks_changes_nothing():
+    wl = SCORE_CASES["g7_ragged_unaligned"]
+    cpu, dev = H.make(wl, 16)
+    dev["free_top"].fill_(1)
+    pool = K.PagedPool.from_cache(dev)
+    before = {k2: dev[k2].clone() for k2 in ("block_table", "ctx_len", "free_top")}
+    kb = H.bits(dev["k"][0]).copy()
+    scores = K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window)[None]
+    na = K.anchors_for(wl.anchor_frac, wl.keep)
+    st = K.kara_compress(scores, dev["k"], dev["v"], pool, wl.window, wl.keep, na, wl.gap_limit,
+                         wl.widen)
+    torch.cuda.synchronize()
+    assert K.read_status(st) == K.ERR_OUT_OF_BLOCKS
+    for k2, t in before.items():
+        assert torch.equal(dev[k2], t)
+    assert np.array_equal(H.bits(dev["k"][0]), kb)
