@@ -74,6 +74,16 @@ def test_host_side_validation_returns_before_any_launch(lib_path):
     assert L.kara_reset_tails(one, one, 0, 4, null) == K.OK             # nothing to reset
     assert L.kara_score_ring(one, one, ctypes.byref(pool), null, 1, 5000, 4, 1.0, one, one,
                              1 << 20, one, null) == K.ERR_INVALID_ARG
+    # fused selection: more anchors than kept, k above the window; fused compression: the same,
+    # and a missing free list
+    assert L.kara_select_chunks(one, 2, 64, 8, 9, 8, 1, null, one, null) == K.ERR_INVALID_ARG
+    assert L.kara_select_chunks(one, 2, 64, 65, 4, 8, 1, null, one, null) == K.ERR_INVALID_ARG
+    assert L.kara_select_chunks(one, 0, 64, 8, 4, 8, 1, null, one, null) == K.OK
+    assert L.kara_compress(one, layers, 1, ctypes.byref(pool), null, 1, 64, 8, 9, 8, 1, null, one,
+                           1 << 20, one, null) == K.ERR_INVALID_ARG
+    nofree = K._Pool(1, 1, 0, 0, 1, 8, 64, 16, 2, 128)
+    assert L.kara_compress(one, layers, 1, ctypes.byref(nofree), null, 1, 64, 8, 4, 8, 1, null,
+                           one, 1 << 20, one, null) == K.ERR_INVALID_ARG
     # none of these reached a kernel launch
     assert K.kara_launch_count() == launches
 
