@@ -50,12 +50,6 @@ __device__ __forceinline__ int block_scan_add(int v, int* buf, int* total) {
 }
 
 // ---------------------------------------------------------------------------------------
-// bf16 <-> fp32 (bit-level; bf16 -> fp32 is exact)
-// ---------------------------------------------------------------------------------------
-__device__ __forceinline__ float bf16lo_to_f32(uint32_t packed) { return __uint_as_float(packed << 16); }
-__device__ __forceinline__ float bf16hi_to_f32(uint32_t packed) { return __uint_as_float(packed & 0xffff0000u); }
-
-// ---------------------------------------------------------------------------------------
 // Shared-memory addresses
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -242,25 +236,6 @@ __device__ __forceinline__ float lg2(float x) {
   return y;
 }
 
-// On the FMA pipe, so that part of the exponentials leaves the SFU: x = n + f with
-// n = round-to-nearest(x) (adding and subtracting 1.5 * 2^23 leaves n in the low mantissa
-// bits of the sum), f in [-1/2, 1/2]; 2^f by a degree-4 polynomial fitted for minimum
-// maximum relative error (csrc/gen_exp2_poly.py); 2^n by adding n to the exponent field,
-// which is (bits of the shifted sum) << 23 because the shifter's own bits vanish modulo 2^32.
-// Inputs below -125 are clamped (result ~2^-125 instead of a denormal or 0). Maximum
-// relative error over [-125, 0]: 2.7e-6.
-__device__ __forceinline__ float ex2_fma(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float n = t - 12582912.0f;
-  const float f = x - n;
-  float p = fmaf(0.009570102207362652f, f, 0.05591785907745361f);
-  p = fmaf(p, f, 0.240247443318367f);
-  p = fmaf(p, f, 0.6931217908859253f);
-  p = fmaf(p, f, 0.9999992847442627f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Packed fp32 pair arithmetic (one instruction for two lanes of work on sm_100).
 __device__ __forceinline__ uint64_t f2_bits(float2 a) { return *reinterpret_cast<uint64_t*>(&a); }
 __device__ __forceinline__ float2 bits_f2(uint64_t r) { return *reinterpret_cast<float2*>(&r); }
@@ -280,7 +255,13 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
   return bits_f2(r);
 }
 
-// ex2_fma on a pair, with packed fp32 arithmetic (same method and error as ex2_fma).
+// 2^x of a pair on the FMA pipe (packed fp32), so that part of the exponentials leaves the
+// SFU: x = n + f with n = round-to-nearest(x) (adding and subtracting 1.5 * 2^23 leaves n in
+// the low mantissa bits of the sum), f in [-1/2, 1/2]; 2^f by a degree-4 polynomial fitted for
+// minimum maximum relative error (csrc/gen_exp2_poly.py); 2^n by adding n to the exponent field,
+// which is (bits of the shifted sum) << 23 because the shifter's own bits vanish modulo 2^32.
+// Inputs below -125 are clamped (result ~2^-125 instead of a denormal or 0). Maximum
+// relative error over [-125, 0]: 2.7e-6.
 __device__ __forceinline__ float2 ex2_fma2(float2 x) {
   x.x = fmaxf(x.x, -125.0f);
   x.y = fmaxf(x.y, -125.0f);
@@ -323,13 +304,6 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t local, uint32_t rank) {
 }
 // Stores two floats into another CTA's shared memory and counts their 8 bytes on that CTA's
 // mbarrier (both addresses from map_to_rank).
-__device__ __forceinline__ void st_async_f2(uint32_t remote, float x, float y, uint32_t remote_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
-          remote),
-      "f"(x), "f"(y), "r"(remote_bar)
-      : "memory");
-}
 __device__ __forceinline__ void st_async_f32(uint32_t remote, float x, uint32_t remote_bar) {
   asm volatile(
       "st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote),
