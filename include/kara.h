@@ -52,7 +52,7 @@ extern "C" {
 typedef enum kara_status {
   KARA_OK = 0,
   KARA_ERR_INVALID_ARG = 1,   /* bad shape, size, pointer or parameter combination */
-  KARA_ERR_UNSUPPORTED = 2,   /* valid request outside what this build implements */
+  KARA_ERR_UNSUPPORTED = 2,   /* valid request outside what the library implements */
   KARA_ERR_OUT_OF_BLOCKS = 3, /* free list holds fewer blocks than the compaction needs */
   KARA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
   KARA_ERR_TIMEOUT = 5,       /* a bounded on-device wait ran out (kernel returned early) */
