@@ -533,6 +533,79 @@ def decode_loop_run(dev, steps: int = 300, period: int = 100, warm: int = 20) ->
                         f"steps, tails spread over [0, W)"}
 
 
+def lacache_loop_run(dev, steps: int = 200, period: int = 100, warm: int = 10) -> dict:
+    """LaCache inside the decode loop on the layer workload's shapes with 4 layers (batch 32,
+    28 query / 4 KV heads, d=128, 4096-token contexts): every step kara_step_begin, one
+    kara_decode_append per layer and kara_step_end with the capacity trigger; the ladder
+    (S = 2, O = 1, rung 64, sink 64, recent 64, budget 2048 per layer, so capacity
+    64 + 64 + 1920 * 4 / 2 = 3968 slots) runs on the sequences due at a check step. Timed with
+    CUDA events per step; a check step includes the host read of the due count."""
+    from decode_kv_cache_kara_b200 import kara as K
+    wl = WORKLOAD.with_(layers=4)
+    B, L = wl.batch, wl.layers
+    span, overlap, rung, budget, sink, recent = 2, 1, 64, 2048, 64, 64
+    cap = sink + recent + (budget - sink - recent) * L // span
+    # spare blocks: the steps' new pages, and a ladder pass pops budget / 16 fresh blocks per
+    # due sequence before it frees the old ones
+    cache = synth.make_cache(wl, 1234 + 7, dev, with_queries=False,
+                             extra_pages=(steps + warm) // wl.page + 2 + budget // wl.page)
+    pool = K.PagedPool.from_cache(cache)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + 8)
+    inputs = [[torch.randn(shape, generator=gen, device=dev).to(torch.bfloat16)
+               for shape in ((B, wl.hq, wl.head_dim), (B, wl.hkv, wl.head_dim),
+                             (B, wl.hkv, wl.head_dim))] for _ in range(8)]
+    out = torch.empty((B, wl.hq, wl.head_dim), dtype=torch.bfloat16, device=dev)
+    ws_dec = torch.empty(K.kara_workspace_bytes(K.OP_DECODE, pool, 0, 0, wl.hq, 0),
+                         dtype=torch.uint8, device=dev)
+    ws_lac = torch.empty(K.kara_workspace_bytes(K.OP_LACACHE, pool, B, 0, 0, budget),
+                         dtype=torch.uint8, device=dev)
+    due = torch.zeros(B, dtype=torch.int32, device=dev)
+    due_count = torch.zeros(1, dtype=torch.int32, device=dev)
+    status = K.new_status(dev)
+
+    def step(t, check):
+        q, kn, vn = inputs[t % len(inputs)]
+        K.kara_step_begin(pool, status)
+        for layer in range(L):
+            K.kara_decode_append(q, kn, vn, cache["k"][layer], cache["v"][layer], pool, out=out,
+                                 workspace=ws_dec, status=status)
+        K.kara_step_end(pool, None, 0, check, due, due_count, capacity=cap)
+        if not check:
+            return 0
+        cnt = int(due_count.item())
+        if cnt:
+            K.lacache_compact(cache["k"], cache["v"], pool, span, overlap, rung, budget, sink,
+                              recent, seq_ids=due[:cnt], workspace=ws_lac, status=status)
+        return cnt
+
+    for t in range(warm):
+        step(t, False)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    dues, checks = [], []
+    for t in range(steps):
+        check = (t + 1) % period == 0
+        ev[t][0].record()
+        n = step(warm + t, check)
+        ev[t][1].record()
+        if check:
+            dues.append(n)
+            checks.append(t)
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    plain = sorted(m for t, m in enumerate(ms) if t not in checks)
+    total = sum(ms)
+    return {"steps": steps, "period": period, "layers": L, "capacity": cap,
+            "ms_per_step": total / steps, "decode_step_ms": plain[len(plain) // 2],
+            "check_step_ms": [ms[t] for t in checks], "due_per_check": dues,
+            "tokens_per_s": B * steps / (total / 1e3), "status": K.read_status(status),
+            "workload": "LaCache in the decode loop: batch 32, 4 layers, 28 query / 4 KV heads, "
+                        "d=128, 4096-token contexts, S=2, O=1, rung 64, sink 64, recent 64, "
+                        f"budget {budget} per layer, capacity {cap}, check every {period} steps"}
+
+
 def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
     import torch.distributed as dist
     from decode_kv_cache_kara_b200 import kara as K
@@ -639,6 +712,7 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
         kernels["lacache_compact"] = lac
     if world == 1 and not args.no_loop:
         kernels["decode_loop"] = decode_loop_run(dev)
+        kernels["lacache_loop"] = lacache_loop_run(dev)
         kernels["variants"] = variants_run(step)
 
     cpu = None
