@@ -44,3 +44,30 @@ def test_neighbour_queries_follow_previous_key():
         kprev = c["k"][0][blk, s % 16].float()                     # [Hkv, d]
         diff = q[b, 5] - kprev.repeat_interleave(wl.group, 0)
         assert 0.3 < float(diff.std()) < 0.7
+
+
+def test_decode_step_inputs_are_seeded_and_shaped():
+    wl = synth.Workload("s", batch=3, layers=2, hq=8, hkv=2, head_dim=64, ctx_lo=20, ctx_hi=40,
+                        window=16, keep=4)
+    a = synth.decode_step_inputs(wl, 7, 3)
+    b = synth.decode_step_inputs(wl, 7, 3)
+    c = synth.decode_step_inputs(wl, 7, 4)
+    assert len(a) == wl.layers
+    for la, lb, lc in zip(a, b, c):
+        assert la["q"].shape == (3, 8, 64) and la["k"].shape == (3, 2, 64)
+        assert all(x.dtype == torch.bfloat16 for x in la.values())
+        assert all(torch.equal(la[n], lb[n]) for n in la)          # same (seed, step)
+        assert not torch.equal(la["k"], lc["k"])                   # another step differs
+    # each query head is its KV head's new key plus noise of scale 0.5
+    d = (a[0]["q"].float() - a[0]["k"].float().repeat_interleave(4, dim=1))
+    assert 0.3 < float(d.std()) < 0.7
+
+
+def test_extra_pages_add_table_columns_and_spare_blocks():
+    wl = synth.Workload("s", batch=3, layers=1, hq=2, hkv=1, head_dim=64, ctx_lo=20, ctx_hi=40,
+                        window=16, keep=4)
+    base = synth.make_cache(wl, 5, "cpu", with_queries=False)
+    more = synth.make_cache(wl, 5, "cpu", with_queries=False, extra_pages=4)
+    assert more["max_blocks"] == base["max_blocks"] + 4
+    assert more["num_blocks"] == base["num_blocks"] + 3 * 4
+    assert int(more["free_top"][0]) == int(base["free_top"][0]) + 3 * 4
