@@ -104,3 +104,34 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(K, "library_path", lambda: str(tmp_path / "nope.so"))
     with pytest.raises(K.KaraLibraryError):
         K.lib()
+
+
+def test_binding_refuses_host_tensors():
+    """No CPU fallback: every compute call of the binding refuses host tensors before it
+    reaches the library (there is no other path to take)."""
+    import torch
+
+    w, k = 32, 8
+    s = torch.zeros((2, 2, w))
+    q = torch.zeros((2, w, 4, 64), dtype=torch.bfloat16)
+    kv = torch.zeros((4, 16, 2, 64), dtype=torch.bfloat16)
+    sel = torch.zeros((2, 2, k), dtype=torch.int32)
+    pool = K.PagedPool(torch.zeros((2, 4), dtype=torch.int32), torch.zeros(2, dtype=torch.int32),
+                       torch.zeros(4, dtype=torch.int32), torch.zeros(1, dtype=torch.int32), 4, 2,
+                       64)
+    calls = {
+        "kara_score": lambda: K.kara_score(q, kv, pool, w),
+        "kara_score_ex": lambda: K.kara_score_ex(q, kv, pool, w),
+        "kara_select": lambda: K.kara_select(s, k),
+        "kara_token2chunk": lambda: K.kara_token2chunk(s, sel, 4, 8, 1),
+        "kara_select_chunks": lambda: K.kara_select_chunks(s, k, 4, 8, 1),
+        "kara_sum_heads": lambda: K.kara_sum_heads(s),
+        "kara_expand_keep": lambda: K.kara_expand_keep(sel[:, 0].contiguous(), 2),
+        "kara_compact": lambda: K.kara_compact([kv], [kv], pool, w, sel[None]),
+        "kara_compress": lambda: K.kara_compress(s[None], [kv], [kv], pool, w, k, 4, 8, 1),
+        "paged_decode_attn": lambda: K.paged_decode_attn(q[:, 0], kv, kv, pool),
+        "kara_decode_append": lambda: K.kara_decode_append(q[:, 0], kv[0], kv[0], kv, kv, pool),
+    }
+    for name, fn in calls.items():
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            fn()
