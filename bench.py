@@ -740,8 +740,9 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
     return line
 
 
-def cpu_baseline(seed: int, target_s: float = 12.0) -> dict:
-    """The oracle as it stands on the host cores, on a bounded sample of the same workload."""
+def cpu_baseline(seed: int, target_s: float = 15.0) -> dict:
+    """The oracle as it stands on the host cores, on a bounded sample of the same workload:
+    as many (sequence, KV head) units as take about target_s seconds (at most 256)."""
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
@@ -750,7 +751,7 @@ def cpu_baseline(seed: int, target_s: float = 12.0) -> dict:
     cache_cpu = synth.make_cache(WORKLOAD, seed, "cpu")
     dt, tokens = time_cpu_oracle_sample(cache_cpu, WORKLOAD, units=1, seed=seed)
     units = max(1, int(target_s / max(dt, 1e-3)))
-    units = min(units, 64)
+    units = min(units, 256)
     dt, tokens = time_cpu_oracle_sample(cache_cpu, WORKLOAD, units=units, seed=seed + 1)
     return {"value": tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{units} (sequence, KV head) units of the layer workload: window scoring "
