@@ -184,7 +184,7 @@ class Step:
                  K.kara_workspace_bytes(K.OP_COMPACT, self.pool, r, wl.window, 0, wl.keep),
                  K.kara_workspace_bytes(K.OP_DECODE, self.pool, 0, 0, hq, 0))
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
-        self.na = K.anchors_for(wl.anchor_frac, wl.keep)
+        self.na = wl.anchor_frac
         # scoring: the fused cluster kernel for windows of 128/256/512/1024 keys (plus the
         # split-item sum when a cluster range ends inside an item), else two passes and a
         # merge; select + Token2Chunk in one kernel; compaction plan + gather; decode + combine
@@ -483,7 +483,7 @@ def decode_loop_run(dev, steps: int = 300, period: int = 100, warm: int = 20) ->
     due = torch.zeros(B, dtype=torch.int32, device=dev)
     due_count = torch.zeros(1, dtype=torch.int32, device=dev)
     status = K.new_status(dev)
-    na = K.anchors_for(wl.anchor_frac, wl.keep)
+    na = wl.anchor_frac
 
     def step(t, check):
         q, kn, vn = inputs[t % len(inputs)]

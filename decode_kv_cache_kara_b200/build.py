@@ -49,14 +49,23 @@ def build(verbose: bool = False, extra_flags=None) -> str:
     """Compile every source to an object, then link libkara.so. Returns the library path."""
     os.makedirs(BUILD_DIR, exist_ok=True)
     cc = nvcc()
-    objs = []
     flags = NVCC_FLAGS + ARCH + ["-I", INCLUDE, "-I", CSRC] + list(extra_flags or [])
-    for src in sources():
+
+    def compile_one(src):
         obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
         cmd = [cc, "-c", src, "-o", obj] + flags
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        return src, obj, cmd, res
+
+    # one nvcc process per source, in parallel
+    from concurrent.futures import ThreadPoolExecutor
+    srcs = sources()
+    with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as pool:
+        results = list(pool.map(compile_one, srcs))
+    objs = []
+    for src, obj, cmd, res in results:
         if verbose:
             print(" ".join(cmd), flush=True)
-        res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError(f"nvcc failed for {src}:\n{res.stdout}\n{res.stderr}")
         if verbose and res.stderr.strip():

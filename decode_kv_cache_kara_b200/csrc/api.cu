@@ -1,6 +1,7 @@
 // C-ABI entry points of libkara: host-side argument checks, workspace carving, launches.
 // Semantics of every call are documented in include/kara.h.
 #include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -50,6 +51,17 @@ kara_status check_pool(const kara_pool* pool) {
   if (pool->head_dim != 64 && pool->head_dim != 128) return KARA_ERR_UNSUPPORTED;
   if (pool->num_kv_heads <= 0) return KARA_ERR_INVALID_ARG;
   return KARA_OK;
+}
+
+// Token2Chunk step (a): the anchors are the top ceil(anchor_frac * k) of the selection. The
+// product is rounded to 6 decimals before the ceiling, so that a float fraction such as 0.2f
+// (0.2000000030) gives ceil(0.2 * 5) = 1 as the decimal fraction would. Returns -1 for a
+// fraction outside [0, 1] (or NaN).
+int anchors_from_frac(float anchor_frac, int32_t k) {
+  if (!(anchor_frac >= 0.f && anchor_frac <= 1.f)) return -1;
+  const double x = std::nearbyint(static_cast<double>(anchor_frac) * k * 1e6) / 1e6;
+  const int n = static_cast<int>(std::ceil(x));
+  return n < 0 ? 0 : (n > k ? k : n);
 }
 
 kara_status check_heads(const kara_pool* pool, int32_t num_q_heads) {
@@ -252,12 +264,12 @@ kara_status kara_select(const float* scores, int32_t rows, int32_t window, int32
 }
 
 kara_status kara_token2chunk(const float* scores, const int32_t* sel, int32_t rows,
-                             int32_t window, int32_t k, int32_t num_anchors, int32_t gap_limit,
+                             int32_t window, int32_t k, float anchor_frac, int32_t gap_limit,
                              int32_t widen, int32_t* keep, cudaStream_t stream) {
   if (rows < 0 || window < 1 || window > KARA_MAX_WINDOW || k < 1 || k > window)
     return KARA_ERR_INVALID_ARG;
-  if (num_anchors < 0 || num_anchors > k || gap_limit < 0 || widen < 0)
-    return KARA_ERR_INVALID_ARG;
+  const int num_anchors = anchors_from_frac(anchor_frac, k);
+  if (num_anchors < 0 || gap_limit < 0 || widen < 0) return KARA_ERR_INVALID_ARG;
   if (rows == 0) return KARA_OK;
   if (scores == nullptr || sel == nullptr || keep == nullptr) return KARA_ERR_INVALID_ARG;
   return launch_token2chunk(scores, sel, rows, window, k, num_anchors, gap_limit, widen, keep,
@@ -265,12 +277,12 @@ kara_status kara_token2chunk(const float* scores, const int32_t* sel, int32_t ro
 }
 
 kara_status kara_select_chunks(const float* scores, int32_t rows, int32_t window, int32_t k,
-                               int32_t num_anchors, int32_t gap_limit, int32_t widen,
+                               float anchor_frac, int32_t gap_limit, int32_t widen,
                                int32_t* sel, int32_t* keep, cudaStream_t stream) {
   if (rows < 0 || window < 1 || window > KARA_MAX_WINDOW || k < 1 || k > window)
     return KARA_ERR_INVALID_ARG;
-  if (num_anchors < 0 || num_anchors > k || gap_limit < 0 || widen < 0)
-    return KARA_ERR_INVALID_ARG;
+  const int num_anchors = anchors_from_frac(anchor_frac, k);
+  if (num_anchors < 0 || gap_limit < 0 || widen < 0) return KARA_ERR_INVALID_ARG;
   if (rows == 0) return KARA_OK;
   if (scores == nullptr || keep == nullptr) return KARA_ERR_INVALID_ARG;
   return launch_select_chunks(scores, rows, window, k, num_anchors, gap_limit, widen, sel, keep,
@@ -315,7 +327,7 @@ kara_status kara_compact(const kara_layer_kv* layers, int32_t num_layers, const 
 
 kara_status kara_compress(const float* scores, const kara_layer_kv* layers, int32_t num_layers,
                           const kara_pool* pool, const int32_t* seq_ids, int32_t num_seqs,
-                          int32_t window, int32_t k, int32_t num_anchors, int32_t gap_limit,
+                          int32_t window, int32_t k, float anchor_frac, int32_t gap_limit,
                           int32_t widen, int32_t* keep, void* workspace, size_t workspace_bytes,
                           int32_t* dev_status, cudaStream_t stream) {
   kara_status st = check_pool(pool);
@@ -323,8 +335,8 @@ kara_status kara_compress(const float* scores, const kara_layer_kv* layers, int3
   if (pool->free_list == nullptr || pool->free_top == nullptr) return KARA_ERR_INVALID_ARG;
   if (num_seqs < 0 || window < 1 || window > KARA_MAX_WINDOW || k < 1 || k > window)
     return KARA_ERR_INVALID_ARG;
-  if (num_anchors < 0 || num_anchors > k || gap_limit < 0 || widen < 0)
-    return KARA_ERR_INVALID_ARG;
+  const int num_anchors = anchors_from_frac(anchor_frac, k);
+  if (num_anchors < 0 || gap_limit < 0 || widen < 0) return KARA_ERR_INVALID_ARG;
   if (num_seqs == 0) return KARA_OK;
   if (scores == nullptr || dev_status == nullptr) return KARA_ERR_INVALID_ARG;
   CompactLaunch L;

@@ -6,7 +6,10 @@
 // ...": states outside the ladder are dropped and the rest packed into a smaller cache
 // (method details), re-applied when the cache is full (iterative compaction).
 //
-// Two stream-ordered kernels per call:
+// Stream-ordered kernels per call:
+//   check    (kara_compact only, a few CTAs) checks the caller's keep sets: every entry a
+//                        window position, every row strictly ascending; the plan reads the
+//                        verdicts and refuses the whole call on a bad entry.
 //   plan     (one CTA)   validates every due sequence, computes its page geometry and pops its
 //                        fresh blocks from the free list (sequence order, stack top first); on
 //                        any error it records the status and marks the plan invalid.
@@ -22,6 +25,7 @@
 //                        then. The plan sets free_top (nothing later in the call reads it).
 // The gather reads only blocks that belong to the sequences and writes only fresh blocks, so
 // sources never alias destinations; nothing is modified unless the plan is valid.
+#include <algorithm>
 #include <cstdint>
 #include <mutex>
 
@@ -34,7 +38,12 @@ namespace kara {
 namespace {
 
 constexpr int kPlanThreads = 1024;
-constexpr int kPlanHeader = 16;   // valid, total_new, total_old, top
+// Header: [0..4) valid, total_new, total_old, top; [16, 16 + kCheckCtas) the verdicts of the
+// keep check's CTAs (nonzero = a bad entry in that CTA's rows)
+constexpr int kCheckCtas = 128;
+constexpr int kCheckThreads = 512;
+constexpr int kHdrCheck = 16;
+constexpr int kPlanHeader = kHdrCheck + kCheckCtas;
 constexpr int kPlanStride = 12;   // b, n, start, off, p0, n_old, n_new, base_new, base_old, done
 enum { P_B = 0, P_N, P_START, P_OFF, P_P0, P_NOLD, P_NNEW, P_BNEW, P_BOLD, P_DONE };
 
@@ -50,7 +59,41 @@ struct PlanParams {
   int R, batch, max_blocks, num_blocks;
   // Kara: window W and budget k. LaCache: W = 0, k = budget, min_len = sink+recent+R_max.
   int W, k, lacache, min_len;
+  int check_ctas;   // CTAs of the keep check that ran before the plan (0: no check)
 };
+
+// The caller's keep sets, before anything is planned: every entry of every (layer, sequence,
+// KV head) row must be a window position (0 <= pos < W) and each row strictly ascending.
+// Each CTA writes its verdict to its own header slot (so nothing has to be cleared first);
+// the plan refuses the call, moving and freeing nothing, when any verdict is nonzero.
+struct KeepCheck {
+  const int32_t* keep;
+  int32_t* plan;
+  long long rows;
+  int k, W;
+};
+
+__global__ void __launch_bounds__(kCheckThreads) keep_check_kernel(const KeepCheck c) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // keep is complete (PDL launch)
+  __shared__ int s_bad;
+  if (threadIdx.x == 0) s_bad = 0;
+  __syncthreads();
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  constexpr int kWarps = kCheckThreads / 32;
+  int bad = 0;
+  for (long long row = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+       row < c.rows; row += static_cast<long long>(gridDim.x) * kWarps) {
+    const int32_t* kr = c.keep + row * c.k;
+    for (int t = lane; t < c.k; t += 32) {
+      const int pos = kr[t];
+      if (pos < 0 || pos >= c.W || (t > 0 && kr[t - 1] >= pos)) bad = 1;
+    }
+  }
+  if (bad) s_bad = 1;
+  __syncthreads();
+  if (threadIdx.x == 0) c.plan[kHdrCheck + blockIdx.x] = s_bad;
+}
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
@@ -129,6 +172,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
     if (top >= 0 && top <= p.num_blocks && carry_new <= top)
       for (int i = threadIdx.x; i < carry_new; i += kPlanThreads) fresh[i] = p.free_list[top - 1 - i];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x < p.check_ctas && hdr[kHdrCheck + threadIdx.x] != 0)
+      atomicCAS(&err, 0, KARA_ERR_INVALID_ARG);     // a keep entry outside the window
     for (int r = warp; r < p.R; r += kPlanThreads / 32) {
       const int32_t* row = rows + static_cast<size_t>(r) * kPlanStride;
       const int n_old = row[P_NOLD];
@@ -270,8 +315,7 @@ __global__ void __launch_bounds__(kGatherThreads) kara_gather_kernel(const KaraG
       } else {
         const int t = t0 + (i - npre);
         const int pos = s_keep[i - npre];
-        if (pos < 0 || pos >= g.W) {      // keep entry outside the window: row left unwritten
-          report(g.status, KARA_ERR_INVALID_ARG);
+        if (pos < 0 || pos >= g.W) {      // refused by the plan already; never read outside
           act[u] = false;
           continue;
         }
@@ -526,6 +570,19 @@ kara_status launch_compact(const CompactLaunch& L, cudaStream_t stream) {
   pp.k = L.k;
   pp.lacache = 0;
   pp.min_len = 0;
+  pp.check_ctas = 0;
+  if (L.scores == nullptr) {   // the caller's keep sets: checked before the plan
+    KeepCheck kc;
+    kc.keep = L.keep;
+    kc.plan = L.plan;
+    kc.rows = static_cast<long long>(L.L) * L.R * L.Hkv;
+    kc.k = L.k;
+    kc.W = L.W;
+    const long long per_cta = kCheckThreads / 32;
+    const int ctas = static_cast<int>(std::min<long long>(kCheckCtas, (kc.rows + per_cta - 1) / per_cta));
+    launch_pdl(keep_check_kernel, dim3(ctas), dim3(kCheckThreads), 0, stream, kc);
+    pp.check_ctas = ctas;
+  }
   launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), 0, stream, pp);
   KaraGather g;
   g.layers = L.layers;
@@ -592,6 +649,7 @@ kara_status launch_lacache(const LacacheLaunch& L, cudaStream_t stream) {
   pp.k = L.budget;
   pp.lacache = 1;
   pp.min_len = L.sink + L.recent + r_max;
+  pp.check_ctas = 0;
   launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), 0, stream, pp);
   LadderGather g;
   g.layers = L.layers;

@@ -71,7 +71,7 @@ _Z = ctypes.c_size_t
 _SIGNATURES = {
     "kara_score": ([_P, _P, ctypes.POINTER(_Pool), _P, _I, _I, _I, _F, _P, _P, _Z, _P, _P], _I),
     "kara_select": ([_P, _I, _I, _I, _P, _P], _I),
-    "kara_token2chunk": ([_P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
+    "kara_token2chunk": ([_P, _P, _I, _I, _I, _F, _I, _I, _P, _P], _I),
     "kara_compact": ([ctypes.POINTER(_LayerKV), _I, ctypes.POINTER(_Pool), _P, _I, _I, _I, _P, _P,
                       _Z, _P, _P], _I),
     "kara_compact_noalloc": ([ctypes.POINTER(_LayerKV), _I, ctypes.POINTER(_Pool), _P, _I, _I, _I,
@@ -96,8 +96,8 @@ _SIGNATURES = {
                        _P], _I),
     "kara_sum_heads": ([_P, _I, _I, _I, _P, _P], _I),
     "kara_expand_keep": ([_P, _I, _I, _I, _P, _P], _I),
-    "kara_select_chunks": ([_P, _I, _I, _I, _I, _I, _I, _P, _P, _P], _I),
-    "kara_compress": ([_P, ctypes.POINTER(_LayerKV), _I, ctypes.POINTER(_Pool), _P, _I, _I, _I, _I,
+    "kara_select_chunks": ([_P, _I, _I, _I, _F, _I, _I, _P, _P, _P], _I),
+    "kara_compress": ([_P, ctypes.POINTER(_LayerKV), _I, ctypes.POINTER(_Pool), _P, _I, _I, _I, _F,
                        _I, _I, _P, _P, _Z, _P, _P], _I),
 }
 
@@ -212,9 +212,19 @@ def kara_workspace_bytes(op: int, pool: PagedPool | None = None, num_seqs: int =
 
 
 def _workspace(nbytes: int, device, workspace):
+    """The caller's workspace (a contiguous CUDA uint8 tensor), or a new one of nbytes."""
     if workspace is not None:
+        _require(workspace, torch.uint8, "workspace")
         return workspace
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def _status(status, device):
+    """The caller's status word (a CUDA int32 tensor), or a new zeroed one."""
+    if status is None:
+        return new_status(device)
+    _require(status, torch.int32, "status")
+    return status
 
 
 def kara_score(q_win: torch.Tensor, k_cache: torch.Tensor, pool: PagedPool, window: int,
@@ -235,7 +245,7 @@ def kara_score(q_win: torch.Tensor, k_cache: torch.Tensor, pool: PagedPool, wind
     _require(scores, torch.float32, "scores")
     if seq_ids is not None:
         _require(seq_ids, torch.int32, "seq_ids")
-    status = status if status is not None else new_status(q_win.device)
+    status = _status(status, q_win.device)
     ps = pool.c_struct()
     nbytes = kara_workspace_bytes(OP_SCORE, pool, r, window, hq)
     ws = _workspace(nbytes, q_win.device, workspace)
@@ -270,7 +280,7 @@ def kara_score_ex(q: torch.Tensor, k_cache: torch.Tensor, pool: PagedPool, windo
         scores = torch.empty((num_seqs, pool.num_kv_heads, window), dtype=torch.float32,
                              device=q.device)
     _require(scores, torch.float32, "scores")
-    status = status if status is not None else new_status(q.device)
+    status = _status(status, q.device)
     ps = pool.c_struct()
     ws = _workspace(kara_workspace_bytes(OP_SCORE, pool, num_seqs, window, hq), q.device,
                     workspace)
@@ -281,7 +291,7 @@ def kara_score_ex(q: torch.Tensor, k_cache: torch.Tensor, pool: PagedPool, windo
     return scores
 
 
-def kara_select_chunks(scores: torch.Tensor, k: int, num_anchors: int, gap_limit: int,
+def kara_select_chunks(scores: torch.Tensor, k: int, anchor_frac: float, gap_limit: int,
                        widen: int, keep: torch.Tensor | None = None,
                        sel: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """kara_select + kara_token2chunk in one kernel: keep [..., k] int32 (sel, if given, gets
@@ -294,14 +304,14 @@ def kara_select_chunks(scores: torch.Tensor, k: int, num_anchors: int, gap_limit
     _require(keep, torch.int32, "keep")
     if sel is not None:
         _require(sel, torch.int32, "sel")
-    _check(lib().kara_select_chunks(_ptr(scores), rows, w, k, num_anchors, gap_limit, widen,
+    _check(lib().kara_select_chunks(_ptr(scores), rows, w, k, float(anchor_frac), gap_limit, widen,
                                     _ptr(sel), _ptr(keep), _stream(stream)),
            "kara_select_chunks")
     return keep
 
 
 def kara_compress(scores: torch.Tensor, k_layers, v_layers, pool: PagedPool, window: int, k: int,
-                  num_anchors: int, gap_limit: int, widen: int,
+                  anchor_frac: float, gap_limit: int, widen: int,
                   seq_ids: torch.Tensor | None = None, keep: torch.Tensor | None = None,
                   workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
                   stream=None) -> torch.Tensor:
@@ -316,12 +326,12 @@ def kara_compress(scores: torch.Tensor, k_layers, v_layers, pool: PagedPool, win
         _require(seq_ids, torch.int32, "seq_ids")
     if keep is not None:
         _require(keep, torch.int32, "keep")
-    status = status if status is not None else new_status(scores.device)
+    status = _status(status, scores.device)
     ps = pool.c_struct()
     ws = _workspace(kara_workspace_bytes(OP_COMPACT, pool, r, window, 0, k), scores.device,
                     workspace)
     _check(lib().kara_compress(_ptr(scores), arr, nl, ctypes.byref(ps), _ptr(seq_ids), r, window,
-                               k, num_anchors, gap_limit, widen, _ptr(keep), _ptr(ws),
+                               k, float(anchor_frac), gap_limit, widen, _ptr(keep), _ptr(ws),
                                ws.numel(), _ptr(status), _stream(stream)), "kara_compress")
     return status
 
@@ -334,6 +344,7 @@ def kara_sum_heads(scores: torch.Tensor, out: torch.Tensor | None = None,
     rows = scores.numel() // (hkv * w) if hkv * w else 0
     if out is None:
         out = torch.empty(scores.shape[:-2] + (w,), dtype=torch.float32, device=scores.device)
+    _require(out, torch.float32, "out")
     _check(lib().kara_sum_heads(_ptr(scores), rows, hkv, w, _ptr(out), _stream(stream)),
            "kara_sum_heads")
     return out
@@ -348,6 +359,7 @@ def kara_expand_keep(keep_shared: torch.Tensor, num_kv_heads: int,
     if keep is None:
         keep = torch.empty(keep_shared.shape[:-1] + (num_kv_heads, k), dtype=torch.int32,
                            device=keep_shared.device)
+    _require(keep, torch.int32, "keep")
     _check(lib().kara_expand_keep(_ptr(keep_shared), rows, num_kv_heads, k, _ptr(keep),
                                   _stream(stream)), "kara_expand_keep")
     return keep
@@ -366,9 +378,10 @@ def kara_select(scores: torch.Tensor, k: int, sel: torch.Tensor | None = None,
     return sel
 
 
-def kara_token2chunk(scores: torch.Tensor, sel: torch.Tensor, num_anchors: int, gap_limit: int,
+def kara_token2chunk(scores: torch.Tensor, sel: torch.Tensor, anchor_frac: float, gap_limit: int,
                      widen: int, keep: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Token2Chunk expansion and trim: [..., k] int32 ascending."""
+    """Token2Chunk expansion and trim with ceil(anchor_frac * k) anchors: [..., k] int32
+    ascending."""
     _require(scores, torch.float32, "scores")
     _require(sel, torch.int32, "sel")
     w = scores.shape[-1]
@@ -377,7 +390,7 @@ def kara_token2chunk(scores: torch.Tensor, sel: torch.Tensor, num_anchors: int, 
     if keep is None:
         keep = torch.empty_like(sel)
     _require(keep, torch.int32, "keep")
-    _check(lib().kara_token2chunk(_ptr(scores), _ptr(sel), rows, w, k, int(num_anchors),
+    _check(lib().kara_token2chunk(_ptr(scores), _ptr(sel), rows, w, k, float(anchor_frac),
                                   int(gap_limit), int(widen), _ptr(keep), _stream(stream)),
            "kara_token2chunk")
     return keep
@@ -407,7 +420,7 @@ def kara_compact(k_layers, v_layers, pool: PagedPool, window: int, keep: torch.T
         raise ValueError("keep's first dimension must equal the number of layers")
     if seq_ids is not None:
         _require(seq_ids, torch.int32, "seq_ids")
-    status = status if status is not None else new_status(keep.device)
+    status = _status(status, keep.device)
     ps = pool.c_struct()
     nbytes = kara_workspace_bytes(OP_COMPACT, pool, r, window, 0, k)
     ws = _workspace(nbytes, keep.device, workspace)
@@ -432,6 +445,7 @@ def kara_compact_noalloc(k_layers, v_layers, pool: PagedPool, window: int, keep:
         _require(seq_ids, torch.int32, "seq_ids")
     if status is None:
         raise ValueError("pass a preallocated status tensor (this call allocates nothing)")
+    _require(status, torch.int32, "status")
     ps = pool.c_struct()
     _check(lib().kara_compact_noalloc(arr, nl, ctypes.byref(ps), _ptr(seq_ids), r, window, k,
                                       _ptr(keep), _ptr(status), _stream(stream)),
@@ -453,7 +467,7 @@ def paged_decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Ten
     if out is None:
         out = torch.empty_like(q)
     _require(out, torch.bfloat16, "out")
-    status = status if status is not None else new_status(q.device)
+    status = _status(status, q.device)
     ps = pool.c_struct()
     nbytes = kara_workspace_bytes(OP_DECODE, pool, 0, 0, hq, 0)
     ws = _workspace(nbytes, q.device, workspace)
@@ -481,7 +495,7 @@ def kara_score_ring(q_ring: torch.Tensor, k_cache: torch.Tensor, pool: PagedPool
         scores = torch.empty((num_seqs, pool.num_kv_heads, window), dtype=torch.float32,
                              device=q_ring.device)
     _require(scores, torch.float32, "scores")
-    status = status if status is not None else new_status(q_ring.device)
+    status = _status(status, q_ring.device)
     ps = pool.c_struct()
     ws = _workspace(kara_workspace_bytes(OP_SCORE, pool, num_seqs, window, hq), q_ring.device,
                     workspace)
@@ -510,7 +524,7 @@ def kara_decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor
     if out is None:
         out = torch.empty_like(q)
     _require(out, torch.bfloat16, "out")
-    status = status if status is not None else new_status(q.device)
+    status = _status(status, q.device)
     ps = pool.c_struct()
     ws = _workspace(kara_workspace_bytes(OP_DECODE, pool, 0, 0, hq, 0), q.device, workspace)
     _check(lib().kara_decode_append(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
@@ -522,6 +536,7 @@ def kara_decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor
 
 def kara_step_begin(pool: PagedPool, status: torch.Tensor, stream=None) -> None:
     """Blocks for the slots a decode step appends (see include/kara.h)."""
+    _require(status, torch.int32, "status")
     ps = pool.c_struct()
     _check(lib().kara_step_begin(ctypes.byref(ps), _ptr(status), _stream(stream)),
            "kara_step_begin")
@@ -535,6 +550,9 @@ def kara_step_end(pool: PagedPool, tail: torch.Tensor | None = None, window: int
     ctx_len >= capacity) and their count."""
     if tail is not None:
         _require(tail, torch.int32, "tail")
+    for t, name in ((due, "due"), (due_count, "due_count")):
+        if t is not None:
+            _require(t, torch.int32, name)
     ps = pool.c_struct()
     _check(lib().kara_step_end(ctypes.byref(ps), _ptr(tail), int(window), int(capacity),
                                1 if check else 0, _ptr(due), _ptr(due_count), _stream(stream)),
@@ -559,7 +577,7 @@ def lacache_compact(k_layers, v_layers, pool: PagedPool, span: int, overlap: int
     r = int(seq_ids.numel()) if seq_ids is not None else int(pool.block_table.shape[0])
     if seq_ids is not None:
         _require(seq_ids, torch.int32, "seq_ids")
-    status = status if status is not None else new_status(device)
+    status = _status(status, device)
     ps = pool.c_struct()
     prm = _LacacheParams(span, overlap, rung, budget, sink, recent)
     nbytes = kara_workspace_bytes(OP_LACACHE, pool, r, 0, 0, budget)
@@ -574,12 +592,7 @@ def kara_wait_probe(wait_ms: int, status: torch.Tensor | None = None, device="cu
                     stream=None) -> torch.Tensor:
     """Runs the bounded-wait probe (a wait that times out after about `wait_ms`). Returns the
     status tensor, which holds KARA_ERR_TIMEOUT once the stream completes."""
-    status = status if status is not None else new_status(torch.device(device))
+    status = _status(status, torch.device(device))
     _check(lib().kara_wait_probe(int(wait_ms), _ptr(status), _stream(stream)), "kara_wait_probe")
     return status
 
-
-def anchors_for(anchor_frac: float, k: int) -> int:
-    """ceil(anchor_frac * k) clipped to [0, k]: the num_anchors argument of Token2Chunk."""
-    n = int(math.ceil(round(anchor_frac * k, 9)))
-    return max(0, min(k, n))

@@ -186,17 +186,20 @@ kara_status kara_select(const float* scores, int32_t rows, int32_t window, int32
  * to budget ([KARA] abstract: a Token2Chunk module grows some of the selected KV pairs into
  * chunks; [GIST] section 2: the span between two important points is kept as one chunk).
  *
- * Per row, in window positions: anchors = the num_anchors selected positions with the largest
- * scores (ties: lower position); every position strictly between two consecutive anchors is
+ * Per row, in window positions: anchors = the num_anchors = ceil(anchor_frac * k) selected
+ * positions with the largest scores (ties: lower position; the product is rounded to 6
+ * decimals before the ceiling, so that a float fraction such as 0.2f counts as 0.2); every
+ * position strictly between two consecutive anchors is
  * added when there are 1..gap_limit of them; every position within `widen` of an anchor is
  * added; the union U (which contains sel) is trimmed to the k members with the largest
  * (priority, score, -position), priority 2 = anchor, 1 = in a run of consecutive U positions
  * that contains an anchor, 0 = other. keep [rows, k] is written ascending.
  *  scores fp32 [rows, window]; sel int32 [rows, k] ascending (as from kara_select).
- *  0 <= num_anchors <= k (callers use ceil(anchor_frac * k)), gap_limit >= 0, widen >= 0.
+ *  0 <= anchor_frac <= 1 (the step workload: 0.5), gap_limit >= 0, widen >= 0; otherwise
+ *  KARA_ERR_INVALID_ARG.
  */
 kara_status kara_token2chunk(const float* scores, const int32_t* sel, int32_t rows,
-                             int32_t window, int32_t k, int32_t num_anchors, int32_t gap_limit,
+                             int32_t window, int32_t k, float anchor_frac, int32_t gap_limit,
                              int32_t widen, int32_t* keep, cudaStream_t stream);
 
 /*
@@ -206,7 +209,7 @@ kara_status kara_token2chunk(const float* scores, const int32_t* sel, int32_t ro
  * the selection is written there too. Arguments and limits as the two calls.
  */
 kara_status kara_select_chunks(const float* scores, int32_t rows, int32_t window, int32_t k,
-                               int32_t num_anchors, int32_t gap_limit, int32_t widen,
+                               float anchor_frac, int32_t gap_limit, int32_t widen,
                                int32_t* sel, int32_t* keep, cudaStream_t stream);
 
 /*
@@ -222,7 +225,7 @@ kara_status kara_select_chunks(const float* scores, int32_t rows, int32_t window
  */
 kara_status kara_compress(const float* scores, const kara_layer_kv* layers, int32_t num_layers,
                           const kara_pool* pool, const int32_t* seq_ids, int32_t num_seqs,
-                          int32_t window, int32_t k, int32_t num_anchors, int32_t gap_limit,
+                          int32_t window, int32_t k, float anchor_frac, int32_t gap_limit,
                           int32_t widen, int32_t* keep, void* workspace, size_t workspace_bytes,
                           int32_t* dev_status, cudaStream_t stream);
 
@@ -241,10 +244,12 @@ kara_status kara_compress(const float* scores, const kara_layer_kv* layers, int3
  * unwritten.
  *  layers     HOST array of num_layers (1 .. KARA_MAX_LAYERS) pool pointers.
  *  seq_ids    device int32 [num_seqs], strictly increasing, or NULL (rows 0..num_seqs-1).
- *  keep       int32 [num_layers, num_seqs, num_kv_heads, k], ascending window positions.
+ *  keep       int32 [num_layers, num_seqs, num_kv_heads, k], strictly ascending window
+ *             positions (0 <= keep < window), checked on the device before anything moves.
  *  workspace  >= kara_workspace_bytes(KARA_OP_COMPACT, ...).
- *  dev_status KARA_ERR_OUT_OF_BLOCKS / KARA_ERR_INVALID_ARG / KARA_ERR_BAD_BLOCK: then no
- *             pool, table, length or free-list entry is modified.
+ *  dev_status KARA_ERR_OUT_OF_BLOCKS / KARA_ERR_INVALID_ARG (a short context, a bad seq_ids
+ *             entry, or a keep entry outside the window or out of order) / KARA_ERR_BAD_BLOCK:
+ *             then no pool, table, length or free-list entry is modified.
  */
 kara_status kara_compact(const kara_layer_kv* layers, int32_t num_layers, const kara_pool* pool,
                          const int32_t* seq_ids, int32_t num_seqs, int32_t window, int32_t k,
@@ -262,9 +267,13 @@ kara_status kara_compact(const kara_layer_kv* layers, int32_t num_layers, const 
  * Same arguments, semantics and device-side errors as kara_compact. Differences:
  *  - Returns KARA_ERR_WORKSPACE, without enqueueing anything, when the plan for num_seqs
  *    sequences and budget k would exceed the fixed array (plan size in bytes:
- *    4 * (16 + 12 * num_seqs + num_seqs * ceil((15 + k) / 16))).
+ *    4 * (144 + 12 * num_seqs + num_seqs * ceil((15 + k) / 16)); at k = 204 that admits up
+ *    to 624 sequences).
  *  - The first call on each device looks up the array's device address (once per device,
- *    with that device current); make that first call before any stream capture.
+ *    with that device current); make that first call before any stream capture. The address
+ *    is kept for the life of the process: after cudaDeviceReset (or any teardown of the
+ *    device's primary context) it is stale, so do not call this entry point again in that
+ *    process after such a reset.
  *  - Every call on a device shares the one array, which keeps the last call's contents:
  *    calls that overlap on the GPU (other streams, or threads sharing a device without
  *    ordering) race on it. Order them on one stream.

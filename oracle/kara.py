@@ -246,8 +246,10 @@ def token2chunk_batch(scores: np.ndarray, sel: np.ndarray, num_anchors: int, gap
 
 
 def anchors_for(anchor_frac: float, k: int) -> int:
-    """Number of anchors for an anchor fraction: ceil(anchor_frac * k), clipped to [0, k]."""
-    n = int(np.ceil(round(anchor_frac * k, 9)))
+    """Number of anchors for an anchor fraction: ceil(anchor_frac * k), clipped to [0, k]. The
+    product is rounded to 6 decimals first, so that a fraction given in single precision (0.2
+    as 0.2000000030) counts as the decimal it stands for."""
+    n = int(np.ceil(np.rint(anchor_frac * k * 1e6) / 1e6))
     return max(0, min(k, n))
 
 
@@ -271,6 +273,9 @@ def compact(k_pools, v_pools, block_table, ctx_len, free_list, free_top: int, se
     at [p0+n_new, p0+n_old); ctx_len becomes n-W+k; once every sequence has popped, the old
     window blocks are pushed (sequence order, page order). If the free list holds fewer blocks
     than the sequences need together, nothing changes and the status is ERR_OUT_OF_BLOCKS.
+    Every keep row must list window positions (0 <= keep < W) in strictly ascending order
+    (the compressed window keeps the order of the tokens it retains); otherwise nothing
+    changes and the status is ERR_INVALID_ARG.
 
     Returns (status, k_pools, v_pools, block_table, ctx_len, free_list, free_top, fresh_ids),
     all new arrays; fresh_ids maps each due sequence to its fresh block ids.
@@ -282,6 +287,11 @@ def compact(k_pools, v_pools, block_table, ctx_len, free_list, free_top: int, se
     fl = free_list.copy()
     top = int(free_top)
     k = keep.shape[-1]
+
+    rows = keep.reshape(-1, k) if keep.size else keep.reshape(0, max(k, 1))
+    for row in rows:
+        if (row < 0).any() or (row >= window).any() or (np.diff(row) <= 0).any():
+            return (ERR_INVALID_ARG, kp, vp, bt, cl, fl, top, {})
 
     plans = []
     need = 0

@@ -33,8 +33,9 @@ def test_host_side_validation_returns_before_any_launch(lib_path):
     assert L.kara_select(null, 4, 16, 17, null, null) == K.ERR_INVALID_ARG
     assert L.kara_select(null, 4, 5000, 8, null, null) == K.ERR_INVALID_ARG
     assert L.kara_select(null, 0, 16, 4, null, null) == K.OK          # empty input
-    # more anchors than kept tokens
-    assert L.kara_token2chunk(null, null, 1, 16, 4, 5, 8, 1, null, null) == K.ERR_INVALID_ARG
+    # anchor fractions outside [0, 1] (and NaN)
+    for frac in (5.0, 1.01, -0.1, float("nan")):
+        assert L.kara_token2chunk(null, null, 1, 16, 4, frac, 8, 1, null, null) == K.ERR_INVALID_ARG
     # page size other than 16, head_dim other than 64/128
     pool = K._Pool(1, 1, 1, 1, 1, 8, 64, 8, 2, 128)
     assert L.paged_decode_attn(null, null, null, ctypes.byref(pool), 4, 1.0, null, null, 0, null,
@@ -74,15 +75,15 @@ def test_host_side_validation_returns_before_any_launch(lib_path):
     assert L.kara_reset_tails(one, one, 0, 4, null) == K.OK             # nothing to reset
     assert L.kara_score_ring(one, one, ctypes.byref(pool), null, 1, 5000, 4, 1.0, one, one,
                              1 << 20, one, null) == K.ERR_INVALID_ARG
-    # fused selection: more anchors than kept, k above the window; fused compression: the same,
-    # and a missing free list
-    assert L.kara_select_chunks(one, 2, 64, 8, 9, 8, 1, null, one, null) == K.ERR_INVALID_ARG
-    assert L.kara_select_chunks(one, 2, 64, 65, 4, 8, 1, null, one, null) == K.ERR_INVALID_ARG
-    assert L.kara_select_chunks(one, 0, 64, 8, 4, 8, 1, null, one, null) == K.OK
-    assert L.kara_compress(one, layers, 1, ctypes.byref(pool), null, 1, 64, 8, 9, 8, 1, null, one,
-                           1 << 20, one, null) == K.ERR_INVALID_ARG
+    # fused selection: an anchor fraction above 1, k above the window; fused compression: the
+    # same, and a missing free list
+    assert L.kara_select_chunks(one, 2, 64, 8, 9.0, 8, 1, null, one, null) == K.ERR_INVALID_ARG
+    assert L.kara_select_chunks(one, 2, 64, 65, 0.5, 8, 1, null, one, null) == K.ERR_INVALID_ARG
+    assert L.kara_select_chunks(one, 0, 64, 8, 0.5, 8, 1, null, one, null) == K.OK
+    assert L.kara_compress(one, layers, 1, ctypes.byref(pool), null, 1, 64, 8, 1.5, 8, 1, null,
+                           one, 1 << 20, one, null) == K.ERR_INVALID_ARG
     nofree = K._Pool(1, 1, 0, 0, 1, 8, 64, 16, 2, 128)
-    assert L.kara_compress(one, layers, 1, ctypes.byref(nofree), null, 1, 64, 8, 4, 8, 1, null,
+    assert L.kara_compress(one, layers, 1, ctypes.byref(nofree), null, 1, 64, 8, 0.5, 8, 1, null,
                            one, 1 << 20, one, null) == K.ERR_INVALID_ARG
     # none of these reached a kernel launch
     assert K.kara_launch_count() == launches
@@ -96,7 +97,7 @@ def test_workspace_sizes(lib_path):
     dec = K.lib().kara_workspace_bytes(K.OP_DECODE, ctypes.byref(pool), 0, 0, 28, 0)
     assert dec == 32 * 28 * 33 * 130 * 4              # 33 units of 8 pages, d + 2 floats
     comp = K.lib().kara_workspace_bytes(K.OP_COMPACT, None, 32, 1024, 0, 204)
-    assert comp == (16 + 32 * 12 + 32 * 14) * 4
+    assert comp == (144 + 32 * 12 + 32 * 14) * 4      # header with the keep check's verdicts
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
@@ -116,6 +117,9 @@ def test_binding_refuses_host_tensors():
     q = torch.zeros((2, w, 4, 64), dtype=torch.bfloat16)
     kv = torch.zeros((4, 16, 2, 64), dtype=torch.bfloat16)
     sel = torch.zeros((2, 2, k), dtype=torch.int32)
+    ring = torch.zeros((2, 2 * w, 4, 64), dtype=torch.bfloat16)
+    seq = torch.zeros(2, dtype=torch.int32)
+    status = torch.zeros(1, dtype=torch.int32)
     pool = K.PagedPool(torch.zeros((2, 4), dtype=torch.int32), torch.zeros(2, dtype=torch.int32),
                        torch.zeros(4, dtype=torch.int32), torch.zeros(1, dtype=torch.int32), 4, 2,
                        64)
@@ -123,14 +127,23 @@ def test_binding_refuses_host_tensors():
         "kara_score": lambda: K.kara_score(q, kv, pool, w),
         "kara_score_ex": lambda: K.kara_score_ex(q, kv, pool, w),
         "kara_select": lambda: K.kara_select(s, k),
-        "kara_token2chunk": lambda: K.kara_token2chunk(s, sel, 4, 8, 1),
-        "kara_select_chunks": lambda: K.kara_select_chunks(s, k, 4, 8, 1),
+        "kara_token2chunk": lambda: K.kara_token2chunk(s, sel, 0.5, 8, 1),
+        "kara_select_chunks": lambda: K.kara_select_chunks(s, k, 0.5, 8, 1),
         "kara_sum_heads": lambda: K.kara_sum_heads(s),
         "kara_expand_keep": lambda: K.kara_expand_keep(sel[:, 0].contiguous(), 2),
         "kara_compact": lambda: K.kara_compact([kv], [kv], pool, w, sel[None]),
-        "kara_compress": lambda: K.kara_compress(s[None], [kv], [kv], pool, w, k, 4, 8, 1),
+        "kara_compress": lambda: K.kara_compress(s[None], [kv], [kv], pool, w, k, 0.5, 8, 1),
+        "kara_compact_noalloc": lambda: K.kara_compact_noalloc([kv], [kv], pool, w, sel[None],
+                                                               status=status),
+        "lacache_compact": lambda: K.lacache_compact([kv], [kv], pool, 1, 0, 16, 64),
         "paged_decode_attn": lambda: K.paged_decode_attn(q[:, 0], kv, kv, pool),
         "kara_decode_append": lambda: K.kara_decode_append(q[:, 0], kv[0], kv[0], kv, kv, pool),
+        "kara_score_ring": lambda: K.kara_score_ring(ring, kv, pool, w, seq, 2),
+        "kara_step_begin": lambda: K.kara_step_begin(pool, status),
+        "kara_step_end": lambda: K.kara_step_end(pool, seq, w, True, seq, seq[:1]),
+        "kara_reset_tails": lambda: K.kara_reset_tails(seq, seq, 2),
+        # a host status word or workspace is refused as well (its address is no device address)
+        "kara_wait_probe": lambda: K.kara_wait_probe(100, status=status),
     }
     for name, fn in calls.items():
         with pytest.raises(ValueError, match="CUDA tensor"):

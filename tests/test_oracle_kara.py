@@ -278,6 +278,11 @@ def test_anchor_count():
     assert ok.anchors_for(0.0, 32) == 0
     assert ok.anchors_for(1.0, 32) == 32
     assert ok.anchors_for(0.1, 30) == 3
+    assert ok.anchors_for(0.5, 61) == 31                      # ceil(30.5)
+    # a fraction that arrives in single precision counts as its decimal: 0.2 as 0.2000000030
+    # gives ceil(0.2 * 5) = 1, not 2 (the product is rounded to 6 decimals before the ceiling)
+    assert ok.anchors_for(float(np.float32(0.2)), 5) == 1
+    assert ok.anchors_for(float(np.float32(0.2)), 61) == 13
 
 
 # ------------------------------------------------------------------ compaction
@@ -374,6 +379,33 @@ def test_compact_out_of_blocks_changes_nothing():
     st, kp, vp, bt, cl, fl, top, _ = ok.compact(ks, vs, table, ctx, free, 0, [0], 12, keep, page)
     assert st == ok.ERR_OUT_OF_BLOCKS
     assert (bt == table).all() and (cl == ctx).all() and top == 0
+
+
+@pytest.mark.parametrize("bad", ["below", "past_window", "repeat", "descending"])
+def test_compact_bad_keep_changes_nothing(bad):
+    page = 4
+    ks, vs = small_pool(5, page=page, nb=10, hkv=2, d=2, layers=2)
+    table = np.array([[0, 1, 2, 3, -1]], dtype=np.int32)
+    ctx = np.array([16], dtype=np.int32)
+    free = np.array([4, 5, 6, 7, 8, 9, 0, 0, 0, 0], dtype=np.int32)
+    keep = np.tile(np.arange(0, 12, 2, dtype=np.int32), (2, 1, 2, 1))   # W = 12, k = 6
+    st, *_ = ok.compact(ks, vs, table, ctx, free, 6, [0], 12, keep, page)
+    assert st == ok.OK
+    keep = keep.copy()
+    if bad == "below":
+        keep[1, 0, 1, 0] = -1
+    elif bad == "past_window":
+        keep[0, 0, 1, 5] = 12
+    elif bad == "repeat":
+        keep[1, 0, 0, 3] = keep[1, 0, 0, 2]
+    else:
+        keep[0, 0, 0, 2], keep[0, 0, 0, 3] = keep[0, 0, 0, 3], keep[0, 0, 0, 2]
+    st, kp, vp, bt, cl, fl, top, fresh = ok.compact(ks, vs, table, ctx, free, 6, [0], 12, keep,
+                                                    page)
+    assert st == ok.ERR_INVALID_ARG and fresh == {}
+    assert (bt == table).all() and (cl == ctx).all() and top == 6 and (fl == free).all()
+    for layer in range(2):
+        assert (kp[layer] == ks[layer]).all() and (vp[layer] == vs[layer]).all()
 
 
 # ---- aggregation variants and the shared selection (variants the pages leave open) ----

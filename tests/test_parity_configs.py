@@ -45,7 +45,7 @@ def test_config_path_sampled(name):
     fl0, top0 = H.i32(cache["free_list"]), int(cache["free_top"][0])
     qw = [q.cpu() for q in cache["q_win"]]
     pool = K.PagedPool.from_cache(cache)
-    na = K.anchors_for(wl.anchor_frac, wl.keep)
+    na = wl.anchor_frac
     status = K.new_status()
     keep = torch.empty((wl.layers, wl.batch, wl.hkv, wl.keep), dtype=torch.int32, device="cuda")
     scores, sels = [], []
@@ -74,8 +74,9 @@ def test_config_path_sampled(name):
             q = qw[layer][r][:, heads].double().numpy()
             H.assert_scores_close(s[r, g], ok.window_scores(q, kw, scale)[0])
             assert np.array_equal(sl[r, g], ok.select_topk(s[r, g], wl.keep))
-            assert np.array_equal(kp[r, g], ok.token2chunk(s[r, g], sl[r, g], na, wl.gap_limit,
-                                                           wl.widen))
+            assert np.array_equal(kp[r, g], ok.token2chunk(s[r, g], sl[r, g],
+                                                           ok.anchors_for(na, wl.keep),
+                                                           wl.gap_limit, wl.widen))
 
     # compaction of all layers, bit-exact
     ws = torch.empty(K.kara_workspace_bytes(K.OP_COMPACT, pool, wl.batch, wl.window, 0, wl.keep),

@@ -55,7 +55,7 @@ def test_decode_loop_matches_oracle(name):
     seed = 21
     W, L, page = wl.window, wl.layers, wl.page
     scale = 1 / math.sqrt(wl.head_dim)
-    na = K.anchors_for(wl.anchor_frac, wl.keep)
+    na = wl.anchor_frac
     cpu = synth.make_cache(wl, seed, "cpu", with_queries=False, extra_pages=steps // page + 2)
     dev = H.to_device(cpu)
     pool = K.PagedPool.from_cache(dev)
@@ -132,8 +132,9 @@ def test_decode_loop_matches_oracle(name):
                 for g in range(wl.hkv):
                     sel = ok.select_topk(s_gpu[r, g], wl.keep)
                     assert np.array_equal(kk[layer, r, g],
-                                          ok.token2chunk(s_gpu[r, g], sel, na, wl.gap_limit,
-                                                         wl.widen))
+                                          ok.token2chunk(s_gpu[r, g], sel,
+                                                         ok.anchors_for(na, wl.keep),
+                                                         wl.gap_limit, wl.widen))
         st, kp, vp, bt, cl, fl, top, _ = ok.compact(kp, vp, bt, cl, fl, top, odue, W, kk, page)
         assert st == ok.OK
         otail = dl.reset_tails(otail, odue)

@@ -141,14 +141,15 @@ def test_select_and_token2chunk(name):
     pool = K.PagedPool.from_cache(dev)
     scores = K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window)
     sel = K.kara_select(scores, wl.keep)
-    na = K.anchors_for(wl.anchor_frac, wl.keep)
+    na = wl.anchor_frac
     keep = K.kara_token2chunk(scores, sel, na, wl.gap_limit, wl.widen)
     torch.cuda.synchronize()
     s_gpu = H.f64(scores)
     # identical inputs -> identical outputs
     assert np.array_equal(H.i32(sel), ok.select_batch(s_gpu, wl.keep))
-    assert np.array_equal(H.i32(keep), ok.token2chunk_batch(s_gpu, H.i32(sel), na, wl.gap_limit,
-                                                            wl.widen))
+    assert np.array_equal(H.i32(keep), ok.token2chunk_batch(s_gpu, H.i32(sel),
+                                                            ok.anchors_for(na, wl.keep),
+                                                            wl.gap_limit, wl.widen))
     # against the oracle's own scores: equal up to near-ties
     ref = oracle_scores(cpu, wl)
     H.assert_selection_matches(H.i32(sel), ok.select_batch(ref, wl.keep), ref)
@@ -164,14 +165,36 @@ def test_select_ties_and_token2chunk_params(seed):
     s[0, :8] = -0.0
     scores = torch.from_numpy(s).cuda()
     sel = K.kara_select(scores, k)
-    na = int(rng.integers(0, k + 1))
+    # an anchor fraction in single precision, as the C ABI takes it; the oracle gets the same
+    # value (ceil of the product rounded to 6 decimals on both sides)
+    frac = float(np.float32(rng.choice([0.0, 0.1, 0.2, 0.25, 0.5, 0.75, 1.0, rng.random()])))
     gap = int(rng.integers(0, 12))
     wid = int(rng.integers(0, 4))
-    keep = K.kara_token2chunk(scores, sel, na, gap, wid)
+    keep = K.kara_token2chunk(scores, sel, frac, gap, wid)
     torch.cuda.synchronize()
     assert np.array_equal(H.i32(sel), ok.select_batch(s.astype(np.float64), k))
-    assert np.array_equal(H.i32(keep), ok.token2chunk_batch(s.astype(np.float64), H.i32(sel), na,
-                                                            gap, wid))
+    assert np.array_equal(H.i32(keep), ok.token2chunk_batch(s.astype(np.float64), H.i32(sel),
+                                                            ok.anchors_for(frac, k), gap, wid))
+
+
+@pytest.mark.parametrize("frac,k,count", [(0.0, 61, 0), (0.5, 61, 31), (1.0, 61, 61),
+                                          (0.2, 61, 13), (0.2, 5, 1)])
+def test_anchor_fraction_through_the_c_abi(frac, k, count):
+    # the C ABI takes anchor_frac and counts ceil(frac * k) anchors itself (0.2 arrives as the
+    # float 0.2000000030, still one anchor of five)
+    assert ok.anchors_for(frac, k) == count
+    rng = np.random.default_rng(11)
+    s = rng.random((4, 300)).astype(np.float32)
+    scores = torch.from_numpy(s).cuda()
+    sel = K.kara_select(scores, k)
+    keep = K.kara_token2chunk(scores, sel, frac, 8, 1)
+    keep2 = K.kara_select_chunks(scores, k, frac, 8, 1)
+    torch.cuda.synchronize()
+    assert torch.equal(keep, keep2)
+    s64 = s.astype(np.float64)
+    for r in range(4):
+        ref = ok.token2chunk(s64[r], ok.select_topk(s64[r], k), count, 8, 1)
+        assert np.array_equal(H.i32(keep[r]), ref)
 
 
 def test_select_max_window_and_k_equals_w():
@@ -184,8 +207,8 @@ def test_select_max_window_and_k_equals_w():
         assert np.array_equal(H.i32(sel), ok.select_batch(s.astype(np.float64), k))
     # Token2Chunk at the largest window (58 KB of shared memory), separately and fused
     sel = K.kara_select(scores, 819)
-    keep = K.kara_token2chunk(scores, sel, 410, 8, 1)
-    keep2 = K.kara_select_chunks(scores, 819, 410, 8, 1)
+    keep = K.kara_token2chunk(scores, sel, 0.5, 8, 1)          # ceil(0.5 * 819) = 410 anchors
+    keep2 = K.kara_select_chunks(scores, 819, 0.5, 8, 1)
     torch.cuda.synchronize()
     assert torch.equal(keep, keep2)
     s64 = s.astype(np.float64)
@@ -269,6 +292,35 @@ def test_compact_out_of_blocks_changes_nothing():
     assert torch.equal(dev["k"][0], kb)
 
 
+@pytest.mark.parametrize("bad", ["past_window", "negative", "out_of_order"])
+def test_compact_bad_keep_changes_nothing(bad):
+    # one bad entry in the last layer's last row: the whole call is refused before anything
+    # moves (the check runs before the plan pops or frees a block)
+    wl = SCORE_CASES["g7_ragged_unaligned"]
+    cpu, dev = H.make(wl, 5, layers=2)
+    rng = np.random.default_rng(3)
+    keep = np.stack([synth.random_keep(rng, wl.batch * wl.hkv, wl.window, wl.keep)
+                     .reshape(wl.batch, wl.hkv, wl.keep) for _ in range(2)])
+    if bad == "past_window":
+        keep[1, -1, -1, -1] = wl.window
+    elif bad == "negative":
+        keep[1, -1, -1, 0] = -1
+    else:
+        keep[1, -1, -1, [3, 4]] = keep[1, -1, -1, [4, 3]]
+    st_ref = oracle_compact(cpu, wl, keep, list(range(wl.batch)), 2)[0]
+    assert st_ref == ok.ERR_INVALID_ARG
+    before = {k: dev[k].clone() for k in ("block_table", "ctx_len", "free_list", "free_top")}
+    pools = [t.clone() for t in dev["k"] + dev["v"]]
+    pool = K.PagedPool.from_cache(dev)
+    status = K.kara_compact(dev["k"], dev["v"], pool, wl.window, torch.from_numpy(keep).cuda())
+    torch.cuda.synchronize()
+    assert K.read_status(status) == K.ERR_INVALID_ARG
+    for k, t in before.items():
+        assert torch.equal(dev[k], t), k
+    for t, t0 in zip(dev["k"] + dev["v"], pools):
+        assert torch.equal(t, t0)
+
+
 def test_compact_bad_block_id_is_reported_not_faulted():
     wl = SCORE_CASES["g7_ragged_unaligned"]
     cpu, dev = H.make(wl, 4)
@@ -338,7 +390,7 @@ def test_select_chunks_equals_select_then_token2chunk(name):
     cpu, dev = H.make(wl, 12)
     pool = K.PagedPool.from_cache(dev)
     sc = K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window)
-    na = K.anchors_for(wl.anchor_frac, wl.keep)
+    na = wl.anchor_frac
     sel = K.kara_select(sc, wl.keep)
     keep = K.kara_token2chunk(sc, sel, na, wl.gap_limit, wl.widen)
     sel2 = torch.empty_like(sel)
@@ -349,8 +401,8 @@ def test_select_chunks_equals_select_then_token2chunk(name):
     s = H.f64(sc)
     for r in range(wl.batch):
         for g in range(wl.hkv):
-            ref = ok.token2chunk(s[r, g], ok.select_topk(s[r, g], wl.keep), na, wl.gap_limit,
-                                 wl.widen)
+            ref = ok.token2chunk(s[r, g], ok.select_topk(s[r, g], wl.keep),
+                                 ok.anchors_for(na, wl.keep), wl.gap_limit, wl.widen)
             assert np.array_equal(H.i32(keep2[r, g]), ref)
 
 
@@ -367,7 +419,7 @@ def test_compress_equals_select_chunks_then_compact(name, layers, subset):
     ids = [1, 3] if subset else list(range(wl.batch))
     assert wl.batch > max(ids)
     seq = torch.tensor(ids, dtype=torch.int32, device="cuda")
-    na = K.anchors_for(wl.anchor_frac, wl.keep)
+    na = wl.anchor_frac
     pool_a, pool_b = K.PagedPool.from_cache(dev_a), K.PagedPool.from_cache(dev_b)
     scores = torch.stack([K.kara_score(dev_a["q_win"][l][ids].contiguous(), dev_a["k"][l], pool_a,
                                        wl.window, seq_ids=seq) for l in range(layers)])
@@ -406,7 +458,7 @@ def test_compress_out_of_blocks_changes_nothing():
     before = {k2: dev[k2].clone() for k2 in ("block_table", "ctx_len", "free_top")}
     kb = H.bits(dev["k"][0]).copy()
     scores = K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window)[None]
-    na = K.anchors_for(wl.anchor_frac, wl.keep)
+    na = wl.anchor_frac
     st = K.kara_compress(scores, dev["k"], dev["v"], pool, wl.window, wl.keep, na, wl.gap_limit,
                          wl.widen)
     torch.cuda.synchronize()

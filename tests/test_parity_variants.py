@@ -78,7 +78,7 @@ def test_shared_selection_across_kv_heads():
     wl = LAYER.with_(batch=3, ctx_lo=600, ctx_hi=900, window=256, keep=52, layers=2)
     cpu, dev = H.make(wl, 10)
     pool = K.PagedPool.from_cache(dev)
-    na = K.anchors_for(wl.anchor_frac, wl.keep)
+    na = wl.anchor_frac
     status = K.new_status()
     keep = torch.empty((wl.layers, wl.batch, wl.hkv, wl.keep), dtype=torch.int32, device="cuda")
     sums, shared = [], []
@@ -101,7 +101,8 @@ def test_shared_selection_across_kv_heads():
         for r in range(wl.batch):
             # selection and Token2Chunk of the oracle on the same (fp32) head sums
             tot = sums[layer][1][r].double().cpu().numpy()
-            own = ok.token2chunk(tot, ok.select_topk(tot, wl.keep), na, wl.gap_limit, wl.widen)
+            own = ok.token2chunk(tot, ok.select_topk(tot, wl.keep), ok.anchors_for(na, wl.keep),
+                                 wl.gap_limit, wl.widen)
             assert np.array_equal(H.i32(shared[layer][r]), own)
             assert all(np.array_equal(H.i32(keep[layer, r, g]), own) for g in range(wl.hkv))
     # compaction with the shared keep sets, bit-exact against the oracle

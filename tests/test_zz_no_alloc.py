@@ -77,6 +77,6 @@ def test_noalloc_rejects_plans_larger_than_its_array():
     null = ctypes.c_void_p(0)
     arr = K._layers(dev["k"], dev["v"])
     ps = pool.c_struct()
-    # 4 * (16 + 12 R + R * ceil((15 + k) / 16)) > 64 KiB for R = 4096, k = 204
+    # 4 * (144 + 12 R + R * ceil((15 + k) / 16)) > 64 KiB for R = 4096, k = 204
     rc = limit(arr, 1, ctypes.byref(ps), null, 4096, 1024, 204, null, null, null)
     assert rc == K.ERR_WORKSPACE
