@@ -1,11 +1,21 @@
 """Throughput benchmark of the Kara decode-time compression step on B200.
 
-One step = one pass of the whole hot path over one batch of the "layer" workload (one
-7B-class layer, batch 32, 28 query / 4 KV heads, d = 128, 4096-token paged caches, window
-1024, keep 204): kara_score -> kara_select_chunks (select and Token2Chunk in one kernel) ->
-kara_compact -> paged_decode_attn over the compressed cache, then the block table, lengths and free list are
-restored so that every step sees the same input. Metric: compressed KV tokens per second
-(window tokens of all due sequences / step time), whole job over all ranks.
+One step = one pass of the whole hot path over the "step" workload: a 28-layer 7B-class model
+(28 query / 4 KV heads, d = 128) with a batch of 128 sequences whose paged caches hold ragged
+contexts of 2K-16K tokens (page 16, so windows start at unaligned slots), every sequence due
+(the worst-case check step of the 100-step schedule), window W = 1024, keep 204 (20 %),
+Token2Chunk anchors 50 % / gap 8 / widen 1:
+
+    kara_score per layer -> kara_select_chunks per layer -> one kara_compact over all layers
+    -> paged_decode_attn per layer over the compressed cache
+
+then the block table, lengths and free list are restored, so that every step sees the same
+input (compaction writes only fresh blocks, so the old rows are still in place). Metric:
+compressed KV tokens per second (window tokens of all due sequences / step time), whole job
+over all ranks. Beside it, in `kernels`: the amortised cost under the 100-step schedule
+(the decode loop with the tail-W trigger on the same shapes), the one-layer workload
+(batch 32, 4096-token caches), the LaCache workload's three iterative ladder passes and the
+score / selection variants.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -35,12 +45,27 @@ from decode_kv_cache_kara_b200 import synth  # noqa: E402
 
 METRIC = "compressed KV tokens/sec on 1 B200; % tensor/HBM roofline per kernel"
 UNIT = "tokens/s"
-WORKLOAD = synth.WORKLOADS["layer"]
-WORKLOAD_DESC = ("layer: one 7B-class layer, batch 32, 28 query / 4 KV heads, head_dim 128, "
-                 "4096-token paged caches (page 16), window W=1024 (last 1024 tokens), keep 204 "
-                 "(20%), Token2Chunk anchors 50% / gap 8 / widen 1, then paged GQA decode over "
-                 "the compressed cache")
+WORKLOAD = synth.WORKLOADS["step"]
+WORKLOAD_INDEX = 2            # its position among the five workloads (seed 1234 + index)
+LAYER_WORKLOAD = synth.WORKLOADS["layer"]
+WORKLOAD_DESC = ("step: 28-layer 7B-class model (28 query / 4 KV heads, head_dim 128), batch "
+                 "128, ragged contexts uniform in [2048, 16384] tokens in 16-token pages, "
+                 "window W=1024 (the last 1024 tokens), keep 204 (20%), Token2Chunk anchors 50% "
+                 "/ gap 8 / widen 1, every sequence due (the worst-case check step of the "
+                 "100-step schedule); score and select per layer, one compaction of all 28 "
+                 "layers, then paged GQA decode of every layer over the compressed cache")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def bench_config(wl: synth.Workload, world: int) -> dict:
+    """The `config` of both arms' JSON lines (the same workload, so the same dict)."""
+    return {"workload": WORKLOAD_DESC, "batch_per_gpu": wl.batch, "layers": wl.layers,
+            "q_heads": wl.hq, "kv_heads": wl.hkv, "head_dim": wl.head_dim,
+            "context": [wl.ctx_lo, wl.ctx_hi], "window": wl.window, "keep": wl.keep,
+            "page": wl.page, "anchor_frac": wl.anchor_frac, "gap_limit": wl.gap_limit,
+            "widen": wl.widen, "due_per_step": wl.batch,
+            "parallelism": f"dp{world} (independent sequences per rank)",
+            "l2": "inputs larger than L2 (window queries 26.3 GB, KV pools about 70 GB per GPU)"}
 
 
 def captured_traffic(op: str):
@@ -62,10 +87,10 @@ def captured_traffic(op: str):
     return None
 
 
-def rank_seed(rank: int) -> int:
-    """Seed of a rank's batch: the layer workload's seed (1234 + config index 1), offset per
-    rank so that every rank compresses its own, independent sequences."""
-    return 1234 + 1 + 1000 * rank
+def rank_seed(rank: int, index: int = WORKLOAD_INDEX) -> int:
+    """Seed of a rank's batch: the workload's seed (1234 + its index), offset per rank so that
+    every rank compresses its own, independent sequences."""
+    return 1234 + index + 1000 * rank
 
 
 def max_over_ranks(x: float, device, world: int) -> float:
@@ -91,6 +116,14 @@ def load_peaks():
         return p, "measured"
     except Exception:
         return FALLBACK_PEAKS, "fallback"
+
+
+def host_cores() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
 
 
 # ------------------------------------------------------------------------------------------
@@ -152,8 +185,24 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------
 # GPU arm
 # ------------------------------------------------------------------------------------------
+def decode_queries(cache: dict) -> list:
+    """One decode query [B, Hq, d] per layer: the cache's own for layer 0, seeded N(0, 1) draws
+    for the others."""
+    q0 = cache["q_dec"]
+    gen = torch.Generator(device=q0.device)
+    gen.manual_seed(cache["seed"] + 77)
+    out = [q0]
+    for _ in range(1, len(cache["k"])):
+        out.append(torch.randn(q0.shape, generator=gen, device=q0.device).to(q0.dtype))
+    return out
+
+
 class Step:
-    """One compression step of the whole path on a device-resident workload."""
+    """One compression step of the whole path, over every layer of a device-resident cache:
+    scores of every layer, selection + Token2Chunk of every layer, one compaction of all
+    layers, decode of every layer over the compressed cache."""
+
+    OPS = ("kara_score", "select+token2chunk", "kara_compact", "paged_decode_attn")
 
     def __init__(self, cache: dict, wl: synth.Workload):
         from decode_kv_cache_kara_b200 import kara as K
@@ -161,6 +210,8 @@ class Step:
         self.wl = wl
         self.c = cache
         dev = cache["k"][0].device
+        L = len(cache["k"])
+        self.L = L
         # the pool bookkeeping as views into one int32 buffer, so that the per-step restore
         # is a single copy
         names = ("block_table", "ctx_len", "free_list", "free_top")
@@ -176,18 +227,19 @@ class Step:
         self.pool = K.PagedPool.from_cache(cache)
         self.status = K.new_status(dev)
         r, hq = wl.batch, wl.hq
-        self.scores = torch.empty((r, wl.hkv, wl.window), dtype=torch.float32, device=dev)
-        self.sel = torch.empty((r, wl.hkv, wl.keep), dtype=torch.int32, device=dev)
-        self.keep = torch.empty((1, r, wl.hkv, wl.keep), dtype=torch.int32, device=dev)
-        self.out = torch.empty((wl.batch, hq, wl.head_dim), dtype=torch.bfloat16, device=dev)
+        self.q_dec = decode_queries(cache)
+        self.scores = torch.empty((L, r, wl.hkv, wl.window), dtype=torch.float32, device=dev)
+        self.sel = torch.empty((L, r, wl.hkv, wl.keep), dtype=torch.int32, device=dev)
+        self.keep = torch.empty((L, r, wl.hkv, wl.keep), dtype=torch.int32, device=dev)
+        self.out = torch.empty((L, wl.batch, hq, wl.head_dim), dtype=torch.bfloat16, device=dev)
         ws = max(K.kara_workspace_bytes(K.OP_SCORE, self.pool, r, wl.window, hq),
                  K.kara_workspace_bytes(K.OP_COMPACT, self.pool, r, wl.window, 0, wl.keep),
                  K.kara_workspace_bytes(K.OP_DECODE, self.pool, 0, 0, hq, 0))
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
-        self.na = wl.anchor_frac
         # scoring: the fused cluster kernel for windows of 128/256/512/1024 keys (plus the
         # split-item sum when a cluster range ends inside an item), else two passes and a
-        # merge; select + Token2Chunk in one kernel; compaction plan + gather; decode + combine
+        # merge; select + Token2Chunk in one kernel; compaction check + plan + gather; decode
+        # stream + combine
         self.score_fused = wl.window in (128, 256, 512, 1024)
 
     def restore(self):
@@ -197,40 +249,123 @@ class Step:
         K, wl, c = self.K, self.wl, self.c
         rec = (lambda i: events[i].record()) if events is not None else (lambda i: None)
         rec(0)
-        K.kara_score(c["q_win"][0], c["k"][0], self.pool, wl.window, scores=self.scores,
-                     workspace=self.ws, status=self.status)
+        for layer in range(self.L):
+            K.kara_score(c["q_win"][layer], c["k"][layer], self.pool, wl.window,
+                         scores=self.scores[layer], workspace=self.ws, status=self.status)
         rec(1)
-        K.kara_select_chunks(self.scores, wl.keep, self.na, wl.gap_limit, wl.widen,
-                             keep=self.keep[0], sel=self.sel)
+        for layer in range(self.L):
+            K.kara_select_chunks(self.scores[layer], wl.keep, wl.anchor_frac, wl.gap_limit,
+                                 wl.widen, keep=self.keep[layer], sel=self.sel[layer])
         rec(2)
         K.kara_compact(c["k"], c["v"], self.pool, wl.window, self.keep, workspace=self.ws,
                        status=self.status)
         rec(3)
-        K.paged_decode_attn(c["q_dec"], c["k"][0], c["v"][0], self.pool, out=self.out,
-                            workspace=self.ws, status=self.status)
+        for layer in range(self.L):
+            K.paged_decode_attn(self.q_dec[layer], c["k"][layer], c["v"][layer], self.pool,
+                                out=self.out[layer], workspace=self.ws, status=self.status)
         rec(4)
         if restore:
             self.restore()
 
 
 def algorithmic_work(wl: synth.Workload, cache: dict) -> dict:
-    """Per-launch algorithmic flops / bytes of each op (inputs before the step)."""
+    """Algorithmic flops / bytes of each op over one step (all layers; inputs before the
+    step). Scoring: one Q K^T per (sequence, layer). Compaction: the K and V head-rows moved
+    (the prefix rows of the first window page and the k kept rows per KV head), read and
+    written. Decode: the K and V rows of the compressed contexts, plus q and out."""
+    L = len(cache["k"])
     ctx = cache["ctx_len"].cpu().numpy().astype(np.int64)
     r, W, d, hq, hkv, k = wl.batch, wl.window, wl.head_dim, wl.hq, wl.hkv, wl.keep
-    score_flops = 2.0 * W * W * d * hq * r                       # one Q K^T, useful
+    score_flops = 2.0 * W * W * d * hq * r * L
     off = (ctx - W) % wl.page
-    rows = (hkv * (k + off)).sum()                               # head-rows copied
-    compact_bytes = float(rows * d * 2 * 2 * 2)                  # K and V, read + write
+    rows = (hkv * (k + off)).sum()                               # head-rows per layer
+    compact_bytes = float(rows * d * 2 * 2 * 2 * L)              # K and V, read + write
     n_after = ctx - W + k
-    decode_bytes = float(n_after.sum() * hkv * d * 2 * 2 + 2 * r * hq * d * 2)
+    decode_bytes = float((n_after.sum() * hkv * d * 2 * 2 + 2 * r * hq * d * 2) * L)
     return {"score_flops": score_flops, "compact_bytes": compact_bytes,
             "decode_bytes": decode_bytes}
 
 
-def time_cpu_oracle_sample(cache_cpu: dict, wl: synth.Workload, units: int = 1, seed: int = 0):
-    """The oracle as it stands on one (sequence, KV head) unit per call: score (its G query
-    heads), select, Token2Chunk, compaction of its rows, decode of its G query heads.
-    Returns (seconds, window tokens equivalent)."""
+def time_step(step: Step, steps: int, warmup: int, world: int = 1, sampler=None):
+    """Warm-up, then `steps` timed steps between a barrier and a synchronize on both sides.
+    Returns (total ms, per-op average ms, launches in the timed region, clocks)."""
+    K = step.K
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    if K.read_status(step.status) != 0:
+        raise RuntimeError(f"device status after warm-up: {K.status_str(K.read_status(step.status))}")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if sampler is not None:
+        sampler.start()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = K.kara_launch_count()
+    t0.record()
+    for i in range(steps):
+        step.run(ev[i])
+    t1.record()
+    launches = K.kara_launch_count() - launches0
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    clocks = sampler.stop() if sampler is not None else None
+    if K.read_status(step.status) != 0:
+        raise RuntimeError(f"device status: {K.status_str(K.read_status(step.status))}")
+    avg = {}
+    for j, name in enumerate(Step.OPS):
+        avg[name] = sum(e[j].elapsed_time(e[j + 1]) for e in ev) / steps
+    return t0.elapsed_time(t1), avg, launches, clocks
+
+
+def kernel_entries(wl: synth.Workload, work: dict, avg: dict, step: Step, peaks: dict,
+                   src: str) -> dict:
+    """Per-op times of a step and their fractions of the measured peaks."""
+    L = step.L
+    n_exp = wl.window * wl.window * wl.hq * wl.batch * L
+    sfu_floor_ms = n_exp / (16 * 148 * 1.965e9) * 1e3
+    if step.score_fused:
+        score_exec, score_note = 1.25, ("fused single-exponential kernel: S over 144 key rows "
+                                        "per 128 owned keys (x1.125) plus the P'^T W column-sum "
+                                        "product (N = 16, x0.125): executed = 1.25 x useful")
+    else:
+        score_exec, score_note = 2.0, ("two UMMA passes (row log-sum-exp, then column sums): "
+                                       "executed flops are twice the useful Q K^T")
+    ms_score = avg["kara_score"]
+    kernels = {
+        "kara_score": {"ms": ms_score, "bound": "tensor", "launches_of_op": L,
+                       "useful_tflops": work["score_flops"] / ms_score / 1e9,
+                       "executed_tflops": score_exec * work["score_flops"] / ms_score / 1e9,
+                       "note": score_note, "exp2_count": n_exp, "sfu_floor_ms": sfu_floor_ms,
+                       "frac_of_sfu_floor": sfu_floor_ms / ms_score},
+        "select+token2chunk": {"ms": avg["select+token2chunk"], "bound": "latency",
+                               "launches_of_op": L},
+        "kara_compact": {"ms": avg["kara_compact"], "bound": "hbm", "launches_of_op": 1,
+                         "gbs": work["compact_bytes"] / avg["kara_compact"] / 1e6,
+                         "bytes": work["compact_bytes"]},
+        "paged_decode_attn": {"ms": avg["paged_decode_attn"], "bound": "hbm", "launches_of_op": L,
+                              "gbs": work["decode_bytes"] / avg["paged_decode_attn"] / 1e6,
+                              "bytes": work["decode_bytes"]},
+    }
+    for v in kernels.values():
+        if v["bound"] == "hbm":
+            v["frac_of_hbm_" + src] = v["gbs"] / peaks["hbm_gbs"]
+        elif v["bound"] == "tensor":
+            v["frac_of_bf16_" + src] = v["useful_tflops"] / peaks["bf16_tflops"]
+    return kernels
+
+
+def time_cpu_oracle_sample(cache_cpu: dict, wl: synth.Workload, units: int = 1, seed: int = 0,
+                           layers_per_step: int = 1):
+    """The oracle as it stands on `units` (sequence, KV head) units of one layer of a CPU
+    cache: score (the unit's G query heads), select, Token2Chunk, compaction of its rows,
+    decode of its G query heads over the compressed sequence. Returns (seconds, tokens):
+    a unit is W / (Hkv * layers_per_step) window tokens of a step that compresses
+    `layers_per_step` layers."""
     from oracle import decode as od
     from oracle import kara as ok
     rng = np.random.default_rng(seed)
@@ -269,49 +404,49 @@ def time_cpu_oracle_sample(cache_cpu: dict, wl: synth.Workload, units: int = 1, 
         # the compacted sequence as one block of nn slots
         od.decode_attention(q, kk[None], vv[None], np.array([[0]]), np.array([nn]), scale, nn)
     dt = time.perf_counter() - t0
-    return dt, units * wl.window / wl.hkv
+    return dt, units * wl.window / (wl.hkv * layers_per_step)
 
 
-def e2e_run(cache: dict, wl: synth.Workload, steps: int, warmup: int) -> dict:
-    """The same step through the public API with HOST inputs: every step copies the inputs from
-    pinned host memory to the device and reads the results back."""
-    from decode_kv_cache_kara_b200 import kara as K
-    dev = cache["k"][0].device
-    names_in = ["q_win", "k", "v", "q_dec", "block_table", "ctx_len", "free_list", "free_top"]
-    host = {}
-    for n in names_in:
-        val = cache[n]
-        host[n] = ([t.cpu().pin_memory() for t in val] if isinstance(val, list)
-                   else val.cpu().pin_memory())
-    dcache = {n: ([torch.empty_like(t, device=dev) for t in host[n]] if isinstance(host[n], list)
-                  else torch.empty_like(host[n], device=dev)) for n in names_in}
-    dcache["num_blocks"] = cache["num_blocks"]
-    out_host = {"out": torch.empty((wl.batch, wl.hq, wl.head_dim), dtype=torch.bfloat16).pin_memory(),
-                "keep": torch.empty((1, wl.batch, wl.hkv, wl.keep), dtype=torch.int32).pin_memory(),
-                "block_table": torch.empty_like(host["block_table"]).pin_memory(),
-                "ctx_len": torch.empty_like(host["ctx_len"]).pin_memory()}
+def oracle_sample_cache(seed: int) -> dict:
+    """A CPU cache with the step workload's shapes and value recipe (four sequences, one
+    layer), for timing the oracle on units of the same workload."""
+    return synth.make_cache(WORKLOAD.with_(batch=4, layers=1), seed, "cpu")
 
-    def h2d():
-        for n in names_in:
-            if isinstance(host[n], list):
-                for d_, h_ in zip(dcache[n], host[n]):
-                    d_.copy_(h_, non_blocking=True)
-            else:
-                dcache[n].copy_(host[n], non_blocking=True)
 
-    h2d_bytes = sum(t.numel() * t.element_size() for n in names_in
-                    for t in (host[n] if isinstance(host[n], list) else [host[n]]))
+def e2e_run(step: Step, steps: int, warmup: int) -> dict:
+    """The same step through the public API with HOST inputs: every step copies the window
+    queries of every layer, the decode queries and the pool bookkeeping from pinned host
+    memory into the step's device buffers, runs the step and reads back every layer's decode
+    output, the keep sets, the block table and the lengths. The KV pools are the serving
+    engine's device-resident cache (state kept across steps, not an input of one step)."""
+    c = step.c
+
+    def pinned_copy(t):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    host_q = [pinned_copy(t) for t in c["q_win"]]
+    host_qd = [pinned_copy(t) for t in step.q_dec]
+    host_book = pinned_copy(step.saved_book)
+    out_host = {"out": torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory(),
+                "keep": torch.empty(step.keep.shape, dtype=torch.int32).pin_memory(),
+                "block_table": torch.empty(c["block_table"].shape, dtype=torch.int32).pin_memory(),
+                "ctx_len": torch.empty(c["ctx_len"].shape, dtype=torch.int32).pin_memory()}
+    h2d_bytes = sum(t.numel() * t.element_size() for t in host_q + host_qd + [host_book])
     d2h_bytes = sum(t.numel() * t.element_size() for t in out_host.values())
-    h2d()
-    step = Step(dcache, wl)
 
     def one():
-        h2d()                       # the next step's copy replaces the compacted state
+        for d_, h_ in zip(c["q_win"], host_q):
+            d_.copy_(h_, non_blocking=True)
+        for d_, h_ in zip(step.q_dec, host_qd):
+            d_.copy_(h_, non_blocking=True)
+        step.book.copy_(host_book, non_blocking=True)   # the step's bookkeeping from the host
         step.run(restore=False)
         out_host["out"].copy_(step.out, non_blocking=True)
         out_host["keep"].copy_(step.keep, non_blocking=True)
-        out_host["block_table"].copy_(dcache["block_table"], non_blocking=True)
-        out_host["ctx_len"].copy_(dcache["ctx_len"], non_blocking=True)
+        out_host["block_table"].copy_(c["block_table"], non_blocking=True)
+        out_host["ctx_len"].copy_(c["ctx_len"], non_blocking=True)
 
     for _ in range(warmup):
         one()
@@ -322,15 +457,40 @@ def e2e_run(cache: dict, wl: synth.Workload, steps: int, warmup: int) -> dict:
         one()
     e1.record()
     torch.cuda.synchronize()
+    step.restore()
     ms = e0.elapsed_time(e1) / steps
+    del host_q, host_qd
     return {"ms_per_step": ms, "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes}
 
 
-def lacache_run(dev, batch: int, reps: int = 5, warmup: int = 3) -> dict:
-    """One LaCache ladder-compaction pass (all 32 layers, 64K -> 8192 slots per layer) on the
-    LaCache workload, timed with CUDA events; the block table, lengths and free list are
-    restored between passes (the pass only writes fresh blocks), so every pass sees the same
-    full cache."""
+def layer_workload_run(dev, steps: int, warmup: int, peaks: dict, src: str) -> dict:
+    """The one-layer workload (batch 32, 28 query / 4 KV heads, 4096-token caches, W=1024,
+    keep 204) through the same step, for comparison with the per-layer numbers."""
+    wl = LAYER_WORKLOAD
+    cache = synth.make_cache(wl, 1234 + 1, dev)
+    step = Step(cache, wl)
+    work = algorithmic_work(wl, cache)
+    total, avg, launches, _ = time_step(step, steps, warmup)
+    out = {"workload": "layer: one 7B-class layer, batch 32, 28 query / 4 KV heads, d=128, "
+                       "4096-token caches, W=1024, keep 204",
+           "ms_per_step": total / steps,
+           "tokens_per_s": wl.batch * wl.window / (total / steps / 1e3),
+           "gpu_launches_per_step": launches / steps,
+           "kernels": kernel_entries(wl, work, avg, step, peaks, src)}
+    out["variants"] = variants_run(step)
+    del step, cache
+    torch.cuda.empty_cache()
+    return out
+
+
+def lacache_run(dev, batch: int, peaks: dict, src: str) -> dict:
+    """The LaCache workload's three iterative ladder passes (batch 8, 32 layers, 8 KV heads,
+    64K-token caches, S=8, O=4, rung 64, budget 8192 per layer): pass 1 keeps 8192 slots per
+    layer of the full cache (the oldest 32768 slots are dropped in every layer), then 24576
+    new tokens are appended to every sequence (untimed: blocks popped from the free list,
+    their K/V drawn from N(0, 1)), refilling the cache to its capacity, and the ladder runs
+    again; passes 2 and 3 compress pass 1's survivors further. Each pass is timed with CUDA
+    events. A warm-up pass runs first and its bookkeeping is restored."""
     from decode_kv_cache_kara_b200 import kara as K
     wl = synth.WORKLOADS["lacache"].with_(batch=batch)
     ex = wl.extra
@@ -340,65 +500,93 @@ def lacache_run(dev, batch: int, reps: int = 5, warmup: int = 3) -> dict:
     ws = torch.empty(K.kara_workspace_bytes(K.OP_LACACHE, pool, wl.batch, 0, 0, ex["budget"]),
                      dtype=torch.uint8, device=dev)
     status = K.new_status(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + 9)
 
     def one():
         K.lacache_compact(cache["k"], cache["v"], pool, ex["span"], ex["overlap"], ex["rung"],
                           ex["budget"], ex["sink"], ex["recent"], workspace=ws, status=status)
 
-    def restore():
-        for k, t in saved.items():
-            cache[k].copy_(t)
+    def refill(tokens: int):
+        # append `tokens` slots to every sequence: their pages are popped from the free list
+        # (stack top first, sequences in order), their K/V rows drawn from N(0, 1)
+        pages = tokens // wl.page
+        top = int(cache["free_top"][0])
+        need = wl.batch * pages
+        if need > top:
+            raise RuntimeError("LaCache refill: free list too short")
+        ids = cache["free_list"][top - need:top].flip(0).view(wl.batch, pages)
+        p0 = cache["ctx_len"].long() // wl.page
+        cols = p0[:, None] + torch.arange(pages, device=dev)[None, :]
+        cache["block_table"].scatter_(1, cols, ids)
+        cache["free_top"][0] = top - need
+        cache["ctx_len"] += tokens
+        flat = ids.reshape(-1).long()
+        for layer in range(wl.layers):
+            for pool_t in (cache["k"][layer], cache["v"][layer]):
+                pool_t[flat] = torch.randn((flat.numel(),) + tuple(pool_t.shape[1:]),
+                                           generator=gen, device=dev).to(pool_t.dtype)
 
-    for _ in range(warmup):
-        one()
-        restore()
+    one()                                   # warm-up pass, then back to the full cache
     torch.cuda.synchronize()
-    times = []
-    for _ in range(reps):
+    for k, t in saved.items():
+        cache[k].copy_(t)
+    passes = []
+    for i in range(ex["passes"]):
+        if i > 0:
+            refill(ex["refill"])
+        torch.cuda.synchronize()
+        n_before = int(cache["ctx_len"][0])
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         one()
         e1.record()
         torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
-        restore()
-    torch.cuda.synchronize()
+        passes.append({"ms": e0.elapsed_time(e1), "ctx_before": n_before,
+                       "ctx_after": int(cache["ctx_len"][0])})
     st = K.read_status(status)
-    ms = sum(times) / len(times)
     # every layer keeps `budget` slots: K and V rows of [Hkv, d] read once and written once
     nbytes = 2 * 2 * wl.batch * wl.layers * ex["budget"] * wl.hkv * wl.head_dim * 2
+    for p in passes:
+        p["gbs"] = nbytes / p["ms"] / 1e6
+        p["frac_of_hbm_" + src] = p["gbs"] / peaks["hbm_gbs"]
+    ms = sum(p["ms"] for p in passes) / len(passes)
     del cache, saved, ws
     torch.cuda.empty_cache()
-    return {"ms": ms, "bound": "hbm", "gbs": nbytes / ms / 1e6, "bytes": nbytes, "status": st,
+    return {"ms": ms, "bound": "hbm", "gbs": nbytes / ms / 1e6, "bytes_per_pass": nbytes,
+            "frac_of_hbm_" + src: nbytes / ms / 1e6 / peaks["hbm_gbs"], "passes": passes,
+            "status": st,
             "workload": f"lacache: batch {wl.batch}, 32 layers, 8 KV heads, d=128, 64K-token "
-                        f"caches, S=8, O=4, rung 64, budget 8192 per layer; one pass (all layers)"}
+                        f"caches, S=8, O=4, rung 64, budget 8192 per layer; three iterative "
+                        f"passes (all layers each), 24576 tokens appended before passes 2 and 3"}
 
 
 def variants_run(step, reps: int = 10) -> dict:
-    """The score and selection variants on the layer workload (its window queries and cache,
-    not changed by them): kara_score_ex with the mean and with the max aggregation, and the
-    selection shared across KV heads (head sums, select, Token2Chunk, expansion to every
+    """The score and selection variants on the one-layer workload (its window queries and
+    cache, not changed by them): kara_score_ex with the mean and with the max aggregation, and
+    the selection shared across KV heads (head sums, select, Token2Chunk, expansion to every
     head). Average times with CUDA events over `reps` calls after one untimed call."""
     K, wl, c = step.K, step.wl, step.c
-    tot = torch.empty((wl.batch, wl.window), dtype=torch.float32, device=step.scores.device)
+    scores, keep, sel = step.scores[0], step.keep[0], step.sel[0]
+    tot = torch.empty((wl.batch, wl.window), dtype=torch.float32, device=scores.device)
     shared = torch.empty((wl.batch, wl.keep), dtype=torch.int32, device=tot.device)
-    sel = torch.empty((wl.batch, wl.keep), dtype=torch.int32, device=tot.device)
+    sel_t = torch.empty((wl.batch, wl.keep), dtype=torch.int32, device=tot.device)
 
     def score(agg):
         K.kara_score_ex(c["q_win"][0], c["k"][0], step.pool, wl.window, agg=agg,
-                        scores=step.scores, workspace=step.ws, status=step.status)
+                        scores=scores, workspace=step.ws, status=step.status)
 
     def shared_select():
-        K.kara_sum_heads(step.scores, out=tot)
-        K.kara_select(tot, wl.keep, sel=sel)
-        K.kara_token2chunk(tot, sel, step.na, wl.gap_limit, wl.widen, keep=shared)
-        K.kara_expand_keep(shared, wl.hkv, keep=step.keep[0])
+        K.kara_sum_heads(scores, out=tot)
+        K.kara_select(tot, wl.keep, sel=sel_t)
+        K.kara_token2chunk(tot, sel_t, wl.anchor_frac, wl.gap_limit, wl.widen, keep=shared)
+        K.kara_expand_keep(shared, wl.hkv, keep=keep)
 
     out = {}
+
     def select_then_chunks():
-        K.kara_select(step.scores, wl.keep, sel=step.sel)
-        K.kara_token2chunk(step.scores, step.sel, step.na, wl.gap_limit, wl.widen,
-                           keep=step.keep[0])
+        K.kara_select(scores, wl.keep, sel=sel)
+        K.kara_token2chunk(scores, sel, wl.anchor_frac, wl.gap_limit, wl.widen, keep=keep)
 
     for name, fn in (("score_mean_ms", lambda: score(K.AGG_MEAN)),
                      ("score_max_ms", lambda: score(K.AGG_MAX)),
@@ -413,18 +601,18 @@ def variants_run(step, reps: int = 10) -> dict:
         e1.record()
         torch.cuda.synchronize()
         out[name] = e0.elapsed_time(e1) / reps
-    # selection, Token2Chunk and compaction: two calls (three kernels) against kara_compress
-    # (plan + one fused kernel); the bookkeeping is restored between repetitions, untimed
+
+    # selection, Token2Chunk and compaction: two calls against kara_compress (plan + one
+    # fused kernel); the bookkeeping is restored between repetitions, untimed
     def compact_pair():
-        K.kara_select_chunks(step.scores, wl.keep, step.na, wl.gap_limit, wl.widen,
-                             keep=step.keep[0])
+        K.kara_select_chunks(scores, wl.keep, wl.anchor_frac, wl.gap_limit, wl.widen, keep=keep)
         K.kara_compact(c["k"], c["v"], step.pool, wl.window, step.keep, workspace=step.ws,
                        status=step.status)
 
     def compress():
-        K.kara_compress(step.scores[None], c["k"], c["v"], step.pool, wl.window, wl.keep, step.na,
-                        wl.gap_limit, wl.widen, keep=step.keep, workspace=step.ws,
-                        status=step.status)
+        K.kara_compress(step.scores, c["k"], c["v"], step.pool, wl.window, wl.keep,
+                        wl.anchor_frac, wl.gap_limit, wl.widen, keep=step.keep,
+                        workspace=step.ws, status=step.status)
 
     for name, fn in (("select_chunks_then_compact_ms", compact_pair), ("compress_ms", compress)):
         fn()
@@ -441,66 +629,69 @@ def variants_run(step, reps: int = 10) -> dict:
             total += e0.elapsed_time(e1)
         out[name] = total / reps
     out["status"] = K.read_status(step.status)
-    out["note"] = ("layer workload; max runs the two-pass kernels (a max, not a sum, per key); "
-                   "shared = head sums, one select + Token2Chunk per (sequence, layer), keep "
-                   "copied to the 4 KV heads; select_then_token2chunk = the two calls the "
+    out["note"] = ("one-layer workload; max runs the two-pass kernels (a max, not a sum, per "
+                   "key); shared = head sums, one select + Token2Chunk per (sequence, layer), "
+                   "keep copied to the 4 KV heads; select_then_token2chunk = the two calls the "
                    "step's fused kara_select_chunks replaces")
     return out
 
 
-def decode_loop_run(dev, steps: int = 300, period: int = 100, warm: int = 20) -> dict:
-    """The decode loop on the layer workload's shapes (batch 32, 28 query / 4 KV heads, d=128,
-    4096-token contexts, W=1024, keep 204, one layer): every step kara_step_begin,
-    kara_decode_append and kara_step_end; every `period` steps the due sequences (tail >= W)
-    are compressed (kara_score_ring, kara_select_chunks, kara_compact,
-    kara_reset_tails). Tails start spread over [0, W) and the query ring holds seeded queries,
-    as in the middle of a generation. Timed with CUDA events per step; a check step includes
-    the host read of the due count that sizes its compression."""
+def decode_loop_run(dev, wl: synth.Workload, seed: int, steps: int = 200, period: int = 100,
+                    warm: int = 10) -> dict:
+    """The amortised step under the 100-step schedule, on the bench workload's shapes (every
+    layer): every decode step runs kara_step_begin, kara_decode_append per layer (the new
+    token's attention, its K/V into the cache, its query into the layer's window-query ring)
+    and kara_step_end; every `period` steps the sequences whose uncompressed tail reached W
+    are due and are compressed (kara_score_ring and kara_select_chunks per layer, one
+    kara_compact of all layers, kara_reset_tails). Tails start uniform over [0, W) and the
+    rings hold N(0, 1) queries, as in the middle of a generation, so that each check finds
+    about batch * period / W due sequences. Timed with CUDA events per step; a check step
+    includes the host read of the due count that sizes its compression."""
     from decode_kv_cache_kara_b200 import kara as K
-    wl = WORKLOAD
-    W, B = wl.window, wl.batch
-    cache = synth.make_cache(wl, 1234 + 5, dev, with_queries=False,
+    W, B, L = wl.window, wl.batch, wl.layers
+    cache = synth.make_cache(wl, seed, dev, with_queries=False,
                              extra_pages=(steps + warm) // wl.page + 2)
     pool = K.PagedPool.from_cache(cache)
-    k0, v0 = cache["k"][0], cache["v"][0]
     gen = torch.Generator(device=dev)
-    gen.manual_seed(1234 + 6)
-    ring = torch.randn((B, 2 * W, wl.hq, wl.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+    gen.manual_seed(seed + 5)
+    rings = [torch.randn((B, 2 * W, wl.hq, wl.head_dim), generator=gen, device=dev)
+             .to(torch.bfloat16) for _ in range(L)]
     tail = torch.randint(0, W, (B,), generator=gen, device=dev, dtype=torch.int32)
-    inputs = [[torch.randn(shape, generator=gen, device=dev).to(torch.bfloat16)
-               for shape in ((B, wl.hq, wl.head_dim), (B, wl.hkv, wl.head_dim),
-                             (B, wl.hkv, wl.head_dim))] for _ in range(16)]
-    out = torch.empty((B, wl.hq, wl.head_dim), dtype=torch.bfloat16, device=dev)
+    inputs = [[[torch.randn(shape, generator=gen, device=dev).to(torch.bfloat16)
+                for shape in ((B, wl.hq, wl.head_dim), (B, wl.hkv, wl.head_dim),
+                              (B, wl.hkv, wl.head_dim))] for _ in range(L)] for _ in range(4)]
+    out = torch.empty((L, B, wl.hq, wl.head_dim), dtype=torch.bfloat16, device=dev)
     ws_dec = torch.empty(K.kara_workspace_bytes(K.OP_DECODE, pool, 0, 0, wl.hq, 0),
                          dtype=torch.uint8, device=dev)
-    ws_sc = torch.empty(K.kara_workspace_bytes(K.OP_SCORE, pool, B, W, wl.hq), dtype=torch.uint8,
-                        device=dev)
-    ws_cp = torch.empty(K.kara_workspace_bytes(K.OP_COMPACT, pool, B, W, 0, wl.keep),
-                        dtype=torch.uint8, device=dev)
-    scores = torch.empty((B, wl.hkv, W), dtype=torch.float32, device=dev)
-    sel = torch.empty((B, wl.hkv, wl.keep), dtype=torch.int32, device=dev)
-    keep = torch.empty((1, B, wl.hkv, wl.keep), dtype=torch.int32, device=dev)
+    ws = torch.empty(max(K.kara_workspace_bytes(K.OP_SCORE, pool, B, W, wl.hq),
+                         K.kara_workspace_bytes(K.OP_COMPACT, pool, B, W, 0, wl.keep)),
+                     dtype=torch.uint8, device=dev)
+    scores = torch.empty((L, B, wl.hkv, W), dtype=torch.float32, device=dev)
+    keep = torch.empty((L, B, wl.hkv, wl.keep), dtype=torch.int32, device=dev)
     due = torch.zeros(B, dtype=torch.int32, device=dev)
     due_count = torch.zeros(1, dtype=torch.int32, device=dev)
     status = K.new_status(dev)
-    na = wl.anchor_frac
 
     def step(t, check):
-        q, kn, vn = inputs[t % len(inputs)]
         K.kara_step_begin(pool, status)
-        K.kara_decode_append(q, kn, vn, k0, v0, pool, ring, W, out=out, workspace=ws_dec,
-                             status=status)
+        for layer in range(L):
+            q, kn, vn = inputs[t % len(inputs)][layer]
+            K.kara_decode_append(q, kn, vn, cache["k"][layer], cache["v"][layer], pool,
+                                 rings[layer], W, out=out[layer], workspace=ws_dec, status=status)
         K.kara_step_end(pool, tail, W, check, due, due_count)
         if not check:
             return 0
         cnt = int(due_count.item())
         if cnt:
             seq = due[:cnt]
-            K.kara_score_ring(ring, k0, pool, W, seq, cnt, scores=scores[:cnt], workspace=ws_sc,
-                              status=status)
-            K.kara_select_chunks(scores[:cnt], wl.keep, na, wl.gap_limit, wl.widen,
-                                 keep=keep[0, :cnt])
-            K.kara_compact([k0], [v0], pool, W, keep[:, :cnt], seq_ids=seq, workspace=ws_cp,
+            # the keep sets of the due sequences, [L, cnt, Hkv, k] contiguous
+            kp = keep.view(-1)[:L * cnt * wl.hkv * wl.keep].view(L, cnt, wl.hkv, wl.keep)
+            for layer in range(L):
+                K.kara_score_ring(rings[layer], cache["k"][layer], pool, W, seq, cnt,
+                                  scores=scores[layer, :cnt], workspace=ws, status=status)
+                K.kara_select_chunks(scores[layer, :cnt], wl.keep, wl.anchor_frac, wl.gap_limit,
+                                     wl.widen, keep=kp[layer])
+            K.kara_compact(cache["k"], cache["v"], pool, W, kp, seq_ids=seq, workspace=ws,
                            status=status)
             K.kara_reset_tails(tail, seq, cnt)
         return cnt
@@ -524,24 +715,33 @@ def decode_loop_run(dev, steps: int = 300, period: int = 100, warm: int = 20) ->
     plain = sorted(m for t, m in enumerate(ms) if t not in checks)
     st = K.read_status(status)
     total = sum(ms)
-    return {"steps": steps, "period": period, "ms_per_step": total / steps,
-            "decode_step_ms": plain[len(plain) // 2],
-            "check_step_ms": [ms[t] for t in checks], "due_per_check": dues,
-            "tokens_per_s": B * steps / (total / 1e3), "status": st,
-            "workload": f"decode loop: batch {B}, 28 query / 4 KV heads, d=128, 4096-token "
-                        f"contexts, W={W}, keep {wl.keep}, one layer, check every {period} "
-                        f"steps, tails spread over [0, W)"}
+    plain_ms = plain[len(plain) // 2]
+    extra = [ms[t] - plain_ms for t in checks]
+    comp_tokens = sum(dues) * W
+    res = {"steps": steps, "period": period, "layers": L, "ms_per_step": total / steps,
+           "decode_step_ms": plain_ms, "check_step_ms": [ms[t] for t in checks],
+           "due_per_check": dues, "compression_ms_per_check": extra,
+           "compressed_tokens_per_s": (comp_tokens / (sum(extra) / 1e3)
+                                       if sum(extra) > 0 else None),
+           "compression_share_of_time": sum(extra) / total,
+           "decode_tokens_per_s": B * steps / (total / 1e3), "status": st,
+           "workload": f"decode loop: batch {B}, {L} layers, 28 query / 4 KV heads, d=128, "
+                       f"ragged contexts [{wl.ctx_lo}, {wl.ctx_hi}], W={W}, keep {wl.keep}, "
+                       f"check every {period} steps (tail-W trigger), tails uniform over [0, W)"}
+    del cache, rings, inputs
+    torch.cuda.empty_cache()
+    return res
 
 
 def lacache_loop_run(dev, steps: int = 200, period: int = 100, warm: int = 10) -> dict:
-    """LaCache inside the decode loop on the layer workload's shapes with 4 layers (batch 32,
-    28 query / 4 KV heads, d=128, 4096-token contexts): every step kara_step_begin, one
+    """LaCache inside the decode loop on the one-layer workload's shapes with 4 layers (batch
+    32, 28 query / 4 KV heads, d=128, 4096-token contexts): every step kara_step_begin, one
     kara_decode_append per layer and kara_step_end with the capacity trigger; the ladder
     (S = 2, O = 1, rung 64, sink 64, recent 64, budget 2048 per layer, so capacity
     64 + 64 + 1920 * 4 / 2 = 3968 slots) runs on the sequences due at a check step. Timed with
     CUDA events per step; a check step includes the host read of the due count."""
     from decode_kv_cache_kara_b200 import kara as K
-    wl = WORKLOAD.with_(layers=4)
+    wl = LAYER_WORKLOAD.with_(layers=4)
     B, L = wl.batch, wl.layers
     span, overlap, rung, budget, sink, recent = 2, 1, 64, 2048, 64, 64
     cap = sink + recent + (budget - sink - recent) * L // span
@@ -597,123 +797,70 @@ def lacache_loop_run(dev, steps: int = 200, period: int = 100, warm: int = 10) -
     ms = [a.elapsed_time(b) for a, b in ev]
     plain = sorted(m for t, m in enumerate(ms) if t not in checks)
     total = sum(ms)
-    return {"steps": steps, "period": period, "layers": L, "capacity": cap,
-            "ms_per_step": total / steps, "decode_step_ms": plain[len(plain) // 2],
-            "check_step_ms": [ms[t] for t in checks], "due_per_check": dues,
-            "tokens_per_s": B * steps / (total / 1e3), "status": K.read_status(status),
-            "workload": "LaCache in the decode loop: batch 32, 4 layers, 28 query / 4 KV heads, "
-                        "d=128, 4096-token contexts, S=2, O=1, rung 64, sink 64, recent 64, "
-                        f"budget {budget} per layer, capacity {cap}, check every {period} steps"}
+    res = {"steps": steps, "period": period, "layers": L, "capacity": cap,
+           "ms_per_step": total / steps, "decode_step_ms": plain[len(plain) // 2],
+           "check_step_ms": [ms[t] for t in checks], "due_per_check": dues,
+           "tokens_per_s": B * steps / (total / 1e3), "status": K.read_status(status),
+           "workload": "LaCache in the decode loop: batch 32, 4 layers, 28 query / 4 KV heads, "
+                       "d=128, 4096-token contexts, S=2, O=1, rung 64, sink 64, recent 64, "
+                       f"budget {budget} per layer, capacity {cap}, check every {period} steps"}
+    del cache
+    torch.cuda.empty_cache()
+    return res
 
 
 def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
-    import torch.distributed as dist
-    from decode_kv_cache_kara_b200 import kara as K
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = WORKLOAD
     seed = rank_seed(rank)
+    peaks, src = load_peaks()
     cache = synth.make_cache(wl, seed, dev)
     work = algorithmic_work(wl, cache)
     step = Step(cache, wl)
-    for _ in range(args.warmup):
-        step.run()
-    torch.cuda.synchronize()
-    if K.read_status(step.status) != 0:
-        raise RuntimeError(f"device status after warm-up: {K.status_str(K.read_status(step.status))}")
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local_rank)
-    sampler.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    launches0 = K.kara_launch_count()
-    t0.record()
-    for i in range(args.steps):
-        step.run(ev[i])
-    t1.record()
-    launches = K.kara_launch_count() - launches0
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop()
-    total_ms = t0.elapsed_time(t1)
-    if K.read_status(step.status) != 0:
-        raise RuntimeError(f"device status: {K.status_str(K.read_status(step.status))}")
-
-    op_ms = {"kara_score": [], "select+token2chunk": [], "kara_compact": [],
-             "paged_decode_attn": []}
-    for e in ev:
-        op_ms["kara_score"].append(e[0].elapsed_time(e[1]))
-        op_ms["select+token2chunk"].append(e[1].elapsed_time(e[2]))
-        op_ms["kara_compact"].append(e[2].elapsed_time(e[3]))
-        op_ms["paged_decode_attn"].append(e[3].elapsed_time(e[4]))
-    avg = {k: sum(v) / len(v) for k, v in op_ms.items()}
-
+    total_ms, avg, launches, clocks = time_step(step, args.steps, args.warmup, world, sampler)
     total_ms = max_over_ranks(total_ms, dev, world)
     ms_step = total_ms / args.steps
-    tokens_step = wl.batch * wl.window * world
-    value = whole_job_value(wl.batch * wl.window, world, ms_step)
+    tokens_step = wl.batch * wl.window          # window tokens compressed per step and rank
+    value = whole_job_value(tokens_step, world, ms_step)
 
-    e2e = e2e_run(cache, wl, steps=min(args.steps, args.e2e_steps), warmup=2)
-    e2e_ms = max_over_ranks(e2e["ms_per_step"], dev, world)
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_run(step, steps=args.e2e_steps, warmup=1)
+        e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], dev, world)
+    kernels = kernel_entries(wl, work, avg, step, peaks, src)
+    del step, cache
+    torch.cuda.empty_cache()
     if rank != 0:
         return None
 
-    peaks, src = load_peaks()
-    # the exponentials bound scoring: one per softmax element, 16 per clock per SM on the SFU
-    n_exp = wl.window * wl.window * wl.hq * wl.batch
-    sfu_floor_ms = n_exp / (16 * 148 * 1.965e9) * 1e3
-    if step.score_fused:
-        score_exec, score_note = 1.25, ("fused single-exponential kernel: S over 144 key rows "
-                                        "per 128 owned keys (x1.125) plus the P'^T W column-sum "
-                                        "product (N = 16, x0.125): executed = 1.25 x useful")
-    else:
-        score_exec, score_note = 2.0, ("two UMMA passes (row log-sum-exp, then column sums): "
-                                       "executed flops are twice the useful Q K^T")
-    kernels = {
-        "kara_score": {"ms": avg["kara_score"], "bound": "tensor",
-                       "useful_tflops": work["score_flops"] / avg["kara_score"] / 1e9,
-                       "executed_tflops": score_exec * work["score_flops"] / avg["kara_score"] / 1e9,
-                       "note": score_note,
-                       "exp2_count": n_exp,
-                       "sfu_floor_ms": sfu_floor_ms,
-                       "frac_of_sfu_floor": sfu_floor_ms / avg["kara_score"]},
-        "select+token2chunk": {"ms": avg["select+token2chunk"], "bound": "latency"},
-        "kara_compact": {"ms": avg["kara_compact"], "bound": "hbm",
-                         "gbs": work["compact_bytes"] / avg["kara_compact"] / 1e6},
-        "paged_decode_attn": {"ms": avg["paged_decode_attn"], "bound": "hbm",
-                              "gbs": work["decode_bytes"] / avg["paged_decode_attn"] / 1e6},
-    }
-    for k, v in kernels.items():
-        if v["bound"] == "hbm":
-            v["frac_of_hbm_" + src] = v["gbs"] / peaks["hbm_gbs"]
-        elif v["bound"] == "tensor":
-            v["frac_of_bf16_" + src] = v["useful_tflops"] / peaks["bf16_tflops"]
     dom = max((k for k in kernels if kernels[k]["bound"] in ("tensor", "hbm")),
               key=lambda k: kernels[k]["ms"])
     dk = kernels[dom]
     traffic = captured_traffic(dom)
+    per_launch = (f"the op runs as {dk['launches_of_op']} launches per step (one per layer); "
+                  "achieved = useful work of all of them / their summed duration")
     if dk["bound"] == "tensor":
         roof = {"kernel": dom, "bound": "tensor", "achieved": dk["useful_tflops"],
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": dk["useful_tflops"] / peaks["bf16_tflops"], "traffic": traffic,
-                "peak_source": f"{src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)"}
+                "peak_source": f"{src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)",
+                "per_launch": per_launch}
     else:
         roof = {"kernel": dom, "bound": "hbm", "achieved": dk["gbs"], "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": dk["gbs"] / peaks["hbm_gbs"], "traffic": traffic,
-                "peak_source": f"{src} HBM copy (MEASURED_PEAKS.json hbm_gbs)"}
+                "peak_source": f"{src} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
+                "per_launch": per_launch}
 
-    if world == 1 and not args.no_lacache:
-        lac = lacache_run(dev, args.lacache_batch)
-        lac["frac_of_hbm_" + src] = lac["gbs"] / peaks["hbm_gbs"]
-        kernels["lacache_compact"] = lac
     if world == 1 and not args.no_loop:
-        kernels["decode_loop"] = decode_loop_run(dev)
+        kernels["amortised_100_step_schedule"] = decode_loop_run(dev, wl, seed + 50)
+    if world == 1 and not args.no_layer:
+        kernels["layer"] = layer_workload_run(dev, max(3, min(args.steps, 20)), 3, peaks, src)
+    if world == 1 and not args.no_lacache:
+        kernels["lacache_compact"] = lacache_run(dev, args.lacache_batch, peaks, src)
+    if world == 1 and not args.no_loop:
         kernels["lacache_loop"] = lacache_loop_run(dev)
-        kernels["variants"] = variants_run(step)
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -722,72 +869,69 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD_DESC, "batch_per_gpu": wl.batch, "layers": wl.layers,
-                   "q_heads": wl.hq, "kv_heads": wl.hkv, "head_dim": wl.head_dim,
-                   "context": wl.ctx_lo, "window": wl.window, "keep": wl.keep, "page": wl.page,
-                   "anchor_frac": wl.anchor_frac, "gap_limit": wl.gap_limit, "widen": wl.widen,
-                   "parallelism": f"dp{world} (independent sequences per rank)",
-                   "l2": "inputs larger than L2 (window queries 235 MB, KV pool 302 MB per GPU)"},
+        "config": bench_config(wl, world),
         "roofline": roof,
         "kernels": kernels,
         "cpu_baseline": cpu,
-        "e2e": {"value": tokens_step / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
-                "d2h_bytes_per_step": e2e["d2h_bytes_per_step"], "ms_per_step": e2e_ms},
         "gpu_launches": launches,
         "clocks": clocks,
     }
+    if e2e is not None:
+        line["e2e"] = {"value": tokens_step * world / (e2e["ms_per_step"] / 1e3), "unit": UNIT,
+                       "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                       "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
+                       "ms_per_step": e2e["ms_per_step"],
+                       "note": "window queries of every layer, decode queries and the pool "
+                               "bookkeeping copied from pinned host memory every step; decode "
+                               "outputs, keep sets, block table and lengths read back; the KV "
+                               "pools stay resident on the device"}
     return line
 
 
 def cpu_baseline(seed: int, target_s: float = 15.0) -> dict:
     """The oracle as it stands on the host cores, on a bounded sample of the same workload:
-    as many (sequence, KV head) units as take about target_s seconds (at most 256)."""
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count() or 1
-    cache_cpu = synth.make_cache(WORKLOAD, seed, "cpu")
-    dt, tokens = time_cpu_oracle_sample(cache_cpu, WORKLOAD, units=1, seed=seed)
+    as many (sequence, layer, KV head) units as take about target_s seconds (at most 256)."""
+    cores = host_cores()
+    cache_cpu = oracle_sample_cache(seed)
+    wl = WORKLOAD.with_(batch=4, layers=1)
+    dt, tokens = time_cpu_oracle_sample(cache_cpu, wl, units=1, seed=seed,
+                                        layers_per_step=WORKLOAD.layers)
     units = max(1, int(target_s / max(dt, 1e-3)))
     units = min(units, 256)
-    dt, tokens = time_cpu_oracle_sample(cache_cpu, WORKLOAD, units=units, seed=seed + 1)
+    dt, tokens = time_cpu_oracle_sample(cache_cpu, wl, units=units, seed=seed + 1,
+                                        layers_per_step=WORKLOAD.layers)
     return {"value": tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{units} (sequence, KV head) units of the layer workload: window scoring "
-                      f"of its 7 query heads, top-k, Token2Chunk, compaction of its rows and "
-                      f"decode of its 7 query heads; tokens counted as W/Hkv per unit",
+            "sample": f"{units} (sequence, layer, KV head) units of the step workload (ragged "
+                      f"contexts 2K-16K, W=1024, keep 204): window scoring of the unit's 7 query "
+                      f"heads, top-k, Token2Chunk, compaction of its rows and decode of its 7 "
+                      f"query heads; tokens counted as W / (Hkv * 28 layers) per unit",
             "seconds": dt}
 
 
 def reference_arm(args, rank: int) -> dict | None:
     if rank != 0:
         return None
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count() or 1
-    wl = WORKLOAD
-    cache_cpu = synth.make_cache(wl, rank_seed(0), "cpu")
+    cores = host_cores()
+    wl = WORKLOAD.with_(batch=4, layers=1)
+    cache_cpu = oracle_sample_cache(rank_seed(0))
     for i in range(args.warmup):
-        time_cpu_oracle_sample(cache_cpu, wl, units=1, seed=i)
+        time_cpu_oracle_sample(cache_cpu, wl, units=1, seed=i, layers_per_step=WORKLOAD.layers)
     total, tokens = 0.0, 0.0
     for i in range(args.steps):
-        dt, tk = time_cpu_oracle_sample(cache_cpu, wl, units=1, seed=10_000 + i)
+        dt, tk = time_cpu_oracle_sample(cache_cpu, wl, units=1, seed=10_000 + i,
+                                        layers_per_step=WORKLOAD.layers)
         total += dt
         tokens += tk
     value = tokens / total
-    sample = ("each step: one (sequence, KV head) unit of the layer workload through the fp64 "
-              "oracle (scoring of 7 query heads x 1024 x 1024, top-k, Token2Chunk, compaction, "
-              "decode); tokens counted as W/Hkv per unit")
+    sample = ("each step: one (sequence, layer, KV head) unit of the step workload through the "
+              "fp64 oracle (scoring of 7 query heads x 1024 x 1024, top-k, Token2Chunk, "
+              "compaction, decode); tokens counted as W / (Hkv * 28 layers) per unit")
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD_DESC, "batch_per_gpu": wl.batch, "window": wl.window,
-                   "keep": wl.keep, "parallelism": "host cores (oracle)"},
+        "config": bench_config(WORKLOAD, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -797,16 +941,19 @@ def reference_arm(args, rank: int) -> dict | None:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["kara", "reference"], default="kara")
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-input measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-lacache", action="store_true",
                     help="skip the LaCache ladder-compaction measurement (1 GPU only)")
     ap.add_argument("--lacache-batch", type=int, default=8)
     ap.add_argument("--no-loop", action="store_true",
-                    help="skip the decode-loop measurement (kernels.decode_loop)")
+                    help="skip the decode-loop measurements (amortised schedule, LaCache loop)")
+    ap.add_argument("--no-layer", action="store_true",
+                    help="skip the one-layer workload and the variants")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

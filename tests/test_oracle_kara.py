@@ -453,6 +453,28 @@ def test_max_closed_forms():
     assert np.allclose(mx[0], [p0, 0.5])      # query 1 has equal logits: 0.5 for both keys
 
 
+def test_shared_keep_golden_cases():
+    # hand-worked cases (tests/golden/shared_keep_cases.txt) in which the shared keep set is
+    # neither a per-head selection, nor the selection of the maximum over heads
+    cases = load_golden("shared_keep_cases.txt")
+    assert len(cases) >= 3
+    for c in cases:
+        heads = sorted(key for key in c if key.startswith("h"))
+        sc = np.array([c[h] for h in heads])
+        k, na = int(c["k"][0]), int(c["num_anchors"][0])
+        gap, wid = int(c["gap_limit"][0]), int(c["widen"][0])
+        keep = ok.shared_keep(sc, k, na, gap, wid)
+        expect = [int(x) for x in c["keep"]]
+        assert keep.shape == (len(heads), k)
+        assert all(row.tolist() == expect for row in keep)
+        assert sc.sum(axis=0).tolist() == c["sum"]
+        assert ok.select_topk(sc.sum(axis=0), k).tolist() == [int(x) for x in c["sel"]]
+        for h in range(len(heads)):
+            assert ok.token2chunk(sc[h], ok.select_topk(sc[h], k), na, gap, wid).tolist() != expect
+        mx = sc.max(axis=0)
+        assert ok.token2chunk(mx, ok.select_topk(mx, k), na, gap, wid).tolist() != expect
+
+
 def test_shared_keep_is_the_selection_of_the_head_sum():
     rng = np.random.default_rng(4)
     sc = rng.random((3, 40))
