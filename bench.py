@@ -68,16 +68,17 @@ def bench_config(wl: synth.Workload, world: int) -> dict:
             "l2": "inputs larger than L2 (window queries 26.3 GB, KV pools about 70 GB per GPU)"}
 
 
-def captured_traffic(op: str):
+def captured_traffic(op: str, workload: str):
     """DRAM bytes per launch of `op` from the committed ncu summary (profiles/traffic.txt),
-    or None when the kernel source changed since the capture (its sha256 no longer matches)."""
+    captured on a launch of `workload`'s shape; None when there is no such capture or the
+    kernel source changed since (its sha256 no longer matches)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
     for line in open(path):
         parts = line.split()
-        if len(parts) != 4 or line.startswith("#") or parts[0] != op:
+        if len(parts) != 5 or line.startswith("#") or parts[0] != op or parts[4] != workload:
             continue
         src = os.path.join(ROOT, "decode_kv_cache_kara_b200", parts[1])
         if not os.path.exists(src):
@@ -812,7 +813,7 @@ def lacache_loop_run(dev, steps: int = 200, period: int = 100, warm: int = 10) -
 def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl = WORKLOAD
+    wl = WORKLOAD if args.layers is None else WORKLOAD.with_(layers=args.layers)
     seed = rank_seed(rank)
     peaks, src = load_peaks()
     cache = synth.make_cache(wl, seed, dev)
@@ -838,7 +839,7 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
     dom = max((k for k in kernels if kernels[k]["bound"] in ("tensor", "hbm")),
               key=lambda k: kernels[k]["ms"])
     dk = kernels[dom]
-    traffic = captured_traffic(dom)
+    traffic = captured_traffic(dom, wl.name)
     per_launch = (f"the op runs as {dk['launches_of_op']} launches per step (one per layer); "
                   "achieved = useful work of all of them / their summed duration")
     if dk["bound"] == "tensor":
@@ -954,6 +955,9 @@ def main():
                     help="skip the decode-loop measurements (amortised schedule, LaCache loop)")
     ap.add_argument("--no-layer", action="store_true",
                     help="skip the one-layer workload and the variants")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layers of the step workload (default: all 28); fewer layers keep a "
+                         "profiler capture of one layer's launches small")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
