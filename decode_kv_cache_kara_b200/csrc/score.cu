@@ -747,27 +747,25 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
 // 128-query tile each CTA
 //   1. computes S = Q K^T over its keys (UMMA M = 128 queries, N = 144 key rows: the 9 pages
 //      that cover its 128 keys at any slot offset; only the owned columns are read);
-//   2. in the epilogue (8 warps: a TMEM lane quadrant and 64 owned keys each) takes the row
-//      max m_p over its 64 keys, P' = 2^(s*c - m_p + 15) and the row sum l_p, and stores P' as
-//      fp16 in shared memory, MN-major (rows along K) for the next product;
-//   3. combines the two parts of each row and sends the partial log-sum-exp of its 128 keys,
-//      lse = m + log2(l), to every CTA of the cluster (st.async into their shared memory,
-//      counted on their mbarrier);
+//   2. in the epilogue (4 warps, one per TMEM lane quadrant: a thread owns one query row and
+//      the CTA's 128 keys) takes the row max m over its keys, P' = 2^(s*c - m + 15) and the
+//      row sum l, and stores P' as fp16 in shared memory, MN-major (rows along K) for the next
+//      product;
+//   3. sends the row's partial log-sum-exp over its 128 keys, lse = m + log2(l), to every CTA
+//      of the cluster (st.async into their shared memory, counted on their mbarrier);
 //   4. once all CL partials of a row are in: M = max lse, L = sum 2^(lse - M), and the row
-//      weight of part p is w = 2^(m_p - M + 15) / L (so that P' w = 2^15 softmax); w goes to
-//      fp16 as three B columns (w1 + w2 + 2^-24 w3, exact to about 2^-36);
+//      weight w = 2^(m - M + 15) / L (so that P' w = 2^15 softmax); w goes to fp16 as three B
+//      columns (w1 + w2 + 2^-24 w3, exact to about 2^-36);
 //   5. D (128 keys x 16) += P'^T W: the column sums of the tile's softmax rows on the tensor
 //      cores (UMMA M = 128 keys, K = 128 queries, N = 16), accumulated over the item's tiles.
-// Two teams of epilogue warps take alternate tiles, so one team's exponentials overlap the
-// other's exchange and weights. P' and the weights have three buffers, taken round-robin by
-// tile: a team's next tile writes the buffer of the other team's previous tile, so the wait
-// for a buffer (exchange, weights and column-sum product of its last tile) gets one more tile
-// of slack than with a buffer per team. After the item's last tile, D (times 2^-15) holds the
-// per-key scores summed over the item's G heads.
+// Three teams of 4 epilogue warps take the tiles in turn, each with its own S accumulator in
+// TMEM and its own P' and weight buffers, so that a team's wait for the cluster exchange and
+// its weights overlap the other two teams' exponentials. After the item's last tile, D (times
+// 2^-15) holds the // per-key scores summed over the item's G heads.
 // ----------------------------------------------------------------------------------------
-constexpr int kFEpiWarps = 16;                    // two teams of 8, tiles alternate between them
-constexpr int kFParts = 2;                        // per team: 2 warps per TMEM lane quadrant
-constexpr int kFPartKeys = 128 / kFParts;         // 64 keys per warp
+constexpr int kFTeams = 3;                        // epilogue teams, tile T goes to team T mod 3
+constexpr int kFEpiWarps = 4 * kFTeams;           // a team: one warp per TMEM lane quadrant
+constexpr int kFTeamThreads = 128;                // a thread owns one query row of the tile
 // warps 0-3: TMA producer, S issuer, column-sum issuer, and a spare, so that each of the four
 // SM sub-partitions holds one such warp beside its four epilogue warps
 constexpr int kFThreads = 128 + 32 * kFEpiWarps;
@@ -776,14 +774,14 @@ constexpr int kFKeys = 128;            // window keys owned per CTA
 constexpr int kFKRows = 144;           // key rows loaded per CTA (9 pages)
 constexpr int kFQRows = 128;           // queries per tile
 constexpr int kFMaxCluster = 8;
-constexpr int kFPBufs = 3;             // P' and weight buffers, tile T in buffer T mod 3
+constexpr int kFPBufs = kFTeams;       // S, P' and weight buffers, tile T in buffer T mod 3
 constexpr int kFQSlots = 3;            // query ring slots of one 64-channel chunk each
-constexpr int kFXStages = 5;           // exchange slots: a peer sends tile T + 5 only after this
-                                       // CTA's exponentials of tile T + 2, which its team starts
-                                       // after reading the partials of tile T
-constexpr uint32_t kFEpiBarrier = 1;
-constexpr uint32_t kFSCols = 256;      // TMEM column stride of the two S buffers
-constexpr uint32_t kFDCol = 160;       // TMEM columns of the two D buffers: 160, 176
+constexpr int kFXStages = 6;           // exchange slots: a peer sends its record of tile T + 6
+                                       // only after its weights of tile T + 3, which need this
+                                       // CTA's record of tile T + 3, which the team of tile T
+                                       // sends after it has read the partials of tile T
+constexpr uint32_t kFSCols = kFKRows;  // TMEM column stride of the three S buffers: 0, 144, 288
+constexpr uint32_t kFDCol = kFTeams * kFSCols;   // TMEM columns of the two D buffers: 432, 448
 
 // Work items (r, g): KV head g of sequence r with all G of its query heads, TPI = G * W / 128
 // query tiles (tile tq: head g * G + tq / CL, queries 128 (tq % CL) ..). Cluster c of ncl takes
@@ -841,9 +839,8 @@ struct FusedSmem {
   static constexpr uint32_t p_off = q_off + kFQSlots * kQChunk;
   static constexpr uint32_t w_off = p_off + kFPBufs * kPBytes;
   static constexpr uint32_t x_off = w_off + kFPBufs * kWBytes;
-  static constexpr uint32_t comb_off = x_off + kXBytes;  // [team][tile parity][part][128] float2
-  static constexpr uint32_t bar_off = comb_off + 2 * 2 * 2 * kFQRows * 8;
-  static constexpr uint32_t kBars = 2 + 2 * kFQSlots + 2 * 2 + 3 * kFPBufs + 2 * 2 + kFXStages;
+  static constexpr uint32_t bar_off = x_off + kXBytes;
+  static constexpr uint32_t kBars = 2 + 2 * kFQSlots + 2 * kFTeams + 3 * kFPBufs + 2 * 2 + kFXStages;
   static constexpr uint32_t end = bar_off + kBars * 8 + 16;
   static constexpr size_t bytes = 1024 + end;
   static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
@@ -872,15 +869,14 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint8_t* p_buf = smem + L::p_off;
   uint8_t* w_buf = smem + L::w_off;
   float* x_buf = reinterpret_cast<float*>(smem + L::x_off);       // [stage][src rank][row]: lse
-  float2* comb = reinterpret_cast<float2*>(smem + L::comb_off);   // [team][par][part][row]: (m, l)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bar_off);
   uint64_t* k_full = bars;
   uint64_t* k_empty = bars + 1;
   uint64_t* q_full = bars + 2;                     // [kFQSlots]
   uint64_t* q_empty = q_full + kFQSlots;
-  uint64_t* s_full = q_empty + kFQSlots;           // [2]
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;                  // [kFPBufs]
+  uint64_t* s_full = q_empty + kFQSlots;           // [kFTeams]
+  uint64_t* s_empty = s_full + kFTeams;
+  uint64_t* p_full = s_empty + kFTeams;            // [kFPBufs]
   uint64_t* w_full = p_full + kFPBufs;
   uint64_t* p_empty = w_full + kFPBufs;
   uint64_t* d_full = p_empty + kFPBufs;            // [2]
@@ -903,27 +899,29 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&q_empty[i], 1);
     }
     for (int i = 0; i < kFPBufs; ++i) {
-      mbar_init(&p_full[i], kFEpiThreads / 2);      // one team per tile
-      mbar_init(&w_full[i], kFEpiThreads / 4);      // the team's part-1 threads
+      mbar_init(&p_full[i], kFTeamThreads);         // one team per tile
+      mbar_init(&w_full[i], kFTeamThreads);
       mbar_init(&p_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kFTeams; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], kFEpiThreads / 2);
+      mbar_init(&s_empty[i], kFTeamThreads);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&d_full[i], 1);
-      mbar_init(&d_empty[i], kFEpiThreads / 2);
+      mbar_init(&d_empty[i], kFTeamThreads);       // the team that reads the segment's sums
     }
     for (int i = 0; i < kFXStages; ++i) mbar_init(&x_full[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp >= 4) {
-    // the weight operands' unused rows (n = 3 * parts .. 15) stay zero
-    constexpr int kZ = 16 - 3 * kFParts;
+    // the weight operands' unused rows (n = 3 .. 15) stay zero
+    constexpr int kZ = 16 - 3;
     const int t = threadIdx.x - 128;
     for (int i = t; i < kFPBufs * 2 * kZ * 8; i += kFEpiThreads) {
       const int buf = i / (16 * kZ), rem = i % (16 * kZ), kc = rem / (8 * kZ);
-      const int n = 3 * kFParts + (rem % (8 * kZ)) / 8, c = rem % 8;
+      const int n = 3 + (rem % (8 * kZ)) / 8, c = rem % 8;
       *reinterpret_cast<uint4*>(w_buf + buf * L::kWBytes + kc * 2048 + n * 128 + c * 16) =
           make_uint4(0u, 0u, 0u, 0u);
     }
@@ -1015,8 +1013,8 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!mbar_wait(k_full, I & 1, abort_flag, a.status)) break;
         const uint32_t k_addr = smem_u32(k_buf);
         for (int tq = cur.q0; tq < cur.q1 && ok; ++tq, ++T) {
-          const int st = T & 1;
-          const uint32_t ph = (T >> 1) & 1;
+          const int st = T % kFTeams;
+          const uint32_t ph = (T / kFTeams) & 1;
           if (!mbar_wait(&s_empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
           const uint32_t d_tmem = tmem_base + st * kFSCols;
           for (int ch = 0; ch < NCH; ++ch, ++C) {
@@ -1075,13 +1073,13 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
   } else if (warp >= 4) {
-    // ---- epilogue: two teams of 8 warps take alternate tiles (team = tile parity), so that
-    // one team's exponentials overlap the other's exchange and weights. In a team, warp
-    // (quad, part) owns TMEM lane quadrant `quad` and keys [64 part, 64 part + 64). ----
+    // ---- epilogue: three teams of 4 warps take the tiles in turn (team = tile mod 3), so
+    // that a team's exchange wait and weights overlap the other teams' exponentials. In a
+    // team, warp `quad` owns TMEM lane quadrant `quad`: each thread one query row and all
+    // 128 keys of this CTA. ----
     const int e = warp - 4;
-    const int team = e >> 3;
+    const int team = e >> 2;
     const int quad = warp & 3;
-    const int part = (e & 7) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     const float2 cs2 = make_float2(a.cs, a.cs);
@@ -1107,15 +1105,17 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       ++I;
       have = cur.next(a, TPI);
     }
-    // running T mod 3 / T div 3 (P' and weight buffers) and T mod 5 / T div 5 (exchange slots)
-    int pb = team, pq = 0, xs = team, xq = 0;
-    for (int T = team; have; T += 2) {
-      const int st = T & 1;     // = team: S buffer
-      const uint32_t ph = (T >> 1) & 1;
-      const uint32_t pph = pq & 1;
+    // this team's buffers: S, P' and weights `team`, used every third tile (phase = T div 3);
+    // exchange slot T mod 6 (xs) and its phase T div 6 (xq)
+    const int st = team;
+    uint8_t* const prow = p_buf + st * L::kPBytes + (row >> 3) * 1024 + (row & 7) * 128;
+    uint32_t sq = 0;
+    int xs = team, xq = 0;
+    for (int T = team; have; T += kFTeams, ++sq) {
+      const uint32_t ph = sq & 1;
       const uint32_t scol = lane_base + st * kFSCols +
-                            ((cur.s.start + static_cast<int>(rank) * kFKeys) % 16) + part * kFPartKeys;
-      // (1) row max over this warp's 64 keys (first pass over TMEM)
+                            ((cur.s.start + static_cast<int>(rank) * kFKeys) % 16);
+      // (1) row max over this CTA's 128 keys (first pass over TMEM)
       wait_cta(&s_full[st], ph);
       float mx = 0.f, l = 0.f;
       if (!aborted) {
@@ -1123,7 +1123,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
         float v[32];
         float mm = -INFINITY;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 4; ++h) {
           tmem_ld16(scol + 32 * h, v);
           tmem_ld16(scol + 32 * h + 16, v + 16);
           tmem_wait_ld();
@@ -1137,25 +1137,25 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
           mm = fmaxf(fmax3(m0, m1, m2), m3);
         }
         mx = mm * a.cs;
-        wait_cta(&p_empty[pb], pph ^ 1);
+        wait_cta(&p_empty[st], ph ^ 1);
       }
-      // (2) P' = 2^(s c - m + 15) as fp16 in shared memory (second pass), and the row sum
+      // (2) P' = 2^(s c - m + 15) as fp16 in shared memory (second pass), and the row sum;
+      // keys [32 h, 32 h + 32) go to atom h / 2, granules 4 (h mod 2) .. + 3
       if (!aborted) {
         const float2 nb2 = make_float2(15.f - mx, 15.f - mx);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-        uint8_t* prow = p_buf + pb * L::kPBytes + part * L::kPAtom + (row >> 3) * 1024 +
-                        (row & 7) * 128;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 4; ++h) {
           float v[32];
           tmem_ld16(scol + 32 * h, v);
           tmem_ld16(scol + 32 * h + 16, v + 16);
           tmem_wait_ld();
           reg_fence<32>(v);
-          if (h == 1) {
+          if (h == 3) {
             tc_fence_before();
             mbar_arrive(&s_empty[st]);
           }
+          uint8_t* patom = prow + (h >> 1) * L::kPAtom;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t pk[4];
@@ -1171,36 +1171,28 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
               pk[i / 2] = pack_f16x2(e0.x, e0.y);
               pk[i / 2 + 1] = pack_f16x2(e1.x, e1.y);
             }
-            const int cc = 4 * h + c;
-            *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) =
+            const int cc = 4 * (h & 1) + c;
+            *reinterpret_cast<uint4*>(patom + ((cc ^ (row & 7)) << 4)) =
                 make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
         l = (acc0.x + acc0.y) + (acc1.x + acc1.y);
         fence_proxy_async();
-        mbar_arrive(&p_full[pb]);
+        mbar_arrive(&p_full[st]);
       }
-      // (3) the CTA's partial log-sum-exp of each row to every CTA of the cluster
-      if ((e & 7) == 0 && lane == 0) mbar_expect_tx(&x_full[xs], CL * kFQRows * 4);
-      // two halves by the team's tile parity: part 0 rewrites a half only after the named
-      // barrier of the team's next tile, which part 1 reaches after reading it for this one
-      float2* cb = comb + (team * 2 + static_cast<int>(ph)) * 2 * kFQRows;
-      cb[part * kFQRows + row] = make_float2(mx, l);
-      named_barrier(kFEpiBarrier + team * 4 + quad, 64);   // the two warps sharing these rows
-      if (part == 0 && !aborted) {
-        const float2 o = cb[kFQRows + row];
-        const float M = fmaxf(mx, o.x);
-        const float lse = M + lg2(l * ex2(mx - M) + o.y * ex2(o.x - M));
+      // (3) the CTA's partial log-sum-exp of the row to every CTA of the cluster
+      if ((e & 3) == 0 && lane == 0) mbar_expect_tx(&x_full[xs], CL * kFQRows * 4);
+      if (!aborted) {
+        const float lse = mx + lg2(l);
         const uint32_t slot = x_buf_u32 + ((xs * kFMaxCluster + rank) * kFQRows + row) * 4;
         const uint32_t xb = x_full_u32 + xs * 8;
 #pragma unroll
         for (int c = 0; c < CL; ++c) st_async_f32(map_to_rank(slot, c), lse, map_to_rank(xb, c));
       }
-      // (4) meanwhile, once every CTA's partials are in, the row's thread of part 1 writes the
-      // weights of both parts, w_p = 2^(m_p - M + 15) / L, as three fp16 columns each of the B
-      // operand
-      if (part == 1) wait_cluster(&x_full[xs], xq & 1);
-      if (part == 1 && !aborted) {
+      // (4) once every CTA's partials are in: the row weight w = 2^(m - M + 15) / L as three
+      // fp16 columns of the B operand
+      wait_cluster(&x_full[xs], xq & 1);
+      if (!aborted) {
         const float* xr = x_buf + xs * kFMaxCluster * kFQRows + row;
         float xv[CL];
 #pragma unroll
@@ -1211,57 +1203,48 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
         float Lsum = 0.f;
 #pragma unroll
         for (int c = 0; c < CL; ++c) Lsum += ex2(xv[c] - M);
-        const float inv = 1.f / Lsum;
-        const float m_part0 = cb[row].x;
-        uint8_t* wb = w_buf + pb * L::kWBytes;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const float w = ex2((q == 0 ? m_part0 : mx) - M + 15.f) * inv;
-          const __half w1 = __float2half_rn(w);
-          const float r1 = w - __half2float(w1);
-          const __half w2 = __float2half_rn(r1);
-          const float r2 = r1 - __half2float(w2);
-          const __half w3 = __float2half_rn(r2 * 16777216.f);
-          *reinterpret_cast<__half*>(wb + w_offset(3 * q, row)) = w1;
-          *reinterpret_cast<__half*>(wb + w_offset(3 * q + 1, row)) = w2;
-          *reinterpret_cast<__half*>(wb + w_offset(3 * q + 2, row)) = w3;
-        }
+        const float w = ex2(mx - M + 15.f) / Lsum;
+        const __half w1 = __float2half_rn(w);
+        const float r1 = w - __half2float(w1);
+        const __half w2 = __float2half_rn(r1);
+        const float r2 = r1 - __half2float(w2);
+        const __half w3 = __float2half_rn(r2 * 16777216.f);
+        uint8_t* wb = w_buf + st * L::kWBytes;
+        *reinterpret_cast<__half*>(wb + w_offset(0, row)) = w1;
+        *reinterpret_cast<__half*>(wb + w_offset(1, row)) = w2;
+        *reinterpret_cast<__half*>(wb + w_offset(2, row)) = w3;
         fence_proxy_async();
-        mbar_arrive(&w_full[pb]);
+        mbar_arrive(&w_full[st]);
       }
       // (5) the segment's last tile: the per-key sums over its heads, read by this team
       if (tp == cur.q1 - cur.q0 - 1) {
         wait_cta(&d_full[I & 1], (I >> 1) & 1);
         if (!aborted) {
           tc_fence_after();
-          if (part == 0) {
-            // lane quadrant `quad` holds keys [32 quad, 32 quad + 32): part quad / 2's columns
-            float d[4];
-            tmem_ld4(lane_base + kFDCol + (I & 1) * 16 + 3 * (quad >> 1), d);
-            tmem_wait_ld();
-            reg_fence<4>(d);
-            const float val =
-                (d[0] + d[1] + d[2] * (1.f / 16777216.f)) * (1.f / 32768.f) * a.out_scale;
-            float* dst;
-            if (cur.q0 == 0 && cur.q1 == TPI) {
-              dst = a.scores + (static_cast<size_t>(cur.r) * a.Hkv + cur.g) * a.W;
-            } else {   // the head part ends this cluster's range (split cid + 1), the tail
-                       // part starts it (split cid)
-              const int side = cur.q0 == 0 ? 0 : 1;
-              const int split = side == 0 ? cid + 1 : cid;
-              dst = a.part + (static_cast<size_t>(split - 1) * 2 + side) * a.W;
-            }
-            dst[rank * kFKeys + row] = val;
+          // TMEM lane `row` of D holds key `row` of this CTA
+          float d[4];
+          tmem_ld4(lane_base + kFDCol + (I & 1) * 16, d);
+          tmem_wait_ld();
+          reg_fence<4>(d);
+          const float val =
+              (d[0] + d[1] + d[2] * (1.f / 16777216.f)) * (1.f / 32768.f) * a.out_scale;
+          float* dst;
+          if (cur.q0 == 0 && cur.q1 == TPI) {
+            dst = a.scores + (static_cast<size_t>(cur.r) * a.Hkv + cur.g) * a.W;
+          } else {   // the head part ends this cluster's range (split cid + 1), the tail
+                     // part starts it (split cid)
+            const int side = cur.q0 == 0 ? 0 : 1;
+            const int split = side == 0 ? cid + 1 : cid;
+            dst = a.part + (static_cast<size_t>(split - 1) * 2 + side) * a.W;
           }
+          dst[rank * kFKeys + row] = val;
           tc_fence_before();
           mbar_arrive(&d_empty[I & 1]);
         }
       }
-      pb += 2;
-      if (pb >= kFPBufs) { pb -= kFPBufs; ++pq; }
-      xs += 2;
+      xs += kFTeams;
       if (xs >= kFXStages) { xs -= kFXStages; ++xq; }
-      tp += 2;
+      tp += kFTeams;
       while (have && tp >= cur.q1 - cur.q0) {
         tp -= cur.q1 - cur.q0;
         ++I;
