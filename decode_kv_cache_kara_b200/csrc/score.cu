@@ -761,7 +761,7 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
 // Three teams of 4 epilogue warps take the tiles in turn, each with its own S accumulator in
 // TMEM and its own P' and weight buffers, so that a team's wait for the cluster exchange and
 // its weights overlap the other two teams' exponentials. After the item's last tile, D (times
-// 2^-15) holds the // per-key scores summed over the item's G heads.
+// 2^-15) holds the per-key scores summed over the item's G heads.
 // ----------------------------------------------------------------------------------------
 constexpr int kFTeams = 3;                        // epilogue teams, tile T goes to team T mod 3
 constexpr int kFEpiWarps = 4 * kFTeams;           // a team: one warp per TMEM lane quadrant
