@@ -1203,7 +1203,9 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
         float Lsum = 0.f;
 #pragma unroll
         for (int c = 0; c < CL; ++c) Lsum += ex2(xv[c] - M);
-        const float w = ex2(mx - M + 15.f) / Lsum;
+        float inv;   // 1 / L to about 2^-23 (rcp.approx), well inside the score tolerance
+        asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(Lsum));
+        const float w = ex2(mx - M + 15.f) * inv;
         const __half w1 = __float2half_rn(w);
         const float r1 = w - __half2float(w1);
         const __half w2 = __float2half_rn(r1);
