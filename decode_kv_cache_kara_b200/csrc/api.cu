@@ -263,30 +263,47 @@ kara_status kara_select(const float* scores, int32_t rows, int32_t window, int32
   return launch_select(scores, rows, window, k, sel, stream);
 }
 
-kara_status kara_token2chunk(const float* scores, const int32_t* sel, int32_t rows,
-                             int32_t window, int32_t k, float anchor_frac, int32_t gap_limit,
-                             int32_t widen, int32_t* keep, cudaStream_t stream) {
+kara_status kara_token2chunk_ex(const float* scores, const int32_t* sel, int32_t rows,
+                                int32_t window, int32_t k, float anchor_frac, int32_t gap_limit,
+                                int32_t widen, int32_t trim, int32_t* keep, cudaStream_t stream) {
   if (rows < 0 || window < 1 || window > KARA_MAX_WINDOW || k < 1 || k > window)
     return KARA_ERR_INVALID_ARG;
   const int num_anchors = anchors_from_frac(anchor_frac, k);
   if (num_anchors < 0 || gap_limit < 0 || widen < 0) return KARA_ERR_INVALID_ARG;
+  if (trim != KARA_TRIM_TOKEN && trim != KARA_TRIM_CHUNK) return KARA_ERR_INVALID_ARG;
   if (rows == 0) return KARA_OK;
   if (scores == nullptr || sel == nullptr || keep == nullptr) return KARA_ERR_INVALID_ARG;
   return launch_token2chunk(scores, sel, rows, window, k, num_anchors, gap_limit, widen, keep,
-                            stream);
+                            stream, trim);
+}
+
+kara_status kara_token2chunk(const float* scores, const int32_t* sel, int32_t rows,
+                             int32_t window, int32_t k, float anchor_frac, int32_t gap_limit,
+                             int32_t widen, int32_t* keep, cudaStream_t stream) {
+  return kara_token2chunk_ex(scores, sel, rows, window, k, anchor_frac, gap_limit, widen,
+                             KARA_TRIM_TOKEN, keep, stream);
+}
+
+kara_status kara_select_chunks_ex(const float* scores, int32_t rows, int32_t window, int32_t k,
+                                  float anchor_frac, int32_t gap_limit, int32_t widen,
+                                  int32_t trim, int32_t* sel, int32_t* keep,
+                                  cudaStream_t stream) {
+  if (rows < 0 || window < 1 || window > KARA_MAX_WINDOW || k < 1 || k > window)
+    return KARA_ERR_INVALID_ARG;
+  const int num_anchors = anchors_from_frac(anchor_frac, k);
+  if (num_anchors < 0 || gap_limit < 0 || widen < 0) return KARA_ERR_INVALID_ARG;
+  if (trim != KARA_TRIM_TOKEN && trim != KARA_TRIM_CHUNK) return KARA_ERR_INVALID_ARG;
+  if (rows == 0) return KARA_OK;
+  if (scores == nullptr || keep == nullptr) return KARA_ERR_INVALID_ARG;
+  return launch_select_chunks(scores, rows, window, k, num_anchors, gap_limit, widen, sel, keep,
+                              stream, trim);
 }
 
 kara_status kara_select_chunks(const float* scores, int32_t rows, int32_t window, int32_t k,
                                float anchor_frac, int32_t gap_limit, int32_t widen,
                                int32_t* sel, int32_t* keep, cudaStream_t stream) {
-  if (rows < 0 || window < 1 || window > KARA_MAX_WINDOW || k < 1 || k > window)
-    return KARA_ERR_INVALID_ARG;
-  const int num_anchors = anchors_from_frac(anchor_frac, k);
-  if (num_anchors < 0 || gap_limit < 0 || widen < 0) return KARA_ERR_INVALID_ARG;
-  if (rows == 0) return KARA_OK;
-  if (scores == nullptr || keep == nullptr) return KARA_ERR_INVALID_ARG;
-  return launch_select_chunks(scores, rows, window, k, num_anchors, gap_limit, widen, sel, keep,
-                              stream);
+  return kara_select_chunks_ex(scores, rows, window, k, anchor_frac, gap_limit, widen,
+                               KARA_TRIM_TOKEN, sel, keep, stream);
 }
 
 kara_status kara_compact(const kara_layer_kv* layers, int32_t num_layers, const kara_pool* pool,

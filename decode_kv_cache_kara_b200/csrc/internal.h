@@ -69,14 +69,14 @@ kara_status launch_select(const float* scores, int rows, int W, int k, int32_t* 
                           cudaStream_t stream);
 kara_status launch_select_chunks(const float* scores, int rows, int W, int k, int num_anchors,
                                  int gap_limit, int widen, int32_t* sel, int32_t* keep,
-                                 cudaStream_t stream);
+                                 cudaStream_t stream, int trim = KARA_TRIM_TOKEN);
 kara_status launch_sum_heads(const float* scores, int rows, int hkv, int W, float* out,
                              cudaStream_t stream);
 kara_status launch_expand_keep(const int32_t* keep_shared, int rows, int hkv, int k,
                                int32_t* keep, cudaStream_t stream);
 kara_status launch_token2chunk(const float* scores, const int32_t* sel, int rows, int W, int k,
                                int num_anchors, int gap_limit, int widen, int32_t* keep,
-                               cudaStream_t stream);
+                               cudaStream_t stream, int trim = KARA_TRIM_TOKEN);
 
 struct LayerPtrs {
   void* k[KARA_MAX_LAYERS];

@@ -33,22 +33,24 @@ select_kernel(const float* __restrict__ scores, int W, int k, int32_t* __restric
 
 __global__ void __launch_bounds__(kSelThreads)
 token2chunk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ sel, int W,
-                   int k, int num_anchors, int gap_limit, int widen, int32_t* __restrict__ keep) {
+                   int k, int num_anchors, int gap_limit, int widen, int32_t* __restrict__ keep,
+                   int trim) {
   asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
   extern __shared__ __align__(16) uint8_t smem[];
   const size_t row = blockIdx.x;
   token2chunk_row(scores + row * W, sel + row * k, nullptr, W, k, num_anchors, gap_limit, widen,
-                  keep + row * k, smem);
+                  keep + row * k, smem, trim);
 }
 
 __global__ void __launch_bounds__(kSelThreads)
 select_chunks_kernel(const float* __restrict__ scores, int32_t* __restrict__ sel, int W, int k,
-                     int num_anchors, int gap_limit, int widen, int32_t* __restrict__ keep) {
+                     int num_anchors, int gap_limit, int widen, int32_t* __restrict__ keep,
+                     int trim) {
   asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
   extern __shared__ __align__(16) uint8_t smem[];
   const size_t row = blockIdx.x;
   token2chunk_row(scores + row * W, nullptr, sel != nullptr ? sel + row * k : nullptr, W, k,
-                  num_anchors, gap_limit, widen, keep + row * k, smem);
+                  num_anchors, gap_limit, widen, keep + row * k, smem, trim);
 }
 
 
@@ -62,11 +64,16 @@ kara_status launch_select(const float* scores, int rows, int W, int k, int32_t* 
   return check_launch(__func__);
 }
 
-// Windows above about 3400 keys need more than the default 48 KB of dynamic shared memory.
+// Windows above about 3400 keys (about 1500 with the chunk-aware trim) need more than the
+// default 48 KB of dynamic shared memory.
+size_t t2c_launch_smem(int W, int trim) {
+  return t2c_smem(W) + (trim == KARA_TRIM_CHUNK ? chunk_smem(W) : 0);
+}
+
 void allow_t2c_smem() {
   static bool done = false;
   if (done) return;
-  const int bytes = static_cast<int>(t2c_smem(KARA_MAX_WINDOW));
+  const int bytes = static_cast<int>(t2c_launch_smem(KARA_MAX_WINDOW, KARA_TRIM_CHUNK));
   cudaFuncSetAttribute(token2chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   cudaFuncSetAttribute(select_chunks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   done = true;
@@ -74,21 +81,21 @@ void allow_t2c_smem() {
 
 kara_status launch_token2chunk(const float* scores, const int32_t* sel, int rows, int W, int k,
                                int num_anchors, int gap_limit, int widen, int32_t* keep,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, int trim) {
   if (rows == 0) return KARA_OK;
   allow_t2c_smem();
-  launch_pdl(token2chunk_kernel, dim3(rows), dim3(kSelThreads), t2c_smem(W), stream, scores, sel,
-             W, k, num_anchors, gap_limit, widen, keep);
+  launch_pdl(token2chunk_kernel, dim3(rows), dim3(kSelThreads), t2c_launch_smem(W, trim), stream,
+             scores, sel, W, k, num_anchors, gap_limit, widen, keep, trim);
   return check_launch(__func__);
 }
 
 kara_status launch_select_chunks(const float* scores, int rows, int W, int k, int num_anchors,
                                  int gap_limit, int widen, int32_t* sel, int32_t* keep,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, int trim) {
   if (rows == 0) return KARA_OK;
   allow_t2c_smem();
-  launch_pdl(select_chunks_kernel, dim3(rows), dim3(kSelThreads), t2c_smem(W), stream, scores,
-             sel, W, k, num_anchors, gap_limit, widen, keep);
+  launch_pdl(select_chunks_kernel, dim3(rows), dim3(kSelThreads), t2c_launch_smem(W, trim),
+             stream, scores, sel, W, k, num_anchors, gap_limit, widen, keep, trim);
   return check_launch(__func__);
 }
 

@@ -13,6 +13,10 @@
 // previous/next non-member positions by block-wide max/min scans over the window; gap fill,
 // widening, run priorities and the trim back to k follow from those per position.
 //
+// The chunk-aware trim (a variant the pages leave open) first drops whole runs of the union
+// that hold no anchor, weakest first by their best score (ties: the later run), while a whole
+// run fits in the excess; the token-level trim then takes the rest.
+//
 // Threads own contiguous chunks of positions, so every scan is one in-chunk pass plus one
 // block-level exclusive scan of chunk aggregates. Every function here is block-collective
 // over kSelThreads threads.
@@ -70,6 +74,11 @@ struct SelectSmem {
   int digit;
   int above;
 };
+
+// Bytes of token2chunk_row's base arrays (the chunk-aware trim's arrays follow them).
+__host__ __device__ constexpr size_t t2c_base_bytes(int W) {
+  return sizeof(SelectSmem) + static_cast<size_t>(W) * 14;
+}
 
 // Among positions with cand[j] != 0, sets flag[j] = 1 for the `count` largest keys (ties:
 // lower position first). Requires count <= number of candidates. Block-collective.
@@ -131,13 +140,91 @@ __device__ void block_compact_write(const uint8_t* flag, int W, int E, int32_t* 
     if (flag[j]) out[pos++] = j;
 }
 
+// Chunk-aware trim, before the token-level trim: the runs of U that hold no anchor (all their
+// members have priority 0) are dropped whole, weakest first by their best key (ties: the later
+// run first), while the whole run fits in the excess |U| - k; their members get priority -1.
+// run_s[j] is the start of the run of U around member j. Work arrays (in `cs`, chunk_smem(W)
+// bytes): rkey / rlen / rrank per run start, the run starts listed ascending, the lengths by
+// rank. Ranks are counted pairwise (O(R^2) for R unanchored runs, R <= k).
+__device__ void drop_weak_runs(const uint32_t* key, const uint8_t* in_u, int8_t* prio,
+                               const int16_t* run_s, int W, int E, int k, SelectSmem* ss,
+                               uint8_t* cs) {
+  uint32_t* rkey = reinterpret_cast<uint32_t*>(cs);
+  int* rlen = reinterpret_cast<int*>(rkey + W);
+  int* rrank = rlen + W;
+  int* bylen = rrank + W;
+  int16_t* list = reinterpret_cast<int16_t*>(bylen + W);
+  __shared__ int s_total, s_runs, s_drop;
+  const int tid = threadIdx.x;
+  const int lo = tid * E, hi = min(W, lo + E);
+  for (int j = tid; j < W; j += kSelThreads) {
+    rkey[j] = 0u;
+    rlen[j] = 0;
+  }
+  __syncthreads();
+  int members = 0, starts = 0;
+  for (int j = lo; j < hi; ++j) {
+    if (!in_u[j]) continue;
+    ++members;
+    if (prio[j] != 0) continue;
+    atomicMax(&rkey[run_s[j]], key[j]);
+    atomicAdd(&rlen[run_s[j]], 1);
+    if (run_s[j] == j) ++starts;
+  }
+  const int mem_before = block_exclusive_scan<true>(members, 0, op_add, ss->ibuf);
+  int pos = block_exclusive_scan<true>(starts, 0, op_add, ss->ibuf);
+  if (tid == kSelThreads - 1) {
+    s_total = mem_before + members;
+    s_runs = pos + starts;
+  }
+  for (int j = lo; j < hi; ++j)
+    if (in_u[j] && prio[j] == 0 && run_s[j] == j) list[pos++] = static_cast<int16_t>(j);
+  __syncthreads();
+  const int R = s_runs, excess = s_total - k;
+  // rank of each run: the number of weaker runs (smaller best key, or equal and later start)
+  for (int r = tid; r < R; r += kSelThreads) {
+    const int sr = list[r];
+    const uint32_t kr = rkey[sr];
+    int rank = 0;
+    for (int q = 0; q < R; ++q) {
+      const int sq = list[q];
+      const uint32_t kq = rkey[sq];
+      rank += (kq < kr || (kq == kr && sq > sr)) ? 1 : 0;
+    }
+    rrank[sr] = rank;
+    bylen[rank] = rlen[sr];
+  }
+  __syncthreads();
+  // the weakest runs whose lengths add up to at most the excess: ranks [0, s_drop)
+  const int ER = (R + kSelThreads - 1) / kSelThreads;
+  const int rlo = tid * ER, rhi = min(R, rlo + ER);
+  int sum = 0;
+  for (int r = rlo; r < rhi; ++r) sum += bylen[r];
+  int acc = block_exclusive_scan<true>(sum, 0, op_add, ss->ibuf);
+  int fits = 0;
+  for (int r = rlo; r < rhi; ++r) {
+    acc += bylen[r];
+    if (acc <= excess) ++fits;
+  }
+  const int fits_before = block_exclusive_scan<true>(fits, 0, op_add, ss->ibuf);
+  if (tid == kSelThreads - 1) s_drop = fits_before + fits;
+  __syncthreads();
+  const int ndrop = s_drop;
+  for (int j = lo; j < hi; ++j)
+    if (in_u[j] && prio[j] == 0 && rrank[run_s[j]] < ndrop) prio[j] = -1;
+  __syncthreads();
+}
+
 // Token2Chunk of one row (block-level): s = the row's W scores, keep = where its k kept
 // positions go (global or shared memory). The selection comes from sel_in (k positions), or,
 // when sel_in is null, is selected here first (written to sel_out unless that is null).
-// smem: t2c_smem(W) bytes of shared memory, 16-byte aligned.
+// trim: KARA_TRIM_TOKEN, or KARA_TRIM_CHUNK (whole unanchored runs dropped first).
+// smem: t2c_smem(W) bytes of shared memory, plus chunk_smem(W) more for the chunk-aware trim,
+// 16-byte aligned.
 __device__ void token2chunk_row(const float* __restrict__ s, const int32_t* sel_in,
                                 int32_t* sel_out, int W, int k, int num_anchors, int gap_limit,
-                                int widen, int32_t* keep, uint8_t* smem) {
+                                int widen, int32_t* keep, uint8_t* smem,
+                                int trim = KARA_TRIM_TOKEN) {
   const bool kSelIn = sel_in != nullptr;
   SelectSmem* ss = reinterpret_cast<SelectSmem*>(smem);
   uint32_t* key = reinterpret_cast<uint32_t*>(smem + sizeof(SelectSmem));
@@ -149,6 +236,9 @@ __device__ void token2chunk_row(const float* __restrict__ s, const int32_t* sel_
   int8_t* prio = reinterpret_cast<int8_t*>(in_u + W);
   uint8_t* cand = reinterpret_cast<uint8_t*>(prio + W);
   uint8_t* flag = cand + W;
+  // chunk-aware trim only: the start of each member's run, then the work arrays
+  int16_t* run_s = reinterpret_cast<int16_t*>(smem + ((t2c_base_bytes(W) + 15) / 16) * 16);
+  uint8_t* chunk_ws = reinterpret_cast<uint8_t*>(run_s) + ((2 * W + 15) / 16) * 16;
 
   const int32_t* sl = sel_in;
   const int tid = threadIdx.x;
@@ -223,6 +313,7 @@ __device__ void token2chunk_row(const float* __restrict__ s, const int32_t* sel_
       if (anchor[j]) prio[j] = 2;
       else if (in_u[j]) prio[j] = (prev_a[j] > last_gap) ? 1 : 0;
       else prio[j] = -1;
+      if (trim == KARA_TRIM_CHUNK) run_s[j] = static_cast<int16_t>(last_gap + 1);
     }
     int next_gap = carry_gap_next;
     for (int j = hi - 1; j >= lo; --j) {
@@ -231,6 +322,7 @@ __device__ void token2chunk_row(const float* __restrict__ s, const int32_t* sel_
     }
   }
   __syncthreads();
+  if (trim == KARA_TRIM_CHUNK) drop_weak_runs(key, in_u, prio, run_s, W, E, k, ss, chunk_ws);
 
   // f. trim to k by (priority, score, -position)
   int c1 = 0;
@@ -262,6 +354,10 @@ __host__ __device__ constexpr size_t select_smem(int W) {
 }
 __host__ __device__ constexpr size_t t2c_smem(int W) {
   return sizeof(SelectSmem) + static_cast<size_t>(W) * 14 + 64;
+}
+// The chunk-aware trim's extra shared memory: run starts (int16) and five W-long work arrays.
+__host__ __device__ constexpr size_t chunk_smem(int W) {
+  return (static_cast<size_t>(2 * W) + 15) / 16 * 16 + static_cast<size_t>(W) * 18 + 64;
 }
 
 }  // namespace

@@ -29,6 +29,7 @@ ERR_WORKSPACE = 6
 ERR_BAD_BLOCK = 7
 
 OP_SCORE, OP_COMPACT, OP_DECODE, OP_LACACHE = 1, 2, 3, 4
+TRIM_TOKEN, TRIM_CHUNK = 0, 1      # Token2Chunk's trim: token by token, or whole chunks first
 MAX_LAYERS = 128
 
 
@@ -97,6 +98,8 @@ _SIGNATURES = {
     "kara_sum_heads": ([_P, _I, _I, _I, _P, _P], _I),
     "kara_expand_keep": ([_P, _I, _I, _I, _P, _P], _I),
     "kara_select_chunks": ([_P, _I, _I, _I, _F, _I, _I, _P, _P, _P], _I),
+    "kara_select_chunks_ex": ([_P, _I, _I, _I, _F, _I, _I, _I, _P, _P, _P], _I),
+    "kara_token2chunk_ex": ([_P, _P, _I, _I, _I, _F, _I, _I, _I, _P, _P], _I),
     "kara_compress": ([_P, ctypes.POINTER(_LayerKV), _I, ctypes.POINTER(_Pool), _P, _I, _I, _I, _F,
                        _I, _I, _P, _P, _Z, _P, _P], _I),
 }
@@ -293,9 +296,10 @@ def kara_score_ex(q: torch.Tensor, k_cache: torch.Tensor, pool: PagedPool, windo
 
 def kara_select_chunks(scores: torch.Tensor, k: int, anchor_frac: float, gap_limit: int,
                        widen: int, keep: torch.Tensor | None = None,
-                       sel: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                       sel: torch.Tensor | None = None, trim: int = TRIM_TOKEN,
+                       stream=None) -> torch.Tensor:
     """kara_select + kara_token2chunk in one kernel: keep [..., k] int32 (sel, if given, gets
-    the selection)."""
+    the selection). trim=TRIM_CHUNK runs kara_select_chunks_ex with the chunk-aware trim."""
     _require(scores, torch.float32, "scores")
     w = scores.shape[-1]
     rows = scores.numel() // w if w else 0
@@ -304,9 +308,14 @@ def kara_select_chunks(scores: torch.Tensor, k: int, anchor_frac: float, gap_lim
     _require(keep, torch.int32, "keep")
     if sel is not None:
         _require(sel, torch.int32, "sel")
-    _check(lib().kara_select_chunks(_ptr(scores), rows, w, k, float(anchor_frac), gap_limit, widen,
-                                    _ptr(sel), _ptr(keep), _stream(stream)),
-           "kara_select_chunks")
+    if trim == TRIM_TOKEN:
+        _check(lib().kara_select_chunks(_ptr(scores), rows, w, k, float(anchor_frac), gap_limit,
+                                        widen, _ptr(sel), _ptr(keep), _stream(stream)),
+               "kara_select_chunks")
+    else:
+        _check(lib().kara_select_chunks_ex(_ptr(scores), rows, w, k, float(anchor_frac),
+                                           gap_limit, widen, int(trim), _ptr(sel), _ptr(keep),
+                                           _stream(stream)), "kara_select_chunks_ex")
     return keep
 
 
@@ -379,9 +388,10 @@ def kara_select(scores: torch.Tensor, k: int, sel: torch.Tensor | None = None,
 
 
 def kara_token2chunk(scores: torch.Tensor, sel: torch.Tensor, anchor_frac: float, gap_limit: int,
-                     widen: int, keep: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                     widen: int, keep: torch.Tensor | None = None, trim: int = TRIM_TOKEN,
+                     stream=None) -> torch.Tensor:
     """Token2Chunk expansion and trim with ceil(anchor_frac * k) anchors: [..., k] int32
-    ascending."""
+    ascending. trim=TRIM_CHUNK runs kara_token2chunk_ex with the chunk-aware trim."""
     _require(scores, torch.float32, "scores")
     _require(sel, torch.int32, "sel")
     w = scores.shape[-1]
@@ -390,9 +400,14 @@ def kara_token2chunk(scores: torch.Tensor, sel: torch.Tensor, anchor_frac: float
     if keep is None:
         keep = torch.empty_like(sel)
     _require(keep, torch.int32, "keep")
-    _check(lib().kara_token2chunk(_ptr(scores), _ptr(sel), rows, w, k, float(anchor_frac),
-                                  int(gap_limit), int(widen), _ptr(keep), _stream(stream)),
-           "kara_token2chunk")
+    if trim == TRIM_TOKEN:
+        _check(lib().kara_token2chunk(_ptr(scores), _ptr(sel), rows, w, k, float(anchor_frac),
+                                      int(gap_limit), int(widen), _ptr(keep), _stream(stream)),
+               "kara_token2chunk")
+    else:
+        _check(lib().kara_token2chunk_ex(_ptr(scores), _ptr(sel), rows, w, k, float(anchor_frac),
+                                         int(gap_limit), int(widen), int(trim), _ptr(keep),
+                                         _stream(stream)), "kara_token2chunk_ex")
     return keep
 
 

@@ -102,6 +102,14 @@ typedef enum kara_agg {
   KARA_AGG_MAX = 2     /* the largest probability any of those queries gives the key */
 } kara_agg;
 
+/* Trims of Token2Chunk's expanded set back to k (the pages leave the trim open): the main
+ * reading keeps the k members with the largest (priority, score, -position); the chunk-aware
+ * trim first drops whole runs of the set that hold no anchor. */
+typedef enum kara_trim {
+  KARA_TRIM_TOKEN = 0,
+  KARA_TRIM_CHUNK = 1
+} kara_trim;
+
 /* Operation ids for kara_workspace_bytes(). */
 typedef enum kara_op {
   KARA_OP_SCORE = 1,
@@ -211,6 +219,25 @@ kara_status kara_token2chunk(const float* scores, const int32_t* sel, int32_t ro
 kara_status kara_select_chunks(const float* scores, int32_t rows, int32_t window, int32_t k,
                                float anchor_frac, int32_t gap_limit, int32_t widen,
                                int32_t* sel, int32_t* keep, cudaStream_t stream);
+
+/*
+ * kara_token2chunk_ex / kara_select_chunks_ex - kara_token2chunk / kara_select_chunks with a
+ * choice of trim (kara_trim; the pages leave the trim open). KARA_TRIM_TOKEN gives the same
+ * keep sets as the calls without the suffix. KARA_TRIM_CHUNK, the chunk-aware trim, treats
+ * the runs of consecutive members of the expanded set U that hold no anchor as chunks ([GIST]
+ * section 2: a chunk has no fixed size and the span between two important points is kept
+ * whole): they are dropped whole, weakest first (a run's strength is its best score; equal
+ * strengths: the later run first), as long as the whole run fits in the excess |U| - k; at
+ * the first run that does not fit the dropping stops, and the rest of the excess is trimmed
+ * token by token as in kara_token2chunk. Other arguments and limits as the calls without the
+ * suffix; an unknown trim is KARA_ERR_INVALID_ARG.
+ */
+kara_status kara_token2chunk_ex(const float* scores, const int32_t* sel, int32_t rows,
+                                int32_t window, int32_t k, float anchor_frac, int32_t gap_limit,
+                                int32_t widen, int32_t trim, int32_t* keep, cudaStream_t stream);
+kara_status kara_select_chunks_ex(const float* scores, int32_t rows, int32_t window, int32_t k,
+                                  float anchor_frac, int32_t gap_limit, int32_t widen,
+                                  int32_t trim, int32_t* sel, int32_t* keep, cudaStream_t stream);
 
 /*
  * kara_compress - selection, Token2Chunk and compaction in two kernels (the compaction plan,

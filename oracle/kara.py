@@ -28,17 +28,18 @@ Readings taken where the pages are silent (each one is used identically by the C
 * Compaction = deterministic allocation of fresh blocks from a LIFO free list, copy of the
   first window page's prefix rows and of the kept rows, block-table rewrite, free of the old
   window blocks; see ``compact``.
-* Variants the pages leave open (``window_scores_agg``, ``shared_keep``): the mean (the sum
-  over its G * W pairs) and the max (the largest probability any query gives the key) in
-  place of the sum, and one selection per layer shared by its KV heads (selection and
-  Token2Chunk on the head-summed scores).
+* Variants the pages leave open (``window_scores_agg``, ``shared_keep``, ``trim="chunk"``):
+  the mean (the sum over its G * W pairs) and the max (the largest probability any query
+  gives the key) in place of the sum; one selection per layer shared by its KV heads
+  (selection and Token2Chunk on the head-summed scores); and a chunk-aware trim that drops
+  whole unanchored runs of the union, weakest first, before it trims single tokens.
 
 Parity pins (tests/test_oracle_kara.py): closed forms for two keys, a dominant key (catches a
 transposed sum), equal keys, GQA group mapping, scale, the W*G total, brute force by pairwise
 dominance for selection and trim, hand-worked golden cases, invariants of Token2Chunk and of
 compaction (conservation, untouched blocks); for the variants, a brute-force max with its
-bounds, closed forms, the mean against the sum, and the shared selection against the selection
-of the head sum. No function here is unpinned.
+bounds, closed forms, the mean against the sum, hand-worked golden cases of the shared
+selection and of the chunk-aware trim. No function here is unpinned.
 """
 
 from __future__ import annotations
@@ -168,7 +169,7 @@ def select_batch(scores: np.ndarray, k: int) -> np.ndarray:
 # --------------------------------------------------------------------------------------------
 
 def token2chunk_detail(scores: np.ndarray, sel: np.ndarray, num_anchors: int, gap_limit: int,
-                       widen: int) -> dict:
+                       widen: int, trim: str = "token") -> dict:
     """Token2Chunk on one window, step by step, in window coordinates.
 
     a. Anchors: the ``num_anchors`` selected positions with the largest scores (ties: lower
@@ -180,6 +181,11 @@ def token2chunk_detail(scores: np.ndarray, sel: np.ndarray, num_anchors: int, ga
     e. Priority: 2 for an anchor; 1 for a non-anchor member of U that lies in a maximal run of
        consecutive U positions containing an anchor; 0 otherwise.
     f. Keep: the k members of U with the largest (priority, score, -index), ascending.
+
+    trim="chunk" (the chunk-aware trim, a variant the pages leave open) first drops whole
+    runs of U that hold no anchor: weakest first, a run's strength being its best score (ties:
+    the later run first), as long as the whole run fits in the excess |U| - k; at the first run
+    that does not fit it stops, and the rest of the excess is trimmed as in f.
     """
     w = scores.shape[0]
     k = len(sel)
@@ -219,28 +225,54 @@ def token2chunk_detail(scores: np.ndarray, sel: np.ndarray, num_anchors: int, ga
             priority[x] = 2 if is_anchor[x] else (1 if run_has_anchor else 0)
         p = q
 
-    members = np.array(sorted(union), dtype=np.int64)
+    dropped = set()
+    if trim == "chunk":
+        runs = []                       # (best score, start, positions) of unanchored runs
+        p = 0
+        while p < w:
+            if not in_u[p]:
+                p += 1
+                continue
+            q = p
+            while q < w and in_u[q]:
+                q += 1
+            if not is_anchor[p:q].any():
+                runs.append((float(scores[p:q].max()), p, list(range(p, q))))
+            p = q
+        excess = len(union) - k
+        for best, start, pos in sorted(runs, key=lambda r: (r[0], -r[1])):
+            if len(pos) > excess:
+                break
+            dropped.update(pos)
+            excess -= len(pos)
+    elif trim != "token":
+        raise ValueError(trim)
+
+    members = np.array(sorted(union - dropped), dtype=np.int64)
     order = np.lexsort((members, -scores[members], -priority[members]))
     keep = np.sort(members[order[:k]])
     return {
         "anchors": anchors, "fill": np.array(sorted(fill), dtype=np.int64),
-        "widen": np.array(sorted(wide), dtype=np.int64), "union": members,
+        "widen": np.array(sorted(wide), dtype=np.int64),
+        "union": np.array(sorted(union), dtype=np.int64),
+        "dropped_runs": np.array(sorted(dropped), dtype=np.int64),
         "priority": priority, "keep": keep,
     }
 
 
 def token2chunk(scores: np.ndarray, sel: np.ndarray, num_anchors: int, gap_limit: int,
-                widen: int) -> np.ndarray:
+                widen: int, trim: str = "token") -> np.ndarray:
     """Kept window positions after Token2Chunk (exactly len(sel) of them, ascending)."""
-    return token2chunk_detail(scores, sel, num_anchors, gap_limit, widen)["keep"]
+    return token2chunk_detail(scores, sel, num_anchors, gap_limit, widen, trim)["keep"]
 
 
 def token2chunk_batch(scores: np.ndarray, sel: np.ndarray, num_anchors: int, gap_limit: int,
-                      widen: int) -> np.ndarray:
+                      widen: int, trim: str = "token") -> np.ndarray:
     """token2chunk over every leading index: scores [..., W], sel [..., k] -> [..., k]."""
     fs = scores.reshape(-1, scores.shape[-1])
     fk = sel.reshape(-1, sel.shape[-1])
-    out = [token2chunk(fs[i], fk[i], num_anchors, gap_limit, widen) for i in range(fs.shape[0])]
+    out = [token2chunk(fs[i], fk[i], num_anchors, gap_limit, widen, trim)
+           for i in range(fs.shape[0])]
     out = np.stack(out) if out else np.zeros((0, sel.shape[-1]))
     return out.reshape(sel.shape).astype(np.int32)
 

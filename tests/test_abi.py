@@ -33,6 +33,10 @@ def test_host_side_validation_returns_before_any_launch(lib_path):
     assert L.kara_select(null, 4, 16, 17, null, null) == K.ERR_INVALID_ARG
     assert L.kara_select(null, 4, 5000, 8, null, null) == K.ERR_INVALID_ARG
     assert L.kara_select(null, 0, 16, 4, null, null) == K.OK          # empty input
+    # an unknown trim
+    assert L.kara_token2chunk_ex(null, null, 1, 16, 4, 0.5, 8, 1, 2, null, null) == K.ERR_INVALID_ARG
+    assert L.kara_select_chunks_ex(null, 1, 16, 4, 0.5, 8, 1, -1, null, null, null) == K.ERR_INVALID_ARG
+    assert L.kara_select_chunks_ex(null, 0, 16, 4, 0.5, 8, 1, K.TRIM_CHUNK, null, null, null) == K.OK
     # anchor fractions outside [0, 1] (and NaN)
     for frac in (5.0, 1.01, -0.1, float("nan")):
         assert L.kara_token2chunk(null, null, 1, 16, 4, frac, 8, 1, null, null) == K.ERR_INVALID_ARG

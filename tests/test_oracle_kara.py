@@ -196,6 +196,46 @@ def test_token2chunk_golden_cases():
         assert det["keep"].tolist() == [int(x) for x in c["keep"]]
 
 
+def test_chunk_trim_golden_cases():
+    # hand-worked cases (tests/golden/chunk_trim_cases.txt): whole unanchored runs dropped
+    # weakest first while they fit, the stop rule, equal strengths, several runs
+    cases = load_golden("chunk_trim_cases.txt")
+    assert len(cases) >= 4
+    for c in cases:
+        scores = np.array(c["scores"])
+        sel = np.array(c["sel"], dtype=np.int64)
+        args = (scores, sel, int(c["num_anchors"][0]), int(c["gap_limit"][0]), int(c["widen"][0]))
+        det = ok.token2chunk_detail(*args, trim="chunk")
+        assert det["union"].tolist() == [int(x) for x in c["union"]]
+        assert det["dropped_runs"].tolist() == [int(x) for x in c["dropped_runs"]]
+        assert det["keep"].tolist() == [int(x) for x in c["keep"]]
+        assert ok.token2chunk(*args).tolist() == [int(x) for x in c["keep_token"]]
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_chunk_trim_invariants(seed):
+    # |keep| = k, anchors kept, keep within U, every run dropped whole is an unanchored run of
+    # U, and no kept token of an unanchored run is weaker than a dropped run's best token
+    # unless the trim fell back to tokens; with no excess both trims keep U
+    scores, sel, na, gap, wid = t2c_random_case(seed)
+    k = len(sel)
+    det = ok.token2chunk_detail(scores, sel, na, gap, wid, trim="chunk")
+    keep = set(det["keep"].tolist())
+    union = set(det["union"].tolist())
+    assert len(keep) == k and set(det["anchors"].tolist()) <= keep <= union
+    dropped = set(det["dropped_runs"].tolist())
+    assert not (dropped & keep) and not (dropped & set(det["anchors"].tolist()))
+    assert len(union) - len(dropped) >= k
+    for p in dropped:                       # dropped positions form whole runs of U
+        for q in (p - 1, p + 1):
+            if q in union:
+                assert q in dropped
+    if len(union) == k:
+        assert keep == union
+    if not dropped:
+        assert det["keep"].tolist() == ok.token2chunk(scores, sel, na, gap, wid).tolist()
+
+
 def t2c_random_case(seed):
     rng = np.random.default_rng(seed)
     w = int(rng.integers(4, 40))

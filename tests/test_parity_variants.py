@@ -143,3 +143,79 @@ def test_mean_from_the_ring_equals_mean_from_q_win_and_one_head_sums():
     torch.cuda.synchronize()
     assert torch.equal(a, b)
     assert torch.equal(one, a[:, 0])
+
+
+# ---- the chunk-aware trim (kara_token2chunk_ex / kara_select_chunks_ex, KARA_TRIM_CHUNK) ----
+
+def _golden(name):
+    from tests.test_oracle_kara import load_golden
+    return load_golden(name)
+
+
+def test_chunk_trim_golden_cases_on_the_gpu():
+    # the hand-worked cases through the kernels (fp32 scores keep the cases' orderings)
+    for c in _golden("chunk_trim_cases.txt"):
+        s = torch.tensor([c["scores"]], dtype=torch.float32, device="cuda")
+        sel = torch.tensor([[int(x) for x in c["sel"]]], dtype=torch.int32, device="cuda")
+        k = sel.shape[1]
+        frac = int(c["num_anchors"][0]) / k
+        args = (frac, int(c["gap_limit"][0]), int(c["widen"][0]))
+        keep = K.kara_token2chunk(s, sel, *args, trim=K.TRIM_CHUNK)
+        keep_tok = K.kara_token2chunk(s, sel, *args)
+        keep_fused = K.kara_select_chunks(s, k, *args, trim=K.TRIM_CHUNK)
+        torch.cuda.synchronize()
+        assert H.i32(keep[0]).tolist() == [int(x) for x in c["keep"]]
+        assert H.i32(keep_tok[0]).tolist() == [int(x) for x in c["keep_token"]]
+        assert torch.equal(keep, keep_fused)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_chunk_trim_matches_oracle(seed):
+    # coarse scores (many ties, many short runs of U), random parameters, identical inputs on
+    # both sides: identical keep sets; the fused kernel equals select then Token2Chunk
+    rng = np.random.default_rng(100 + seed)
+    rows, w = 6, int(rng.choice([64, 200, 1024, 2048]))
+    k = int(rng.integers(1, max(2, w // 3)))
+    s = (rng.integers(0, 7, size=(rows, w)).astype(np.float32) * 0.5
+         + rng.random((rows, w)).astype(np.float32) * float(seed % 2))
+    scores = torch.from_numpy(s).cuda()
+    frac = float(np.float32(rng.choice([0.1, 0.25, 0.5, 1.0])))
+    gap, wid = int(rng.integers(0, 10)), int(rng.integers(0, 3))
+    sel = K.kara_select(scores, k)
+    keep = K.kara_token2chunk(scores, sel, frac, gap, wid, trim=K.TRIM_CHUNK)
+    sel2 = torch.empty_like(sel)
+    keep2 = K.kara_select_chunks(scores, k, frac, gap, wid, sel=sel2, trim=K.TRIM_CHUNK)
+    torch.cuda.synchronize()
+    assert torch.equal(sel, sel2) and torch.equal(keep, keep2)
+    s64 = s.astype(np.float64)
+    na = ok.anchors_for(frac, k)
+    for r in range(rows):
+        ref = ok.token2chunk(s64[r], H.i32(sel[r]), na, gap, wid, trim="chunk")
+        assert np.array_equal(H.i32(keep[r]), ref), r
+
+
+def test_chunk_trim_on_window_scores_and_largest_window():
+    # real window scores of the one-layer workload's shapes, and the largest window (4096 keys,
+    # about 131 KB of shared memory with the chunk-aware trim's work arrays)
+    wl = LAYER.with_(batch=2, ctx_lo=1100, ctx_hi=1400, window=1024, keep=204)
+    cpu, dev = H.make(wl, 14)
+    pool = K.PagedPool.from_cache(dev)
+    sc = K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window)
+    keep = K.kara_select_chunks(sc, wl.keep, wl.anchor_frac, wl.gap_limit, wl.widen,
+                                trim=K.TRIM_CHUNK)
+    rng = np.random.default_rng(3)
+    big = torch.from_numpy(rng.random((2, 4096)).astype(np.float32)).cuda()
+    keep_big = K.kara_select_chunks(big, 819, 0.25, 8, 1, trim=K.TRIM_CHUNK)
+    torch.cuda.synchronize()
+    s = H.f64(sc)
+    na = ok.anchors_for(wl.anchor_frac, wl.keep)
+    for r in range(wl.batch):
+        for g in range(wl.hkv):
+            ref = ok.token2chunk(s[r, g], ok.select_topk(s[r, g], wl.keep), na, wl.gap_limit,
+                                 wl.widen, trim="chunk")
+            assert np.array_equal(H.i32(keep[r, g]), ref)
+    b64 = big.double().cpu().numpy()
+    for r in range(2):
+        ref = ok.token2chunk(b64[r], ok.select_topk(b64[r], 819), ok.anchors_for(0.25, 819), 8, 1,
+                             trim="chunk")
+        assert np.array_equal(H.i32(keep_big[r]), ref)
