@@ -562,6 +562,78 @@ def lacache_run(dev, batch: int, peaks: dict, src: str) -> dict:
                         f"passes (all layers each), 24576 tokens appended before passes 2 and 3"}
 
 
+def gqa8b_run(dev, peaks: dict, src: str, steps: int = 5, warmup: int = 3) -> dict:
+    """The 8B-GQA workload (32 query / 8 KV heads, d=128, batch 256, ragged contexts uniform in
+    [8192, 32768], W=2048, keep 409), one layer: its 32 layers' KV pools (about 690 GB) do not
+    fit on one GPU, so one layer's pool (about 21.5 GB, plus 4.3 GB of window queries) is
+    resident, the per-layer step (score, select + Token2Chunk, compaction, decode) is timed like
+    the headline step, and the 32-layer step is extrapolated as 32 x the per-layer time
+    (labelled as such). Then block free and reuse: W new tokens are appended to every sequence
+    (untimed; their pages popped from the free list, so they reuse blocks the first compaction
+    freed) and a second compression over the new window is timed."""
+    from decode_kv_cache_kara_b200 import kara as K
+    wl = synth.WORKLOADS["gqa8b"].with_(layers=1)
+    cache = synth.make_cache(wl, 1234 + 3, dev, extra_pages=wl.window // wl.page + 2)
+    work = algorithmic_work(wl, cache)
+    step = Step(cache, wl)
+    total, avg, launches, _ = time_step(step, steps, warmup)
+    per_layer = total / steps
+    kernels = kernel_entries(wl, work, avg, step, peaks, src)
+    # block free and reuse: compact once (kept), append W tokens, time the second compression
+    step.run(restore=False)
+    torch.cuda.synchronize()
+    freed_top = int(cache["free_top"][0])
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + 13)
+    pages = wl.window // wl.page
+    n = cache["ctx_len"].long()
+    first = (n + wl.page - 1) // wl.page            # first page the new tokens need
+    last = (n + wl.window + wl.page - 1) // wl.page
+    need = (last - first).cpu().tolist()
+    top = freed_top
+    table = cache["block_table"]
+    for b in range(wl.batch):                        # pages popped from the stack top, in order
+        cnt = need[b]
+        ids = cache["free_list"][top - cnt:top].flip(0)
+        table[b, int(first[b]):int(first[b]) + cnt] = ids
+        top -= cnt
+    cache["free_top"][0] = top
+    slots = n[:, None] + torch.arange(wl.window, device=dev)[None, :]
+    blk = torch.gather(table.long(), 1, slots // wl.page)
+    for pool_t in (cache["k"][0], cache["v"][0]):
+        pool_t[blk, slots % wl.page] = torch.randn((wl.batch, wl.window, wl.hkv, wl.head_dim),
+                                                   generator=gen, device=dev).to(pool_t.dtype)
+    cache["ctx_len"] += wl.window
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    K.kara_score(cache["q_win"][0], cache["k"][0], step.pool, wl.window, scores=step.scores[0],
+                 workspace=step.ws, status=step.status)
+    K.kara_select_chunks(step.scores[0], wl.keep, wl.anchor_frac, wl.gap_limit, wl.widen,
+                         keep=step.keep[0])
+    K.kara_compact(cache["k"], cache["v"], step.pool, wl.window, step.keep, workspace=step.ws,
+                   status=step.status)
+    e1.record()
+    torch.cuda.synchronize()
+    st = K.read_status(step.status)
+    tokens = wl.batch * wl.window
+    out = {"workload": "gqa8b: 8B-class GQA, 32 query / 8 KV heads, d=128, batch 256, ragged "
+                       "contexts [8192, 32768], W=2048, keep 409; one layer resident, the "
+                       "32-layer step extrapolated as 32 x the per-layer step",
+           "per_layer_ms": per_layer,
+           "step_ms_extrapolated_x32": 32 * per_layer,
+           "tokens_per_s_extrapolated": tokens / (32 * per_layer / 1e3),
+           "gpu_launches_per_layer_step": launches / steps,
+           "kernels_per_layer": kernels,
+           "second_compression_after_reuse_ms": e0.elapsed_time(e1),
+           "second_compression_status": st,
+           "note": "scoring at W=2048 takes the two-pass kernels (the fused scorer covers windows "
+                   "of up to 1024 keys); the second compression pops blocks freed by the first"}
+    del step, cache
+    torch.cuda.empty_cache()
+    return out
+
+
 def variants_run(step, reps: int = 10) -> dict:
     """The score and selection variants on the one-layer workload (its window queries and
     cache, not changed by them): kara_score_ex with the mean and with the max aggregation, and
@@ -860,6 +932,8 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
         kernels["layer"] = layer_workload_run(dev, max(3, min(args.steps, 20)), 3, peaks, src)
     if world == 1 and not args.no_lacache:
         kernels["lacache_compact"] = lacache_run(dev, args.lacache_batch, peaks, src)
+    if world == 1 and not args.no_gqa8b:
+        kernels["gqa8b"] = gqa8b_run(dev, peaks, src)
     if world == 1 and not args.no_loop:
         kernels["lacache_loop"] = lacache_loop_run(dev)
 
@@ -895,9 +969,10 @@ def cpu_baseline(seed: int, target_s: float = 15.0) -> dict:
     cores = host_cores()
     cache_cpu = oracle_sample_cache(seed)
     wl = WORKLOAD.with_(batch=4, layers=1)
-    dt, tokens = time_cpu_oracle_sample(cache_cpu, wl, units=1, seed=seed,
+    time_cpu_oracle_sample(cache_cpu, wl, units=1, seed=seed, layers_per_step=WORKLOAD.layers)
+    dt, tokens = time_cpu_oracle_sample(cache_cpu, wl, units=2, seed=seed + 7,
                                         layers_per_step=WORKLOAD.layers)
-    units = max(1, int(target_s / max(dt, 1e-3)))
+    units = max(1, int(target_s / max(dt / 2, 1e-3)))
     units = min(units, 256)
     dt, tokens = time_cpu_oracle_sample(cache_cpu, wl, units=units, seed=seed + 1,
                                         layers_per_step=WORKLOAD.layers)
@@ -955,6 +1030,8 @@ def main():
                     help="skip the decode-loop measurements (amortised schedule, LaCache loop)")
     ap.add_argument("--no-layer", action="store_true",
                     help="skip the one-layer workload and the variants")
+    ap.add_argument("--no-gqa8b", action="store_true",
+                    help="skip the 8B-GQA workload's per-layer measurement")
     ap.add_argument("--layers", type=int, default=None,
                     help="layers of the step workload (default: all 28); fewer layers keep a "
                          "profiler capture of one layer's launches small")

@@ -28,6 +28,12 @@ void count_launch(cudaError_t err) {
   if (err == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
 }
 
+int device_slot() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
 kara_status check_launch(const char* where) {
   const cudaError_t err = cudaGetLastError();
   if (err == cudaSuccess) return KARA_OK;

@@ -611,13 +611,18 @@ kara_status launch_compact(const CompactLaunch& L, cudaStream_t stream) {
     c.gap_limit = L.gap_limit;
     c.widen = L.widen;
     const size_t smem = compress_keep_off(L.W) + static_cast<size_t>(L.k) * sizeof(int32_t);
-    static bool attr = false;
-    if (!attr) {
+    static std::atomic<int> attr_done[kMaxDevices];   // per device: the limit is set
+    const int dev = device_slot();
+    if (dev < 0) {
+      set_last_error("kara_compress", "no usable current CUDA device");
+      return KARA_ERR_CUDA;
+    }
+    if (!attr_done[dev].load()) {
       const int most = static_cast<int>(compress_keep_off(KARA_MAX_WINDOW) +
                                         KARA_MAX_WINDOW * sizeof(int32_t));
       cudaFuncSetAttribute(compress_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
       cudaFuncSetAttribute(compress_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
-      attr = true;
+      attr_done[dev].store(1);
     }
     const dim3 grid(1, L.R * L.Hkv, L.L);
     if (L.D == 128) launch_pdl(compress_kernel<128>, grid, dim3(kSelThreads), smem, stream, c);
@@ -696,15 +701,14 @@ constexpr size_t kNoAllocScratchBytes = KARA_COMPACT_NOALLOC_SCRATCH_BYTES;
 // Every GPU that loads this library holds one copy of this array until the process exits.
 static __device__ __align__(256) int32_t g_compact_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
 int32_t* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device, looked up once per device
 // (in host code the array's name is only a host-side handle, not a device address).
 kara_status scratch_for_current_device(int32_t** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KARA_ERR_CUDA;
+  const int dev = device_slot();
+  if (dev < 0) return KARA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;

@@ -542,19 +542,23 @@ template <int D, int G>
 kara_status launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, void* out,
                       cudaStream_t stream) {
   constexpr size_t smem = stream_smem_bytes<D, G>();
-  static int per_sm = 0;   // resident CTAs per SM, queried once
-  if (per_sm == 0) {
+  static std::atomic<int> per_sm[kMaxDevices];   // resident CTAs per SM, queried once per device
+  const int dev = device_slot();
+  if (dev < 0) {
+    set_last_error("paged_decode_attn", "no usable current CUDA device");
+    return KARA_ERR_CUDA;
+  }
+  if (per_sm[dev].load() == 0) {
     cudaFuncSetAttribute(decode_stream_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
     int n = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_stream_kernel<D, G>, kDecThreads, smem);
-    per_sm = n > 0 ? n : 1;
+    per_sm[dev].store(n > 0 ? n : 1);
   }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
+  int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  launch_pdl(decode_stream_kernel<D, G>, dim3(per_sm * sms), dim3(kDecThreads), smem, stream, tk,
-             tv, a);
+  launch_pdl(decode_stream_kernel<D, G>, dim3(per_sm[dev].load() * sms), dim3(kDecThreads), smem,
+             stream, tk, tv, a);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.B * a.Hq);
   cfg.blockDim = dim3(32 * kCombWarps);

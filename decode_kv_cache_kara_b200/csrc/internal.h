@@ -1,6 +1,7 @@
 // Internal launch interface between the C-ABI entry points (api.cu) and the kernel files.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
@@ -12,6 +13,14 @@ namespace kara {
 
 // Counts a kernel launch call that returned cudaSuccess (kara_launch_count). Defined in api.cu.
 void count_launch(cudaError_t err);
+
+// Kernel attributes (shared-memory limits) and occupancy are set and measured per device: every
+// device holds its own instance of the library's kernels. Tables indexed by device_slot() hold
+// that per-device state for device ordinals 0 .. kMaxDevices - 1.
+constexpr int kMaxDevices = 64;
+// The current CUDA device's index into such tables, or -1 (no current device, or an ordinal of
+// kMaxDevices or more). Defined in api.cu.
+int device_slot();
 
 // Launches `kernel` as a programmatic dependent of the previous kernel in `stream`: it may
 // start while that kernel finishes, and it must execute griddepcontrol.wait (which returns once

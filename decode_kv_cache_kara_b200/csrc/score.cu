@@ -1337,13 +1337,14 @@ bool make_map(CUtensorMap* m, const void* base, const uint64_t dims[4], const ui
   return res == CUDA_SUCCESS;
 }
 
-int sm_count() {
-  static int n = 0;
+// SMs of device slot `dev` (queried once per device).
+int sm_count(int dev) {
+  static std::atomic<int> count[kMaxDevices];
+  int n = count[dev].load();
   if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (n <= 0) n = 148;
+    count[dev].store(n);
   }
   return n;
 }
@@ -1391,6 +1392,11 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   a.streamk = 0;
   a.out_scale = L.agg == KARA_AGG_MEAN ? 1.f / (static_cast<float>(a.G) * L.W) : 1.f;
   const bool agg_max = L.agg == KARA_AGG_MAX;
+  const int dev = device_slot();
+  if (dev < 0) {
+    set_last_error("kara_score", "no usable current CUDA device");
+    return KARA_ERR_CUDA;
+  }
 
 
   // Windows of 128, 256, 512 or 1024 keys: the fused single-exponential kernel on clusters of
@@ -1401,7 +1407,8 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
               : CL == 2 ? score_fused_kernel<D, 2>
               : CL == 4 ? score_fused_kernel<D, 4> : score_fused_kernel<D, 8>;
     constexpr size_t smem = FusedSmem<D>::bytes;
-    static int max_clusters[kFMaxCluster + 1] = {0};   // per cluster size, queried once
+    // per device and cluster size: resident clusters, queried once
+    static std::atomic<int> max_clusters[kMaxDevices][kFMaxCluster + 1];
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kFThreads);
     cfg.dynamicSmemBytes = smem;
@@ -1415,10 +1422,10 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (max_clusters[CL] == 0) {
+    if (max_clusters[dev][CL].load() == 0) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
-      cfg.gridDim = dim3(CL * (sm_count() / CL));
+      cfg.gridDim = dim3(CL * (sm_count(dev) / CL));
       cfg.numAttrs = 1;                    // the query sees the cluster shape only
       int n = 0;
       const cudaError_t qe = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
@@ -1427,10 +1434,11 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
         check_launch("score_fused_kernel occupancy");
         return KARA_ERR_CUDA;
       }
-      max_clusters[CL] = n;
+      max_clusters[dev][CL].store(n);
     }
     const long long items = static_cast<long long>(L.R) * L.Hkv;
-    const int ncl = static_cast<int>(std::max<long long>(1, std::min<long long>(max_clusters[CL], items)));
+    const int ncl = static_cast<int>(
+        std::max<long long>(1, std::min<long long>(max_clusters[dev][CL].load(), items)));
     // Tile-granular ranges whenever the split slots fit in the workspace (they do whenever
     // ncl <= items, which the grid guarantees; checked all the same). The ranges are then at
     // least TPI tiles long, as the kernel assumes.
@@ -1456,20 +1464,20 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
     return KARA_OK;
   }
 
-  static bool attr_set = false;
-  if (!attr_set) {
+  static std::atomic<int> attr_set[kMaxDevices];   // per device: the limits are set
+  if (!attr_set[dev].load()) {
     cudaFuncSetAttribute(score_rowstats_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(rowstats_smem<D>()));
     cudaFuncSetAttribute(score_colsum_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(colsum_smem<D>()));
     cudaFuncSetAttribute(score_colsum_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(colsum_smem<D>()));
-    attr_set = true;
+    attr_set[dev].store(1);
   }
   const int tiles1 = L.R * L.Hkv * score_chunks(L.W) * (L.Hq / L.Hkv);   // upper bound
   const int KT = ((L.W + 15 + 15) / 16 + 7) / 8;   // at most this many key tiles per (r, g)
   const int tiles2 = L.R * L.Hkv * KT;
-  const int sms = sm_count();
+  const int sms = sm_count(dev);
   launch_pdl(score_rowstats_kernel<D>, dim3(min(tiles1, sms)), dim3(kThreads), rowstats_smem<D>(),
              stream, tq1, tk, a);
   if (check_launch("score_rowstats_kernel") != KARA_OK) {

@@ -70,13 +70,15 @@ size_t t2c_launch_smem(int W, int trim) {
   return t2c_smem(W) + (trim == KARA_TRIM_CHUNK ? chunk_smem(W) : 0);
 }
 
+// Per device (every device holds its own instance of the kernels).
 void allow_t2c_smem() {
-  static bool done = false;
-  if (done) return;
+  static std::atomic<int> done[kMaxDevices];
+  const int dev = device_slot();
+  if (dev < 0 || done[dev].load()) return;   // no device: the launch reports the error
   const int bytes = static_cast<int>(t2c_launch_smem(KARA_MAX_WINDOW, KARA_TRIM_CHUNK));
   cudaFuncSetAttribute(token2chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   cudaFuncSetAttribute(select_chunks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  done = true;
+  done[dev].store(1);
 }
 
 kara_status launch_token2chunk(const float* scores, const int32_t* sel, int rows, int W, int k,

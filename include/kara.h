@@ -19,10 +19,9 @@
  *    kara_workspace_bytes(), 256-byte aligned).
  *  - Every call is asynchronous on `stream` (a cudaStream_t; 0 = legacy default stream) and
  *    returns after enqueueing its kernels, on the current CUDA device.
- *  - One GPU per process (the model the multi-GPU benchmark follows): the library sets its
- *    kernels' shared-memory limits and measures cluster occupancy once per process, on the
- *    first device it launches on. A process that then launches on another device gets
- *    KARA_ERR_CUDA from the calls whose kernels need more than 48 KB of shared memory.
+ *  - Calls run on the current CUDA device. The library sets its kernels' shared-memory limits
+ *    and measures their occupancy once per device, the first time a call runs there; devices
+ *    with ordinals 0 .. 63 are supported (a higher ordinal gives KARA_ERR_CUDA).
  *  - The return value reports what the host can check: argument shapes, alignment (16-byte
  *    aligned tensors), supported sizes, workspace size, and CUDA launch errors
  *    (KARA_ERR_CUDA). On any non-OK return nothing was enqueued.

@@ -105,3 +105,79 @@ def test_config_path_sampled(name):
     ref = od.decode_attention(H.f64(cache["q_dec"]), H.f64(cache["k"][0]), H.f64(cache["v"][0]),
                               bt, cl, scale, wl.page)
     assert np.allclose(H.f64(out), ref, atol=2e-2, rtol=1e-2)
+
+
+def test_gqa8b_free_and_reuse():
+    # The 8B-GQA workload's shapes (32 q / 8 kv heads, ragged 8K-32K contexts, W=2048, keep
+    # 409; 3 sequences, 1 layer): a compaction, then W new tokens per sequence whose pages come
+    # from the free list top (so they reuse blocks the first compaction freed), then a second
+    # compaction over the new window. Both bit-exact against the oracle.
+    wl = synth.WORKLOADS["gqa8b"].with_(batch=3, layers=1)
+    cpu = synth.make_cache(wl, 1234 + 3, "cpu", with_queries=False,
+                           extra_pages=wl.window // 16 + 2)
+    dev = H.to_device(cpu)
+    pool = K.PagedPool.from_cache(dev)
+    rng = np.random.default_rng(21)
+    ids = list(range(wl.batch))
+
+    def compact_both(state, keep):
+        ref = ok.compact([H.bits(state["k"][0])], [H.bits(state["v"][0])],
+                         H.i32(state["block_table"]), H.i32(state["ctx_len"]),
+                         H.i32(state["free_list"]), int(state["free_top"][0]), ids, wl.window,
+                         keep, wl.page)
+        st = K.kara_compact(dev["k"], dev["v"], pool, wl.window, torch.from_numpy(keep).cuda())
+        torch.cuda.synchronize()
+        assert K.read_status(st) == 0 and ref[0] == ok.OK
+        _, kp, vp, bt, cl, fl, top, fresh = ref
+        assert np.array_equal(H.i32(dev["block_table"]), bt)
+        assert np.array_equal(H.i32(dev["ctx_len"]), cl)
+        assert int(dev["free_top"][0]) == top
+        assert np.array_equal(H.i32(dev["free_list"])[:top], fl[:top])
+        kg, vg = H.bits(dev["k"][0]), H.bits(dev["v"][0])
+        for b in ids:
+            n = int(cl[b])
+            assert np.array_equal(H.logical_rows(kg, bt[b], n), H.logical_rows(kp[0], bt[b], n))
+            assert np.array_equal(H.logical_rows(vg, bt[b], n), H.logical_rows(vp[0], bt[b], n))
+        return kp, vp, bt, cl, fl, top, fresh
+
+    keep1 = synth.random_keep(rng, wl.batch * wl.hkv, wl.window, wl.keep).reshape(
+        1, wl.batch, wl.hkv, wl.keep)
+    kp, vp, bt, cl, fl, top, _ = compact_both(cpu, keep1)
+    old = H.i32(cpu["block_table"])
+    freed = set(old[old >= 0].tolist()) - set(bt[bt >= 0].tolist())
+    assert len(freed) >= wl.batch * (wl.window // 16)
+
+    # W new tokens per sequence: pages popped from the free list top (sequence order), their
+    # K/V rows drawn from N(0, 1); the same on the host state and on the device
+    bt, cl, fl = bt.copy(), cl.copy(), fl.copy()
+    kp0, vp0 = kp[0].copy(), vp[0].copy()
+    popped = []
+    for b in ids:
+        n = int(cl[b])
+        for p in range((n + 15) // 16, (n + wl.window + 15) // 16):
+            top -= 1
+            bt[b, p] = fl[top]
+            popped.append(int(fl[top]))
+        slots = np.arange(n, n + wl.window)
+        rows = rng.standard_normal((2, wl.window, wl.hkv, wl.head_dim)).astype(np.float32)
+        kb = torch.from_numpy(rows[0]).to(torch.bfloat16).view(torch.int16).numpy()
+        vb = torch.from_numpy(rows[1]).to(torch.bfloat16).view(torch.int16).numpy()
+        kp0[bt[b][slots // 16], slots % 16] = kb
+        vp0[bt[b][slots // 16], slots % 16] = vb
+        cl[b] = n + wl.window
+    assert set(popped) & freed                      # the new pages reuse freed blocks
+    state2 = {"k": [torch.from_numpy(kp0).view(torch.bfloat16)],
+              "v": [torch.from_numpy(vp0).view(torch.bfloat16)],
+              "block_table": torch.from_numpy(bt.astype(np.int32)),
+              "ctx_len": torch.from_numpy(cl.astype(np.int32)),
+              "free_list": torch.from_numpy(fl.astype(np.int32)),
+              "free_top": torch.tensor([top], dtype=torch.int32)}
+    for key in ("block_table", "ctx_len", "free_list", "free_top"):
+        dev[key].copy_(state2[key].cuda())
+    dev["k"][0].copy_(state2["k"][0].cuda())
+    dev["v"][0].copy_(state2["v"][0].cuda())
+    keep2 = synth.random_keep(rng, wl.batch * wl.hkv, wl.window, wl.keep).reshape(
+        1, wl.batch, wl.hkv, wl.keep)
+    _, _, bt2, _, _, _, fresh2 = compact_both(state2, keep2)
+    reused = set(x for ids_ in fresh2.values() for x in ids_) & freed
+    assert reused                                    # the second compaction pops freed blocks too
