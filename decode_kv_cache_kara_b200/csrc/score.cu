@@ -773,9 +773,11 @@ constexpr int kFEpiThreads = 32 * kFEpiWarps;
 constexpr int kFKeys = 128;            // window keys owned per CTA
 constexpr int kFKRows = 144;           // key rows loaded per CTA (9 pages)
 constexpr int kFQRows = 128;           // queries per tile
-constexpr int kFMaxCluster = 8;
+constexpr int kFMaxCluster = 16;      // W = 2048: a non-portable cluster of 16 CTAs
 constexpr int kFPBufs = kFTeams;       // S, P' and weight buffers, tile T in buffer T mod 3
-constexpr int kFQSlots = 3;            // query ring slots of one 64-channel chunk each
+// query ring slots of one 64-channel chunk each: three, or two for a cluster of 16 (whose
+// exchange records need the room)
+__host__ __device__ constexpr int fq_slots(int CL) { return CL > 8 ? 2 : 3; }
 constexpr int kFXStages = 6;           // exchange slots: a peer sends its record of tile T + 6
                                        // only after its weights of tile T + 3, which need this
                                        // CTA's record of tile T + 3, which the team of tile T
@@ -824,7 +826,7 @@ struct SegCursor {
   }
 };
 
-template <int D>
+template <int D, int CL>
 struct FusedSmem {
   static constexpr int NCH = D / 64;
   static constexpr uint32_t kKChunk = kFKRows * kRowBytes;     // one 64-channel chunk of K
@@ -833,14 +835,15 @@ struct FusedSmem {
   static constexpr uint32_t kPAtom = 64 * kFQRows * 2;         // 64 keys x 128 queries, fp16
   static constexpr uint32_t kPBytes = 2 * kPAtom;
   static constexpr uint32_t kWBytes = 2 * 16 * kRowBytes;      // [k chunk][16 n rows][128 B]
-  static constexpr uint32_t kXBytes = kFXStages * kFMaxCluster * kFQRows * 4;
+  static constexpr int kQSlots = fq_slots(CL);
+  static constexpr uint32_t kXBytes = kFXStages * CL * kFQRows * 4;   // [stage][rank][row]
   static constexpr uint32_t k_off = 0;
   static constexpr uint32_t q_off = k_off + kKBytes;            // [slot] one chunk each
-  static constexpr uint32_t p_off = q_off + kFQSlots * kQChunk;
+  static constexpr uint32_t p_off = q_off + kQSlots * kQChunk;
   static constexpr uint32_t w_off = p_off + kFPBufs * kPBytes;
   static constexpr uint32_t x_off = w_off + kFPBufs * kWBytes;
   static constexpr uint32_t bar_off = x_off + kXBytes;
-  static constexpr uint32_t kBars = 2 + 2 * kFQSlots + 2 * kFTeams + 3 * kFPBufs + 2 * 2 + kFXStages;
+  static constexpr uint32_t kBars = 2 + 2 * kQSlots + 2 * kFTeams + 3 * kFPBufs + 2 * 2 + kFXStages;
   static constexpr uint32_t end = bar_off + kBars * 8 + 16;
   static constexpr size_t bytes = 1024 + end;
   static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
@@ -857,7 +860,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
 score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
-  using L = FusedSmem<D>;
+  using L = FusedSmem<D, CL>;
+  constexpr int kFQSlots = L::kQSlots;
   constexpr int NCH = L::NCH;
   constexpr uint32_t kPageBytes = 16 * kRowBytes;
 
@@ -1184,7 +1188,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       if ((e & 3) == 0 && lane == 0) mbar_expect_tx(&x_full[xs], CL * kFQRows * 4);
       if (!aborted) {
         const float lse = mx + lg2(l);
-        const uint32_t slot = x_buf_u32 + ((xs * kFMaxCluster + rank) * kFQRows + row) * 4;
+        const uint32_t slot = x_buf_u32 + ((xs * CL + rank) * kFQRows + row) * 4;
         const uint32_t xb = x_full_u32 + xs * 8;
 #pragma unroll
         for (int c = 0; c < CL; ++c) st_async_f32(map_to_rank(slot, c), lse, map_to_rank(xb, c));
@@ -1193,7 +1197,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       // fp16 columns of the B operand
       wait_cluster(&x_full[xs], xq & 1);
       if (!aborted) {
-        const float* xr = x_buf + xs * kFMaxCluster * kFQRows + row;
+        const float* xr = x_buf + xs * CL * kFQRows + row;
         float xv[CL];
 #pragma unroll
         for (int c = 0; c < CL; ++c) xv[c] = xr[c * kFQRows];
@@ -1399,16 +1403,23 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   }
 
 
-  // Windows of 128, 256, 512 or 1024 keys: the fused single-exponential kernel on clusters of
-  // W / 128 CTAs (sum and mean; the max aggregation takes the two-pass path).
-  if (!agg_max && (L.W == 128 || L.W == 256 || L.W == 512 || L.W == 1024)) {
+  // Windows of 128, 256, 512, 1024 or 2048 keys: the fused single-exponential kernel on
+  // clusters of W / 128 CTAs (sum and mean; the max aggregation takes the two-pass path). A
+  // cluster of 16 is non-portable: where the device cannot hold one, W = 2048 takes the
+  // two-pass path too.
+  // per device and cluster size: resident clusters, queried once (-1: none fits)
+  static std::atomic<int> max_clusters[kMaxDevices][kFMaxCluster + 1];
+  const bool fused_window = L.W == 128 || L.W == 256 || L.W == 512 || L.W == 1024 || L.W == 2048;
+  if (!agg_max && fused_window && max_clusters[dev][L.W / kFKeys].load() >= 0) {
     const int CL = L.W / kFKeys;
     auto kern = CL == 1 ? score_fused_kernel<D, 1>
               : CL == 2 ? score_fused_kernel<D, 2>
-              : CL == 4 ? score_fused_kernel<D, 4> : score_fused_kernel<D, 8>;
-    constexpr size_t smem = FusedSmem<D>::bytes;
-    // per device and cluster size: resident clusters, queried once
-    static std::atomic<int> max_clusters[kMaxDevices][kFMaxCluster + 1];
+              : CL == 4 ? score_fused_kernel<D, 4>
+              : CL == 8 ? score_fused_kernel<D, 8> : score_fused_kernel<D, 16>;
+    const size_t smem = CL == 1 ? FusedSmem<D, 1>::bytes
+                      : CL == 2 ? FusedSmem<D, 2>::bytes
+                      : CL == 4 ? FusedSmem<D, 4>::bytes
+                      : CL == 8 ? FusedSmem<D, 8>::bytes : FusedSmem<D, 16>::bytes;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kFThreads);
     cfg.dynamicSmemBytes = smem;
@@ -1425,43 +1436,50 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
     if (max_clusters[dev][CL].load() == 0) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
+      if (CL > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       cfg.gridDim = dim3(CL * (sm_count(dev) / CL));
       cfg.numAttrs = 1;                    // the query sees the cluster shape only
       int n = 0;
       const cudaError_t qe = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
       cfg.numAttrs = 2;
       if (qe != cudaSuccess || n <= 0) {
-        check_launch("score_fused_kernel occupancy");
-        return KARA_ERR_CUDA;
+        if (CL <= 8) {
+          check_launch("score_fused_kernel occupancy");
+          return KARA_ERR_CUDA;
+        }
+        cudaGetLastError();                // no cluster of 16 fits: the two-pass path below
+        n = -1;
       }
       max_clusters[dev][CL].store(n);
     }
-    const long long items = static_cast<long long>(L.R) * L.Hkv;
-    const int ncl = static_cast<int>(
-        std::max<long long>(1, std::min<long long>(max_clusters[dev][CL].load(), items)));
-    // Tile-granular ranges whenever the split slots fit in the workspace (they do whenever
-    // ncl <= items, which the grid guarantees; checked all the same). The ranges are then at
-    // least TPI tiles long, as the kernel assumes.
-    const int TPI = a.G * CL;
-    const long long ntiles = items * TPI;
-    const size_t part_bytes = static_cast<size_t>(ncl - 1) * 2 * L.W * sizeof(float);
-    a.part = L.lse;
-    a.streamk = ncl > 1 && ntiles / ncl >= TPI &&
-                part_bytes <= score_workspace_bytes(L.R, L.W, L.Hq);
-    bool any_split = false;
-    for (int k = 1; a.streamk && k < ncl && !any_split; ++k)
-      any_split = (k * ntiles / ncl) % TPI != 0;
-    cfg.gridDim = dim3(ncl * CL);
-    count_launch(cudaLaunchKernelEx(&cfg, kern, tq1, tk, a));
-    if (check_launch("score_fused_kernel") != KARA_OK) {
-      describe_kernel("score_fused_kernel", reinterpret_cast<const void*>(kern), kFThreads, smem);
-      return KARA_ERR_CUDA;
+    if (max_clusters[dev][CL].load() > 0) {
+      const long long items = static_cast<long long>(L.R) * L.Hkv;
+      const int ncl = static_cast<int>(
+          std::max<long long>(1, std::min<long long>(max_clusters[dev][CL].load(), items)));
+      // Tile-granular ranges whenever the split slots fit in the workspace (they do whenever
+      // ncl <= items, which the grid guarantees; checked all the same). The ranges are then at
+      // least TPI tiles long, as the kernel assumes.
+      const int TPI = a.G * CL;
+      const long long ntiles = items * TPI;
+      const size_t part_bytes = static_cast<size_t>(ncl - 1) * 2 * L.W * sizeof(float);
+      a.part = L.lse;
+      a.streamk = ncl > 1 && ntiles / ncl >= TPI &&
+                  part_bytes <= score_workspace_bytes(L.R, L.W, L.Hq);
+      bool any_split = false;
+      for (int k = 1; a.streamk && k < ncl && !any_split; ++k)
+        any_split = (k * ntiles / ncl) % TPI != 0;
+      cfg.gridDim = dim3(ncl * CL);
+      count_launch(cudaLaunchKernelEx(&cfg, kern, tq1, tk, a));
+      if (check_launch("score_fused_kernel") != KARA_OK) {
+        describe_kernel("score_fused_kernel", reinterpret_cast<const void*>(kern), kFThreads, smem);
+        return KARA_ERR_CUDA;
+      }
+      if (any_split) {
+        launch_pdl(score_split_sum_kernel, dim3(ncl - 1), dim3(256), 0, stream, a, ncl, TPI);
+        if (check_launch("score_split_sum_kernel") != KARA_OK) return KARA_ERR_CUDA;
+      }
+      return KARA_OK;
     }
-    if (any_split) {
-      launch_pdl(score_split_sum_kernel, dim3(ncl - 1), dim3(256), 0, stream, a, ncl, TPI);
-      if (check_launch("score_split_sum_kernel") != KARA_OK) return KARA_ERR_CUDA;
-    }
-    return KARA_OK;
   }
 
   static std::atomic<int> attr_set[kMaxDevices];   // per device: the limits are set

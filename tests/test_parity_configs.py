@@ -2,10 +2,10 @@
 
 Every per-sequence size is the workload's own; only the batch and the layer count are cut so
 that the oracle can check the results:
-- step: 28 q / 4 kv heads, d=128, ragged contexts 2K-16K, W=1024 (fused cluster scorer),
-  keep 204, Token2Chunk anchors 50 % / gap 8 / widen 1; 5 sequences, 3 layers;
-- gqa8b: 32 q / 8 kv heads, d=128, ragged contexts 8K-32K, W=2048 (two-pass scorer),
-  keep 409; 3 sequences, 2 layers.
+- step: 28 q / 4 kv heads, d=128, ragged contexts 2K-16K, W=1024 (fused scorer on clusters of
+  8), keep 204, Token2Chunk anchors 50 % / gap 8 / widen 1; 5 sequences, 3 layers;
+- gqa8b: 32 q / 8 kv heads, d=128, ragged contexts 8K-32K, W=2048 (fused scorer on clusters of
+  16), keep 409; 3 sequences, 2 layers.
 Each layer is scored, selected and expanded, all layers are compacted in one call, and layer
 0 of the compacted cache is decoded. Checks: sampled score rows against the oracle, select and
 Token2Chunk exactly on those rows, compaction bit-exact on every layer and sequence, decode on
@@ -50,7 +50,11 @@ def test_config_path_sampled(name):
     keep = torch.empty((wl.layers, wl.batch, wl.hkv, wl.keep), dtype=torch.int32, device="cuda")
     scores, sels = [], []
     for layer in range(wl.layers):
+        n0 = K.kara_launch_count()
         sc = K.kara_score(cache["q_win"][layer], cache["k"][layer], pool, wl.window, status=status)
+        # the fused kernel (and the split-item sum when a cluster's range ends inside an item);
+        # the two-pass path takes three launches
+        assert K.kara_launch_count() - n0 <= 2
         sel = K.kara_select(sc, wl.keep)
         K.kara_token2chunk(sc, sel, na, wl.gap_limit, wl.widen, keep=keep[layer])
         scores.append(sc)

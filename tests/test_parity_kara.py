@@ -46,6 +46,15 @@ SCORE_CASES = {
     "w256_split_items": synth.Workload("w256_split", batch=24, layers=1, hq=8, hkv=4,
                                        head_dim=128, ctx_lo=260, ctx_hi=420, window=256, keep=51,
                                        heavy_frac=0.05, spare_blocks=8),
+    # W = 2048: clusters of 16 CTAs (non-portable size); whole items per cluster, then more
+    # items than resident clusters of 16 (at most 148 / 16 of them)
+    "g4_w2048_ragged": synth.Workload("g4_w2048", batch=3, layers=1, hq=8, hkv=2, head_dim=128,
+                                      ctx_lo=2050, ctx_hi=2900, window=2048, keep=409,
+                                      heavy_frac=0.03, run_hi=16, spare_blocks=8),
+    "w2048_split_items": synth.Workload("w2048_split", batch=8, layers=1, hq=4, hkv=2,
+                                        head_dim=128, ctx_lo=2048, ctx_hi=2400, window=2048,
+                                        keep=409, heavy_frac=0.05, q_mode="neighbour",
+                                        spare_blocks=8),
 }
 
 
@@ -121,7 +130,8 @@ def test_score_split_items_skip_short_contexts():
     H.assert_scores_close(H.f64(scores[good]), oracle_scores(cpu, wl, good))
 
 
-@pytest.mark.parametrize("name,launches", [("g7_w1024_unaligned", 1), ("w128_split_items", 2)])
+@pytest.mark.parametrize("name,launches", [("g7_w1024_unaligned", 1), ("w128_split_items", 2),
+                                           ("g4_w2048_ragged", 1), ("w2048_split_items", 2)])
 def test_score_launch_count(name, launches):
     """The fused kernel alone when every cluster range holds whole items; with the split sum
     when more items than resident clusters make ranges end inside items."""
