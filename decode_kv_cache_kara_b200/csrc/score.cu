@@ -778,6 +778,9 @@ constexpr int kFPBufs = kFTeams;       // S, P' and weight buffers, tile T in bu
 // query ring slots of one 64-channel chunk each: three, or two for a cluster of 16 (whose
 // exchange records need the room)
 __host__ __device__ constexpr int fq_slots(int CL) { return CL > 8 ? 2 : 3; }
+// query tiles between a tile's L2 prefetch and its load; only a ring of two slots (a cluster
+// of 16) gains from it, three slots already cover the load latency
+__host__ __device__ constexpr int fq_ahead(int CL) { return fq_slots(CL) < 3 ? 2 : 0; }
 constexpr int kFXStages = 6;           // exchange slots: a peer sends its record of tile T + 6
                                        // only after its weights of tile T + 3, which need this
                                        // CTA's record of tile T + 3, which the team of tile T
@@ -988,6 +991,15 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (lane == 0) {
         for (int tq = q0; tq < q1 && !stop; ++tq) {
           const int h = gi * a.G + tq / CL, qt = tq % CL;
+          // L2 prefetch of the query tile fq_ahead(CL) tiles on (the CTAs of the cluster take
+          // turns; the others' loads of it then hit L2)
+          const int tp = tq + fq_ahead(CL);
+          if (fq_ahead(CL) > 0 && tp < q1 && tq % CL == static_cast<int>(rank)) {
+            const int hp = gi * a.G + tp / CL, qp = tp % CL;
+            for (int ch = 0; ch < NCH; ++ch)
+              tma_prefetch_l2_4d(&tm_q, ch * 64, hp, q_tile_row(a, si, qp * kFQRows),
+                                 q_tile_batch(a, si, r));
+          }
           for (int ch = 0; ch < NCH; ++ch) {   // chunk C of the ring: slot C mod 3
             const int slot = C % kFQSlots;
             if (!mbar_wait(&q_empty[slot], ((C / kFQSlots) & 1) ^ 1, abort_flag, a.status)) {
