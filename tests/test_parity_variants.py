@@ -24,6 +24,10 @@ LAYER = synth.WORKLOADS["layer"]
 CASES = {
     "w512_fused": LAYER.with_(batch=3, ctx_lo=520, ctx_hi=900, window=512, keep=102),
     "w200_twopass": LAYER.with_(batch=3, ctx_lo=300, ctx_hi=700, window=200, keep=40),
+    # clusters of 16 CTAs (mean) and the two-pass kernels (max) at the largest fused window
+    "w2048_fused": synth.Workload("w2048", batch=2, layers=1, hq=8, hkv=2, head_dim=128,
+                                  ctx_lo=2050, ctx_hi=2600, window=2048, keep=409,
+                                  heavy_frac=0.03, spare_blocks=8),
 }
 AGGS = {"mean": K.AGG_MEAN, "max": K.AGG_MAX}
 
@@ -127,8 +131,9 @@ def test_shared_selection_across_kv_heads():
             assert np.array_equal(H.logical_rows(vg, bt[b], n), H.logical_rows(vpo[layer], bt[b], n))
 
 
-def test_mean_from_the_ring_equals_mean_from_q_win_and_one_head_sums():
-    wl = CASES["w512_fused"]
+@pytest.mark.parametrize("name", ["w512_fused", "w2048_fused"])
+def test_mean_from_the_ring_equals_mean_from_q_win_and_one_head_sums(name):
+    wl = CASES[name]
     cpu, dev = H.make(wl, 14)
     pool = K.PagedPool.from_cache(dev)
     W = wl.window
