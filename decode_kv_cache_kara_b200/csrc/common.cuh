@@ -195,6 +195,25 @@ __device__ __forceinline__ void reg_fence(float* v) {
 }
 
 // 16 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
+// One column of 32 lanes (one value per thread of the warp) into tensor memory; the stores
+// are complete after tmem_wait_st.
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float x) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr),
+               "r"(__float_as_uint(x))
+               : "memory");
+}
+// The same value into 16 consecutive columns (column address a multiple of 16).
+__device__ __forceinline__ void tmem_st16_fill(uint32_t taddr, float x) {
+  const uint32_t r = __float_as_uint(x);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
+      "r"(r)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   uint32_t r[16];
   asm volatile(

@@ -739,12 +739,14 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
 }
 
 // ----------------------------------------------------------------------------------------
-// Fused scoring: one exponential per score, on a cluster of CL = W / 128 CTAs.
+// Fused scoring: one exponential per score, on a cluster of CL = ceil(W / 128) CTAs (W <= 1024,
+// or W = 2048 on 16).
 //
 // Work items are (r, g): the G query heads of KV head g of a valid sequence r against the
-// window keys of that KV head (G * W / 128 query tiles); all CTAs of a cluster take the same
-// items, CTA `rank` owns the 128 window keys [start + 128 rank, start + 128 rank + 128). Per
-// 128-query tile each CTA
+// window keys of that KV head (G * ceil(W / 128) query tiles); all CTAs of a cluster take the
+// same items, CTA `rank` owns the window keys [start + 128 rank, start + 128 rank + 128) that
+// exist (a window that is not a multiple of 128 leaves the last CTA fewer; its other S columns
+// are set to -inf in tensor memory, so that they count nowhere). Per 128-query tile each CTA
 //   1. computes S = Q K^T over its keys (UMMA M = 128 queries, N = 144 key rows: the 9 pages
 //      that cover its 128 keys at any slot offset; only the owned columns are read);
 //   2. in the epilogue (4 warps, one per TMEM lane quadrant: a thread owns one query row and
@@ -788,8 +790,9 @@ constexpr int kFXStages = 6;           // exchange slots: a peer sends its recor
 constexpr uint32_t kFSCols = kFKRows;  // TMEM column stride of the three S buffers: 0, 144, 288
 constexpr uint32_t kFDCol = kFTeams * kFSCols;   // TMEM columns of the two D buffers: 432, 448
 
-// Work items (r, g): KV head g of sequence r with all G of its query heads, TPI = G * W / 128
-// query tiles (tile tq: head g * G + tq / CL, queries 128 (tq % CL) ..). Cluster c of ncl takes
+// Work items (r, g): KV head g of sequence r with all G of its query heads, TPI = G * CL query
+// tiles (tile tq: head g * G + tq / CL, queries 128 (tq % CL) ..; rows past W weigh nothing).
+// Cluster c of ncl takes
 // a contiguous range of the sequence of (item, tile) pairs, items in order:
 //  - streamk: tiles [c N / ncl, (c + 1) N / ncl) of N = R * Hkv * TPI, so every cluster has the
 //    same share within a tile. A boundary inside an item splits it into a head part (ending
@@ -858,7 +861,7 @@ __device__ __forceinline__ uint32_t w_offset(int n, int k) {
                                (k & 7) * 2);
 }
 
-template <int D, int CL>
+template <int D, int CL, bool PARTIAL>
 __global__ void __launch_bounds__(kFThreads, 1)
 score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
@@ -897,6 +900,12 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t rank = cluster_ctarank();
   const int cid = static_cast<int>(cluster_id_x());
   const int ncl = static_cast<int>(cluster_count_x());
+  // query tiles per head: CL = ceil(W / 128) (a cluster of 16 serves W = 2048 only); this
+  // CTA's window keys: 128, fewer in the last CTA when W is not a multiple of 128 (PARTIAL,
+  // an instantiation of its own so that the other windows' code stays as it is)
+  constexpr int QT = CL;
+  const int TPI = a.G * QT;
+  const int kcount = PARTIAL ? min(kFKeys, a.W - static_cast<int>(rank) * kFKeys) : kFKeys;
 
   if (threadIdx.x == 0) {
     mbar_init(k_full, 1);
@@ -956,14 +965,13 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
     }
-    const int TPI = a.G * CL;
     SegCursor cur;
     cur.init(a, cid, ncl, TPI);
     int C = 0;   // query chunks issued
     bool have = cur.next(a, TPI);
     auto page_ids = [&](const SeqInfo& s, int& npg) {
       const int key0 = s.start + static_cast<int>(rank) * kFKeys;
-      npg = (key0 % 16) != 0 ? 9 : 8;
+      npg = kcount <= 0 ? 0 : (key0 + kcount - 1) / 16 - key0 / 16 + 1;   // 8 or 9 when full
       return lane < npg ? page_block(a, s.b, key0 / 16 + lane) : 0;
     };
     int npg = 0;
@@ -990,12 +998,12 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       bool stop = false;
       if (lane == 0) {
         for (int tq = q0; tq < q1 && !stop; ++tq) {
-          const int h = gi * a.G + tq / CL, qt = tq % CL;
+          const int h = gi * a.G + tq / QT, qt = tq % QT;
           // L2 prefetch of the query tile fq_ahead(CL) tiles on (the CTAs of the cluster take
           // turns; the others' loads of it then hit L2)
           const int tp = tq + fq_ahead(CL);
           if (fq_ahead(CL) > 0 && tp < q1 && tq % CL == static_cast<int>(rank)) {
-            const int hp = gi * a.G + tp / CL, qp = tp % CL;
+            const int hp = gi * a.G + tp / QT, qp = tp % QT;
             for (int ch = 0; ch < NCH; ++ch)
               tma_prefetch_l2_4d(&tm_q, ch * 64, hp, q_tile_row(a, si, qp * kFQRows),
                                  q_tile_batch(a, si, r));
@@ -1020,7 +1028,6 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     // ---- UMMA issuer for S: runs ahead of the epilogue by one tile ----
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, kFKRows);
-      const int TPI = a.G * CL;
       SegCursor cur;
       cur.init(a, cid, ncl, TPI);
       int T = 0, I = 0, C = 0;   // tiles, segments, query chunks
@@ -1056,7 +1063,6 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     // ---- UMMA issuer for the column sums: D += P'^T W, tile by tile ----
     if (lane == 0) {
       const uint32_t idesc_c = idesc_f16_f32(128, 16, true);
-      const int TPI = a.G * CL;
       SegCursor cur;
       cur.init(a, cid, ncl, TPI);
       int Tc = 0, Ic = 0;
@@ -1111,7 +1117,6 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       const bool ok = aborted ? false : mbar_wait_cluster(bar, parity, abort_flag, a.status);
       aborted = __any_sync(0xffffffffu, !ok) != 0;
     };
-    const int TPI = a.G * CL;
     SegCursor cur;
     cur.init(a, cid, ncl, TPI);
     int I = 0, tp = team;                 // segment index and tile within the segment (no
@@ -1136,6 +1141,19 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
       float mx = 0.f, l = 0.f;
       if (!aborted) {
         tc_fence_after();
+        if (PARTIAL && kcount < kFKeys) {
+          // keys past the window (the last CTA of a window that is not a multiple of 128):
+          // their S columns become -inf, so that they set no row max and give P' = 0. Single
+          // columns up to a multiple of 16, then 16 at a time (past column 128 + offset lie
+          // columns the passes do not read).
+          uint32_t c = scol + kcount;
+          const uint32_t c_end = scol + kFKeys;
+#pragma unroll 1
+          for (; (c & 15u) != 0 && c < c_end; ++c) tmem_st1(c, -INFINITY);
+#pragma unroll 1
+          for (; c < c_end; c += 16) tmem_st16_fill(c, -INFINITY);
+          tmem_wait_st();
+        }
         float v[32];
         float mm = -INFINITY;
 #pragma unroll
@@ -1152,7 +1170,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
           const float m2 = fmax3(mq[6], mq[7], mq[8]), m3 = fmax3(mq[9], mq[10], mm);
           mm = fmaxf(fmax3(m0, m1, m2), m3);
         }
-        mx = mm * a.cs;
+        mx = mm == -INFINITY ? 0.f : mm * a.cs;   // a CTA without keys: P' = 0, lse = -inf
         wait_cta(&p_empty[st], ph ^ 1);
       }
       // (2) P' = 2^(s c - m + 15) as fp16 in shared memory (second pass), and the row sum;
@@ -1221,7 +1239,10 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int c = 0; c < CL; ++c) Lsum += ex2(xv[c] - M);
         float inv;   // 1 / L to about 2^-23 (rcp.approx), well inside the score tolerance
         asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(Lsum));
-        const float w = ex2(mx - M + 15.f) * inv;
+        float w = ex2(mx - M + 15.f) * inv;
+        // query rows past the window (the last tile of a window that is not a multiple of
+        // 128): weight 0
+        if (PARTIAL && ((cur.q0 + tp) % QT) * kFQRows + row >= a.W) w = 0.f;
         const __half w1 = __float2half_rn(w);
         const float r1 = w - __half2float(w1);
         const __half w2 = __float2half_rn(r1);
@@ -1255,7 +1276,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
             const int split = side == 0 ? cid + 1 : cid;
             dst = a.part + (static_cast<size_t>(split - 1) * 2 + side) * a.W;
           }
-          dst[rank * kFKeys + row] = val;
+          if (!PARTIAL || static_cast<int>(rank) * kFKeys + row < a.W) dst[rank * kFKeys + row] = val;
           tc_fence_before();
           mbar_arrive(&d_empty[I & 1]);
         }
@@ -1415,23 +1436,30 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   }
 
 
-  // Windows of 128, 256, 512, 1024 or 2048 keys: the fused single-exponential kernel on
-  // clusters of W / 128 CTAs (sum and mean; the max aggregation takes the two-pass path). A
+  // Windows of up to 1024 keys, and of 2048: the fused single-exponential kernel (sum and
+  // mean; the max aggregation takes the two-pass path) on clusters of ceil(W / 128) CTAs. A
   // cluster of 16 is non-portable: where the device cannot hold one, W = 2048 takes the
-  // two-pass path too.
+  // two-pass path too, as do the other windows.
   // per device and cluster size: resident clusters, queried once (-1: none fits)
-  static std::atomic<int> max_clusters[kMaxDevices][kFMaxCluster + 1];
-  const bool fused_window = L.W == 128 || L.W == 256 || L.W == 512 || L.W == 1024 || L.W == 2048;
-  if (!agg_max && fused_window && max_clusters[dev][L.W / kFKeys].load() >= 0) {
-    const int CL = L.W / kFKeys;
-    auto kern = CL == 1 ? score_fused_kernel<D, 1>
-              : CL == 2 ? score_fused_kernel<D, 2>
-              : CL == 4 ? score_fused_kernel<D, 4>
-              : CL == 8 ? score_fused_kernel<D, 8> : score_fused_kernel<D, 16>;
-    const size_t smem = CL == 1 ? FusedSmem<D, 1>::bytes
-                      : CL == 2 ? FusedSmem<D, 2>::bytes
-                      : CL == 4 ? FusedSmem<D, 4>::bytes
-                      : CL == 8 ? FusedSmem<D, 8>::bytes : FusedSmem<D, 16>::bytes;
+  static std::atomic<int> max_clusters[kMaxDevices][kFMaxCluster + 1][2];
+  const bool fused_window = (L.W >= 1 && L.W <= 8 * kFKeys) || L.W == kFMaxCluster * kFKeys;
+  const int CL = (L.W + kFKeys - 1) / kFKeys;            // query tiles per head too
+  const int PT = L.W % kFKeys != 0 ? 1 : 0;             // the last CTA owns fewer keys
+  if (!agg_max && fused_window && max_clusters[dev][CL][PT].load() >= 0) {
+    using KernT = void (*)(CUtensorMap, CUtensorMap, ScoreArgs);
+    KernT kern = nullptr;
+    size_t smem = 0;
+    switch (CL) {
+#define KARA_FUSED_CASE(c)                                                                \
+      case c:                                                                             \
+        kern = PT ? score_fused_kernel<D, c, true> : score_fused_kernel<D, c, false>;     \
+        smem = FusedSmem<D, c>::bytes;                                                    \
+        break;
+      KARA_FUSED_CASE(1) KARA_FUSED_CASE(2) KARA_FUSED_CASE(3) KARA_FUSED_CASE(4)
+      KARA_FUSED_CASE(5) KARA_FUSED_CASE(6) KARA_FUSED_CASE(7) KARA_FUSED_CASE(8)
+#undef KARA_FUSED_CASE
+      default: kern = score_fused_kernel<D, 16, false>; smem = FusedSmem<D, 16>::bytes; break;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kFThreads);
     cfg.dynamicSmemBytes = smem;
@@ -1445,7 +1473,7 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (max_clusters[dev][CL].load() == 0) {
+    if (max_clusters[dev][CL][PT].load() == 0) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
       if (CL > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -1462,12 +1490,12 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
         cudaGetLastError();                // no cluster of 16 fits: the two-pass path below
         n = -1;
       }
-      max_clusters[dev][CL].store(n);
+      max_clusters[dev][CL][PT].store(n);
     }
-    if (max_clusters[dev][CL].load() > 0) {
+    if (max_clusters[dev][CL][PT].load() > 0) {
       const long long items = static_cast<long long>(L.R) * L.Hkv;
       const int ncl = static_cast<int>(
-          std::max<long long>(1, std::min<long long>(max_clusters[dev][CL].load(), items)));
+          std::max<long long>(1, std::min<long long>(max_clusters[dev][CL][PT].load(), items)));
       // Tile-granular ranges whenever the split slots fit in the workspace (they do whenever
       // ncl <= items, which the grid guarantees; checked all the same). The ranges are then at
       // least TPI tiles long, as the kernel assumes.

@@ -29,8 +29,9 @@ CASES = {
     "w128_fused": (synth.Workload("loop128", batch=3, layers=2, hq=8, hkv=2, head_dim=64,
                                   ctx_lo=20, ctx_hi=40, window=128, keep=26, spare_blocks=4),
                    16, 300),
-    # W = 64: the two-pass scorer; G = 2, d = 128, a check every 8 steps
-    "w64_twopass": (synth.Workload("loop64", batch=3, layers=2, hq=4, hkv=2, head_dim=128,
+    # W = 64: the fused scorer with one CTA owning 64 keys and half-empty query tiles, reading
+    # the window-query ring; G = 2, d = 128, a check every 8 steps
+    "w64_partial": (synth.Workload("loop64", batch=3, layers=2, hq=4, hkv=2, head_dim=128,
                                    ctx_lo=17, ctx_hi=50, window=64, keep=13, spare_blocks=4),
                     8, 150),
 }

@@ -56,6 +56,18 @@ SCORE_CASES = {
     "w1024_g2": synth.Workload("w1024_g2", batch=12, layers=1, hq=8, hkv=4,
                                    head_dim=128, ctx_lo=1024, ctx_hi=1800, window=1024,
                                    keep=204, heavy_frac=0.05, spare_blocks=8),
+    # windows that are not a multiple of 128: the last CTA of the cluster owns fewer keys
+    # (W = 1000 on 8 CTAs, the last with 104); windows between 1024 and 2048 and above 2048
+    # take the two-pass kernels
+    "w1000_partial": synth.Workload("w1000", batch=3, layers=1, hq=8, hkv=2, head_dim=128,
+                                    ctx_lo=1000, ctx_hi=1400, window=1000, keep=200,
+                                    heavy_frac=0.05, q_mode="neighbour", spare_blocks=8),
+    "w1100_twopass": synth.Workload("w1100", batch=3, layers=1, hq=4, hkv=2, head_dim=128,
+                                 ctx_lo=1100, ctx_hi=1500, window=1100, keep=220,
+                                 heavy_frac=0.05, spare_blocks=8),
+    "w2500_twopass": synth.Workload("w2500", batch=2, layers=1, hq=4, hkv=2, head_dim=128,
+                                    ctx_lo=2500, ctx_hi=2900, window=2500, keep=500,
+                                    heavy_frac=0.03, spare_blocks=8),
     # W = 2048: clusters of 16 CTAs (non-portable size); whole items per cluster, then more
     # items than resident clusters of 16 (at most 148 / 16 of them)
     "g4_w2048_ragged": synth.Workload("g4_w2048", batch=3, layers=1, hq=8, hkv=2, head_dim=128,
@@ -164,10 +176,13 @@ def test_score_split_items_skip_short_contexts():
 
 @pytest.mark.parametrize("name,launches", [("g7_w1024_unaligned", (1,)), ("w128_split_items", (2,)),
                                            ("w1024_split_items", (2,)),
+                                           ("g7_ragged_unaligned", (1, 2)), ("w1100_twopass", (3,)),
+                                           ("w2500_twopass", (3,)),
                                            ("g4_w2048_ragged", (1,)), ("w2048_split_items", (2,))])
 def test_score_launch_count(name, launches):
     """The fused kernel alone when every cluster range holds whole items; with the split sum
-    when more items than resident clusters make ranges end inside items."""
+    when more items than resident clusters make ranges end inside items; three two-pass
+    kernels above W = 2048."""
     wl = SCORE_CASES[name]
     cpu, dev = H.make(wl, 1)
     pool = K.PagedPool.from_cache(dev)

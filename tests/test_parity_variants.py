@@ -23,7 +23,8 @@ pytestmark = pytest.mark.gpu
 LAYER = synth.WORKLOADS["layer"]
 CASES = {
     "w512_fused": LAYER.with_(batch=3, ctx_lo=520, ctx_hi=900, window=512, keep=102),
-    "w200_twopass": LAYER.with_(batch=3, ctx_lo=300, ctx_hi=700, window=200, keep=40),
+    # W = 200: mean on the fused kernel (a last CTA with 72 keys), max on the two-pass kernels
+    "w200": LAYER.with_(batch=3, ctx_lo=300, ctx_hi=700, window=200, keep=40),
     # clusters of 16 CTAs (mean) and the two-pass kernels (max) at the largest fused window
     "w2048_fused": synth.Workload("w2048", batch=2, layers=1, hq=8, hkv=2, head_dim=128,
                                   ctx_lo=2050, ctx_hi=2600, window=2048, keep=409,
@@ -63,7 +64,7 @@ def test_score_aggregation_matches_oracle(name, agg):
 
 def test_max_from_the_ring_equals_max_from_q_win():
     """The ring form reads the same query rows: the same tiles, the same result, bit for bit."""
-    wl = CASES["w200_twopass"]
+    wl = CASES["w200"]
     cpu, dev = H.make(wl, 9)
     pool = K.PagedPool.from_cache(dev)
     W = wl.window
