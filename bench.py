@@ -726,8 +726,9 @@ def variants_run(step, reps: int = 10) -> dict:
             total += e0.elapsed_time(e1)
         out[name] = total / reps
     out["status"] = K.read_status(step.status)
-    out["note"] = ("one-layer workload; max runs the two-pass kernels (a max, not a sum, per "
-                   "key); shared = head sums, one select + Token2Chunk per (sequence, layer), "
+    out["note"] = ("one-layer workload; max runs the fused kernel with a per-key column "
+                   "maximum in place of the column-sum product; shared = head sums, one "
+                   "select + Token2Chunk per (sequence, layer), "
                    "keep copied to the 4 KV heads; select_then_token2chunk = the two calls the "
                    "step's fused kara_select_chunks replaces")
     return out

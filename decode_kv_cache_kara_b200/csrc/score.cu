@@ -76,6 +76,7 @@ struct ScoreArgs {
   int streamk;      // fused kernel: cluster ranges split items (else they hold whole items)
   int ring;         // queries from the window-query ring [batch, 2W, Hq, d] (else q_win)
   float out_scale;  // 1, or 1 / (G W) for the mean aggregation
+  int max_agg;      // the max aggregation (split parts combine by max)
   int32_t* status;
   int R, W, Wp, Hq, Hkv, G;
   int batch, max_blocks, num_blocks;
@@ -861,7 +862,7 @@ __device__ __forceinline__ uint32_t w_offset(int n, int k) {
                                (k & 7) * 2);
 }
 
-template <int D, int CL, bool PARTIAL>
+template <int D, int CL, bool PARTIAL, bool AGGMAX>
 __global__ void __launch_bounds__(kFThreads, 1)
 score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
@@ -917,7 +918,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int i = 0; i < kFPBufs; ++i) {
       mbar_init(&p_full[i], kFTeamThreads);         // one team per tile
       mbar_init(&w_full[i], kFTeamThreads);
-      mbar_init(&p_empty[i], 1);
+      mbar_init(&p_empty[i], AGGMAX ? kFTeamThreads : 1);   // the product, or the team
     }
     for (int i = 0; i < kFTeams; ++i) {
       mbar_init(&s_full[i], 1);
@@ -1059,7 +1060,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
       }
     }
-  } else if (warp == 2) {
+  } else if (warp == 2 && !AGGMAX) {
     // ---- UMMA issuer for the column sums: D += P'^T W, tile by tile ----
     if (lane == 0) {
       const uint32_t idesc_c = idesc_f16_f32(128, 16, true);
@@ -1132,6 +1133,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     uint8_t* const prow = p_buf + st * L::kPBytes + (row >> 3) * 1024 + (row & 7) * 128;
     uint32_t sq = 0;
     int xs = team, xq = 0;
+    float kmax0 = 0.f, kmax1 = 0.f;   // the max aggregation: this thread's two keys
     for (int T = team; have; T += kFTeams, ++sq) {
       const uint32_t ph = sq & 1;
       const uint32_t scol = lane_base + st * kFSCols +
@@ -1243,20 +1245,77 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
         // query rows past the window (the last tile of a window that is not a multiple of
         // 128): weight 0
         if (PARTIAL && ((cur.q0 + tp) % QT) * kFQRows + row >= a.W) w = 0.f;
-        const __half w1 = __float2half_rn(w);
-        const float r1 = w - __half2float(w1);
-        const __half w2 = __float2half_rn(r1);
-        const float r2 = r1 - __half2float(w2);
-        const __half w3 = __float2half_rn(r2 * 16777216.f);
-        uint8_t* wb = w_buf + st * L::kWBytes;
-        *reinterpret_cast<__half*>(wb + w_offset(0, row)) = w1;
-        *reinterpret_cast<__half*>(wb + w_offset(1, row)) = w2;
-        *reinterpret_cast<__half*>(wb + w_offset(2, row)) = w3;
-        fence_proxy_async();
-        mbar_arrive(&w_full[st]);
+        if (AGGMAX) {
+          // the row's softmax factor, P' w / 2^15, for the column maxima below
+          reinterpret_cast<float*>(w_buf + st * L::kWBytes)[row] = w * (1.f / 32768.f);
+        } else {
+          const __half w1 = __float2half_rn(w);
+          const float r1 = w - __half2float(w1);
+          const __half w2 = __float2half_rn(r1);
+          const float r2 = r1 - __half2float(w2);
+          const __half w3 = __float2half_rn(r2 * 16777216.f);
+          uint8_t* wb = w_buf + st * L::kWBytes;
+          *reinterpret_cast<__half*>(wb + w_offset(0, row)) = w1;
+          *reinterpret_cast<__half*>(wb + w_offset(1, row)) = w2;
+          *reinterpret_cast<__half*>(wb + w_offset(2, row)) = w3;
+          fence_proxy_async();
+          mbar_arrive(&w_full[st]);
+        }
+      }
+      if (AGGMAX) {
+        // (4') the max aggregation: per key, the largest softmax value over the tile's rows,
+        // from P' in shared memory times the row factors (thread: keys 2p, 2p + 1 of this
+        // CTA, rows 64 h .. 64 h + 63); kept in registers over the team's tiles of the
+        // segment, then merged into the output with an atomic max (non-negative floats order
+        // as their bits)
+        named_barrier(1 + team, kFTeamThreads);     // the team's P' rows and factors are in
+        const int kp = row & 63, rh = row >> 6;
+        if (!aborted) {
+          const float* wr = reinterpret_cast<const float*>(w_buf + st * L::kWBytes);
+          const uint8_t* pb = p_buf + st * L::kPBytes + (kp >> 5) * L::kPAtom + 4 * (kp & 3);
+          const int gq = (kp & 31) >> 2;               // the keys' 16-byte granule in a row
+          float m0 = 0.f, m1 = 0.f;
+          const float2 zero2 = make_float2(0.f, 0.f);
+#pragma unroll 4
+          for (int i = 64 * rh; i < 64 * rh + 64; i += 2) {   // two rows at a time
+            const uint32_t pa = *reinterpret_cast<const uint32_t*>(
+                pb + (i >> 3) * 1024 + (i & 7) * 128 + ((gq ^ (i & 7)) << 4));
+            const uint32_t pc = *reinterpret_cast<const uint32_t*>(
+                pb + (i >> 3) * 1024 + ((i + 1) & 7) * 128 + ((gq ^ ((i + 1) & 7)) << 4));
+            const float2 wi = *reinterpret_cast<const float2*>(wr + i);
+            const float2 fa = ffma2(__half22float2(*reinterpret_cast<const __half2*>(&pa)),
+                                    make_float2(wi.x, wi.x), zero2);
+            const float2 fc = ffma2(__half22float2(*reinterpret_cast<const __half2*>(&pc)),
+                                    make_float2(wi.y, wi.y), zero2);
+            m0 = fmax3(m0, fa.x, fc.x);
+            m1 = fmax3(m1, fa.y, fc.y);
+          }
+          kmax0 = fmaxf(kmax0, m0);
+          kmax1 = fmaxf(kmax1, m1);
+        }
+        mbar_arrive(&p_empty[st]);                  // this thread is done with P'
+        if (tp + kFTeams >= cur.q1 - cur.q0) {      // the team's last tile of the segment
+          if (!aborted) {
+            float* dst;
+            if (cur.q0 == 0 && cur.q1 == TPI) {
+              dst = a.scores + (static_cast<size_t>(cur.r) * a.Hkv + cur.g) * a.W;
+            } else {
+              const int side = cur.q0 == 0 ? 0 : 1;
+              const int split = side == 0 ? cid + 1 : cid;
+              dst = a.part + (static_cast<size_t>(split - 1) * 2 + side) * a.W;
+            }
+            const int k0 = static_cast<int>(rank) * kFKeys + 2 * kp;
+            if (!PARTIAL || 2 * kp < kcount)
+              atomicMax(reinterpret_cast<unsigned int*>(dst + k0), __float_as_uint(kmax0));
+            if (!PARTIAL || 2 * kp + 1 < kcount)
+              atomicMax(reinterpret_cast<unsigned int*>(dst + k0 + 1), __float_as_uint(kmax1));
+          }
+          kmax0 = 0.f;
+          kmax1 = 0.f;
+        }
       }
       // (5) the segment's last tile: the per-key sums over its heads, read by this team
-      if (tp == cur.q1 - cur.q0 - 1) {
+      if (!AGGMAX && tp == cur.q1 - cur.q0 - 1) {
         wait_cta(&d_full[I & 1], (I >> 1) & 1);
         if (!aborted) {
           tc_fence_after();
@@ -1318,7 +1377,8 @@ score_split_sum_kernel(const ScoreArgs a, int ncl, int TPI) {
   const float* head = a.part + static_cast<size_t>(k - 1) * 2 * a.W;
   const float* tail = head + a.W;
   float* dst = a.scores + (static_cast<size_t>(r) * a.Hkv + g) * a.W;
-  for (int j = threadIdx.x; j < a.W; j += blockDim.x) dst[j] = head[j] + tail[j];
+  for (int j = threadIdx.x; j < a.W; j += blockDim.x)
+    dst[j] = a.max_agg ? fmaxf(head[j], tail[j]) : head[j] + tail[j];
 }
 
 template <int D>
@@ -1428,6 +1488,7 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   a.part = nullptr;
   a.streamk = 0;
   a.out_scale = L.agg == KARA_AGG_MEAN ? 1.f / (static_cast<float>(a.G) * L.W) : 1.f;
+  a.max_agg = 0;
   const bool agg_max = L.agg == KARA_AGG_MAX;
   const int dev = device_slot();
   if (dev < 0) {
@@ -1436,29 +1497,42 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   }
 
 
-  // Windows of up to 1024 keys, and of 2048: the fused single-exponential kernel (sum and
-  // mean; the max aggregation takes the two-pass path) on clusters of ceil(W / 128) CTAs. A
-  // cluster of 16 is non-portable: where the device cannot hold one, W = 2048 takes the
-  // two-pass path too, as do the other windows.
-  // per device and cluster size: resident clusters, queried once (-1: none fits)
-  static std::atomic<int> max_clusters[kMaxDevices][kFMaxCluster + 1][2];
-  const bool fused_window = (L.W >= 1 && L.W <= 8 * kFKeys) || L.W == kFMaxCluster * kFKeys;
+  // Windows of up to 1024 keys, and of 2048: the fused single-exponential kernel on clusters
+  // of ceil(W / 128) CTAs (the max aggregation: head_dim 128 and up to 1024 keys). A cluster
+  // of 16 is non-portable: where the device cannot hold one, W = 2048 takes the two-pass path
+  // too, as do the other windows.
+  // per device, cluster size, partial last CTA and aggregation: resident clusters, queried
+  // once (-1: none fits)
+  static std::atomic<int> max_clusters[kMaxDevices][kFMaxCluster + 1][2][2];
   const int CL = (L.W + kFKeys - 1) / kFKeys;            // query tiles per head too
   const int PT = L.W % kFKeys != 0 ? 1 : 0;             // the last CTA owns fewer keys
-  if (!agg_max && fused_window && max_clusters[dev][CL][PT].load() >= 0) {
+  const int AG = agg_max ? 1 : 0;
+  const bool fused_window = agg_max ? (D == 128 && L.W >= 1 && L.W <= 8 * kFKeys)
+                                    : (L.W >= 1 && L.W <= 8 * kFKeys) || L.W == kFMaxCluster * kFKeys;
+  if (fused_window && max_clusters[dev][CL][PT][AG].load() >= 0) {
     using KernT = void (*)(CUtensorMap, CUtensorMap, ScoreArgs);
     KernT kern = nullptr;
     size_t smem = 0;
     switch (CL) {
-#define KARA_FUSED_CASE(c)                                                                \
-      case c:                                                                             \
-        kern = PT ? score_fused_kernel<D, c, true> : score_fused_kernel<D, c, false>;     \
-        smem = FusedSmem<D, c>::bytes;                                                    \
+#define KARA_FUSED_CASE(c)                                                                  \
+      case c:                                                                               \
+        if constexpr (D == 128) {                                                           \
+          if (AG) {                                                                         \
+            kern = PT ? score_fused_kernel<D, c, true, true> : score_fused_kernel<D, c, false, true>; \
+            smem = FusedSmem<D, c>::bytes;                                                  \
+            break;                                                                          \
+          }                                                                                 \
+        }                                                                                   \
+        kern = PT ? score_fused_kernel<D, c, true, false> : score_fused_kernel<D, c, false, false>; \
+        smem = FusedSmem<D, c>::bytes;                                                      \
         break;
       KARA_FUSED_CASE(1) KARA_FUSED_CASE(2) KARA_FUSED_CASE(3) KARA_FUSED_CASE(4)
       KARA_FUSED_CASE(5) KARA_FUSED_CASE(6) KARA_FUSED_CASE(7) KARA_FUSED_CASE(8)
 #undef KARA_FUSED_CASE
-      default: kern = score_fused_kernel<D, 16, false>; smem = FusedSmem<D, 16>::bytes; break;
+      default:
+        kern = score_fused_kernel<D, 16, false, false>;
+        smem = FusedSmem<D, 16>::bytes;
+        break;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kFThreads);
@@ -1473,7 +1547,7 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (max_clusters[dev][CL][PT].load() == 0) {
+    if (max_clusters[dev][CL][PT][AG].load() == 0) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
       if (CL > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -1490,12 +1564,12 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
         cudaGetLastError();                // no cluster of 16 fits: the two-pass path below
         n = -1;
       }
-      max_clusters[dev][CL][PT].store(n);
+      max_clusters[dev][CL][PT][AG].store(n);
     }
-    if (max_clusters[dev][CL][PT].load() > 0) {
+    if (max_clusters[dev][CL][PT][AG].load() > 0) {
       const long long items = static_cast<long long>(L.R) * L.Hkv;
       const int ncl = static_cast<int>(
-          std::max<long long>(1, std::min<long long>(max_clusters[dev][CL][PT].load(), items)));
+          std::max<long long>(1, std::min<long long>(max_clusters[dev][CL][PT][AG].load(), items)));
       // Tile-granular ranges whenever the split slots fit in the workspace (they do whenever
       // ncl <= items, which the grid guarantees; checked all the same). The ranges are then at
       // least TPI tiles long, as the kernel assumes.
@@ -1505,6 +1579,16 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
       a.part = L.lse;
       a.streamk = ncl > 1 && ntiles / ncl >= TPI &&
                   part_bytes <= score_workspace_bytes(L.R, L.W, L.Hq);
+      a.max_agg = AG;
+      if (AG) {
+        // the max aggregation merges into zeroed outputs with atomic maxima (softmax >= 0)
+        if (cudaMemsetAsync(L.scores, 0, static_cast<size_t>(L.R) * L.Hkv * L.W * sizeof(float),
+                            stream) != cudaSuccess ||
+            (a.streamk && cudaMemsetAsync(a.part, 0, part_bytes, stream) != cudaSuccess)) {
+          check_launch("kara_score max zero fill");
+          return KARA_ERR_CUDA;
+        }
+      }
       bool any_split = false;
       for (int k = 1; a.streamk && k < ncl && !any_split; ++k)
         any_split = (k * ntiles / ncl) % TPI != 0;

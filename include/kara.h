@@ -154,10 +154,10 @@ kara_status kara_score(const void* q_win, const void* k_cache, const kara_pool* 
 /*
  * kara_score_ex - kara_score (q_is_ring == 0: q is q_win [R, W, Hq, d]) or kara_score_ring
  * (q_is_ring != 0: q is the window-query ring [batch, 2W, Hq, d]) with the aggregation `agg`
- * (kara_agg). KARA_AGG_MAX runs the two-pass kernels for every window; sum and mean run the
- * fused kernel for windows of up to 1024 keys and of 2048 (the latter on a cluster of 16 CTAs,
- * where the device holds one), the two-pass kernels for the others. Other arguments, output
- * and errors as kara_score; an unknown agg is KARA_ERR_INVALID_ARG.
+ * (kara_agg). Sum and mean run the fused kernel for windows of up to 1024 keys and of 2048
+ * (the latter on a cluster of 16 CTAs, where the device holds one); the max runs it for
+ * windows of up to 1024 keys with head_dim 128; the other cases run the two-pass kernels.
+ * Other arguments, output and errors as kara_score; an unknown agg is KARA_ERR_INVALID_ARG.
  */
 kara_status kara_score_ex(const void* q, int32_t q_is_ring, const void* k_cache,
                           const kara_pool* pool, const int32_t* seq_ids, int32_t num_seqs,

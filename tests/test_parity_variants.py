@@ -23,8 +23,13 @@ pytestmark = pytest.mark.gpu
 LAYER = synth.WORKLOADS["layer"]
 CASES = {
     "w512_fused": LAYER.with_(batch=3, ctx_lo=520, ctx_hi=900, window=512, keep=102),
-    # W = 200: mean on the fused kernel (a last CTA with 72 keys), max on the two-pass kernels
+    # W = 200: the fused kernel with a last CTA of 72 keys (mean and max)
     "w200": LAYER.with_(batch=3, ctx_lo=300, ctx_hi=700, window=200, keep=40),
+    # more items than resident clusters: cluster ranges end inside items, the two parts are
+    # added (mean) or maxed (max) by the split kernel
+    "w256_split": synth.Workload("w256_split", batch=24, layers=1, hq=8, hkv=4, head_dim=128,
+                                 ctx_lo=260, ctx_hi=420, window=256, keep=51, heavy_frac=0.05,
+                                 spare_blocks=8),
     # clusters of 16 CTAs (mean) and the two-pass kernels (max) at the largest fused window
     "w2048_fused": synth.Workload("w2048", batch=2, layers=1, hq=8, hkv=2, head_dim=128,
                                   ctx_lo=2050, ctx_hi=2600, window=2048, keep=409,
@@ -33,13 +38,13 @@ CASES = {
 AGGS = {"mean": K.AGG_MEAN, "max": K.AGG_MAX}
 
 
-def oracle_agg(cpu, wl, agg):
+def oracle_agg(cpu, wl, agg, rows=None):
     q = H.f64(cpu["q_win"][0])
     kf = H.f64(cpu["k"][0])
     bt, cl = H.i32(cpu["block_table"]), H.i32(cpu["ctx_len"])
     scale = 1 / math.sqrt(wl.head_dim)
     out = []
-    for r in range(wl.batch):
+    for r in (range(wl.batch) if rows is None else rows):
         slots = ok.window_slots(int(cl[r]), wl.window)
         kw = ok.gather_rows(kf, bt[r], slots, wl.page)
         out.append(ok.window_scores_agg(q[r], kw, scale, agg))
@@ -53,13 +58,38 @@ def test_score_aggregation_matches_oracle(name, agg):
     cpu, dev = H.make(wl, 8)
     pool = K.PagedPool.from_cache(dev)
     status = K.new_status()
+    n0 = K.kara_launch_count()
     sc = K.kara_score_ex(dev["q_win"][0], dev["k"][0], pool, wl.window, agg=AGGS[agg],
                          status=status)
     torch.cuda.synchronize()
+    launches = K.kara_launch_count() - n0
     assert K.read_status(status) == 0
     H.assert_scores_close(H.f64(sc), oracle_agg(cpu, wl, agg))
+    # the fused kernel (and the split sum / max) for windows up to 1024 keys, and for the mean
+    # at 2048; else the three two-pass kernels
+    fused = wl.window <= 1024 or (agg == "mean" and wl.window == 2048)
+    assert (launches <= 2) == fused and (fused or launches == 3)
     if agg == "mean":   # the mean of each (sequence, KV head) row sums to 1
         assert np.allclose(H.f64(sc).sum(-1), 1.0, rtol=1e-4)
+
+
+def test_max_skips_short_contexts_in_split_items():
+    """The max aggregation with every third sequence too short for the window and cluster
+    ranges ending inside items: those rows are zero and reported, the rest match the oracle."""
+    wl = CASES["w256_split"]
+    cpu, dev = H.make(wl, 4)
+    bad = list(range(1, wl.batch, 3))
+    good = [r for r in range(wl.batch) if r not in bad]
+    dev["ctx_len"][bad] = wl.window - 1
+    pool = K.PagedPool.from_cache(dev)
+    status = K.new_status()
+    sc = K.kara_score_ex(dev["q_win"][0], dev["k"][0], pool, wl.window, agg=K.AGG_MAX,
+                         status=status)
+    torch.cuda.synchronize()
+    assert K.read_status(status) == K.ERR_INVALID_ARG
+    assert (sc[bad] == 0).all()
+    cpu["ctx_len"][bad] = wl.window - 1
+    H.assert_scores_close(H.f64(sc[good]), oracle_agg(cpu, wl, "max", good))
 
 
 def test_max_from_the_ring_equals_max_from_q_win():
