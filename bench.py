@@ -6,8 +6,8 @@ contexts of 2K-16K tokens (page 16, so windows start at unaligned slots), every 
 (the worst-case check step of the 100-step schedule), window W = 1024, keep 204 (20 %),
 Token2Chunk anchors 50 % / gap 8 / widen 1:
 
-    kara_score per layer -> kara_select_chunks per layer -> one kara_compact over all layers
-    -> paged_decode_attn per layer over the compressed cache
+    kara_score per layer -> one kara_select_chunks over the rows of all layers -> one
+    kara_compact over all layers -> paged_decode_attn per layer over the compressed cache
 
 then the block table, lengths and free list are restored, so that every step sees the same
 input (compaction writes only fresh blocks, so the old rows are still in place). Metric:
@@ -265,9 +265,10 @@ class Step:
             if layer_scored is not None:
                 layer_scored[layer].record()
         rec(1)
-        for layer in range(self.L):
-            K.kara_select_chunks(self.scores[layer], wl.keep, wl.anchor_frac, wl.gap_limit,
-                                 wl.widen, keep=self.keep[layer], sel=self.sel[layer])
+        # selection and Token2Chunk are per (sequence, KV head) row: one launch over the rows
+        # of every layer
+        K.kara_select_chunks(self.scores, wl.keep, wl.anchor_frac, wl.gap_limit, wl.widen,
+                             keep=self.keep, sel=self.sel)
         rec(2)
         K.kara_compact(c["k"], c["v"], self.pool, wl.window, self.keep, workspace=self.ws,
                        status=self.status)
