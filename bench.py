@@ -659,6 +659,45 @@ def gqa8b_run(dev, peaks: dict, src: str, steps: int = 5, warmup: int = 3) -> di
     return out
 
 
+def compress_compare(step: Step, reps: int = 5) -> dict:
+    """The step's selection + Token2Chunk and compaction of all layers as the two calls it
+    times (kara_select_chunks, kara_compact) against the fused kara_compress, on the step's
+    own scores; the bookkeeping is restored before every run (not timed)."""
+    K, wl, c = step.K, step.wl, step.c
+
+    def timed(fn):
+        out = []
+        for _ in range(reps + 1):
+            step.restore()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            out.append(e0.elapsed_time(e1))
+        return sorted(out[1:])[reps // 2]
+
+    def two_calls():
+        K.kara_select_chunks(step.scores, wl.keep, wl.anchor_frac, wl.gap_limit, wl.widen,
+                             keep=step.keep, sel=step.sel)
+        K.kara_compact(c["k"], c["v"], step.pool, wl.window, step.keep, workspace=step.ws,
+                       status=step.status)
+
+    def fused():
+        K.kara_compress(step.scores, c["k"], c["v"], step.pool, wl.window, wl.keep,
+                        wl.anchor_frac, wl.gap_limit, wl.widen, keep=step.keep,
+                        workspace=step.ws, status=step.status)
+
+    res = {"select_chunks_then_compact_ms": timed(two_calls), "compress_ms": timed(fused)}
+    step.restore()
+    torch.cuda.synchronize()
+    res["status"] = K.read_status(step.status)
+    res["note"] = ("all 28 layers of the step workload from the step's scores; median of "
+                   f"{reps} runs")
+    return res
+
+
 def variants_run(step, reps: int = 10) -> dict:
     """The score and selection variants on the one-layer workload (its window queries and
     cache, not changed by them): kara_score_ex with the mean and with the max aggregation, and
@@ -929,6 +968,7 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
         e2e = e2e_run(step, steps=args.e2e_steps, warmup=1)
         e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], dev, world)
     kernels = kernel_entries(wl, work, avg, step, peaks, src)
+    fused_compression = (compress_compare(step) if world == 1 and not args.no_layer else None)
     del step, cache
     torch.cuda.empty_cache()
     if rank != 0:
@@ -952,6 +992,8 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
                 "peak_source": f"{src} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
                 "per_launch": per_launch}
 
+    if fused_compression is not None:
+        kernels["fused_compression"] = fused_compression
     if world == 1 and not args.no_loop:
         kernels["amortised_100_step_schedule"] = decode_loop_run(dev, wl, seed + 50)
     if world == 1 and not args.no_layer:
