@@ -30,6 +30,10 @@ CASES = {
     "w256_split": synth.Workload("w256_split", batch=24, layers=1, hq=8, hkv=4, head_dim=128,
                                  ctx_lo=260, ctx_hi=420, window=256, keep=51, heavy_frac=0.05,
                                  spare_blocks=8),
+    # head_dim 64: mean on the fused kernel, max on the two-pass kernels
+    "d64_w256": synth.Workload("d64_w256", batch=3, layers=1, hq=8, hkv=2, head_dim=64,
+                               ctx_lo=260, ctx_hi=400, window=256, keep=51, heavy_frac=0.05,
+                               q_mode="neighbour", spare_blocks=8),
     # clusters of 16 CTAs (mean) and the two-pass kernels (max) at the largest fused window
     "w2048_fused": synth.Workload("w2048", batch=2, layers=1, hq=8, hkv=2, head_dim=128,
                                   ctx_lo=2050, ctx_hi=2600, window=2048, keep=409,
@@ -67,7 +71,8 @@ def test_score_aggregation_matches_oracle(name, agg):
     H.assert_scores_close(H.f64(sc), oracle_agg(cpu, wl, agg))
     # the fused kernel (and the split sum / max) for windows up to 1024 keys, and for the mean
     # at 2048; else the three two-pass kernels
-    fused = wl.window <= 1024 or (agg == "mean" and wl.window == 2048)
+    fused = ((wl.window <= 1024 and (agg == "mean" or wl.head_dim == 128))
+             or (agg == "mean" and wl.window == 2048))
     assert (launches <= 2) == fused and (fused or launches == 3)
     if agg == "mean":   # the mean of each (sequence, KV head) row sums to 1
         assert np.allclose(H.f64(sc).sum(-1), 1.0, rtol=1e-4)
