@@ -992,6 +992,11 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
                 "peak_source": f"{src} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
                 "per_launch": per_launch}
 
+    comp_ms = sum(kernels[op]["ms"] for op in ("kara_score", "select+token2chunk", "kara_compact"))
+    kernels["compression_only"] = {
+        "ms": comp_ms, "tokens_per_s": whole_job_value(tokens_step, world, comp_ms),
+        "note": "the step without its decode: scoring, selection + Token2Chunk and compaction "
+                "of all layers (per-op event times of the timed steps)"}
     if fused_compression is not None:
         kernels["fused_compression"] = fused_compression
     if world == 1 and not args.no_loop:
