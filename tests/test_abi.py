@@ -152,3 +152,37 @@ def test_binding_refuses_host_tensors():
     for name, fn in calls.items():
         with pytest.raises(ValueError, match="CUDA tensor"):
             fn()
+
+
+def test_empty_inputs_return_ok_without_a_launch(lib_path):
+    """No rows, no due sequences, an empty batch: every compute call returns KARA_OK on the
+    host and launches nothing (the buffers are never touched, so null pointers do)."""
+    L = K.lib()
+    null = ctypes.c_void_p(0)
+    launches = K.kara_launch_count()
+    pool = K._Pool(8, 8, 8, 8, 3, 64, 64, 16, 2, 128)       # dummy table pointers, 3 sequences
+    empty = K._Pool(8, 8, 8, 8, 0, 64, 64, 16, 2, 128)      # no sequence at all
+    layers = (K._LayerKV * 1)()
+    prm = K._LacacheParams(2, 1, 64, 2048, 64, 64)
+    calls = {
+        "kara_score": L.kara_score(null, null, ctypes.byref(pool), null, 0, 16, 4, 1.0, null,
+                                   null, 0, null, null),
+        "kara_score_ex max": L.kara_score_ex(null, 0, null, ctypes.byref(pool), null, 0, 16, 4,
+                                             1.0, K.AGG_MAX, null, null, 0, null, null),
+        "kara_score_ring": L.kara_score_ring(null, null, ctypes.byref(pool), null, 0, 16, 4, 1.0,
+                                             null, null, 0, null, null),
+        "kara_token2chunk": L.kara_token2chunk(null, null, 0, 16, 4, 0.5, 8, 1, null, null),
+        "kara_select_chunks": L.kara_select_chunks(null, 0, 16, 4, 0.5, 8, 1, null, null, null),
+        "kara_sum_heads": L.kara_sum_heads(null, 0, 2, 16, null, null),
+        "kara_expand_keep": L.kara_expand_keep(null, 0, 2, 4, null, null),
+        "kara_compact": L.kara_compact(layers, 1, ctypes.byref(pool), null, 0, 16, 4, null, null,
+                                       0, null, null),
+        "kara_compress": L.kara_compress(null, layers, 1, ctypes.byref(pool), null, 0, 16, 4, 0.5,
+                                         8, 1, null, null, 0, null, null),
+        "lacache_compact": L.lacache_compact(layers, 4, ctypes.byref(pool), null, 0,
+                                             ctypes.byref(prm), null, 0, null, null),
+        "paged_decode_attn": L.paged_decode_attn(null, null, null, ctypes.byref(empty), 4, 1.0,
+                                                 null, null, 0, null, null),
+    }
+    assert {name: code for name, code in calls.items() if code != K.OK} == {}
+    assert K.kara_launch_count() == launches
