@@ -412,8 +412,8 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
 // first query head writes k_new / v_new to slot n of the cache (its block was taken by
 // kara_step_begin), and every CTA writes its query to rows n mod W and n mod W + W of the
 // window-query ring. The stream kernel, which reads slots [0, n) only, has finished by then.
-constexpr int kCombWarps = 4;
-constexpr int kCombBatch = 8;
+constexpr int kCombWarps = 8;
+constexpr int kCombBatch = 4;
 
 template <int D>
 __global__ void __launch_bounds__(32 * kCombWarps)

@@ -58,13 +58,16 @@ SCORE_CASES = {
                                    keep=204, heavy_frac=0.05, spare_blocks=8),
     # windows that are not a multiple of 128: the last CTA of the cluster owns fewer keys
     # (W = 1000 on 8 CTAs, the last with 104); windows between 1024 and 2048 and above 2048
-    # take the two-pass kernels
+    # (up to the largest, 4096) take the two-pass kernels
     "w1000_partial": synth.Workload("w1000", batch=3, layers=1, hq=8, hkv=2, head_dim=128,
                                     ctx_lo=1000, ctx_hi=1400, window=1000, keep=200,
                                     heavy_frac=0.05, q_mode="neighbour", spare_blocks=8),
     "w1100_twopass": synth.Workload("w1100", batch=3, layers=1, hq=4, hkv=2, head_dim=128,
                                  ctx_lo=1100, ctx_hi=1500, window=1100, keep=220,
                                  heavy_frac=0.05, spare_blocks=8),
+    "w4096_largest": synth.Workload("w4096", batch=1, layers=1, hq=2, hkv=1, head_dim=128,
+                                    ctx_lo=4100, ctx_hi=4200, window=4096, keep=819,
+                                    heavy_frac=0.03, spare_blocks=8),
     "w2500_twopass": synth.Workload("w2500", batch=2, layers=1, hq=4, hkv=2, head_dim=128,
                                     ctx_lo=2500, ctx_hi=2900, window=2500, keep=500,
                                     heavy_frac=0.03, spare_blocks=8),
