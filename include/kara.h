@@ -139,8 +139,9 @@ typedef enum kara_op {
  *  seq_ids    device int32 [num_seqs] or NULL (row r is cache row r).
  *  window     1 .. KARA_MAX_WINDOW.      scale  usually 1/sqrt(head_dim).
  *  scores     fp32 [num_seqs, num_kv_heads, window] (written).
- *  workspace  >= kara_workspace_bytes(KARA_OP_SCORE, ...): per-query log-sum-exp of every
- *             16-page key chunk of the window.
+ *  workspace  >= kara_workspace_bytes(KARA_OP_SCORE, ...): the fused kernel's partial key
+ *             sums of items split between two clusters, or the two-pass kernels' per-query
+ *             log-sum-exp of every 16-page key chunk of the window.
  *  dev_status device int32: KARA_ERR_INVALID_ARG if n < window or n exceeds the table,
  *             KARA_ERR_BAD_BLOCK for a window block id outside [0, num_blocks),
  *             KARA_ERR_TIMEOUT if a pipeline wait ran out; the scores of such a sequence are
