@@ -474,6 +474,7 @@ __device__ __forceinline__ int ladder_source(const LadderGather& g, int layer, i
 }
 
 __global__ void __launch_bounds__(kGatherThreads) ladder_gather_kernel(const LadderGather g) {
+  __shared__ size_t s_src[kLadderSlots], s_dst[kLadderSlots];   // row starts, in 16-byte units
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int32_t* hdr = g.plan;
   if (hdr[0] != 1) return;
@@ -492,7 +493,18 @@ __global__ void __launch_bounds__(kGatherThreads) ladder_gather_kernel(const Lad
   uint4* vdst = reinterpret_cast<uint4*>(g.layers.v[layer]);
   const int t0 = chunk * kLadderSlots;
   const int t1 = min(g.budget, t0 + kLadderSlots);
+  // the chunk's source and destination rows, once per slot (not per 16-byte piece)
+  if (threadIdx.x < t1 - t0) {
+    const int t = t0 + threadIdx.x;
+    const int src = ladder_source(g, layer, t, n);
+    s_src[threadIdx.x] = (static_cast<size_t>(tab[src >> 4]) * 16 + (src & 15)) * g.row_vecs;
+    s_dst[threadIdx.x] = (static_cast<size_t>(fr[t >> 4]) * 16 + (t & 15)) * g.row_vecs;
+  }
+  __syncthreads();
   const int pieces = (t1 - t0) * g.row_vecs;
+  // row_vecs (Hkv * d * 2 / 16) is a power of two for power-of-two head counts: shifts then
+  const bool pow2 = (g.row_vecs & (g.row_vecs - 1)) == 0;
+  const int shift = __ffs(g.row_vecs) - 1;
   constexpr int kUnroll = 4;
   for (int base = threadIdx.x; base < pieces; base += kGatherThreads * kUnroll) {
     uint4 kv[kUnroll], vv[kUnroll];
@@ -503,13 +515,10 @@ __global__ void __launch_bounds__(kGatherThreads) ladder_gather_kernel(const Lad
       const int i = base + u * kGatherThreads;
       act[u] = i < pieces;
       if (!act[u]) continue;
-      const int t = t0 + i / g.row_vecs;
-      const int v = i % g.row_vecs;
-      const int src = ladder_source(g, layer, t, n);
-      const int sblk = tab[src >> 4];
-      const int dblk = fr[t >> 4];
-      const size_t si = (static_cast<size_t>(sblk) * 16 + (src & 15)) * g.row_vecs + v;
-      dsti[u] = (static_cast<size_t>(dblk) * 16 + (t & 15)) * g.row_vecs + v;
+      const int tl = pow2 ? i >> shift : i / g.row_vecs;
+      const int v = i - tl * g.row_vecs;
+      const size_t si = s_src[tl] + v;
+      dsti[u] = s_dst[tl] + v;
       kv[u] = ksrc[si];
       vv[u] = vsrc[si];
     }
