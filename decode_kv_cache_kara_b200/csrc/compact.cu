@@ -265,6 +265,9 @@ __global__ void __launch_bounds__(kGatherThreads) kara_gather_kernel(const KaraG
   __shared__ int s_old[kMaxWindowPages];     // old block ids of the window's pages
   __shared__ int s_fresh[kMaxWindowPages];   // the sequence's fresh block ids
   __shared__ int s_keep[kChunkRows];         // this chunk's kept positions
+  // the CTA's rows (prefix rows, then kept rows): source and destination row starts in
+  // 16-byte units, once per row rather than per piece; ~0 marks a row that is not copied
+  __shared__ size_t s_src[kChunkRows + 16], s_dst[kChunkRows + 16];
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int32_t* hdr = g.plan;
   if (hdr[0] != 1) return;
@@ -289,16 +292,33 @@ __global__ void __launch_bounds__(kGatherThreads) kara_gather_kernel(const KaraG
   for (int i = threadIdx.x; i < n_new; i += kGatherThreads) s_fresh[i] = fr[i];
   for (int i = threadIdx.x; i < t1 - t0; i += kGatherThreads) s_keep[i] = kp[t0 + i];
   __syncthreads();
+  // rows handled by this CTA: prefix rows (chunk 0 only), then kept rows of the chunk
+  const int npre = (chunk == 0) ? off : 0;
+  const int total = npre + max(0, t1 - t0);
+  for (int i = threadIdx.x; i < total; i += kGatherThreads) {
+    int src_slot, dst_slot;
+    bool ok = true;
+    if (i < npre) {
+      src_slot = dst_slot = p0 * 16 + i;
+    } else {
+      const int pos = s_keep[i - npre];
+      ok = pos >= 0 && pos < g.W;          // refused by the plan already; never read outside
+      src_slot = start + (ok ? pos : 0);
+      dst_slot = start + t0 + (i - npre);
+    }
+    const int sblk = s_old[(src_slot >> 4) - p0];
+    const int dblk = s_fresh[(dst_slot >> 4) - p0];
+    s_src[i] = ok ? ((static_cast<size_t>(sblk) * 16 + (src_slot & 15)) * g.Hkv + head) * kVecPerRow
+                  : ~size_t(0);
+    s_dst[i] = ((static_cast<size_t>(dblk) * 16 + (dst_slot & 15)) * g.Hkv + head) * kVecPerRow;
+  }
+  __syncthreads();
   const uint4* ksrc = reinterpret_cast<const uint4*>(g.layers.k[layer]);
   const uint4* vsrc = reinterpret_cast<const uint4*>(g.layers.v[layer]);
   uint4* kdst = reinterpret_cast<uint4*>(g.layers.k[layer]);
   uint4* vdst = reinterpret_cast<uint4*>(g.layers.v[layer]);
   const int vec = threadIdx.x % kVecPerRow;
   const int sub = threadIdx.x / kVecPerRow;
-
-  // rows handled by this CTA: prefix rows (chunk 0 only), then kept rows of the chunk
-  const int npre = (chunk == 0) ? off : 0;
-  const int total = npre + max(0, t1 - t0);
   constexpr int kUnroll = 8;
   for (int base = sub; base < total; base += kRowsPerPass * kUnroll) {
     uint4 kv[kUnroll], vv[kUnroll];
@@ -307,27 +327,10 @@ __global__ void __launch_bounds__(kGatherThreads) kara_gather_kernel(const KaraG
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int i = base + u * kRowsPerPass;
-      act[u] = i < total;
+      act[u] = i < total && s_src[i] != ~size_t(0);
       if (!act[u]) continue;
-      int src_slot, dst_slot;
-      if (i < npre) {
-        src_slot = dst_slot = p0 * 16 + i;
-      } else {
-        const int t = t0 + (i - npre);
-        const int pos = s_keep[i - npre];
-        if (pos < 0 || pos >= g.W) {      // refused by the plan already; never read outside
-          act[u] = false;
-          continue;
-        }
-        src_slot = start + pos;
-        dst_slot = start + t;
-      }
-      const int sblk = s_old[(src_slot >> 4) - p0];
-      const int dblk = s_fresh[(dst_slot >> 4) - p0];
-      const size_t si = ((static_cast<size_t>(sblk) * 16 + (src_slot & 15)) * g.Hkv + head) *
-                            kVecPerRow + vec;
-      dsti[u] = ((static_cast<size_t>(dblk) * 16 + (dst_slot & 15)) * g.Hkv + head) *
-                    kVecPerRow + vec;
+      const size_t si = s_src[i] + vec;
+      dsti[u] = s_dst[i] + vec;
       kv[u] = ksrc[si];
       vv[u] = vsrc[si];
     }
