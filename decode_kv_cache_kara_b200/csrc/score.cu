@@ -77,6 +77,17 @@ struct ScoreArgs {
   int ring;         // queries from the window-query ring [batch, 2W, Hq, d] (else q_win)
   float out_scale;  // 1, or 1 / (G W) for the mean aggregation
   int max_agg;      // the max aggregation (split parts combine by max)
+  // A launch may cover part of the work: due rows [row0, row0 + R) (seq_ids and the query
+  // rows are indexed by the global row; scores and the workspace by the local one, their
+  // pointers starting at the range) and KV heads [g0, g0 + HkvN) of each (every head is
+  // indexed globally); the fused kernel takes the first `items` (row, KV head) items.
+  int row0, g0, HkvN;
+  long long items;
+  // The fused kernel with a helper beside it (a one-CTA-per-item two-pass kernel on the SMs
+  // the clusters leave idle): each fused CTA adds 1 to *done_count when it leaves; CTA 0 of
+  // the helper waits for done_target of them, so that what follows sees both kernels' work.
+  int* done_count;
+  int done_target;
   int32_t* status;
   int R, W, Wp, Hq, Hkv, G;
   int batch, max_blocks, num_blocks;
@@ -90,7 +101,7 @@ struct SeqInfo {
 
 __device__ __forceinline__ SeqInfo seq_info(const ScoreArgs& a, int r) {
   SeqInfo s;
-  s.b = a.seq_ids ? a.seq_ids[r] : r;
+  s.b = a.seq_ids ? a.seq_ids[a.row0 + r] : a.row0 + r;
   s.ok = s.b >= 0 && s.b < a.batch;
   s.n = s.ok ? a.ctx_len[s.b] : 0;
   s.ok = s.ok && s.n >= a.W && s.n <= a.max_blocks * 16;
@@ -108,7 +119,7 @@ __device__ __forceinline__ int q_tile_row(const ScoreArgs& a, const SeqInfo& s, 
   return a.ring ? s.start % a.W + row0 : row0;
 }
 __device__ __forceinline__ int q_tile_batch(const ScoreArgs& a, const SeqInfo& s, int r) {
-  return a.ring ? s.b : r;
+  return a.ring ? s.b : a.row0 + r;
 }
 
 // Block id of page p of sequence row b, with range check (an out-of-range id is reported and
@@ -136,13 +147,13 @@ struct TileCursor {
         s = seq_info(a, r);
         per = s.ok ? (s.np + 7) / 8 : (a.W + kKRows2 - 1) / kKRows2;
       }
-      if (t < base + a.Hkv * per) break;
-      base += a.Hkv * per;
+      if (t < base + a.HkvN * per) break;
+      base += a.HkvN * per;
       ++r;
       per = -1;
     }
     const int local = t - base;
-    g = local / per;
+    g = a.g0 + local / per;
     kt = local % per;
     return true;
   }
@@ -160,7 +171,7 @@ struct RowTileCursor {
       if (per < 0) {
         s = seq_info(a, r);
         nc = s.ok ? (s.np + 15) / 16 : 0;
-        per = a.Hkv * nc * a.G;
+        per = a.HkvN * nc * a.G;
       }
       if (t < base + per) break;
       base += per;
@@ -171,7 +182,7 @@ struct RowTileCursor {
     hl = local % a.G;
     local /= a.G;
     c = local % nc;
-    g = local / nc;
+    g = a.g0 + local / nc;
     return true;
   }
 };
@@ -182,19 +193,18 @@ struct RowTileCursor {
 // stream through it: S = Q K^T (UMMA M = 128 queries, N = the chunk's keys). The partial
 // results of the chunks are merged when pass 2 stages them.
 // ----------------------------------------------------------------------------------------
+// The pass as a device function over the tiles t0, t0 + tstep, ... of the cursor (a kernel
+// passes its CTA index and the grid size; the one-CTA item kernel 0 and 1), on the
+// 1024-aligned shared memory `smem`. `relinquish`: release the CTA's right to allocate
+// tensor memory after this pass's allocation (the item kernel allocates again).
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
-                      const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
+__device__ __forceinline__ void rowstats_pass(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                              const ScoreArgs& a, uint8_t* smem, int t0,
+                                              int tstep, bool relinquish) {
   constexpr int NCH = D / 64;
   constexpr uint32_t kQBytes = NCH * kQRows1 * kRowBytes;
   constexpr uint32_t kKBytes = NCH * kKRows1 * kRowBytes;
   constexpr uint32_t kPageBytes = 16 * kRowBytes;
-
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
   uint8_t* k_buf = smem;                      // 2 x kKBytes (key chunks)
   uint8_t* q_buf = smem + 2 * kKBytes;        // kQStages1 x kQBytes (query tiles)
   float2* comb = reinterpret_cast<float2*>(q_buf + kQStages1 * kQBytes);   // [kParts-1][128]
@@ -228,7 +238,7 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if (relinquish) tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
@@ -245,7 +255,7 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
     uint32_t kph = 0, qph = 0;
     RowTileCursor cur;
     int g, c, hl;
-    for (int t = blockIdx.x; cur.seek(a, t, g, c, hl); t += gridDim.x) {
+    for (int t = t0; cur.seek(a, t, g, c, hl); t += tstep) {
       if (__shfl_sync(0xffffffffu, *abort_flag != 0 ? 1 : 0, 0)) break;
       const SeqInfo& s = cur.s;
       const int r = cur.r;
@@ -289,7 +299,7 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
       uint32_t kph = 0, qph = 0, aph = 0;
       RowTileCursor cur;
       int g, c, hl;
-      for (int t = blockIdx.x; !*abort_flag && cur.seek(a, t, g, c, hl); t += gridDim.x) {
+      for (int t = t0; !*abort_flag && cur.seek(a, t, g, c, hl); t += tstep) {
         const SeqInfo& s = cur.s;
         const int pages = min(16, s.np - c * 16);
         if (!mbar_wait(&k_full[ki], kph, abort_flag, a.status)) break;
@@ -332,7 +342,7 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
     bool aborted = false;
     RowTileCursor cur;
     int g, c, hl;
-    for (int t = blockIdx.x; cur.seek(a, t, g, c, hl); t += gridDim.x) {
+    for (int t = t0; cur.seek(a, t, g, c, hl); t += tstep) {
       const SeqInfo& s = cur.s;
       const int r = cur.r;
       const int h = g * a.G + hl;
@@ -447,7 +457,23 @@ score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
+  if (threadIdx.x == 0) {   // the barriers' memory may be reused by a later pass
+    for (int i = 0; i < 4 + 2 * kQStages1 + 4; ++i) mbar_inval(&bars[i]);
+  }
+  __syncthreads();
 }
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+score_rowstats_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  rowstats_pass<D>(tm_q, tm_k, a, smem, blockIdx.x, gridDim.x, true);
+}
+
 
 // ----------------------------------------------------------------------------------------
 // Merge of the per-chunk partial log-sum-exps: lse = log2(sum_c 2^lse_c), one thread per query.
@@ -482,19 +508,15 @@ __global__ void __launch_bounds__(256) score_lse_merge_kernel(const ScoreArgs a)
 // ----------------------------------------------------------------------------------------
 // kMax: the largest probability of each key over the group's queries in place of the sum:
 // max_i 2^(s c - lse_i) = 2^(max_i (s c - lse_i)), one exponential per key.
+// The pass as a device function, as rowstats_pass.
 template <int D, bool kMax>
-__global__ void __launch_bounds__(kThreads, 1)
-score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
-                    const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
+__device__ __forceinline__ void colsum_pass(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                            const ScoreArgs& a, uint8_t* smem, int t0,
+                                            int tstep, bool relinquish) {
   constexpr int NCH = D / 64;
   constexpr uint32_t kABytes = NCH * kKRows2 * kRowBytes;
   constexpr uint32_t kBBytes = NCH * kQRows2 * kRowBytes;
   constexpr uint32_t kPageBytes = 16 * kRowBytes;
-
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
   uint8_t* a_buf = smem;                    // 2 x kABytes (key tiles)
   uint8_t* b_buf = smem + 2 * kABytes;      // kQStages2 x kBBytes (query tiles)
   float* lse_s = reinterpret_cast<float*>(b_buf + kQStages2 * kBBytes);   // [2][256]
@@ -530,7 +552,7 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if (relinquish) tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
@@ -547,7 +569,7 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
     uint32_t aph = 0, bph = 0;
     TileCursor cur;
     int g, kt;
-    for (int t = blockIdx.x; cur.seek(a, t, g, kt); t += gridDim.x) {
+    for (int t = t0; cur.seek(a, t, g, kt); t += tstep) {
       if (__shfl_sync(0xffffffffu, *abort_flag != 0 ? 1 : 0, 0)) break;
       const SeqInfo& s = cur.s;
       if (!s.ok) continue;
@@ -593,7 +615,7 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t idesc = idesc_bf16_f32(128, kQRows2);
       TileCursor cur;
       int g, kt;
-      for (int t = blockIdx.x; !*abort_flag && cur.seek(a, t, g, kt); t += gridDim.x) {
+      for (int t = t0; !*abort_flag && cur.seek(a, t, g, kt); t += tstep) {
         if (!cur.s.ok) continue;
         if (!mbar_wait(&a_full[ai], aph, abort_flag, a.status)) break;
         const uint32_t a_addr = smem_u32(a_buf + ai * kABytes);
@@ -635,7 +657,7 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
     bool aborted = false;
     TileCursor cur;
     int g, kt;
-    for (int t = blockIdx.x; cur.seek(a, t, g, kt); t += gridDim.x) {
+    for (int t = t0; cur.seek(a, t, g, kt); t += tstep) {
       const SeqInfo& s = cur.s;
       const int r = cur.r;
       float* out = a.scores + (static_cast<size_t>(r) * a.Hkv + g) * a.W;
@@ -737,6 +759,87 @@ score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
+  if (threadIdx.x == 0) {   // the barriers' memory may be reused by a later pass
+    for (int i = 0; i < 4 + 2 * kQStages2 + 4; ++i) mbar_inval(&bars[i]);
+  }
+  __syncthreads();
+}
+
+template <int D, bool kMax>
+__global__ void __launch_bounds__(kThreads, 1)
+score_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  colsum_pass<D, kMax>(tm_q, tm_k, a, smem, blockIdx.x, gridDim.x, true);
+}
+
+// ----------------------------------------------------------------------------------------
+// The helper beside the fused kernel: one CTA takes whole (row, KV head) items, items
+// item0 + blockIdx.x, + gridDim.x, ..., through both passes of the two-pass path (the row
+// log-sum-exps of the item's G query heads, their merge over the key chunks, the column
+// sums), so that it needs nothing from other CTAs. Launched as the fused kernel's
+// programmatic dependent once that kernel's CTAs all run, on the SMs its clusters leave idle;
+// it reads only what was complete before the fused kernel started, so it does not wait at
+// entry. CTA 0 waits at the end for every fused CTA (a.done_count), so that the kernels after
+// this one see both kernels' scores. Workspace: one row's two-pass region per CTA.
+// ----------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+score_item_kernel(const __grid_constant__ CUtensorMap tm_q1,
+                  const __grid_constant__ CUtensorMap tm_q2,
+                  const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a, long long item0,
+                  long long nitems) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const size_t region = static_cast<size_t>(a.Hq) * (a.CM + 1) * a.Wp;   // floats per CTA
+  float* ws = a.lse + blockIdx.x * region;
+  for (long long it = blockIdx.x; it < nitems; it += gridDim.x) {
+    const long long item = item0 + it;
+    const int r = static_cast<int>(item / a.Hkv);
+    const int g = static_cast<int>(item - static_cast<long long>(r) * a.Hkv);
+    ScoreArgs b = a;
+    b.R = 1;
+    b.row0 = r;
+    b.g0 = g;
+    b.HkvN = 1;
+    b.scores = a.scores + static_cast<size_t>(r) * a.Hkv * a.W;
+    b.lse = ws;
+    b.lse_merged = ws + static_cast<size_t>(a.Hq) * a.CM * a.Wp;
+    rowstats_pass<D>(tm_q1, tm_k, b, smem, 0, 1, false);
+    // merge of the key chunks' partial log-sum-exps, the item's G query heads
+    const SeqInfo s = seq_info(b, 0);
+    const int nc = s.ok ? (s.np + 15) / 16 : 0;
+    for (int i = threadIdx.x; i < a.G * a.Wp; i += blockDim.x) {
+      const int h = g * a.G + i / a.Wp;
+      const int token = i % a.Wp;
+      float out = INFINITY;
+      if (s.ok && token < a.W) {
+        const float* p = b.lse + static_cast<size_t>(h) * a.CM * a.Wp + token;
+        float mx = -INFINITY;
+        for (int c = 0; c < nc; ++c) mx = fmaxf(mx, p[static_cast<size_t>(c) * a.Wp]);
+        float sum = 0.f;
+        for (int c = 0; c < nc; ++c) sum += ex2(p[static_cast<size_t>(c) * a.Wp] - mx);
+        out = mx + __log2f(sum);
+      }
+      b.lse_merged[static_cast<size_t>(h) * a.Wp + token] = out;
+    }
+    __syncthreads();
+    colsum_pass<D, false>(tm_q2, tm_k, b, smem, 0, 1, false);
+  }
+  if (a.done_count != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(a.done_count) < a.done_target) {
+      if (clock64() - t0 > kWaitBudgetCycles) {
+        report(a.status, KARA_ERR_TIMEOUT);
+        break;
+      }
+      __nanosleep(500);
+    }
+  }
 }
 
 // ----------------------------------------------------------------------------------------
@@ -776,6 +879,12 @@ constexpr int kFEpiThreads = 32 * kFEpiWarps;
 constexpr int kFKeys = 128;            // window keys owned per CTA
 constexpr int kFKRows = 144;           // key rows loaded per CTA (9 pages)
 constexpr int kFQRows = 128;           // queries per tile
+// the helper beside the fused kernel (score_item_kernel): used from this many idle SMs; an
+// item's cost per SM on the two-pass path against the fused kernel's (clusters of up to 8,
+// clusters of 16), measured: step workload 1.04 against 0.42 ms; 8B-GQA 2.07 against 1.05
+constexpr int kHelperMinSms = 8;
+constexpr double kHelperCost = 2.5;
+constexpr double kHelperCost16 = 2.0;
 constexpr int kFMaxCluster = 16;      // W = 2048: a non-portable cluster of 16 CTAs
 constexpr int kFPBufs = kFTeams;       // S, P' and weight buffers, tile T in buffer T mod 3
 // query ring slots of one 64-channel chunk each: three, or two for a cluster of 16 (whose
@@ -808,7 +917,7 @@ struct SegCursor {
   int r = 0, g = 0, q0 = 0, q1 = 0;
   SeqInfo s;
   __device__ __forceinline__ void init(const ScoreArgs& a, int c, int ncl, int TPI) {
-    const long long items = static_cast<long long>(a.R) * a.Hkv;
+    const long long items = a.items;
     if (a.streamk) {
       const long long n = items * TPI;
       t = c * n / ncl;
@@ -867,6 +976,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
 score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
+  // with a helper: it may start now, on the SMs this grid leaves idle
+  if (a.done_count != nullptr) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   using L = FusedSmem<D, CL>;
   constexpr int kFQSlots = L::kQSlots;
   constexpr int NCH = L::NCH;
@@ -1358,6 +1469,10 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     tmem_dealloc(tmem_base, kTmemCols);
   }
   cluster_sync_all();     // no CTA leaves while a peer may still write into its shared memory
+  if (a.done_count != nullptr && threadIdx.x == 0) {
+    __threadfence();      // this CTA's writes (ordered by the barrier above) before the count
+    atomicAdd(a.done_count, 1);
+  }
 }
 
 // Items split between two clusters of the fused kernel: scores = head part + tail part (in
@@ -1367,7 +1482,7 @@ __global__ void __launch_bounds__(256)
 score_split_sum_kernel(const ScoreArgs a, int ncl, int TPI) {
   asm volatile("griddepcontrol.wait;" ::: "memory");   // the fused kernel's writes are visible
   const int k = blockIdx.x + 1;
-  const long long n = static_cast<long long>(a.R) * a.Hkv * TPI;
+  const long long n = a.items * TPI;
   const long long t = k * n / ncl;
   const long long item = t / TPI;
   if (t == item * TPI) return;
@@ -1446,6 +1561,33 @@ int sm_count(int dev) {
   return n;
 }
 
+// The helper: items [item0, item0 + h) on F CTAs (one per idle SM), as the fused kernel's
+// programmatic dependent; CTA 0 waits for `target` fused CTAs at its end.
+template <int D>
+kara_status launch_helper(ScoreArgs a, const ScoreLaunch& L, const CUtensorMap& tq1,
+                          const CUtensorMap& tq2, const CUtensorMap& tk, long long item0,
+                          long long h, int F, int target, cudaStream_t stream) {
+  static std::atomic<int> attr_done[kMaxDevices];   // per device: the smem limit is set
+  const int dev = device_slot();
+  constexpr size_t smem = rowstats_smem<D>() > colsum_smem<D>() ? rowstats_smem<D>()
+                                                               : colsum_smem<D>();
+  if (!attr_done[dev].load()) {
+    cudaFuncSetAttribute(score_item_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+    attr_done[dev].store(1);
+  }
+  a.lse = L.lse;
+  a.done_target = target;
+  launch_pdl(score_item_kernel<D>, dim3(F), dim3(kThreads), smem, stream, tq1, tq2, tk, a,
+             item0, h);
+  if (check_launch("score_item_kernel") != KARA_OK) {
+    describe_kernel("score_item_kernel", reinterpret_cast<const void*>(score_item_kernel<D>),
+                    kThreads, smem);
+    return KARA_ERR_CUDA;
+  }
+  return KARA_OK;
+}
+
 template <int D>
 kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   // queries: q_win [R, W, Hq, d], or the window-query ring [batch, 2W, Hq, d]
@@ -1489,6 +1631,12 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
   a.streamk = 0;
   a.out_scale = L.agg == KARA_AGG_MEAN ? 1.f / (static_cast<float>(a.G) * L.W) : 1.f;
   a.max_agg = 0;
+  a.row0 = 0;
+  a.g0 = 0;
+  a.HkvN = L.Hkv;
+  a.items = static_cast<long long>(L.R) * L.Hkv;
+  a.done_count = nullptr;
+  a.done_target = 0;
   const bool agg_max = L.agg == KARA_AGG_MAX;
   const int dev = device_slot();
   if (dev < 0) {
@@ -1567,18 +1715,47 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
       max_clusters[dev][CL][PT][AG].store(n);
     }
     if (max_clusters[dev][CL][PT][AG].load() > 0) {
-      const long long items = static_cast<long long>(L.R) * L.Hkv;
+      const int maxc = max_clusters[dev][CL][PT][AG].load();
+      const long long all_items = static_cast<long long>(L.R) * L.Hkv;
+      const size_t ws_bytes = score_workspace_bytes(L.R, L.W, L.Hq);
+      // Helper items: when the clusters fill the GPU and leave at least kHelperMinSms SMs
+      // idle, score_item_kernel takes the last m * F items there (F = the idle SMs, m items
+      // each), m from the per-SM cost of an item on the two-pass path against the fused one
+      // (kHelperCost: 2.5 on clusters of up to 8, 2.0 on clusters of 16, measured), so that
+      // both kernels end together. Sum and mean, head_dim 128. Workspace: [F one-row two-pass
+      // regions][split parts][done counter].
+      const int F = sm_count(dev) - maxc * CL;
+      long long h = 0;
+      if (!AG && D == 128 && F >= kHelperMinSms && all_items >= maxc) {
+        const double cost = CL > 8 ? kHelperCost16 : kHelperCost;
+        const long long m = static_cast<long long>(all_items / (cost * maxc * CL + F));
+        h = m * F;
+        const size_t need = static_cast<size_t>(F) * score_workspace_bytes(1, L.W, L.Hq) +
+                            static_cast<size_t>(maxc - 1) * 2 * L.W * sizeof(float) + 16;
+        if (all_items - h < maxc || need > ws_bytes) h = 0;
+      }
+      const long long items = all_items - h;
+      a.items = items;
       const int ncl = static_cast<int>(
-          std::max<long long>(1, std::min<long long>(max_clusters[dev][CL][PT][AG].load(), items)));
+          std::max<long long>(1, std::min<long long>(maxc, items)));
       // Tile-granular ranges whenever the split slots fit in the workspace (they do whenever
       // ncl <= items, which the grid guarantees; checked all the same). The ranges are then at
       // least TPI tiles long, as the kernel assumes.
       const int TPI = a.G * CL;
       const long long ntiles = items * TPI;
       const size_t part_bytes = static_cast<size_t>(ncl - 1) * 2 * L.W * sizeof(float);
-      a.part = L.lse;
+      const size_t helper_floats =
+          h > 0 ? static_cast<size_t>(F) * score_workspace_bytes(1, L.W, L.Hq) / sizeof(float) : 0;
+      a.part = L.lse + helper_floats;
       a.streamk = ncl > 1 && ntiles / ncl >= TPI &&
-                  part_bytes <= score_workspace_bytes(L.R, L.W, L.Hq);
+                  helper_floats * sizeof(float) + part_bytes <= ws_bytes;
+      if (h > 0) {
+        a.done_count = reinterpret_cast<int*>(a.part + static_cast<size_t>(ncl - 1) * 2 * L.W);
+        if (cudaMemsetAsync(a.done_count, 0, sizeof(int), stream) != cudaSuccess) {
+          check_launch("kara_score helper counter");
+          return KARA_ERR_CUDA;
+        }
+      }
       a.max_agg = AG;
       if (AG) {
         // the max aggregation merges into zeroed outputs with atomic maxima (softmax >= 0)
@@ -1597,6 +1774,13 @@ kara_status launch_score(const ScoreLaunch& L, cudaStream_t stream) {
       if (check_launch("score_fused_kernel") != KARA_OK) {
         describe_kernel("score_fused_kernel", reinterpret_cast<const void*>(kern), kFThreads, smem);
         return KARA_ERR_CUDA;
+      }
+      if (h > 0) {
+        if constexpr (D == 128) {
+          const kara_status hs = launch_helper<D>(a, L, tq1, tq2, tk, items, h, F, ncl * CL,
+                                                  stream);
+          if (hs != KARA_OK) return hs;
+        }
       }
       if (any_split) {
         launch_pdl(score_split_sum_kernel, dim3(ncl - 1), dim3(256), 0, stream, a, ncl, TPI);

@@ -151,7 +151,11 @@ def test_step_workload_scores_sampled(full_step):
     assert np.allclose(sums, wl.window * wl.group, rtol=1e-4)
     rng = np.random.default_rng(5)
     scale = 1 / math.sqrt(wl.head_dim)
-    for layer, r in zip(rng.integers(0, wl.layers, 4), rng.integers(0, wl.batch, 4)):
+    # random rows, plus the last row (its items go to the helper beside the fused kernel when
+    # the clusters leave SMs idle) and the first
+    picks = list(zip(rng.integers(0, wl.layers, 4), rng.integers(0, wl.batch, 4)))
+    picks += [(wl.layers - 1, wl.batch - 1), (0, 0)]
+    for layer, r in picks:
         slots = ok.window_slots(int(cl0[r]), wl.window)
         kw = _window_rows(cache["k"][layer], bt0[r], slots)    # old rows, still in place
         qw = cache["q_win"][layer][r].double().cpu().numpy()

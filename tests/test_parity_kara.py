@@ -53,6 +53,12 @@ SCORE_CASES = {
                                         head_dim=128, ctx_lo=1030, ctx_hi=1500, window=1024,
                                         keep=204, heavy_frac=0.05, q_mode="neighbour",
                                         spare_blocks=8),
+    # 332 (row, KV head) items at W = 1024: the clusters fill the GPU, and the last 28 items
+    # go to the one-CTA-per-item two-pass helper on the SMs the clusters leave idle
+    "w1024_helper": synth.Workload("w1024_helper", batch=83, layers=1, hq=4, hkv=4,
+                                   head_dim=128, ctx_lo=1030, ctx_hi=1200, window=1024,
+                                   keep=204, heavy_frac=0.05, q_mode="neighbour",
+                                   spare_blocks=8),
     "w1024_g2": synth.Workload("w1024_g2", batch=12, layers=1, hq=8, hkv=4,
                                    head_dim=128, ctx_lo=1024, ctx_hi=1800, window=1024,
                                    keep=204, heavy_frac=0.05, spare_blocks=8),
@@ -112,9 +118,11 @@ def test_score_matches_oracle(name):
 
 
 @pytest.mark.parametrize("name,ids", [("g7_ragged_unaligned", [1, 3]), ("g7_w512_ragged", [1, 3]),
-                                      ("w1024_g2", [7, 0, 11, 3, 9, 1, 5, 10, 2, 8, 4, 6])])
+                                      ("w1024_g2", [7, 0, 11, 3, 9, 1, 5, 10, 2, 8, 4, 6]),
+                                      ("w1024_helper", list(range(82, -1, -1)))])
 def test_score_subset_of_sequences(name, ids):
-    """Due rows given by seq_ids: a subset, or every row in another order."""
+    """Due rows given by seq_ids: a subset, or every row in another order (with the helper's
+    rows looked up through seq_ids too)."""
     wl = SCORE_CASES[name]
     cpu, dev = H.make(wl, 5)
     assert wl.batch > max(ids)
@@ -139,6 +147,24 @@ def test_score_reports_short_context():
     cpu["ctx_len"][1] = wl.window - 1
     ref = oracle_scores(cpu, wl, [0, 2])
     H.assert_scores_close(H.f64(scores[[0, 2]]), ref)
+
+
+def test_score_helper_rows_report_short_contexts():
+    """Too-short contexts among the helper's rows and the fused kernel's: their rows are zero
+    and reported, the rest match the oracle."""
+    wl = SCORE_CASES["w1024_helper"]
+    cpu, dev = H.make(wl, 7)
+    bad = [wl.batch - 1, wl.batch - 4, 3]
+    good = [r for r in range(wl.batch) if r not in bad]
+    dev["ctx_len"][bad] = wl.window - 1
+    pool = K.PagedPool.from_cache(dev)
+    status = K.new_status()
+    scores = K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window, status=status)
+    torch.cuda.synchronize()
+    assert K.read_status(status) == K.ERR_INVALID_ARG
+    assert (scores[bad] == 0).all()
+    cpu["ctx_len"][bad] = wl.window - 1
+    H.assert_scores_close(H.f64(scores[good]), oracle_scores(cpu, wl, good))
 
 
 def test_score_w1024_reports_short_contexts():
@@ -178,13 +204,14 @@ def test_score_split_items_skip_short_contexts():
 
 
 @pytest.mark.parametrize("name,launches", [("g7_w1024_unaligned", (1,)), ("w128_split_items", (2,)),
-                                           ("w1024_split_items", (2,)),
+                                           ("w1024_split_items", (2,)), ("w1024_helper", (2, 3)),
                                            ("g7_ragged_unaligned", (1, 2)), ("w1100_twopass", (3,)),
                                            ("w2500_twopass", (3,)),
                                            ("g4_w2048_ragged", (1,)), ("w2048_split_items", (2,))])
 def test_score_launch_count(name, launches):
     """The fused kernel alone when every cluster range holds whole items; with the split sum
-    when more items than resident clusters make ranges end inside items; three two-pass
+    when more items than resident clusters make ranges end inside items; with the one-kernel
+    helper when the clusters fill the GPU and there are items enough for it; three two-pass
     kernels above W = 2048."""
     wl = SCORE_CASES[name]
     cpu, dev = H.make(wl, 1)
