@@ -237,15 +237,17 @@ class Step:
                  K.kara_workspace_bytes(K.OP_COMPACT, self.pool, r, wl.window, 0, wl.keep),
                  K.kara_workspace_bytes(K.OP_DECODE, self.pool, 0, 0, hq, 0))
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
-        # scoring: the fused cluster kernel for windows of 128/256/512/1024/2048 keys (plus the
-        # split-item sum when a cluster range ends inside an item), else two passes and a
-        # merge (three launches); select + Token2Chunk in one kernel; compaction check + plan +
-        # gather; decode stream + combine. Which scorer runs is read from one call's launches.
+        # scoring: the fused cluster kernel for windows of up to 1024 keys and of 2048 (plus
+        # the split-item sum when a cluster range ends inside an item, and the one-kernel
+        # two-pass helper on the SMs the clusters leave idle when there are items enough),
+        # else the three two-pass kernels; select + Token2Chunk in one kernel; compaction
+        # check + plan + gather; decode stream + combine. One call's launches are recorded.
         n0 = K.kara_launch_count()
         K.kara_score(cache["q_win"][0], cache["k"][0], self.pool, wl.window,
                      scores=self.scores[0], workspace=self.ws, status=self.status)
         torch.cuda.synchronize()
-        self.score_fused = K.kara_launch_count() - n0 <= 2
+        self.score_launches = K.kara_launch_count() - n0
+        self.score_fused = wl.window <= 1024 or wl.window == 2048
 
     def restore(self):
         self.book.copy_(self.saved_book, non_blocking=True)
@@ -342,9 +344,12 @@ def kernel_entries(wl: synth.Workload, work: dict, avg: dict, step: Step, peaks:
     n_exp = wl.window * wl.window * wl.hq * wl.batch * L
     sfu_floor_ms = n_exp / (16 * 148 * 1.965e9) * 1e3
     if step.score_fused:
-        score_exec, score_note = 1.25, ("fused single-exponential kernel: S over 144 key rows "
-                                        "per 128 owned keys (x1.125) plus the P'^T W column-sum "
-                                        "product (N = 16, x0.125): executed = 1.25 x useful")
+        score_exec, score_note = None, ("fused single-exponential kernel (executed = 1.25 x "
+                                        "useful: S over 144 key rows per 128 owned keys plus the "
+                                        "P'^T W column-sum product), and beside it, on the SMs "
+                                        "its clusters leave idle, the one-kernel two-pass helper "
+                                        "for a few percent of the items (executed 2 x useful) "
+                                        "when the batch is large enough")
     else:
         score_exec, score_note = 2.0, ("two UMMA passes (row log-sum-exp, then column sums): "
                                        "executed flops are twice the useful Q K^T")
@@ -352,11 +357,13 @@ def kernel_entries(wl: synth.Workload, work: dict, avg: dict, step: Step, peaks:
     kernels = {
         "kara_score": {"ms": ms_score, "bound": "tensor", "launches_of_op": L,
                        "useful_tflops": work["score_flops"] / ms_score / 1e9,
-                       "executed_tflops": score_exec * work["score_flops"] / ms_score / 1e9,
+                       "executed_tflops": (score_exec * work["score_flops"] / ms_score / 1e9
+                                           if score_exec is not None else None),
+                       "launches_per_call": step.score_launches,
                        "note": score_note, "exp2_count": n_exp, "sfu_floor_ms": sfu_floor_ms,
                        "frac_of_sfu_floor": sfu_floor_ms / ms_score},
         "select+token2chunk": {"ms": avg["select+token2chunk"], "bound": "latency",
-                               "launches_of_op": L},
+                               "launches_of_op": 1},
         "kara_compact": {"ms": avg["kara_compact"], "bound": "hbm", "launches_of_op": 1,
                          "gbs": work["compact_bytes"] / avg["kara_compact"] / 1e6,
                          "bytes": work["compact_bytes"]},
