@@ -149,6 +149,27 @@ def test_score_reports_short_context():
     H.assert_scores_close(H.f64(scores[[0, 2]]), ref)
 
 
+def test_score_w2048_helper_rows():
+    """W = 2048 with items enough for the helper beside clusters of 16 (65 rows of 4 KV heads:
+    the last 36 items, rows 56-64, on the idle SMs): the helper's rows and a few of the fused
+    kernel's against the oracle, every row's sum W * G."""
+    wl = synth.Workload("w2048_helper", batch=65, layers=1, hq=4, hkv=4, head_dim=128,
+                        ctx_lo=2050, ctx_hi=2200, window=2048, keep=409, heavy_frac=0.03,
+                        spare_blocks=8)
+    cpu, dev = H.make(wl, 9)
+    pool = K.PagedPool.from_cache(dev)
+    status = K.new_status()
+    c0 = K.kara_launch_count()
+    scores = K.kara_score(dev["q_win"][0], dev["k"][0], pool, wl.window, status=status)
+    torch.cuda.synchronize()
+    assert K.read_status(status) == 0
+    assert K.kara_launch_count() - c0 in (1, 2, 3)
+    sums = scores.double().sum(-1).cpu().numpy()
+    assert np.allclose(sums, wl.window * wl.group, rtol=1e-4)
+    rows = [0, 1, 30] + list(range(wl.batch - 10, wl.batch))
+    H.assert_scores_close(H.f64(scores[rows]), oracle_scores(cpu, wl, rows))
+
+
 def test_score_helper_rows_report_short_contexts():
     """Too-short contexts among the helper's rows and the fused kernel's: their rows are zero
     and reported, the rest match the oracle."""
