@@ -344,9 +344,9 @@ def kernel_entries(wl: synth.Workload, work: dict, avg: dict, step: Step, peaks:
     n_exp = wl.window * wl.window * wl.hq * wl.batch * L
     sfu_floor_ms = n_exp / (16 * 148 * 1.965e9) * 1e3
     if step.score_fused:
-        score_exec, score_note = None, ("fused single-exponential kernel (executed = 1.25 x "
-                                        "useful: S over 144 key rows per 128 owned keys plus the "
-                                        "P'^T W column-sum product), and beside it, on the SMs "
+        score_exec, score_note = None, ("fused single-exponential kernel (executed = 1.125 x "
+                                        "useful: S over the 128 owned keys plus the P'^T W "
+                                        "column-sum product, N = 16), and beside it, on the SMs "
                                         "its clusters leave idle, the one-kernel two-pass helper "
                                         "for a few percent of the items (executed 2 x useful) "
                                         "when the batch is large enough")

@@ -851,8 +851,11 @@ score_item_kernel(const __grid_constant__ CUtensorMap tm_q1,
 // same items, CTA `rank` owns the window keys [start + 128 rank, start + 128 rank + 128) that
 // exist (a window that is not a multiple of 128 leaves the last CTA fewer; its other S columns
 // are set to -inf in tensor memory, so that they count nowhere). Per 128-query tile each CTA
-//   1. computes S = Q K^T over its keys (UMMA M = 128 queries, N = 144 key rows: the 9 pages
-//      that cover its 128 keys at any slot offset; only the owned columns are read);
+//   1. computes S = Q K^T over its keys (UMMA M = 128 queries, N = 128 keys). The 9 pages that
+//      cover the 128 keys at any slot offset are loaded whole; the B operand starts at the
+//      first owned key's row inside them (the 128-byte swizzle is a function of the shared
+//      memory address, so a start at any row of a 1024-byte-aligned buffer reads the rows as
+//      the TMA wrote them);
 //   2. in the epilogue (4 warps, one per TMEM lane quadrant: a thread owns one query row and
 //      the CTA's 128 keys) takes the row max m over its keys, P' = 2^(s*c - m + 15) and the
 //      row sum l, and stores P' as fp16 in shared memory, MN-major (rows along K) for the next
@@ -897,8 +900,8 @@ constexpr int kFXStages = 6;           // exchange slots: a peer sends its recor
                                        // only after its weights of tile T + 3, which need this
                                        // CTA's record of tile T + 3, which the team of tile T
                                        // sends after it has read the partials of tile T
-constexpr uint32_t kFSCols = kFKRows;  // TMEM column stride of the three S buffers: 0, 144, 288
-constexpr uint32_t kFDCol = kFTeams * kFSCols;   // TMEM columns of the two D buffers: 432, 448
+constexpr uint32_t kFSCols = kFKeys;  // TMEM column stride of the three S buffers: 0, 128, 256
+constexpr uint32_t kFDCol = kFTeams * kFSCols;   // TMEM columns of the two D buffers: 384, 400
 
 // Work items (r, g): KV head g of sequence r with all G of its query heads, TPI = G * CL query
 // tiles (tile tq: head g * G + tq / CL, queries 128 (tq % CL) ..; rows past W weigh nothing).
@@ -1139,14 +1142,16 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (warp == 1) {
     // ---- UMMA issuer for S: runs ahead of the epilogue by one tile ----
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, kFKRows);
+      const uint32_t idesc_s = idesc_bf16_f32(128, kFKeys);
       SegCursor cur;
       cur.init(a, cid, ncl, TPI);
       int T = 0, I = 0, C = 0;   // tiles, segments, query chunks
       bool ok = true;
       for (; ok && !*abort_flag && cur.next(a, TPI); ++I) {
         if (!mbar_wait(k_full, I & 1, abort_flag, a.status)) break;
-        const uint32_t k_addr = smem_u32(k_buf);
+        // the S product starts at the CTA's first key, row `off` of the loaded pages
+        const int koff = (cur.s.start + static_cast<int>(rank) * kFKeys) % 16;
+        const uint32_t k_addr = smem_u32(k_buf) + koff * kRowBytes;
         for (int tq = cur.q0; tq < cur.q1 && ok; ++tq, ++T) {
           const int st = T % kFTeams;
           const uint32_t ph = (T / kFTeams) & 1;
@@ -1247,8 +1252,7 @@ score_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
     float kmax0 = 0.f, kmax1 = 0.f;   // the max aggregation: this thread's two keys
     for (int T = team; have; T += kFTeams, ++sq) {
       const uint32_t ph = sq & 1;
-      const uint32_t scol = lane_base + st * kFSCols +
-                            ((cur.s.start + static_cast<int>(rank) * kFKeys) % 16);
+      const uint32_t scol = lane_base + st * kFSCols;
       // (1) row max over this CTA's 128 keys (first pass over TMEM)
       wait_cta(&s_full[st], ph);
       float mx = 0.f, l = 0.f;

@@ -170,6 +170,24 @@ def test_score_w2048_helper_rows():
     H.assert_scores_close(H.f64(scores[rows]), oracle_scores(cpu, wl, rows))
 
 
+def test_score_ring_equals_dense_with_the_helper():
+    """The window-query ring form with the helper active (83 due rows at W = 1024, seq_ids
+    given): the same tiles in the same order as the dense form, so the same bits."""
+    wl = SCORE_CASES["w1024_helper"]
+    cpu, dev = H.make(wl, 10)
+    pool = K.PagedPool.from_cache(dev)
+    W = wl.window
+    ring = torch.zeros((wl.batch, 2 * W, wl.hq, wl.head_dim), device="cuda", dtype=torch.bfloat16)
+    for b in range(wl.batch):
+        off = (int(cpu["ctx_len"][b]) - W) % W
+        ring[b, off:off + W] = dev["q_win"][0][b]
+    seq = torch.arange(wl.batch, dtype=torch.int32, device="cuda")
+    a = K.kara_score(dev["q_win"][0], dev["k"][0], pool, W)
+    b = K.kara_score_ex(ring, dev["k"][0], pool, W, ring=True, seq_ids=seq)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
 def test_score_helper_rows_report_short_contexts():
     """Too-short contexts among the helper's rows and the fused kernel's: their rows are zero
     and reported, the rest match the oracle."""
