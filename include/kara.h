@@ -146,6 +146,9 @@ typedef enum kara_op {
  *             KARA_ERR_BAD_BLOCK for a window block id outside [0, num_blocks),
  *             KARA_ERR_TIMEOUT if a pipeline wait ran out; the scores of such a sequence are
  *             then zero or unspecified.
+ * With enough (sequence, KV head) items the call runs a second kernel beside the cluster
+ * kernel, on the SMs its clusters leave idle, for the last few items; both are in `stream`
+ * and whatever the caller enqueues after the call sees all scores, as usual.
  */
 kara_status kara_score(const void* q_win, const void* k_cache, const kara_pool* pool,
                        const int32_t* seq_ids, int32_t num_seqs, int32_t window,
