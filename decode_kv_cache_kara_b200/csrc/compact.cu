@@ -245,7 +245,7 @@ __device__ void finalize_if_last(const FinalizeParams& p, int r, int per_seq,
 // prefix rows of the first window page for its head.
 // ------------------------------------------------------------------------------------------
 constexpr int kGatherThreads = 128;
-constexpr int kChunkRows = 64;
+constexpr int kChunkRows = 256;
 
 struct KaraGather {
   LayerPtrs layers;
