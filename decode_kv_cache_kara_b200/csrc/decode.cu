@@ -57,8 +57,8 @@ struct DecodeArgs {
 
 template <int D>
 __host__ __device__ constexpr int page_bytes() { return 16 * D * 2; }   // one page, one KV head
-constexpr int kStages = 4;          // TMA ring depth per warp, in single pages (K or V)
-constexpr int kDecMinBlocks = 3;    // resident CTAs per SM the register budget is sized for
+constexpr int kStages = 3;          // TMA ring depth per warp, in single pages (K or V)
+constexpr int kDecMinBlocks = 4;    // resident CTAs per SM the register budget is sized for
 
 template <int D, int G>
 constexpr size_t stream_smem_bytes() {
