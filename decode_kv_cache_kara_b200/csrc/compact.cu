@@ -508,7 +508,7 @@ __global__ void __launch_bounds__(kGatherThreads) ladder_gather_kernel(const Lad
   // row_vecs (Hkv * d * 2 / 16) is a power of two for power-of-two head counts: shifts then
   const bool pow2 = (g.row_vecs & (g.row_vecs - 1)) == 0;
   const int shift = __ffs(g.row_vecs) - 1;
-  constexpr int kUnroll = 4;
+  constexpr int kUnroll = 8;
   for (int base = threadIdx.x; base < pieces; base += kGatherThreads * kUnroll) {
     uint4 kv[kUnroll], vv[kUnroll];
     size_t dsti[kUnroll];
