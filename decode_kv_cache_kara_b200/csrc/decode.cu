@@ -57,13 +57,18 @@ struct DecodeArgs {
 
 template <int D>
 __host__ __device__ constexpr int page_bytes() { return 16 * D * 2; }   // one page, one KV head
-constexpr int kStages = 3;          // TMA ring depth per warp, in single pages (K or V)
-constexpr int kDecMinBlocks = 4;    // resident CTAs per SM the register budget is sized for
+// Two ring shapes with the same bytes in flight per SM: DEEP = 3 CTAs per SM with 4-page rings
+// per warp, else 4 CTAs per SM (128 registers a thread) with 3-page rings.
+template <bool DEEP>
+__host__ __device__ constexpr int dec_stages() { return DEEP ? 4 : 3; }   // ring depth, pages
+template <bool DEEP>
+__host__ __device__ constexpr int dec_min_blocks() { return DEEP ? 3 : 4; }
 
-template <int D, int G>
+template <int D, bool DEEP>
 constexpr size_t stream_smem_bytes() {
   // [warp][stage] one page (1024-aligned) + the warps' ring barriers
-  return 1024 + static_cast<size_t>(kDecWarps) * kStages * page_bytes<D>() + 8 * kStages * kDecWarps;
+  return 1024 + static_cast<size_t>(kDecWarps) * dec_stages<DEEP>() * page_bytes<D>() +
+         8 * dec_stages<DEEP>() * kDecWarps;
 }
 
 // Byte offset of 16-byte granule `gi` of row `r` in a 128-byte-swizzled 16-row box.
@@ -141,7 +146,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 // Persistent, one independent stream per warp: the warp walks units u = warp_id, +num_warps,
-// ...; its TMA ring (kStages single pages) streams, per unit, the unit's K pages and then its
+// ...; its TMA ring (dec_stages single pages) streams, per unit, the unit's K pages and then its
 // V pages, and keeps streaming across unit boundaries (the next unit's block ids and queries
 // are fetched ahead). Every unit leaves one partial (m, l, o) per query head for the combine
 // kernel.
@@ -153,11 +158,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // head over the unit fixes the exponent base, so the accumulators are never rescaled. P^T goes
 // to bf16 and, transposed in registers by movmatrix, becomes the B operand of O^T (d x 8) +=
 // V^T (d x 16) P^T (16 x 8), with V^T fragments read by ldmatrix.trans.
-template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
+template <int D, int G, bool DEEP>
+__global__ void __launch_bounds__(kDecThreads, dec_min_blocks<DEEP>())
 decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
   static_assert(G <= 8, "at most 8 query heads per KV head");
+  constexpr int kStages = dec_stages<DEEP>();
   asm volatile("griddepcontrol.wait;" ::: "memory");   // previous kernel done (PDL launch)
   constexpr int NCH = D / 64;                 // 64-channel chunks per row
   constexpr int KS = D / 16;                  // k-steps of S^T, m-tiles of O^T
@@ -538,10 +544,10 @@ decode_combine_kernel(const DecodeArgs a, __nv_bfloat16* __restrict__ out) {
   }
 }
 
-template <int D, int G>
+template <int D, int G, bool DEEP>
 kara_status launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, void* out,
                       cudaStream_t stream) {
-  constexpr size_t smem = stream_smem_bytes<D, G>();
+  constexpr size_t smem = stream_smem_bytes<D, DEEP>();
   static std::atomic<int> per_sm[kMaxDevices];   // resident CTAs per SM, queried once per device
   const int dev = device_slot();
   if (dev < 0) {
@@ -549,15 +555,15 @@ kara_status launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensor
     return KARA_ERR_CUDA;
   }
   if (per_sm[dev].load() == 0) {
-    cudaFuncSetAttribute(decode_stream_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(decode_stream_kernel<D, G, DEEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
     int n = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_stream_kernel<D, G>, kDecThreads, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_stream_kernel<D, G, DEEP>, kDecThreads, smem);
     per_sm[dev].store(n > 0 ? n : 1);
   }
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  launch_pdl(decode_stream_kernel<D, G>, dim3(per_sm[dev].load() * sms), dim3(kDecThreads), smem,
+  launch_pdl(decode_stream_kernel<D, G, DEEP>, dim3(per_sm[dev].load() * sms), dim3(kDecThreads), smem,
              stream, tk, tv, a);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.B * a.Hq);
@@ -573,18 +579,26 @@ kara_status launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensor
   return check_launch(__func__);
 }
 
+// Ring shape per instantiation. At 128 registers (4 CTAs per SM) the d = 128 stream spills
+// 4-12 bytes for G <= 6 (ptxas); those run 3 CTAs per SM with 4-page rings, which measured 8 %
+// faster at G = 4 with 4 and with 8 KV heads. G = 7 and 8 fit 128 registers without spills and
+// run 4 CTAs per SM with 3-page rings, 0.8-0.9 % faster with 4 and with 8 KV heads. d = 64 fits
+// either way (at most 125 registers) and keeps the shallow rings.
+template <int D, int G>
+constexpr bool deep_ring() { return D == 128 && G <= 6; }
+
 template <int D>
 kara_status launch_d(const DecodeArgs& a, int G, const CUtensorMap& tk, const CUtensorMap& tv,
                      void* out, cudaStream_t stream) {
   switch (G) {
-    case 1: return launch_dg<D, 1>(a, tk, tv, out, stream);
-    case 2: return launch_dg<D, 2>(a, tk, tv, out, stream);
-    case 3: return launch_dg<D, 3>(a, tk, tv, out, stream);
-    case 4: return launch_dg<D, 4>(a, tk, tv, out, stream);
-    case 5: return launch_dg<D, 5>(a, tk, tv, out, stream);
-    case 6: return launch_dg<D, 6>(a, tk, tv, out, stream);
-    case 7: return launch_dg<D, 7>(a, tk, tv, out, stream);
-    case 8: return launch_dg<D, 8>(a, tk, tv, out, stream);
+    case 1: return launch_dg<D, 1, deep_ring<D, 1>()>(a, tk, tv, out, stream);
+    case 2: return launch_dg<D, 2, deep_ring<D, 2>()>(a, tk, tv, out, stream);
+    case 3: return launch_dg<D, 3, deep_ring<D, 3>()>(a, tk, tv, out, stream);
+    case 4: return launch_dg<D, 4, deep_ring<D, 4>()>(a, tk, tv, out, stream);
+    case 5: return launch_dg<D, 5, deep_ring<D, 5>()>(a, tk, tv, out, stream);
+    case 6: return launch_dg<D, 6, deep_ring<D, 6>()>(a, tk, tv, out, stream);
+    case 7: return launch_dg<D, 7, deep_ring<D, 7>()>(a, tk, tv, out, stream);
+    case 8: return launch_dg<D, 8, deep_ring<D, 8>()>(a, tk, tv, out, stream);
     default: return KARA_ERR_UNSUPPORTED;
   }
 }
