@@ -381,6 +381,42 @@ def kernel_entries(wl: synth.Workload, work: dict, avg: dict, step: Step, peaks:
     return kernels
 
 
+def roofline_entry(kernels: dict, peaks: dict, src: str, total_ms: float, clocks,
+                   traffic_of) -> dict:
+    """The bench line's `roofline`: the dominant kernel (the longest op bound by the tensor
+    pipe or by HBM), its achieved rate over its summed launch time and the measured peak it is
+    held against. A tensor-bound kernel timed inside a long run (a timed region of a second or
+    more, or with sw_power_cap seen in the clock samples) is held against the sustained bf16
+    figure, one timed alone against the burst figure; both fractions are reported."""
+    dom = max((k for k in kernels if kernels[k]["bound"] in ("tensor", "hbm")),
+              key=lambda k: kernels[k]["ms"])
+    dk = kernels[dom]
+    traffic = traffic_of(dom)
+    per_launch = (f"the op runs as {dk['launches_of_op']} launches per step (one per layer); "
+                  "achieved = useful work of all of them / their summed duration")
+    if dk["bound"] == "hbm":
+        return {"kernel": dom, "bound": "hbm", "achieved": dk["gbs"], "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": dk["gbs"] / peaks["hbm_gbs"], "traffic": traffic,
+                "peak_source": f"{src} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
+                "per_launch": per_launch}
+    timed_s = total_ms / 1e3
+    capped = bool(clocks) and "sw_power_cap" in (clocks.get("reasons") or [])
+    sustained = timed_s >= 1.0 or capped
+    sus_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    peak = sus_peak if sustained else peaks["bf16_tflops"]
+    if sustained:
+        source = (f"{src} bf16 sustained (MEASURED_PEAKS.json bf16_tflops_sustained): timed "
+                  f"region {timed_s:.2f} s{', sw_power_cap active' if capped else ''}")
+    else:
+        source = (f"{src} bf16 burst (MEASURED_PEAKS.json bf16_tflops): timed region "
+                  f"{timed_s:.2f} s, no power cap seen")
+    return {"kernel": dom, "bound": "tensor", "achieved": dk["useful_tflops"], "peak": peak,
+            "unit": "TFLOP/s", "frac": dk["useful_tflops"] / peak, "traffic": traffic,
+            "frac_of_burst": dk["useful_tflops"] / peaks["bf16_tflops"],
+            "frac_of_sustained": dk["useful_tflops"] / sus_peak,
+            "peak_source": source, "per_launch": per_launch}
+
+
 def time_cpu_oracle_sample(cache_cpu: dict, wl: synth.Workload, units: int = 1, seed: int = 0,
                            layers_per_step: int = 1):
     """The oracle as it stands on `units` (sequence, KV head) units of one layer of a CPU
@@ -989,37 +1025,8 @@ def gpu_arm(args, rank: int, world: int, local_rank: int) -> dict | None:
     if rank != 0:
         return None
 
-    dom = max((k for k in kernels if kernels[k]["bound"] in ("tensor", "hbm")),
-              key=lambda k: kernels[k]["ms"])
-    dk = kernels[dom]
-    traffic = captured_traffic(dom, wl.name)
-    per_launch = (f"the op runs as {dk['launches_of_op']} launches per step (one per layer); "
-                  "achieved = useful work of all of them / their summed duration")
-    if dk["bound"] == "tensor":
-        # The burst GEMM figure is the denominator for a kernel timed alone; one timed inside a
-        # long run (a second or more of back-to-back steps, or under the power cap) takes the
-        # sustained figure. Both fractions are reported.
-        timed_s = total_ms / 1e3
-        capped = bool(clocks) and "sw_power_cap" in (clocks.get("reasons") or [])
-        sustained = timed_s >= 1.0 or capped
-        sus_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        peak = sus_peak if sustained else peaks["bf16_tflops"]
-        roof = {"kernel": dom, "bound": "tensor", "achieved": dk["useful_tflops"],
-                "peak": peak, "unit": "TFLOP/s",
-                "frac": dk["useful_tflops"] / peak, "traffic": traffic,
-                "frac_of_burst": dk["useful_tflops"] / peaks["bf16_tflops"],
-                "frac_of_sustained": dk["useful_tflops"] / sus_peak,
-                "peak_source": (f"{src} bf16 sustained (MEASURED_PEAKS.json "
-                                f"bf16_tflops_sustained): timed region {timed_s:.2f} s"
-                                f"{', sw_power_cap active' if capped else ''}" if sustained else
-                                f"{src} bf16 burst (MEASURED_PEAKS.json bf16_tflops): timed "
-                                f"region {timed_s:.2f} s, no power cap seen"),
-                "per_launch": per_launch}
-    else:
-        roof = {"kernel": dom, "bound": "hbm", "achieved": dk["gbs"], "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": dk["gbs"] / peaks["hbm_gbs"], "traffic": traffic,
-                "peak_source": f"{src} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
-                "per_launch": per_launch}
+    roof = roofline_entry(kernels, peaks, src, total_ms, clocks,
+                          lambda op: captured_traffic(op, wl.name))
 
     comp_ms = sum(kernels[op]["ms"] for op in ("kara_score", "select+token2chunk", "kara_compact"))
     kernels["compression_only"] = {
